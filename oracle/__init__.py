@@ -1,0 +1,208 @@
+"""fp64 CPU oracle for the DiT block memory-bound operators.
+
+TEST INFRASTRUCTURE ONLY.  Only the test-suite, ``__graft_entry__.smoke()``
+and the CPU-baseline leg of ``bench.py`` may import this package.  The CUDA
+library never loads it and shares no code with it; a product call that reached
+this module would be a CPU fallback, which the library does not have.
+
+This module is argument marshalling around ``dit_oracle.c`` (numpy arrays in,
+numpy arrays out).  bf16 tensors travel as ``uint16`` bit patterns; modulation
+vectors and norm weights as ``float64`` (a float32 value widens exactly).
+Outputs come back unrounded in fp64; ``f64_to_bf16`` rounds them once.
+"""
+from __future__ import annotations
+
+import ctypes
+import threading
+
+import numpy as np
+
+from . import build as _build
+
+_u16p = ctypes.POINTER(ctypes.c_uint16)
+_u8p = ctypes.POINTER(ctypes.c_uint8)
+_i32p = ctypes.POINTER(ctypes.c_int32)
+_f64p = ctypes.POINTER(ctypes.c_double)
+_i64 = ctypes.c_int64
+_int = ctypes.c_int
+_dbl = ctypes.c_double
+
+
+def _c(a: np.ndarray, dtype) -> np.ndarray:
+    return np.ascontiguousarray(a, dtype=dtype)
+
+
+def _p(a: np.ndarray, ptype):
+    return a.ctypes.data_as(ptype)
+
+
+def _check(rc: int, what: str) -> None:
+    if rc != 0:
+        raise ValueError(f"oracle {what}: bad arguments (code {rc})")
+
+
+class Oracle:
+    """The oracle library at ``path`` (the built dit_oracle.c by default)."""
+
+    def __init__(self, path: str | None = None):
+        L = ctypes.CDLL(path or _build.build())
+        L.dito_bf16_to_f64.argtypes = [ctypes.c_uint16]
+        L.dito_bf16_to_f64.restype = _dbl
+        L.dito_f64_to_bf16.argtypes = [_dbl]
+        L.dito_f64_to_bf16.restype = ctypes.c_uint16
+        L.dito_round_bf16.argtypes = [_f64p, _u16p, _i64]
+        L.dito_widen_bf16.argtypes = [_u16p, _f64p, _i64]
+        L.dito_adaln_modulate.argtypes = [_u16p, _f64p, _f64p, _i64, _int, _i64, _int,
+                                          _dbl, _f64p, _f64p]
+        L.dito_gated_residual_adaln.argtypes = [_u16p, _u16p, _f64p, _f64p, _f64p, _i64,
+                                                _int, _i64, _int, _dbl, _u16p, _f64p, _f64p]
+        L.dito_swiglu.argtypes = [_u16p, _i64, _int, _f64p]
+        L.dito_grid_positions.argtypes = [_int, _int, _int, _i64, _i64, _i32p]
+        L.dito_qk_rmsnorm_rope3d.argtypes = [_u16p, _i64, _f64p, _int, _i64, _int, _int,
+                                             _i32p, _int, _int, _int, _dbl, _dbl, _f64p, _f64p]
+        L.dito_cachedit_sums.argtypes = [_u16p, _u16p, _i64, _f64p, _f64p]
+        L.dito_cachedit_decide.argtypes = [_dbl, _dbl, _dbl, _f64p]
+        L.dito_cachedit_decide.restype = _int
+        L.dito_cachedit_residual_diff.argtypes = [_u16p, _u16p, _int, _i64, _int, _dbl,
+                                                  _f64p, _u8p]
+        for name in ("dito_adaln_modulate", "dito_gated_residual_adaln", "dito_swiglu",
+                     "dito_grid_positions", "dito_qk_rmsnorm_rope3d",
+                     "dito_cachedit_residual_diff"):
+            getattr(L, name).restype = _int
+        self.lib = L
+
+    # ------------------------------------------------------------- bf16
+
+    def bf16_to_f64(self, h: np.ndarray) -> np.ndarray:
+        h = _c(h, np.uint16)
+        out = np.empty(h.shape, dtype=np.float64)
+        self.lib.dito_widen_bf16(_p(h, _u16p), _p(out, _f64p), h.size)
+        return out
+
+    def f64_to_bf16(self, v: np.ndarray) -> np.ndarray:
+        v = _c(v, np.float64)
+        out = np.empty(v.shape, dtype=np.uint16)
+        self.lib.dito_round_bf16(_p(v, _f64p), _p(out, _u16p), v.size)
+        return out
+
+    def f64_to_bf16_scalar(self, v: float) -> int:
+        return int(self.lib.dito_f64_to_bf16(float(v)))
+
+    # -------------------------------------------------------- operators
+
+    def adaln_modulate(self, x, shift, scale, eps):
+        """x: [B,N,D] bf16 bits; shift, scale: [B,D]. Returns y [B,N,D] fp64."""
+        x = _c(x, np.uint16)
+        B, N, D = x.shape
+        shift = _c(shift, np.float64).reshape(B, D)
+        scale = _c(scale, np.float64).reshape(B, D)
+        y = np.empty((B, N, D), dtype=np.float64)
+        work = np.empty(D, dtype=np.float64)
+        _check(self.lib.dito_adaln_modulate(_p(x, _u16p), _p(shift, _f64p), _p(scale, _f64p), D,
+                                            B, N, D, eps, _p(y, _f64p), _p(work, _f64p)),
+               "adaln_modulate")
+        return y
+
+    def gated_residual_adaln(self, x, r, gate, shift, scale, eps):
+        """x, r: [B,N,D] bf16 bits; gate/shift/scale [B,D].
+        Returns (x_out [B,N,D] bf16 bits, y [B,N,D] fp64)."""
+        x = _c(x, np.uint16)
+        r = _c(r, np.uint16)
+        B, N, D = x.shape
+        gate = _c(gate, np.float64).reshape(B, D)
+        shift = _c(shift, np.float64).reshape(B, D)
+        scale = _c(scale, np.float64).reshape(B, D)
+        x_out = np.empty((B, N, D), dtype=np.uint16)
+        y = np.empty((B, N, D), dtype=np.float64)
+        work = np.empty(D, dtype=np.float64)
+        _check(self.lib.dito_gated_residual_adaln(_p(x, _u16p), _p(r, _u16p), _p(gate, _f64p),
+                                                  _p(shift, _f64p), _p(scale, _f64p), D, B, N, D,
+                                                  eps, _p(x_out, _u16p), _p(y, _f64p),
+                                                  _p(work, _f64p)),
+               "gated_residual_adaln")
+        return x_out, y
+
+    def swiglu(self, inp):
+        """inp: [M, 2F] bf16 bits. Returns [M, F] fp64."""
+        inp = _c(inp, np.uint16)
+        M, F2 = inp.shape
+        if F2 % 2:
+            raise ValueError("swiglu input width must be even")
+        F = F2 // 2
+        out = np.empty((M, F), dtype=np.float64)
+        _check(self.lib.dito_swiglu(_p(inp, _u16p), M, F, _p(out, _f64p)), "swiglu")
+        return out
+
+    def grid_positions(self, T, Hg, Wg, offset, N):
+        """[N, 3] int32 (t, h, w) of global tokens offset .. offset+N-1."""
+        pos = np.empty((N, 3), dtype=np.int32)
+        _check(self.lib.dito_grid_positions(T, Hg, Wg, offset, N, _p(pos, _i32p)),
+               "grid_positions")
+        return pos
+
+    def qk_rmsnorm_rope3d(self, x, w, H, hd, pos, pairs, theta, eps, row_stride=None):
+        """x: token rows of bf16 bits ([R, row_stride] or [..., H*hd]); w: [hd];
+        pos: [R, 3] int32. Returns [R, H*hd] fp64."""
+        x = _c(x, np.uint16)
+        if row_stride is None:
+            row_stride = x.shape[-1]
+        R = x.size // row_stride
+        w = _c(w, np.float64).reshape(hd)
+        pos = _c(pos, np.int32).reshape(R, 3)
+        out = np.empty((R, H * hd), dtype=np.float64)
+        work = np.empty(hd, dtype=np.float64)
+        pt, ph, pw = pairs
+        _check(self.lib.dito_qk_rmsnorm_rope3d(_p(x, _u16p), row_stride, _p(w, _f64p), 1, R, H,
+                                               hd, _p(pos, _i32p), pt, ph, pw, theta, eps,
+                                               _p(out, _f64p), _p(work, _f64p)),
+               "qk_rmsnorm_rope3d")
+        return out
+
+    def cachedit_sums(self, prev, cur):
+        """(sum |cur - prev|, sum |prev|) over all elements, fp64."""
+        prev = _c(prev, np.uint16)
+        cur = _c(cur, np.uint16)
+        if prev.size != cur.size:
+            raise ValueError("size mismatch")
+        num = ctypes.c_double()
+        den = ctypes.c_double()
+        self.lib.dito_cachedit_sums(_p(prev, _u16p), _p(cur, _u16p), prev.size,
+                                    ctypes.byref(num), ctypes.byref(den))
+        return num.value, den.value
+
+    def cachedit_decide(self, num, den, threshold):
+        """(rel, reuse) from the two sums."""
+        rel = ctypes.c_double()
+        reuse = self.lib.dito_cachedit_decide(num, den, threshold, ctypes.byref(rel))
+        return rel.value, int(reuse)
+
+    def cachedit_residual_diff(self, prev, cur, threshold):
+        """prev, cur: [B,N,D] bf16 bits. Returns (rel [B] fp64, reuse [B] uint8)."""
+        prev = _c(prev, np.uint16)
+        cur = _c(cur, np.uint16)
+        B, N, D = prev.shape
+        rel = np.empty(B, dtype=np.float64)
+        reuse = np.empty(B, dtype=np.uint8)
+        _check(self.lib.dito_cachedit_residual_diff(_p(prev, _u16p), _p(cur, _u16p), B, N, D,
+                                                    threshold, _p(rel, _f64p), _p(reuse, _u8p)),
+               "cachedit_residual_diff")
+        return rel, reuse
+
+
+_default = None
+_lock = threading.Lock()
+
+
+def default() -> Oracle:
+    global _default
+    with _lock:
+        if _default is None:
+            _default = Oracle()
+    return _default
+
+
+def __getattr__(name):
+    # module-level access to the default oracle's methods: oracle.swiglu(...)
+    if name.startswith("_"):
+        raise AttributeError(name)
+    return getattr(default(), name)

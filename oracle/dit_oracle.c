@@ -1,0 +1,312 @@
+/*
+ * dit_oracle.c -- plain, slow, fp64 CPU oracle for the per-block memory-bound
+ * operators of a dense single-stream video+audio DiT (MiniMax-H3 shaped).
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing in the product path may link, load or
+ * call this file: only the test-suite, the smoke check and the CPU-baseline
+ * leg of the benchmark use it.  It shares no code, header, table or helper
+ * with the CUDA library.
+ *
+ * Sources.  The operators are named, not defined, by:
+ *   [REPORT]  "MiniMax-H3 no SGLang em H200" (news.cocoloop.cn, LMSYS report
+ *             summary), section "Só com três camadas de aceleração somadas
+ *             chega-se a 6 vezes": fused AdaLN update, gated residual, SwiGLU,
+ *             QK RMSNorm with 3D RoPE; the fused layer changes no result;
+ *             Cache-DiT reuses results between neighbouring denoising steps
+ *             when a residual-difference threshold (0.04 conservative, 0.08
+ *             stride mode) allows it.
+ *   [CEVIU]   "SGLang acelera MiniMax-H3 em GPUs H200 e redefine geração de
+ *             vídeo por IA" (ceviu.com.br), first paragraph: the three
+ *             pillars (fused kernels for AdaLN, SwiGLU, QK RMSNorm, 3D RoPE;
+ *             Cache-DiT; SubBlock attention).
+ *   [H3BASE]  "MiniMax H3 mở trọng số: H3-Base có gì và còn thiếu gì?"
+ *             (studioglobal.ai), section "Kiến trúc: tạo hình và tiếng trong
+ *             cùng một luồng": dense single-stream transformer whose AdaLN
+ *             branch outputs can be precomputed and cached.
+ * The pages print no formula; every function below is the textbook definition
+ * of the named operator, with the readings listed beside it.
+ *
+ * Arithmetic.  Every stored input (bf16 bit patterns, fp64 modulation or
+ * weights) is read exactly into fp64; the definition is evaluated in fp64 in
+ * the plainest order; callers round a final output to bf16 once with
+ * dito_f64_to_bf16 (round to nearest, ties to even, straight from fp64).
+ *
+ * Parity pins: closed forms, invariants, hand-worked golden values and exact
+ * rational brute force live in the test-suite (tests/test_oracle_*.py).
+ */
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+
+/* ------------------------------------------------------------------ bf16 */
+
+/* bf16 is the upper half of an IEEE binary32 word: widen and reinterpret. */
+double dito_bf16_to_f64(uint16_t h)
+{
+    uint32_t w = ((uint32_t)h) << 16;
+    float f;
+    memcpy(&f, &w, sizeof f);
+    return (double)f;
+}
+
+/*
+ * Round an fp64 value to the nearest bf16 (ties to even) in ONE step.
+ * bf16 keeps 8 significant bits, the binary32 exponent range, subnormals down
+ * to 2^-133 and overflows to infinity at (2 - 2^-8) * 2^127 and above.
+ * Method: find the value's binade [2^(e-1), 2^e), take the bf16 spacing q of
+ * that binade (2^(e-8); 2^-133 below the normal range), round a/q to an
+ * integer with rint() in the default ties-to-even mode (a/q is an exact
+ * power-of-two scaling), scale back and re-encode.  No intermediate rounding
+ * to binary32 happens, so there is no double rounding.
+ */
+uint16_t dito_f64_to_bf16(double v)
+{
+    uint16_t sign = signbit(v) ? 0x8000u : 0u;
+    if (isnan(v)) return (uint16_t)(sign | 0x7FC0u);
+    double a = fabs(v);
+    if (isinf(a)) return (uint16_t)(sign | 0x7F80u);
+    if (a == 0.0) return sign;
+    int e;
+    (void)frexp(a, &e);                 /* a in [2^(e-1), 2^e) */
+    int qexp = (e - 1 >= -126) ? (e - 8) : -133;
+    double k = ldexp(a, -qexp);         /* exact */
+    double r = rint(k);                 /* ties to even */
+    double res = ldexp(r, qexp);        /* exact */
+    if (res >= 0x1p128) return (uint16_t)(sign | 0x7F80u);
+    if (res == 0.0) return sign;
+    float f = (float)res;               /* exact: <= 8 significant bits */
+    uint32_t w;
+    memcpy(&w, &f, sizeof w);
+    return (uint16_t)(sign | (uint16_t)(w >> 16));
+}
+
+void dito_round_bf16(const double* v, uint16_t* out, int64_t n)
+{
+    for (int64_t i = 0; i < n; ++i) out[i] = dito_f64_to_bf16(v[i]);
+}
+
+void dito_widen_bf16(const uint16_t* h, double* out, int64_t n)
+{
+    for (int64_t i = 0; i < n; ++i) out[i] = dito_bf16_to_f64(h[i]);
+}
+
+/* --------------------------------------------------- AdaLN modulation (a1) */
+
+/*
+ * Non-affine LayerNorm of one row of D values, then the AdaLN modulation
+ *     y_d = (x_d - mu) / sqrt(var + eps) * (1 + scale_d) + shift_d
+ * with mu the row mean and var the biased (divide by D) variance, computed in
+ * two passes.  Readings: the "(1 + scale)" form (zero modulation must give a
+ * plain LayerNorm), eps inside the square root.  [REPORT] "atualização do
+ * AdaLN"; [H3BASE] modulation vectors come precomputed from the AdaLN branch.
+ */
+static void adaln_row(const double* x, const double* shift, const double* scale,
+                      int D, double eps, double* y)
+{
+    double mu = 0.0;
+    for (int d = 0; d < D; ++d) mu += x[d];
+    mu /= (double)D;
+    double var = 0.0;
+    for (int d = 0; d < D; ++d) var += (x[d] - mu) * (x[d] - mu);
+    var /= (double)D;
+    double inv = 1.0 / sqrt(var + eps);
+    for (int d = 0; d < D; ++d)
+        y[d] = (x[d] - mu) * inv * (1.0 + scale[d]) + shift[d];
+}
+
+/*
+ * x: [B,N,D] bf16 bits.  shift, scale: fp64, sample b's vector starts at
+ * b*mod_batch_stride.  y: [B,N,D] fp64 (unrounded).  work: D doubles.
+ */
+int dito_adaln_modulate(const uint16_t* x, const double* shift, const double* scale,
+                        int64_t mod_batch_stride, int B, int64_t N, int D, double eps,
+                        double* y, double* work)
+{
+    if (D <= 0 || B < 0 || N < 0) return -2;
+    for (int b = 0; b < B; ++b)
+        for (int64_t n = 0; n < N; ++n) {
+            int64_t row = ((int64_t)b * N + n) * D;
+            for (int d = 0; d < D; ++d) work[d] = dito_bf16_to_f64(x[row + d]);
+            adaln_row(work, shift + b * mod_batch_stride, scale + b * mod_batch_stride,
+                      D, eps, y + row);
+        }
+    return 0;
+}
+
+/* ------------------------------------- gated residual fused with AdaLN (a2) */
+
+/*
+ * x' = bf16(x + gate * r)  (one rounding, stored: it is the new residual
+ * stream), then y = AdaLN(x') as in a1 on the ROUNDED x'.  Reading: the fused
+ * operator must give what the unfused chain gives ([REPORT]: the fused layer
+ * "does not change any calculation result"), and the unfused chain stores x'
+ * in bf16 before the next LayerNorm reads it.  Plain (not tanh) gate.
+ */
+int dito_gated_residual_adaln(const uint16_t* x, const uint16_t* r,
+                              const double* gate, const double* shift, const double* scale,
+                              int64_t mod_batch_stride, int B, int64_t N, int D, double eps,
+                              uint16_t* x_out, double* y, double* work)
+{
+    if (D <= 0 || B < 0 || N < 0) return -2;
+    for (int b = 0; b < B; ++b) {
+        const double* g = gate + b * mod_batch_stride;
+        for (int64_t n = 0; n < N; ++n) {
+            int64_t row = ((int64_t)b * N + n) * D;
+            for (int d = 0; d < D; ++d) {
+                double v = dito_bf16_to_f64(x[row + d]) + g[d] * dito_bf16_to_f64(r[row + d]);
+                uint16_t h = dito_f64_to_bf16(v);
+                x_out[row + d] = h;
+                work[d] = dito_bf16_to_f64(h);
+            }
+            adaln_row(work, shift + b * mod_batch_stride, scale + b * mod_batch_stride,
+                      D, eps, y + row);
+        }
+    }
+    return 0;
+}
+
+/* ------------------------------------------------------------ SwiGLU (a3) */
+
+/*
+ * in: [M, 2F]; out[m, j] = silu(a) * b with a = in[m, j] (first half, the
+ * gate) and b = in[m, F + j] (second half), silu(a) = a / (1 + exp(-a)).
+ * [REPORT] "a ativação SwiGLU".  Reading: first half is the gate.
+ */
+int dito_swiglu(const uint16_t* in, int64_t M, int F, double* out)
+{
+    if (F <= 0 || M < 0) return -2;
+    for (int64_t m = 0; m < M; ++m)
+        for (int j = 0; j < F; ++j) {
+            double a = dito_bf16_to_f64(in[m * 2 * (int64_t)F + j]);
+            double b = dito_bf16_to_f64(in[m * 2 * (int64_t)F + F + j]);
+            double silu = a / (1.0 + exp(-a));
+            out[m * (int64_t)F + j] = silu * b;
+        }
+    return 0;
+}
+
+/* ------------------------------------------ QK RMSNorm + 3D RoPE (a4) */
+
+/*
+ * Row-major flattening of a (T, Hg, Wg) latent grid: token g sits at
+ * t = g / (Hg*Wg), h = (g / Wg) % Hg, w = g % Wg.  Tokens n = 0..N-1 of each
+ * sample get the positions of global tokens offset + n.
+ */
+int dito_grid_positions(int T, int Hg, int Wg, int64_t offset, int64_t N, int32_t* pos)
+{
+    if (T <= 0 || Hg <= 0 || Wg <= 0 || offset < 0) return -2;
+    if (offset + N > (int64_t)T * Hg * Wg) return -2;
+    for (int64_t n = 0; n < N; ++n) {
+        int64_t g = offset + n;
+        pos[3 * n + 0] = (int32_t)(g / ((int64_t)Hg * Wg));
+        pos[3 * n + 1] = (int32_t)((g / Wg) % Hg);
+        pos[3 * n + 2] = (int32_t)(g % Wg);
+    }
+    return 0;
+}
+
+/*
+ * One head of hd values: RMSNorm with weight w, then 3D rotary embedding.
+ *   u_j = x_j / sqrt(mean_j(x_j^2) + eps) * w_j
+ * The hd/2 rotation pairs are (u_{2p}, u_{2p+1}) (interleaved reading).  Pairs
+ * [0, pt) follow the temporal position, [pt, pt+ph) the height position and
+ * [pt+ph, hd/2) the width position.  Inside an axis with P pairs, local pair i
+ * turns by phi = pos_axis * theta^(-2i / (2P)):
+ *   (u0, u1) -> (u0 cos phi - u1 sin phi,  u0 sin phi + u1 cos phi).
+ * [REPORT] "QK RMSNorm com 3D RoPE"; [CEVIU] "QK RMSNorm e 3D RoPE".
+ */
+static void qk_head(const double* x, const double* w, int hd, const int32_t* p3,
+                    int pt, int ph, int pw, double theta, double eps, double* out)
+{
+    double ms = 0.0;
+    for (int j = 0; j < hd; ++j) ms += x[j] * x[j];
+    ms /= (double)hd;
+    double inv = 1.0 / sqrt(ms + eps);
+    for (int p = 0; p < hd / 2; ++p) {
+        int axis, i, P;
+        if (p < pt)           { axis = 0; i = p;           P = pt; }
+        else if (p < pt + ph) { axis = 1; i = p - pt;      P = ph; }
+        else                  { axis = 2; i = p - pt - ph; P = pw; }
+        double omega = pow(theta, -2.0 * (double)i / (2.0 * (double)P));
+        double phi = (double)p3[axis] * omega;
+        double u0 = x[2 * p] * inv * w[2 * p];
+        double u1 = x[2 * p + 1] * inv * w[2 * p + 1];
+        out[2 * p]     = u0 * cos(phi) - u1 * sin(phi);
+        out[2 * p + 1] = u0 * sin(phi) + u1 * cos(phi);
+    }
+}
+
+/*
+ * x: rows of B*N tokens, token i's H*hd values start at x + i*row_stride.
+ * w: [hd] fp64.  pos: [B*N, 3] int32 (t, h, w) per token.  out: [B*N, H*hd]
+ * fp64, dense.  work: hd doubles.  Requires pt+ph+pw == hd/2, each > 0.
+ */
+int dito_qk_rmsnorm_rope3d(const uint16_t* x, int64_t row_stride, const double* w,
+                           int B, int64_t N, int H, int hd, const int32_t* pos,
+                           int pt, int ph, int pw, double theta, double eps,
+                           double* out, double* work)
+{
+    if (hd <= 0 || hd % 2 || pt <= 0 || ph <= 0 || pw <= 0 || pt + ph + pw != hd / 2)
+        return -2;
+    if (row_stride < (int64_t)H * hd) return -2;
+    int64_t rows = (int64_t)B * N;
+    for (int64_t i = 0; i < rows; ++i)
+        for (int h = 0; h < H; ++h) {
+            const uint16_t* src = x + i * row_stride + (int64_t)h * hd;
+            for (int j = 0; j < hd; ++j) work[j] = dito_bf16_to_f64(src[j]);
+            qk_head(work, w, hd, pos + 3 * i, pt, ph, pw, theta, eps,
+                    out + i * (int64_t)H * hd + (int64_t)h * hd);
+        }
+    return 0;
+}
+
+/* ----------------------------------------- Cache-DiT residual check (a5) */
+
+/*
+ * Sums over `count` elements: num = sum |cur - prev|, den = sum |prev|.
+ * [REPORT] Cache-DiT paragraph: a residual-difference threshold decides reuse.
+ */
+void dito_cachedit_sums(const uint16_t* prev, const uint16_t* cur, int64_t count,
+                        double* num, double* den)
+{
+    double s_num = 0.0, s_den = 0.0;
+    for (int64_t i = 0; i < count; ++i) {
+        double p = dito_bf16_to_f64(prev[i]);
+        double c = dito_bf16_to_f64(cur[i]);
+        s_num += fabs(c - p);
+        s_den += fabs(p);
+    }
+    *num = s_num;
+    *den = s_den;
+}
+
+/*
+ * rel = num / den, with 0/0 read as 0 (identical residuals are reusable) and
+ * x/0 as +inf; reuse = rel < threshold (strict).  Returns reuse (0 or 1).
+ */
+int dito_cachedit_decide(double num, double den, double threshold, double* rel)
+{
+    double q;
+    if (den == 0.0) q = (num == 0.0) ? 0.0 : INFINITY;
+    else q = num / den;
+    *rel = q;
+    return q < threshold ? 1 : 0;
+}
+
+/*
+ * prev, cur: [B,N,D] bf16.  Per sample b: rel[b] = relative L1 difference of
+ * its N*D elements, reuse[b] = rel[b] < threshold.
+ */
+int dito_cachedit_residual_diff(const uint16_t* prev, const uint16_t* cur,
+                                int B, int64_t N, int D, double threshold,
+                                double* rel, uint8_t* reuse)
+{
+    if (B < 0 || N < 0 || D <= 0) return -2;
+    for (int b = 0; b < B; ++b) {
+        double num, den;
+        int64_t off = (int64_t)b * N * D;
+        dito_cachedit_sums(prev + off, cur + off, N * (int64_t)D, &num, &den);
+        reuse[b] = (uint8_t)dito_cachedit_decide(num, den, threshold, &rel[b]);
+    }
+    return 0;
+}

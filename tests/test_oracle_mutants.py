@@ -1,0 +1,88 @@
+"""Planted mistakes: each mutant is a copy of the oracle's C source with one
+plausible error (a dropped term, a wrong sign, index or divisor, a transposed
+operand).  It is compiled on the CPU into a temporary library and the whole
+battery of oracle pins runs against it: at least one pin must fail.  This is
+the evidence that the pins constrain every part of the oracle."""
+import importlib
+import inspect
+import os
+import subprocess
+
+import pytest
+
+from conftest import ROOT
+
+SRC = os.path.join(ROOT, "oracle", "dit_oracle.c")
+
+MUTANTS = {
+    "ln_unbiased_variance": ("var /= (double)D;", "var /= (double)(D - 1);"),
+    "ln_eps_outside_root": ("1.0 / sqrt(var + eps)", "1.0 / (sqrt(var) + eps)"),
+    "ln_scale_without_one": ("(1.0 + scale[d])", "scale[d]"),
+    "ln_shift_scale_swapped": ("(1.0 + scale[d]) + shift[d]", "(1.0 + shift[d]) + scale[d]"),
+    "ln_mean_dropped": ("(x[d] - mu) * inv", "x[d] * inv"),
+    "gate_adds_instead_of_multiplies": ("+ g[d] * dito_bf16_to_f64(r[row + d])",
+                                        "+ g[d] + dito_bf16_to_f64(r[row + d])"),
+    "gate_ln_reads_unrounded": ("work[d] = dito_bf16_to_f64(h);", "work[d] = v;"),
+    "swiglu_exp_sign": ("a / (1.0 + exp(-a))", "a / (1.0 + exp(a))"),
+    "swiglu_halves_swapped": ("double a = dito_bf16_to_f64(in[m * 2 * (int64_t)F + j]);",
+                              "double a = dito_bf16_to_f64(in[m * 2 * (int64_t)F + F + j]);"),
+    "swiglu_row_stride": ("double b = dito_bf16_to_f64(in[m * 2 * (int64_t)F + F + j]);",
+                          "double b = dito_bf16_to_f64(in[m * (int64_t)F + F + j]);"),
+    "rms_mean_over_half_head": ("ms /= (double)hd;", "ms /= (double)(hd / 2);"),
+    "rms_eps_outside_root": ("1.0 / sqrt(ms + eps)", "1.0 / (sqrt(ms) + eps)"),
+    "rms_weight_index": ("double u1 = x[2 * p + 1] * inv * w[2 * p + 1];",
+                         "double u1 = x[2 * p + 1] * inv * w[2 * p];"),
+    "rope_rotation_sign": ("u0 * cos(phi) - u1 * sin(phi)", "u0 * cos(phi) + u1 * sin(phi)"),
+    "rope_rotate_half_layout": ("double u1 = x[2 * p + 1] * inv * w[2 * p + 1];",
+                                "double u1 = x[(p + hd / 2) % hd] * inv * w[(p + hd / 2) % hd];"),
+    "rope_axis_h_w_swapped": ("axis = 1; i = p - pt;", "axis = 2; i = p - pt;"),
+    "rope_frequency_over_head": ("-2.0 * (double)i / (2.0 * (double)P)",
+                                 "-2.0 * (double)i / (double)hd"),
+    "rope_pos_axis_index": ("double phi = (double)p3[axis] * omega;",
+                            "double phi = (double)p3[0] * omega;"),
+    "grid_h_w_confused": ("pos[3 * n + 1] = (int32_t)((g / Wg) % Hg);",
+                          "pos[3 * n + 1] = (int32_t)((g / Hg) % Wg);"),
+    "cache_denominator_uses_cur": ("s_den += fabs(p);", "s_den += fabs(c);"),
+    "cache_not_strict": ("return q < threshold ? 1 : 0;", "return q <= threshold ? 1 : 0;"),
+    "cache_zero_over_zero": ("q = (num == 0.0) ? 0.0 : INFINITY;", "q = num / den;"),
+    "cache_sample_offset": ("int64_t off = (int64_t)b * N * D;", "int64_t off = (int64_t)b * N;"),
+    "bf16_double_rounding": ("uint16_t sign = signbit(v) ? 0x8000u : 0u;",
+                             "v = (double)(float)v; uint16_t sign = signbit(v) ? 0x8000u : 0u;"),
+    "bf16_ties_away": ("double r = rint(k);", "double r = floor(k + 0.5);"),
+    "bf16_subnormal_quantum": ("int qexp = (e - 1 >= -126) ? (e - 8) : -133;",
+                               "int qexp = e - 8;"),
+}
+
+PIN_MODULES = ["test_oracle_bf16", "test_oracle_adaln", "test_oracle_swiglu", "test_oracle_qk",
+               "test_oracle_cachedit"]
+
+
+def _pins():
+    pins = []
+    for modname in PIN_MODULES:
+        mod = importlib.import_module(modname)
+        for name, fn in inspect.getmembers(mod, inspect.isfunction):
+            if name.startswith("test_") and list(inspect.signature(fn).parameters) == ["orc"]:
+                pins.append((f"{modname}.{name}", fn))
+    return pins
+
+
+@pytest.mark.parametrize("mutant", sorted(MUTANTS))
+def test_every_planted_mistake_is_caught(mutant, tmp_path):
+    import oracle
+    old, new = MUTANTS[mutant]
+    src = open(SRC).read()
+    assert src.count(old) == 1, f"mutation site for {mutant} not unique"
+    path_c = tmp_path / "mutant.c"
+    path_c.write_text(src.replace(old, new))
+    lib = tmp_path / "libmutant.so"
+    subprocess.run(["gcc", "-std=c11", "-O2", "-fPIC", "-shared", "-ffp-contract=off",
+                    "-o", str(lib), str(path_c), "-lm"], check=True)
+    orc = oracle.Oracle(str(lib))
+    caught = []
+    for name, fn in _pins():
+        try:
+            fn(orc)
+        except Exception:  # an assertion, or a crash of the mutant's arithmetic
+            caught.append(name)
+    assert caught, f"no pin catches the planted mistake {mutant}"
