@@ -1,0 +1,506 @@
+"""Benchmark of the per-block memory-bound op chain on B200.
+
+One step = one pass of the whole hot path over one H3-shaped 5 s clip
+(B=1, 31x48x84 latent grid = 124,992 tokens, D=5120, 40 heads x 128,
+SwiGLU 27,648 -> 13,824), in block order:
+  AdaLN modulation -> QK RMSNorm + 3D RoPE (in place on a fused qkv buffer)
+  -> gated residual + next AdaLN -> SwiGLU, plus the Cache-DiT residual check.
+
+Metric: block op-chain tokens/s (whole job), with per-op GB/s and fraction
+of the measured HBM peak.  Every input is larger than L2 (126 MB), so no L2
+flush is needed between steps.  Device time comes from CUDA events on the
+launching stream, bracketed by a barrier and a synchronize, max over ranks.
+
+Usage:
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+Under torchrun each rank runs an independent clip (weak scaling; the ops are
+token-local, so the data path has no collective).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = ("fused DiT op GB/s & % of B200 HBM peak; block op-chain tokens/s at 125k tokens")
+FALLBACK_HBM_GBS = 6650.0
+OPS = ["adaln_modulate", "qk_rmsnorm_rope3d", "gated_residual_adaln", "swiglu",
+       "cachedit_residual_diff"]
+DOMINANT = "swiglu"
+
+# DRAM traffic per launch from ncu (dram__bytes_read.sum + dram__bytes_write.sum),
+# valid only while the kernel source is unchanged (sha256 of the .cu file).
+NCU_TRAFFIC = {}
+
+
+def algorithmic_bytes(wl) -> dict:
+    """Bytes each op must move: every input read once, every output written
+    once (bf16 = 2 bytes; modulation vectors, weights and positions are
+    under 0.01% and left out)."""
+    M, D, F = wl.M, wl.D, wl.F
+    return {
+        "adaln_modulate": 4 * M * D,            # read x, write y
+        "qk_rmsnorm_rope3d": 8 * M * D,         # read and write q and k
+        "gated_residual_adaln": 8 * M * D,      # read x, r; write x', y
+        "swiglu": 6 * M * F,                    # read [M, 2F], write [M, F]
+        "cachedit_residual_diff": 4 * M * D,    # read prev, cur
+    }
+
+
+def hbm_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            v = float(json.load(f)["hbm_gbs"])
+        return v, "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+# ------------------------------------------------------------- clocks
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons during a region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100", "-i", str(self.gpu)],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.reader = threading.Thread(target=self._read, daemon=True)
+            self.reader.start()
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            self.reader.join(timeout=2)
+
+    def summary(self):
+        rows = []
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append({"sm": float(parts[1]), "max": float(parts[2]),
+                             "power": float(parts[3]), "hw": parts[5], "hwt": parts[6],
+                             "swt": parts[7], "pcap": parts[8]})
+            except ValueError:
+                continue
+        if not rows:
+            return None
+        reasons = set()
+        for r in rows:
+            for key, name in (("hw", "hw_slowdown"), ("hwt", "hw_thermal_slowdown"),
+                              ("swt", "sw_thermal_slowdown"), ("pcap", "sw_power_cap")):
+                if r[key].lower().startswith("active"):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(r["sm"] for r in rows),
+                "sm_max_mhz": max(r["max"] for r in rows),
+                "power_w_max": max(r["power"] for r in rows),
+                "samples": len(rows), "reasons": sorted(reasons)}
+
+
+# ------------------------------------------------------------ the step
+
+
+class Chain:
+    """Device buffers of one clip and the op chain over them."""
+
+    def __init__(self, wl, device):
+        import torch
+        from dit_block_pass_b200 import workloads as W
+        self.wl = wl
+        self.dev = device
+        B, N, D, M, F = wl.B, wl.N, wl.D, wl.M, wl.F
+        g = lambda s, w: W.token_rows(wl, s, w, device=device)
+        self.x = g(W.S_X, D).view(B, N, D)
+        self.r = g(W.S_R, D).view(B, N, D)
+        self.qkv = g(W.S_QKV, 3 * D).view(B, N, 3 * D)
+        self.swi = g(W.S_SWIGLU, 2 * F)
+        prev, cur = W.cache_pair(wl, device=device)
+        self.prev, self.cur = prev.view(B, N, D), cur.view(B, N, D)
+        self.mod = W.modulation(wl, device=device)
+        self.wq, self.wk = W.norm_weights(wl, device=device)
+        self.pos = W.positions(wl, device=device)
+        self.y1 = torch.empty_like(self.x)
+        self.xo = torch.empty_like(self.x)
+        self.y2 = torch.empty_like(self.x)
+        self.out = torch.empty(M, F, dtype=torch.bfloat16, device=device)
+        import dit_block_pass_b200 as dbp
+        self.ws = torch.empty(dbp.cachedit_workspace_bytes(B, N, D), dtype=torch.uint8,
+                              device=device)
+        self.rel = torch.empty(B, dtype=torch.float64, device=device)
+        self.reuse = torch.empty(B, dtype=torch.uint8, device=device)
+        torch.cuda.synchronize(device)
+
+    def ops(self):
+        import dit_block_pass_b200 as dbp
+        wl, D, m = self.wl, self.wl.D, self.mod
+        grid = None if self.pos is not None else (wl.T, wl.Hg, wl.Wg)
+        return [
+            lambda: dbp.adaln_modulate(self.x, m[:, 0], m[:, 1], wl.eps, out=self.y1),
+            lambda: dbp.qk_rmsnorm_rope3d(self.qkv[:, :, :D], self.qkv[:, :, D:2 * D], self.wq,
+                                          self.wk, wl.H, wl.pairs, grid=grid, pos=self.pos,
+                                          theta=wl.theta, eps=wl.eps),
+            lambda: dbp.gated_residual_adaln(self.x, self.r, m[:, 2], m[:, 3], m[:, 4], wl.eps,
+                                             x_out=self.xo, y=self.y2),
+            lambda: dbp.swiglu(self.swi, out=self.out),
+            lambda: dbp.cachedit_residual_diff(self.prev, self.cur, wl.thresholds[0],
+                                               workspace=self.ws, rel=self.rel,
+                                               reuse=self.reuse),
+        ]
+
+    def launches_per_step(self):
+        import dit_block_pass_b200 as dbp
+        return sum(dbp.launch_counts[o] for o in OPS)
+
+
+def dist_setup(args):
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device(f"cuda:{local}"))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return world, rank, local
+
+
+def barrier_sync(world):
+    import torch
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize()
+
+
+def max_over_ranks(v: float, world: int) -> float:
+    if world == 1:
+        return v
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def time_device(chain, steps, warmup, world):
+    """Per-op and per-step device times (ms) over `steps` timed steps."""
+    import torch
+    ops = chain.ops()
+    for _ in range(warmup):
+        for op in ops:
+            op()
+    barrier_sync(world)
+    stream = torch.cuda.current_stream()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(ops) + 1)]
+          for _ in range(steps)]
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for s in range(steps):
+        ev[s][0].record(stream)
+        for i, op in enumerate(ops):
+            op()
+            ev[s][i + 1].record(stream)
+    stop.record(stream)
+    barrier_sync(world)
+    total_ms = start.elapsed_time(stop)
+    per_op = [sum(ev[s][i].elapsed_time(ev[s][i + 1]) for s in range(steps)) / steps
+              for i in range(len(ops))]
+    return total_ms, per_op
+
+
+def time_e2e(chain, steps, warmup, world):
+    """The same chain through the public API with inputs on the host: every
+    step copies its inputs host->device from pinned memory, runs the chain and
+    reads every output back device->host.  Returns (ms per step, h2d bytes,
+    d2h bytes)."""
+    import torch
+    c = chain
+    ins = [c.x, c.r, c.qkv, c.swi, c.prev, c.cur]
+    outs = [c.y1, c.qkv, c.xo, c.y2, c.out, c.rel, c.reuse]
+    host_in = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in ins]
+    for h, t in zip(host_in, ins):
+        h.copy_(t)
+    host_out = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in outs]
+    h2d = sum(t.numel() * t.element_size() for t in ins)
+    d2h = sum(t.numel() * t.element_size() for t in outs)
+    ops = c.ops()
+    stream = torch.cuda.current_stream()
+
+    def step():
+        for h, t in zip(host_in, ins):
+            t.copy_(h, non_blocking=True)
+        for op in ops:
+            op()
+        for h, t in zip(host_out, outs):
+            h.copy_(t, non_blocking=True)
+
+    for _ in range(warmup):
+        step()
+    barrier_sync(world)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(steps):
+        step()
+    b.record(stream)
+    barrier_sync(world)
+    ms = max_over_ranks(a.elapsed_time(b), world) / steps
+    del host_in, host_out
+    return ms, h2d, d2h
+
+
+# ------------------------------------------------------- CPU oracle leg
+
+
+def oracle_chain_rate(wl, budget_s: float, threads: int, steps: int = 1, pool_cap: int = 4096):
+    """Tokens/s of the fp64 oracle running the whole chain on token rows of
+    the workload, the rows split across `threads` host threads (the ctypes
+    calls release the GIL).  A pool of at most `pool_cap` random rows is
+    generated once; each of `steps` timed steps makes enough passes over the
+    pool to take about budget_s/steps.  Returns (tokens/s, pool rows, passes
+    per step, threads)."""
+    import concurrent.futures
+
+    import numpy as np
+    import torch
+
+    import oracle
+    from dit_block_pass_b200 import workloads as W
+    orc = oracle.default()
+    D, F, H, hd = wl.D, wl.F, wl.H, wl.hd
+    mod = W.modulation(wl).double().numpy()
+    wq, wk = (w.double().numpy() for w in W.norm_weights(wl))
+    pos_all = W.positions(wl)
+
+    def inputs(rows):
+        rid = torch.as_tensor(rows, dtype=torch.int64)
+        bits = W.bits_u16
+        x = bits(W.token_rows(wl, W.S_X, D, row_ids=rid))
+        r = bits(W.token_rows(wl, W.S_R, D, row_ids=rid))
+        qkv = bits(W.token_rows(wl, W.S_QKV, 3 * D, row_ids=rid))
+        swi = bits(W.token_rows(wl, W.S_SWIGLU, 2 * F, row_ids=rid))
+        prev, cur = (bits(t) for t in W.cache_pair(wl, row_ids=rid))
+        if pos_all is not None:
+            pos = pos_all.numpy()[rows]
+        else:
+            pos = orc.grid_positions(wl.T, wl.Hg, wl.Wg, 0, wl.N)[np.asarray(rows) % wl.N]
+        samp = np.asarray(rows) // wl.N
+        return x, r, qkv, swi, prev, cur, pos, samp
+
+    def chain(x, r, qkv, swi, prev, cur, pos, samp):
+        n = x.shape[0]
+        b = int(samp[0])
+        orc.adaln_modulate(x.reshape(1, n, D), mod[b:b + 1, 0], mod[b:b + 1, 1], wl.eps)
+        orc.qk_rmsnorm_rope3d(qkv[:, :D], wq, H, hd, pos, wl.pairs, wl.theta, wl.eps)
+        orc.qk_rmsnorm_rope3d(qkv[:, D:2 * D], wk, H, hd, pos, wl.pairs, wl.theta, wl.eps)
+        orc.gated_residual_adaln(x.reshape(1, n, D), r.reshape(1, n, D), mod[b:b + 1, 2],
+                                 mod[b:b + 1, 3], mod[b:b + 1, 4], wl.eps)
+        orc.swiglu(swi)
+        return orc.cachedit_sums(prev, cur)
+
+    rng = np.random.default_rng(0)
+    cal = inputs(np.sort(rng.choice(wl.M, 16, replace=False)))
+    t0 = time.perf_counter()
+    chain(*cal)
+    per_token = (time.perf_counter() - t0) / 16          # one thread
+    step_s = budget_s / max(1, steps)
+    want = max(threads, int(step_s / per_token * threads))
+    pool = min(want, pool_cap, wl.M)
+    passes = max(1, round(want / pool))
+    rows = np.sort(rng.choice(wl.M, pool, replace=False))
+    data = inputs(rows)
+    # rows of one sample per chunk (the modulation is per sample)
+    chunks = [c for c in np.array_split(np.arange(pool), threads) if c.size]
+    chunks = [part for c in chunks for part in np.split(c, np.nonzero(np.diff(data[7][c]))[0] + 1)]
+    total_t = 0.0
+    with concurrent.futures.ThreadPoolExecutor(max_workers=threads) as ex:
+        for _ in range(max(1, steps)):
+            t0 = time.perf_counter()
+            for _ in range(passes):
+                list(ex.map(lambda c: chain(*(a[c] for a in data)), chunks))
+            total_t += time.perf_counter() - t0
+    return pool * passes * max(1, steps) / total_t, pool, passes, threads
+
+
+def host_threads():
+    try:
+        return len(os.sched_getaffinity(0))
+    except Exception:
+        return os.cpu_count() or 1
+
+
+# ---------------------------------------------------------------- main
+
+
+def source_sha(kernel_file: str) -> str:
+    p = os.path.join(ROOT, "dit_block_pass_b200", "csrc", kernel_file)
+    with open(p, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def run_reference(args, wl):
+    """The reference arm: the fp64 oracle as it stands, on the host cores."""
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if world > 1 and rank != 0:
+        return
+    rate, pool, passes, threads = oracle_chain_rate(
+        wl, budget_s=args.ref_budget, threads=host_threads(), steps=max(1, args.steps))
+    per_step = pool * passes
+    line = {
+        "impl": "reference", "metric": METRIC, "value": rate, "unit": "tokens/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1000.0 * per_step / rate, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": wl.describe(), "tokens_per_step_sampled": per_step},
+        "cpu_baseline": {"value": rate, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+                         "sample": f"{pool} random token rows of the clip, {passes} pass(es) "
+                                   f"per step over them, {args.steps} steps, whole chain per "
+                                   f"row, rows split over {threads} host threads"},
+        "e2e": {"value": rate, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=250)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--config", default="h3_5s")
+    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--no-clocks", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--ref-budget", type=float, default=60.0)
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "native" and args.steps > 20:
+        raise SystemExit("use at least 3 warm-up steps for a timed run")
+
+    from dit_block_pass_b200 import workloads as W
+    wl = W.CONFIGS[args.config]
+    if args.impl == "reference":
+        run_reference(args, wl)
+        return
+
+    import torch
+    import dit_block_pass_b200 as dbp
+    from dit_block_pass_b200 import build
+    build.build()
+    world, rank, local = dist_setup(args)
+    dev = torch.device(f"cuda:{local}")
+    chain = Chain(wl, dev)
+
+    sampler = ClockSampler(local) if not args.no_clocks else None
+    if sampler:
+        sampler.__enter__()
+    try:
+        total_ms, per_op = time_device(chain, args.steps, args.warmup, world)
+    finally:
+        if sampler:
+            sampler.__exit__(None, None, None)
+    total_ms = max_over_ranks(total_ms, world)
+    ms_step = total_ms / args.steps
+    tokens = wl.M
+    value = world * tokens * args.steps / (total_ms / 1000.0)
+
+    peak, peak_kind = hbm_peak()
+    nbytes = algorithmic_bytes(wl)
+    ops = {}
+    for name, ms in zip(OPS, per_op):
+        gbs = nbytes[name] / (ms / 1000.0) / 1e9
+        ops[name] = {"ms": round(ms, 4), "GB/s": round(gbs, 1),
+                     "frac_of_peak": round(gbs / peak, 4),
+                     "tokens_per_s": round(tokens / (ms / 1000.0), 1)}
+    dom_ms = per_op[OPS.index(DOMINANT)]
+    achieved = nbytes[DOMINANT] / (dom_ms / 1000.0) / 1e9
+    tr = NCU_TRAFFIC.get(DOMINANT)
+    traffic = tr["bytes"] if tr and tr["sha"] == source_sha("swiglu.cu") else None
+    roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                "frac": round(achieved / peak, 4), "traffic": traffic,
+                "kernel": "swiglu_kernel", "peak_source": f"{peak_kind} hbm_gbs (copy)",
+                "algorithmic_bytes": nbytes[DOMINANT]}
+
+    e2e = None
+    if not args.no_e2e:
+        ms_e2e, h2d, d2h = time_e2e(chain, args.e2e_steps, 1, world)
+        e2e = {"value": world * tokens / (ms_e2e / 1000.0), "unit": "tokens/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "ms_per_step": round(ms_e2e, 3)}
+
+    cpu = None
+    if world == 1 and not args.no_cpu and rank == 0:
+        rate, pool, passes, threads = oracle_chain_rate(wl, args.cpu_budget, host_threads())
+        cpu = {"value": rate, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+               "sample": f"{pool} random token rows of the clip, {passes} pass(es) over them "
+                         f"(about {args.cpu_budget:.0f} s), whole chain per row, rows split "
+                         f"over {threads} host threads"}
+
+    clocks = sampler.summary() if sampler else None
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded counter-based generator, H3-shaped)",
+            "config": {"workload": wl.describe(),
+                       "chain": "adaln_modulate -> qk_rmsnorm_rope3d -> gated_residual_adaln "
+                                "-> swiglu, + cachedit_residual_diff",
+                       "tokens_per_step_per_gpu": tokens,
+                       "l2": "every input is larger than L2 (126 MB); no flush",
+                       "parallelism": f"{world} independent clip(s), one per GPU"},
+            "ops": ops, "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+            "gpu_launches": chain.launches_per_step() * args.steps, "clocks": clocks,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,2 +1,324 @@
-"""dit_block_pass_b200: B200-native (sm_100a) memory-bound operators of a dense
-single-stream video+audio DiT block."""
+"""dit_block_pass_b200: B200-native (sm_100a) memory-bound operators of one
+block of a dense single-stream video+audio diffusion transformer
+(MiniMax-H3 shaped).
+
+The compute lives in ``libdit_block.so`` (hand-written CUDA, C ABI declared in
+``include/dit_block.h``).  This module only marshals torch tensors into that
+ABI: it checks devices, dtypes and strides, passes raw pointers and the
+current CUDA stream, and turns a negative status into an exception.  There
+is no CPU fallback: without the built library every call raises.
+
+Operators (see the header for the definitions):
+  adaln_modulate, gated_residual_adaln, swiglu, qk_rmsnorm_rope3d,
+  cachedit_residual_diff, cachedit_residual_sums, cachedit_decide.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+from typing import Optional, Sequence
+
+import torch
+
+__all__ = [
+    "DitError", "library", "library_path", "adaln_modulate", "gated_residual_adaln", "swiglu",
+    "qk_rmsnorm_rope3d", "cachedit_workspace_bytes", "cachedit_residual_diff",
+    "cachedit_residual_sums", "cachedit_decide", "launch_counts", "F32", "BF16",
+]
+
+F32, BF16 = 0, 1
+_PKG = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_PKG, "libdit_block.so")
+_lib = None
+_lock = threading.Lock()
+
+# kernels launched per call of each entry point (for launch accounting)
+launch_counts = {
+    "adaln_modulate": 1, "gated_residual_adaln": 1, "swiglu": 1, "qk_rmsnorm_rope3d": 1,
+    "cachedit_residual_diff": 2, "cachedit_residual_sums": 2, "cachedit_decide": 1,
+}
+
+
+class DitError(RuntimeError):
+    def __init__(self, fn: str, status: int, msg: str):
+        super().__init__(f"{fn} failed with status {status}: {msg}")
+        self.status = status
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def library() -> ctypes.CDLL:
+    """The loaded C library; raises if it has not been built."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(_LIB_PATH):
+                raise RuntimeError(
+                    f"{_LIB_PATH} is missing: build it with "
+                    "`python -m dit_block_pass_b200.build` (nvcc, sm_100a). "
+                    "There is no CPU fallback.")
+            L = ctypes.CDLL(_LIB_PATH)
+            vp, i64, i32, dbl, sz = (ctypes.c_void_p, ctypes.c_int64, ctypes.c_int,
+                                     ctypes.c_double, ctypes.c_size_t)
+            L.dit_abi_version.restype = i32
+            L.dit_status_string.restype = ctypes.c_char_p
+            L.dit_status_string.argtypes = [i32]
+            L.dit_adaln_modulate.argtypes = [vp, vp, vp, vp, i32, i64, i32, i64, i32, dbl, vp]
+            L.dit_gated_residual_adaln.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, i64, i32,
+                                                   i64, i32, dbl, vp]
+            L.dit_swiglu.argtypes = [vp, vp, i64, i32, vp]
+            L.dit_qk_rmsnorm_rope3d.argtypes = [vp, vp, i64, vp, vp, i32, i32, i64, i32, i32,
+                                                i32, i32, i32, vp, i64, i32, i32, i32, dbl, dbl,
+                                                vp]
+            L.cachedit_workspace_bytes.restype = sz
+            L.cachedit_workspace_bytes.argtypes = [i32, i64, i32]
+            L.cachedit_residual_diff.argtypes = [vp, vp, i32, i64, i32, dbl, vp, vp, vp, sz, vp]
+            L.cachedit_residual_sums.argtypes = [vp, vp, i32, i64, i32, vp, vp, sz, vp]
+            L.cachedit_decide.argtypes = [vp, i32, i32, dbl, vp, vp, vp]
+            for name in ("dit_adaln_modulate", "dit_gated_residual_adaln", "dit_swiglu",
+                         "dit_qk_rmsnorm_rope3d", "cachedit_residual_diff",
+                         "cachedit_residual_sums", "cachedit_decide"):
+                getattr(L, name).restype = i32
+            _lib = L
+    return _lib
+
+
+def _call(name: str, *args) -> None:
+    L = library()
+    st = getattr(L, name)(*args)
+    if st != 0:
+        raise DitError(name, st, L.dit_status_string(st).decode())
+
+
+def _stream(t: torch.Tensor) -> int:
+    return torch.cuda.current_stream(t.device).cuda_stream
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def _need_cuda_bf16(name: str, t: torch.Tensor) -> None:
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor (there is no CPU path)")
+    if t.dtype != torch.bfloat16:
+        raise ValueError(f"{name} must be bfloat16, got {t.dtype}")
+
+
+def _mod_dtype(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return F32
+    if t.dtype == torch.bfloat16:
+        return BF16
+    raise ValueError(f"modulation/weight dtype must be float32 or bfloat16, got {t.dtype}")
+
+
+def _mod_views(B: int, D: int, *mods: torch.Tensor):
+    """Modulation vectors as [B, D] views (any batch stride, unit inner
+    stride); returns (dtype code, batch stride in elements)."""
+    dt = _mod_dtype(mods[0])
+    stride = None
+    for m in mods:
+        if m.dtype != mods[0].dtype or not m.is_cuda or m.device != mods[0].device:
+            raise ValueError("modulation vectors must share dtype and device")
+        if m.dim() == 1:
+            m = m.reshape(1, -1)
+        if m.shape[-1] != D or m.stride(-1) != 1 or m.shape[0] not in (1, B):
+            raise ValueError(f"modulation must be [B, D] (or [D]) with unit inner stride, got "
+                             f"{tuple(m.shape)}")
+        s = 0 if m.shape[0] == 1 else m.stride(0)
+        if stride is None:
+            stride = s
+        elif s != stride:
+            raise ValueError("modulation vectors must share one batch stride")
+    return dt, stride
+
+
+def _rows3(name: str, t: torch.Tensor):
+    if t.dim() != 3 or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous [B, N, D] tensor")
+    return t.shape
+
+
+# ---------------------------------------------------------------- operators
+
+
+def adaln_modulate(x: torch.Tensor, shift: torch.Tensor, scale: torch.Tensor, eps: float = 1e-6,
+                   out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """y = LN(x) * (1 + scale) + shift per sample; x [B, N, D] bf16."""
+    _need_cuda_bf16("x", x)
+    B, N, D = _rows3("x", x)
+    dt, ms = _mod_views(B, D, shift, scale)
+    y = torch.empty_like(x) if out is None else out
+    _need_cuda_bf16("out", y)
+    if y.shape != x.shape or not y.is_contiguous():
+        raise ValueError("out must match x")
+    _call("dit_adaln_modulate", x.data_ptr(), y.data_ptr(), shift.data_ptr(), scale.data_ptr(),
+          dt, ms, B, N, D, float(eps), _stream(x))
+    return y
+
+
+def gated_residual_adaln(x: torch.Tensor, r: torch.Tensor, gate: torch.Tensor,
+                         shift: torch.Tensor, scale: torch.Tensor, eps: float = 1e-6,
+                         x_out: Optional[torch.Tensor] = None, y: Optional[torch.Tensor] = None):
+    """x' = bf16(x + gate * r); y = AdaLN(x'). Returns (x', y)."""
+    _need_cuda_bf16("x", x)
+    _need_cuda_bf16("r", r)
+    B, N, D = _rows3("x", x)
+    if r.shape != x.shape or not r.is_contiguous():
+        raise ValueError("r must match x")
+    dt, ms = _mod_views(B, D, gate, shift, scale)
+    x_out = torch.empty_like(x) if x_out is None else x_out
+    y = torch.empty_like(x) if y is None else y
+    for nm, t in (("x_out", x_out), ("y", y)):
+        _need_cuda_bf16(nm, t)
+        if t.shape != x.shape or not t.is_contiguous():
+            raise ValueError(f"{nm} must match x")
+    _call("dit_gated_residual_adaln", x.data_ptr(), r.data_ptr(), x_out.data_ptr(), y.data_ptr(),
+          gate.data_ptr(), shift.data_ptr(), scale.data_ptr(), dt, ms, B, N, D, float(eps),
+          _stream(x))
+    return x_out, y
+
+
+def swiglu(inp: torch.Tensor, out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """out = silu(inp[..., :F]) * inp[..., F:]; inp [..., 2F] bf16 contiguous."""
+    _need_cuda_bf16("inp", inp)
+    if not inp.is_contiguous() or inp.shape[-1] % 2:
+        raise ValueError("inp must be contiguous with an even last dimension")
+    F = inp.shape[-1] // 2
+    M = inp.numel() // max(1, inp.shape[-1])
+    if out is None:
+        out = torch.empty(*inp.shape[:-1], F, dtype=inp.dtype, device=inp.device)
+    _need_cuda_bf16("out", out)
+    if out.numel() != M * F or not out.is_contiguous():
+        raise ValueError("out must be contiguous [..., F]")
+    _call("dit_swiglu", inp.data_ptr(), out.data_ptr(), M, F, _stream(inp))
+    return out
+
+
+def _token_rows(name: str, t: torch.Tensor, B: int, N: int, width: int) -> int:
+    """Row stride (elements) of a [B, N, width] view with unit inner stride and
+    uniformly strided token rows."""
+    _need_cuda_bf16(name, t)
+    if t.dim() != 3 or tuple(t.shape) != (B, N, width) or t.stride(2) != 1:
+        raise ValueError(f"{name} must be a [B, N, H*hd] view with unit inner stride")
+    rs = t.stride(1)
+    if B > 1 and t.stride(0) != N * rs:
+        raise ValueError(f"{name}: samples must be uniformly strided token rows")
+    return rs
+
+
+def qk_rmsnorm_rope3d(q: Optional[torch.Tensor], k: Optional[torch.Tensor],
+                      w_q: Optional[torch.Tensor], w_k: Optional[torch.Tensor], heads: int,
+                      pairs: Sequence[int], grid: Optional[Sequence[int]] = None,
+                      pos: Optional[torch.Tensor] = None, pos_offset: int = 0,
+                      theta: float = 10000.0, eps: float = 1e-6) -> None:
+    """In place on q and k ([B, N, H*hd] views, e.g. slices of a fused qkv
+    buffer): per-head RMSNorm with weight w, then 3D RoPE with pair split
+    ``pairs`` = (t, h, w).  Positions come from ``grid`` = (T, Hg, Wg) (token
+    n at global index pos_offset + n) or from ``pos`` [B*N, 3] int32."""
+    ref = q if q is not None else k
+    if ref is None:
+        raise ValueError("q and k cannot both be None")
+    B, N, width = ref.shape
+    if width % heads:
+        raise ValueError("last dimension must be heads * head_dim")
+    hd = width // heads
+    rs = None
+    for nm, t in (("q", q), ("k", k)):
+        if t is not None:
+            s = _token_rows(nm, t, B, N, width)
+            if rs is not None and s != rs:
+                raise ValueError("q and k must share the row stride")
+            rs = s
+    w_dt = None
+    for nm, t, w in (("w_q", q, w_q), ("w_k", k, w_k)):
+        if t is not None:
+            if w is None or w.numel() != hd or not w.is_contiguous() or not w.is_cuda:
+                raise ValueError(f"{nm} must be a contiguous CUDA [{hd}] tensor")
+            d = _mod_dtype(w)
+            if w_dt is not None and d != w_dt:
+                raise ValueError("w_q and w_k must share a dtype")
+            w_dt = d
+    if pos is not None:
+        if pos.dtype != torch.int32 or not pos.is_contiguous() or pos.numel() != B * N * 3 \
+                or not pos.is_cuda:
+            raise ValueError("pos must be a contiguous CUDA int32 [B*N, 3] tensor")
+        T = Hg = Wg = 0
+    else:
+        if grid is None:
+            raise ValueError("give grid=(T, Hg, Wg) or pos")
+        T, Hg, Wg = grid
+    pt, ph, pw = pairs
+    _call("dit_qk_rmsnorm_rope3d", _ptr(q), _ptr(k), rs, _ptr(w_q), _ptr(w_k), w_dt, B, N, heads,
+          hd, T, Hg, Wg, _ptr(pos), int(pos_offset), pt, ph, pw, float(theta), float(eps),
+          _stream(ref))
+
+
+def cachedit_workspace_bytes(B: int, N: int, D: int) -> int:
+    return int(library().cachedit_workspace_bytes(B, N, D))
+
+
+def _workspace(prev: torch.Tensor, workspace: Optional[torch.Tensor]) -> torch.Tensor:
+    B, N, D = prev.shape
+    need = cachedit_workspace_bytes(B, N, D)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=prev.device)
+    if workspace.numel() * workspace.element_size() < need or not workspace.is_contiguous():
+        raise ValueError(f"workspace needs {need} contiguous bytes")
+    return workspace
+
+
+def cachedit_residual_diff(prev: torch.Tensor, cur: torch.Tensor, threshold: float,
+                           workspace: Optional[torch.Tensor] = None, rel: Optional[torch.Tensor] = None,
+                           reuse: Optional[torch.Tensor] = None):
+    """Per sample rel = sum|cur-prev| / sum|prev| and reuse = rel < threshold.
+    Returns device tensors (rel [B] float64, reuse [B] uint8)."""
+    _need_cuda_bf16("prev", prev)
+    _need_cuda_bf16("cur", cur)
+    B, N, D = _rows3("prev", prev)
+    if cur.shape != prev.shape or not cur.is_contiguous():
+        raise ValueError("cur must match prev")
+    ws = _workspace(prev, workspace)
+    rel = torch.empty(B, dtype=torch.float64, device=prev.device) if rel is None else rel
+    reuse = torch.empty(B, dtype=torch.uint8, device=prev.device) if reuse is None else reuse
+    _call("cachedit_residual_diff", prev.data_ptr(), cur.data_ptr(), B, N, D, float(threshold),
+          rel.data_ptr(), reuse.data_ptr(), ws.data_ptr(), ws.numel() * ws.element_size(),
+          _stream(prev))
+    return rel, reuse
+
+
+def cachedit_residual_sums(prev: torch.Tensor, cur: torch.Tensor,
+                           workspace: Optional[torch.Tensor] = None,
+                           sums: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """[B, 2] float64 device tensor: (sum|cur-prev|, sum|prev|) per sample."""
+    _need_cuda_bf16("prev", prev)
+    _need_cuda_bf16("cur", cur)
+    B, N, D = _rows3("prev", prev)
+    if cur.shape != prev.shape or not cur.is_contiguous():
+        raise ValueError("cur must match prev")
+    ws = _workspace(prev, workspace)
+    sums = torch.empty(B, 2, dtype=torch.float64, device=prev.device) if sums is None else sums
+    _call("cachedit_residual_sums", prev.data_ptr(), cur.data_ptr(), B, N, D, sums.data_ptr(),
+          ws.data_ptr(), ws.numel() * ws.element_size(), _stream(prev))
+    return sums
+
+
+def cachedit_decide(sums: torch.Tensor, threshold: float):
+    """sums: [R, B, 2] float64 device tensor of partial sums (R shards).
+    Returns (rel [B] float64, reuse [B] uint8) device tensors."""
+    if sums.dtype != torch.float64 or not sums.is_cuda or not sums.is_contiguous():
+        raise ValueError("sums must be a contiguous CUDA float64 tensor")
+    if sums.dim() == 2:
+        sums = sums.unsqueeze(0)
+    R, B, two = sums.shape
+    if two != 2:
+        raise ValueError("sums must be [R, B, 2]")
+    rel = torch.empty(B, dtype=torch.float64, device=sums.device)
+    reuse = torch.empty(B, dtype=torch.uint8, device=sums.device)
+    _call("cachedit_decide", sums.data_ptr(), R, B, float(threshold), rel.data_ptr(),
+          reuse.data_ptr(), _stream(sums))
+    return rel, reuse

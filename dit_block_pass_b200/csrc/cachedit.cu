@@ -1,0 +1,199 @@
+// cachedit.cu -- Cache-DiT residual-difference check, one pass over HBM.
+//
+// "MiniMax-H3 no SGLang em H200", section "Só com três camadas de aceleração
+// somadas chega-se a 6 vezes", Cache-DiT paragraph: cached results are reused
+// between neighbouring denoising steps when a residual-difference threshold
+// allows it (0.04 conservative, 0.08 in the more aggressive stride mode).
+// The check is the relative L1 difference of two residual tensors.
+//
+// Design: a partial-sum kernel on a (G, B) grid streams prev and cur once;
+// thread sums are fp32 per 8-element vector (|cur - prev| of two bf16 values
+// is exact in fp32 unless their exponents are more than 16 apart) and fp64
+// above that.  Each CTA reduces with a fixed butterfly and writes its fp64
+// pair to the workspace as part[g][b][2].  A one-warp-per-sample kernel then
+// adds the G pairs in a fixed order and takes the decision in fp64.  There
+// are no floating-point atomics, so the result is identical run to run.
+#include <math.h>
+
+#include "common.cuh"
+
+namespace dit {
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kUnroll = 4;
+constexpr int kSlotCap = 2048;  // partial-sum slots per sample in a workspace
+
+__global__ void __launch_bounds__(kThreads)
+cachedit_partials_kernel(const uint4* __restrict__ prev, const uint4* __restrict__ cur,
+                         int64_t nvs, double* __restrict__ part, int B) {
+    const int g = blockIdx.x, b = blockIdx.y, G = gridDim.x;
+    const uint4* P = prev + static_cast<int64_t>(b) * nvs;
+    const uint4* C = cur + static_cast<int64_t>(b) * nvs;
+    const int64_t step = static_cast<int64_t>(G) * kThreads;
+    double acc_n = 0.0, acc_d = 0.0;
+    for (int64_t v = static_cast<int64_t>(g) * kThreads + threadIdx.x; v < nvs;
+         v += kUnroll * step) {
+        uint4 pv[kUnroll], cv[kUnroll];
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) {
+            if (v + u * step < nvs) {
+                pv[u] = ld_stream(P + v + u * step);
+                cv[u] = ld_stream(C + v + u * step);
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) {
+            if (v + u * step < nvs) {
+                float fp[8], fc[8];
+                unpack8(pv[u], fp);
+                unpack8(cv[u], fc);
+                float sn = 0.0f, sd = 0.0f;
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    sn += fabsf(fc[i] - fp[i]);
+                    sd += fabsf(fp[i]);
+                }
+                acc_n += static_cast<double>(sn);
+                acc_d += static_cast<double>(sd);
+            }
+        }
+    }
+    acc_n = warp_sum(acc_n);
+    acc_d = warp_sum(acc_d);
+    __shared__ double sh[2][kThreads / 32];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    if (lane == 0) {
+        sh[0][warp] = acc_n;
+        sh[1][warp] = acc_d;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        double n = 0.0, d = 0.0;
+#pragma unroll
+        for (int w = 0; w < kThreads / 32; ++w) {
+            n += sh[0][w];
+            d += sh[1][w];
+        }
+        double* out = part + (static_cast<int64_t>(g) * B + b) * 2;
+        out[0] = n;
+        out[1] = d;
+    }
+}
+
+// One warp per sample: add R partial pairs (part[r][b][2]) lane-strided and
+// through a fixed butterfly, then write the sums and/or the decision.
+__global__ void cachedit_finalize_kernel(const double* __restrict__ part, int R, int B,
+                                         double threshold, double* sums_out, double* rel_out,
+                                         uint8_t* reuse_out) {
+    const int b = blockIdx.x, lane = threadIdx.x;
+    double n = 0.0, d = 0.0;
+    for (int r = lane; r < R; r += 32) {
+        n += part[(static_cast<int64_t>(r) * B + b) * 2];
+        d += part[(static_cast<int64_t>(r) * B + b) * 2 + 1];
+    }
+    n = warp_sum(n);
+    d = warp_sum(d);
+    if (lane == 0) {
+        if (sums_out) {
+            sums_out[2 * b] = n;
+            sums_out[2 * b + 1] = d;
+        }
+        if (rel_out) {
+            double rel;
+            if (d == 0.0) rel = (n == 0.0) ? 0.0 : INFINITY;
+            else rel = n / d;
+            rel_out[b] = rel;
+            reuse_out[b] = rel < threshold ? 1 : 0;
+        }
+    }
+}
+
+int partial_slots(int B, int64_t nvs) {
+    const int sms = device_sm_count();
+    if (sms <= 0) return 0;
+    const int occ = occupancy(reinterpret_cast<const void*>(cachedit_partials_kernel), kThreads, 0);
+    int64_t g = static_cast<int64_t>(sms) * occ / B;
+    const int64_t need = (nvs + kThreads - 1) / kThreads;
+    if (g > need) g = need;
+    if (g > kSlotCap) g = kSlotCap;
+    if (g < 1) g = 1;
+    return static_cast<int>(g);
+}
+
+int check_inputs(const uint16_t* prev, const uint16_t* cur, int B, int64_t N, int D) {
+    if (!prev || !cur) return DIT_ERR_NULL;
+    if (B < 1 || N < 0 || D <= 0) return DIT_ERR_SHAPE;
+    if (B > 65535 || N > (INT64_MAX / 8) / D / B) return DIT_ERR_SHAPE;
+    if (D % 8 || !aligned16(prev) || !aligned16(cur)) return DIT_ERR_ALIGN;
+    return DIT_OK;
+}
+
+int run_partials(const uint16_t* prev, const uint16_t* cur, int B, int64_t N, int D,
+                 void* workspace, size_t workspace_bytes, cudaStream_t stream, int* slots) {
+    if (!workspace || !aligned16(workspace)) return DIT_ERR_WORKSPACE;
+    if (workspace_bytes < cachedit_workspace_bytes(B, N, D)) return DIT_ERR_WORKSPACE;
+    const int64_t nvs = N * D / 8;
+    const int G = partial_slots(B, nvs);
+    if (G < 1) return DIT_ERR_LAUNCH;
+    dim3 grid(static_cast<unsigned>(G), static_cast<unsigned>(B));
+    cachedit_partials_kernel<<<grid, kThreads, 0, stream>>>(
+        reinterpret_cast<const uint4*>(prev), reinterpret_cast<const uint4*>(cur), nvs,
+        static_cast<double*>(workspace), B);
+    *slots = G;
+    return launch_status();
+}
+
+}  // namespace
+}  // namespace dit
+
+extern "C" size_t cachedit_workspace_bytes(int B, int64_t N, int D) {
+    (void)N;
+    (void)D;
+    if (B < 1) return 0;
+    return static_cast<size_t>(B) * dit::kSlotCap * 2 * sizeof(double);
+}
+
+extern "C" int cachedit_residual_diff(const uint16_t* prev, const uint16_t* cur, int B, int64_t N,
+                                      int D, double threshold, double* rel_out,
+                                      uint8_t* reuse_out, void* workspace,
+                                      size_t workspace_bytes, void* stream) {
+    using namespace dit;
+    int st = check_inputs(prev, cur, B, N, D);
+    if (st) return st;
+    if (!rel_out || !reuse_out) return DIT_ERR_NULL;
+    if (isnan(threshold)) return DIT_ERR_VALUE;
+    int G = 0;
+    if ((st = run_partials(prev, cur, B, N, D, workspace, workspace_bytes, as_stream(stream), &G)))
+        return st;
+    cachedit_finalize_kernel<<<B, 32, 0, as_stream(stream)>>>(
+        static_cast<const double*>(workspace), G, B, threshold, nullptr, rel_out, reuse_out);
+    return launch_status();
+}
+
+extern "C" int cachedit_residual_sums(const uint16_t* prev, const uint16_t* cur, int B, int64_t N,
+                                      int D, double* sums_out, void* workspace,
+                                      size_t workspace_bytes, void* stream) {
+    using namespace dit;
+    int st = check_inputs(prev, cur, B, N, D);
+    if (st) return st;
+    if (!sums_out) return DIT_ERR_NULL;
+    int G = 0;
+    if ((st = run_partials(prev, cur, B, N, D, workspace, workspace_bytes, as_stream(stream), &G)))
+        return st;
+    cachedit_finalize_kernel<<<B, 32, 0, as_stream(stream)>>>(
+        static_cast<const double*>(workspace), G, B, 0.0, sums_out, nullptr, nullptr);
+    return launch_status();
+}
+
+extern "C" int cachedit_decide(const double* sums, int R, int B, double threshold,
+                               double* rel_out, uint8_t* reuse_out, void* stream) {
+    using namespace dit;
+    if (!sums || !rel_out || !reuse_out) return DIT_ERR_NULL;
+    if (R < 1 || B < 1 || B > 65535) return DIT_ERR_SHAPE;
+    if (reinterpret_cast<uintptr_t>(sums) % 8) return DIT_ERR_ALIGN;
+    if (isnan(threshold)) return DIT_ERR_VALUE;
+    cachedit_finalize_kernel<<<B, 32, 0, dit::as_stream(stream)>>>(sums, R, B, threshold, nullptr,
+                                                                  rel_out, reuse_out);
+    return launch_status();
+}

@@ -162,11 +162,14 @@ def _normal_f32(seed: int, stream: int, idx: torch.Tensor, sigma: float, mean: f
 
 def normal(seed: int, stream: int, rows: int, cols: int, sigma: float = 1.0, mean: float = 0.0,
            dtype=torch.bfloat16, device="cpu", row_ids: Optional[torch.Tensor] = None,
-           chunk: int = 1 << 24) -> torch.Tensor:
+           chunk: Optional[int] = None) -> torch.Tensor:
     """A [rows, cols] tensor (or [len(row_ids), cols] with row_ids) of
     ~N(mean, sigma^2) values of the given dtype; element (r, c) has index
-    r*cols + c in the stream."""
+    r*cols + c in the stream.  `chunk` elements are hashed at a time (only
+    speed and memory depend on it)."""
     device = torch.device(device)
+    if chunk is None:
+        chunk = (1 << 24) if device.type == "cuda" else (1 << 20)
     if row_ids is not None:
         row_ids = row_ids.to(device=device, dtype=torch.int64)
         out_rows = row_ids.numel()

@@ -1,0 +1,205 @@
+/*
+ * dit_block.h -- C ABI of libdit_block.so: the per-block memory-bound
+ * operators of a dense single-stream video+audio diffusion transformer
+ * (MiniMax-H3 shaped), as hand-written CUDA kernels for B200 (sm_100a).
+ *
+ * Sources.  The operators are the ones the SGLang-Diffusion H200 report fuses
+ * and the Cache-DiT check it uses:
+ *   "MiniMax-H3 no SGLang em H200" (news.cocoloop.cn, summary of the LMSYS
+ *   report), section "Só com três camadas de aceleração somadas chega-se a 6
+ *   vezes": the fused AdaLN update, gated residual, SwiGLU activation and
+ *   QK RMSNorm with 3D RoPE ("changes no calculation result"), and Cache-DiT
+ *   reuse decided by a residual-difference threshold (0.04 conservative,
+ *   0.08 stride mode);
+ *   "SGLang acelera MiniMax-H3 em GPUs H200 e redefine geração de vídeo por
+ *   IA" (ceviu.com.br), first paragraph: fused kernels for AdaLN, SwiGLU,
+ *   QK RMSNorm and 3D RoPE cut memory traffic and kernel launches;
+ *   "MiniMax H3 mở trọng số: H3-Base có gì và còn thiếu gì?"
+ *   (studioglobal.ai), section "Kiến trúc: tạo hình và tiếng trong cùng một
+ *   luồng": a dense single-stream transformer whose AdaLN-branch outputs can
+ *   be precomputed and cached (so modulation vectors are inputs here).
+ * The pages give names, not formulas; each function states the definition it
+ * computes.
+ *
+ * Conventions for every entry point.
+ *  - bf16 tensors are passed as uint16_t* (raw bf16 bit patterns) in DEVICE
+ *    memory, token-major and contiguous in the feature dimension.
+ *  - `stream` is a cudaStream_t (NULL = the legacy default stream).  Every
+ *    call is asynchronous on that stream; outputs are valid once the stream
+ *    has reached the call.
+ *  - The caller owns every buffer and the stream.  The library allocates no
+ *    memory and keeps no state between calls except a per-device cache of
+ *    device attributes, so calls are thread-safe.
+ *  - Arguments are checked on the host before anything is launched.  A bad
+ *    argument returns a negative dit_status and launches nothing; nothing
+ *    aborts, nothing throws.  DIT_ERR_LAUNCH carries a CUDA launch error
+ *    (cudaGetLastError after the launch); it may also report an earlier
+ *    asynchronous error already pending on the device.
+ *  - An empty problem (B == 0 or N == 0 / M == 0) returns DIT_OK and launches
+ *    nothing, except where a function says otherwise.
+ *  - Pointer alignment: every bf16 tensor pointer must be 16-byte aligned,
+ *    and row lengths must be multiples of 8 elements, because each kernel
+ *    moves rows as 128-bit vectors.  There is no scalar or CPU fallback.
+ */
+#ifndef DIT_BLOCK_H
+#define DIT_BLOCK_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    DIT_OK = 0,
+    DIT_ERR_NULL = -1,      /* a required pointer is NULL */
+    DIT_ERR_SHAPE = -2,     /* a size is negative, zero where it may not be, or too large */
+    DIT_ERR_ALIGN = -3,     /* a pointer or row length breaks the 16-byte rule */
+    DIT_ERR_DTYPE = -4,     /* unknown dit_dtype */
+    DIT_ERR_LAUNCH = -5,    /* CUDA reported an error at launch */
+    DIT_ERR_WORKSPACE = -6, /* workspace NULL or smaller than required */
+    DIT_ERR_OVERLAP = -7,   /* buffers overlap where they may not */
+    DIT_ERR_VALUE = -8      /* a scalar argument (eps, theta) is out of range */
+} dit_status;
+
+/* Element type of modulation vectors and norm weights. */
+typedef enum { DIT_F32 = 0, DIT_BF16 = 1 } dit_dtype;
+
+/* Largest model width the row kernels accept (a row is held in registers). */
+#define DIT_MAX_D 8192
+
+/* ABI version, bumped on any signature change. */
+int dit_abi_version(void);
+
+/* Human-readable name of a dit_status value (static string). */
+const char* dit_status_string(int status);
+
+/*
+ * AdaLN modulation (the fused "AdaLN update").
+ *   For every token row x (D values) of sample b:
+ *     mu  = mean(x),  var = mean((x - mu)^2)            (biased variance)
+ *     y_d = (x_d - mu) / sqrt(var + eps) * (1 + scale_b[d]) + shift_b[d]
+ *   Non-affine LayerNorm; the (1 + scale) form makes zero modulation a plain
+ *   LayerNorm.  Statistics in fp32, one rounding to bf16 per output.
+ * x, y        [B, N, D] bf16, 16-byte aligned.  y may equal x (in place) but
+ *             must not partially overlap it.
+ * shift,scale modulation of dtype mod_dtype; sample b's D values start at
+ *             element b * mod_batch_stride (>= 0; 0 broadcasts one vector;
+ *             6*D walks a [B, 6, D] AdaLN-branch output).  Naturally aligned.
+ * D           multiple of 8, 8 <= D <= DIT_MAX_D.  eps >= 0.
+ */
+int dit_adaln_modulate(const uint16_t* x, uint16_t* y,
+                       const void* shift, const void* scale, int mod_dtype,
+                       int64_t mod_batch_stride,
+                       int B, int64_t N, int D, double eps, void* stream);
+
+/*
+ * Gated residual fused with the next AdaLN.
+ *   x'_d = bf16(x_d + gate_b[d] * r_d)          (one rounding; the new residual)
+ *   y    = AdaLN(x'; shift_b, scale_b, eps)     (as dit_adaln_modulate, on the
+ *                                                ROUNDED x', so the fused op
+ *                                                equals the unfused chain)
+ * x'  is computed so that it is bit-identical to a single round-to-nearest-
+ * even of the exact x + gate*r.
+ * x, r, x_out, y  [B, N, D] bf16, 16-byte aligned.  x_out may equal x (in
+ *                 place); otherwise no two of x, r, x_out, y may overlap.
+ * gate, shift, scale  as in dit_adaln_modulate (same dtype and batch stride).
+ */
+int dit_gated_residual_adaln(const uint16_t* x, const uint16_t* r,
+                             uint16_t* x_out, uint16_t* y,
+                             const void* gate, const void* shift, const void* scale,
+                             int mod_dtype, int64_t mod_batch_stride,
+                             int B, int64_t N, int D, double eps, void* stream);
+
+/*
+ * SwiGLU activation between the MLP up-projection and down-projection.
+ *   out[m, j] = silu(in[m, j]) * in[m, F + j],   silu(a) = a / (1 + exp(-a))
+ * (first half of each row is the gate, second half the linear branch).
+ * in   [M, 2F] bf16, 16-byte aligned.    out [M, F] bf16, 16-byte aligned,
+ *      disjoint from in.                 F multiple of 8, F > 0, M >= 0.
+ */
+int dit_swiglu(const uint16_t* in, uint16_t* out, int64_t M, int F, void* stream);
+
+/*
+ * Per-head QK RMSNorm fused with 3D (t, h, w) rotary position embedding,
+ * in place on q and k.
+ *   For each token and head (hd values x, weight w of the tensor):
+ *     u_j = x_j / sqrt(mean_j(x_j^2) + eps) * w_j
+ *   The hd/2 rotation pairs are (u_{2p}, u_{2p+1}).  Pairs [0, pairs_t) use
+ *   the token's t position, the next pairs_h its h position, the last pairs_w
+ *   its w position.  Pair i of an axis with P pairs turns by
+ *     phi = pos_axis * theta^(-2i / (2P))
+ *   as (u0, u1) -> (u0 cos phi - u1 sin phi, u0 sin phi + u1 cos phi).
+ *   Angles are formed and reduced in fp64, sin/cos taken in fp32.
+ * q, k        token rows: token i (i = b*N + n) of q starts at q + i*row_stride
+ *             elements and holds H*hd values; same for k.  Either may be NULL
+ *             (then only the other is processed), not both.  16-byte
+ *             aligned; q and k rows must not overlap.
+ * row_stride  elements between tokens, multiple of 8, >= H*hd (3*H*hd for a
+ *             fused qkv buffer).
+ * w_q, w_k    [hd] weights of dtype w_dtype (needed for each non-NULL tensor).
+ * hd          one of 32, 64, 128, 256; pairs_t + pairs_h + pairs_w == hd/2,
+ *             each >= 1.  H >= 1.
+ * pos         device [B*N, 3] int32 (t, h, w) per token, or NULL: then token
+ *             n of every sample sits at global grid index g = pos_offset + n
+ *             of a row-major (T, Hg, Wg) grid, t = g/(Hg*Wg), h = (g/Wg)%Hg,
+ *             w = g%Wg, and pos_offset + N <= T*Hg*Wg is required (a sequence
+ *             shard passes its first token's global index as pos_offset).
+ * theta > 0, eps >= 0.
+ */
+int dit_qk_rmsnorm_rope3d(uint16_t* q, uint16_t* k, int64_t row_stride,
+                          const void* w_q, const void* w_k, int w_dtype,
+                          int B, int64_t N, int H, int hd,
+                          int T, int Hg, int Wg, const int32_t* pos, int64_t pos_offset,
+                          int pairs_t, int pairs_h, int pairs_w,
+                          double theta, double eps, void* stream);
+
+/*
+ * Cache-DiT residual-difference check between neighbouring denoising steps.
+ *   Per sample b:  rel_b   = sum_{n,d} |cur - prev| / sum_{n,d} |prev|
+ *                  reuse_b = rel_b < threshold       (strict)
+ *   0/0 reads as rel = 0 (identical residuals are reusable); x/0 as +inf.
+ *   |cur - prev| and |prev| are summed in fp32 per 8-element vector and in
+ *   fp64 above that, in a fixed order: the result is deterministic run to run
+ *   on a given device.
+ * prev, cur   [B, N, D] bf16, 16-byte aligned.  D multiple of 8.
+ * rel_out     device [B] double;  reuse_out device [B] uint8 (0 or 1).
+ * workspace   device scratch of at least cachedit_workspace_bytes(B, N, D)
+ *             bytes, 16-byte aligned; its contents on entry do not matter.
+ *             Calls that share a workspace must be ordered on the device.
+ * N == 0 is allowed and yields rel = 0, reuse = threshold > 0.
+ */
+size_t cachedit_workspace_bytes(int B, int64_t N, int D);
+int cachedit_residual_diff(const uint16_t* prev, const uint16_t* cur,
+                           int B, int64_t N, int D, double threshold,
+                           double* rel_out, uint8_t* reuse_out,
+                           void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * The two sums of the Cache-DiT check without the decision, for a sequence
+ * shard: sums_out[b][0] = sum |cur - prev|, sums_out[b][1] = sum |prev| over
+ * this call's N*D elements of sample b (device [B][2] double).  Ranks that
+ * each hold a shard exchange these 2*B doubles (an all-gather) and call
+ * cachedit_decide on the gathered [R][B][2] array, so every rank reaches the
+ * same decision.  Arguments otherwise as cachedit_residual_diff.
+ */
+int cachedit_residual_sums(const uint16_t* prev, const uint16_t* cur,
+                           int B, int64_t N, int D, double* sums_out,
+                           void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Decision from R sets of partial sums: sums is device [R][B][2] double;
+ * per sample the R partials are added in a fixed order that depends only on
+ * R (so ranks that hold the same gathered array reach bit-identical results),
+ * then rel and reuse follow as in cachedit_residual_diff.  R >= 1, B >= 1.
+ * sums must be 8-byte aligned.
+ */
+int cachedit_decide(const double* sums, int R, int B, double threshold,
+                    double* rel_out, uint8_t* reuse_out, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DIT_BLOCK_H */

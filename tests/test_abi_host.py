@@ -1,0 +1,169 @@
+"""The C ABI without a GPU: the library loads, exports every function the
+header declares, and rejects bad arguments on the host before touching CUDA
+(only checks that return before any CUDA call are exercised here)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from conftest import ROOT
+
+HEADER = os.path.join(ROOT, "include", "dit_block.h")
+E = {"NULL": -1, "SHAPE": -2, "ALIGN": -3, "DTYPE": -4, "WORKSPACE": -6, "OVERLAP": -7,
+     "VALUE": -8}
+A = 0x10000  # a 16-byte aligned fake address: never dereferenced by these calls
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    src = re.sub(r"//[^\n]*", "", src)
+    names = re.findall(r"^[A-Za-z_][\w\s\*]*?\b([A-Za-z_]\w*)\s*\([^;{]*\)\s*;", src, flags=re.M)
+    return sorted(set(names))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from dit_block_pass_b200 import build
+    import dit_block_pass_b200 as dbp
+    build.build()
+    return dbp.library()
+
+
+def test_header_declares_the_hot_path():
+    names = declared_functions()
+    for n in ("dit_adaln_modulate", "dit_gated_residual_adaln", "dit_swiglu",
+              "dit_qk_rmsnorm_rope3d", "cachedit_residual_diff", "cachedit_workspace_bytes",
+              "cachedit_residual_sums", "cachedit_decide", "dit_status_string",
+              "dit_abi_version"):
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+
+
+def test_header_is_plain_c():
+    """The header compiles as C99 with no CUDA include path."""
+    import subprocess
+    import tempfile
+    with tempfile.TemporaryDirectory() as d:
+        c = os.path.join(d, "t.c")
+        open(c, "w").write('#include "dit_block.h"\nint main(void){return dit_abi_version();}\n')
+        subprocess.run(["gcc", "-std=c99", "-Wall", "-Werror", "-fsyntax-only",
+                        "-I", os.path.dirname(HEADER), c], check=True)
+
+
+def test_status_strings_and_version(lib):
+    assert lib.dit_abi_version() == 1
+    assert lib.dit_status_string(0) == b"ok"
+    for code in E.values():
+        assert lib.dit_status_string(code) not in (b"ok", b"unknown status")
+
+
+def test_workspace_size_is_host_only(lib):
+    assert lib.cachedit_workspace_bytes(1, 124992, 5120) > 0
+    assert lib.cachedit_workspace_bytes(2, 0, 8) == 2 * lib.cachedit_workspace_bytes(1, 0, 8)
+    assert lib.cachedit_workspace_bytes(0, 10, 8) == 0
+
+
+def test_swiglu_argument_errors(lib):
+    f = lib.dit_swiglu
+    assert f(None, A, 4, 8, None) == E["NULL"]
+    assert f(A, A + 0x1000, -1, 8, None) == E["SHAPE"]
+    assert f(A, A + 0x1000, 4, 0, None) == E["SHAPE"]
+    assert f(A, A + 0x1000, 4, 12, None) == E["ALIGN"]         # F % 8
+    assert f(A + 2, A + 0x1000, 4, 8, None) == E["ALIGN"]      # misaligned in
+    assert f(A, A + 16, 4, 8, None) == E["OVERLAP"]            # out inside in
+    assert f(A, A + 0x1000, 0, 8, None) == 0                   # empty: no launch
+
+
+def test_adaln_argument_errors(lib):
+    f = lib.dit_adaln_modulate
+    ok = (A, A + 0x100000, A + 0x200000, A + 0x300000, 0, 0, 1, 4, 64, 1e-6, None)
+
+    def call(**kw):
+        names = ["x", "y", "shift", "scale", "dt", "ms", "B", "N", "D", "eps", "s"]
+        a = dict(zip(names, ok))
+        a.update(kw)
+        return f(*[a[n] for n in names])
+
+    assert call(x=None) == E["NULL"]
+    assert call(shift=None) == E["NULL"]
+    assert call(D=60) == E["ALIGN"]
+    assert call(D=8200) == E["SHAPE"]
+    assert call(B=-1) == E["SHAPE"]
+    assert call(dt=7) == E["DTYPE"]
+    assert call(eps=-1.0) == E["VALUE"]
+    assert call(eps=float("nan")) == E["VALUE"]
+    assert call(x=A + 8) == E["ALIGN"]
+    assert call(scale=A + 0x300002) == E["ALIGN"]              # fp32 scale not 4-aligned
+    assert call(y=A + 64) == E["OVERLAP"]                      # partial overlap
+    assert call(N=0) == 0
+    g = lib.dit_gated_residual_adaln
+    base = [A, A + 0x100000, A + 0x200000, A + 0x300000, A + 0x400000, A + 0x500000,
+            A + 0x600000, 0, 0, 1, 4, 64, 1e-6, None]
+    bad = list(base)
+    bad[1] = A  # r == x
+    assert g(*bad) == E["OVERLAP"]
+    bad = list(base)
+    bad[2] = A  # x_out == x is allowed (in place): empty N makes it a no-op
+    bad[10] = 0
+    assert g(*bad) == 0
+    bad = list(base)
+    bad[4] = None
+    assert g(*bad) == E["NULL"]
+
+
+def test_qk_argument_errors(lib):
+    f = lib.dit_qk_rmsnorm_rope3d
+    names = ["q", "k", "rs", "wq", "wk", "wdt", "B", "N", "H", "hd", "T", "Hg", "Wg", "pos",
+             "off", "pt", "ph", "pw", "theta", "eps", "s"]
+    ok = dict(zip(names, [A, A + 2 * 256, 768, A + 0x900000, A + 0x900100, 0, 1, 48, 4, 64, 2, 4,
+                          6, None, 0, 12, 10, 10, 1e4, 1e-6, None]))
+
+    def call(**kw):
+        a = dict(ok)
+        a.update(kw)
+        return f(*[a[n] for n in names])
+
+    assert call(q=None, k=None) == E["NULL"]
+    assert call(wq=None) == E["NULL"]
+    assert call(hd=48, H=4) == E["SHAPE"]                       # unsupported head dim
+    assert call(pt=11) == E["SHAPE"]                            # pairs do not sum to hd/2
+    assert call(rs=200) == E["SHAPE"]                           # stride < H*hd
+    assert call(rs=772) == E["ALIGN"]
+    assert call(N=49) == E["SHAPE"]                             # beyond the grid
+    assert call(off=1) == E["SHAPE"]
+    assert call(k=A + 2 * 128) == E["OVERLAP"]                  # k inside q's row
+    assert call(theta=0.0) == E["VALUE"]
+    assert call(wdt=3) == E["DTYPE"]
+    assert call(q=A + 4) == E["ALIGN"]
+    assert call(N=0) == 0
+
+
+def test_cachedit_argument_errors(lib):
+    f = lib.cachedit_residual_diff
+    ws = lib.cachedit_workspace_bytes(1, 4, 64)
+    assert f(None, A, 1, 4, 64, 0.04, A, A, A, ws, None) == E["NULL"]
+    assert f(A, A, 0, 4, 64, 0.04, A, A, A, ws, None) == E["SHAPE"]
+    assert f(A, A, 1, 4, 60, 0.04, A, A, A, ws, None) == E["ALIGN"]
+    assert f(A, A, 1, 4, 64, 0.04, None, A, A, ws, None) == E["NULL"]
+    assert f(A, A, 1, 4, 64, float("nan"), A, A, A, ws, None) == E["VALUE"]
+    assert f(A, A, 1, 4, 64, 0.04, A, A, None, ws, None) == E["WORKSPACE"]
+    assert f(A, A, 1, 4, 64, 0.04, A, A, A, ws - 1, None) == E["WORKSPACE"]
+    assert lib.cachedit_decide(None, 1, 1, 0.04, A, A, None) == E["NULL"]
+    assert lib.cachedit_decide(A, 0, 1, 0.04, A, A, None) == E["SHAPE"]
+    assert lib.cachedit_decide(A + 4, 1, 1, 0.04, A, A, None) == E["ALIGN"]
+
+
+def test_binding_refuses_cpu_tensors():
+    import torch
+    import dit_block_pass_b200 as dbp
+    x = torch.zeros(1, 4, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        dbp.adaln_modulate(x, torch.zeros(1, 64), torch.zeros(1, 64))
+    with pytest.raises(ValueError):
+        dbp.swiglu(torch.zeros(4, 16, dtype=torch.bfloat16))
