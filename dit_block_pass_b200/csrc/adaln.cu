@@ -10,7 +10,8 @@
 //
 // Design: one warp owns one token row at a time and holds the whole row in
 // registers (VPL 16-byte vectors per lane; D = 5120 -> 20), so x is read
-// once.  Row statistics are two warp-shuffle reductions (a mean of values
+// once.  The gated variant splits each row across a warp pair and brings the
+// branch row r through a per-warp shared-memory stage with cp.async.  Row statistics are two warp-shuffle reductions (a mean of values
 // shifted by the row's first element, then the centred sum of squares).
 // The modulation vectors of the CTA's sample are staged once in shared
 // memory as fp32, split into low and high float4 halves so that a warp's
@@ -46,19 +47,31 @@ __device__ __forceinline__ float mod_at(const void* p, int dtype, int64_t i) {
     return __uint_as_float(static_cast<uint32_t>(static_cast<const uint16_t*>(p)[i]) << 16);
 }
 
-// bf16(x + g*r) with ONE rounding of the exact value.  The fp32 fma rounds
-// once to 24 bits; rounding that to bf16 can differ from rounding the exact
-// value only when the fp32 result sits exactly on a bf16 tie (low 16 bits
-// 0x8000).  Then the sum is redone in fp64, where g*r (<= 32 significant
-// bits) is exact, and rounded straight to bf16.
-__device__ __forceinline__ float gated_add(float x, float g, float r) {
-    const float s = __fmaf_rn(g, r, x);
-    if ((__float_as_uint(s) & 0xFFFFu) == 0x8000u) {
-        const double e = fma(static_cast<double>(g), static_cast<double>(r),
-                             static_cast<double>(x));
-        return __bfloat162float(__double2bfloat16(e));
-    }
-    return __bfloat162float(__float2bfloat16_rn(s));
+// bf16(x + g*r) for two elements with ONE rounding of each exact value.
+// The fp32 fma rounds once to 24 bits; rounding that to bf16 can differ
+// from rounding the exact value only when the fp32 result sits exactly on a
+// bf16 tie (low 16 bits 0x8000).  The pair is then redone in fp64, where
+// g*r (<= 32 significant bits) is exact, and rounded straight to bf16.  The
+// packed fp32 -> bf16x2 conversion runs on the ALU, not the conversion unit.
+__device__ __noinline__ uint32_t gated_pair_fp64(float x0, float g0, float r0, float x1, float g1,
+                                                 float r1) {
+    const __nv_bfloat16 lo = __double2bfloat16(
+        fma(static_cast<double>(g0), static_cast<double>(r0), static_cast<double>(x0)));
+    const __nv_bfloat16 hi = __double2bfloat16(
+        fma(static_cast<double>(g1), static_cast<double>(r1), static_cast<double>(x1)));
+    return static_cast<uint32_t>(__bfloat16_as_ushort(lo)) |
+           (static_cast<uint32_t>(__bfloat16_as_ushort(hi)) << 16);
+}
+
+__device__ __forceinline__ uint32_t gated_pair(uint32_t xw, uint32_t rw, float g0, float g1) {
+    const float x0 = bf16_lo(xw), x1 = bf16_hi(xw);
+    const float r0 = bf16_lo(rw), r1 = bf16_hi(rw);
+    const float s0 = __fmaf_rn(g0, r0, x0);
+    const float s1 = __fmaf_rn(g1, r1, x1);
+    const bool tie = ((__float_as_uint(s0) & 0xFFFFu) == 0x8000u) |
+                     ((__float_as_uint(s1) & 0xFFFFu) == 0x8000u);
+    if (tie) return gated_pair_fp64(x0, g0, r0, x1, g1, r1);
+    return pack2(s0, s1);
 }
 
 __device__ __forceinline__ void lds8(const float4* lo, const float4* hi, int v, float (&f)[8]) {
@@ -67,17 +80,16 @@ __device__ __forceinline__ void lds8(const float4* lo, const float4* hi, int v, 
     f[4] = b.x; f[5] = b.y; f[6] = b.z; f[7] = b.w;
 }
 
-template <int VPL, bool GATED>
-__global__ void __launch_bounds__(kThreads)
-adaln_rows_kernel(RowParams p) {
-    extern __shared__ float4 smem[];
+// Stage the modulation vectors of sample blockIdx.y in shared memory:
+// shift and (1 + scale) (and gate), each as [lo Dv][hi Dv] float4 halves.
+template <bool GATED>
+__device__ __forceinline__ void stage_modulation(const RowParams& p, float4* smem, int nthreads) {
     const int Dv = p.Dv;
-    float4* s_sh = smem;            // shift:     [lo Dv][hi Dv]
-    float4* s_sc = smem + 2 * Dv;   // 1 + scale: [lo Dv][hi Dv]
-    float4* s_g = smem + 4 * Dv;    // gate:      [lo Dv][hi Dv] (GATED)
-    const int b = blockIdx.y;
-    const int64_t mb = static_cast<int64_t>(b) * p.mod_stride;
-    for (int v = threadIdx.x; v < Dv; v += kThreads) {
+    float4* s_sh = smem;
+    float4* s_sc = smem + 2 * Dv;
+    float4* s_g = smem + 4 * Dv;
+    const int64_t mb = static_cast<int64_t>(blockIdx.y) * p.mod_stride;
+    for (int v = threadIdx.x; v < Dv; v += nthreads) {
         float sh[8], sc[8], g[8];
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
@@ -94,60 +106,185 @@ adaln_rows_kernel(RowParams p) {
             s_g[Dv + v] = make_float4(g[4], g[5], g[6], g[7]);
         }
     }
-    __syncthreads();
+}
 
+// Second half of the LayerNorm of the warp's register-resident row, given
+// the shift x0 and the warp's sum of (x - x0): the centred sum of squares,
+// then y = (x - mu) * rstd * (1 + scale) + shift.
+template <int VPL>
+__device__ __forceinline__ void ln_finish_store(const RowParams& p, const float4* smem,
+                                                const uint4 (&xv)[VPL], int64_t base, int lane,
+                                                float x0, float s) {
+    const int Dv = p.Dv;
+    const float4* s_sh = smem;
+    const float4* s_sc = smem + 2 * Dv;
+    s = warp_sum(s);
+    const float mu = x0 + s * p.inv_D;
+    float q = 0.0f;
+#pragma unroll
+    for (int j = 0; j < VPL; ++j) {
+        if (j * 32 + lane < Dv) {
+            float f[8];
+            unpack8(xv[j], f);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const float d = f[i] - mu;
+                q = __fmaf_rn(d, d, q);
+            }
+        }
+    }
+    q = warp_sum(q);
+    const float rstd = rsqrtf(__fmaf_rn(q, p.inv_D, p.eps));
+#pragma unroll
+    for (int j = 0; j < VPL; ++j) {
+        const int v = j * 32 + lane;
+        if (v < Dv) {
+            float f[8], sh[8], sc[8];
+            unpack8(xv[j], f);
+            lds8(s_sh, s_sh + Dv, v, sh);
+            lds8(s_sc, s_sc + Dv, v, sc);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) f[i] = __fmaf_rn((f[i] - mu) * rstd, sc[i], sh[i]);
+            st_stream(p.y + base + v, pack8(f));
+        }
+    }
+}
+
+// The LayerNorm of the row with the mean accumulated relative to the row's
+// first element (a shift that keeps the fp32 sum small when |mean| >> std).
+template <int VPL>
+__device__ __forceinline__ void ln_modulate_store(const RowParams& p, const float4* smem,
+                                                  const uint4 (&xv)[VPL], int64_t base,
+                                                  int lane) {
+    const float x0 = __shfl_sync(0xffffffffu, bf16_lo(xv[0].x), 0);
+    float s = 0.0f;
+#pragma unroll
+    for (int j = 0; j < VPL; ++j) {
+        if (j * 32 + lane < p.Dv) {
+            float f[8];
+            unpack8(xv[j], f);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) s += f[i] - x0;
+        }
+    }
+    ln_finish_store<VPL>(p, smem, xv, base, lane, x0, s);
+}
+
+// AdaLN: one warp per row, the row in registers (VPL vectors per lane).
+template <int VPL>
+__global__ void __launch_bounds__(kThreads)
+adaln_rows_kernel(RowParams p) {
+    extern __shared__ float4 smem[];
+    stage_modulation<false>(p, smem, kThreads);
+    __syncthreads();
     const int lane = threadIdx.x & 31;
-    const int warp = threadIdx.x >> 5;
-    const int64_t row0 = static_cast<int64_t>(b) * p.N;
+    const int64_t row0 = static_cast<int64_t>(blockIdx.y) * p.N;
     const int64_t wstep = static_cast<int64_t>(gridDim.x) * kWarps;
-    for (int64_t n = static_cast<int64_t>(blockIdx.x) * kWarps + warp; n < p.N; n += wstep) {
-        const int64_t base = (row0 + n) * Dv;
+    for (int64_t n = static_cast<int64_t>(blockIdx.x) * kWarps + (threadIdx.x >> 5); n < p.N;
+         n += wstep) {
+        const int64_t base = (row0 + n) * p.Dv;
         uint4 xv[VPL];
 #pragma unroll
         for (int j = 0; j < VPL; ++j) {
             const int v = j * 32 + lane;
+            xv[j] = (v < p.Dv) ? ld_inplace(p.x + base + v) : make_uint4(0, 0, 0, 0);
+        }
+        ln_modulate_store<VPL>(p, smem, xv, base, lane);
+    }
+}
+
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gsrc) {
+    const unsigned d = static_cast<unsigned>(__cvta_generic_to_shared(smem_dst));
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d), "l"(gsrc) : "memory");
+}
+
+// Gated residual + AdaLN: one warp PAIR per row.  Warp h (0, 1) of a pair
+// holds vectors v = 64*j + 32*h + lane of the row (each warp instruction
+// still covers 512 contiguous bytes), so a lane keeps VPL = ceil(D/512)
+// vectors in registers and twice as many warps fit on an SM as with one
+// warp per row.  The branch row r goes to a per-warp shared-memory stage
+// with cp.async, issued together with the x loads.  The two row statistics
+// are exchanged through shared memory with one named barrier per pair each;
+// both warps add the two halves in the same order, so they agree exactly.
+template <int VPL, int WARPS>
+__global__ void __launch_bounds__(WARPS * 32, 1)
+gated_rows_kernel(RowParams p) {
+    constexpr int PAIRS = WARPS / 2;
+    extern __shared__ float4 smem[];
+    __shared__ float red[PAIRS][2][2];          // [pair][statistic][half]
+    __shared__ float shift[PAIRS][2];           // [pair][half]: each half's shift
+    stage_modulation<true>(p, smem, WARPS * 32);
+    __syncthreads();
+    const int Dv = p.Dv;
+    const float4* s_g = smem + 4 * Dv;
+    const float4* s_sh = smem;
+    const float4* s_sc = smem + 2 * Dv;
+    const int lane = threadIdx.x & 31;
+    const int warp = threadIdx.x >> 5;
+    const int half = warp & 1, pair = warp >> 1;
+    const int bar = 1 + pair;                   // named barrier of the pair (0 = __syncthreads)
+    uint4* stage = reinterpret_cast<uint4*>(smem + 6 * Dv) + warp * (VPL * 32);
+    // elements held by half 1: vectors 64j + 32 + lane < Dv
+    const int rem = Dv % 64;
+    const float n1 = 8.0f * static_cast<float>((Dv / 64) * 32 + (rem > 32 ? rem - 32 : 0));
+    const int64_t row0 = static_cast<int64_t>(blockIdx.y) * p.N;
+    const int64_t rstep = static_cast<int64_t>(gridDim.x) * PAIRS;
+    for (int64_t n = static_cast<int64_t>(blockIdx.x) * PAIRS + pair; n < p.N; n += rstep) {
+        const int64_t base = (row0 + n) * Dv;
+#pragma unroll
+        for (int j = 0; j < VPL; ++j) {
+            const int v = 64 * j + 32 * half + lane;
+            if (v < Dv) cp_async16(stage + j * 32 + lane, p.r + base + v);
+        }
+        asm volatile("cp.async.commit_group;" ::: "memory");
+        uint4 xv[VPL];
+#pragma unroll
+        for (int j = 0; j < VPL; ++j) {
+            const int v = 64 * j + 32 * half + lane;
             xv[j] = (v < Dv) ? ld_inplace(p.x + base + v) : make_uint4(0, 0, 0, 0);
         }
-        if constexpr (GATED) {
-            uint4 rv[VPL];
-#pragma unroll
-            for (int j = 0; j < VPL; ++j) {
-                const int v = j * 32 + lane;
-                rv[j] = (v < Dv) ? ld_stream(p.r + base + v) : make_uint4(0, 0, 0, 0);
-            }
-#pragma unroll
-            for (int j = 0; j < VPL; ++j) {
-                const int v = j * 32 + lane;
-                if (v < Dv) {
-                    float fx[8], fr[8], fg[8];
-                    unpack8(xv[j], fx);
-                    unpack8(rv[j], fr);
-                    lds8(s_g, s_g + Dv, v, fg);
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) fx[i] = gated_add(fx[i], fg[i], fr[i]);
-                    xv[j] = pack8(fx);  // exact: every fx[i] is a bf16 value
-                    st_stream(p.x_out + base + v, xv[j]);
-                }
-            }
-        }
-        // mean, accumulated relative to the row's first element
+        // shift for this half's sum: the first element the warp holds (x may be
+        // overwritten in place by the other warp, so each warp uses its own)
         const float x0 = __shfl_sync(0xffffffffu, bf16_lo(xv[0].x), 0);
+        // each lane reads back only the vectors it copied itself
+        asm volatile("cp.async.wait_group 0;" ::: "memory");
         float s = 0.0f;
 #pragma unroll
         for (int j = 0; j < VPL; ++j) {
-            if (j * 32 + lane < Dv) {
+            const int v = 64 * j + 32 * half + lane;
+            if (v < Dv) {
+                const uint4 rv = stage[j * 32 + lane];
+                float g[8];
+                lds8(s_g, s_g + Dv, v, g);
+                uint4 o;
+                o.x = gated_pair(xv[j].x, rv.x, g[0], g[1]);
+                o.y = gated_pair(xv[j].y, rv.y, g[2], g[3]);
+                o.z = gated_pair(xv[j].z, rv.z, g[4], g[5]);
+                o.w = gated_pair(xv[j].w, rv.w, g[6], g[7]);
+                xv[j] = o;
+                st_stream(p.x_out + base + v, o);
                 float f[8];
-                unpack8(xv[j], f);
+                unpack8(o, f);
+                float t = 0.0f;
 #pragma unroll
-                for (int i = 0; i < 8; ++i) s += f[i] - x0;
+                for (int i = 0; i < 8; ++i) t += f[i];
+                s += __fmaf_rn(-8.0f, x0, t);
             }
         }
         s = warp_sum(s);
-        const float mu = x0 + s * p.inv_D;
+        if (lane == 0) {
+            red[pair][0][half] = s;
+            shift[pair][half] = x0;
+        }
+        asm volatile("bar.sync %0, 64;" ::"r"(bar) : "memory");
+        // sum = s0 + n0*x00 + s1 + n1*x01; both warps evaluate the same expression
+        const float x00 = shift[pair][0];
+        const float mu =
+            x00 + __fmaf_rn(n1, shift[pair][1] - x00, red[pair][0][0] + red[pair][0][1]) * p.inv_D;
         float q = 0.0f;
 #pragma unroll
         for (int j = 0; j < VPL; ++j) {
-            if (j * 32 + lane < Dv) {
+            if (64 * j + 32 * half + lane < Dv) {
                 float f[8];
                 unpack8(xv[j], f);
 #pragma unroll
@@ -158,10 +295,13 @@ adaln_rows_kernel(RowParams p) {
             }
         }
         q = warp_sum(q);
-        const float rstd = rsqrtf(__fmaf_rn(q, p.inv_D, p.eps));
+        if (lane == 0) red[pair][1][half] = q;
+        asm volatile("bar.sync %0, 64;" ::"r"(bar) : "memory");
+        const float rstd =
+            rsqrtf(__fmaf_rn(red[pair][1][0] + red[pair][1][1], p.inv_D, p.eps));
 #pragma unroll
         for (int j = 0; j < VPL; ++j) {
-            const int v = j * 32 + lane;
+            const int v = 64 * j + 32 * half + lane;
             if (v < Dv) {
                 float f[8], sh[8], sc[8];
                 unpack8(xv[j], f);
@@ -175,21 +315,57 @@ adaln_rows_kernel(RowParams p) {
     }
 }
 
-template <bool GATED>
 using RowKernel = void (*)(RowParams);
 
-template <bool GATED>
-RowKernel<GATED> pick_kernel(int vpl_needed, int* vpl) {
-#define DIT_VPL_CASE(V)                              \
-    if (vpl_needed <= V) {                           \
-        *vpl = V;                                    \
-        return adaln_rows_kernel<V, GATED>;          \
-    }
-    DIT_VPL_CASE(1) DIT_VPL_CASE(2) DIT_VPL_CASE(3) DIT_VPL_CASE(4) DIT_VPL_CASE(6)
-    DIT_VPL_CASE(8) DIT_VPL_CASE(10) DIT_VPL_CASE(12) DIT_VPL_CASE(16) DIT_VPL_CASE(20)
-    DIT_VPL_CASE(24) DIT_VPL_CASE(32)
+struct RowLaunch {
+    RowKernel kernel;
+    int threads;
+    size_t smem;
+};
+
+RowLaunch pick_kernel(bool gated, int Dv) {
+    const size_t mod = static_cast<size_t>(gated ? 6 : 4) * Dv * sizeof(float4);
+    if (!gated) {
+        const int need = (Dv + 31) / 32;
+#define DIT_VPL_CASE(V) \
+    if (need <= V) return {adaln_rows_kernel<V>, kThreads, mod};
+        DIT_VPL_CASE(1) DIT_VPL_CASE(2) DIT_VPL_CASE(3) DIT_VPL_CASE(4) DIT_VPL_CASE(6)
+        DIT_VPL_CASE(8) DIT_VPL_CASE(10) DIT_VPL_CASE(12) DIT_VPL_CASE(16) DIT_VPL_CASE(20)
+        DIT_VPL_CASE(24) DIT_VPL_CASE(32)
 #undef DIT_VPL_CASE
-    return nullptr;
+        return {nullptr, 0, 0};
+    }
+    const int need = (Dv + 63) / 64;   // a warp pair shares a row
+#define DIT_VPL_CASE(V)                                                                   \
+    if (need <= V) {                                                                      \
+        constexpr int WG = (V <= 10) ? 24 : 16;                                           \
+        return {gated_rows_kernel<V, WG>, WG * 32,                                        \
+                mod + static_cast<size_t>(WG) * V * 32 * sizeof(uint4)};                  \
+    }
+    DIT_VPL_CASE(1) DIT_VPL_CASE(2) DIT_VPL_CASE(3) DIT_VPL_CASE(4) DIT_VPL_CASE(5)
+    DIT_VPL_CASE(6) DIT_VPL_CASE(8) DIT_VPL_CASE(10) DIT_VPL_CASE(12) DIT_VPL_CASE(16)
+#undef DIT_VPL_CASE
+    return {nullptr, 0, 0};
+}
+
+int launch_rows(const RowParams& p, bool gated, int B, cudaStream_t stream) {
+    const RowLaunch L = pick_kernel(gated, p.Dv);
+    if (!L.kernel) return DIT_ERR_SHAPE;
+    if (L.smem > 48 * 1024 &&
+        cudaFuncSetAttribute(L.kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(L.smem)) != cudaSuccess)
+        return DIT_ERR_LAUNCH;
+    const int sms = device_sm_count();
+    if (sms <= 0) return DIT_ERR_LAUNCH;
+    const int occ = occupancy(reinterpret_cast<const void*>(L.kernel), L.threads, L.smem);
+    int64_t per_sample = (static_cast<int64_t>(sms) * occ) / B;
+    if (per_sample < 1) per_sample = 1;
+    const int rows_per_cta = gated ? L.threads / 64 : L.threads / 32;
+    const int64_t need = (p.N + rows_per_cta - 1) / rows_per_cta;
+    if (per_sample > need) per_sample = need;
+    dim3 grid(static_cast<unsigned>(per_sample), static_cast<unsigned>(B));
+    L.kernel<<<grid, L.threads, L.smem, stream>>>(p);
+    return launch_status();
 }
 
 int check_mod(const void* p, int dtype) {
@@ -197,28 +373,6 @@ int check_mod(const void* p, int dtype) {
     const uintptr_t a = reinterpret_cast<uintptr_t>(p);
     if (a % (dtype == DIT_F32 ? 4 : 2)) return DIT_ERR_ALIGN;
     return DIT_OK;
-}
-
-template <bool GATED>
-int launch_rows(const RowParams& p, int B, cudaStream_t stream) {
-    int vpl = 0;
-    RowKernel<GATED> kernel = pick_kernel<GATED>((p.Dv + 31) / 32, &vpl);
-    if (!kernel) return DIT_ERR_SHAPE;
-    const size_t smem = static_cast<size_t>(GATED ? 6 : 4) * p.Dv * sizeof(float4);
-    if (smem > 48 * 1024 &&
-        cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(smem)) != cudaSuccess)
-        return DIT_ERR_LAUNCH;
-    const int sms = device_sm_count();
-    if (sms <= 0) return DIT_ERR_LAUNCH;
-    const int occ = occupancy(reinterpret_cast<const void*>(kernel), kThreads, smem);
-    int64_t per_sample = (static_cast<int64_t>(sms) * occ) / B;
-    if (per_sample < 1) per_sample = 1;
-    const int64_t need = (p.N + kWarps - 1) / kWarps;
-    if (per_sample > need) per_sample = need;
-    dim3 grid(static_cast<unsigned>(per_sample), static_cast<unsigned>(B));
-    kernel<<<grid, kThreads, smem, stream>>>(p);
-    return launch_status();
 }
 
 int common_checks(int B, int64_t N, int D, int mod_dtype, int64_t mod_stride, double eps) {
@@ -238,14 +392,14 @@ extern "C" int dit_adaln_modulate(const uint16_t* x, uint16_t* y, const void* sh
                                   const void* scale, int mod_dtype, int64_t mod_batch_stride,
                                   int B, int64_t N, int D, double eps, void* stream) {
     using namespace dit;
-    if (!x || !y) return DIT_ERR_NULL;
     int st = common_checks(B, N, D, mod_dtype, mod_batch_stride, eps);
     if (st) return st;
+    if (B == 0 || N == 0) return DIT_OK;
+    if (!x || !y) return DIT_ERR_NULL;
     if ((st = check_mod(shift, mod_dtype)) || (st = check_mod(scale, mod_dtype))) return st;
     if (!aligned16(x) || !aligned16(y)) return DIT_ERR_ALIGN;
     const size_t bytes = static_cast<size_t>(B) * N * D * 2;
     if (x != y && overlaps(x, bytes, y, bytes)) return DIT_ERR_OVERLAP;
-    if (B == 0 || N == 0) return DIT_OK;
     RowParams p{};
     p.x = reinterpret_cast<const uint4*>(x);
     p.y = reinterpret_cast<uint4*>(y);
@@ -257,7 +411,7 @@ extern "C" int dit_adaln_modulate(const uint16_t* x, uint16_t* y, const void* sh
     p.Dv = D / 8;
     p.inv_D = 1.0f / static_cast<float>(D);
     p.eps = static_cast<float>(eps);
-    return launch_rows<false>(p, B, as_stream(stream));
+    return launch_rows(p, false, B, as_stream(stream));
 }
 
 extern "C" int dit_gated_residual_adaln(const uint16_t* x, const uint16_t* r, uint16_t* x_out,
@@ -266,9 +420,10 @@ extern "C" int dit_gated_residual_adaln(const uint16_t* x, const uint16_t* r, ui
                                         int64_t mod_batch_stride, int B, int64_t N, int D,
                                         double eps, void* stream) {
     using namespace dit;
-    if (!x || !r || !x_out || !y) return DIT_ERR_NULL;
     int st = common_checks(B, N, D, mod_dtype, mod_batch_stride, eps);
     if (st) return st;
+    if (B == 0 || N == 0) return DIT_OK;
+    if (!x || !r || !x_out || !y) return DIT_ERR_NULL;
     if ((st = check_mod(gate, mod_dtype)) || (st = check_mod(shift, mod_dtype)) ||
         (st = check_mod(scale, mod_dtype)))
         return st;
@@ -279,7 +434,6 @@ extern "C" int dit_gated_residual_adaln(const uint16_t* x, const uint16_t* r, ui
         overlaps(x, bytes, y, bytes) || overlaps(r, bytes, x_out, bytes) ||
         overlaps(r, bytes, y, bytes) || overlaps(x_out, bytes, y, bytes))
         return DIT_ERR_OVERLAP;
-    if (B == 0 || N == 0) return DIT_OK;
     RowParams p{};
     p.x = reinterpret_cast<const uint4*>(x);
     p.r = reinterpret_cast<const uint4*>(r);
@@ -294,5 +448,5 @@ extern "C" int dit_gated_residual_adaln(const uint16_t* x, const uint16_t* r, ui
     p.Dv = D / 8;
     p.inv_D = 1.0f / static_cast<float>(D);
     p.eps = static_cast<float>(eps);
-    return launch_rows<true>(p, B, as_stream(stream));
+    return launch_rows(p, true, B, as_stream(stream));
 }

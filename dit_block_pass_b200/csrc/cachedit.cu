@@ -122,10 +122,12 @@ int partial_slots(int B, int64_t nvs) {
 }
 
 int check_inputs(const uint16_t* prev, const uint16_t* cur, int B, int64_t N, int D) {
-    if (!prev || !cur) return DIT_ERR_NULL;
     if (B < 1 || N < 0 || D <= 0) return DIT_ERR_SHAPE;
     if (B > 65535 || N > (INT64_MAX / 8) / D / B) return DIT_ERR_SHAPE;
-    if (D % 8 || !aligned16(prev) || !aligned16(cur)) return DIT_ERR_ALIGN;
+    if (D % 8) return DIT_ERR_ALIGN;
+    if (N == 0) return DIT_OK;  // nothing is read: prev and cur may be NULL
+    if (!prev || !cur) return DIT_ERR_NULL;
+    if (!aligned16(prev) || !aligned16(cur)) return DIT_ERR_ALIGN;
     return DIT_OK;
 }
 

@@ -29,6 +29,30 @@ __device__ __forceinline__ void st_stream(uint4* p, const uint4& v) {
                  : "memory");
 }
 
+// 256-bit forms (sm_100): 32-byte aligned, eight 32-bit words.
+struct alignas(32) u32x8 {
+    uint32_t w[8];
+};
+
+__device__ __forceinline__ u32x8 ld_stream256(const void* p) {
+    u32x8 v;
+    asm volatile(
+        "ld.global.nc.L1::no_allocate.L2::evict_first.v8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+        : "=r"(v.w[0]), "=r"(v.w[1]), "=r"(v.w[2]), "=r"(v.w[3]), "=r"(v.w[4]), "=r"(v.w[5]),
+          "=r"(v.w[6]), "=r"(v.w[7])
+        : "l"(p));
+    return v;
+}
+
+__device__ __forceinline__ void st_stream256(void* p, const u32x8& v) {
+    asm volatile("st.global.cs.v8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"l"(p), "r"(v.w[0]),
+                 "r"(v.w[1]), "r"(v.w[2]), "r"(v.w[3]), "r"(v.w[4]), "r"(v.w[5]), "r"(v.w[6]),
+                 "r"(v.w[7])
+                 : "memory");
+}
+
+inline bool aligned32(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 31u) == 0; }
+
 // In-place data (read then written by the same thread): a plain coherent
 // load that still skips L1.
 __device__ __forceinline__ uint4 ld_inplace(const uint4* p) {

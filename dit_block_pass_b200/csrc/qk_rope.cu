@@ -16,8 +16,10 @@
 // (computed once per thread), angles pos*omega are formed and reduced modulo
 // 2*pi in fp64, and sin/cos are taken in fp32 on the reduced angle, which
 // keeps the rotation accurate to a few fp32 ulp for positions in the hundreds.
-// q and k are loaded CH vectors per lane at a time (both tensors in one
-// stream of vectors) to keep enough bytes in flight.  HBM bound.
+// q and k stream through a per-warp, kStages-deep cp.async pipeline of
+// kChunk lane-vectors per stage (each lane copies and later reads back only
+// its own vectors, so no barrier is needed): the next chunks are in flight
+// while the current one is normalised and rotated.  HBM bound.
 #include "common.cuh"
 
 namespace dit {
@@ -25,7 +27,9 @@ namespace {
 
 constexpr int kWarps = 8;
 constexpr int kThreads = kWarps * 32;
-constexpr int kChunk = 8;
+constexpr int kChunk = 10;   // lane-vectors per pipeline stage
+constexpr int kStages = 2;   // cp.async stages per warp
+constexpr size_t kSmem = static_cast<size_t>(kWarps) * kStages * kChunk * 32 * sizeof(uint4);
 
 struct QKParams {
     uint4* t0;              // first tensor processed (q, or k when q is NULL)
@@ -50,12 +54,25 @@ __device__ __forceinline__ float w_at(const void* p, int dtype, int i) {
     return __uint_as_float(static_cast<uint32_t>(static_cast<const uint16_t*>(p)[i]) << 16);
 }
 
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gsrc) {
+    const unsigned d = static_cast<unsigned>(__cvta_generic_to_shared(smem_dst));
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d), "l"(gsrc) : "memory");
+}
+
+// Work of one warp is a sequence of jobs: chunk c (0 .. cpt-1) of each of
+// the warp's tokens in turn.  Chunks 0 .. cq-1 cover the q row and chunks
+// cq .. 2cq-1 the k row, kChunk lane-vectors each (lane-vector i of a row is
+// its vector i * 32 + lane), so the tensor, its weights and its row pointer
+// are uniform inside a chunk.
 template <int HD>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, 2)
 qk_rmsnorm_rope3d_kernel(QKParams p) {
     constexpr int LPH = HD / 8;             // lanes per head
+    extern __shared__ uint4 qk_stage[];
     const int lane = threadIdx.x & 31;
+    const int warp = threadIdx.x >> 5;
     const int sub = lane % LPH;             // this lane's vector within a head
+    uint4* stage = qk_stage + warp * (kStages * kChunk * 32) + lane;
 
     // this lane's rotation pairs: p = 4*sub + j
     int axis[4];
@@ -80,75 +97,110 @@ qk_rmsnorm_rope3d_kernel(QKParams p) {
         w1[i] = p.t1 ? w_at(p.w1, p.w_dtype, 8 * sub + i) : 0.0f;
     }
     const float inv_hd = 1.0f / static_cast<float>(HD);
-    const int nvl = (p.nvr + 31) / 32;      // vectors per lane per tensor row
-    const int lanes_total = (p.t1 ? 2 : 1) * nvl;
+    const int nvl = (p.nvr + 31) / 32;              // lane-vectors per row
+    const int cq = (nvl + kChunk - 1) / kChunk;     // chunks per row
+    const int cpt = (p.t1 ? 2 : 1) * cq;            // chunks per token
+    const int hw = p.Hg * p.Wg;
     const double kTwoPi = 6.283185307179586;
     const double kInvTwoPi = 0.15915494309189535;
-
     const int64_t wstep = static_cast<int64_t>(gridDim.x) * kWarps;
-    for (int64_t tok = static_cast<int64_t>(blockIdx.x) * kWarps + (threadIdx.x >> 5);
-         tok < p.rows; tok += wstep) {
-        int pos3[3];
-        if (p.pos) {
-            pos3[0] = p.pos[3 * tok + 0];
-            pos3[1] = p.pos[3 * tok + 1];
-            pos3[2] = p.pos[3 * tok + 2];
-        } else {
-            const int64_t g = p.pos_offset + tok % p.N;
-            const int64_t hw = static_cast<int64_t>(p.Hg) * p.Wg;
-            const int64_t t = g / hw;
-            const int64_t rem = g - t * hw;
-            const int64_t h = rem / p.Wg;
-            pos3[0] = static_cast<int>(t);
-            pos3[1] = static_cast<int>(h);
-            pos3[2] = static_cast<int>(rem - h * p.Wg);
+
+    // copy chunk `chunk` of token `tok` into stage slot `slot` (one commit group)
+    auto issue = [&](int64_t tok, int chunk, int slot) {
+        if (tok < p.rows) {
+            const int tensor = chunk >= cq ? 1 : 0;
+            const int first = (chunk - tensor * cq) * kChunk;
+            const uint4* row = (tensor ? p.t1 : p.t0) + tok * p.stride_v;
+            uint4* dst = stage + slot * (kChunk * 32);
+#pragma unroll
+            for (int u = 0; u < kChunk; ++u) {
+                const int idx = (first + u) * 32 + lane;
+                if (first + u < nvl && idx < p.nvr) cp_async16(dst + u * 32, row + idx);
+            }
         }
-        float cs[4], sn[4];
+        asm volatile("cp.async.commit_group;" ::: "memory");
+    };
+
+    int64_t itok = static_cast<int64_t>(blockIdx.x) * kWarps + warp, ctok = itok;
+    int ichunk = 0, cchunk = 0, islot = 0, cslot = 0;
+#pragma unroll
+    for (int s = 0; s < kStages - 1; ++s) {
+        issue(itok, ichunk, islot);
+        if (++ichunk == cpt) { ichunk = 0; itok += wstep; }
+        islot = islot + 1 == kStages ? 0 : islot + 1;
+    }
+    float cs[4], sn[4];
+    while (ctok < p.rows) {
+        issue(itok, ichunk, islot);
+        if (++ichunk == cpt) { ichunk = 0; itok += wstep; }
+        islot = islot + 1 == kStages ? 0 : islot + 1;
+        // groups complete in order: all but the newest kStages-1 are done
+        asm volatile("cp.async.wait_group %0;" ::"n"(kStages - 1) : "memory");
+        if (cchunk == 0) {
+            int pos3[3];
+            if (p.pos) {
+                pos3[0] = p.pos[3 * ctok + 0];
+                pos3[1] = p.pos[3 * ctok + 1];
+                pos3[2] = p.pos[3 * ctok + 2];
+            } else {
+                // grid index < 2^31 (checked on the host)
+                const int g = static_cast<int>(p.pos_offset + ctok % p.N);
+                const int t = g / hw;
+                const int rem = g - t * hw;
+                const int h = rem / p.Wg;
+                pos3[0] = t;
+                pos3[1] = h;
+                pos3[2] = rem - h * p.Wg;
+            }
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int pa = axis[j] == 0 ? pos3[0] : (axis[j] == 1 ? pos3[1] : pos3[2]);
+                const double phi = static_cast<double>(pa) * omega[j];
+                const double kk = rint(phi * kInvTwoPi);
+                const float red = static_cast<float>(fma(-kk, kTwoPi, phi));
+                sincosf(red, &sn[j], &cs[j]);
+            }
+        }
+        const int tensor = cchunk >= cq ? 1 : 0;
+        const int first = (cchunk - tensor * cq) * kChunk;
+        uint4* row = (tensor ? p.t1 : p.t0) + ctok * p.stride_v;
+        // rotation with the weight folded in: (u0, u1) = inv * (f0 w0, f1 w1)
+        //   out0 = inv * (f0 * w0 cos - f1 * w1 sin), out1 = inv * (f0 * w0 sin + f1 * w1 cos)
+        float A[4], Bn[4], C[4], Dd[4];
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-            const int pa = axis[j] == 0 ? pos3[0] : (axis[j] == 1 ? pos3[1] : pos3[2]);
-            const double phi = static_cast<double>(pa) * omega[j];
-            const double k = rint(phi * kInvTwoPi);
-            const float red = static_cast<float>(fma(-k, kTwoPi, phi));
-            sincosf(red, &sn[j], &cs[j]);
+            const float wa = tensor ? w1[2 * j] : w0[2 * j];
+            const float wb = tensor ? w1[2 * j + 1] : w0[2 * j + 1];
+            A[j] = wa * cs[j];
+            Bn[j] = -(wb * sn[j]);
+            C[j] = wa * sn[j];
+            Dd[j] = wb * cs[j];
         }
-
-        for (int c0 = 0; c0 < lanes_total; c0 += kChunk) {
-            uint4 v[kChunk];
-            uint4* addr[kChunk];
-            bool act[kChunk];
+        const uint4* src = stage + cslot * (kChunk * 32);
 #pragma unroll
-            for (int u = 0; u < kChunk; ++u) {
-                const int jl = c0 + u;
-                const int tsel = jl >= nvl ? 1 : 0;
-                const int idx = (jl - tsel * nvl) * 32 + lane;
-                act[u] = jl < lanes_total && idx < p.nvr;
-                addr[u] = (tsel ? p.t1 : p.t0) + tok * p.stride_v + idx;
-                v[u] = act[u] ? ld_inplace(addr[u]) : make_uint4(0, 0, 0, 0);
+        for (int u = 0; u < kChunk; ++u) {
+            const int idx = (first + u) * 32 + lane;
+            const bool valid = first + u < nvl && idx < p.nvr;
+            float f[8];
+            unpack8(valid ? src[u * 32] : make_uint4(0, 0, 0, 0), f);
+            float ss = 0.0f;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) ss = __fmaf_rn(f[i], f[i], ss);
+#pragma unroll
+            for (int o = LPH / 2; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+            const float inv = rsqrtf(__fmaf_rn(ss, inv_hd, p.eps));
+            float o8[8];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                o8[2 * j] = inv * __fmaf_rn(f[2 * j], A[j], f[2 * j + 1] * Bn[j]);
+                o8[2 * j + 1] = inv * __fmaf_rn(f[2 * j], C[j], f[2 * j + 1] * Dd[j]);
             }
-#pragma unroll
-            for (int u = 0; u < kChunk; ++u) {
-                const bool second = (c0 + u) >= nvl;
-                float f[8];
-                unpack8(v[u], f);
-                float ss = 0.0f;
-#pragma unroll
-                for (int i = 0; i < 8; ++i) ss = __fmaf_rn(f[i], f[i], ss);
-#pragma unroll
-                for (int o = LPH / 2; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-                const float inv = rsqrtf(__fmaf_rn(ss, inv_hd, p.eps));
-                float o8[8];
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const float u0 = f[2 * j] * inv * (second ? w1[2 * j] : w0[2 * j]);
-                    const float u1 = f[2 * j + 1] * inv * (second ? w1[2 * j + 1] : w0[2 * j + 1]);
-                    o8[2 * j] = __fmaf_rn(u0, cs[j], -u1 * sn[j]);
-                    o8[2 * j + 1] = __fmaf_rn(u0, sn[j], u1 * cs[j]);
-                }
-                if (act[u]) st_stream(addr[u], pack8(o8));
-            }
+            if (valid) st_stream(row + idx, pack8(o8));
         }
+        if (++cchunk == cpt) { cchunk = 0; ctok += wstep; }
+        cslot = cslot + 1 == kStages ? 0 : cslot + 1;
     }
+    asm volatile("cp.async.wait_all;" ::: "memory");
 }
 
 using QKKernel = void (*)(QKParams);
@@ -161,6 +213,27 @@ QKKernel pick(int hd) {
         case 256: return qk_rmsnorm_rope3d_kernel<256>;
         default: return nullptr;
     }
+}
+
+// Rows i of q ([q + i*rs, q + i*rs + w), elements) and rows j of k overlap
+// for some 0 <= i, j < rows iff |d - m*rs| < w for an integer
+// m = i - j in (-rows, rows), d = k - q; the distance is smallest for m next
+// to d/rs, so the two integers around it (clamped to the range) decide.
+bool rows_overlap(const void* q, const void* k, int64_t rows, int64_t rs, int64_t w) {
+    const intptr_t bq = reinterpret_cast<intptr_t>(q), bk = reinterpret_cast<intptr_t>(k);
+    const intptr_t db = bk - bq;
+    if (db % 2) return true;  // not on the same element grid: be conservative
+    const int64_t d = static_cast<int64_t>(db / 2);
+    int64_t m0 = d >= 0 ? d / rs : -((-d + rs - 1) / rs);  // floor(d / rs)
+    for (int64_t m = m0; m <= m0 + 1; ++m) {
+        int64_t mc = m;
+        if (mc > rows - 1) mc = rows - 1;
+        if (mc < -(rows - 1)) mc = -(rows - 1);
+        int64_t dist = d - mc * rs;
+        if (dist < 0) dist = -dist;
+        if (dist < w) return true;
+    }
+    return false;
 }
 
 int check_w(const void* p, int dtype) {
@@ -179,11 +252,7 @@ extern "C" int dit_qk_rmsnorm_rope3d(uint16_t* q, uint16_t* k, int64_t row_strid
                                      int pairs_h, int pairs_w, double theta, double eps,
                                      void* stream) {
     using namespace dit;
-    if (!q && !k) return DIT_ERR_NULL;
     if (w_dtype != DIT_F32 && w_dtype != DIT_BF16) return DIT_ERR_DTYPE;
-    int st;
-    if (q && (st = check_w(w_q, w_dtype))) return st;
-    if (k && (st = check_w(w_k, w_dtype))) return st;
     if (B < 0 || N < 0 || H < 1) return DIT_ERR_SHAPE;
     QKKernel kernel = pick(hd);
     if (!kernel) return DIT_ERR_SHAPE;
@@ -192,7 +261,6 @@ extern "C" int dit_qk_rmsnorm_rope3d(uint16_t* q, uint16_t* k, int64_t row_strid
     const int64_t width = static_cast<int64_t>(H) * hd;
     if (width > (int64_t(1) << 30) || row_stride < width) return DIT_ERR_SHAPE;
     if (row_stride % 8) return DIT_ERR_ALIGN;
-    if ((q && !aligned16(q)) || (k && !aligned16(k))) return DIT_ERR_ALIGN;
     if (!(theta > 0.0) || theta > 1e300 || !(eps >= 0.0) || eps > 1e30) return DIT_ERR_VALUE;
     const int64_t rows = static_cast<int64_t>(B) * N;
     if (B > 0 && N > (INT64_MAX / 4) / row_stride / B) return DIT_ERR_SHAPE;
@@ -203,14 +271,13 @@ extern "C" int dit_qk_rmsnorm_rope3d(uint16_t* q, uint16_t* k, int64_t row_strid
     } else if (reinterpret_cast<uintptr_t>(pos) % 4) {
         return DIT_ERR_ALIGN;
     }
-    if (q && k) {
-        // q and k rows share the stride; they must not overlap in any row
-        const int64_t d = (reinterpret_cast<intptr_t>(k) - reinterpret_cast<intptr_t>(q)) / 2;
-        int64_t m = d % row_stride;
-        if (m < 0) m += row_stride;
-        if (m < width || row_stride - m < width) return DIT_ERR_OVERLAP;
-    }
     if (rows == 0) return DIT_OK;
+    if (!q && !k) return DIT_ERR_NULL;
+    int st;
+    if (q && (st = check_w(w_q, w_dtype))) return st;
+    if (k && (st = check_w(w_k, w_dtype))) return st;
+    if ((q && !aligned16(q)) || (k && !aligned16(k))) return DIT_ERR_ALIGN;
+    if (q && k && rows_overlap(q, k, rows, row_stride, width)) return DIT_ERR_OVERLAP;
 
     QKParams p{};
     p.t0 = reinterpret_cast<uint4*>(q ? q : k);
@@ -234,10 +301,13 @@ extern "C" int dit_qk_rmsnorm_rope3d(uint16_t* q, uint16_t* k, int64_t row_strid
 
     const int sms = device_sm_count();
     if (sms <= 0) return DIT_ERR_LAUNCH;
-    const int occ = occupancy(reinterpret_cast<const void*>(kernel), kThreads, 0);
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(kSmem)) != cudaSuccess)
+        return DIT_ERR_LAUNCH;
+    const int occ = occupancy(reinterpret_cast<const void*>(kernel), kThreads, kSmem);
     int64_t blocks = static_cast<int64_t>(sms) * occ;
     const int64_t need = (rows + kWarps - 1) / kWarps;
     if (blocks > need) blocks = need;
-    kernel<<<static_cast<unsigned>(blocks), kThreads, 0, as_stream(stream)>>>(p);
+    kernel<<<static_cast<unsigned>(blocks), kThreads, kSmem, as_stream(stream)>>>(p);
     return launch_status();
 }

@@ -4,8 +4,10 @@
 // somadas chega-se a 6 vezes": the SwiGLU activation is one of the fused
 // operators.  out[m, j] = silu(in[m, j]) * in[m, F + j].
 //
-// Design: a persistent grid (SM count x resident CTAs) walks the M*F/8
-// output vectors with a grid stride.  Each thread keeps its (row, column)
+// Design: a persistent grid (SM count x resident CTAs) walks the output
+// vectors with a grid stride: 32-byte vectors (16 values, the 256-bit
+// loads and stores of sm_100) when F is a multiple of 16 and the pointers
+// are 32-byte aligned, else 16-byte vectors.  Each thread keeps its (row, column)
 // position and advances it by a precomputed (rows, columns) step, so the
 // loop has no integer division.  U independent vectors are in flight per
 // thread (2U 16-byte loads), which covers HBM latency at full occupancy.
@@ -36,22 +38,55 @@ __device__ __forceinline__ uint4 swiglu8(const uint4& a, const uint4& b) {
     return pack8(o);
 }
 
-template <int U>
+// Vector of E bf16 values: E = 8 (16-byte accesses) or E = 16 (32-byte).
+template <int E>
+struct Vec;
+template <>
+struct Vec<8> {
+    using T = uint4;
+    static __device__ __forceinline__ T load(const T* p) { return ld_stream(p); }
+    static __device__ __forceinline__ void store(T* p, const T& v) { st_stream(p, v); }
+    static __device__ __forceinline__ T apply(const T& a, const T& b) { return swiglu8(a, b); }
+};
+template <>
+struct Vec<16> {
+    using T = u32x8;
+    static __device__ __forceinline__ T load(const T* p) { return ld_stream256(p); }
+    static __device__ __forceinline__ void store(T* p, const T& v) { st_stream256(p, v); }
+    static __device__ __forceinline__ T apply(const T& a, const T& b) {
+        const uint4 a0 = make_uint4(a.w[0], a.w[1], a.w[2], a.w[3]);
+        const uint4 a1 = make_uint4(a.w[4], a.w[5], a.w[6], a.w[7]);
+        const uint4 b0 = make_uint4(b.w[0], b.w[1], b.w[2], b.w[3]);
+        const uint4 b1 = make_uint4(b.w[4], b.w[5], b.w[6], b.w[7]);
+        const uint4 o0 = swiglu8(a0, b0), o1 = swiglu8(a1, b1);
+        T o;
+        o.w[0] = o0.x; o.w[1] = o0.y; o.w[2] = o0.z; o.w[3] = o0.w;
+        o.w[4] = o1.x; o.w[5] = o1.y; o.w[6] = o1.z; o.w[7] = o1.w;
+        return o;
+    }
+};
+
+// Fv = vectors per output row (F / E); total = M * Fv.
+template <int E, int U>
 __global__ void __launch_bounds__(kThreads)
-swiglu_kernel(const uint4* __restrict__ in, uint4* __restrict__ out, int64_t Fv, int64_t total,
+swiglu_kernel(const void* __restrict__ in_, void* __restrict__ out_, int64_t Fv, int64_t total,
               int64_t step_r, int64_t step_c) {
-    const int64_t T = static_cast<int64_t>(gridDim.x) * kThreads;
+    using V = Vec<E>;
+    using T = typename V::T;
+    const T* in = static_cast<const T*>(in_);
+    T* out = static_cast<T*>(out_);
+    const int64_t nthreads = static_cast<int64_t>(gridDim.x) * kThreads;
     int64_t v = static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x;
     int64_t row = v / Fv;
     int64_t col = v - row * Fv;
-    for (; v < total; v += U * T) {
-        uint4 a[U], b[U];
+    for (; v < total; v += U * nthreads) {
+        T a[U], b[U];
 #pragma unroll
         for (int u = 0; u < U; ++u) {
-            if (v + u * T < total) {
-                const uint4* src = in + row * 2 * Fv + col;
-                a[u] = ld_stream(src);
-                b[u] = ld_stream(src + Fv);
+            if (v + u * nthreads < total) {
+                const T* src = in + row * 2 * Fv + col;
+                a[u] = V::load(src);
+                b[u] = V::load(src + Fv);
             }
             row += step_r;
             col += step_c;
@@ -62,7 +97,7 @@ swiglu_kernel(const uint4* __restrict__ in, uint4* __restrict__ out, int64_t Fv,
         }
 #pragma unroll
         for (int u = 0; u < U; ++u)
-            if (v + u * T < total) st_stream(out + v + u * T, swiglu8(a[u], b[u]));
+            if (v + u * nthreads < total) V::store(out + v + u * nthreads, V::apply(a[u], b[u]));
     }
 }
 
@@ -71,27 +106,30 @@ swiglu_kernel(const uint4* __restrict__ in, uint4* __restrict__ out, int64_t Fv,
 
 extern "C" int dit_swiglu(const uint16_t* in, uint16_t* out, int64_t M, int F, void* stream) {
     using namespace dit;
-    if (!in || !out) return DIT_ERR_NULL;
     if (M < 0 || F <= 0) return DIT_ERR_SHAPE;
-    if (F % 8 || !aligned16(in) || !aligned16(out)) return DIT_ERR_ALIGN;
+    if (F % 8) return DIT_ERR_ALIGN;
     if (M > (INT64_MAX / 8) / F) return DIT_ERR_SHAPE;
+    if (M == 0) return DIT_OK;
+    if (!in || !out) return DIT_ERR_NULL;
+    if (!aligned16(in) || !aligned16(out)) return DIT_ERR_ALIGN;
     const size_t in_bytes = static_cast<size_t>(M) * 2 * F * 2;
     const size_t out_bytes = static_cast<size_t>(M) * F * 2;
     if (overlaps(in, in_bytes, out, out_bytes)) return DIT_ERR_OVERLAP;
-    if (M == 0) return DIT_OK;
 
-    const int64_t Fv = F / 8;
+    // 32-byte vectors when the rows allow them, else 16-byte vectors
+    const bool wide = (F % 16 == 0) && aligned32(in) && aligned32(out);
+    const int E = wide ? 16 : 8;
+    const int64_t Fv = F / E;
     const int64_t total = M * Fv;
     const int sms = device_sm_count();
     if (sms <= 0) return DIT_ERR_LAUNCH;
-    auto kernel = swiglu_kernel<kUnroll>;
+    auto kernel = wide ? swiglu_kernel<16, kUnroll> : swiglu_kernel<8, kUnroll>;
     const int occ = occupancy(reinterpret_cast<const void*>(kernel), kThreads, 0);
     int64_t blocks = static_cast<int64_t>(sms) * occ;
     const int64_t need = (total + kThreads - 1) / kThreads;
     if (blocks > need) blocks = need;
     const int64_t T = blocks * kThreads;
-    kernel<<<static_cast<unsigned>(blocks), kThreads, 0, as_stream(stream)>>>(
-        reinterpret_cast<const uint4*>(in), reinterpret_cast<uint4*>(out), Fv, total, T / Fv,
-        T % Fv);
+    kernel<<<static_cast<unsigned>(blocks), kThreads, 0, as_stream(stream)>>>(in, out, Fv, total,
+                                                                            T / Fv, T % Fv);
     return launch_status();
 }

@@ -36,7 +36,8 @@
  *    (cudaGetLastError after the launch); it may also report an earlier
  *    asynchronous error already pending on the device.
  *  - An empty problem (B == 0 or N == 0 / M == 0) returns DIT_OK and launches
- *    nothing, except where a function says otherwise.
+ *    nothing, except where a function says otherwise; its tensor pointers
+ *    are not read and may be NULL.
  *  - Pointer alignment: every bf16 tensor pointer must be 16-byte aligned,
  *    and row lengths must be multiples of 8 elements, because each kernel
  *    moves rows as 128-bit vectors.  There is no scalar or CPU fallback.
@@ -168,7 +169,8 @@ int dit_qk_rmsnorm_rope3d(uint16_t* q, uint16_t* k, int64_t row_stride,
  * workspace   device scratch of at least cachedit_workspace_bytes(B, N, D)
  *             bytes, 16-byte aligned; its contents on entry do not matter.
  *             Calls that share a workspace must be ordered on the device.
- * N == 0 is allowed and yields rel = 0, reuse = threshold > 0.
+ * N == 0 is allowed (prev and cur may then be NULL) and yields rel = 0,
+ * reuse = (threshold > 0); the kernels still run to write rel and reuse.
  */
 size_t cachedit_workspace_bytes(int B, int64_t N, int D);
 int cachedit_residual_diff(const uint16_t* prev, const uint16_t* cur,

@@ -155,15 +155,25 @@ def test_gated_residual_ties_and_in_place(orc):
     compare_bf16(bits(y), ref_y, "gated ties")
 
 
-def test_gated_zero_gate_equals_adaln():
+def test_gated_zero_gate_equals_adaln(orc):
+    """gate = 0: the residual passes through bit for bit, and y is the AdaLN
+    of x (both kernels within the tolerance of the oracle, and within one
+    bf16 ulp of each other: they sum the row statistics in different
+    orders)."""
     wl = ragged(B=2, N=30, D=640)
-    x = rows(wl, W.S_X, wl.D).view(2, 30, 640).to(DEV)
-    r = rows(wl, W.S_R, wl.D).view(2, 30, 640).to(DEV)
-    mod = W.modulation(wl).to(DEV)
-    xo, y = dbp.gated_residual_adaln(x, r, torch.zeros_like(mod[:, 2]), mod[:, 3], mod[:, 4])
-    y1 = dbp.adaln_modulate(x, mod[:, 3], mod[:, 4])
-    assert torch.equal(xo.view(torch.int16), x.view(torch.int16))
-    assert torch.equal(y.view(torch.int16), y1.view(torch.int16))
+    x = rows(wl, W.S_X, wl.D).view(2, 30, 640)
+    r = rows(wl, W.S_R, wl.D).view(2, 30, 640)
+    mod = W.modulation(wl)
+    mod[:, 2] = 0.0
+    ref = orc.adaln_modulate(bits(x), mod[:, 3].double().numpy(), mod[:, 4].double().numpy(),
+                             wl.eps)
+    xg, modg = x.to(DEV), mod.to(DEV)
+    xo, y = dbp.gated_residual_adaln(xg, r.to(DEV), modg[:, 2], modg[:, 3], modg[:, 4])
+    y1 = dbp.adaln_modulate(xg, modg[:, 3], modg[:, 4])
+    assert torch.equal(xo.view(torch.int16), xg.view(torch.int16))
+    compare_bf16(bits(y), ref, "gated with zero gate")
+    compare_bf16(bits(y1), ref, "adaln")
+    assert compare_bf16(bits(y), orc.bf16_to_f64(bits(y1)), "gated vs adaln", max_ulps=1.0)
 
 
 # ------------------------------------------------------------------ SwiGLU
@@ -184,6 +194,21 @@ def test_swiglu(orc, name):
     torch.cuda.synchronize()
     check()
     compare_bf16(bits(out), ref, f"swiglu {name}")
+
+
+def test_swiglu_narrow_vectors_when_not_32_byte_aligned(orc):
+    """F divisible by 16 but pointers only 16-byte aligned: the 16-byte path."""
+    M, F = 333, 512
+    inp = W.normal(0, 41, M, 2 * F, sigma=2.0)
+    ref = orc.swiglu(bits(inp))
+    ibuf = torch.zeros(M * 2 * F + 8, dtype=torch.bfloat16, device=DEV)
+    ig = ibuf[8:].view(M, 2 * F)            # 16 bytes past a 256-byte boundary
+    ig.copy_(inp.to(DEV))
+    out, check = guarded((M, F), pad=72)    # 144-byte pad: 16 past a 32-byte boundary
+    dbp.swiglu(ig, out=out)
+    torch.cuda.synchronize()
+    check()
+    compare_bf16(bits(out), ref, "swiglu 16-byte path")
 
 
 def test_swiglu_extremes(orc):
