@@ -322,3 +322,4 @@ def cachedit_decide(sums: torch.Tensor, threshold: float):
     _call("cachedit_decide", sums.data_ptr(), R, B, float(threshold), rel.data_ptr(),
           reuse.data_ptr(), _stream(sums))
     return rel, reuse
+

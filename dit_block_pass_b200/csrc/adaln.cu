@@ -1,7 +1,8 @@
 // adaln.cu -- AdaLN modulation, and the gated residual fused with the next
 // AdaLN, each in one pass over HBM.
 //
-// "MiniMax-H3 no SGLang em H200", section "Só com três camadas de aceleração
+// The LMSYS report summary at news.cocoloop.cn ("minimax-h3-sglang-h200"),
+// section "Só com três camadas de aceleração
 // somadas chega-se a 6 vezes": the fused AdaLN update and the gated residual
 // ("residual com gate"); the fused layer changes no result, so the gated
 // variant normalises the residual exactly as stored in bf16.  "MiniMax H3 mở

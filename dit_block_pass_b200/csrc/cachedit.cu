@@ -1,6 +1,7 @@
 // cachedit.cu -- Cache-DiT residual-difference check, one pass over HBM.
 //
-// "MiniMax-H3 no SGLang em H200", section "Só com três camadas de aceleração
+// The LMSYS report summary at news.cocoloop.cn ("minimax-h3-sglang-h200"),
+// section "Só com três camadas de aceleração
 // somadas chega-se a 6 vezes", Cache-DiT paragraph: cached results are reused
 // between neighbouring denoising steps when a residual-difference threshold
 // allows it (0.04 conservative, 0.08 in the more aggressive stride mode).
@@ -199,3 +200,4 @@ extern "C" int cachedit_decide(const double* sums, int R, int B, double threshol
                                                                   rel_out, reuse_out);
     return launch_status();
 }
+

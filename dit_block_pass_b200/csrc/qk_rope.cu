@@ -1,7 +1,8 @@
 // qk_rope.cu -- per-head QK RMSNorm fused with 3D (t, h, w) rotary position
 // embedding, in place, in one pass over HBM.
 //
-// "MiniMax-H3 no SGLang em H200", section "Só com três camadas de aceleração
+// The LMSYS report summary at news.cocoloop.cn ("minimax-h3-sglang-h200"),
+// section "Só com três camadas de aceleração
 // somadas chega-se a 6 vezes": "QK RMSNorm com 3D RoPE" is one fused operator;
 // "SGLang acelera MiniMax-H3 em GPUs H200", first paragraph, lists QK RMSNorm
 // and 3D RoPE among the fused low-level operations.

@@ -1,6 +1,7 @@
 // swiglu.cu -- SwiGLU activation, one streaming pass over HBM.
 //
-// "MiniMax-H3 no SGLang em H200", section "Só com três camadas de aceleração
+// The LMSYS report summary at news.cocoloop.cn ("minimax-h3-sglang-h200"),
+// section "Só com três camadas de aceleração
 // somadas chega-se a 6 vezes": the SwiGLU activation is one of the fused
 // operators.  out[m, j] = silu(in[m, j]) * in[m, F + j].
 //

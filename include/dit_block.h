@@ -5,8 +5,8 @@
  *
  * Sources.  The operators are the ones the SGLang-Diffusion H200 report fuses
  * and the Cache-DiT check it uses:
- *   "MiniMax-H3 no SGLang em H200" (news.cocoloop.cn, summary of the LMSYS
- *   report), section "Só com três camadas de aceleração somadas chega-se a 6
+ *   the LMSYS report summary at news.cocoloop.cn (page "minimax-h3-sglang-h200",
+ *   untitled in the text), section "Só com três camadas de aceleração somadas chega-se a 6
  *   vezes": the fused AdaLN update, gated residual, SwiGLU activation and
  *   QK RMSNorm with 3D RoPE ("changes no calculation result"), and Cache-DiT
  *   reuse decided by a residual-difference threshold (0.04 conservative,

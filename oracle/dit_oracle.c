@@ -8,9 +8,10 @@
  * with the CUDA library.
  *
  * Sources.  The operators are named, not defined, by:
- *   [REPORT]  "MiniMax-H3 no SGLang em H200" (news.cocoloop.cn, LMSYS report
- *             summary), section "Só com três camadas de aceleração somadas
- *             chega-se a 6 vezes": fused AdaLN update, gated residual, SwiGLU,
+ *   [REPORT]  the LMSYS report summary at news.cocoloop.cn (page
+ *             "minimax-h3-sglang-h200", untitled in the text), section
+ *             "Só com três camadas de aceleração somadas chega-se a 6
+ *             vezes": fused AdaLN update, gated residual, SwiGLU,
  *             QK RMSNorm with 3D RoPE; the fused layer changes no result;
  *             Cache-DiT reuses results between neighbouring denoising steps
  *             when a residual-difference threshold (0.04 conservative, 0.08
