@@ -24,7 +24,8 @@ import torch
 __all__ = [
     "DitError", "library", "library_path", "adaln_modulate", "gated_residual_adaln", "swiglu",
     "qk_rmsnorm_rope3d", "cachedit_workspace_bytes", "cachedit_residual_diff",
-    "cachedit_residual_sums", "cachedit_decide", "launch_counts", "F32", "BF16",
+    "cachedit_residual_sums", "cachedit_decide", "cachedit_residual_diff_noalloc",
+    "launch_counts", "F32", "BF16",
 ]
 
 F32, BF16 = 0, 1
@@ -37,6 +38,7 @@ _lock = threading.Lock()
 launch_counts = {
     "adaln_modulate": 1, "gated_residual_adaln": 1, "swiglu": 1, "qk_rmsnorm_rope3d": 1,
     "cachedit_residual_diff": 2, "cachedit_residual_sums": 2, "cachedit_decide": 1,
+    "cachedit_residual_diff_noalloc": 2,
 }
 
 
@@ -78,6 +80,8 @@ def library() -> ctypes.CDLL:
             L.cachedit_residual_diff.argtypes = [vp, vp, i32, i64, i32, dbl, vp, vp, vp, sz, vp]
             L.cachedit_residual_sums.argtypes = [vp, vp, i32, i64, i32, vp, vp, sz, vp]
             L.cachedit_decide.argtypes = [vp, i32, i32, dbl, vp, vp, vp]
+            L.cachedit_residual_diff_noalloc.argtypes = [vp, vp, i32, i64, i32, dbl, vp, vp, vp]
+            L.cachedit_residual_diff_noalloc.restype = i32
             for name in ("dit_adaln_modulate", "dit_gated_residual_adaln", "dit_swiglu",
                          "dit_qk_rmsnorm_rope3d", "cachedit_residual_diff",
                          "cachedit_residual_sums", "cachedit_decide"):
@@ -323,3 +327,22 @@ def cachedit_decide(sums: torch.Tensor, threshold: float):
           reuse.data_ptr(), _stream(sums))
     return rel, reuse
 
+
+def cachedit_residual_diff_noalloc(prev: torch.Tensor, cur: torch.Tensor, threshold: float,
+                                   rel: Optional[torch.Tensor] = None,
+                                   reuse: Optional[torch.Tensor] = None):
+    """The Cache-DiT check for callers that cannot allocate device memory: the
+    library keeps the partial sums in its own fixed 64 KB device array
+    instead of a workspace (at most 64 samples).  Pass preallocated ``rel``
+    [B] float64 and ``reuse`` [B] uint8 to allocate nothing at all.  Calls
+    on one device share that array: order them (one stream, or synchronise)."""
+    _need_cuda_bf16("prev", prev)
+    _need_cuda_bf16("cur", cur)
+    B, N, D = _rows3("prev", prev)
+    if cur.shape != prev.shape or not cur.is_contiguous():
+        raise ValueError("cur must match prev")
+    rel = torch.empty(B, dtype=torch.float64, device=prev.device) if rel is None else rel
+    reuse = torch.empty(B, dtype=torch.uint8, device=prev.device) if reuse is None else reuse
+    _call("cachedit_residual_diff_noalloc", prev.data_ptr(), cur.data_ptr(), B, N, D,
+          float(threshold), rel.data_ptr(), reuse.data_ptr(), _stream(prev))
+    return rel, reuse

@@ -16,6 +16,8 @@
 // are no floating-point atomics, so the result is identical run to run.
 #include <math.h>
 
+#include <mutex>
+
 #include "common.cuh"
 
 namespace dit {
@@ -201,3 +203,72 @@ extern "C" int cachedit_decide(const double* sums, int R, int B, double threshol
     return launch_status();
 }
 
+// ---------------------------------------------------------------------------
+// Cache-DiT check without a caller-provided workspace.
+//
+// Some callers cannot call cudaMalloc or hand this library a scratch buffer:
+// for example a plugin inside a serving engine that owns every byte of device
+// memory through its own pool and forbids raw allocations, or a caller on a
+// latency-critical path that cannot afford the device-wide synchronisation a
+// fresh cudaMalloc can cause.  For them the partial sums live in a fixed
+// array in this library's device memory: kStaticPairs (sum, sum) pairs, 64 KB,
+// which every GPU that loads the library holds until the process exits.
+//
+// Host code must not pass the array's name to a kernel (on the host it is a
+// stand-in, not a device address); the device address is looked up once per
+// device with cudaGetSymbolAddress, on the first call made with that device
+// current, and cached.
+namespace dit {
+namespace {
+
+constexpr int kStaticMaxSamples = 64;
+constexpr int kStaticPairs = 4096;
+static __device__ __align__(256) double g_cachedit_scratch[kStaticPairs * 2];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_scratch_mu;
+double* g_scratch_ptr[kMaxDevices] = {};
+
+// Device address of the scratch array on the current device (looked up once).
+double* scratch_address() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+    std::lock_guard<std::mutex> lock(g_scratch_mu);
+    if (!g_scratch_ptr[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_cachedit_scratch) != cudaSuccess) return nullptr;
+        g_scratch_ptr[dev] = static_cast<double*>(p);
+    }
+    return g_scratch_ptr[dev];
+}
+
+}  // namespace
+}  // namespace dit
+
+extern "C" int cachedit_residual_diff_noalloc(const uint16_t* prev, const uint16_t* cur, int B,
+                                              int64_t N, int D, double threshold,
+                                              double* rel_out, uint8_t* reuse_out,
+                                              void* stream) {
+    using namespace dit;
+    int st = check_inputs(prev, cur, B, N, D);
+    if (st) return st;
+    if (B > kStaticMaxSamples) return DIT_ERR_SHAPE;
+    if (!rel_out || !reuse_out) return DIT_ERR_NULL;
+    if (isnan(threshold)) return DIT_ERR_VALUE;
+    double* scratch = scratch_address();
+    if (!scratch) return DIT_ERR_LAUNCH;
+    const int64_t nvs = N * D / 8;
+    const int G = partial_slots(B, nvs);
+    if (G < 1) return DIT_ERR_LAUNCH;
+    if (static_cast<int64_t>(G) * B > kStaticPairs) return DIT_ERR_WORKSPACE;
+    // Every slot the finalize kernel reads is written by the partials kernel
+    // of the same call, so the array needs no clearing between calls.
+    dim3 grid(static_cast<unsigned>(G), static_cast<unsigned>(B));
+    cachedit_partials_kernel<<<grid, kThreads, 0, as_stream(stream)>>>(
+        reinterpret_cast<const uint4*>(prev), reinterpret_cast<const uint4*>(cur), nvs, scratch,
+        B);
+    if ((st = launch_status())) return st;
+    cachedit_finalize_kernel<<<B, 32, 0, as_stream(stream)>>>(scratch, G, B, threshold, nullptr,
+                                                              rel_out, reuse_out);
+    return launch_status();
+}

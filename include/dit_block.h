@@ -200,6 +200,34 @@ int cachedit_residual_sums(const uint16_t* prev, const uint16_t* cur,
 int cachedit_decide(const double* sums, int R, int B, double threshold,
                     double* rel_out, uint8_t* reuse_out, void* stream);
 
+/*
+ * The Cache-DiT check of cachedit_residual_diff for callers that cannot
+ * allocate device memory or pass a workspace (the pages have no counterpart
+ * to this entry point; it exists for such callers).  Some callers cannot
+ * call cudaMalloc: a plugin inside a serving engine that owns all device
+ * memory through its own pool and forbids raw allocations, or a caller on a
+ * latency-critical path that cannot accept the device-wide synchronisation a
+ * fresh allocation can cause.
+ * The partial sums go to a fixed 64 KB array inside the library (4096 pairs
+ * of doubles per device, held by every GPU that loads the library until the
+ * process exits).  This entry point allocates nothing and calls no
+ * allocating routine.
+ * Limits: B <= 64 samples, and (partial-sum slots per sample) x B <= 4096
+ * (always true for B <= 64 on current GPUs); beyond them it returns
+ * DIT_ERR_SHAPE (B) or DIT_ERR_WORKSPACE (slots) and launches nothing.
+ * Set-up: the first call on each device looks up the array's device address
+ * (cudaGetSymbolAddress) with that device current and caches it; make that
+ * first call before any stream capture on the device.
+ * Sharing: every call on a device uses the same array, which keeps the last
+ * call's contents; each call writes every slot it reads before reading it,
+ * so nothing needs clearing, but calls that overlap on the GPU (different
+ * streams, or host threads without ordering) race on the array: order them.
+ * Arguments and results otherwise as cachedit_residual_diff.
+ */
+int cachedit_residual_diff_noalloc(const uint16_t* prev, const uint16_t* cur,
+                                   int B, int64_t N, int D, double threshold,
+                                   double* rel_out, uint8_t* reuse_out, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -1,0 +1,78 @@
+"""The Cache-DiT check for callers that cannot allocate device memory.
+
+Some callers cannot call cudaMalloc or pass this library a workspace: a
+plugin inside a serving engine that owns all device memory through its own
+pool, or a caller on a latency-critical path that cannot take the device-wide
+synchronisation a fresh allocation can cause.  cachedit_residual_diff_noalloc
+serves them from a fixed array inside the library.  Its results must match
+the workspace entry point's, call after call, although every call reuses the
+same array and finds the previous call's partial sums in it.
+
+This file sorts last so that a run which stops at the first failure has
+already run every other test.
+"""
+import ctypes
+
+import numpy as np
+import pytest
+import torch
+
+import dit_block_pass_b200 as dbp
+from dit_block_pass_b200 import workloads as W
+
+A = 0x10000  # a 16-byte aligned fake address, never dereferenced by the host checks
+
+
+def _lib():
+    from dit_block_pass_b200 import build
+    build.build()
+    return dbp.library()
+
+
+def test_noalloc_rejects_bad_arguments_on_the_host():
+    """Checks that return before any CUDA call: too many samples, NULLs."""
+    L = _lib()
+    f = L.cachedit_residual_diff_noalloc
+    assert f(A, A, 65, 4, 64, 0.04, A, A, None) == -2          # more than 64 samples
+    assert f(A, A, 0, 4, 64, 0.04, A, A, None) == -2
+    assert f(None, A, 1, 4, 64, 0.04, A, A, None) == -1
+    assert f(A, A, 1, 4, 64, 0.04, None, A, None) == -1
+    assert f(A, A, 1, 4, 60, 0.04, A, A, None) == -3
+    assert f(A, A, 1, 4, 64, float("nan"), A, A, None) == -8
+
+
+@pytest.mark.gpu
+def test_noalloc_matches_the_workspace_entry_point_on_consecutive_calls():
+    _lib()
+    dev = "cuda:0"
+    cases = [
+        W.Workload("a", B=3, T=1, Hg=1, Wg=301, D=512, H=4, hd=128, F=8, pairs=(22, 21, 21),
+                   sigma_cache=(0.03, 0.05, 0.1)),
+        W.Workload("b", B=2, T=2, Hg=24, Wg=42, D=3072, H=24, hd=128, F=8, pairs=(22, 21, 21),
+                   sigma_cache=(0.1, 0.03), seed=7),
+    ]
+    inputs = []
+    for wl in cases:
+        prev, cur = W.cache_pair(wl, device=dev)
+        inputs.append((prev.view(wl.B, wl.N, wl.D), cur.view(wl.B, wl.N, wl.D)))
+    # two calls in a row, on different inputs, through the C ABI
+    got = [dbp.cachedit_residual_diff_noalloc(p, c, 0.04) for p, c in inputs]
+    got = [(r.cpu().numpy(), u.cpu().numpy()) for r, u in got]
+    for (p, c), (rel, reuse) in zip(inputs, got):
+        ref_rel, ref_reuse = dbp.cachedit_residual_diff(p, c, 0.04)
+        ref_rel, ref_reuse = ref_rel.cpu().numpy(), ref_reuse.cpu().numpy()
+        assert np.allclose(rel, ref_rel, rtol=1e-7, atol=0), (rel, ref_rel)
+        assert np.array_equal(reuse, ref_reuse)
+    # and the first input again, after the array holds the second call's sums
+    rel, reuse = dbp.cachedit_residual_diff_noalloc(*inputs[0], 0.04)
+    assert np.allclose(rel.cpu().numpy(), got[0][0], rtol=1e-7, atol=0)
+    assert np.array_equal(reuse.cpu().numpy(), got[0][1])
+
+
+@pytest.mark.gpu
+def test_noalloc_too_many_samples_is_a_clear_error():
+    _lib()
+    x = torch.zeros(65, 2, 64, dtype=torch.bfloat16, device="cuda:0")
+    with pytest.raises(dbp.DitError) as e:
+        dbp.cachedit_residual_diff_noalloc(x, x, 0.04)
+    assert e.value.status == -2
