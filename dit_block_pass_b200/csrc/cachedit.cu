@@ -7,10 +7,12 @@
 // allows it (0.04 conservative, 0.08 in the more aggressive stride mode).
 // The check is the relative L1 difference of two residual tensors.
 //
-// Design: a partial-sum kernel on a (G, B) grid streams prev and cur once;
-// thread sums are fp32 per 8-element vector (|cur - prev| of two bf16 values
-// is exact in fp32 unless their exponents are more than 16 apart) and fp64
-// above that.  Each CTA reduces with a fixed butterfly and writes its fp64
+// Design: a partial-sum kernel on a (G, B) grid streams prev and cur once,
+// 32 bytes per load when the rows allow it; G is a few device-fulls of CTAs
+// (more than fit at once, which let the scheduler interleave them);
+// thread sums are fp32 per 8- or 16-element vector (|cur - prev| of two bf16
+// values is exact in fp32 unless their exponents are more than 16 apart) and
+// fp64 above that.  Each CTA reduces with a fixed butterfly and writes its fp64
 // pair to the workspace as part[g][b][2].  A one-warp-per-sample kernel then
 // adds the G pairs in a fixed order and takes the decision in fp64.  There
 // are no floating-point atomics, so the result is identical run to run.
@@ -26,37 +28,72 @@ namespace {
 constexpr int kThreads = 256;
 constexpr int kUnroll = 4;
 constexpr int kSlotCap = 2048;  // partial-sum slots per sample in a workspace
+constexpr int kWaves = 4;       // partial CTAs per sample: this many device-fulls
 
+// Sum of |c - p| and |p| over the 8 (or 16) bf16 values of a vector pair,
+// in fp32.
+__device__ __forceinline__ void absdiff_sums(const uint4& pv, const uint4& cv, float& sn,
+                                             float& sd) {
+    float fp[8], fc[8];
+    unpack8(pv, fp);
+    unpack8(cv, fc);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        sn += fabsf(fc[i] - fp[i]);
+        sd += fabsf(fp[i]);
+    }
+}
+
+template <int E>
+struct CacheVec;
+template <>
+struct CacheVec<8> {
+    using T = uint4;
+    static __device__ __forceinline__ T load(const T* p) { return ld_stream(p); }
+    static __device__ __forceinline__ void sums(const T& p, const T& c, float& sn, float& sd) {
+        absdiff_sums(p, c, sn, sd);
+    }
+};
+template <>
+struct CacheVec<16> {
+    using T = u32x8;
+    static __device__ __forceinline__ T load(const T* p) { return ld_stream256(p); }
+    static __device__ __forceinline__ void sums(const T& p, const T& c, float& sn, float& sd) {
+        absdiff_sums(make_uint4(p.w[0], p.w[1], p.w[2], p.w[3]),
+                     make_uint4(c.w[0], c.w[1], c.w[2], c.w[3]), sn, sd);
+        absdiff_sums(make_uint4(p.w[4], p.w[5], p.w[6], p.w[7]),
+                     make_uint4(c.w[4], c.w[5], c.w[6], c.w[7]), sn, sd);
+    }
+};
+
+// Grid (G, B): CTA g of sample b sums vectors g*T + t + k*G*T of the
+// sample (T threads) and writes its fp64 pair to part[g][b][2].
+template <int E>
 __global__ void __launch_bounds__(kThreads)
-cachedit_partials_kernel(const uint4* __restrict__ prev, const uint4* __restrict__ cur,
+cachedit_partials_kernel(const void* __restrict__ prev_, const void* __restrict__ cur_,
                          int64_t nvs, double* __restrict__ part, int B) {
+    using V = CacheVec<E>;
+    using T = typename V::T;
     const int g = blockIdx.x, b = blockIdx.y, G = gridDim.x;
-    const uint4* P = prev + static_cast<int64_t>(b) * nvs;
-    const uint4* C = cur + static_cast<int64_t>(b) * nvs;
+    const T* P = static_cast<const T*>(prev_) + static_cast<int64_t>(b) * nvs;
+    const T* C = static_cast<const T*>(cur_) + static_cast<int64_t>(b) * nvs;
     const int64_t step = static_cast<int64_t>(G) * kThreads;
     double acc_n = 0.0, acc_d = 0.0;
     for (int64_t v = static_cast<int64_t>(g) * kThreads + threadIdx.x; v < nvs;
          v += kUnroll * step) {
-        uint4 pv[kUnroll], cv[kUnroll];
+        T pv[kUnroll], cv[kUnroll];
 #pragma unroll
         for (int u = 0; u < kUnroll; ++u) {
             if (v + u * step < nvs) {
-                pv[u] = ld_stream(P + v + u * step);
-                cv[u] = ld_stream(C + v + u * step);
+                pv[u] = V::load(P + v + u * step);
+                cv[u] = V::load(C + v + u * step);
             }
         }
 #pragma unroll
         for (int u = 0; u < kUnroll; ++u) {
             if (v + u * step < nvs) {
-                float fp[8], fc[8];
-                unpack8(pv[u], fp);
-                unpack8(cv[u], fc);
                 float sn = 0.0f, sd = 0.0f;
-#pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    sn += fabsf(fc[i] - fp[i]);
-                    sd += fabsf(fp[i]);
-                }
+                V::sums(pv[u], cv[u], sn, sd);
                 acc_n += static_cast<double>(sn);
                 acc_d += static_cast<double>(sd);
             }
@@ -112,11 +149,15 @@ __global__ void cachedit_finalize_kernel(const double* __restrict__ part, int R,
     }
 }
 
-int partial_slots(int B, int64_t nvs) {
+// Partial-sum slots per sample: `waves` times the CTAs that fit on the
+// device at once (more CTAs than fit lets the scheduler interleave them),
+// at most kSlotCap, at least 1.
+int partial_slots(int B, int64_t nvs, int waves) {
     const int sms = device_sm_count();
     if (sms <= 0) return 0;
-    const int occ = occupancy(reinterpret_cast<const void*>(cachedit_partials_kernel), kThreads, 0);
-    int64_t g = static_cast<int64_t>(sms) * occ / B;
+    const int occ =
+        occupancy(reinterpret_cast<const void*>(cachedit_partials_kernel<8>), kThreads, 0);
+    int64_t g = static_cast<int64_t>(sms) * occ * waves / B;
     const int64_t need = (nvs + kThreads - 1) / kThreads;
     if (g > need) g = need;
     if (g > kSlotCap) g = kSlotCap;
@@ -138,13 +179,18 @@ int run_partials(const uint16_t* prev, const uint16_t* cur, int B, int64_t N, in
                  void* workspace, size_t workspace_bytes, cudaStream_t stream, int* slots) {
     if (!workspace || !aligned16(workspace)) return DIT_ERR_WORKSPACE;
     if (workspace_bytes < cachedit_workspace_bytes(B, N, D)) return DIT_ERR_WORKSPACE;
-    const int64_t nvs = N * D / 8;
-    const int G = partial_slots(B, nvs);
+    // 32-byte vectors when every sample's rows allow them
+    const bool wide = D % 16 == 0 && aligned32(prev) && aligned32(cur);
+    const int64_t nvs = N * D / (wide ? 16 : 8);
+    const int G = partial_slots(B, nvs, kWaves);
     if (G < 1) return DIT_ERR_LAUNCH;
     dim3 grid(static_cast<unsigned>(G), static_cast<unsigned>(B));
-    cachedit_partials_kernel<<<grid, kThreads, 0, stream>>>(
-        reinterpret_cast<const uint4*>(prev), reinterpret_cast<const uint4*>(cur), nvs,
-        static_cast<double*>(workspace), B);
+    if (wide)
+        cachedit_partials_kernel<16><<<grid, kThreads, 0, stream>>>(
+            prev, cur, nvs, static_cast<double*>(workspace), B);
+    else
+        cachedit_partials_kernel<8><<<grid, kThreads, 0, stream>>>(
+            prev, cur, nvs, static_cast<double*>(workspace), B);
     *slots = G;
     return launch_status();
 }
@@ -258,15 +304,14 @@ extern "C" int cachedit_residual_diff_noalloc(const uint16_t* prev, const uint16
     double* scratch = scratch_address();
     if (!scratch) return DIT_ERR_LAUNCH;
     const int64_t nvs = N * D / 8;
-    const int G = partial_slots(B, nvs);
+    const int G = partial_slots(B, nvs, 1);
     if (G < 1) return DIT_ERR_LAUNCH;
     if (static_cast<int64_t>(G) * B > kStaticPairs) return DIT_ERR_WORKSPACE;
     // Every slot the finalize kernel reads is written by the partials kernel
     // of the same call, so the array needs no clearing between calls.
     dim3 grid(static_cast<unsigned>(G), static_cast<unsigned>(B));
-    cachedit_partials_kernel<<<grid, kThreads, 0, as_stream(stream)>>>(
-        reinterpret_cast<const uint4*>(prev), reinterpret_cast<const uint4*>(cur), nvs, scratch,
-        B);
+    cachedit_partials_kernel<8><<<grid, kThreads, 0, as_stream(stream)>>>(prev, cur, nvs, scratch,
+                                                                         B);
     if ((st = launch_status())) return st;
     cachedit_finalize_kernel<<<B, 32, 0, as_stream(stream)>>>(scratch, G, B, threshold, nullptr,
                                                               rel_out, reuse_out);

@@ -29,7 +29,8 @@ __device__ __forceinline__ void st_stream(uint4* p, const uint4& v) {
                  : "memory");
 }
 
-// 256-bit forms (sm_100): 32-byte aligned, eight 32-bit words.
+// 256-bit forms (sm_100): 32-byte aligned, eight 32-bit words.  Loads are
+// evict-first with a 256-byte L2 fetch hint (whole DRAM bursts).
 struct alignas(32) u32x8 {
     uint32_t w[8];
 };
@@ -37,7 +38,8 @@ struct alignas(32) u32x8 {
 __device__ __forceinline__ u32x8 ld_stream256(const void* p) {
     u32x8 v;
     asm volatile(
-        "ld.global.nc.L1::no_allocate.L2::evict_first.v8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+        "ld.global.nc.L1::no_allocate.L2::evict_first.L2::256B.v8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, "
+        "[%8];"
         : "=r"(v.w[0]), "=r"(v.w[1]), "=r"(v.w[2]), "=r"(v.w[3]), "=r"(v.w[4]), "=r"(v.w[5]),
           "=r"(v.w[6]), "=r"(v.w[7])
         : "l"(p));

@@ -2,25 +2,27 @@
 // embedding, in place, in one pass over HBM.
 //
 // The LMSYS report summary at news.cocoloop.cn ("minimax-h3-sglang-h200"),
-// section "Só com três camadas de aceleração
-// somadas chega-se a 6 vezes": "QK RMSNorm com 3D RoPE" is one fused operator;
-// "SGLang acelera MiniMax-H3 em GPUs H200", first paragraph, lists QK RMSNorm
-// and 3D RoPE among the fused low-level operations.
+// section "Só com três camadas de aceleração somadas chega-se a 6 vezes":
+// "QK RMSNorm com 3D RoPE" is one fused operator; "SGLang acelera MiniMax-H3
+// em GPUs H200", first paragraph, lists QK RMSNorm and 3D RoPE among the
+// fused low-level operations.
 //
-// Design: one warp per token.  A token row of H heads x hd is H*hd/8
-// consecutive 16-byte vectors; warp pass i reads vectors 32*i + lane, so each
-// load instruction covers 512 contiguous bytes and a head occupies hd/8
-// adjacent lanes.  The head's sum of squares is a shuffle reduction inside
-// that lane group.  A lane always holds the same 4 rotation pairs of a head
+// Design: one warp per token, one-shot grid (a CTA of 8 warps takes 8 tokens
+// and exits; on B200 this sustained more HBM bandwidth than persistent CTAs).
+// A token row of H heads x hd is H*hd/8 consecutive 16-byte vectors; warp
+// pass j reads vectors 32*j + lane, so each load instruction covers 512
+// contiguous bytes and a head occupies hd/8 adjacent lanes.  The head's sum
+// of squares is a shuffle reduction inside that lane group.  The q row is
+// loaded into registers while the k row is copied into the warp's
+// shared-memory stage with cp.async, so both are in flight before any
+// arithmetic.  A lane always holds the same 4 rotation pairs of a head
 // (pairs 4*(lane mod hd/8) .. +3), so it computes their 4 angles once per
-// token and reuses them for every head of q and k.  Frequencies are fp64
-// (computed once per thread), angles pos*omega are formed and reduced modulo
-// 2*pi in fp64, and sin/cos are taken in fp32 on the reduced angle, which
-// keeps the rotation accurate to a few fp32 ulp for positions in the hundreds.
-// q and k stream through a per-warp, kStages-deep cp.async pipeline of
-// kChunk lane-vectors per stage (each lane copies and later reads back only
-// its own vectors, so no barrier is needed): the next chunks are in flight
-// while the current one is normalised and rotated.  HBM bound.
+// token and reuses them for every head of q and k.  Frequencies and the
+// angles pos*omega are formed and reduced modulo 2*pi in fp64, and sin/cos
+// are taken in fp32 on the reduced angle, which keeps the rotation accurate
+// to a few fp32 ulp for positions in the hundreds.  The RMSNorm weight is
+// folded into the rotation coefficients once per token and tensor.  HBM
+// bound.
 #include "common.cuh"
 
 namespace dit {
@@ -28,9 +30,6 @@ namespace {
 
 constexpr int kWarps = 8;
 constexpr int kThreads = kWarps * 32;
-constexpr int kChunk = 10;   // lane-vectors per pipeline stage
-constexpr int kStages = 2;   // cp.async stages per warp
-constexpr size_t kSmem = static_cast<size_t>(kWarps) * kStages * kChunk * 32 * sizeof(uint4);
 
 struct QKParams {
     uint4* t0;              // first tensor processed (q, or k when q is NULL)
@@ -60,158 +59,146 @@ __device__ __forceinline__ void cp_async16(void* smem_dst, const void* gsrc) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d), "l"(gsrc) : "memory");
 }
 
-// Work of one warp is a sequence of jobs: chunk c (0 .. cpt-1) of each of
-// the warp's tokens in turn.  Chunks 0 .. cq-1 cover the q row and chunks
-// cq .. 2cq-1 the k row, kChunk lane-vectors each (lane-vector i of a row is
-// its vector i * 32 + lane), so the tensor, its weights and its row pointer
-// are uniform inside a chunk.
-template <int HD>
-__global__ void __launch_bounds__(kThreads, 2)
+// One warp per token (one-shot grid: a CTA takes 8 tokens and exits).  The
+// first tensor's row goes to registers and the second's to the warp's
+// shared-memory stage with cp.async, both issued before any arithmetic;
+// lane-vector j of a row is its vector j * 32 + lane.
+template <int HD, int NVL>
+__device__ __forceinline__ void qk_row(const uint4 (&v)[NVL], uint4* row, int nvr, int lane,
+                                       const float (&A)[4], const float (&Bn)[4],
+                                       const float (&C)[4], const float (&Dd)[4], float eps,
+                                       float inv_hd) {
+    constexpr int LPH = HD / 8;
+#pragma unroll
+    for (int j = 0; j < NVL; ++j) {
+        const int idx = j * 32 + lane;
+        float f[8];
+        unpack8(v[j], f);
+        float ss = 0.0f;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) ss = __fmaf_rn(f[i], f[i], ss);
+#pragma unroll
+        for (int o = LPH / 2; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+        const float inv = rsqrtf(__fmaf_rn(ss, inv_hd, eps));
+        float o8[8];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            o8[2 * k] = inv * __fmaf_rn(f[2 * k], A[k], f[2 * k + 1] * Bn[k]);
+            o8[2 * k + 1] = inv * __fmaf_rn(f[2 * k], C[k], f[2 * k + 1] * Dd[k]);
+        }
+        if (idx < nvr) st_stream(row + idx, pack8(o8));
+    }
+}
+
+template <int HD, int NVL>
+__global__ void __launch_bounds__(kThreads, (NVL <= 20 ? 2 : 1))
 qk_rmsnorm_rope3d_kernel(QKParams p) {
     constexpr int LPH = HD / 8;             // lanes per head
     extern __shared__ uint4 qk_stage[];
     const int lane = threadIdx.x & 31;
     const int warp = threadIdx.x >> 5;
+    const int64_t tok = static_cast<int64_t>(blockIdx.x) * kWarps + warp;
+    if (tok >= p.rows) return;
     const int sub = lane % LPH;             // this lane's vector within a head
-    uint4* stage = qk_stage + warp * (kStages * kChunk * 32) + lane;
+    uint4* row0 = p.t0 + tok * p.stride_v;
+    uint4* row1 = p.t1 ? p.t1 + tok * p.stride_v : nullptr;
+    uint4* stage = qk_stage + warp * (NVL * 32) + lane;
+    if (row1) {
+#pragma unroll
+        for (int j = 0; j < NVL; ++j)
+            if (j * 32 + lane < p.nvr) cp_async16(stage + j * 32, row1 + j * 32 + lane);
+        asm volatile("cp.async.commit_group;" ::: "memory");
+    }
+    uint4 v[NVL];
+#pragma unroll
+    for (int j = 0; j < NVL; ++j)
+        v[j] = (j * 32 + lane < p.nvr) ? ld_inplace(row0 + j * 32 + lane) : make_uint4(0, 0, 0, 0);
 
-    // this lane's rotation pairs: p = 4*sub + j
-    int axis[4];
-    double omega[4];
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-        const int pr = 4 * sub + j;
-        int i, P;
-        if (pr < p.pt) {
-            axis[j] = 0; i = pr; P = p.pt;
-        } else if (pr < p.pt + p.ph) {
-            axis[j] = 1; i = pr - p.pt; P = p.ph;
-        } else {
-            axis[j] = 2; i = pr - p.pt - p.ph; P = p.pw;
-        }
-        omega[j] = pow(p.theta, -2.0 * static_cast<double>(i) / (2.0 * static_cast<double>(P)));
+    // token position and this lane's 4 rotation angles (pairs 4*sub + k)
+    int pos3[3];
+    if (p.pos) {
+        pos3[0] = p.pos[3 * tok + 0];
+        pos3[1] = p.pos[3 * tok + 1];
+        pos3[2] = p.pos[3 * tok + 2];
+    } else {
+        // grid index < 2^31 (checked on the host)
+        const int hw = p.Hg * p.Wg;
+        const int g = static_cast<int>(p.pos_offset + tok % p.N);
+        const int t = g / hw;
+        const int rem = g - t * hw;
+        const int h = rem / p.Wg;
+        pos3[0] = t;
+        pos3[1] = h;
+        pos3[2] = rem - h * p.Wg;
     }
-    float w0[8], w1[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        w0[i] = w_at(p.w0, p.w_dtype, 8 * sub + i);
-        w1[i] = p.t1 ? w_at(p.w1, p.w_dtype, 8 * sub + i) : 0.0f;
-    }
-    const float inv_hd = 1.0f / static_cast<float>(HD);
-    const int nvl = (p.nvr + 31) / 32;              // lane-vectors per row
-    const int cq = (nvl + kChunk - 1) / kChunk;     // chunks per row
-    const int cpt = (p.t1 ? 2 : 1) * cq;            // chunks per token
-    const int hw = p.Hg * p.Wg;
     const double kTwoPi = 6.283185307179586;
     const double kInvTwoPi = 0.15915494309189535;
-    const int64_t wstep = static_cast<int64_t>(gridDim.x) * kWarps;
-
-    // copy chunk `chunk` of token `tok` into stage slot `slot` (one commit group)
-    auto issue = [&](int64_t tok, int chunk, int slot) {
-        if (tok < p.rows) {
-            const int tensor = chunk >= cq ? 1 : 0;
-            const int first = (chunk - tensor * cq) * kChunk;
-            const uint4* row = (tensor ? p.t1 : p.t0) + tok * p.stride_v;
-            uint4* dst = stage + slot * (kChunk * 32);
-#pragma unroll
-            for (int u = 0; u < kChunk; ++u) {
-                const int idx = (first + u) * 32 + lane;
-                if (first + u < nvl && idx < p.nvr) cp_async16(dst + u * 32, row + idx);
-            }
-        }
-        asm volatile("cp.async.commit_group;" ::: "memory");
-    };
-
-    int64_t itok = static_cast<int64_t>(blockIdx.x) * kWarps + warp, ctok = itok;
-    int ichunk = 0, cchunk = 0, islot = 0, cslot = 0;
-#pragma unroll
-    for (int s = 0; s < kStages - 1; ++s) {
-        issue(itok, ichunk, islot);
-        if (++ichunk == cpt) { ichunk = 0; itok += wstep; }
-        islot = islot + 1 == kStages ? 0 : islot + 1;
-    }
     float cs[4], sn[4];
-    while (ctok < p.rows) {
-        issue(itok, ichunk, islot);
-        if (++ichunk == cpt) { ichunk = 0; itok += wstep; }
-        islot = islot + 1 == kStages ? 0 : islot + 1;
-        // groups complete in order: all but the newest kStages-1 are done
-        asm volatile("cp.async.wait_group %0;" ::"n"(kStages - 1) : "memory");
-        if (cchunk == 0) {
-            int pos3[3];
-            if (p.pos) {
-                pos3[0] = p.pos[3 * ctok + 0];
-                pos3[1] = p.pos[3 * ctok + 1];
-                pos3[2] = p.pos[3 * ctok + 2];
-            } else {
-                // grid index < 2^31 (checked on the host)
-                const int g = static_cast<int>(p.pos_offset + ctok % p.N);
-                const int t = g / hw;
-                const int rem = g - t * hw;
-                const int h = rem / p.Wg;
-                pos3[0] = t;
-                pos3[1] = h;
-                pos3[2] = rem - h * p.Wg;
-            }
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const int pa = axis[j] == 0 ? pos3[0] : (axis[j] == 1 ? pos3[1] : pos3[2]);
-                const double phi = static_cast<double>(pa) * omega[j];
-                const double kk = rint(phi * kInvTwoPi);
-                const float red = static_cast<float>(fma(-kk, kTwoPi, phi));
-                sincosf(red, &sn[j], &cs[j]);
-            }
+    for (int k = 0; k < 4; ++k) {
+        const int pr = 4 * sub + k;
+        int i, P, pa;
+        if (pr < p.pt) {
+            i = pr; P = p.pt; pa = pos3[0];
+        } else if (pr < p.pt + p.ph) {
+            i = pr - p.pt; P = p.ph; pa = pos3[1];
+        } else {
+            i = pr - p.pt - p.ph; P = p.pw; pa = pos3[2];
         }
-        const int tensor = cchunk >= cq ? 1 : 0;
-        const int first = (cchunk - tensor * cq) * kChunk;
-        uint4* row = (tensor ? p.t1 : p.t0) + ctok * p.stride_v;
-        // rotation with the weight folded in: (u0, u1) = inv * (f0 w0, f1 w1)
-        //   out0 = inv * (f0 * w0 cos - f1 * w1 sin), out1 = inv * (f0 * w0 sin + f1 * w1 cos)
-        float A[4], Bn[4], C[4], Dd[4];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const float wa = tensor ? w1[2 * j] : w0[2 * j];
-            const float wb = tensor ? w1[2 * j + 1] : w0[2 * j + 1];
-            A[j] = wa * cs[j];
-            Bn[j] = -(wb * sn[j]);
-            C[j] = wa * sn[j];
-            Dd[j] = wb * cs[j];
-        }
-        const uint4* src = stage + cslot * (kChunk * 32);
-#pragma unroll
-        for (int u = 0; u < kChunk; ++u) {
-            const int idx = (first + u) * 32 + lane;
-            const bool valid = first + u < nvl && idx < p.nvr;
-            float f[8];
-            unpack8(valid ? src[u * 32] : make_uint4(0, 0, 0, 0), f);
-            float ss = 0.0f;
-#pragma unroll
-            for (int i = 0; i < 8; ++i) ss = __fmaf_rn(f[i], f[i], ss);
-#pragma unroll
-            for (int o = LPH / 2; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-            const float inv = rsqrtf(__fmaf_rn(ss, inv_hd, p.eps));
-            float o8[8];
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                o8[2 * j] = inv * __fmaf_rn(f[2 * j], A[j], f[2 * j + 1] * Bn[j]);
-                o8[2 * j + 1] = inv * __fmaf_rn(f[2 * j], C[j], f[2 * j + 1] * Dd[j]);
-            }
-            if (valid) st_stream(row + idx, pack8(o8));
-        }
-        if (++cchunk == cpt) { cchunk = 0; ctok += wstep; }
-        cslot = cslot + 1 == kStages ? 0 : cslot + 1;
+        const double omega =
+            pow(p.theta, -2.0 * static_cast<double>(i) / (2.0 * static_cast<double>(P)));
+        const double phi = static_cast<double>(pa) * omega;
+        const double kk = rint(phi * kInvTwoPi);
+        sincosf(static_cast<float>(fma(-kk, kTwoPi, phi)), &sn[k], &cs[k]);
     }
-    asm volatile("cp.async.wait_all;" ::: "memory");
+    // rotation with the weight folded in: (u0, u1) = inv * (f0 w0, f1 w1)
+    //   out0 = inv * (f0 w0 cos - f1 w1 sin), out1 = inv * (f0 w0 sin + f1 w1 cos)
+    const float inv_hd = 1.0f / static_cast<float>(HD);
+    float A[4], Bn[4], C[4], Dd[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        const float wa = w_at(p.w0, p.w_dtype, 8 * sub + 2 * k);
+        const float wb = w_at(p.w0, p.w_dtype, 8 * sub + 2 * k + 1);
+        A[k] = wa * cs[k]; Bn[k] = -(wb * sn[k]); C[k] = wa * sn[k]; Dd[k] = wb * cs[k];
+    }
+    qk_row<HD, NVL>(v, row0, p.nvr, lane, A, Bn, C, Dd, p.eps, inv_hd);
+    if (row1) {
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const float wa = w_at(p.w1, p.w_dtype, 8 * sub + 2 * k);
+            const float wb = w_at(p.w1, p.w_dtype, 8 * sub + 2 * k + 1);
+            A[k] = wa * cs[k]; Bn[k] = -(wb * sn[k]); C[k] = wa * sn[k]; Dd[k] = wb * cs[k];
+        }
+        asm volatile("cp.async.wait_group 0;" ::: "memory");
+#pragma unroll
+        for (int j = 0; j < NVL; ++j)
+            v[j] = (j * 32 + lane < p.nvr) ? stage[j * 32] : make_uint4(0, 0, 0, 0);
+        qk_row<HD, NVL>(v, row1, p.nvr, lane, A, Bn, C, Dd, p.eps, inv_hd);
+    }
 }
 
 using QKKernel = void (*)(QKParams);
 
-QKKernel pick(int hd) {
+template <int HD>
+QKKernel pick_nvl(int nvl, int* nvl_out) {
+#define DIT_NVL_CASE(V)                                   \
+    if (nvl <= V) {                                       \
+        *nvl_out = V;                                     \
+        return qk_rmsnorm_rope3d_kernel<HD, V>;           \
+    }
+    DIT_NVL_CASE(1) DIT_NVL_CASE(2) DIT_NVL_CASE(3) DIT_NVL_CASE(4) DIT_NVL_CASE(6)
+    DIT_NVL_CASE(8) DIT_NVL_CASE(10) DIT_NVL_CASE(12) DIT_NVL_CASE(16) DIT_NVL_CASE(20)
+    DIT_NVL_CASE(24) DIT_NVL_CASE(32)
+#undef DIT_NVL_CASE
+    return nullptr;
+}
+
+QKKernel pick(int hd, int nvl, int* nvl_out) {
     switch (hd) {
-        case 32: return qk_rmsnorm_rope3d_kernel<32>;
-        case 64: return qk_rmsnorm_rope3d_kernel<64>;
-        case 128: return qk_rmsnorm_rope3d_kernel<128>;
-        case 256: return qk_rmsnorm_rope3d_kernel<256>;
+        case 32: return pick_nvl<32>(nvl, nvl_out);
+        case 64: return pick_nvl<64>(nvl, nvl_out);
+        case 128: return pick_nvl<128>(nvl, nvl_out);
+        case 256: return pick_nvl<256>(nvl, nvl_out);
         default: return nullptr;
     }
 }
@@ -255,12 +242,11 @@ extern "C" int dit_qk_rmsnorm_rope3d(uint16_t* q, uint16_t* k, int64_t row_strid
     using namespace dit;
     if (w_dtype != DIT_F32 && w_dtype != DIT_BF16) return DIT_ERR_DTYPE;
     if (B < 0 || N < 0 || H < 1) return DIT_ERR_SHAPE;
-    QKKernel kernel = pick(hd);
-    if (!kernel) return DIT_ERR_SHAPE;
+    if (hd != 32 && hd != 64 && hd != 128 && hd != 256) return DIT_ERR_SHAPE;
     if (pairs_t < 1 || pairs_h < 1 || pairs_w < 1 || pairs_t + pairs_h + pairs_w != hd / 2)
         return DIT_ERR_SHAPE;
     const int64_t width = static_cast<int64_t>(H) * hd;
-    if (width > (int64_t(1) << 30) || row_stride < width) return DIT_ERR_SHAPE;
+    if (width > DIT_MAX_D || row_stride < width) return DIT_ERR_SHAPE;
     if (row_stride % 8) return DIT_ERR_ALIGN;
     if (!(theta > 0.0) || theta > 1e300 || !(eps >= 0.0) || eps > 1e30) return DIT_ERR_VALUE;
     const int64_t rows = static_cast<int64_t>(B) * N;
@@ -300,15 +286,16 @@ extern "C" int dit_qk_rmsnorm_rope3d(uint16_t* q, uint16_t* k, int64_t row_strid
     p.theta = theta;
     p.eps = static_cast<float>(eps);
 
-    const int sms = device_sm_count();
-    if (sms <= 0) return DIT_ERR_LAUNCH;
-    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(kSmem)) != cudaSuccess)
+    int nvl = 0;
+    QKKernel kernel = pick(hd, (p.nvr + 31) / 32, &nvl);
+    if (!kernel) return DIT_ERR_SHAPE;
+    const size_t smem = p.t1 ? static_cast<size_t>(kWarps) * nvl * 32 * sizeof(uint4) : 0;
+    if (smem > 48 * 1024 &&
+        cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem)) != cudaSuccess)
         return DIT_ERR_LAUNCH;
-    const int occ = occupancy(reinterpret_cast<const void*>(kernel), kThreads, kSmem);
-    int64_t blocks = static_cast<int64_t>(sms) * occ;
-    const int64_t need = (rows + kWarps - 1) / kWarps;
-    if (blocks > need) blocks = need;
-    kernel<<<static_cast<unsigned>(blocks), kThreads, kSmem, as_stream(stream)>>>(p);
+    const int64_t ctas = (rows + kWarps - 1) / kWarps;
+    if (ctas > 0x7FFFFFFF) return DIT_ERR_SHAPE;
+    kernel<<<static_cast<unsigned>(ctas), kThreads, smem, as_stream(stream)>>>(p);
     return launch_status();
 }

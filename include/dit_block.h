@@ -161,9 +161,9 @@ int dit_qk_rmsnorm_rope3d(uint16_t* q, uint16_t* k, int64_t row_stride,
  *   Per sample b:  rel_b   = sum_{n,d} |cur - prev| / sum_{n,d} |prev|
  *                  reuse_b = rel_b < threshold       (strict)
  *   0/0 reads as rel = 0 (identical residuals are reusable); x/0 as +inf.
- *   |cur - prev| and |prev| are summed in fp32 per 8-element vector and in
- *   fp64 above that, in a fixed order: the result is deterministic run to run
- *   on a given device.
+ *   |cur - prev| and |prev| are summed in fp32 per 8- or 16-element vector
+ *   and in fp64 above that, in a fixed order: the result is deterministic run
+ *   to run on a given device.
  * prev, cur   [B, N, D] bf16, 16-byte aligned.  D multiple of 8.
  * rel_out     device [B] double;  reuse_out device [B] uint8 (0 or 1).
  * workspace   device scratch of at least cachedit_workspace_bytes(B, N, D)
