@@ -352,7 +352,9 @@ RowLaunch pick_kernel(bool gated, int Dv) {
 int launch_rows(const RowParams& p, bool gated, int B, cudaStream_t stream) {
     const RowLaunch L = pick_kernel(gated, p.Dv);
     if (!L.kernel) return DIT_ERR_SHAPE;
-    if (L.smem > 48 * 1024 &&
+    // opt in whenever dynamic shared memory is used (static arrays count
+    // toward the 48 KB default too)
+    if (L.smem > 0 &&
         cudaFuncSetAttribute(L.kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(L.smem)) != cudaSuccess)
         return DIT_ERR_LAUNCH;

@@ -17,10 +17,11 @@
 // shared-memory stage with cp.async, so both are in flight before any
 // arithmetic.  A lane always holds the same 4 rotation pairs of a head
 // (pairs 4*(lane mod hd/8) .. +3), so it computes their 4 angles once per
-// token and reuses them for every head of q and k.  Frequencies and the
-// angles pos*omega are formed and reduced modulo 2*pi in fp64, and sin/cos
-// are taken in fp32 on the reduced angle, which keeps the rotation accurate
-// to a few fp32 ulp for positions in the hundreds.  The RMSNorm weight is
+// token and reuses them for every head of q and k.  The hd/2 frequencies
+// are computed in fp64 once per CTA into shared memory while the rows load;
+// the angles pos*omega are formed and reduced modulo 2*pi in fp64, and
+// sin/cos are taken in fp32 on the reduced angle, which keeps the rotation
+// accurate to a few fp32 ulp for positions in the hundreds.  The RMSNorm weight is
 // folded into the rotation coefficients once per token and tensor.  HBM
 // bound.
 #include "common.cuh"
@@ -95,24 +96,43 @@ __global__ void __launch_bounds__(kThreads, (NVL <= 20 ? 2 : 1))
 qk_rmsnorm_rope3d_kernel(QKParams p) {
     constexpr int LPH = HD / 8;             // lanes per head
     extern __shared__ uint4 qk_stage[];
+    __shared__ double s_omega[HD / 2];      // frequency of each rotation pair
     const int lane = threadIdx.x & 31;
     const int warp = threadIdx.x >> 5;
     const int64_t tok = static_cast<int64_t>(blockIdx.x) * kWarps + warp;
-    if (tok >= p.rows) return;
+    const bool live = tok < p.rows;
     const int sub = lane % LPH;             // this lane's vector within a head
     uint4* row0 = p.t0 + tok * p.stride_v;
     uint4* row1 = p.t1 ? p.t1 + tok * p.stride_v : nullptr;
     uint4* stage = qk_stage + warp * (NVL * 32) + lane;
-    if (row1) {
+    uint4 v[NVL];
+    if (live) {
+        if (row1) {
+#pragma unroll
+            for (int j = 0; j < NVL; ++j)
+                if (j * 32 + lane < p.nvr) cp_async16(stage + j * 32, row1 + j * 32 + lane);
+            asm volatile("cp.async.commit_group;" ::: "memory");
+        }
 #pragma unroll
         for (int j = 0; j < NVL; ++j)
-            if (j * 32 + lane < p.nvr) cp_async16(stage + j * 32, row1 + j * 32 + lane);
-        asm volatile("cp.async.commit_group;" ::: "memory");
+            v[j] = (j * 32 + lane < p.nvr) ? ld_inplace(row0 + j * 32 + lane)
+                                           : make_uint4(0, 0, 0, 0);
     }
-    uint4 v[NVL];
-#pragma unroll
-    for (int j = 0; j < NVL; ++j)
-        v[j] = (j * 32 + lane < p.nvr) ? ld_inplace(row0 + j * 32 + lane) : make_uint4(0, 0, 0, 0);
+    // pair pr of an axis with P pairs, local index i: omega = theta^(-2i/(2P)),
+    // once per CTA while the rows are in flight
+    for (int pr = threadIdx.x; pr < HD / 2; pr += kThreads) {
+        int i, P;
+        if (pr < p.pt) {
+            i = pr; P = p.pt;
+        } else if (pr < p.pt + p.ph) {
+            i = pr - p.pt; P = p.ph;
+        } else {
+            i = pr - p.pt - p.ph; P = p.pw;
+        }
+        s_omega[pr] = pow(p.theta, -2.0 * static_cast<double>(i) / (2.0 * static_cast<double>(P)));
+    }
+    __syncthreads();
+    if (!live) return;
 
     // token position and this lane's 4 rotation angles (pairs 4*sub + k)
     int pos3[3];
@@ -137,17 +157,8 @@ qk_rmsnorm_rope3d_kernel(QKParams p) {
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
         const int pr = 4 * sub + k;
-        int i, P, pa;
-        if (pr < p.pt) {
-            i = pr; P = p.pt; pa = pos3[0];
-        } else if (pr < p.pt + p.ph) {
-            i = pr - p.pt; P = p.ph; pa = pos3[1];
-        } else {
-            i = pr - p.pt - p.ph; P = p.pw; pa = pos3[2];
-        }
-        const double omega =
-            pow(p.theta, -2.0 * static_cast<double>(i) / (2.0 * static_cast<double>(P)));
-        const double phi = static_cast<double>(pa) * omega;
+        const int pa = pr < p.pt ? pos3[0] : (pr < p.pt + p.ph ? pos3[1] : pos3[2]);
+        const double phi = static_cast<double>(pa) * s_omega[pr];
         const double kk = rint(phi * kInvTwoPi);
         sincosf(static_cast<float>(fma(-kk, kTwoPi, phi)), &sn[k], &cs[k]);
     }
@@ -290,7 +301,9 @@ extern "C" int dit_qk_rmsnorm_rope3d(uint16_t* q, uint16_t* k, int64_t row_strid
     QKKernel kernel = pick(hd, (p.nvr + 31) / 32, &nvl);
     if (!kernel) return DIT_ERR_SHAPE;
     const size_t smem = p.t1 ? static_cast<size_t>(kWarps) * nvl * 32 * sizeof(uint4) : 0;
-    if (smem > 48 * 1024 &&
+    // opt in whenever dynamic shared memory is used: with the static
+    // frequency table the total can pass the 48 KB default
+    if (smem > 0 &&
         cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(smem)) != cudaSuccess)
         return DIT_ERR_LAUNCH;

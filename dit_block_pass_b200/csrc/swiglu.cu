@@ -72,21 +72,28 @@ struct Vec<16> {
 // b*T*U + u*T + t, loads first, then the U results.
 template <int E, int U>
 __global__ void __launch_bounds__(kThreads)
-swiglu_kernel(const void* __restrict__ in_, void* __restrict__ out_, int64_t Fv, int64_t total) {
+swiglu_kernel(const void* __restrict__ in_, void* __restrict__ out_, int64_t Fv, int64_t total,
+              int64_t step_r, int64_t step_c) {
     using V = Vec<E>;
     using T = typename V::T;
     const T* in = static_cast<const T*>(in_);
     T* out = static_cast<T*>(out_);
     const int64_t v0 = static_cast<int64_t>(blockIdx.x) * (kThreads * U) + threadIdx.x;
+    // (row, col) of v0 + u*kThreads, advanced by (step_r, step_c) = divmod(kThreads, Fv)
+    int64_t row = v0 / Fv, col = v0 - row * Fv;
     T a[U], b[U];
 #pragma unroll
     for (int u = 0; u < U; ++u) {
-        const int64_t v = v0 + u * kThreads;
-        if (v < total) {
-            const int64_t row = v / Fv;
-            const T* src = in + row * 2 * Fv + (v - row * Fv);
+        if (v0 + u * kThreads < total) {
+            const T* src = in + row * 2 * Fv + col;
             a[u] = V::load(src);
             b[u] = V::load(src + Fv);
+        }
+        row += step_r;
+        col += step_c;
+        if (col >= Fv) {
+            col -= Fv;
+            ++row;
         }
     }
 #pragma unroll
@@ -119,6 +126,7 @@ extern "C" int dit_swiglu(const uint16_t* in, uint16_t* out, int64_t M, int F, v
     auto kernel = wide ? swiglu_kernel<16, kUnroll> : swiglu_kernel<8, kUnroll>;
     const int64_t blocks = (total + kThreads * kUnroll - 1) / (kThreads * kUnroll);
     if (blocks > 0x7FFFFFFF) return DIT_ERR_SHAPE;
-    kernel<<<static_cast<unsigned>(blocks), kThreads, 0, as_stream(stream)>>>(in, out, Fv, total);
+    kernel<<<static_cast<unsigned>(blocks), kThreads, 0, as_stream(stream)>>>(
+        in, out, Fv, total, kThreads / Fv, kThreads % Fv);
     return launch_status();
 }
