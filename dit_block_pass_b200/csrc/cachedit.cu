@@ -13,7 +13,7 @@
 // thread sums are fp32 per 8- or 16-element vector (|cur - prev| of two bf16
 // values is exact in fp32 unless their exponents are more than 16 apart) and
 // fp64 above that.  Each CTA reduces with a fixed butterfly and writes its fp64
-// pair to the workspace as part[g][b][2].  A one-warp-per-sample kernel then
+// pair to the workspace as part[g][b][2].  A one-CTA-per-sample kernel then
 // adds the G pairs in a fixed order and takes the decision in fp64.  There
 // are no floating-point atomics, so the result is identical run to run.
 #include <math.h>
@@ -121,20 +121,36 @@ cachedit_partials_kernel(const void* __restrict__ prev_, const void* __restrict_
     }
 }
 
-// One warp per sample: add R partial pairs (part[r][b][2]) lane-strided and
-// through a fixed butterfly, then write the sums and/or the decision.
-__global__ void cachedit_finalize_kernel(const double* __restrict__ part, int R, int B,
-                                         double threshold, double* sums_out, double* rel_out,
-                                         uint8_t* reuse_out) {
-    const int b = blockIdx.x, lane = threadIdx.x;
+// One CTA of kThreads per sample: thread t adds partial pairs t, t + T, ...
+// (part[r][b][2]) in order, then the CTA combines the thread sums through a
+// fixed butterfly and a fixed warp order, and thread 0 writes the sums and/or
+// the decision.  The order depends only on R, so equal inputs give equal bits.
+__global__ void __launch_bounds__(kThreads)
+cachedit_finalize_kernel(const double* __restrict__ part, int R, int B, double threshold,
+                         double* sums_out, double* rel_out, uint8_t* reuse_out) {
+    const int b = blockIdx.x;
     double n = 0.0, d = 0.0;
-    for (int r = lane; r < R; r += 32) {
+    for (int r = threadIdx.x; r < R; r += kThreads) {
         n += part[(static_cast<int64_t>(r) * B + b) * 2];
         d += part[(static_cast<int64_t>(r) * B + b) * 2 + 1];
     }
     n = warp_sum(n);
     d = warp_sum(d);
+    __shared__ double sh[2][kThreads / 32];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     if (lane == 0) {
+        sh[0][warp] = n;
+        sh[1][warp] = d;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        n = 0.0;
+        d = 0.0;
+#pragma unroll
+        for (int w = 0; w < kThreads / 32; ++w) {
+            n += sh[0][w];
+            d += sh[1][w];
+        }
         if (sums_out) {
             sums_out[2 * b] = n;
             sums_out[2 * b + 1] = d;
@@ -217,7 +233,7 @@ extern "C" int cachedit_residual_diff(const uint16_t* prev, const uint16_t* cur,
     int G = 0;
     if ((st = run_partials(prev, cur, B, N, D, workspace, workspace_bytes, as_stream(stream), &G)))
         return st;
-    cachedit_finalize_kernel<<<B, 32, 0, as_stream(stream)>>>(
+    cachedit_finalize_kernel<<<B, kThreads, 0, as_stream(stream)>>>(
         static_cast<const double*>(workspace), G, B, threshold, nullptr, rel_out, reuse_out);
     return launch_status();
 }
@@ -232,7 +248,7 @@ extern "C" int cachedit_residual_sums(const uint16_t* prev, const uint16_t* cur,
     int G = 0;
     if ((st = run_partials(prev, cur, B, N, D, workspace, workspace_bytes, as_stream(stream), &G)))
         return st;
-    cachedit_finalize_kernel<<<B, 32, 0, as_stream(stream)>>>(
+    cachedit_finalize_kernel<<<B, kThreads, 0, as_stream(stream)>>>(
         static_cast<const double*>(workspace), G, B, 0.0, sums_out, nullptr, nullptr);
     return launch_status();
 }
@@ -244,7 +260,7 @@ extern "C" int cachedit_decide(const double* sums, int R, int B, double threshol
     if (R < 1 || B < 1 || B > 65535) return DIT_ERR_SHAPE;
     if (reinterpret_cast<uintptr_t>(sums) % 8) return DIT_ERR_ALIGN;
     if (isnan(threshold)) return DIT_ERR_VALUE;
-    cachedit_finalize_kernel<<<B, 32, 0, dit::as_stream(stream)>>>(sums, R, B, threshold, nullptr,
+    cachedit_finalize_kernel<<<B, kThreads, 0, dit::as_stream(stream)>>>(sums, R, B, threshold, nullptr,
                                                                   rel_out, reuse_out);
     return launch_status();
 }
@@ -313,7 +329,7 @@ extern "C" int cachedit_residual_diff_noalloc(const uint16_t* prev, const uint16
     cachedit_partials_kernel<8><<<grid, kThreads, 0, as_stream(stream)>>>(prev, cur, nvs, scratch,
                                                                          B);
     if ((st = launch_status())) return st;
-    cachedit_finalize_kernel<<<B, 32, 0, as_stream(stream)>>>(scratch, G, B, threshold, nullptr,
+    cachedit_finalize_kernel<<<B, kThreads, 0, as_stream(stream)>>>(scratch, G, B, threshold, nullptr,
                                                               rel_out, reuse_out);
     return launch_status();
 }
