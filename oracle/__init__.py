@@ -60,6 +60,9 @@ class Oracle:
         L.dito_grid_positions.argtypes = [_int, _int, _int, _i64, _i64, _i32p]
         L.dito_qk_rmsnorm_rope3d.argtypes = [_u16p, _i64, _f64p, _int, _i64, _int, _int,
                                              _i32p, _int, _int, _int, _dbl, _dbl, _f64p, _f64p]
+        L.dito_qk_rmsnorm_rope3d_ex.argtypes = [_u16p, _i64, _f64p, _int, _i64, _int, _int,
+                                                _i32p, _int, _int, _int, _dbl, _dbl, _int, _int,
+                                                _f64p, _f64p]
         L.dito_cachedit_sums.argtypes = [_u16p, _u16p, _i64, _f64p, _f64p]
         L.dito_cachedit_decide.argtypes = [_dbl, _dbl, _dbl, _f64p]
         L.dito_cachedit_decide.restype = _int
@@ -67,7 +70,7 @@ class Oracle:
                                                   _f64p, _u8p]
         for name in ("dito_adaln_modulate", "dito_gated_residual_adaln", "dito_swiglu",
                      "dito_grid_positions", "dito_qk_rmsnorm_rope3d",
-                     "dito_cachedit_residual_diff"):
+                     "dito_qk_rmsnorm_rope3d_ex", "dito_cachedit_residual_diff"):
             getattr(L, name).restype = _int
         self.lib = L
 
@@ -156,6 +159,28 @@ class Oracle:
                                                hd, _p(pos, _i32p), pt, ph, pw, theta, eps,
                                                _p(out, _f64p), _p(work, _f64p)),
                "qk_rmsnorm_rope3d")
+        return out
+
+    def qk_rmsnorm_rope3d_ex(self, x, w, H, hd, pos, pairs, theta, eps, layout=0, norm=0,
+                             row_stride=None):
+        """As qk_rmsnorm_rope3d with the two options: layout 0 interleaved pairs,
+        1 rotate-half pairs; norm 0 per-head RMS with w [hd], 1 whole-row RMS with
+        w [H*hd]. Returns [R, H*hd] fp64."""
+        x = _c(x, np.uint16)
+        if row_stride is None:
+            row_stride = x.shape[-1]
+        R = x.size // row_stride
+        w = _c(w, np.float64).reshape(-1)
+        if w.size != (hd if norm == 0 else H * hd):
+            raise ValueError("weight size does not match the norm option")
+        pos = _c(pos, np.int32).reshape(R, 3)
+        out = np.empty((R, H * hd), dtype=np.float64)
+        work = np.empty(H * hd, dtype=np.float64)
+        pt, ph, pw = pairs
+        _check(self.lib.dito_qk_rmsnorm_rope3d_ex(_p(x, _u16p), row_stride, _p(w, _f64p), 1, R, H,
+                                                  hd, _p(pos, _i32p), pt, ph, pw, theta, eps,
+                                                  layout, norm, _p(out, _f64p), _p(work, _f64p)),
+               "qk_rmsnorm_rope3d_ex")
         return out
 
     def cachedit_sums(self, prev, cur):

@@ -261,6 +261,66 @@ int dito_qk_rmsnorm_rope3d(const uint16_t* x, int64_t row_stride, const double* 
     return 0;
 }
 
+/*
+ * The same operator with two options the pages leave open.
+ *   layout 0: rotation pairs (u_{2p}, u_{2p+1})        (interleaved)
+ *   layout 1: rotation pairs (u_p, u_{p + hd/2})        (rotate-half)
+ *   norm 0:   RMS over each head's hd values, weight w[hd]
+ *   norm 1:   RMS over the token's whole row of H*hd values, weight w[H*hd]
+ * Pair p's axis, frequency and angle are as in dito_qk_rmsnorm_rope3d.
+ * work: H*hd doubles.
+ */
+int dito_qk_rmsnorm_rope3d_ex(const uint16_t* x, int64_t row_stride, const double* w,
+                              int B, int64_t N, int H, int hd, const int32_t* pos,
+                              int pt, int ph, int pw, double theta, double eps,
+                              int layout, int norm, double* out, double* work)
+{
+    if (hd <= 0 || hd % 2 || pt <= 0 || ph <= 0 || pw <= 0 || pt + ph + pw != hd / 2)
+        return -2;
+    if (row_stride < (int64_t)H * hd || (layout != 0 && layout != 1) || (norm != 0 && norm != 1))
+        return -2;
+    int64_t rows = (int64_t)B * N;
+    int width = H * hd;
+    for (int64_t r = 0; r < rows; ++r) {
+        for (int j = 0; j < width; ++j) work[j] = dito_bf16_to_f64(x[r * row_stride + j]);
+        double inv_row = 0.0;
+        if (norm == 1) {
+            double ms = 0.0;
+            for (int j = 0; j < width; ++j) ms += work[j] * work[j];
+            ms /= (double)width;
+            inv_row = 1.0 / sqrt(ms + eps);
+        }
+        const int32_t* p3 = pos + 3 * r;
+        for (int h = 0; h < H; ++h) {
+            const double* xh = work + (int64_t)h * hd;
+            const double* wh = norm == 1 ? w + (int64_t)h * hd : w;
+            double* oh = out + r * width + (int64_t)h * hd;
+            double inv = inv_row;
+            if (norm == 0) {
+                double ms = 0.0;
+                for (int j = 0; j < hd; ++j) ms += xh[j] * xh[j];
+                ms /= (double)hd;
+                inv = 1.0 / sqrt(ms + eps);
+            }
+            for (int q = 0; q < hd / 2; ++q) {
+                int axis, i, P;
+                if (q < pt)           { axis = 0; i = q;           P = pt; }
+                else if (q < pt + ph) { axis = 1; i = q - pt;      P = ph; }
+                else                  { axis = 2; i = q - pt - ph; P = pw; }
+                double omega = pow(theta, -2.0 * (double)i / (2.0 * (double)P));
+                double phi = (double)p3[axis] * omega;
+                int a = layout == 0 ? 2 * q : q;
+                int b = layout == 0 ? 2 * q + 1 : q + hd / 2;
+                double u0 = xh[a] * inv * wh[a];
+                double u1 = xh[b] * inv * wh[b];
+                oh[a] = u0 * cos(phi) - u1 * sin(phi);
+                oh[b] = u0 * sin(phi) + u1 * cos(phi);
+            }
+        }
+    }
+    return 0;
+}
+
 /* ----------------------------------------- Cache-DiT residual check (a5) */
 
 /*

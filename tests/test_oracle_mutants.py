@@ -28,18 +28,36 @@ MUTANTS = {
                               "double a = dito_bf16_to_f64(in[m * 2 * (int64_t)F + F + j]);"),
     "swiglu_row_stride": ("double b = dito_bf16_to_f64(in[m * 2 * (int64_t)F + F + j]);",
                           "double b = dito_bf16_to_f64(in[m * (int64_t)F + F + j]);"),
-    "rms_mean_over_half_head": ("ms /= (double)hd;", "ms /= (double)(hd / 2);"),
-    "rms_eps_outside_root": ("1.0 / sqrt(ms + eps)", "1.0 / (sqrt(ms) + eps)"),
+    "rms_mean_over_half_head": ("ms /= (double)hd;\n    double inv = 1.0 / sqrt(ms + eps);",
+                                "ms /= (double)(hd / 2);\n    double inv = 1.0 / sqrt(ms + eps);"),
+    "rms_eps_outside_root": ("double inv = 1.0 / sqrt(ms + eps);",
+                             "double inv = 1.0 / (sqrt(ms) + eps);"),
+    "ex_head_eps_outside_root": ("                inv = 1.0 / sqrt(ms + eps);",
+                                 "                inv = 1.0 / (sqrt(ms) + eps);"),
     "rms_weight_index": ("double u1 = x[2 * p + 1] * inv * w[2 * p + 1];",
                          "double u1 = x[2 * p + 1] * inv * w[2 * p];"),
-    "rope_rotation_sign": ("u0 * cos(phi) - u1 * sin(phi)", "u0 * cos(phi) + u1 * sin(phi)"),
+    "rope_rotation_sign": ("out[2 * p]     = u0 * cos(phi) - u1 * sin(phi);",
+                           "out[2 * p]     = u0 * cos(phi) + u1 * sin(phi);"),
+    "ex_rotation_sign": ("oh[a] = u0 * cos(phi) - u1 * sin(phi);",
+                         "oh[a] = u0 * cos(phi) + u1 * sin(phi);"),
     "rope_rotate_half_layout": ("double u1 = x[2 * p + 1] * inv * w[2 * p + 1];",
                                 "double u1 = x[(p + hd / 2) % hd] * inv * w[(p + hd / 2) % hd];"),
     "rope_axis_h_w_swapped": ("axis = 1; i = p - pt;", "axis = 2; i = p - pt;"),
-    "rope_frequency_over_head": ("-2.0 * (double)i / (2.0 * (double)P)",
-                                 "-2.0 * (double)i / (double)hd"),
-    "rope_pos_axis_index": ("double phi = (double)p3[axis] * omega;",
-                            "double phi = (double)p3[0] * omega;"),
+    "rope_frequency_over_head": ("\n        double omega = pow(theta, -2.0 * (double)i / (2.0 * (double)P));",
+                                 "\n        double omega = pow(theta, -2.0 * (double)i / (double)hd);"),
+    "ex_frequency_over_head": ("\n                double omega = pow(theta, -2.0 * (double)i / (2.0 * (double)P));",
+                               "\n                double omega = pow(theta, -2.0 * (double)i / (double)hd);"),
+    "rope_pos_axis_index": ("\n        double phi = (double)p3[axis] * omega;",
+                            "\n        double phi = (double)p3[0] * omega;"),
+    "ex_pos_axis_index": ("\n                double phi = (double)p3[axis] * omega;",
+                          "\n                double phi = (double)p3[0] * omega;"),
+    "ex_half_partner_index": ("int b = layout == 0 ? 2 * q + 1 : q + hd / 2;",
+                              "int b = layout == 0 ? 2 * q + 1 : hd - 1 - q;"),
+    "ex_half_rotation_sign": ("oh[b] = u0 * sin(phi) + u1 * cos(phi);",
+                              "oh[b] = -u0 * sin(phi) + u1 * cos(phi);"),
+    "ex_row_norm_over_head": ("ms /= (double)width;", "ms /= (double)hd;"),
+    "ex_row_weight_per_head": ("const double* wh = norm == 1 ? w + (int64_t)h * hd : w;",
+                               "const double* wh = w;"),
     "grid_h_w_confused": ("pos[3 * n + 1] = (int32_t)((g / Wg) % Hg);",
                           "pos[3 * n + 1] = (int32_t)((g / Hg) % Wg);"),
     "cache_denominator_uses_cur": ("s_den += fabs(p);", "s_den += fabs(c);"),

@@ -112,3 +112,95 @@ def test_row_stride_reads_a_fused_buffer(orc):
     flat = np.concatenate([qkv.reshape(-1)[D:], np.zeros(D, np.uint16)])
     via_stride = orc.qk_rmsnorm_rope3d(flat, w, H, hd, pos, pairs, 1e4, 1e-6, row_stride=3 * D)
     assert np.array_equal(dense, via_stride)
+
+
+# ------------------------------------------------ layout and norm options
+
+
+def test_options_golden(orc):
+    g = load_golden("qk_rope.json")
+    hd, pairs, theta = g["hd"], tuple(g["pairs"]), g["theta"]
+    for case in g["rotate_half_cases"]:
+        x = orc.f64_to_bf16(np.array(case["x"], dtype=np.float64)).reshape(1, hd)
+        out = orc.qk_rmsnorm_rope3d_ex(x, np.array(case["w"], dtype=np.float64), 1, hd,
+                                       np.array([case["pos"]], np.int32), pairs, theta,
+                                       case["eps"], layout=1)
+        want = np.array([closed_form(e) for e in case["out"]])
+        assert np.allclose(out.reshape(-1), want, rtol=0, atol=1e-14), case["name"]
+    for case in g["row_norm_cases"]:
+        H = case["heads"]
+        x = orc.f64_to_bf16(np.array(case["x"], dtype=np.float64)).reshape(1, H * hd)
+        out = orc.qk_rmsnorm_rope3d_ex(x, np.array(case["w"], dtype=np.float64), H, hd,
+                                       np.array([case["pos"]], np.int32), pairs, theta,
+                                       case["eps"], norm=1)
+        want = np.array([closed_form(e) for e in case["out"]])
+        assert np.allclose(out.reshape(-1), want, rtol=0, atol=1e-14), case["name"]
+
+
+def test_default_options_are_the_pinned_operator(orc):
+    x, w, H, hd, pairs = _setup(orc, seed=8)
+    pos = np.random.default_rng(9).integers(0, 60, (x.shape[0], 3)).astype(np.int32)
+    assert np.array_equal(orc.qk_rmsnorm_rope3d_ex(x, w, H, hd, pos, pairs, 1e4, 1e-6),
+                          orc.qk_rmsnorm_rope3d(x, w, H, hd, pos, pairs, 1e4, 1e-6))
+
+
+def test_rotate_half_is_interleaved_after_a_fixed_permutation(orc):
+    """Moving element p to slot 2p and element p + hd/2 to slot 2p + 1 turns
+    rotate-half pairs into interleaved pairs of the same index, so the
+    rotate-half operator equals the (pinned) interleaved one conjugated by
+    that permutation."""
+    x, w, H, hd, pairs = _setup(orc, seed=10)
+    R = x.shape[0]
+    pos = np.random.default_rng(11).integers(0, 60, (R, 3)).astype(np.int32)
+    perm = np.empty(hd, dtype=np.int64)           # interleaved slot -> rotate-half element
+    perm[0::2] = np.arange(hd // 2)
+    perm[1::2] = np.arange(hd // 2) + hd // 2
+    xi = x.reshape(R, H, hd)[:, :, perm].reshape(R, H * hd)
+    out_i = orc.qk_rmsnorm_rope3d(xi, w[perm], H, hd, pos, pairs, 1e4, 1e-6).reshape(R, H, hd)
+    out_h = orc.qk_rmsnorm_rope3d_ex(x, w, H, hd, pos, pairs, 1e4, 1e-6, layout=1).reshape(R, H, hd)
+    back = np.empty_like(out_i)
+    back[:, :, perm] = out_i
+    assert np.allclose(out_h, back, rtol=0, atol=1e-14)
+
+
+def test_row_norm_at_position_zero_is_library_rms_norm(orc):
+    x, _, H, hd, pairs = _setup(orc, seed=12)
+    w = 1.0 + 0.02 * np.random.default_rng(13).standard_normal(H * hd)
+    out = orc.qk_rmsnorm_rope3d_ex(x, w, H, hd, np.zeros((x.shape[0], 3), np.int32), pairs, 1e4,
+                                   1e-6, norm=1)
+    v = torch.from_numpy(orc.bf16_to_f64(x))
+    ref = torch.nn.functional.rms_norm(v, (H * hd,), weight=torch.from_numpy(w), eps=1e-6)
+    assert np.allclose(out, ref.numpy(), rtol=0, atol=1e-13)
+
+
+def test_row_norm_with_one_head_is_the_head_norm(orc):
+    x, w, _, hd, pairs = _setup(orc, H=1, seed=14)
+    pos = np.random.default_rng(15).integers(0, 60, (x.shape[0], 3)).astype(np.int32)
+    for layout in (0, 1):
+        a = orc.qk_rmsnorm_rope3d_ex(x, w, 1, hd, pos, pairs, 1e4, 1e-6, layout=layout, norm=0)
+        b = orc.qk_rmsnorm_rope3d_ex(x, w, 1, hd, pos, pairs, 1e4, 1e-6, layout=layout, norm=1)
+        assert np.array_equal(a, b)
+
+
+def test_options_keep_norms_and_relative_positions(orc):
+    x, w, H, hd, pairs = _setup(orc, R=2, seed=16)
+    wrow = np.tile(w, H)
+    q, k = x[0:1], x[1:2]
+    p, pp = np.array([[3, 5, 7]], np.int32), np.array([[11, 2, 9]], np.int32)
+    for layout, norm in ((1, 0), (0, 1), (1, 1)):
+        ww = wrow if norm else w
+        f = lambda t, ps: orc.qk_rmsnorm_rope3d_ex(t, ww, H, hd, ps, pairs, 1e4, 1e-6,
+                                                   layout=layout, norm=norm).reshape(H, hd)
+        base = f(q, np.zeros((1, 3), np.int32))
+        rot = f(q, p)
+        half = hd // 2
+        if layout == 0:
+            nb, nr = np.hypot(base[:, 0::2], base[:, 1::2]), np.hypot(rot[:, 0::2], rot[:, 1::2])
+        else:
+            nb, nr = np.hypot(base[:, :half], base[:, half:]), np.hypot(rot[:, :half], rot[:, half:])
+        assert np.allclose(nb, nr, rtol=1e-13)
+        ref = (f(q, p) * f(k, pp)).sum(axis=1)
+        for axis in range(3):
+            d = np.zeros((1, 3), np.int32)
+            d[0, axis] = 13
+            assert np.allclose((f(q, p + d) * f(k, pp + d)).sum(axis=1), ref, rtol=1e-12, atol=1e-12)
