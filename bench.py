@@ -254,6 +254,41 @@ def time_device(chain, steps, warmup, world):
     return total_ms, per_op
 
 
+QK_OPTIONS = {"rope_half+norm_head": (1, 0), "interleaved+norm_row": (0, 1),
+              "rope_half+norm_row": (1, 1)}
+
+
+def time_qk_options(chain, steps, warmup, world):
+    """Device ms per launch of the QK op with its non-default options (rotate-
+    half pairs, whole-row norm) on the chain's q and k, outside the chain."""
+    import torch
+    import dit_block_pass_b200 as dbp
+    from dit_block_pass_b200 import workloads as W
+    c, wl, D = chain, chain.wl, chain.wl.D
+    rq, rk = W.row_norm_weights(wl, device=c.dev)
+    grid = None if c.pos is not None else (wl.T, wl.Hg, wl.Wg)
+    stream = torch.cuda.current_stream()
+    out = {}
+    for name, (layout, norm) in QK_OPTIONS.items():
+        wq, wk = (c.wq, c.wk) if norm == dbp.NORM_HEAD else (rq, rk)
+
+        def op():
+            dbp.qk_rmsnorm_rope3d(c.qkv[:, :, :D], c.qkv[:, :, D:2 * D], wq, wk, wl.H, wl.pairs,
+                                  grid=grid, pos=c.pos, theta=wl.theta, eps=wl.eps,
+                                  rope_layout=layout, norm_width=norm)
+        for _ in range(warmup):
+            op()
+        barrier_sync(world)
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(2 * steps)]
+        for s in range(steps):
+            ev[2 * s].record(stream)
+            op()
+            ev[2 * s + 1].record(stream)
+        barrier_sync(world)
+        out[name] = sum(ev[2 * s].elapsed_time(ev[2 * s + 1]) for s in range(steps)) / steps
+    return out
+
+
 def time_e2e(chain, steps, warmup, world):
     """The same chain through the public API with inputs on the host: every
     step copies its inputs host->device from pinned memory, runs the chain and
@@ -451,6 +486,7 @@ def main():
         sampler.__enter__()
     try:
         total_ms, per_op = time_device(chain, args.steps, args.warmup, world)
+        qk_opt = time_qk_options(chain, args.steps, args.warmup, world)
     finally:
         if sampler:
             sampler.__exit__(None, None, None)
@@ -467,6 +503,12 @@ def main():
         ops[name] = {"ms": round(ms, 4), "GB/s": round(gbs, 1),
                      "frac_of_peak": round(gbs / peak, 4),
                      "tokens_per_s": round(tokens / (ms / 1000.0), 1)}
+    qk_options = {}
+    for name, ms in qk_opt.items():
+        ms = max_over_ranks(ms, world)
+        gbs = nbytes["qk_rmsnorm_rope3d"] / (ms / 1000.0) / 1e9
+        qk_options[name] = {"ms": round(ms, 4), "GB/s": round(gbs, 1),
+                            "frac_of_peak": round(gbs / peak, 4)}
     dom_ms = per_op[OPS.index(DOMINANT)]
     achieved = nbytes[DOMINANT] / (dom_ms / 1000.0) / 1e9
     tr = NCU_TRAFFIC.get(DOMINANT)
@@ -505,7 +547,7 @@ def main():
                        "tokens_per_step_per_gpu": tokens,
                        "l2": "every input is larger than L2 (126 MB); no flush",
                        "parallelism": f"{world} independent clip(s), one per GPU"},
-            "ops": ops, "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+            "ops": ops, "qk_options": qk_options, "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": chain.launches_per_step() * args.steps, "clocks": clocks,
         }
         print(json.dumps(line), flush=True)

@@ -25,10 +25,13 @@ __all__ = [
     "DitError", "library", "library_path", "adaln_modulate", "gated_residual_adaln", "swiglu",
     "qk_rmsnorm_rope3d", "cachedit_workspace_bytes", "cachedit_residual_diff",
     "cachedit_residual_sums", "cachedit_decide", "cachedit_residual_diff_noalloc",
-    "launch_counts", "F32", "BF16",
+    "launch_counts", "F32", "BF16", "ROPE_INTERLEAVED", "ROPE_HALF", "NORM_HEAD", "NORM_ROW",
 ]
 
 F32, BF16 = 0, 1
+# options of qk_rmsnorm_rope3d
+ROPE_INTERLEAVED, ROPE_HALF = 0, 1     # rotation pairs (2p, 2p+1) or (p, p + hd/2)
+NORM_HEAD, NORM_ROW = 0, 1             # RMS over each head or over the whole H*hd row
 _PKG = os.path.dirname(os.path.abspath(__file__))
 _LIB_PATH = os.path.join(_PKG, "libdit_block.so")
 _lib = None
@@ -37,6 +40,7 @@ _lock = threading.Lock()
 # kernels launched per call of each entry point (for launch accounting)
 launch_counts = {
     "adaln_modulate": 1, "gated_residual_adaln": 1, "swiglu": 1, "qk_rmsnorm_rope3d": 1,
+    "qk_rmsnorm_rope3d_ex": 1,
     "cachedit_residual_diff": 2, "cachedit_residual_sums": 2, "cachedit_decide": 1,
     "cachedit_residual_diff_noalloc": 2,
 }
@@ -75,6 +79,9 @@ def library() -> ctypes.CDLL:
             L.dit_qk_rmsnorm_rope3d.argtypes = [vp, vp, i64, vp, vp, i32, i32, i64, i32, i32,
                                                 i32, i32, i32, vp, i64, i32, i32, i32, dbl, dbl,
                                                 vp]
+            L.dit_qk_rmsnorm_rope3d_ex.argtypes = [vp, vp, i64, vp, vp, i32, i32, i64, i32,
+                                                   i32, i32, i32, i32, vp, i64, i32, i32, i32,
+                                                   dbl, dbl, i32, i32, vp]
             L.cachedit_workspace_bytes.restype = sz
             L.cachedit_workspace_bytes.argtypes = [i32, i64, i32]
             L.cachedit_residual_diff.argtypes = [vp, vp, i32, i64, i32, dbl, vp, vp, vp, sz, vp]
@@ -83,7 +90,8 @@ def library() -> ctypes.CDLL:
             L.cachedit_residual_diff_noalloc.argtypes = [vp, vp, i32, i64, i32, dbl, vp, vp, vp]
             L.cachedit_residual_diff_noalloc.restype = i32
             for name in ("dit_adaln_modulate", "dit_gated_residual_adaln", "dit_swiglu",
-                         "dit_qk_rmsnorm_rope3d", "cachedit_residual_diff",
+                         "dit_qk_rmsnorm_rope3d", "dit_qk_rmsnorm_rope3d_ex",
+                         "cachedit_residual_diff",
                          "cachedit_residual_sums", "cachedit_decide"):
                 getattr(L, name).restype = i32
             _lib = L
@@ -219,11 +227,15 @@ def qk_rmsnorm_rope3d(q: Optional[torch.Tensor], k: Optional[torch.Tensor],
                       w_q: Optional[torch.Tensor], w_k: Optional[torch.Tensor], heads: int,
                       pairs: Sequence[int], grid: Optional[Sequence[int]] = None,
                       pos: Optional[torch.Tensor] = None, pos_offset: int = 0,
-                      theta: float = 10000.0, eps: float = 1e-6) -> None:
+                      theta: float = 10000.0, eps: float = 1e-6,
+                      rope_layout: int = ROPE_INTERLEAVED, norm_width: int = NORM_HEAD) -> None:
     """In place on q and k ([B, N, H*hd] views, e.g. slices of a fused qkv
-    buffer): per-head RMSNorm with weight w, then 3D RoPE with pair split
+    buffer): RMSNorm with weight w, then 3D RoPE with pair split
     ``pairs`` = (t, h, w).  Positions come from ``grid`` = (T, Hg, Wg) (token
-    n at global index pos_offset + n) or from ``pos`` [B*N, 3] int32."""
+    n at global index pos_offset + n) or from ``pos`` [B*N, 3] int32.
+    ``norm_width`` NORM_HEAD normalises each head (w: [hd]), NORM_ROW the
+    token's whole row (w: [H*hd]); ``rope_layout`` ROPE_INTERLEAVED rotates
+    pairs (2p, 2p+1), ROPE_HALF pairs (p, p + hd/2)."""
     ref = q if q is not None else k
     if ref is None:
         raise ValueError("q and k cannot both be None")
@@ -241,8 +253,9 @@ def qk_rmsnorm_rope3d(q: Optional[torch.Tensor], k: Optional[torch.Tensor],
     w_dt = None
     for nm, t, w in (("w_q", q, w_q), ("w_k", k, w_k)):
         if t is not None:
-            if w is None or w.numel() != hd or not w.is_contiguous() or not w.is_cuda:
-                raise ValueError(f"{nm} must be a contiguous CUDA [{hd}] tensor")
+            wn = hd if norm_width == NORM_HEAD else width
+            if w is None or w.numel() != wn or not w.is_contiguous() or not w.is_cuda:
+                raise ValueError(f"{nm} must be a contiguous CUDA [{wn}] tensor")
             d = _mod_dtype(w)
             if w_dt is not None and d != w_dt:
                 raise ValueError("w_q and w_k must share a dtype")
@@ -257,9 +270,9 @@ def qk_rmsnorm_rope3d(q: Optional[torch.Tensor], k: Optional[torch.Tensor],
             raise ValueError("give grid=(T, Hg, Wg) or pos")
         T, Hg, Wg = grid
     pt, ph, pw = pairs
-    _call("dit_qk_rmsnorm_rope3d", _ptr(q), _ptr(k), rs, _ptr(w_q), _ptr(w_k), w_dt, B, N, heads,
-          hd, T, Hg, Wg, _ptr(pos), int(pos_offset), pt, ph, pw, float(theta), float(eps),
-          _stream(ref))
+    _call("dit_qk_rmsnorm_rope3d_ex", _ptr(q), _ptr(k), rs, _ptr(w_q), _ptr(w_k), w_dt, B, N,
+          heads, hd, T, Hg, Wg, _ptr(pos), int(pos_offset), pt, ph, pw, float(theta), float(eps),
+          int(rope_layout), int(norm_width), _stream(ref))
 
 
 def cachedit_workspace_bytes(B: int, N: int, D: int) -> int:

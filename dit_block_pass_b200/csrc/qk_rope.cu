@@ -64,37 +64,139 @@ __device__ __forceinline__ void cp_async16(void* smem_dst, const void* gsrc) {
 // first tensor's row goes to registers and the second's to the warp's
 // shared-memory stage with cp.async, both issued before any arithmetic;
 // lane-vector j of a row is its vector j * 32 + lane.
-template <int HD, int NVL>
-__device__ __forceinline__ void qk_row(const uint4 (&v)[NVL], uint4* row, int nvr, int lane,
-                                       const float (&A)[4], const float (&Bn)[4],
-                                       const float (&C)[4], const float (&Dd)[4], float eps,
-                                       float inv_hd) {
+// Eight weights of elements e .. e+7 (fp32 or bf16; 16-byte aligned rows).
+__device__ __forceinline__ void w8_at(const void* w, int dtype, int e, float (&f)[8]) {
+    if (dtype == DIT_F32) {
+        const float4* q = reinterpret_cast<const float4*>(static_cast<const float*>(w) + e);
+        const float4 a = __ldg(q), b = __ldg(q + 1);
+        f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w;
+        f[4] = b.x; f[5] = b.y; f[6] = b.z; f[7] = b.w;
+    } else {
+        unpack8(__ldg(reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(w) + e)), f);
+    }
+}
+
+// Normalise and rotate one tensor row held as NVL lane-vectors v (vector
+// j * 32 + lane of the row), and store it.
+//   LAYOUT 0: pairs (2p, 2p+1) inside a lane's vector: lane pairs 4*sub + k.
+//   LAYOUT 1: pairs (p, p + hd/2): a lane's 8 elements pair with the same
+//             slots of lane ^ (hd/16) (one shuffle of the packed vector);
+//             lane pairs 8*(sub mod hd/16) + i.
+//   NORMW 0:  RMS over each head (a shuffle over its hd/8 lanes); the weight
+//             is folded into per-lane rotation coefficients.
+//   NORMW 1:  RMS over the whole row (a warp reduction); the weight has one
+//             entry per element of the row.
+template <int HD, int NVL, int LAYOUT, int NORMW>
+__device__ __forceinline__ void qk_tensor(uint4 (&v)[NVL], uint4* row, int nvr, int lane,
+                                          const void* w, int w_dtype, const float* cs,
+                                          const float* sn, float eps) {
     constexpr int LPH = HD / 8;
+    constexpr int HALF = LPH / 2;           // partner lane distance for rotate-half
+    const int sub = lane % LPH;
+    const bool first = (sub & HALF) == 0;   // rotate-half: lane holds the first half
+    float inv_row = 0.0f;
+    if (NORMW == 1) {
+        float ss = 0.0f;
+#pragma unroll
+        for (int j = 0; j < NVL; ++j) {
+            float f[8];
+            unpack8(v[j], f);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) ss = __fmaf_rn(f[i], f[i], ss);
+        }
+        ss = warp_sum(ss);
+        inv_row = rsqrtf(__fmaf_rn(ss, 1.0f / static_cast<float>(nvr * 8), eps));
+        // unpack again below rather than keep every unpacked float alive
+        // across the reduction (the packed row needs half the registers)
+#pragma unroll
+        for (int j = 0; j < NVL; ++j)
+            asm volatile("" : "+r"(v[j].x), "+r"(v[j].y), "+r"(v[j].z), "+r"(v[j].w));
+    }
+    // per-lane coefficients with the weight folded in (per-head norm)
+    float A[8], Bc[8], C[4], Dd[4];
+    if (NORMW == 0) {
+        if (LAYOUT == 0) {
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const float wa = w_at(w, w_dtype, 8 * sub + 2 * k);
+                const float wb = w_at(w, w_dtype, 8 * sub + 2 * k + 1);
+                A[k] = wa * cs[k]; Bc[k] = -(wb * sn[k]); C[k] = wa * sn[k]; Dd[k] = wb * cs[k];
+            }
+        } else {
+            // out_e = inv * (f_e w_e cos + sign * f_partner w_partner sin)
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const float wo = w_at(w, w_dtype, 8 * sub + i);
+                const float wp = w_at(w, w_dtype, 8 * (sub ^ HALF) + i);
+                A[i] = wo * cs[i];
+                Bc[i] = (first ? -wp : wp) * sn[i];
+            }
+        }
+    }
 #pragma unroll
     for (int j = 0; j < NVL; ++j) {
         const int idx = j * 32 + lane;
         float f[8];
         unpack8(v[j], f);
-        float ss = 0.0f;
+        float inv = inv_row;
+        if (NORMW == 0) {
+            float ss = 0.0f;
 #pragma unroll
-        for (int i = 0; i < 8; ++i) ss = __fmaf_rn(f[i], f[i], ss);
+            for (int i = 0; i < 8; ++i) ss = __fmaf_rn(f[i], f[i], ss);
 #pragma unroll
-        for (int o = LPH / 2; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-        const float inv = rsqrtf(__fmaf_rn(ss, inv_hd, eps));
+            for (int o = LPH / 2; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+            inv = rsqrtf(__fmaf_rn(ss, 1.0f / static_cast<float>(HD), eps));
+        }
         float o8[8];
+        if (LAYOUT == 0) {
+            if (NORMW == 0) {
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            o8[2 * k] = inv * __fmaf_rn(f[2 * k], A[k], f[2 * k + 1] * Bn[k]);
-            o8[2 * k + 1] = inv * __fmaf_rn(f[2 * k], C[k], f[2 * k + 1] * Dd[k]);
+                for (int k = 0; k < 4; ++k) {
+                    o8[2 * k] = inv * __fmaf_rn(f[2 * k], A[k], f[2 * k + 1] * Bc[k]);
+                    o8[2 * k + 1] = inv * __fmaf_rn(f[2 * k], C[k], f[2 * k + 1] * Dd[k]);
+                }
+            } else {
+                float wv[8];
+                w8_at(w, w_dtype, (idx < nvr ? idx : 0) * 8, wv);
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const float u0 = f[2 * k] * inv * wv[2 * k];
+                    const float u1 = f[2 * k + 1] * inv * wv[2 * k + 1];
+                    o8[2 * k] = __fmaf_rn(u0, cs[k], -u1 * sn[k]);
+                    o8[2 * k + 1] = __fmaf_rn(u0, sn[k], u1 * cs[k]);
+                }
+            }
+        } else if (NORMW == 0) {
+            uint4 pv;
+            pv.x = __shfl_xor_sync(0xffffffffu, v[j].x, HALF);
+            pv.y = __shfl_xor_sync(0xffffffffu, v[j].y, HALF);
+            pv.z = __shfl_xor_sync(0xffffffffu, v[j].z, HALF);
+            pv.w = __shfl_xor_sync(0xffffffffu, v[j].w, HALF);
+            float fp[8];
+            unpack8(pv, fp);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) o8[i] = inv * __fmaf_rn(f[i], A[i], fp[i] * Bc[i]);
+        } else {
+            // weight each element on its own lane, then swap the weighted
+            // values with the partner lane
+            float wo[8];
+            w8_at(w, w_dtype, (idx < nvr ? idx : 0) * 8, wo);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const float u = f[i] * inv * wo[i];
+                const float up = __shfl_xor_sync(0xffffffffu, u, HALF);
+                o8[i] = __fmaf_rn(u, cs[i], (first ? -up : up) * sn[i]);
+            }
         }
         if (idx < nvr) st_stream(row + idx, pack8(o8));
     }
 }
 
-template <int HD, int NVL>
+template <int HD, int NVL, int LAYOUT, int NORMW>
 __global__ void __launch_bounds__(kThreads, (NVL <= 20 ? 2 : 1))
 qk_rmsnorm_rope3d_kernel(QKParams p) {
     constexpr int LPH = HD / 8;             // lanes per head
+    constexpr int NP = LAYOUT == 0 ? 4 : 8; // rotation pairs per lane
     extern __shared__ uint4 qk_stage[];
     __shared__ double s_omega[HD / 2];      // frequency of each rotation pair
     const int lane = threadIdx.x & 31;
@@ -134,7 +236,7 @@ qk_rmsnorm_rope3d_kernel(QKParams p) {
     __syncthreads();
     if (!live) return;
 
-    // token position and this lane's 4 rotation angles (pairs 4*sub + k)
+    // token position and this lane's rotation angles
     int pos3[3];
     if (p.pos) {
         pos3[0] = p.pos[3 * tok + 0];
@@ -153,49 +255,33 @@ qk_rmsnorm_rope3d_kernel(QKParams p) {
     }
     const double kTwoPi = 6.283185307179586;
     const double kInvTwoPi = 0.15915494309189535;
-    float cs[4], sn[4];
+    float cs[NP], sn[NP];
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-        const int pr = 4 * sub + k;
+    for (int k = 0; k < NP; ++k) {
+        const int pr = LAYOUT == 0 ? 4 * sub + k : 8 * (sub % (LPH / 2)) + k;
         const int pa = pr < p.pt ? pos3[0] : (pr < p.pt + p.ph ? pos3[1] : pos3[2]);
         const double phi = static_cast<double>(pa) * s_omega[pr];
         const double kk = rint(phi * kInvTwoPi);
         sincosf(static_cast<float>(fma(-kk, kTwoPi, phi)), &sn[k], &cs[k]);
     }
-    // rotation with the weight folded in: (u0, u1) = inv * (f0 w0, f1 w1)
-    //   out0 = inv * (f0 w0 cos - f1 w1 sin), out1 = inv * (f0 w0 sin + f1 w1 cos)
-    const float inv_hd = 1.0f / static_cast<float>(HD);
-    float A[4], Bn[4], C[4], Dd[4];
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-        const float wa = w_at(p.w0, p.w_dtype, 8 * sub + 2 * k);
-        const float wb = w_at(p.w0, p.w_dtype, 8 * sub + 2 * k + 1);
-        A[k] = wa * cs[k]; Bn[k] = -(wb * sn[k]); C[k] = wa * sn[k]; Dd[k] = wb * cs[k];
-    }
-    qk_row<HD, NVL>(v, row0, p.nvr, lane, A, Bn, C, Dd, p.eps, inv_hd);
+    qk_tensor<HD, NVL, LAYOUT, NORMW>(v, row0, p.nvr, lane, p.w0, p.w_dtype, cs, sn, p.eps);
     if (row1) {
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            const float wa = w_at(p.w1, p.w_dtype, 8 * sub + 2 * k);
-            const float wb = w_at(p.w1, p.w_dtype, 8 * sub + 2 * k + 1);
-            A[k] = wa * cs[k]; Bn[k] = -(wb * sn[k]); C[k] = wa * sn[k]; Dd[k] = wb * cs[k];
-        }
         asm volatile("cp.async.wait_group 0;" ::: "memory");
 #pragma unroll
         for (int j = 0; j < NVL; ++j)
             v[j] = (j * 32 + lane < p.nvr) ? stage[j * 32] : make_uint4(0, 0, 0, 0);
-        qk_row<HD, NVL>(v, row1, p.nvr, lane, A, Bn, C, Dd, p.eps, inv_hd);
+        qk_tensor<HD, NVL, LAYOUT, NORMW>(v, row1, p.nvr, lane, p.w1, p.w_dtype, cs, sn, p.eps);
     }
 }
 
 using QKKernel = void (*)(QKParams);
 
-template <int HD>
+template <int HD, int LAYOUT, int NORMW>
 QKKernel pick_nvl(int nvl, int* nvl_out) {
-#define DIT_NVL_CASE(V)                                   \
-    if (nvl <= V) {                                       \
-        *nvl_out = V;                                     \
-        return qk_rmsnorm_rope3d_kernel<HD, V>;           \
+#define DIT_NVL_CASE(V)                                               \
+    if (nvl <= V) {                                                   \
+        *nvl_out = V;                                                 \
+        return qk_rmsnorm_rope3d_kernel<HD, V, LAYOUT, NORMW>;        \
     }
     DIT_NVL_CASE(1) DIT_NVL_CASE(2) DIT_NVL_CASE(3) DIT_NVL_CASE(4) DIT_NVL_CASE(6)
     DIT_NVL_CASE(8) DIT_NVL_CASE(10) DIT_NVL_CASE(12) DIT_NVL_CASE(16) DIT_NVL_CASE(20)
@@ -204,14 +290,27 @@ QKKernel pick_nvl(int nvl, int* nvl_out) {
     return nullptr;
 }
 
-QKKernel pick(int hd, int nvl, int* nvl_out) {
+template <int LAYOUT, int NORMW>
+QKKernel pick_hd(int hd, int nvl, int* nvl_out) {
     switch (hd) {
-        case 32: return pick_nvl<32>(nvl, nvl_out);
-        case 64: return pick_nvl<64>(nvl, nvl_out);
-        case 128: return pick_nvl<128>(nvl, nvl_out);
-        case 256: return pick_nvl<256>(nvl, nvl_out);
+        case 32: return pick_nvl<32, LAYOUT, NORMW>(nvl, nvl_out);
+        case 64: return pick_nvl<64, LAYOUT, NORMW>(nvl, nvl_out);
+        case 128: return pick_nvl<128, LAYOUT, NORMW>(nvl, nvl_out);
+        case 256: return pick_nvl<256, LAYOUT, NORMW>(nvl, nvl_out);
         default: return nullptr;
     }
+}
+
+QKKernel pick(int hd, int layout, int norm, int nvl, int* nvl_out) {
+    if (layout == DIT_ROPE_INTERLEAVED && norm == DIT_NORM_HEAD)
+        return pick_hd<DIT_ROPE_INTERLEAVED, DIT_NORM_HEAD>(hd, nvl, nvl_out);
+    if (layout == DIT_ROPE_HALF && norm == DIT_NORM_HEAD)
+        return pick_hd<DIT_ROPE_HALF, DIT_NORM_HEAD>(hd, nvl, nvl_out);
+    if (layout == DIT_ROPE_INTERLEAVED && norm == DIT_NORM_ROW)
+        return pick_hd<DIT_ROPE_INTERLEAVED, DIT_NORM_ROW>(hd, nvl, nvl_out);
+    if (layout == DIT_ROPE_HALF && norm == DIT_NORM_ROW)
+        return pick_hd<DIT_ROPE_HALF, DIT_NORM_ROW>(hd, nvl, nvl_out);
+    return nullptr;
 }
 
 // Rows i of q ([q + i*rs, q + i*rs + w), elements) and rows j of k overlap
@@ -244,16 +343,18 @@ int check_w(const void* p, int dtype) {
 }  // namespace
 }  // namespace dit
 
-extern "C" int dit_qk_rmsnorm_rope3d(uint16_t* q, uint16_t* k, int64_t row_stride,
-                                     const void* w_q, const void* w_k, int w_dtype, int B,
-                                     int64_t N, int H, int hd, int T, int Hg, int Wg,
-                                     const int32_t* pos, int64_t pos_offset, int pairs_t,
-                                     int pairs_h, int pairs_w, double theta, double eps,
-                                     void* stream) {
+extern "C" int dit_qk_rmsnorm_rope3d_ex(uint16_t* q, uint16_t* k, int64_t row_stride,
+                                        const void* w_q, const void* w_k, int w_dtype, int B,
+                                        int64_t N, int H, int hd, int T, int Hg, int Wg,
+                                        const int32_t* pos, int64_t pos_offset, int pairs_t,
+                                        int pairs_h, int pairs_w, double theta, double eps,
+                                        int rope_layout, int norm_width, void* stream) {
     using namespace dit;
     if (w_dtype != DIT_F32 && w_dtype != DIT_BF16) return DIT_ERR_DTYPE;
     if (B < 0 || N < 0 || H < 1) return DIT_ERR_SHAPE;
     if (hd != 32 && hd != 64 && hd != 128 && hd != 256) return DIT_ERR_SHAPE;
+    if (rope_layout != DIT_ROPE_INTERLEAVED && rope_layout != DIT_ROPE_HALF) return DIT_ERR_VALUE;
+    if (norm_width != DIT_NORM_HEAD && norm_width != DIT_NORM_ROW) return DIT_ERR_VALUE;
     if (pairs_t < 1 || pairs_h < 1 || pairs_w < 1 || pairs_t + pairs_h + pairs_w != hd / 2)
         return DIT_ERR_SHAPE;
     const int64_t width = static_cast<int64_t>(H) * hd;
@@ -274,6 +375,9 @@ extern "C" int dit_qk_rmsnorm_rope3d(uint16_t* q, uint16_t* k, int64_t row_strid
     int st;
     if (q && (st = check_w(w_q, w_dtype))) return st;
     if (k && (st = check_w(w_k, w_dtype))) return st;
+    // whole-row weights are read 16 bytes at a time
+    if (norm_width == DIT_NORM_ROW && ((q && !aligned16(w_q)) || (k && !aligned16(w_k))))
+        return DIT_ERR_ALIGN;
     if ((q && !aligned16(q)) || (k && !aligned16(k))) return DIT_ERR_ALIGN;
     if (q && k && rows_overlap(q, k, rows, row_stride, width)) return DIT_ERR_OVERLAP;
 
@@ -298,7 +402,7 @@ extern "C" int dit_qk_rmsnorm_rope3d(uint16_t* q, uint16_t* k, int64_t row_strid
     p.eps = static_cast<float>(eps);
 
     int nvl = 0;
-    QKKernel kernel = pick(hd, (p.nvr + 31) / 32, &nvl);
+    QKKernel kernel = pick(hd, rope_layout, norm_width, (p.nvr + 31) / 32, &nvl);
     if (!kernel) return DIT_ERR_SHAPE;
     const size_t smem = p.t1 ? static_cast<size_t>(kWarps) * nvl * 32 * sizeof(uint4) : 0;
     // opt in whenever dynamic shared memory is used: with the static
@@ -311,4 +415,15 @@ extern "C" int dit_qk_rmsnorm_rope3d(uint16_t* q, uint16_t* k, int64_t row_strid
     if (ctas > 0x7FFFFFFF) return DIT_ERR_SHAPE;
     kernel<<<static_cast<unsigned>(ctas), kThreads, smem, as_stream(stream)>>>(p);
     return launch_status();
+}
+
+extern "C" int dit_qk_rmsnorm_rope3d(uint16_t* q, uint16_t* k, int64_t row_stride,
+                                     const void* w_q, const void* w_k, int w_dtype, int B,
+                                     int64_t N, int H, int hd, int T, int Hg, int Wg,
+                                     const int32_t* pos, int64_t pos_offset, int pairs_t,
+                                     int pairs_h, int pairs_w, double theta, double eps,
+                                     void* stream) {
+    return dit_qk_rmsnorm_rope3d_ex(q, k, row_stride, w_q, w_k, w_dtype, B, N, H, hd, T, Hg, Wg,
+                                    pos, pos_offset, pairs_t, pairs_h, pairs_w, theta, eps,
+                                    DIT_ROPE_INTERLEAVED, DIT_NORM_HEAD, stream);
 }

@@ -227,6 +227,14 @@ def norm_weights(wl: Workload, device="cpu"):
     return wq.reshape(wl.hd), wk.reshape(wl.hd)
 
 
+def row_norm_weights(wl: Workload, device="cpu"):
+    """Whole-row RMSNorm weights w_q, w_k: [H*hd] fp32 ~ 1 + N(0, 0.02)."""
+    D = wl.H * wl.hd
+    wq = normal(wl.seed, S_WQ, 1, D, sigma=0.02, mean=1.0, dtype=torch.float32, device=device)
+    wk = normal(wl.seed, S_WK, 1, D, sigma=0.02, mean=1.0, dtype=torch.float32, device=device)
+    return wq.reshape(D), wk.reshape(D)
+
+
 def token_rows(wl: Workload, stream: int, width: int, device="cpu", row_ids=None) -> torch.Tensor:
     """[B*N, width] bf16 ~N(0,1) token-major rows (all rows, or row_ids)."""
     return normal(wl.seed, stream, wl.M, width, device=device, row_ids=row_ids)

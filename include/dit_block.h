@@ -141,7 +141,7 @@ int dit_swiglu(const uint16_t* in, uint16_t* out, int64_t M, int F, void* stream
  *             fused qkv buffer).
  * w_q, w_k    [hd] weights of dtype w_dtype (needed for each non-NULL tensor).
  * hd          one of 32, 64, 128, 256; pairs_t + pairs_h + pairs_w == hd/2,
- *             each >= 1.  H >= 1.
+ *             each >= 1.  H >= 1, H*hd <= DIT_MAX_D.
  * pos         device [B*N, 3] int32 (t, h, w) per token, or NULL: then token
  *             n of every sample sits at global grid index g = pos_offset + n
  *             of a row-major (T, Hg, Wg) grid, t = g/(Hg*Wg), h = (g/Wg)%Hg,
@@ -155,6 +155,31 @@ int dit_qk_rmsnorm_rope3d(uint16_t* q, uint16_t* k, int64_t row_stride,
                           int T, int Hg, int Wg, const int32_t* pos, int64_t pos_offset,
                           int pairs_t, int pairs_h, int pairs_w,
                           double theta, double eps, void* stream);
+
+/* Options of dit_qk_rmsnorm_rope3d_ex. */
+enum { DIT_ROPE_INTERLEAVED = 0, DIT_ROPE_HALF = 1 };
+enum { DIT_NORM_HEAD = 0, DIT_NORM_ROW = 1 };
+
+/*
+ * dit_qk_rmsnorm_rope3d with the two choices the pages leave open (the
+ * "QK RMSNorm com 3D RoPE" the report names does not say which it uses):
+ *   rope_layout  DIT_ROPE_INTERLEAVED: rotation pairs (u_{2p}, u_{2p+1});
+ *                DIT_ROPE_HALF: rotation pairs (u_p, u_{p + hd/2}).  Pair p's
+ *                axis, frequency and angle are the same in both layouts.
+ *   norm_width   DIT_NORM_HEAD: RMS over each head's hd values, weights [hd];
+ *                DIT_NORM_ROW: RMS over the token's whole H*hd row, weights
+ *                [H*hd] (then w_q and w_k must be 16-byte aligned).
+ * Other arguments, errors and limits as dit_qk_rmsnorm_rope3d; an unknown
+ * option returns DIT_ERR_VALUE.  dit_qk_rmsnorm_rope3d is this function with
+ * (DIT_ROPE_INTERLEAVED, DIT_NORM_HEAD).
+ */
+int dit_qk_rmsnorm_rope3d_ex(uint16_t* q, uint16_t* k, int64_t row_stride,
+                             const void* w_q, const void* w_k, int w_dtype,
+                             int B, int64_t N, int H, int hd,
+                             int T, int Hg, int Wg, const int32_t* pos, int64_t pos_offset,
+                             int pairs_t, int pairs_h, int pairs_w,
+                             double theta, double eps, int rope_layout, int norm_width,
+                             void* stream);
 
 /*
  * Cache-DiT residual-difference check between neighbouring denoising steps.

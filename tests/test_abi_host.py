@@ -34,7 +34,8 @@ def lib():
 def test_header_declares_the_hot_path():
     names = declared_functions()
     for n in ("dit_adaln_modulate", "dit_gated_residual_adaln", "dit_swiglu",
-              "dit_qk_rmsnorm_rope3d", "cachedit_residual_diff", "cachedit_workspace_bytes",
+              "dit_qk_rmsnorm_rope3d", "dit_qk_rmsnorm_rope3d_ex", "cachedit_residual_diff",
+              "cachedit_workspace_bytes",
               "cachedit_residual_sums", "cachedit_decide", "dit_status_string",
               "dit_abi_version"):
         assert n in names
@@ -142,6 +143,27 @@ def test_qk_argument_errors(lib):
     assert call(wdt=3) == E["DTYPE"]
     assert call(q=A + 4) == E["ALIGN"]
     assert call(N=0) == 0
+
+
+def test_qk_option_argument_errors(lib):
+    f = lib.dit_qk_rmsnorm_rope3d_ex
+    names = ["q", "k", "rs", "wq", "wk", "wdt", "B", "N", "H", "hd", "T", "Hg", "Wg", "pos",
+             "off", "pt", "ph", "pw", "theta", "eps", "layout", "norm", "s"]
+    ok = dict(zip(names, [A, A + 2 * 256, 768, A + 0x900000, A + 0x900100, 0, 1, 48, 4, 64, 2, 4,
+                          6, None, 0, 12, 10, 10, 1e4, 1e-6, 0, 0, None]))
+
+    def call(**kw):
+        a = dict(ok)
+        a.update(kw)
+        return f(*[a[n] for n in names])
+
+    assert call(layout=2) == E["VALUE"]
+    assert call(layout=-1) == E["VALUE"]
+    assert call(norm=2) == E["VALUE"]
+    assert call(norm=1, wq=A + 0x900004) == E["ALIGN"]     # row weights are read 16 B at a time
+    assert call(norm=1, wq=None) == E["NULL"]
+    assert call(hd=48, H=4, layout=1) == E["SHAPE"]
+    assert call(N=0, layout=1, norm=1) == 0
 
 
 def test_cachedit_argument_errors(lib):

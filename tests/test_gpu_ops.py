@@ -230,24 +230,31 @@ def test_swiglu_empty():
 # ----------------------------------------------------- QK RMSNorm + RoPE
 
 
-def _qk_case(orc, wl, fused, which="qk", pos_mode="grid", w_dtype=torch.float32, offset=0):
+def _qk_case(orc, wl, fused, which="qk", pos_mode="grid", w_dtype=torch.float32, offset=0,
+             layout=dbp.ROPE_INTERLEAVED, norm=dbp.NORM_HEAD):
     B, N, H, hd = wl.B, wl.N, wl.H, wl.hd
     D = H * hd
     qkv = rows(wl, W.S_QKV, 3 * D)
     if not fused:
         q = qkv[:, :D].contiguous()
         k = qkv[:, D:2 * D].contiguous()
-    wq, wk = W.norm_weights(wl)
+    wq, wk = W.norm_weights(wl) if norm == dbp.NORM_HEAD else W.row_norm_weights(wl)
     wq, wk = wq.to(w_dtype), wk.to(w_dtype)
     if pos_mode == "grid":
         pos = np.tile(orc.grid_positions(wl.T, wl.Hg, wl.Wg, offset, N), (B, 1))
     else:
         pos = W.positions(wl).numpy() if wl.explicit_positions else np.tile(
             orc.grid_positions(wl.T, wl.Hg, wl.Wg, 0, N), (B, 1))
-    ref_q = orc.qk_rmsnorm_rope3d(bits(qkv[:, :D]), wq.double().numpy(), H, hd, pos, wl.pairs,
-                                  wl.theta, wl.eps)
-    ref_k = orc.qk_rmsnorm_rope3d(bits(qkv[:, D:2 * D]), wk.double().numpy(), H, hd, pos,
-                                  wl.pairs, wl.theta, wl.eps)
+    if layout == dbp.ROPE_INTERLEAVED and norm == dbp.NORM_HEAD:
+        ref_q = orc.qk_rmsnorm_rope3d(bits(qkv[:, :D]), wq.double().numpy(), H, hd, pos,
+                                      wl.pairs, wl.theta, wl.eps)
+        ref_k = orc.qk_rmsnorm_rope3d(bits(qkv[:, D:2 * D]), wk.double().numpy(), H, hd, pos,
+                                      wl.pairs, wl.theta, wl.eps)
+    else:
+        ref_q = orc.qk_rmsnorm_rope3d_ex(bits(qkv[:, :D]), wq.double().numpy(), H, hd, pos,
+                                         wl.pairs, wl.theta, wl.eps, layout=layout, norm=norm)
+        ref_k = orc.qk_rmsnorm_rope3d_ex(bits(qkv[:, D:2 * D]), wk.double().numpy(), H, hd, pos,
+                                         wl.pairs, wl.theta, wl.eps, layout=layout, norm=norm)
     if fused:
         buf, check = guarded((B * N, 3 * D))
         buf.copy_(qkv.to(DEV))
@@ -263,7 +270,8 @@ def _qk_case(orc, wl, fused, which="qk", pos_mode="grid", w_dtype=torch.float32,
     dbp.qk_rmsnorm_rope3d(qg if "q" in which else None, kg if "k" in which else None,
                           wq.to(DEV), wk.to(DEV), H, wl.pairs,
                           grid=(wl.T, wl.Hg, wl.Wg) if posg is None else None, pos=posg,
-                          pos_offset=offset, theta=wl.theta, eps=wl.eps)
+                          pos_offset=offset, theta=wl.theta, eps=wl.eps, rope_layout=layout,
+                          norm_width=norm)
     torch.cuda.synchronize()
     check()
     q_in = bits(qkv[:, :D])
@@ -324,6 +332,55 @@ def test_qk_shard_offset_matches_full(orc):
         assert torch.equal(part.view(torch.int16), full[:, a:b].view(torch.int16))
     # and the shard against the oracle
     _qk_case(orc, wl, fused=True, offset=0)
+
+
+OPTIONS = [(dbp.ROPE_HALF, dbp.NORM_HEAD), (dbp.ROPE_INTERLEAVED, dbp.NORM_ROW),
+           (dbp.ROPE_HALF, dbp.NORM_ROW)]
+
+
+@pytest.mark.parametrize("layout,norm", OPTIONS)
+@pytest.mark.parametrize("name", ["tiny", "small"])
+def test_qk_options(orc, name, layout, norm):
+    """Rotate-half pairs and the whole-row norm against the oracle, fused qkv."""
+    _qk_case(orc, W.CONFIGS[name], fused=True, layout=layout, norm=norm)
+
+
+@pytest.mark.parametrize("layout,norm", OPTIONS)
+@pytest.mark.parametrize("hd,pairs,H", [(32, (6, 5, 5), 5), (64, (12, 10, 10), 3),
+                                        (128, (22, 21, 21), 3), (256, (44, 42, 42), 2),
+                                        (128, (22, 21, 21), 40)])
+def test_qk_options_head_dims_ragged(orc, hd, pairs, H, layout, norm):
+    """Every head size; widths that leave a ragged last lane-vector pass,
+    up to 5120 (H=40), where the row kernel holds 20 vectors a lane."""
+    wl = W.Workload("ragged", B=2, T=3, Hg=5, Wg=7, D=H * hd, H=H, hd=hd, F=8, pairs=pairs)
+    _qk_case(orc, wl, fused=True, layout=layout, norm=norm)
+
+
+@pytest.mark.parametrize("layout,norm", OPTIONS)
+def test_qk_options_single_tensor_separate_buffers_bf16_weights(orc, layout, norm):
+    wl = W.CONFIGS["tiny"]
+    _qk_case(orc, wl, fused=False, which="k", w_dtype=torch.bfloat16, layout=layout, norm=norm)
+    _qk_case(orc, wl, fused=False, which="q", layout=layout, norm=norm, pos_mode="explicit")
+
+
+def test_qk_option_errors():
+    wl = W.CONFIGS["tiny"]
+    D = wl.H * wl.hd
+    x = torch.zeros(1, 4, 3 * D, dtype=torch.bfloat16, device=DEV)
+    wq, wk = (w.to(DEV) for w in W.norm_weights(wl))
+    rq, rk = (w.to(DEV) for w in W.row_norm_weights(wl))
+    grid = (1, 1, 4)
+    with pytest.raises(dbp.DitError) as e:
+        dbp.qk_rmsnorm_rope3d(x[:, :, :D], x[:, :, D:2 * D], wq, wk, wl.H, wl.pairs, grid=grid,
+                              rope_layout=2)
+    assert e.value.status == -8
+    with pytest.raises(ValueError):      # a head-sized weight for the whole-row norm
+        dbp.qk_rmsnorm_rope3d(x[:, :, :D], None, wq, None, wl.H, wl.pairs, grid=grid,
+                              norm_width=dbp.NORM_ROW)
+    dbp.qk_rmsnorm_rope3d(x[:, :, :D], x[:, :, D:2 * D], rq, rk, wl.H, wl.pairs, grid=grid,
+                          norm_width=dbp.NORM_ROW)
+    torch.cuda.synchronize()
+    assert torch.count_nonzero(x) == 0   # a zero row stays zero under either norm
 
 
 def test_qk_zero_position_is_plain_rms_norm(orc):
