@@ -68,6 +68,13 @@ class Oracle:
         L.dito_cachedit_decide.restype = _int
         L.dito_cachedit_residual_diff.argtypes = [_u16p, _u16p, _int, _i64, _int, _dbl,
                                                   _f64p, _u8p]
+        L.dito_adaln_modulate_tok.argtypes = [_u16p, _f64p, _f64p, _i64, _i64, _u8p, _int, _int,
+                                              _i64, _int, _dbl, _f64p, _f64p]
+        L.dito_gated_residual_adaln_tok.argtypes = [_u16p, _u16p, _f64p, _f64p, _f64p, _i64,
+                                                    _i64, _u8p, _int, _int, _i64, _int, _dbl,
+                                                    _u16p, _f64p, _f64p]
+        L.dito_adaln_modulate_tok.restype = _int
+        L.dito_gated_residual_adaln_tok.restype = _int
         for name in ("dito_adaln_modulate", "dito_gated_residual_adaln", "dito_swiglu",
                      "dito_grid_positions", "dito_qk_rmsnorm_rope3d",
                      "dito_qk_rmsnorm_rope3d_ex", "dito_cachedit_residual_diff"):
@@ -105,6 +112,44 @@ class Oracle:
                                             B, N, D, eps, _p(y, _f64p), _p(work, _f64p)),
                "adaln_modulate")
         return y
+
+    def adaln_modulate_tok(self, x, shift, scale, set_index, eps):
+        """x: [B,N,D] bf16 bits; shift, scale: [B,S,D] (S modulation sets);
+        set_index: [B,N] uint8. Token (b, n) uses set set_index[b, n].
+        Returns y [B,N,D] fp64."""
+        x = _c(x, np.uint16)
+        B, N, D = x.shape
+        shift = _c(shift, np.float64).reshape(B, -1, D)
+        S = shift.shape[1]
+        scale = _c(scale, np.float64).reshape(B, S, D)
+        idx = _c(set_index, np.uint8).reshape(B, N)
+        y = np.empty((B, N, D), dtype=np.float64)
+        work = np.empty(D, dtype=np.float64)
+        _check(self.lib.dito_adaln_modulate_tok(
+            _p(x, _u16p), _p(shift, _f64p), _p(scale, _f64p), S * D, D,
+            _p(idx, _u8p), S, B, N, D, eps, _p(y, _f64p),
+            _p(work, _f64p)), "adaln_modulate_tok")
+        return y
+
+    def gated_residual_adaln_tok(self, x, r, gate, shift, scale, set_index, eps):
+        """As gated_residual_adaln with [B,S,D] modulation sets chosen per
+        token by set_index [B,N] uint8. Returns (x_out bits, y fp64)."""
+        x = _c(x, np.uint16)
+        r = _c(r, np.uint16)
+        B, N, D = x.shape
+        gate = _c(gate, np.float64).reshape(B, -1, D)
+        S = gate.shape[1]
+        shift = _c(shift, np.float64).reshape(B, S, D)
+        scale = _c(scale, np.float64).reshape(B, S, D)
+        idx = _c(set_index, np.uint8).reshape(B, N)
+        x_out = np.empty((B, N, D), dtype=np.uint16)
+        y = np.empty((B, N, D), dtype=np.float64)
+        work = np.empty(D, dtype=np.float64)
+        _check(self.lib.dito_gated_residual_adaln_tok(
+            _p(x, _u16p), _p(r, _u16p), _p(gate, _f64p), _p(shift, _f64p), _p(scale, _f64p),
+            S * D, D, _p(idx, _u8p), S, B, N, D, eps,
+            _p(x_out, _u16p), _p(y, _f64p), _p(work, _f64p)), "gated_residual_adaln_tok")
+        return x_out, y
 
     def gated_residual_adaln(self, x, r, gate, shift, scale, eps):
         """x, r: [B,N,D] bf16 bits; gate/shift/scale [B,D].

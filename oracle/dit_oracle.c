@@ -166,6 +166,62 @@ int dito_gated_residual_adaln(const uint16_t* x, const uint16_t* r,
     return 0;
 }
 
+/* ---------------------------------------- per-token modulation sets (a1, a2) */
+
+/*
+ * The two AdaLN operators with the modulation chosen per token instead of
+ * per sample: token (b, n) takes set s = set_index[b*N + n] (0 <= s <
+ * n_sets) of its sample, whose vectors start at b*mod_batch_stride +
+ * s*mod_set_stride of shift, scale (and gate).  Everything else is the
+ * operator above, row by row.  Reading: [H3BASE], section "Phần nào đã được
+ * phát hành?", names first/last-frame conditioned generation (FL2VA); the
+ * tokens of conditioning frames then carry modulation of their own.  The
+ * pages say no more, so any assignment of tokens to a few sets is allowed.
+ * An index >= n_sets returns -3 (nothing else checked).
+ */
+int dito_adaln_modulate_tok(const uint16_t* x, const double* shift, const double* scale,
+                            int64_t mod_batch_stride, int64_t mod_set_stride,
+                            const uint8_t* set_index, int n_sets, int B, int64_t N, int D,
+                            double eps, double* y, double* work)
+{
+    if (D <= 0 || B < 0 || N < 0 || n_sets < 1) return -2;
+    for (int b = 0; b < B; ++b)
+        for (int64_t n = 0; n < N; ++n) {
+            int64_t tok = (int64_t)b * N + n;
+            int set = set_index[tok];
+            if (set >= n_sets) return -3;
+            int64_t m = b * mod_batch_stride + set * mod_set_stride;
+            for (int d = 0; d < D; ++d) work[d] = dito_bf16_to_f64(x[tok * D + d]);
+            adaln_row(work, shift + m, scale + m, D, eps, y + tok * D);
+        }
+    return 0;
+}
+
+int dito_gated_residual_adaln_tok(const uint16_t* x, const uint16_t* r, const double* gate,
+                                  const double* shift, const double* scale,
+                                  int64_t mod_batch_stride, int64_t mod_set_stride,
+                                  const uint8_t* set_index, int n_sets, int B, int64_t N, int D,
+                                  double eps, uint16_t* x_out, double* y, double* work)
+{
+    if (D <= 0 || B < 0 || N < 0 || n_sets < 1) return -2;
+    for (int b = 0; b < B; ++b)
+        for (int64_t n = 0; n < N; ++n) {
+            int64_t tok = (int64_t)b * N + n;
+            int sg = set_index[tok];
+            if (sg >= n_sets) return -3;
+            int64_t mg = b * mod_batch_stride + sg * mod_set_stride;
+            for (int d = 0; d < D; ++d) {
+                double v = dito_bf16_to_f64(x[tok * D + d]) +
+                           gate[mg + d] * dito_bf16_to_f64(r[tok * D + d]);
+                uint16_t h = dito_f64_to_bf16(v);
+                x_out[tok * D + d] = h;
+                work[d] = dito_bf16_to_f64(h);
+            }
+            adaln_row(work, shift + mg, scale + mg, D, eps, y + tok * D);
+        }
+    return 0;
+}
+
 /* ------------------------------------------------------------ SwiGLU (a3) */
 
 /*

@@ -3,6 +3,7 @@ from decimal import Decimal, getcontext
 from fractions import Fraction
 
 import numpy as np
+import pytest
 import torch
 
 from conftest import closed_form, load_golden
@@ -164,3 +165,74 @@ def test_gated_y_is_adaln_of_rounded_residual(orc):
     sh, sc, gt = (rng.standard_normal((B, D)) * 0.3 for _ in range(3))
     x_out, y = orc.gated_residual_adaln(x, r, gt, sh, sc, eps)
     assert np.array_equal(y, orc.adaln_modulate(x_out, sh, sc, eps))
+
+
+# ------------------------------------------- per-token modulation sets
+
+
+def _token_case(orc, seed, B=2, N=5, D=16, S=3):
+    rng = np.random.default_rng(seed)
+    x = _bf16(orc, rng.standard_normal((B, N, D)))
+    r = _bf16(orc, rng.standard_normal((B, N, D)))
+    mods = [rng.standard_normal((B, S, D)) * 0.3 for _ in range(3)]
+    idx = rng.integers(0, S, (B, N)).astype(np.uint8)
+    return x, r, mods, idx
+
+
+def test_token_sets_all_zero_are_per_sample(orc):
+    """Every token on set 0 is the per-sample operator with set 0's vectors."""
+    x, r, (g, sh, sc), idx = _token_case(orc, 1)
+    idx[:] = 0
+    y = orc.adaln_modulate_tok(x, sh, sc, idx, 1e-6)
+    assert np.array_equal(y, orc.adaln_modulate(x, sh[:, 0], sc[:, 0], 1e-6))
+    xo, y = orc.gated_residual_adaln_tok(x, r, g, sh, sc, idx, 1e-6)
+    xo0, y0 = orc.gated_residual_adaln(x, r, g[:, 0], sh[:, 0], sc[:, 0], 1e-6)
+    assert np.array_equal(xo, xo0) and np.array_equal(y, y0)
+
+
+def test_token_sets_each_token_uses_its_own_set(orc):
+    """Token (b, n) equals the per-sample operator run on that token alone
+    with the vectors of set idx[b, n] of sample b."""
+    x, r, (g, sh, sc), idx = _token_case(orc, 2)
+    B, N, D = x.shape
+    y = orc.adaln_modulate_tok(x, sh, sc, idx, 1e-6)
+    xo, yg = orc.gated_residual_adaln_tok(x, r, g, sh, sc, idx, 1e-6)
+    for b in range(B):
+        for n in range(N):
+            s = idx[b, n]
+            one = orc.adaln_modulate(x[b:b + 1, n:n + 1], sh[b, s], sc[b, s], 1e-6)
+            assert np.array_equal(y[b, n], one[0, 0])
+            xo1, y1 = orc.gated_residual_adaln(x[b:b + 1, n:n + 1], r[b:b + 1, n:n + 1], g[b, s],
+                                               sh[b, s], sc[b, s], 1e-6)
+            assert np.array_equal(xo[b, n], xo1[0, 0]) and np.array_equal(yg[b, n], y1[0, 0])
+
+
+def test_token_sets_closed_forms(orc):
+    """Set 0 has zero modulation (a plain LayerNorm: row [1, 2, 3, 4] gives
+    (x - 2.5) / sqrt(1.25 + eps)); set 1 has scale = -1 (y is its shift) and
+    gate 0 (the residual passes unchanged)."""
+    eps = 1e-6
+    x = _bf16(orc, [[[1, 2, 3, 4], [1, 2, 3, 4], [-8, 0.5, 3, 7]]])
+    r = _bf16(orc, np.full((1, 3, 4), 0.75))
+    sh = np.array([[[0, 0, 0, 0], [0.5, -1.5, 2.0, 3.25]]])
+    sc = np.array([[[0, 0, 0, 0], [-1, -1, -1, -1]]])
+    g = np.array([[[1, 1, 1, 1], [0, 0, 0, 0]]])
+    idx = np.array([[0, 1, 1]], np.uint8)
+    y = orc.adaln_modulate_tok(x, sh, sc, idx, eps)
+    ln = (np.array([1, 2, 3, 4]) - 2.5) / np.sqrt(1.25 + eps)
+    assert np.allclose(y[0, 0], ln, rtol=1e-15, atol=1e-15)
+    assert np.array_equal(y[0, 1], sh[0, 1]) and np.array_equal(y[0, 2], sh[0, 1])
+    xo, yg = orc.gated_residual_adaln_tok(x, r, g, sh, sc, idx, eps)
+    assert np.array_equal(xo[0, 1:], x[0, 1:])                       # gate 0
+    assert np.array_equal(orc.bf16_to_f64(xo[0, 0]), [1.75, 2.75, 3.75, 4.75])
+    assert np.allclose(yg[0, 0], ln, rtol=1e-15, atol=1e-15)        # LN is shift-invariant
+    assert np.array_equal(yg[0, 2], sh[0, 1])
+
+
+def test_token_set_out_of_range_is_an_error(orc):
+    x, r, (g, sh, sc), idx = _token_case(orc, 3, S=2)
+    idx[0, 0] = 2
+    with pytest.raises(ValueError):
+        orc.adaln_modulate_tok(x, sh, sc, idx, 1e-6)
+    with pytest.raises(ValueError):
+        orc.gated_residual_adaln_tok(x, r, g, sh, sc, idx, 1e-6)

@@ -23,6 +23,12 @@ MUTANTS = {
     "gate_adds_instead_of_multiplies": ("+ g[d] * dito_bf16_to_f64(r[row + d])",
                                         "+ g[d] + dito_bf16_to_f64(r[row + d])"),
     "gate_ln_reads_unrounded": ("work[d] = dito_bf16_to_f64(h);", "work[d] = v;"),
+    "tok_set_ignored": ("int64_t m = b * mod_batch_stride + set * mod_set_stride;",
+                        "int64_t m = b * mod_batch_stride;"),
+    "tok_set_strided_as_sample": ("int64_t m = b * mod_batch_stride + set * mod_set_stride;",
+                                  "int64_t m = (b + set) * mod_set_stride;"),
+    "tok_gated_index_per_token_of_sample": ("int sg = set_index[tok];", "int sg = set_index[n];"),
+    "tok_gated_gate_from_set0": ("gate[mg + d]", "gate[b * mod_batch_stride + d]"),
     "swiglu_exp_sign": ("a / (1.0 + exp(-a))", "a / (1.0 + exp(a))"),
     "swiglu_halves_swapped": ("double a = dito_bf16_to_f64(in[m * 2 * (int64_t)F + j]);",
                               "double a = dito_bf16_to_f64(in[m * 2 * (int64_t)F + F + j]);"),
