@@ -22,7 +22,10 @@ MUTANTS = {
     "ln_mean_dropped": ("(x[d] - mu) * inv", "x[d] * inv"),
     "gate_adds_instead_of_multiplies": ("+ g[d] * dito_bf16_to_f64(r[row + d])",
                                         "+ g[d] + dito_bf16_to_f64(r[row + d])"),
-    "gate_ln_reads_unrounded": ("work[d] = dito_bf16_to_f64(h);", "work[d] = v;"),
+    "gate_ln_reads_unrounded": ("x_out[row + d] = h;\n                work[d] = dito_bf16_to_f64(h);",
+                                "x_out[row + d] = h;\n                work[d] = v;"),
+    "tok_gate_ln_reads_unrounded": ("x_out[tok * D + d] = h;\n                work[d] = dito_bf16_to_f64(h);",
+                                    "x_out[tok * D + d] = h;\n                work[d] = v;"),
     "tok_set_ignored": ("int64_t m = b * mod_batch_stride + set * mod_set_stride;",
                         "int64_t m = b * mod_batch_stride;"),
     "tok_set_strided_as_sample": ("int64_t m = b * mod_batch_stride + set * mod_set_stride;",
