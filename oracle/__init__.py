@@ -75,6 +75,8 @@ class Oracle:
                                                     _u16p, _f64p, _f64p]
         L.dito_adaln_modulate_tok.restype = _int
         L.dito_gated_residual_adaln_tok.restype = _int
+        L.dito_residual_store.argtypes = [_u16p, _u16p, _i64, _u16p]
+        L.dito_residual_apply.argtypes = [_u16p, _u16p, _i64, _u16p]
         for name in ("dito_adaln_modulate", "dito_gated_residual_adaln", "dito_swiglu",
                      "dito_grid_positions", "dito_qk_rmsnorm_rope3d",
                      "dito_qk_rmsnorm_rope3d_ex", "dito_cachedit_residual_diff"):
@@ -228,6 +230,27 @@ class Oracle:
                "qk_rmsnorm_rope3d_ex")
         return out
 
+    def residual_store(self, before, after):
+        """R = bf16(after - before), elementwise on bf16 bits."""
+        before = _c(before, np.uint16)
+        after = _c(after, np.uint16)
+        if before.shape != after.shape:
+            raise ValueError("shapes differ")
+        out = np.empty(before.shape, dtype=np.uint16)
+        self.lib.dito_residual_store(_p(before, _u16p), _p(after, _u16p), before.size,
+                                     _p(out, _u16p))
+        return out
+
+    def residual_apply(self, h, residual):
+        """out = bf16(h + R), elementwise on bf16 bits."""
+        h = _c(h, np.uint16)
+        residual = _c(residual, np.uint16)
+        if h.shape != residual.shape:
+            raise ValueError("shapes differ")
+        out = np.empty(h.shape, dtype=np.uint16)
+        self.lib.dito_residual_apply(_p(h, _u16p), _p(residual, _u16p), h.size, _p(out, _u16p))
+        return out
+
     def cachedit_sums(self, prev, cur):
         """(sum |cur - prev|, sum |prev|) over all elements, fp64."""
         prev = _c(prev, np.uint16)
@@ -276,3 +299,29 @@ def __getattr__(name):
     if name.startswith("_"):
         raise AttributeError(name)
     return getattr(default(), name)
+
+
+def cache_policy(rels, threshold, warmup_steps=0, max_cached_steps=0):
+    """The Cache-DiT reuse rule over a denoising run, one decision per step.
+
+    [REPORT], section "Só com três camadas de aceleração somadas chega-se a 6
+    vezes": a residual-difference threshold decides whether a step reuses
+    the results cached between neighbouring steps (0.04 conservative, 0.08 in
+    the more aggressive stride mode).  rels[t] is the relative L1 difference
+    of step t's first-block residual against step t-1's (rels[0] is ignored:
+    the first step has nothing to compare with).  Step t reuses iff
+        t >= 1 and t >= warmup_steps and rels[t] < threshold
+        and (max_cached_steps == 0 or fewer than max_cached_steps steps in a
+             row before t reused).
+    Readings: the comparison is always with the previous step (neighbouring
+    steps); warm-up and the cap on consecutive reuses are optional guards
+    (0 = off) that the pages do not mention.  Returns a list of bools.
+    """
+    out = []
+    run = 0
+    for t, rel in enumerate(rels):
+        reuse = (t >= 1 and t >= warmup_steps and rel < threshold
+                 and (max_cached_steps == 0 or run < max_cached_steps))
+        run = run + 1 if reuse else 0
+        out.append(reuse)
+    return out

@@ -427,3 +427,29 @@ int dito_cachedit_residual_diff(const uint16_t* prev, const uint16_t* cur,
     }
     return 0;
 }
+
+/* --------------------------- Cache-DiT residual cache across steps (f3) */
+
+/*
+ * [REPORT], section "Só com três camadas de aceleração somadas chega-se a 6
+ * vezes": Cache-DiT reuses results cached between neighbouring denoising
+ * steps.  Reading: the cached result is the residual the skipped blocks add
+ * to the hidden state, R = after - before, stored in bf16 like the hidden
+ * state; a reusing step adds it back, out = h + R.  Each is the exact
+ * rational value rounded once to bf16: fp64 holds the sum or difference of
+ * two bf16 values exactly unless their exponents differ by more than 44,
+ * and then the smaller one lies far below half a bf16 ulp of the larger, so
+ * the single rounding of the fp64 value still gives the nearest bf16.
+ */
+void dito_residual_store(const uint16_t* before, const uint16_t* after, int64_t n,
+                         uint16_t* residual)
+{
+    for (int64_t i = 0; i < n; ++i)
+        residual[i] = dito_f64_to_bf16(dito_bf16_to_f64(after[i]) - dito_bf16_to_f64(before[i]));
+}
+
+void dito_residual_apply(const uint16_t* h, const uint16_t* residual, int64_t n, uint16_t* out)
+{
+    for (int64_t i = 0; i < n; ++i)
+        out[i] = dito_f64_to_bf16(dito_bf16_to_f64(h[i]) + dito_bf16_to_f64(residual[i]));
+}

@@ -32,6 +32,12 @@ MUTANTS = {
                                   "int64_t m = (b + set) * mod_set_stride;"),
     "tok_gated_index_per_token_of_sample": ("int sg = set_index[tok];", "int sg = set_index[n];"),
     "tok_gated_gate_from_set0": ("gate[mg + d]", "gate[b * mod_batch_stride + d]"),
+    "store_operands_swapped": ("dito_f64_to_bf16(dito_bf16_to_f64(after[i]) - dito_bf16_to_f64(before[i]))",
+                               "dito_f64_to_bf16(dito_bf16_to_f64(before[i]) - dito_bf16_to_f64(after[i]))"),
+    "apply_subtracts": ("dito_f64_to_bf16(dito_bf16_to_f64(h[i]) + dito_bf16_to_f64(residual[i]))",
+                        "dito_f64_to_bf16(dito_bf16_to_f64(h[i]) - dito_bf16_to_f64(residual[i]))"),
+    "apply_ties_away": ("dito_f64_to_bf16(dito_bf16_to_f64(h[i]) + dito_bf16_to_f64(residual[i]))",
+                        "dito_f64_to_bf16(nextafter(dito_bf16_to_f64(h[i]) + dito_bf16_to_f64(residual[i]), 1e300))"),
     "swiglu_exp_sign": ("a / (1.0 + exp(-a))", "a / (1.0 + exp(a))"),
     "swiglu_halves_swapped": ("double a = dito_bf16_to_f64(in[m * 2 * (int64_t)F + j]);",
                               "double a = dito_bf16_to_f64(in[m * 2 * (int64_t)F + F + j]);"),
@@ -81,7 +87,7 @@ MUTANTS = {
 }
 
 PIN_MODULES = ["test_oracle_bf16", "test_oracle_adaln", "test_oracle_swiglu", "test_oracle_qk",
-               "test_oracle_cachedit"]
+               "test_oracle_cachedit", "test_oracle_cache_step"]
 
 
 def _pins():
