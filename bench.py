@@ -254,13 +254,14 @@ def time_device(chain, steps, warmup, world):
     return total_ms, per_op
 
 
-QK_OPTIONS = {"rope_half+norm_head": (1, 0), "interleaved+norm_row": (0, 1),
-              "rope_half+norm_row": (1, 1)}
+QK_OPTIONS = {"rope_half+norm_head": (1, 0, False), "interleaved+norm_row": (0, 1, False),
+              "rope_half+norm_row": (1, 1, False), "interleaved+norm_head->[B,H,N,hd]": (0, 0, True)}
 
 
 def time_qk_options(chain, steps, warmup, world):
     """Device ms per launch of the QK op with its non-default options (rotate-
-    half pairs, whole-row norm) on the chain's q and k, outside the chain."""
+    half pairs, whole-row norm, results written head-major into separate q/k
+    buffers) on the chain's q and k, outside the chain."""
     import torch
     import dit_block_pass_b200 as dbp
     from dit_block_pass_b200 import workloads as W
@@ -269,13 +270,18 @@ def time_qk_options(chain, steps, warmup, world):
     grid = None if c.pos is not None else (wl.T, wl.Hg, wl.Wg)
     stream = torch.cuda.current_stream()
     out = {}
-    for name, (layout, norm) in QK_OPTIONS.items():
+    B, N, H, hd = wl.B, wl.N, wl.H, wl.hd
+    for name, (layout, norm, head_major) in QK_OPTIONS.items():
         wq, wk = (c.wq, c.wk) if norm == dbp.NORM_HEAD else (rq, rk)
+        qo = ko = None
+        if head_major:
+            qo = torch.empty(B, H, N, hd, dtype=torch.bfloat16, device=c.dev).transpose(1, 2)
+            ko = torch.empty(B, H, N, hd, dtype=torch.bfloat16, device=c.dev).transpose(1, 2)
 
         def op():
             dbp.qk_rmsnorm_rope3d(c.qkv[:, :, :D], c.qkv[:, :, D:2 * D], wq, wk, wl.H, wl.pairs,
                                   grid=grid, pos=c.pos, theta=wl.theta, eps=wl.eps,
-                                  rope_layout=layout, norm_width=norm)
+                                  rope_layout=layout, norm_width=norm, q_out=qo, k_out=ko)
         for _ in range(warmup):
             op()
         barrier_sync(world)
@@ -286,6 +292,76 @@ def time_qk_options(chain, steps, warmup, world):
             ev[2 * s + 1].record(stream)
         barrier_sync(world)
         out[name] = sum(ev[2 * s].elapsed_time(ev[2 * s + 1]) for s in range(steps)) / steps
+        del qo, ko
+    return out
+
+
+def time_token_sets(chain, steps, warmup, world):
+    """Device ms per launch of the two AdaLN operators with per-token
+    modulation sets: the first and last latent frames' tokens (the
+    conditioning frames of first/last-frame generation) on set 1, the rest on
+    set 0; [B, 2, 6, D] fp32 modulation."""
+    import torch
+    import dit_block_pass_b200 as dbp
+    from dit_block_pass_b200 import workloads as W
+    c, wl = chain, chain.wl
+    B, N, D = wl.B, wl.N, wl.D
+    frame = wl.Hg * wl.Wg
+    idx = torch.zeros(B, N, dtype=torch.uint8, device=c.dev)
+    idx[:, :frame] = 1
+    idx[:, max(0, wl.T - 1) * frame:wl.T * frame] = 1
+    base = W.normal(wl.seed, 90, B * 2 * 6, D, sigma=0.1, dtype=torch.float32,
+                    device=c.dev).view(B, 2, 6, D)
+    m = [base[:, :, k] for k in range(6)]
+    ops = {
+        "adaln_modulate": lambda: dbp.adaln_modulate(c.x, m[0], m[1], wl.eps, out=c.y1,
+                                                     set_index=idx),
+        "gated_residual_adaln": lambda: dbp.gated_residual_adaln(
+            c.x, c.r, m[2], m[3], m[4], wl.eps, x_out=c.xo, y=c.y2, set_index=idx),
+    }
+    stream = torch.cuda.current_stream()
+    out = {}
+    for name, op in ops.items():
+        for _ in range(warmup):
+            op()
+        barrier_sync(world)
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(2 * steps)]
+        for s in range(steps):
+            ev[2 * s].record(stream)
+            op()
+            ev[2 * s + 1].record(stream)
+        barrier_sync(world)
+        out[name] = sum(ev[2 * s].elapsed_time(ev[2 * s + 1]) for s in range(steps)) / steps
+    share = float(idx.float().mean().item())
+    return out, share
+
+
+def time_cache_step(chain, steps, warmup, world):
+    """Device ms per launch of the Cache-DiT step-cache operators on the
+    clip's hidden state: storing the skipped blocks' residual
+    (bf16(after - before)) and adding it back on a reusing step."""
+    import torch
+    import dit_block_pass_b200 as dbp
+    c = chain
+    R = torch.empty_like(c.x)
+    ops = {
+        "cachedit_residual_store": lambda: dbp.cachedit_residual_store(c.x, c.r, out=R),
+        "cachedit_residual_apply": lambda: dbp.cachedit_residual_apply(c.x, c.r, out=c.y1),
+    }
+    stream = torch.cuda.current_stream()
+    out = {}
+    for name, op in ops.items():
+        for _ in range(warmup):
+            op()
+        barrier_sync(world)
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(2 * steps)]
+        for s in range(steps):
+            ev[2 * s].record(stream)
+            op()
+            ev[2 * s + 1].record(stream)
+        barrier_sync(world)
+        out[name] = sum(ev[2 * s].elapsed_time(ev[2 * s + 1]) for s in range(steps)) / steps
+    del R
     return out
 
 
@@ -487,6 +563,8 @@ def main():
     try:
         total_ms, per_op = time_device(chain, args.steps, args.warmup, world)
         qk_opt = time_qk_options(chain, args.steps, args.warmup, world)
+        tok_sets, tok_share = time_token_sets(chain, args.steps, args.warmup, world)
+        step_cache = time_cache_step(chain, args.steps, args.warmup, world)
     finally:
         if sampler:
             sampler.__exit__(None, None, None)
@@ -508,6 +586,18 @@ def main():
         ms = max_over_ranks(ms, world)
         gbs = nbytes["qk_rmsnorm_rope3d"] / (ms / 1000.0) / 1e9
         qk_options[name] = {"ms": round(ms, 4), "GB/s": round(gbs, 1),
+                            "frac_of_peak": round(gbs / peak, 4)}
+    token_sets = {"tokens_on_set_1": round(tok_share, 4)}
+    for name, ms in tok_sets.items():
+        ms = max_over_ranks(ms, world)
+        gbs = nbytes[name] / (ms / 1000.0) / 1e9
+        token_sets[name] = {"ms": round(ms, 4), "GB/s": round(gbs, 1),
+                            "frac_of_peak": round(gbs / peak, 4)}
+    cache_step = {}
+    for name, ms in step_cache.items():
+        ms = max_over_ranks(ms, world)
+        gbs = 6 * wl.M * wl.D / (ms / 1000.0) / 1e9        # read two, write one
+        cache_step[name] = {"ms": round(ms, 4), "GB/s": round(gbs, 1),
                             "frac_of_peak": round(gbs / peak, 4)}
     dom_ms = per_op[OPS.index(DOMINANT)]
     achieved = nbytes[DOMINANT] / (dom_ms / 1000.0) / 1e9
@@ -547,7 +637,9 @@ def main():
                        "tokens_per_step_per_gpu": tokens,
                        "l2": "every input is larger than L2 (126 MB); no flush",
                        "parallelism": f"{world} independent clip(s), one per GPU"},
-            "ops": ops, "qk_options": qk_options, "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+            "ops": ops, "qk_options": qk_options, "token_sets": token_sets,
+            "cache_step": cache_step,
+            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": chain.launches_per_step() * args.steps, "clocks": clocks,
         }
         print(json.dumps(line), flush=True)

@@ -25,7 +25,8 @@ __all__ = [
     "DitError", "library", "library_path", "adaln_modulate", "gated_residual_adaln", "swiglu",
     "qk_rmsnorm_rope3d", "cachedit_workspace_bytes", "cachedit_residual_diff",
     "cachedit_residual_sums", "cachedit_decide", "cachedit_residual_diff_noalloc",
-    "launch_counts", "F32", "BF16", "ROPE_INTERLEAVED", "ROPE_HALF", "NORM_HEAD", "NORM_ROW",
+    "launch_counts", "QKOut", "CachePolicy", "cachedit_residual_store",
+    "cachedit_residual_apply", "F32", "BF16", "ROPE_INTERLEAVED", "ROPE_HALF", "NORM_HEAD", "NORM_ROW",
 ]
 
 F32, BF16 = 0, 1
@@ -40,10 +41,24 @@ _lock = threading.Lock()
 # kernels launched per call of each entry point (for launch accounting)
 launch_counts = {
     "adaln_modulate": 1, "gated_residual_adaln": 1, "swiglu": 1, "qk_rmsnorm_rope3d": 1,
-    "qk_rmsnorm_rope3d_ex": 1,
+    "qk_rmsnorm_rope3d_ex": 1, "adaln_modulate_tok": 1, "gated_residual_adaln_tok": 1,
     "cachedit_residual_diff": 2, "cachedit_residual_sums": 2, "cachedit_decide": 1,
-    "cachedit_residual_diff_noalloc": 2,
+    "cachedit_residual_diff_noalloc": 2, "cachedit_residual_store": 1,
+    "cachedit_residual_apply": 1,
 }
+
+
+class QKOut(ctypes.Structure):
+    """dit_qk_out: output buffers and [B, N, H, hd] element strides."""
+    _fields_ = [("q", ctypes.c_void_p), ("k", ctypes.c_void_p), ("stride_b", ctypes.c_int64),
+                ("stride_n", ctypes.c_int64), ("stride_h", ctypes.c_int64)]
+
+
+class CachePolicyStruct(ctypes.Structure):
+    """dit_cache_policy."""
+    _fields_ = [("threshold", ctypes.c_double), ("warmup_steps", ctypes.c_int),
+                ("max_cached_steps", ctypes.c_int), ("step", ctypes.c_int), ("run", ctypes.c_int),
+                ("computed", ctypes.c_int), ("reused", ctypes.c_int)]
 
 
 class DitError(RuntimeError):
@@ -76,12 +91,21 @@ def library() -> ctypes.CDLL:
             L.dit_gated_residual_adaln.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, i64, i32,
                                                    i64, i32, dbl, vp]
             L.dit_swiglu.argtypes = [vp, vp, i64, i32, vp]
+            L.dit_adaln_modulate_tok.argtypes = [vp, vp, vp, vp, i32, i64, i64, vp, i32, i32,
+                                                 i64, i32, dbl, vp]
+            L.dit_gated_residual_adaln_tok.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, i64,
+                                                       i64, vp, i32, i32, i64, i32, dbl, vp]
             L.dit_qk_rmsnorm_rope3d.argtypes = [vp, vp, i64, vp, vp, i32, i32, i64, i32, i32,
                                                 i32, i32, i32, vp, i64, i32, i32, i32, dbl, dbl,
                                                 vp]
             L.dit_qk_rmsnorm_rope3d_ex.argtypes = [vp, vp, i64, vp, vp, i32, i32, i64, i32,
                                                    i32, i32, i32, i32, vp, i64, i32, i32, i32,
-                                                   dbl, dbl, i32, i32, vp]
+                                                   dbl, dbl, i32, i32,
+                                                   ctypes.POINTER(QKOut), vp]
+            L.cachedit_residual_store.argtypes = [vp, vp, vp, i64, vp]
+            L.cachedit_residual_apply.argtypes = [vp, vp, vp, i64, vp]
+            L.dit_cache_policy_init.argtypes = [ctypes.POINTER(CachePolicyStruct), dbl, i32, i32]
+            L.dit_cache_policy_decide.argtypes = [ctypes.POINTER(CachePolicyStruct), dbl]
             L.cachedit_workspace_bytes.restype = sz
             L.cachedit_workspace_bytes.argtypes = [i32, i64, i32]
             L.cachedit_residual_diff.argtypes = [vp, vp, i32, i64, i32, dbl, vp, vp, vp, sz, vp]
@@ -90,6 +114,9 @@ def library() -> ctypes.CDLL:
             L.cachedit_residual_diff_noalloc.argtypes = [vp, vp, i32, i64, i32, dbl, vp, vp, vp]
             L.cachedit_residual_diff_noalloc.restype = i32
             for name in ("dit_adaln_modulate", "dit_gated_residual_adaln", "dit_swiglu",
+                         "dit_adaln_modulate_tok", "dit_gated_residual_adaln_tok",
+                         "cachedit_residual_store", "cachedit_residual_apply",
+                         "dit_cache_policy_init", "dit_cache_policy_decide",
                          "dit_qk_rmsnorm_rope3d", "dit_qk_rmsnorm_rope3d_ex",
                          "cachedit_residual_diff",
                          "cachedit_residual_sums", "cachedit_decide"):
@@ -149,6 +176,31 @@ def _mod_views(B: int, D: int, *mods: torch.Tensor):
     return dt, stride
 
 
+def _set_views(B: int, N: int, D: int, set_index: torch.Tensor, *mods: torch.Tensor):
+    """Per-token modulation: vectors as [B, S, D] views (unit inner stride,
+    shared strides; a sample stride of 0 broadcasts) and set_index [B, N]
+    uint8.  Returns (dtype code, sample stride, set stride, S)."""
+    dt = _mod_dtype(mods[0])
+    if set_index.dtype != torch.uint8 or not set_index.is_cuda or \
+            set_index.numel() != B * N or not set_index.is_contiguous():
+        raise ValueError("set_index must be a contiguous CUDA uint8 [B, N] tensor")
+    strides = None
+    S = None
+    for m in mods:
+        if m.dtype != mods[0].dtype or not m.is_cuda or m.device != set_index.device:
+            raise ValueError("modulation vectors must share dtype and device")
+        if m.dim() != 3 or m.shape[0] not in (1, B) or m.shape[2] != D or m.stride(2) != 1:
+            raise ValueError(f"modulation must be [B, S, D] with unit inner stride, got "
+                             f"{tuple(m.shape)}")
+        st = (0 if m.shape[0] == 1 else m.stride(0), m.stride(1))
+        if strides is not None and (st != strides or m.shape[1] != S):
+            raise ValueError("modulation vectors must share shape and strides")
+        strides, S = st, m.shape[1]
+    if not 1 <= S <= 255:
+        raise ValueError("between 1 and 255 modulation sets")
+    return dt, strides[0], strides[1], S
+
+
 def _rows3(name: str, t: torch.Tensor):
     if t.dim() != 3 or not t.is_contiguous():
         raise ValueError(f"{name} must be a contiguous [B, N, D] tensor")
@@ -159,39 +211,58 @@ def _rows3(name: str, t: torch.Tensor):
 
 
 def adaln_modulate(x: torch.Tensor, shift: torch.Tensor, scale: torch.Tensor, eps: float = 1e-6,
-                   out: Optional[torch.Tensor] = None) -> torch.Tensor:
-    """y = LN(x) * (1 + scale) + shift per sample; x [B, N, D] bf16."""
+                   out: Optional[torch.Tensor] = None,
+                   set_index: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """y = LN(x) * (1 + scale) + shift per sample; x [B, N, D] bf16.  With
+    ``set_index`` ([B, N] uint8) shift and scale are [B, S, D] modulation sets
+    and token (b, n) uses set set_index[b, n] (an index >= S gives NaN)."""
     _need_cuda_bf16("x", x)
     B, N, D = _rows3("x", x)
-    dt, ms = _mod_views(B, D, shift, scale)
     y = torch.empty_like(x) if out is None else out
     _need_cuda_bf16("out", y)
     if y.shape != x.shape or not y.is_contiguous():
         raise ValueError("out must match x")
-    _call("dit_adaln_modulate", x.data_ptr(), y.data_ptr(), shift.data_ptr(), scale.data_ptr(),
-          dt, ms, B, N, D, float(eps), _stream(x))
+    if set_index is None:
+        dt, ms = _mod_views(B, D, shift, scale)
+        _call("dit_adaln_modulate", x.data_ptr(), y.data_ptr(), shift.data_ptr(),
+              scale.data_ptr(), dt, ms, B, N, D, float(eps), _stream(x))
+        return y
+    dt, ms, ss, S = _set_views(B, N, D, set_index, shift, scale)
+    _call("dit_adaln_modulate_tok", x.data_ptr(), y.data_ptr(), shift.data_ptr(),
+          scale.data_ptr(), dt, ms, ss, set_index.data_ptr(), S, B, N, D, float(eps), _stream(x))
     return y
 
 
 def gated_residual_adaln(x: torch.Tensor, r: torch.Tensor, gate: torch.Tensor,
                          shift: torch.Tensor, scale: torch.Tensor, eps: float = 1e-6,
-                         x_out: Optional[torch.Tensor] = None, y: Optional[torch.Tensor] = None):
-    """x' = bf16(x + gate * r); y = AdaLN(x'). Returns (x', y)."""
+                         x_out: Optional[torch.Tensor] = None, y: Optional[torch.Tensor] = None,
+                         set_index: Optional[torch.Tensor] = None):
+    """x' = bf16(x + gate * r); y = AdaLN(x'). Returns (x', y).  With
+    ``set_index`` ([B, N] uint8) gate, shift and scale are [B, S, D]
+    modulation sets chosen per token (an index >= S gives NaN)."""
     _need_cuda_bf16("x", x)
     _need_cuda_bf16("r", r)
     B, N, D = _rows3("x", x)
     if r.shape != x.shape or not r.is_contiguous():
         raise ValueError("r must match x")
-    dt, ms = _mod_views(B, D, gate, shift, scale)
+    if set_index is None:
+        dt, ms = _mod_views(B, D, gate, shift, scale)
+    else:
+        dt, ms, ss, S = _set_views(B, N, D, set_index, gate, shift, scale)
     x_out = torch.empty_like(x) if x_out is None else x_out
     y = torch.empty_like(x) if y is None else y
     for nm, t in (("x_out", x_out), ("y", y)):
         _need_cuda_bf16(nm, t)
         if t.shape != x.shape or not t.is_contiguous():
             raise ValueError(f"{nm} must match x")
-    _call("dit_gated_residual_adaln", x.data_ptr(), r.data_ptr(), x_out.data_ptr(), y.data_ptr(),
-          gate.data_ptr(), shift.data_ptr(), scale.data_ptr(), dt, ms, B, N, D, float(eps),
-          _stream(x))
+    if set_index is None:
+        _call("dit_gated_residual_adaln", x.data_ptr(), r.data_ptr(), x_out.data_ptr(),
+              y.data_ptr(), gate.data_ptr(), shift.data_ptr(), scale.data_ptr(), dt, ms, B, N, D,
+              float(eps), _stream(x))
+    else:
+        _call("dit_gated_residual_adaln_tok", x.data_ptr(), r.data_ptr(), x_out.data_ptr(),
+              y.data_ptr(), gate.data_ptr(), shift.data_ptr(), scale.data_ptr(), dt, ms, ss,
+              set_index.data_ptr(), S, B, N, D, float(eps), _stream(x))
     return x_out, y
 
 
@@ -228,14 +299,19 @@ def qk_rmsnorm_rope3d(q: Optional[torch.Tensor], k: Optional[torch.Tensor],
                       pairs: Sequence[int], grid: Optional[Sequence[int]] = None,
                       pos: Optional[torch.Tensor] = None, pos_offset: int = 0,
                       theta: float = 10000.0, eps: float = 1e-6,
-                      rope_layout: int = ROPE_INTERLEAVED, norm_width: int = NORM_HEAD) -> None:
+                      rope_layout: int = ROPE_INTERLEAVED, norm_width: int = NORM_HEAD,
+                      q_out: Optional[torch.Tensor] = None,
+                      k_out: Optional[torch.Tensor] = None) -> None:
     """In place on q and k ([B, N, H*hd] views, e.g. slices of a fused qkv
     buffer): RMSNorm with weight w, then 3D RoPE with pair split
     ``pairs`` = (t, h, w).  Positions come from ``grid`` = (T, Hg, Wg) (token
     n at global index pos_offset + n) or from ``pos`` [B*N, 3] int32.
     ``norm_width`` NORM_HEAD normalises each head (w: [hd]), NORM_ROW the
     token's whole row (w: [H*hd]); ``rope_layout`` ROPE_INTERLEAVED rotates
-    pairs (2p, 2p+1), ROPE_HALF pairs (p, p + hd/2)."""
+    pairs (2p, 2p+1), ROPE_HALF pairs (p, p + hd/2).  With ``q_out``/``k_out``
+    ([B, N, H, hd] views with any strides and a contiguous last dimension,
+    e.g. ``torch.empty(B, H, N, hd).transpose(1, 2)`` for the head-major
+    layout attention reads) q and k are only read and the results go there."""
     ref = q if q is not None else k
     if ref is None:
         raise ValueError("q and k cannot both be None")
@@ -270,9 +346,28 @@ def qk_rmsnorm_rope3d(q: Optional[torch.Tensor], k: Optional[torch.Tensor],
             raise ValueError("give grid=(T, Hg, Wg) or pos")
         T, Hg, Wg = grid
     pt, ph, pw = pairs
+    out = None
+    if q_out is not None or k_out is not None:
+        strides = None
+        for nm, t, o in (("q_out", q, q_out), ("k_out", k, k_out)):
+            if t is None:
+                continue
+            if o is None:
+                raise ValueError(f"{nm} is needed when the outputs are not in place")
+            if o.shape != (B, N, heads, hd) or o.stride(-1) != 1 or o.dtype != torch.bfloat16 \
+                    or o.device != ref.device:
+                raise ValueError(f"{nm} must be a bfloat16 [B, N, H, hd] view with unit inner "
+                                 f"stride on {ref.device}")
+            s = tuple(o.stride()[:3])
+            if strides is not None and s != strides:
+                raise ValueError("q_out and k_out must share their strides")
+            strides = s
+        out = QKOut(_ptr(q_out) if q is not None else None,
+                    _ptr(k_out) if k is not None else None, *strides)
     _call("dit_qk_rmsnorm_rope3d_ex", _ptr(q), _ptr(k), rs, _ptr(w_q), _ptr(w_k), w_dt, B, N,
           heads, hd, T, Hg, Wg, _ptr(pos), int(pos_offset), pt, ph, pw, float(theta), float(eps),
-          int(rope_layout), int(norm_width), _stream(ref))
+          int(rope_layout), int(norm_width), None if out is None else ctypes.byref(out),
+          _stream(ref))
 
 
 def cachedit_workspace_bytes(B: int, N: int, D: int) -> int:
@@ -359,3 +454,68 @@ def cachedit_residual_diff_noalloc(prev: torch.Tensor, cur: torch.Tensor, thresh
     _call("cachedit_residual_diff_noalloc", prev.data_ptr(), cur.data_ptr(), B, N, D,
           float(threshold), rel.data_ptr(), reuse.data_ptr(), _stream(prev))
     return rel, reuse
+
+
+# ------------------------------------------------------ Cache-DiT step cache
+
+
+def _elementwise(name: str, a: torch.Tensor, b: torch.Tensor, out: Optional[torch.Tensor]):
+    for nm, t in (("a", a), ("b", b)):
+        _need_cuda_bf16(nm, t)
+        if not t.is_contiguous():
+            raise ValueError(f"{name}: inputs must be contiguous")
+    if a.shape != b.shape:
+        raise ValueError(f"{name}: shapes differ")
+    out = torch.empty_like(a) if out is None else out
+    _need_cuda_bf16("out", out)
+    if out.shape != a.shape or not out.is_contiguous():
+        raise ValueError(f"{name}: out must match the inputs")
+    return out
+
+
+def cachedit_residual_store(before: torch.Tensor, after: torch.Tensor,
+                            out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """The residual blocks added: bf16(after - before), elementwise."""
+    out = _elementwise("cachedit_residual_store", before, after, out)
+    _call("cachedit_residual_store", before.data_ptr(), after.data_ptr(), out.data_ptr(),
+          before.numel(), _stream(before))
+    return out
+
+
+def cachedit_residual_apply(h: torch.Tensor, residual: torch.Tensor,
+                            out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """A reusing step: bf16(h + residual), elementwise (out may be h)."""
+    out = _elementwise("cachedit_residual_apply", h, residual, out)
+    _call("cachedit_residual_apply", h.data_ptr(), residual.data_ptr(), out.data_ptr(),
+          h.numel(), _stream(h))
+    return out
+
+
+class CachePolicy:
+    """The Cache-DiT reuse rule (dit_cache_policy in the library): call
+    decide(rel) once per denoising step; True = reuse the cached residual."""
+
+    def __init__(self, threshold: float = 0.04, warmup_steps: int = 0,
+                 max_cached_steps: int = 0):
+        self._s = CachePolicyStruct()
+        _call("dit_cache_policy_init", ctypes.byref(self._s), float(threshold),
+              int(warmup_steps), int(max_cached_steps))
+
+    def decide(self, rel: Optional[float]) -> bool:
+        r = library().dit_cache_policy_decide(ctypes.byref(self._s),
+                                             float("nan") if rel is None else float(rel))
+        if r < 0:
+            raise DitError("dit_cache_policy_decide", r, library().dit_status_string(r).decode())
+        return bool(r)
+
+    @property
+    def step(self) -> int:
+        return self._s.step
+
+    @property
+    def computed(self) -> int:
+        return self._s.computed
+
+    @property
+    def reused(self) -> int:
+        return self._s.reused

@@ -41,6 +41,10 @@ struct RowParams {
     int Dv;
     float inv_D;
     float eps;
+    const uint8_t* set_index;   // per-token modulation set, or NULL (set 0 everywhere)
+    int64_t set_stride;         // elements between the sets of one sample
+    int n_sets;
+    bool mod_vec;               // every set's vectors can be read 16 bytes at a time
 };
 
 __device__ __forceinline__ float mod_at(const void* p, int dtype, int64_t i) {
@@ -81,6 +85,60 @@ __device__ __forceinline__ void lds8(const float4* lo, const float4* hi, int v, 
     f[4] = b.x; f[5] = b.y; f[6] = b.z; f[7] = b.w;
 }
 
+// Eight modulation values at element offset off, from global memory (L1/L2
+// resident: a set is shared by many rows).  Vector loads when the host
+// found every set 16-byte aligned.
+__device__ __forceinline__ void mod8(const RowParams& p, const void* m, int64_t off,
+                                     float (&f)[8]) {
+    if (p.mod_vec) {
+        if (p.mod_dtype == DIT_F32) {
+            const float4* q = reinterpret_cast<const float4*>(static_cast<const float*>(m) + off);
+            const float4 a = __ldg(q), b = __ldg(q + 1);
+            f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w;
+            f[4] = b.x; f[5] = b.y; f[6] = b.z; f[7] = b.w;
+        } else {
+            unpack8(__ldg(reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(m) + off)),
+                    f);
+        }
+    } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) f[i] = mod_at(m, p.mod_dtype, off + i);
+    }
+}
+
+// Modulation set of token n of sample blockIdx.y (0 without an index).  An
+// index past the last set returns -1: the row's outputs are then NaN, since
+// a kernel cannot return an error to the caller.
+template <bool TOK>
+__device__ __forceinline__ int token_set(const RowParams& p, int64_t row) {
+    if (!TOK) return 0;
+    const int s = __ldg(p.set_index + row);
+    return s < p.n_sets ? s : -1;
+}
+
+// shift and 1 + scale (and gate) of vector v for a row of set `set`: set 0
+// from the shared-memory stage, other sets from global memory.
+template <bool TOK>
+__device__ __forceinline__ void modulation8(const RowParams& p, const float4* s_lo, int Dv,
+                                            int v, const void* m, int set, bool one_plus,
+                                            float (&f)[8]) {
+    if (TOK && set != 0) {
+        if (set < 0) {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) f[i] = __int_as_float(0x7fc00000);
+            return;
+        }
+        mod8(p, m, static_cast<int64_t>(blockIdx.y) * p.mod_stride + set * p.set_stride + 8 * v,
+             f);
+        if (one_plus) {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) f[i] = 1.0f + f[i];
+        }
+        return;
+    }
+    lds8(s_lo, s_lo + Dv, v, f);
+}
+
 // Stage the modulation vectors of sample blockIdx.y in shared memory:
 // shift and (1 + scale) (and gate), each as [lo Dv][hi Dv] float4 halves.
 template <bool GATED>
@@ -112,10 +170,10 @@ __device__ __forceinline__ void stage_modulation(const RowParams& p, float4* sme
 // Second half of the LayerNorm of the warp's register-resident row, given
 // the shift x0 and the warp's sum of (x - x0): the centred sum of squares,
 // then y = (x - mu) * rstd * (1 + scale) + shift.
-template <int VPL>
+template <int VPL, bool TOK>
 __device__ __forceinline__ void ln_finish_store(const RowParams& p, const float4* smem,
                                                 const uint4 (&xv)[VPL], int64_t base, int lane,
-                                                float x0, float s) {
+                                                float x0, float s, int set) {
     const int Dv = p.Dv;
     const float4* s_sh = smem;
     const float4* s_sc = smem + 2 * Dv;
@@ -142,8 +200,8 @@ __device__ __forceinline__ void ln_finish_store(const RowParams& p, const float4
         if (v < Dv) {
             float f[8], sh[8], sc[8];
             unpack8(xv[j], f);
-            lds8(s_sh, s_sh + Dv, v, sh);
-            lds8(s_sc, s_sc + Dv, v, sc);
+            modulation8<TOK>(p, s_sh, Dv, v, p.shift, set, false, sh);
+            modulation8<TOK>(p, s_sc, Dv, v, p.scale, set, true, sc);
 #pragma unroll
             for (int i = 0; i < 8; ++i) f[i] = __fmaf_rn((f[i] - mu) * rstd, sc[i], sh[i]);
             st_stream(p.y + base + v, pack8(f));
@@ -153,10 +211,10 @@ __device__ __forceinline__ void ln_finish_store(const RowParams& p, const float4
 
 // The LayerNorm of the row with the mean accumulated relative to the row's
 // first element (a shift that keeps the fp32 sum small when |mean| >> std).
-template <int VPL>
+template <int VPL, bool TOK>
 __device__ __forceinline__ void ln_modulate_store(const RowParams& p, const float4* smem,
                                                   const uint4 (&xv)[VPL], int64_t base,
-                                                  int lane) {
+                                                  int lane, int set) {
     const float x0 = __shfl_sync(0xffffffffu, bf16_lo(xv[0].x), 0);
     float s = 0.0f;
 #pragma unroll
@@ -168,12 +226,13 @@ __device__ __forceinline__ void ln_modulate_store(const RowParams& p, const floa
             for (int i = 0; i < 8; ++i) s += f[i] - x0;
         }
     }
-    ln_finish_store<VPL>(p, smem, xv, base, lane, x0, s);
+    ln_finish_store<VPL, TOK>(p, smem, xv, base, lane, x0, s, set);
 }
 
 // AdaLN: one warp per row, the row in registers (VPL vectors per lane).
-template <int VPL>
-__global__ void __launch_bounds__(kThreads)
+// TOK: modulation sets chosen per token (set 0 staged, others from L1/L2).
+template <int VPL, bool TOK>
+__global__ void __launch_bounds__(kThreads, (TOK && VPL <= 20) ? 2 : 0)
 adaln_rows_kernel(RowParams p) {
     extern __shared__ float4 smem[];
     stage_modulation<false>(p, smem, kThreads);
@@ -190,7 +249,7 @@ adaln_rows_kernel(RowParams p) {
             const int v = j * 32 + lane;
             xv[j] = (v < p.Dv) ? ld_inplace(p.x + base + v) : make_uint4(0, 0, 0, 0);
         }
-        ln_modulate_store<VPL>(p, smem, xv, base, lane);
+        ln_modulate_store<VPL, TOK>(p, smem, xv, base, lane, token_set<TOK>(p, row0 + n));
     }
 }
 
@@ -207,7 +266,7 @@ __device__ __forceinline__ void cp_async16(void* smem_dst, const void* gsrc) {
 // with cp.async, issued together with the x loads.  The two row statistics
 // are exchanged through shared memory with one named barrier per pair each;
 // both warps add the two halves in the same order, so they agree exactly.
-template <int VPL, int WARPS>
+template <int VPL, int WARPS, bool TOK>
 __global__ void __launch_bounds__(WARPS * 32, 1)
 gated_rows_kernel(RowParams p) {
     constexpr int PAIRS = WARPS / 2;
@@ -244,6 +303,7 @@ gated_rows_kernel(RowParams p) {
             const int v = 64 * j + 32 * half + lane;
             xv[j] = (v < Dv) ? ld_inplace(p.x + base + v) : make_uint4(0, 0, 0, 0);
         }
+        const int set = token_set<TOK>(p, row0 + n);
         // shift for this half's sum: the first element the warp holds (x may be
         // overwritten in place by the other warp, so each warp uses its own)
         const float x0 = __shfl_sync(0xffffffffu, bf16_lo(xv[0].x), 0);
@@ -256,7 +316,8 @@ gated_rows_kernel(RowParams p) {
             if (v < Dv) {
                 const uint4 rv = stage[j * 32 + lane];
                 float g[8];
-                lds8(s_g, s_g + Dv, v, g);
+                if (TOK) modulation8<TOK>(p, s_g, Dv, v, p.gate, set, false, g);
+                else lds8(s_g, s_g + Dv, v, g);
                 uint4 o;
                 o.x = gated_pair(xv[j].x, rv.x, g[0], g[1]);
                 o.y = gated_pair(xv[j].y, rv.y, g[2], g[3]);
@@ -306,8 +367,13 @@ gated_rows_kernel(RowParams p) {
             if (v < Dv) {
                 float f[8], sh[8], sc[8];
                 unpack8(xv[j], f);
-                lds8(s_sh, s_sh + Dv, v, sh);
-                lds8(s_sc, s_sc + Dv, v, sc);
+                if (TOK) {
+                    modulation8<TOK>(p, s_sh, Dv, v, p.shift, set, false, sh);
+                    modulation8<TOK>(p, s_sc, Dv, v, p.scale, set, true, sc);
+                } else {
+                    lds8(s_sh, s_sh + Dv, v, sh);
+                    lds8(s_sc, s_sc + Dv, v, sc);
+                }
 #pragma unroll
                 for (int i = 0; i < 8; ++i) f[i] = __fmaf_rn((f[i] - mu) * rstd, sc[i], sh[i]);
                 st_stream(p.y + base + v, pack8(f));
@@ -324,12 +390,13 @@ struct RowLaunch {
     size_t smem;
 };
 
+template <bool TOK>
 RowLaunch pick_kernel(bool gated, int Dv) {
     const size_t mod = static_cast<size_t>(gated ? 6 : 4) * Dv * sizeof(float4);
     if (!gated) {
         const int need = (Dv + 31) / 32;
 #define DIT_VPL_CASE(V) \
-    if (need <= V) return {adaln_rows_kernel<V>, kThreads, mod};
+    if (need <= V) return {adaln_rows_kernel<V, TOK>, kThreads, mod};
         DIT_VPL_CASE(1) DIT_VPL_CASE(2) DIT_VPL_CASE(3) DIT_VPL_CASE(4) DIT_VPL_CASE(6)
         DIT_VPL_CASE(8) DIT_VPL_CASE(10) DIT_VPL_CASE(12) DIT_VPL_CASE(16) DIT_VPL_CASE(20)
         DIT_VPL_CASE(24) DIT_VPL_CASE(32)
@@ -340,7 +407,7 @@ RowLaunch pick_kernel(bool gated, int Dv) {
 #define DIT_VPL_CASE(V)                                                                   \
     if (need <= V) {                                                                      \
         constexpr int WG = (V <= 10) ? 24 : 16;                                           \
-        return {gated_rows_kernel<V, WG>, WG * 32,                                        \
+        return {gated_rows_kernel<V, WG, TOK>, WG * 32,                                   \
                 mod + static_cast<size_t>(WG) * V * 32 * sizeof(uint4)};                  \
     }
     DIT_VPL_CASE(1) DIT_VPL_CASE(2) DIT_VPL_CASE(3) DIT_VPL_CASE(4) DIT_VPL_CASE(5)
@@ -350,7 +417,8 @@ RowLaunch pick_kernel(bool gated, int Dv) {
 }
 
 int launch_rows(const RowParams& p, bool gated, int B, cudaStream_t stream) {
-    const RowLaunch L = pick_kernel(gated, p.Dv);
+    const RowLaunch L = p.set_index ? pick_kernel<true>(gated, p.Dv)
+                                    : pick_kernel<false>(gated, p.Dv);
     if (!L.kernel) return DIT_ERR_SHAPE;
     // opt in whenever dynamic shared memory is used (static arrays count
     // toward the 48 KB default too)
@@ -388,15 +456,34 @@ int common_checks(int B, int64_t N, int D, int mod_dtype, int64_t mod_stride, do
     return DIT_OK;
 }
 
+// Per-token sets: the index and its set stride; whether every set's
+// vectors are 16-byte aligned for vector reads.
+int set_checks(RowParams& p, const uint8_t* set_index, int n_sets, int64_t set_stride,
+               const void* const* mods, int n_mods) {
+    if (!set_index) return DIT_ERR_NULL;
+    if (n_sets < 1 || n_sets > 255 || set_stride < 0) return DIT_ERR_SHAPE;
+    p.set_index = set_index;
+    p.n_sets = n_sets;
+    p.set_stride = set_stride;
+    const int per16 = p.mod_dtype == DIT_F32 ? 4 : 8;     // elements per 16 bytes
+    bool vec = p.mod_stride % per16 == 0 && set_stride % per16 == 0;
+    for (int i = 0; i < n_mods; ++i) vec = vec && aligned16(mods[i]);
+    p.mod_vec = vec;
+    return DIT_OK;
+}
+
 }  // namespace
 }  // namespace dit
 
-extern "C" int dit_adaln_modulate(const uint16_t* x, uint16_t* y, const void* shift,
-                                  const void* scale, int mod_dtype, int64_t mod_batch_stride,
-                                  int B, int64_t N, int D, double eps, void* stream) {
+extern "C" int dit_adaln_modulate_tok(const uint16_t* x, uint16_t* y, const void* shift,
+                                      const void* scale, int mod_dtype, int64_t mod_batch_stride,
+                                      int64_t mod_set_stride, const uint8_t* set_index,
+                                      int n_sets, int B, int64_t N, int D, double eps,
+                                      void* stream) {
     using namespace dit;
     int st = common_checks(B, N, D, mod_dtype, mod_batch_stride, eps);
     if (st) return st;
+    if (set_index && (n_sets < 1 || n_sets > 255 || mod_set_stride < 0)) return DIT_ERR_SHAPE;
     if (B == 0 || N == 0) return DIT_OK;
     if (!x || !y) return DIT_ERR_NULL;
     if ((st = check_mod(shift, mod_dtype)) || (st = check_mod(scale, mod_dtype))) return st;
@@ -414,17 +501,30 @@ extern "C" int dit_adaln_modulate(const uint16_t* x, uint16_t* y, const void* sh
     p.Dv = D / 8;
     p.inv_D = 1.0f / static_cast<float>(D);
     p.eps = static_cast<float>(eps);
+    if (set_index) {
+        const void* mods[2] = {shift, scale};
+        if ((st = set_checks(p, set_index, n_sets, mod_set_stride, mods, 2))) return st;
+    }
     return launch_rows(p, false, B, as_stream(stream));
 }
 
-extern "C" int dit_gated_residual_adaln(const uint16_t* x, const uint16_t* r, uint16_t* x_out,
-                                        uint16_t* y, const void* gate, const void* shift,
-                                        const void* scale, int mod_dtype,
-                                        int64_t mod_batch_stride, int B, int64_t N, int D,
-                                        double eps, void* stream) {
+extern "C" int dit_adaln_modulate(const uint16_t* x, uint16_t* y, const void* shift,
+                                  const void* scale, int mod_dtype, int64_t mod_batch_stride,
+                                  int B, int64_t N, int D, double eps, void* stream) {
+    return dit_adaln_modulate_tok(x, y, shift, scale, mod_dtype, mod_batch_stride, 0, nullptr,
+                                  1, B, N, D, eps, stream);
+}
+
+extern "C" int dit_gated_residual_adaln_tok(const uint16_t* x, const uint16_t* r,
+                                            uint16_t* x_out, uint16_t* y, const void* gate,
+                                            const void* shift, const void* scale, int mod_dtype,
+                                            int64_t mod_batch_stride, int64_t mod_set_stride,
+                                            const uint8_t* set_index, int n_sets, int B,
+                                            int64_t N, int D, double eps, void* stream) {
     using namespace dit;
     int st = common_checks(B, N, D, mod_dtype, mod_batch_stride, eps);
     if (st) return st;
+    if (set_index && (n_sets < 1 || n_sets > 255 || mod_set_stride < 0)) return DIT_ERR_SHAPE;
     if (B == 0 || N == 0) return DIT_OK;
     if (!x || !r || !x_out || !y) return DIT_ERR_NULL;
     if ((st = check_mod(gate, mod_dtype)) || (st = check_mod(shift, mod_dtype)) ||
@@ -451,5 +551,18 @@ extern "C" int dit_gated_residual_adaln(const uint16_t* x, const uint16_t* r, ui
     p.Dv = D / 8;
     p.inv_D = 1.0f / static_cast<float>(D);
     p.eps = static_cast<float>(eps);
+    if (set_index) {
+        const void* mods[3] = {gate, shift, scale};
+        if ((st = set_checks(p, set_index, n_sets, mod_set_stride, mods, 3))) return st;
+    }
     return launch_rows(p, true, B, as_stream(stream));
+}
+
+extern "C" int dit_gated_residual_adaln(const uint16_t* x, const uint16_t* r, uint16_t* x_out,
+                                        uint16_t* y, const void* gate, const void* shift,
+                                        const void* scale, int mod_dtype,
+                                        int64_t mod_batch_stride, int B, int64_t N, int D,
+                                        double eps, void* stream) {
+    return dit_gated_residual_adaln_tok(x, r, x_out, y, gate, shift, scale, mod_dtype,
+                                        mod_batch_stride, 0, nullptr, 1, B, N, D, eps, stream);
 }

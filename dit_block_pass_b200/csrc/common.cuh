@@ -65,6 +65,18 @@ __device__ __forceinline__ uint4 ld_inplace(const uint4* p) {
     return v;
 }
 
+// In-place data, 32 bytes: coherent, skips L1, evict-first in L2.
+__device__ __forceinline__ u32x8 ld_inplace256(const void* p) {
+    u32x8 v;
+    asm volatile(
+        "ld.global.L1::no_allocate.L2::evict_first.L2::256B.v8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, "
+        "[%8];"
+        : "=r"(v.w[0]), "=r"(v.w[1]), "=r"(v.w[2]), "=r"(v.w[3]), "=r"(v.w[4]), "=r"(v.w[5]),
+          "=r"(v.w[6]), "=r"(v.w[7])
+        : "l"(p));
+    return v;
+}
+
 // ------------------------------------------------------ bf16 conversion
 
 // bf16 -> fp32 is exact: the bf16 bits are the high half of the fp32 word.

@@ -1,44 +1,58 @@
-// qk_rope.cu -- per-head QK RMSNorm fused with 3D (t, h, w) rotary position
-// embedding, in place, in one pass over HBM.
+// qk_rope.cu -- QK RMSNorm fused with 3D (t, h, w) rotary position
+// embedding, in one pass over HBM.
 //
 // The LMSYS report summary at news.cocoloop.cn ("minimax-h3-sglang-h200"),
 // section "Só com três camadas de aceleração somadas chega-se a 6 vezes":
 // "QK RMSNorm com 3D RoPE" is one fused operator; "SGLang acelera MiniMax-H3
 // em GPUs H200", first paragraph, lists QK RMSNorm and 3D RoPE among the
-// fused low-level operations.
+// fused low-level operations.  The pages name the operator only: the pair
+// layout and the width of the norm are options here (interleaved pairs and
+// a per-head norm by default), and so is where the result goes (in place,
+// or into separate q/k buffers with any head-major or token-major layout,
+// e.g. the [B, H, N, hd] an attention kernel reads).
 //
-// Design: one warp per token, one-shot grid (a CTA of 8 warps takes 8 tokens
-// and exits; on B200 this sustained more HBM bandwidth than persistent CTAs).
-// A token row of H heads x hd is H*hd/8 consecutive 16-byte vectors; warp
-// pass j reads vectors 32*j + lane, so each load instruction covers 512
-// contiguous bytes and a head occupies hd/8 adjacent lanes.  The head's sum
-// of squares is a shuffle reduction inside that lane group.  The q row is
-// loaded into registers while the k row is copied into the warp's
-// shared-memory stage with cp.async, so both are in flight before any
-// arithmetic.  A lane always holds the same 4 rotation pairs of a head
-// (pairs 4*(lane mod hd/8) .. +3), so it computes their 4 angles once per
-// token and reuses them for every head of q and k.  The hd/2 frequencies
-// are computed in fp64 once per CTA into shared memory while the rows load;
-// the angles pos*omega are formed and reduced modulo 2*pi in fp64, and
-// sin/cos are taken in fp32 on the reduced angle, which keeps the rotation
-// accurate to a few fp32 ulp for positions in the hundreds.  The RMSNorm weight is
-// folded into the rotation coefficients once per token and tensor.  HBM
+// Design: one warp per token, one-shot grid (a CTA takes one token per warp
+// and exits; on B200 this sustained more HBM bandwidth than persistent
+// CTAs).  A token row of H heads x hd is H*hd/8 consecutive 16-byte
+// vectors; warp pass j reads vectors 32*j + lane, so each load instruction
+// covers 512 contiguous bytes and a head occupies hd/8 adjacent lanes.
+//
+// The q row is loaded into registers while the k row is copied into the
+// warp's shared-memory stage with cp.async, so both are in flight before any
+// arithmetic.  Per-head norm: the head's sum of squares is a shuffle
+// reduction inside its lane group, and the RMSNorm weight is folded into
+// per-lane rotation coefficients once per token and tensor.  Whole-row norm:
+// the row's sum of squares is a warp reduction over every vector the lane
+// holds, and the per-element weights are read through L1.
+//
+// Rotation: a lane always holds the same rotation pairs of a head (4 pairs
+// inside its vector when pairs are interleaved; 8 pairs shared with the lane
+// hd/16 away when they are (p, p + hd/2)), so it computes their angles once
+// per token and reuses them for every head of q and k.  The hd/2
+// frequencies are computed in fp64 once per CTA into shared memory while the
+// rows load; the angles pos*omega are formed and reduced modulo 2*pi in
+// fp64, and sin/cos are taken in fp32 on the reduced angle, which keeps the
+// rotation accurate to a few fp32 ulp for positions in the hundreds.  HBM
 // bound.
 #include "common.cuh"
 
 namespace dit {
 namespace {
 
-constexpr int kWarps = 8;
+constexpr int kWarps = 8;                    // tokens per CTA
 constexpr int kThreads = kWarps * 32;
 
 struct QKParams {
-    uint4* t0;              // first tensor processed (q, or k when q is NULL)
-    uint4* t1;              // second tensor or NULL
+    const uint4* t0;        // first tensor processed (q, or k when q is NULL)
+    const uint4* t1;        // second tensor or NULL
+    uint4* o0;              // where t0's result goes (t0 itself when in place)
+    uint4* o1;
     const void* w0;
     const void* w1;
     int w_dtype;
-    int64_t stride_v;       // row stride in 16-byte vectors
+    int64_t stride_v;       // input row stride in 16-byte vectors
+    int64_t osb, osn, osh;  // output strides of sample, token, head (vectors)
+    bool o_rows;            // output token rows are evenly spaced: osb == N * osn
     int64_t rows;           // B * N
     int64_t N;
     int nvr;                // vectors per tensor row = H * hd / 8
@@ -55,15 +69,6 @@ __device__ __forceinline__ float w_at(const void* p, int dtype, int i) {
     return __uint_as_float(static_cast<uint32_t>(static_cast<const uint16_t*>(p)[i]) << 16);
 }
 
-__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gsrc) {
-    const unsigned d = static_cast<unsigned>(__cvta_generic_to_shared(smem_dst));
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d), "l"(gsrc) : "memory");
-}
-
-// One warp per token (one-shot grid: a CTA takes 8 tokens and exits).  The
-// first tensor's row goes to registers and the second's to the warp's
-// shared-memory stage with cp.async, both issued before any arithmetic;
-// lane-vector j of a row is its vector j * 32 + lane.
 // Eight weights of elements e .. e+7 (fp32 or bf16; 16-byte aligned rows).
 __device__ __forceinline__ void w8_at(const void* w, int dtype, int e, float (&f)[8]) {
     if (dtype == DIT_F32) {
@@ -76,153 +81,33 @@ __device__ __forceinline__ void w8_at(const void* w, int dtype, int e, float (&f
     }
 }
 
-// Normalise and rotate one tensor row held as NVL lane-vectors v (vector
-// j * 32 + lane of the row), and store it.
-//   LAYOUT 0: pairs (2p, 2p+1) inside a lane's vector: lane pairs 4*sub + k.
-//   LAYOUT 1: pairs (p, p + hd/2): a lane's 8 elements pair with the same
-//             slots of lane ^ (hd/16) (one shuffle of the packed vector);
-//             lane pairs 8*(sub mod hd/16) + i.
-//   NORMW 0:  RMS over each head (a shuffle over its hd/8 lanes); the weight
-//             is folded into per-lane rotation coefficients.
-//   NORMW 1:  RMS over the whole row (a warp reduction); the weight has one
-//             entry per element of the row.
-template <int HD, int NVL, int LAYOUT, int NORMW>
-__device__ __forceinline__ void qk_tensor(uint4 (&v)[NVL], uint4* row, int nvr, int lane,
-                                          const void* w, int w_dtype, const float* cs,
-                                          const float* sn, float eps) {
-    constexpr int LPH = HD / 8;
-    constexpr int HALF = LPH / 2;           // partner lane distance for rotate-half
-    const int sub = lane % LPH;
-    const bool first = (sub & HALF) == 0;   // rotate-half: lane holds the first half
-    float inv_row = 0.0f;
-    if (NORMW == 1) {
-        float ss = 0.0f;
-#pragma unroll
-        for (int j = 0; j < NVL; ++j) {
-            float f[8];
-            unpack8(v[j], f);
-#pragma unroll
-            for (int i = 0; i < 8; ++i) ss = __fmaf_rn(f[i], f[i], ss);
-        }
-        ss = warp_sum(ss);
-        inv_row = rsqrtf(__fmaf_rn(ss, 1.0f / static_cast<float>(nvr * 8), eps));
-        // unpack again below rather than keep every unpacked float alive
-        // across the reduction (the packed row needs half the registers)
-#pragma unroll
-        for (int j = 0; j < NVL; ++j)
-            asm volatile("" : "+r"(v[j].x), "+r"(v[j].y), "+r"(v[j].z), "+r"(v[j].w));
-    }
-    // per-lane coefficients with the weight folded in (per-head norm)
-    float A[8], Bc[8], C[4], Dd[4];
-    if (NORMW == 0) {
-        if (LAYOUT == 0) {
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const float wa = w_at(w, w_dtype, 8 * sub + 2 * k);
-                const float wb = w_at(w, w_dtype, 8 * sub + 2 * k + 1);
-                A[k] = wa * cs[k]; Bc[k] = -(wb * sn[k]); C[k] = wa * sn[k]; Dd[k] = wb * cs[k];
-            }
-        } else {
-            // out_e = inv * (f_e w_e cos + sign * f_partner w_partner sin)
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const float wo = w_at(w, w_dtype, 8 * sub + i);
-                const float wp = w_at(w, w_dtype, 8 * (sub ^ HALF) + i);
-                A[i] = wo * cs[i];
-                Bc[i] = (first ? -wp : wp) * sn[i];
-            }
-        }
-    }
-#pragma unroll
-    for (int j = 0; j < NVL; ++j) {
-        const int idx = j * 32 + lane;
-        float f[8];
-        unpack8(v[j], f);
-        float inv = inv_row;
-        if (NORMW == 0) {
-            float ss = 0.0f;
-#pragma unroll
-            for (int i = 0; i < 8; ++i) ss = __fmaf_rn(f[i], f[i], ss);
-#pragma unroll
-            for (int o = LPH / 2; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-            inv = rsqrtf(__fmaf_rn(ss, 1.0f / static_cast<float>(HD), eps));
-        }
-        float o8[8];
-        if (LAYOUT == 0) {
-            if (NORMW == 0) {
-#pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    o8[2 * k] = inv * __fmaf_rn(f[2 * k], A[k], f[2 * k + 1] * Bc[k]);
-                    o8[2 * k + 1] = inv * __fmaf_rn(f[2 * k], C[k], f[2 * k + 1] * Dd[k]);
-                }
-            } else {
-                float wv[8];
-                w8_at(w, w_dtype, (idx < nvr ? idx : 0) * 8, wv);
-#pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    const float u0 = f[2 * k] * inv * wv[2 * k];
-                    const float u1 = f[2 * k + 1] * inv * wv[2 * k + 1];
-                    o8[2 * k] = __fmaf_rn(u0, cs[k], -u1 * sn[k]);
-                    o8[2 * k + 1] = __fmaf_rn(u0, sn[k], u1 * cs[k]);
-                }
-            }
-        } else if (NORMW == 0) {
-            uint4 pv;
-            pv.x = __shfl_xor_sync(0xffffffffu, v[j].x, HALF);
-            pv.y = __shfl_xor_sync(0xffffffffu, v[j].y, HALF);
-            pv.z = __shfl_xor_sync(0xffffffffu, v[j].z, HALF);
-            pv.w = __shfl_xor_sync(0xffffffffu, v[j].w, HALF);
-            float fp[8];
-            unpack8(pv, fp);
-#pragma unroll
-            for (int i = 0; i < 8; ++i) o8[i] = inv * __fmaf_rn(f[i], A[i], fp[i] * Bc[i]);
-        } else {
-            // weight each element on its own lane, then swap the weighted
-            // values with the partner lane
-            float wo[8];
-            w8_at(w, w_dtype, (idx < nvr ? idx : 0) * 8, wo);
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const float u = f[i] * inv * wo[i];
-                const float up = __shfl_xor_sync(0xffffffffu, u, HALF);
-                o8[i] = __fmaf_rn(u, cs[i], (first ? -up : up) * sn[i]);
-            }
-        }
-        if (idx < nvr) st_stream(row + idx, pack8(o8));
-    }
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gsrc) {
+    const unsigned d = static_cast<unsigned>(__cvta_generic_to_shared(smem_dst));
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d), "l"(gsrc) : "memory");
 }
 
-template <int HD, int NVL, int LAYOUT, int NORMW>
-__global__ void __launch_bounds__(kThreads, (NVL <= 20 ? 2 : 1))
-qk_rmsnorm_rope3d_kernel(QKParams p) {
-    constexpr int LPH = HD / 8;             // lanes per head
-    constexpr int NP = LAYOUT == 0 ? 4 : 8; // rotation pairs per lane
-    extern __shared__ uint4 qk_stage[];
-    __shared__ double s_omega[HD / 2];      // frequency of each rotation pair
-    const int lane = threadIdx.x & 31;
-    const int warp = threadIdx.x >> 5;
-    const int64_t tok = static_cast<int64_t>(blockIdx.x) * kWarps + warp;
-    const bool live = tok < p.rows;
-    const int sub = lane % LPH;             // this lane's vector within a head
-    uint4* row0 = p.t0 + tok * p.stride_v;
-    uint4* row1 = p.t1 ? p.t1 + tok * p.stride_v : nullptr;
-    uint4* stage = qk_stage + warp * (NVL * 32) + lane;
-    uint4 v[NVL];
-    if (live) {
-        if (row1) {
-#pragma unroll
-            for (int j = 0; j < NVL; ++j)
-                if (j * 32 + lane < p.nvr) cp_async16(stage + j * 32, row1 + j * 32 + lane);
-            asm volatile("cp.async.commit_group;" ::: "memory");
-        }
-#pragma unroll
-        for (int j = 0; j < NVL; ++j)
-            v[j] = (j * 32 + lane < p.nvr) ? ld_inplace(row0 + j * 32 + lane)
-                                           : make_uint4(0, 0, 0, 0);
-    }
-    // pair pr of an axis with P pairs, local index i: omega = theta^(-2i/(2P)),
-    // once per CTA while the rows are in flight
-    for (int pr = threadIdx.x; pr < HD / 2; pr += kThreads) {
+// First vector of token tok's output row: sample b = tok / N, token n.
+__device__ __forceinline__ uint4* out_row(uint4* o, const QKParams& p, int64_t tok) {
+    if (p.o_rows) return o + tok * p.osn;
+    const int64_t b = tok / p.N;
+    return o + b * p.osb + (tok - b * p.N) * p.osn;
+}
+
+// Output address of row vector idx: head idx / (hd/8), vector idx mod hd/8.
+// CONTIG: the heads of a token row are adjacent (in place, or a token-major
+// output), so the address is the row's plus idx.
+template <int HD, bool CONTIG>
+__device__ __forceinline__ uint4* out_vec(uint4* orow, int64_t osh, int idx) {
+    constexpr int LPH = HD / 8;
+    if (CONTIG) return orow + idx;
+    return orow + (idx / LPH) * osh + (idx % LPH);
+}
+
+// Pair pr of an axis with P pairs, local index i: omega = theta^(-2i/(2P)).
+// Computed once per CTA, while the rows are in flight.
+template <int HD>
+__device__ __forceinline__ void omega_table(const QKParams& p, double* s_omega) {
+    for (int pr = threadIdx.x; pr < HD / 2; pr += blockDim.x) {
         int i, P;
         if (pr < p.pt) {
             i = pr; P = p.pt;
@@ -233,10 +118,18 @@ qk_rmsnorm_rope3d_kernel(QKParams p) {
         }
         s_omega[pr] = pow(p.theta, -2.0 * static_cast<double>(i) / (2.0 * static_cast<double>(P)));
     }
-    __syncthreads();
-    if (!live) return;
+}
 
-    // token position and this lane's rotation angles
+// The token's (t, h, w) position and this lane's rotation angles:
+// LAYOUT 0 pairs 4*sub + k (k < 4), LAYOUT 1 pairs 8*(sub mod hd/16) + k
+// (k < 8), sub = the lane's vector within its head.
+template <int HD, int LAYOUT>
+__device__ __forceinline__ void token_angles(const QKParams& p, const double* s_omega,
+                                             int64_t tok, int sub,
+                                             float (&cs)[LAYOUT == 0 ? 4 : 8],
+                                             float (&sn)[LAYOUT == 0 ? 4 : 8]) {
+    constexpr int NP = LAYOUT == 0 ? 4 : 8;
+    constexpr int LPH = HD / 8;
     int pos3[3];
     if (p.pos) {
         pos3[0] = p.pos[3 * tok + 0];
@@ -255,7 +148,6 @@ qk_rmsnorm_rope3d_kernel(QKParams p) {
     }
     const double kTwoPi = 6.283185307179586;
     const double kInvTwoPi = 0.15915494309189535;
-    float cs[NP], sn[NP];
 #pragma unroll
     for (int k = 0; k < NP; ++k) {
         const int pr = LAYOUT == 0 ? 4 * sub + k : 8 * (sub % (LPH / 2)) + k;
@@ -264,59 +156,227 @@ qk_rmsnorm_rope3d_kernel(QKParams p) {
         const double kk = rint(phi * kInvTwoPi);
         sincosf(static_cast<float>(fma(-kk, kTwoPi, phi)), &sn[k], &cs[k]);
     }
-    qk_tensor<HD, NVL, LAYOUT, NORMW>(v, row0, p.nvr, lane, p.w0, p.w_dtype, cs, sn, p.eps);
+}
+
+// Per-head norm of one tensor row held as NVL lane-vectors v (vector
+// j * 32 + lane of the row), rotated and stored.
+//   LAYOUT 0: pairs (2p, 2p+1) inside a lane's vector.
+//   LAYOUT 1: pairs (p, p + hd/2): a lane's 8 elements pair with the same
+//             slots of lane ^ (hd/16), fetched with one shuffle of the
+//             packed vector.
+template <int HD, int NVL, int LAYOUT, bool CONTIG>
+__device__ __forceinline__ void qk_head_tensor(const uint4 (&v)[NVL], uint4* orow, int64_t osh,
+                                               int nvr, int lane, const void* w, int w_dtype,
+                                               const float* cs, const float* sn, float eps) {
+    constexpr int LPH = HD / 8;
+    constexpr int HALF = LPH / 2;           // partner lane distance for rotate-half
+    const int sub = lane % LPH;
+    const bool first = (sub & HALF) == 0;   // rotate-half: lane holds the first half
+    // per-lane coefficients with the weight folded in
+    float A[8], Bc[8], C[4], Dd[4];
+    if (LAYOUT == 0) {
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const float wa = w_at(w, w_dtype, 8 * sub + 2 * k);
+            const float wb = w_at(w, w_dtype, 8 * sub + 2 * k + 1);
+            A[k] = wa * cs[k]; Bc[k] = -(wb * sn[k]); C[k] = wa * sn[k]; Dd[k] = wb * cs[k];
+        }
+    } else {
+        // out_e = inv * (f_e w_e cos -/+ f_partner w_partner sin)
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const float wo = w_at(w, w_dtype, 8 * sub + i);
+            const float wp = w_at(w, w_dtype, 8 * (sub ^ HALF) + i);
+            A[i] = wo * cs[i];
+            Bc[i] = (first ? -wp : wp) * sn[i];
+        }
+    }
+#pragma unroll
+    for (int j = 0; j < NVL; ++j) {
+        const int idx = j * 32 + lane;
+        float f[8];
+        unpack8(v[j], f);
+        float ss = 0.0f;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) ss = __fmaf_rn(f[i], f[i], ss);
+#pragma unroll
+        for (int o = LPH / 2; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+        const float inv = rsqrtf(__fmaf_rn(ss, 1.0f / static_cast<float>(HD), eps));
+        float o8[8];
+        if (LAYOUT == 0) {
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                o8[2 * k] = inv * __fmaf_rn(f[2 * k], A[k], f[2 * k + 1] * Bc[k]);
+                o8[2 * k + 1] = inv * __fmaf_rn(f[2 * k], C[k], f[2 * k + 1] * Dd[k]);
+            }
+        } else {
+            uint4 pv;
+            pv.x = __shfl_xor_sync(0xffffffffu, v[j].x, HALF);
+            pv.y = __shfl_xor_sync(0xffffffffu, v[j].y, HALF);
+            pv.z = __shfl_xor_sync(0xffffffffu, v[j].z, HALF);
+            pv.w = __shfl_xor_sync(0xffffffffu, v[j].w, HALF);
+            float fp[8];
+            unpack8(pv, fp);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) o8[i] = inv * __fmaf_rn(f[i], A[i], fp[i] * Bc[i]);
+        }
+        if (idx < nvr) st_stream(out_vec<HD, CONTIG>(orow, osh, idx), pack8(o8));
+    }
+}
+
+// Whole-row norm of one tensor row held as NVL lane-vectors v: the row's
+// sum of squares first (a warp reduction), then the weighted, rotated
+// values.  The weight has one entry per element of the row.
+template <int HD, int NVL, int LAYOUT>
+__device__ __forceinline__ void qk_row_tensor(uint4 (&v)[NVL], uint4* orow, int64_t osh, int nvr,
+                                              int lane, const void* w, int w_dtype,
+                                              const float* cs, const float* sn, float eps) {
+    constexpr int LPH = HD / 8;
+    constexpr int HALF = LPH / 2;
+    const bool first = ((lane % LPH) & HALF) == 0;
+    float ss = 0.0f;
+#pragma unroll
+    for (int j = 0; j < NVL; ++j) {
+        float f[8];
+        unpack8(v[j], f);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) ss = __fmaf_rn(f[i], f[i], ss);
+    }
+    ss = warp_sum(ss);
+    const float inv = rsqrtf(__fmaf_rn(ss, 1.0f / static_cast<float>(nvr * 8), eps));
+    // unpack again below rather than keep every unpacked float alive across
+    // the reduction (the packed row needs half the registers)
+#pragma unroll
+    for (int j = 0; j < NVL; ++j)
+        asm volatile("" : "+r"(v[j].x), "+r"(v[j].y), "+r"(v[j].z), "+r"(v[j].w));
+#pragma unroll
+    for (int j = 0; j < NVL; ++j) {
+        const int idx = j * 32 + lane;
+        float f[8], wv[8], o8[8];
+        unpack8(v[j], f);
+        w8_at(w, w_dtype, (idx < nvr ? idx : 0) * 8, wv);
+        if (LAYOUT == 0) {
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const float u0 = f[2 * k] * inv * wv[2 * k];
+                const float u1 = f[2 * k + 1] * inv * wv[2 * k + 1];
+                o8[2 * k] = __fmaf_rn(u0, cs[k], -u1 * sn[k]);
+                o8[2 * k + 1] = __fmaf_rn(u0, sn[k], u1 * cs[k]);
+            }
+        } else {
+            // weight each element on its own lane, then swap the weighted
+            // values with the partner lane
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const float u = f[i] * inv * wv[i];
+                const float up = __shfl_xor_sync(0xffffffffu, u, HALF);
+                o8[i] = __fmaf_rn(u, cs[i], (first ? -up : up) * sn[i]);
+            }
+        }
+        if (idx < nvr) st_stream(out_vec<HD, false>(orow, osh, idx), pack8(o8));
+    }
+}
+
+// MODE 0: per-head norm, heads adjacent in the output; 1: per-head norm,
+// strided heads (e.g. a head-major output); 2: whole-row norm.
+template <int HD, int NVL, int LAYOUT, int MODE>
+__global__ void __launch_bounds__(kThreads, (NVL <= 20 ? 2 : 1))
+qk_rmsnorm_rope3d_kernel(QKParams p) {
+    constexpr int LPH = HD / 8;             // lanes per head
+    constexpr int NP = LAYOUT == 0 ? 4 : 8; // rotation pairs per lane
+    extern __shared__ uint4 qk_stage[];
+    __shared__ double s_omega[HD / 2];      // frequency of each rotation pair
+    const int lane = threadIdx.x & 31;
+    const int warp = threadIdx.x >> 5;
+    const int64_t tok = static_cast<int64_t>(blockIdx.x) * kWarps + warp;
+    const bool live = tok < p.rows;
+    const uint4* row0 = p.t0 + tok * p.stride_v;
+    const uint4* row1 = p.t1 ? p.t1 + tok * p.stride_v : nullptr;
+    uint4* stage = qk_stage + warp * (NVL * 32) + lane;
+    uint4 v[NVL];
+    if (live) {
+        if (row1) {
+#pragma unroll
+            for (int j = 0; j < NVL; ++j)
+                if (j * 32 + lane < p.nvr) cp_async16(stage + j * 32, row1 + j * 32 + lane);
+            asm volatile("cp.async.commit_group;" ::: "memory");
+        }
+#pragma unroll
+        for (int j = 0; j < NVL; ++j)
+            v[j] = (j * 32 + lane < p.nvr) ? ld_inplace(row0 + j * 32 + lane)
+                                           : make_uint4(0, 0, 0, 0);
+    }
+    omega_table<HD>(p, s_omega);
+    __syncthreads();
+    if (!live) return;
+
+    float cs[NP], sn[NP];
+    token_angles<HD, LAYOUT>(p, s_omega, tok, lane % LPH, cs, sn);
+    if (MODE == 2)
+        qk_row_tensor<HD, NVL, LAYOUT>(v, out_row(p.o0, p, tok), p.osh, p.nvr, lane, p.w0,
+                                       p.w_dtype, cs, sn, p.eps);
+    else
+        qk_head_tensor<HD, NVL, LAYOUT, MODE == 0>(v, out_row(p.o0, p, tok), p.osh, p.nvr, lane,
+                                                   p.w0, p.w_dtype, cs, sn, p.eps);
     if (row1) {
+        // each lane reads back only the vectors it copied itself
         asm volatile("cp.async.wait_group 0;" ::: "memory");
 #pragma unroll
         for (int j = 0; j < NVL; ++j)
             v[j] = (j * 32 + lane < p.nvr) ? stage[j * 32] : make_uint4(0, 0, 0, 0);
-        qk_tensor<HD, NVL, LAYOUT, NORMW>(v, row1, p.nvr, lane, p.w1, p.w_dtype, cs, sn, p.eps);
+        if (MODE == 2)
+            qk_row_tensor<HD, NVL, LAYOUT>(v, out_row(p.o1, p, tok), p.osh, p.nvr, lane, p.w1,
+                                           p.w_dtype, cs, sn, p.eps);
+        else
+            qk_head_tensor<HD, NVL, LAYOUT, MODE == 0>(v, out_row(p.o1, p, tok), p.osh, p.nvr,
+                                                       lane, p.w1, p.w_dtype, cs, sn, p.eps);
     }
 }
 
 using QKKernel = void (*)(QKParams);
 
-template <int HD, int LAYOUT, int NORMW>
-QKKernel pick_nvl(int nvl, int* nvl_out) {
-#define DIT_NVL_CASE(V)                                               \
-    if (nvl <= V) {                                                   \
-        *nvl_out = V;                                                 \
-        return qk_rmsnorm_rope3d_kernel<HD, V, LAYOUT, NORMW>;        \
-    }
+struct Pick {
+    QKKernel kernel = nullptr;
+    int nvl = 0;            // vectors per lane the kernel holds
+};
+
+template <int HD, int LAYOUT, int MODE>
+Pick pick_nvl(int nvl) {
+#define DIT_NVL_CASE(V) \
+    if (nvl <= V) return Pick{qk_rmsnorm_rope3d_kernel<HD, V, LAYOUT, MODE>, V};
     DIT_NVL_CASE(1) DIT_NVL_CASE(2) DIT_NVL_CASE(3) DIT_NVL_CASE(4) DIT_NVL_CASE(6)
     DIT_NVL_CASE(8) DIT_NVL_CASE(10) DIT_NVL_CASE(12) DIT_NVL_CASE(16) DIT_NVL_CASE(20)
     DIT_NVL_CASE(24) DIT_NVL_CASE(32)
 #undef DIT_NVL_CASE
-    return nullptr;
+    return Pick{};
 }
 
-template <int LAYOUT, int NORMW>
-QKKernel pick_hd(int hd, int nvl, int* nvl_out) {
+template <int LAYOUT, int MODE>
+Pick pick_hd(int hd, int nvl) {
     switch (hd) {
-        case 32: return pick_nvl<32, LAYOUT, NORMW>(nvl, nvl_out);
-        case 64: return pick_nvl<64, LAYOUT, NORMW>(nvl, nvl_out);
-        case 128: return pick_nvl<128, LAYOUT, NORMW>(nvl, nvl_out);
-        case 256: return pick_nvl<256, LAYOUT, NORMW>(nvl, nvl_out);
-        default: return nullptr;
+        case 32: return pick_nvl<32, LAYOUT, MODE>(nvl);
+        case 64: return pick_nvl<64, LAYOUT, MODE>(nvl);
+        case 128: return pick_nvl<128, LAYOUT, MODE>(nvl);
+        case 256: return pick_nvl<256, LAYOUT, MODE>(nvl);
+        default: return Pick{};
     }
 }
 
-QKKernel pick(int hd, int layout, int norm, int nvl, int* nvl_out) {
-    if (layout == DIT_ROPE_INTERLEAVED && norm == DIT_NORM_HEAD)
-        return pick_hd<DIT_ROPE_INTERLEAVED, DIT_NORM_HEAD>(hd, nvl, nvl_out);
-    if (layout == DIT_ROPE_HALF && norm == DIT_NORM_HEAD)
-        return pick_hd<DIT_ROPE_HALF, DIT_NORM_HEAD>(hd, nvl, nvl_out);
-    if (layout == DIT_ROPE_INTERLEAVED && norm == DIT_NORM_ROW)
-        return pick_hd<DIT_ROPE_INTERLEAVED, DIT_NORM_ROW>(hd, nvl, nvl_out);
-    if (layout == DIT_ROPE_HALF && norm == DIT_NORM_ROW)
-        return pick_hd<DIT_ROPE_HALF, DIT_NORM_ROW>(hd, nvl, nvl_out);
-    return nullptr;
+Pick pick(int hd, int layout, int mode, int nvl) {
+    const bool half = layout == DIT_ROPE_HALF;
+    switch (mode) {
+        case 0: return half ? pick_hd<DIT_ROPE_HALF, 0>(hd, nvl)
+                            : pick_hd<DIT_ROPE_INTERLEAVED, 0>(hd, nvl);
+        case 1: return half ? pick_hd<DIT_ROPE_HALF, 1>(hd, nvl)
+                            : pick_hd<DIT_ROPE_INTERLEAVED, 1>(hd, nvl);
+        case 2: return half ? pick_hd<DIT_ROPE_HALF, 2>(hd, nvl)
+                            : pick_hd<DIT_ROPE_INTERLEAVED, 2>(hd, nvl);
+        default: return Pick{};
+    }
 }
 
-// Rows i of q ([q + i*rs, q + i*rs + w), elements) and rows j of k overlap
-// for some 0 <= i, j < rows iff |d - m*rs| < w for an integer
-// m = i - j in (-rows, rows), d = k - q; the distance is smallest for m next
-// to d/rs, so the two integers around it (clamped to the range) decide.
+// Rows i of q and k (i < rows, `rs` elements apart, `w` wide) overlap iff
+// some row difference m in (-rows, rows) puts k within w elements of q.
 bool rows_overlap(const void* q, const void* k, int64_t rows, int64_t rs, int64_t w) {
     const intptr_t bq = reinterpret_cast<intptr_t>(q), bk = reinterpret_cast<intptr_t>(k);
     const intptr_t db = bk - bq;
@@ -340,6 +400,36 @@ int check_w(const void* p, int dtype) {
     return DIT_OK;
 }
 
+// Byte range [lo, hi) a buffer touches.
+struct Span {
+    uintptr_t lo = 0, hi = 0;
+    bool meets(const Span& o) const { return lo < o.hi && o.lo < hi; }
+};
+
+// The output layout [B, N, H, hd] with strides (sb, sn, sh, 1) must give
+// every element its own address: sorted by stride, each dimension of
+// extent > 1 must step over everything the smaller ones span.  Returns
+// the element span of one tensor, or -1.
+int64_t out_extent(int B, int64_t N, int H, int hd, int64_t sb, int64_t sn, int64_t sh) {
+    int64_t ext[3] = {B, N, H}, st[3] = {sb, sn, sh};
+    for (int a = 0; a < 3; ++a)
+        for (int b = a + 1; b < 3; ++b)
+            if (st[b] < st[a]) {
+                const int64_t e = ext[a], s = st[a];
+                ext[a] = ext[b]; st[a] = st[b];
+                ext[b] = e; st[b] = s;
+            }
+    int64_t span = hd;                     // elements covered so far
+    for (int a = 0; a < 3; ++a) {
+        if (ext[a] <= 1) continue;
+        if (st[a] < span) return -1;
+        if (st[a] > (INT64_MAX / 4) / ext[a]) return -1;
+        span = st[a] * (ext[a] - 1) + span;
+        if (span > INT64_MAX / 4) return -1;
+    }
+    return span;
+}
+
 }  // namespace
 }  // namespace dit
 
@@ -348,7 +438,8 @@ extern "C" int dit_qk_rmsnorm_rope3d_ex(uint16_t* q, uint16_t* k, int64_t row_st
                                         int64_t N, int H, int hd, int T, int Hg, int Wg,
                                         const int32_t* pos, int64_t pos_offset, int pairs_t,
                                         int pairs_h, int pairs_w, double theta, double eps,
-                                        int rope_layout, int norm_width, void* stream) {
+                                        int rope_layout, int norm_width, const dit_qk_out* out,
+                                        void* stream) {
     using namespace dit;
     if (w_dtype != DIT_F32 && w_dtype != DIT_BF16) return DIT_ERR_DTYPE;
     if (B < 0 || N < 0 || H < 1) return DIT_ERR_SHAPE;
@@ -370,6 +461,16 @@ extern "C" int dit_qk_rmsnorm_rope3d_ex(uint16_t* q, uint16_t* k, int64_t row_st
     } else if (reinterpret_cast<uintptr_t>(pos) % 4) {
         return DIT_ERR_ALIGN;
     }
+    int64_t osb = N * row_stride, osn = row_stride, osh = hd, oext = 0;
+    if (out) {
+        osb = out->stride_b;
+        osn = out->stride_n;
+        osh = out->stride_h;
+        if (osb < 0 || osn < 0 || osh < 0) return DIT_ERR_SHAPE;
+        if (osb % 8 || osn % 8 || osh % 8) return DIT_ERR_ALIGN;
+        oext = out_extent(B, N, H, hd, osb, osn, osh);
+        if (oext < 0) return DIT_ERR_SHAPE;
+    }
     if (rows == 0) return DIT_OK;
     if (!q && !k) return DIT_ERR_NULL;
     int st;
@@ -379,15 +480,49 @@ extern "C" int dit_qk_rmsnorm_rope3d_ex(uint16_t* q, uint16_t* k, int64_t row_st
     if (norm_width == DIT_NORM_ROW && ((q && !aligned16(w_q)) || (k && !aligned16(w_k))))
         return DIT_ERR_ALIGN;
     if ((q && !aligned16(q)) || (k && !aligned16(k))) return DIT_ERR_ALIGN;
-    if (q && k && rows_overlap(q, k, rows, row_stride, width)) return DIT_ERR_OVERLAP;
+    uint16_t* q_dst = q;
+    uint16_t* k_dst = k;
+    if (out) {
+        if ((q && !out->q) || (k && !out->k)) return DIT_ERR_NULL;
+        q_dst = q ? out->q : nullptr;
+        k_dst = k ? out->k : nullptr;
+        if ((q_dst && !aligned16(q_dst)) || (k_dst && !aligned16(k_dst))) return DIT_ERR_ALIGN;
+        // no output may overlap an input or the other output
+        const uintptr_t in_bytes = 2 * static_cast<uintptr_t>((rows - 1) * row_stride + width);
+        const uintptr_t out_bytes = 2 * static_cast<uintptr_t>(oext);
+        auto span = [](const void* p, uintptr_t n) {
+            Span s;
+            s.lo = reinterpret_cast<uintptr_t>(p);
+            s.hi = s.lo + n;
+            return s;
+        };
+        Span outs[2], ins[2];
+        int no = 0, ni = 0;
+        if (q) { outs[no++] = span(q_dst, out_bytes); ins[ni++] = span(q, in_bytes); }
+        if (k) { outs[no++] = span(k_dst, out_bytes); ins[ni++] = span(k, in_bytes); }
+        for (int a = 0; a < no; ++a) {
+            for (int b = 0; b < ni; ++b)
+                if (outs[a].meets(ins[b])) return DIT_ERR_OVERLAP;
+            for (int b = a + 1; b < no; ++b)
+                if (outs[a].meets(outs[b])) return DIT_ERR_OVERLAP;
+        }
+    } else if (q && k && rows_overlap(q, k, rows, row_stride, width)) {
+        return DIT_ERR_OVERLAP;
+    }
 
     QKParams p{};
-    p.t0 = reinterpret_cast<uint4*>(q ? q : k);
-    p.t1 = q ? reinterpret_cast<uint4*>(k) : nullptr;
+    p.t0 = reinterpret_cast<const uint4*>(q ? q : k);
+    p.t1 = q ? reinterpret_cast<const uint4*>(k) : nullptr;
+    p.o0 = reinterpret_cast<uint4*>(q ? q_dst : k_dst);
+    p.o1 = q ? reinterpret_cast<uint4*>(k_dst) : nullptr;
     p.w0 = q ? w_q : w_k;
     p.w1 = q ? w_k : nullptr;
     p.w_dtype = w_dtype;
     p.stride_v = row_stride / 8;
+    p.osb = osb / 8;
+    p.osn = osn / 8;
+    p.osh = osh / 8;
+    p.o_rows = osb == N * osn;
     p.rows = rows;
     p.N = N;
     p.nvr = static_cast<int>(width / 8);
@@ -401,19 +536,21 @@ extern "C" int dit_qk_rmsnorm_rope3d_ex(uint16_t* q, uint16_t* k, int64_t row_st
     p.theta = theta;
     p.eps = static_cast<float>(eps);
 
-    int nvl = 0;
-    QKKernel kernel = pick(hd, rope_layout, norm_width, (p.nvr + 31) / 32, &nvl);
-    if (!kernel) return DIT_ERR_SHAPE;
-    const size_t smem = p.t1 ? static_cast<size_t>(kWarps) * nvl * 32 * sizeof(uint4) : 0;
+    const int mode = norm_width == DIT_NORM_ROW ? 2 : (osh == hd ? 0 : 1);
+    const Pick pk = pick(hd, rope_layout, mode, (p.nvr + 31) / 32);
+    if (!pk.kernel) return DIT_ERR_SHAPE;
+    // the second tensor's stage
+    const size_t smem =
+        p.t1 ? static_cast<size_t>(kWarps) * pk.nvl * 32 * sizeof(uint4) : 0;
     // opt in whenever dynamic shared memory is used: with the static
     // frequency table the total can pass the 48 KB default
     if (smem > 0 &&
-        cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        cudaFuncSetAttribute(pk.kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(smem)) != cudaSuccess)
         return DIT_ERR_LAUNCH;
     const int64_t ctas = (rows + kWarps - 1) / kWarps;
     if (ctas > 0x7FFFFFFF) return DIT_ERR_SHAPE;
-    kernel<<<static_cast<unsigned>(ctas), kThreads, smem, as_stream(stream)>>>(p);
+    pk.kernel<<<static_cast<unsigned>(ctas), kThreads, smem, as_stream(stream)>>>(p);
     return launch_status();
 }
 
@@ -425,5 +562,5 @@ extern "C" int dit_qk_rmsnorm_rope3d(uint16_t* q, uint16_t* k, int64_t row_strid
                                      void* stream) {
     return dit_qk_rmsnorm_rope3d_ex(q, k, row_stride, w_q, w_k, w_dtype, B, N, H, hd, T, Hg, Wg,
                                     pos, pos_offset, pairs_t, pairs_h, pairs_w, theta, eps,
-                                    DIT_ROPE_INTERLEAVED, DIT_NORM_HEAD, stream);
+                                    DIT_ROPE_INTERLEAVED, DIT_NORM_HEAD, nullptr, stream);
 }

@@ -114,6 +114,36 @@ int dit_gated_residual_adaln(const uint16_t* x, const uint16_t* r,
                              int B, int64_t N, int D, double eps, void* stream);
 
 /*
+ * The two operators above with modulation chosen per token instead of per
+ * sample.  The pages name first/last-frame conditioned generation (FL2VA,
+ * H3-Base page, section "Phần nào đã được phát hành?") without saying how
+ * the conditioning frames are modulated; these entry points let a caller give
+ * such tokens modulation of their own.
+ *   set_index       device [B*N] uint8: token (b, n) uses set set_index[b*N+n].
+ *   n_sets          1..255.  A token whose index is >= n_sets gets NaN outputs
+ *                   (y, and x_out of the gated form); nothing is read for it.
+ *   mod_set_stride  elements between consecutive sets of one sample: the
+ *                   vectors of set s of sample b start at
+ *                   b*mod_batch_stride + s*mod_set_stride (e.g. [B, S, 6, D]
+ *                   modulation: mod_batch_stride = 6*S*D, mod_set_stride = 6*D).
+ * Set 0 is staged in shared memory as in the per-sample operators; other sets
+ * are read through the L1/L2 caches, so rows of set 0 run at full speed and
+ * the others somewhat slower.  set_index == NULL is the per-sample operator.
+ * Other arguments, aliasing rules and errors as above.
+ */
+int dit_adaln_modulate_tok(const uint16_t* x, uint16_t* y,
+                           const void* shift, const void* scale, int mod_dtype,
+                           int64_t mod_batch_stride, int64_t mod_set_stride,
+                           const uint8_t* set_index, int n_sets,
+                           int B, int64_t N, int D, double eps, void* stream);
+int dit_gated_residual_adaln_tok(const uint16_t* x, const uint16_t* r,
+                                 uint16_t* x_out, uint16_t* y,
+                                 const void* gate, const void* shift, const void* scale,
+                                 int mod_dtype, int64_t mod_batch_stride, int64_t mod_set_stride,
+                                 const uint8_t* set_index, int n_sets,
+                                 int B, int64_t N, int D, double eps, void* stream);
+
+/*
  * SwiGLU activation between the MLP up-projection and down-projection.
  *   out[m, j] = silu(in[m, j]) * in[m, F + j],   silu(a) = a / (1 + exp(-a))
  * (first half of each row is the gate, second half the linear branch).
@@ -161,17 +191,37 @@ enum { DIT_ROPE_INTERLEAVED = 0, DIT_ROPE_HALF = 1 };
 enum { DIT_NORM_HEAD = 0, DIT_NORM_ROW = 1 };
 
 /*
- * dit_qk_rmsnorm_rope3d with the two choices the pages leave open (the
- * "QK RMSNorm com 3D RoPE" the report names does not say which it uses):
+ * Where dit_qk_rmsnorm_rope3d_ex writes its result instead of in place: q
+ * and k outputs laid out as [B, N, H, hd] with element strides stride_b,
+ * stride_n, stride_h and hd contiguous.  Token-major separate buffers are
+ * (N*H*hd, H*hd, hd); the head-major [B, H, N, hd] that attention kernels
+ * read is (H*N*hd, hd, N*hd).  Strides are multiples of 8, the pointers
+ * 16-byte aligned, and the layout must give every element its own address
+ * (else DIT_ERR_SHAPE).  Host memory, read during the call only.
+ */
+typedef struct dit_qk_out {
+    uint16_t* q;        /* device; needed when the q input is given */
+    uint16_t* k;        /* device; needed when the k input is given */
+    int64_t stride_b, stride_n, stride_h;
+} dit_qk_out;
+
+/*
+ * dit_qk_rmsnorm_rope3d with the choices the pages leave open (the "QK
+ * RMSNorm com 3D RoPE" the report names says neither which pairs rotate
+ * nor over how many values the RMS is taken) and an output placement:
  *   rope_layout  DIT_ROPE_INTERLEAVED: rotation pairs (u_{2p}, u_{2p+1});
  *                DIT_ROPE_HALF: rotation pairs (u_p, u_{p + hd/2}).  Pair p's
  *                axis, frequency and angle are the same in both layouts.
  *   norm_width   DIT_NORM_HEAD: RMS over each head's hd values, weights [hd];
  *                DIT_NORM_ROW: RMS over the token's whole H*hd row, weights
  *                [H*hd] (then w_q and w_k must be 16-byte aligned).
+ *   out          NULL: in place, as dit_qk_rmsnorm_rope3d.  Else q and k are
+ *                only read, and the results go to out->q / out->k, which
+ *                must overlap neither input nor each other (DIT_ERR_OVERLAP);
+ *                a missing output pointer is DIT_ERR_NULL.
  * Other arguments, errors and limits as dit_qk_rmsnorm_rope3d; an unknown
  * option returns DIT_ERR_VALUE.  dit_qk_rmsnorm_rope3d is this function with
- * (DIT_ROPE_INTERLEAVED, DIT_NORM_HEAD).
+ * (DIT_ROPE_INTERLEAVED, DIT_NORM_HEAD, NULL).
  */
 int dit_qk_rmsnorm_rope3d_ex(uint16_t* q, uint16_t* k, int64_t row_stride,
                              const void* w_q, const void* w_k, int w_dtype,
@@ -179,7 +229,7 @@ int dit_qk_rmsnorm_rope3d_ex(uint16_t* q, uint16_t* k, int64_t row_stride,
                              int T, int Hg, int Wg, const int32_t* pos, int64_t pos_offset,
                              int pairs_t, int pairs_h, int pairs_w,
                              double theta, double eps, int rope_layout, int norm_width,
-                             void* stream);
+                             const dit_qk_out* out, void* stream);
 
 /*
  * Cache-DiT residual-difference check between neighbouring denoising steps.
@@ -224,6 +274,61 @@ int cachedit_residual_sums(const uint16_t* prev, const uint16_t* cur,
  */
 int cachedit_decide(const double* sums, int R, int B, double threshold,
                     double* rel_out, uint8_t* reuse_out, void* stream);
+
+/*
+ * Cache-DiT step cache.  The LMSYS report (news.cocoloop.cn,
+ * "minimax-h3-sglang-h200", section "Só com três camadas de aceleração
+ * somadas chega-se a 6 vezes") reuses results cached between neighbouring
+ * denoising steps when a residual-difference threshold allows (0.04
+ * conservative, 0.08 stride mode).  Reading: the cached result is the
+ * residual the skipped blocks add to the hidden state.  A run:
+ *   step t: h1 = first blocks(h); r1 = cachedit_residual_store(h, h1);
+ *           rel = max over samples of the relative L1 difference of r1
+ *                 against the previous step's r1 (cachedit_residual_diff);
+ *           if dit_cache_policy_decide(&policy, rel):
+ *               out = cachedit_residual_apply(h1, R)
+ *           else:
+ *               out = remaining blocks(h1); R = cachedit_residual_store(h1, out)
+ * (at step 0 rel is ignored and the step computes).
+ *
+ * cachedit_residual_store: residual[i] = bf16(after[i] - before[i]).
+ * cachedit_residual_apply: out[i] = bf16(h[i] + residual[i]).
+ * Each is the exact value rounded once to nearest-even.  Device pointers,
+ * n elements (multiple of 8, >= 0), 16-byte aligned.  The output may be one
+ * of the inputs (in place) or disjoint from both (else DIT_ERR_OVERLAP).
+ * Asynchronous on `stream`.
+ */
+int cachedit_residual_store(const uint16_t* before, const uint16_t* after, uint16_t* residual,
+                            int64_t n, void* stream);
+int cachedit_residual_apply(const uint16_t* h, const uint16_t* residual, uint16_t* out,
+                            int64_t n, void* stream);
+
+/*
+ * The reuse rule, host only.  Step t (counted by the struct) reuses iff
+ *   t >= 1, t >= warmup_steps, rel < threshold (strict; NaN never reuses),
+ *   and max_cached_steps == 0 or fewer than max_cached_steps steps in a row
+ *   reused before it.
+ * warmup_steps and max_cached_steps are guards the pages do not mention
+ * (0 = off).  Every rank that passes the same rel sequence takes the same
+ * decisions (rel from the all-gathered sums is bit-identical on all ranks).
+ * dit_cache_policy_decide returns 1 (reuse) or 0 (compute) and advances
+ * the step; a NULL struct returns DIT_ERR_NULL.  init rejects a NaN
+ * threshold or negative counts with DIT_ERR_VALUE.  Not thread-safe per
+ * struct; the caller owns the struct.
+ */
+typedef struct dit_cache_policy {
+    double threshold;
+    int warmup_steps;
+    int max_cached_steps;
+    int step;           /* next step's index */
+    int run;            /* consecutive reuses just before it */
+    int computed;       /* steps that computed so far */
+    int reused;         /* steps that reused so far */
+} dit_cache_policy;
+
+int dit_cache_policy_init(dit_cache_policy* policy, double threshold, int warmup_steps,
+                          int max_cached_steps);
+int dit_cache_policy_decide(dit_cache_policy* policy, double rel);
 
 /*
  * The Cache-DiT check of cachedit_residual_diff for callers that cannot

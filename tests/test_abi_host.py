@@ -148,9 +148,9 @@ def test_qk_argument_errors(lib):
 def test_qk_option_argument_errors(lib):
     f = lib.dit_qk_rmsnorm_rope3d_ex
     names = ["q", "k", "rs", "wq", "wk", "wdt", "B", "N", "H", "hd", "T", "Hg", "Wg", "pos",
-             "off", "pt", "ph", "pw", "theta", "eps", "layout", "norm", "s"]
+             "off", "pt", "ph", "pw", "theta", "eps", "layout", "norm", "out", "s"]
     ok = dict(zip(names, [A, A + 2 * 256, 768, A + 0x900000, A + 0x900100, 0, 1, 48, 4, 64, 2, 4,
-                          6, None, 0, 12, 10, 10, 1e4, 1e-6, 0, 0, None]))
+                          6, None, 0, 12, 10, 10, 1e4, 1e-6, 0, 0, None, None]))
 
     def call(**kw):
         a = dict(ok)
@@ -164,6 +164,19 @@ def test_qk_option_argument_errors(lib):
     assert call(norm=1, wq=None) == E["NULL"]
     assert call(hd=48, H=4, layout=1) == E["SHAPE"]
     assert call(N=0, layout=1, norm=1) == 0
+
+    # separate outputs: [B, N, H, hd] = [1, 48, 4, 64] with element strides
+    import ctypes
+    from dit_block_pass_b200 import QKOut
+    O = A + 0x1000000                                   # well clear of the inputs
+    head_major = (4 * 48 * 64, 64, 48 * 64)
+    assert call(out=ctypes.byref(QKOut(O, O + 0x100000, *head_major)), N=0) == 0
+    assert call(out=ctypes.byref(QKOut(O, None, *head_major))) == E["NULL"]
+    assert call(out=ctypes.byref(QKOut(O + 4, O + 0x100000, *head_major))) == E["ALIGN"]
+    assert call(out=ctypes.byref(QKOut(O, O + 0x100000, 4 * 48 * 64, 64, 44 * 64))) == E["SHAPE"]
+    assert call(out=ctypes.byref(QKOut(O, O + 0x100000, 4 * 48 * 64, 60, 48 * 64))) == E["ALIGN"]
+    assert call(out=ctypes.byref(QKOut(O, O + 0x100, *head_major))) == E["OVERLAP"]
+    assert call(out=ctypes.byref(QKOut(A + 0x40, O, *head_major))) == E["OVERLAP"]  # on q
 
 
 def test_cachedit_argument_errors(lib):
@@ -189,3 +202,40 @@ def test_binding_refuses_cpu_tensors():
         dbp.adaln_modulate(x, torch.zeros(1, 64), torch.zeros(1, 64))
     with pytest.raises(ValueError):
         dbp.swiglu(torch.zeros(4, 16, dtype=torch.bfloat16))
+
+
+def test_cache_policy_matches_the_rule(lib):
+    """The library's reuse rule against the oracle's, on golden and random
+    runs (host code: no GPU)."""
+    import numpy as np
+    import oracle
+    from conftest import load_golden
+    from dit_block_pass_b200 import CachePolicy
+    cases = [([float(x) for x in c["rels"]], c["threshold"], c["warmup"], c["max_cached"])
+             for c in load_golden("cache_policy.json")["cases"]]
+    rng = np.random.default_rng(11)
+    for _ in range(300):
+        cases.append((list(rng.exponential(0.05, 40)), float(rng.choice([0.04, 0.08])),
+                      int(rng.integers(0, 5)), int(rng.integers(0, 4))))
+    for rels, thr, warm, cap in cases:
+        p = CachePolicy(thr, warm, cap)
+        got = [p.decide(r) for r in rels]
+        assert got == oracle.cache_policy(rels, thr, warm, cap)
+        assert p.step == len(rels) and p.reused == sum(got) and p.computed == len(rels) - sum(got)
+
+
+def test_cache_policy_and_step_cache_errors(lib):
+    import ctypes
+    from dit_block_pass_b200 import CachePolicyStruct
+    s = CachePolicyStruct()
+    assert lib.dit_cache_policy_init(None, 0.04, 0, 0) == E["NULL"]
+    assert lib.dit_cache_policy_init(ctypes.byref(s), float("nan"), 0, 0) == E["VALUE"]
+    assert lib.dit_cache_policy_init(ctypes.byref(s), 0.04, -1, 0) == E["VALUE"]
+    assert lib.dit_cache_policy_decide(None, 0.0) == E["NULL"]
+    for f in (lib.cachedit_residual_store, lib.cachedit_residual_apply):
+        assert f(A, A + 0x10000, A + 0x20000, 0, None) == 0            # empty: no launch
+        assert f(A, A + 0x10000, A + 0x20000, -8, None) == E["SHAPE"]
+        assert f(None, A + 0x10000, A + 0x20000, 8, None) == E["NULL"]
+        assert f(A, A + 0x10000, A + 0x20000, 12, None) == E["ALIGN"]
+        assert f(A + 2, A + 0x10000, A + 0x20000, 8, None) == E["ALIGN"]
+        assert f(A, A + 0x10000, A + 16, 64, None) == E["OVERLAP"]    # partly over an input

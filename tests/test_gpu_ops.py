@@ -176,6 +176,110 @@ def test_gated_zero_gate_equals_adaln(orc):
     assert compare_bf16(bits(y), orc.bf16_to_f64(bits(y1)), "gated vs adaln", max_ulps=1.0)
 
 
+# ------------------------------------------- per-token modulation sets
+
+
+def _fl2va_index(wl, S, seed=0):
+    """Tokens of the first and last latent frames on set 1, a few random
+    tokens on the other sets, the rest on set 0."""
+    B, N = wl.B, wl.N
+    idx = np.zeros((B, N), np.uint8)
+    frame = wl.Hg * wl.Wg
+    idx[:, :frame] = 1 % S
+    idx[:, max(0, N - frame):] = 1 % S
+    rng = np.random.default_rng(seed)
+    pick = rng.random((B, N)) < 0.05
+    idx[pick] = rng.integers(0, S, pick.sum())
+    return idx
+
+
+def _set_views(base, D, pad):
+    """[B, S, D] views of the six DiT modulation vectors in a
+    [B, S, 6, D + pad] buffer (pad > 0 breaks every set's 16-byte alignment)."""
+    B, S = base.shape[:2]
+    flat = base.reshape(B, S, 6 * (D + pad))
+    return [flat[:, :, k * (D + pad):k * (D + pad) + D] for k in range(6)]
+
+
+def _set_mods(wl, S, dtype, pad=0):
+    B, D = wl.B, wl.D
+    base = W.normal(wl.seed, 90, B * S * 6, D + pad, sigma=0.1, dtype=torch.float32)
+    return base.view(B, S, 6, D + pad).to(dtype)
+
+
+TOKEN_SET_CASES = [("ragged", 3, 0), ("twosamples", 3, 0), ("wide8192", 2, 0),
+                   ("small", 4, 0), ("ragged", 3, 1)]
+
+
+@pytest.mark.parametrize("name,S,pad", TOKEN_SET_CASES)
+@pytest.mark.parametrize("mod_dtype", [torch.float32, torch.bfloat16])
+def test_token_sets(orc, name, S, pad, mod_dtype):
+    """AdaLN and the gated residual with a modulation set per token: first
+    and last frames on their own set, scattered tokens on others."""
+    wl = _adaln_wl(name)
+    B, N, D = wl.B, wl.N, wl.D
+    x = rows(wl, W.S_X, D).view(B, N, D)
+    r = rows(wl, W.S_R, D).view(B, N, D)
+    idx = _fl2va_index(wl, S)
+    base = _set_mods(wl, S, mod_dtype, pad)
+    m = [t.contiguous().double().numpy() for t in _set_views(base, D, pad)]
+    ref_y = orc.adaln_modulate_tok(bits(x), m[0], m[1], idx, wl.eps)
+    ref_xo, ref_y2 = orc.gated_residual_adaln_tok(bits(x), bits(r), m[2], m[3], m[4], idx, wl.eps)
+    vg = _set_views(base.to(DEV), D, pad)
+    idg = torch.from_numpy(idx).to(DEV)
+    xg, rg = x.to(DEV), r.to(DEV)
+    y = dbp.adaln_modulate(xg, vg[0], vg[1], wl.eps, set_index=idg)
+    xo, y2 = dbp.gated_residual_adaln(xg, rg, vg[2], vg[3], vg[4], wl.eps, set_index=idg)
+    torch.cuda.synchronize()
+    compare_bf16(bits(y), ref_y, f"adaln sets {name}")
+    assert np.array_equal(bits(xo), ref_xo), "gated x' differs"
+    compare_bf16(bits(y2), ref_y2, f"gated sets {name}")
+    # set 0 everywhere is the per-sample operator, bit for bit
+    zero = torch.zeros_like(idg)
+    y0 = dbp.adaln_modulate(xg, vg[0], vg[1], wl.eps, set_index=zero)
+    y0s = dbp.adaln_modulate(xg, vg[0][:, 0], vg[1][:, 0], wl.eps)
+    assert torch.equal(y0.view(torch.int16), y0s.view(torch.int16))
+
+
+def test_token_set_out_of_range_gives_nan(orc):
+    wl = ragged(B=2, N=40, D=512)
+    B, N, D = wl.B, wl.N, wl.D
+    x = rows(wl, W.S_X, D).view(B, N, D)
+    r = rows(wl, W.S_R, D).view(B, N, D)
+    bad = _fl2va_index(wl, 2)
+    bad[1, 7] = 2
+    bad[0, 0] = 255
+    base = _set_mods(wl, 2, torch.float32)
+    vg = _set_views(base.to(DEV), D, 0)
+    badg = torch.from_numpy(bad).to(DEV)
+    y = dbp.adaln_modulate(x.to(DEV), vg[0], vg[1], wl.eps, set_index=badg)
+    xo, y2 = dbp.gated_residual_adaln(x.to(DEV), r.to(DEV), vg[2], vg[3], vg[4], wl.eps,
+                                      set_index=badg)
+    ok = torch.ones(B, N, dtype=torch.bool)
+    ok[1, 7] = ok[0, 0] = False
+    for t in (y, xo, y2):
+        t = t.float().cpu()
+        assert torch.isnan(t[~ok]).all() and not torch.isnan(t[ok]).any()
+    m = [t.contiguous().double().numpy() for t in _set_views(base, D, 0)]
+    ref = orc.adaln_modulate_tok(bits(x), m[0], m[1], np.where(bad < 2, bad, 0).astype(np.uint8),
+                                 wl.eps)
+    compare_bf16(bits(y.cpu()[ok]), ref[ok.numpy()], "valid rows")
+
+
+def test_token_set_argument_errors():
+    x = torch.zeros(1, 4, 64, dtype=torch.bfloat16, device=DEV)
+    m = torch.zeros(1, 2, 64, device=DEV)
+    with pytest.raises(ValueError):
+        dbp.adaln_modulate(x, m, m, set_index=torch.zeros(1, 4, dtype=torch.int32, device=DEV))
+    L = dbp.library()
+    idx = torch.zeros(4, dtype=torch.uint8, device=DEV)
+    y = torch.empty_like(x)
+    for n_sets in (0, 256):
+        assert L.dit_adaln_modulate_tok(x.data_ptr(), y.data_ptr(), m.data_ptr(), m.data_ptr(),
+                                        0, 128, 64, idx.data_ptr(), n_sets, 1, 4, 64, 1e-6,
+                                        None) == -2
+
+
 # ------------------------------------------------------------------ SwiGLU
 
 
@@ -361,6 +465,36 @@ def test_qk_options_single_tensor_separate_buffers_bf16_weights(orc, layout, nor
     wl = W.CONFIGS["tiny"]
     _qk_case(orc, wl, fused=False, which="k", w_dtype=torch.bfloat16, layout=layout, norm=norm)
     _qk_case(orc, wl, fused=False, which="q", layout=layout, norm=norm, pos_mode="explicit")
+
+
+@pytest.mark.parametrize("layout,norm", [(dbp.ROPE_INTERLEAVED, dbp.NORM_HEAD)] + OPTIONS)
+@pytest.mark.parametrize("order", ["head_major", "token_major"])
+def test_qk_separate_outputs(orc, layout, norm, order):
+    """Results written to separate q/k buffers ([B, H, N, hd] for attention,
+    or [B, N, H, hd]) equal the oracle; the fused qkv input stays as it was."""
+    wl = W.Workload("o", B=2, T=3, Hg=5, Wg=7, D=3 * 128, H=3, hd=128, F=8, pairs=(22, 21, 21))
+    B, N, H, hd, D = wl.B, wl.N, wl.H, wl.hd, wl.D
+    qkv = rows(wl, W.S_QKV, 3 * D)
+    wq, wk = W.norm_weights(wl) if norm == dbp.NORM_HEAD else W.row_norm_weights(wl)
+    pos = np.tile(orc.grid_positions(wl.T, wl.Hg, wl.Wg, 0, N), (B, 1))
+    refs = [orc.qk_rmsnorm_rope3d_ex(bits(qkv[:, a * D:(a + 1) * D]), w.double().numpy(), H, hd,
+                                     pos, wl.pairs, wl.theta, wl.eps, layout=layout, norm=norm)
+            for a, w in ((0, wq), (1, wk))]
+    buf = qkv.to(DEV).view(B, N, 3 * D)
+    before = buf.clone()
+    if order == "head_major":
+        q_out = torch.full((B, H, N, hd), 7.0, dtype=torch.bfloat16, device=DEV).transpose(1, 2)
+        k_out = torch.full((B, H, N, hd), 7.0, dtype=torch.bfloat16, device=DEV).transpose(1, 2)
+    else:
+        q_out = torch.full((B, N, H, hd), 7.0, dtype=torch.bfloat16, device=DEV)
+        k_out = torch.full((B, N, H, hd), 7.0, dtype=torch.bfloat16, device=DEV)
+    dbp.qk_rmsnorm_rope3d(buf[:, :, :D], buf[:, :, D:2 * D], wq.to(DEV), wk.to(DEV), H, wl.pairs,
+                          grid=(wl.T, wl.Hg, wl.Wg), theta=wl.theta, eps=wl.eps,
+                          rope_layout=layout, norm_width=norm, q_out=q_out, k_out=k_out)
+    torch.cuda.synchronize()
+    assert torch.equal(buf.view(torch.int16), before.view(torch.int16)), "input changed"
+    for o, ref, nm in ((q_out, refs[0], "q"), (k_out, refs[1], "k")):
+        compare_bf16(bits(o.reshape(B * N, D)), ref, f"{nm} {order}")
 
 
 def test_qk_option_errors():

@@ -57,6 +57,9 @@ def _oracle_decide(orc):
     return decide_fn
 
 
+POLICY_SIGMAS = [0.02, 0.03, 0.1, 0.02, 0.03, 0.02, 0.02, 0.2, 0.01]
+
+
 def _worker(rank, world, port, mode, q):
     try:
         import sys
@@ -90,6 +93,26 @@ def _worker(rank, world, port, mode, q):
                 q.put((rank, "no error"))
             except Exception as e:          # the survivor learns of it on the host
                 q.put((rank, "error:" + type(e).__name__))
+            return
+        if mode == "policy":
+            # a run of steps: each rank decides from the all-gathered sums
+            # with the library's reuse rule (host code)
+            from dit_block_pass_b200 import CachePolicy
+            pol = CachePolicy(0.04, 0, 2)
+            decisions, rels = [], []
+            for t, sig in enumerate(POLICY_SIGMAS):
+                wt = W.Workload("shard", B=2, T=3, Hg=5, Wg=7, D=256, H=2, hd=128, F=8,
+                                pairs=(22, 21, 21), sigma_cache=(sig, sig / 2), seed=t)
+                prev, cur = (x.view(B, N, D) for x in W.cache_pair(wt))
+                rel, _ = sharding.cachedit_residual_diff_sharded(
+                    prev[:, a:b].contiguous(), cur[:, a:b].contiguous(), 0.04,
+                    sums_fn=_oracle_sums(orc), decide_fn=_oracle_decide(orc))
+                r = float(rel.max())
+                rels.append(r)
+                decisions.append(pol.decide(r if t > 0 else None))
+            q.put((rank, "policy", decisions, rels))
+            dist.barrier()
+            dist.destroy_process_group()
             return
         # Cache-DiT over shards == over the whole clip, identical on every rank
         prev, cur = (t.view(B, N, D) for t in W.cache_pair(wl))
@@ -179,3 +202,31 @@ def test_a_rank_that_leaves_before_the_exchange_is_reported():
     survivors = [o for o in out if o[0] == 0]
     assert survivors, out
     assert survivors[0][1].startswith("error:"), survivors
+
+
+def test_two_ranks_take_the_same_reuse_decisions():
+    """Over a run of steps, both ranks decide from the all-gathered sums with
+    the library's reuse rule, agree step by step, and match the oracle's rule
+    applied to the whole clip's relative differences."""
+    import oracle
+    from dit_block_pass_b200 import workloads as W
+    from parity import bits
+    out = _run(2, "policy")
+    errs = [o for o in out if o[1] == "exception"]
+    assert not errs, errs[0][2]
+    runs = [o for o in out if o[1] == "policy"]
+    assert len(runs) == 2
+    assert runs[0][2] == runs[1][2] and runs[0][3] == runs[1][3]
+    orc = oracle.default()
+    whole = []
+    for t, sig in enumerate(POLICY_SIGMAS):
+        wt = W.Workload("shard", B=2, T=3, Hg=5, Wg=7, D=256, H=2, hd=128, F=8,
+                        pairs=(22, 21, 21), sigma_cache=(sig, sig / 2), seed=t)
+        prev, cur = W.cache_pair(wt)
+        rel, _ = orc.cachedit_residual_diff(bits(prev).reshape(2, wt.N, 256),
+                                            bits(cur).reshape(2, wt.N, 256), 0.04)
+        whole.append(float(rel.max()))
+    assert np.allclose(runs[0][3], whole, rtol=1e-12, atol=0)
+    expect = oracle.cache_policy(whole, 0.04, 0, 2)
+    assert runs[0][2] == expect
+    assert any(expect) and not all(expect[1:])
