@@ -75,6 +75,10 @@ class Oracle:
                                                     _u16p, _f64p, _f64p]
         L.dito_adaln_modulate_tok.restype = _int
         L.dito_gated_residual_adaln_tok.restype = _int
+        _i64p = ctypes.POINTER(ctypes.c_int64)
+        L.dito_swiglu_gemm.argtypes = [_u16p, _u16p, _i64, _int, _int, _i64p, _i64, _f64p,
+                                       _f64p, _f64p]
+        L.dito_swiglu_gemm.restype = _int
         L.dito_residual_store.argtypes = [_u16p, _u16p, _i64, _u16p]
         L.dito_residual_apply.argtypes = [_u16p, _u16p, _i64, _u16p]
         for name in ("dito_adaln_modulate", "dito_gated_residual_adaln", "dito_swiglu",
@@ -229,6 +233,27 @@ class Oracle:
                                                   layout, norm, _p(out, _f64p), _p(work, _f64p)),
                "qk_rmsnorm_rope3d_ex")
         return out
+
+    def swiglu_gemm(self, x, w, rows=None):
+        """x: [M, K] bf16 bits, w: [2F, K] bf16 bits (gate rows, then linear
+        rows). Returns (out [R, F] fp64, g_abs, u_abs) for the rows `rows`
+        of x (all when None); g_abs / u_abs are the sums of |x w| per output."""
+        x = _c(x, np.uint16)
+        w = _c(w, np.uint16)
+        M, K = x.shape
+        F = w.shape[0] // 2
+        if w.shape != (2 * F, K):
+            raise ValueError("w must be [2F, K]")
+        r = None if rows is None else _c(rows, np.int64)
+        R = M if r is None else r.size
+        out = np.empty((R, F), dtype=np.float64)
+        ga = np.empty((R, F), dtype=np.float64)
+        ua = np.empty((R, F), dtype=np.float64)
+        _check(self.lib.dito_swiglu_gemm(
+            _p(x, _u16p), _p(w, _u16p), M, K, F,
+            None if r is None else r.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)), R,
+            _p(out, _f64p), _p(ga, _f64p), _p(ua, _f64p)), "swiglu_gemm")
+        return out, ga, ua
 
     def residual_store(self, before, after):
         """R = bf16(after - before), elementwise on bf16 bits."""

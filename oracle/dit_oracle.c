@@ -453,3 +453,50 @@ void dito_residual_apply(const uint16_t* h, const uint16_t* residual, int64_t n,
     for (int64_t i = 0; i < n; ++i)
         out[i] = dito_f64_to_bf16(dito_bf16_to_f64(h[i]) + dito_bf16_to_f64(residual[i]));
 }
+
+/* ------------------------ SwiGLU fused into the up-projection GEMM (f2) */
+
+/*
+ * out[m, j] = silu(g) * u with
+ *     g = sum_k x[m, k] * w[j, k],   u = sum_k x[m, k] * w[F + j, k]
+ * x: [M, K] bf16 (the block's normalised input), w: [2F, K] bf16 (the
+ * up-projection weight, one row per output feature: rows [0, F) the gate
+ * half, rows [F, 2F) the linear half, the order read for a3).  [REPORT]
+ * names SwiGLU among the fused operators and [CEVIU] says fusion cuts
+ * memory traffic; fusing it into the GEMM that produces its input is the
+ * reading here, with no rounding between the product and the activation.
+ * Dot products in fp64 in the order k = 0 .. K-1.  rows (n_rows entries)
+ * picks the rows of x to compute, or NULL for all M; out is [n_rows, F].
+ * g_abs / u_abs (optional) receive sum_k |x w| for each output, from which
+ * a test bounds the error of a lower-precision accumulation.
+ */
+int dito_swiglu_gemm(const uint16_t* x, const uint16_t* w, int64_t M, int K, int F,
+                     const int64_t* rows, int64_t n_rows, double* out, double* g_abs,
+                     double* u_abs)
+{
+    if (M < 0 || K <= 0 || F <= 0 || n_rows < 0) return -2;
+    if (!rows) n_rows = M;
+    for (int64_t r = 0; r < n_rows; ++r) {
+        int64_t m = rows ? rows[r] : r;
+        if (m < 0 || m >= M) return -3;
+        const uint16_t* xr = x + m * (int64_t)K;
+        for (int j = 0; j < F; ++j) {
+            const uint16_t* wg = w + (int64_t)j * K;
+            const uint16_t* wu = w + ((int64_t)F + j) * K;
+            double g = 0.0, u = 0.0, ga = 0.0, ua = 0.0;
+            for (int k = 0; k < K; ++k) {
+                double xv = dito_bf16_to_f64(xr[k]);
+                double tg = xv * dito_bf16_to_f64(wg[k]);
+                double tu = xv * dito_bf16_to_f64(wu[k]);
+                g += tg;
+                u += tu;
+                ga += fabs(tg);
+                ua += fabs(tu);
+            }
+            out[r * F + j] = g / (1.0 + exp(-g)) * u;
+            if (g_abs) g_abs[r * F + j] = ga;
+            if (u_abs) u_abs[r * F + j] = ua;
+        }
+    }
+    return 0;
+}

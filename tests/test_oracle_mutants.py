@@ -38,6 +38,14 @@ MUTANTS = {
                         "dito_f64_to_bf16(dito_bf16_to_f64(h[i]) - dito_bf16_to_f64(residual[i]))"),
     "apply_ties_away": ("dito_f64_to_bf16(dito_bf16_to_f64(h[i]) + dito_bf16_to_f64(residual[i]))",
                         "dito_f64_to_bf16(nextafter(dito_bf16_to_f64(h[i]) + dito_bf16_to_f64(residual[i]), 1e300))"),
+    "gemm_gate_reads_linear_half": ("const uint16_t* wg = w + (int64_t)j * K;",
+                                    "const uint16_t* wg = w + ((int64_t)F + j) * K;"),
+    "gemm_weight_transposed": ("double tg = xv * dito_bf16_to_f64(wg[k]);",
+                               "double tg = xv * dito_bf16_to_f64(w[(int64_t)k * 2 * F + j]);"),
+    "gemm_last_term_dropped": ("for (int k = 0; k < K; ++k) {\n                double xv",
+                               "for (int k = 0; k < K - 1; ++k) {\n                double xv"),
+    "gemm_silu_sign": ("out[r * F + j] = g / (1.0 + exp(-g)) * u;",
+                       "out[r * F + j] = g / (1.0 + exp(g)) * u;"),
     "swiglu_exp_sign": ("a / (1.0 + exp(-a))", "a / (1.0 + exp(a))"),
     "swiglu_halves_swapped": ("double a = dito_bf16_to_f64(in[m * 2 * (int64_t)F + j]);",
                               "double a = dito_bf16_to_f64(in[m * 2 * (int64_t)F + F + j]);"),
@@ -87,7 +95,7 @@ MUTANTS = {
 }
 
 PIN_MODULES = ["test_oracle_bf16", "test_oracle_adaln", "test_oracle_swiglu", "test_oracle_qk",
-               "test_oracle_cachedit", "test_oracle_cache_step"]
+               "test_oracle_cachedit", "test_oracle_cache_step", "test_oracle_swiglu_gemm"]
 
 
 def _pins():
