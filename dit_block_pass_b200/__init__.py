@@ -25,7 +25,7 @@ __all__ = [
     "DitError", "library", "library_path", "adaln_modulate", "gated_residual_adaln", "swiglu",
     "qk_rmsnorm_rope3d", "cachedit_workspace_bytes", "cachedit_residual_diff",
     "cachedit_residual_sums", "cachedit_decide", "cachedit_residual_diff_noalloc",
-    "launch_counts", "QKOut", "CachePolicy", "cachedit_residual_store",
+    "launch_counts", "QKOut", "CachePolicy", "swiglu_gemm", "cachedit_residual_store",
     "cachedit_residual_apply", "F32", "BF16", "ROPE_INTERLEAVED", "ROPE_HALF", "NORM_HEAD", "NORM_ROW",
 ]
 
@@ -44,7 +44,7 @@ launch_counts = {
     "qk_rmsnorm_rope3d_ex": 1, "adaln_modulate_tok": 1, "gated_residual_adaln_tok": 1,
     "cachedit_residual_diff": 2, "cachedit_residual_sums": 2, "cachedit_decide": 1,
     "cachedit_residual_diff_noalloc": 2, "cachedit_residual_store": 1,
-    "cachedit_residual_apply": 1,
+    "cachedit_residual_apply": 1, "swiglu_gemm": 1,
 }
 
 
@@ -102,6 +102,7 @@ def library() -> ctypes.CDLL:
                                                    i32, i32, i32, i32, vp, i64, i32, i32, i32,
                                                    dbl, dbl, i32, i32,
                                                    ctypes.POINTER(QKOut), vp]
+            L.dit_swiglu_gemm.argtypes = [vp, vp, vp, i64, i32, i32, vp, vp]
             L.cachedit_residual_store.argtypes = [vp, vp, vp, i64, vp]
             L.cachedit_residual_apply.argtypes = [vp, vp, vp, i64, vp]
             L.dit_cache_policy_init.argtypes = [ctypes.POINTER(CachePolicyStruct), dbl, i32, i32]
@@ -115,7 +116,7 @@ def library() -> ctypes.CDLL:
             L.cachedit_residual_diff_noalloc.restype = i32
             for name in ("dit_adaln_modulate", "dit_gated_residual_adaln", "dit_swiglu",
                          "dit_adaln_modulate_tok", "dit_gated_residual_adaln_tok",
-                         "cachedit_residual_store", "cachedit_residual_apply",
+                         "cachedit_residual_store", "cachedit_residual_apply", "dit_swiglu_gemm",
                          "dit_cache_policy_init", "dit_cache_policy_decide",
                          "dit_qk_rmsnorm_rope3d", "dit_qk_rmsnorm_rope3d_ex",
                          "cachedit_residual_diff",
@@ -519,3 +520,33 @@ class CachePolicy:
     @property
     def reused(self) -> int:
         return self._s.reused
+
+
+# ------------------------------------------- SwiGLU fused into the up-projection
+
+
+def swiglu_gemm(x: torch.Tensor, w: torch.Tensor, out: Optional[torch.Tensor] = None,
+                status: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """out = silu(x @ w[:F].T) * (x @ w[F:].T) on the tensor cores, the
+    [M, 2F] product never written.  x [..., K] bf16, w [2F, K] bf16 (gate
+    rows, then linear rows); returns [..., F].  ``status`` (int32 CUDA
+    scalar) is set to 1 if a wait inside the kernel expired."""
+    _need_cuda_bf16("x", x)
+    _need_cuda_bf16("w", w)
+    if not x.is_contiguous() or not w.is_contiguous() or w.dim() != 2 or w.shape[0] % 2:
+        raise ValueError("x must be contiguous [..., K] and w contiguous [2F, K]")
+    K = x.shape[-1]
+    F = w.shape[0] // 2
+    if w.shape[1] != K:
+        raise ValueError("w must be [2F, K] with the K of x")
+    M = x.numel() // max(1, K)
+    if out is None:
+        out = torch.empty(*x.shape[:-1], F, dtype=x.dtype, device=x.device)
+    _need_cuda_bf16("out", out)
+    if out.numel() != M * F or not out.is_contiguous():
+        raise ValueError("out must be contiguous [..., F]")
+    if status is not None and (status.dtype != torch.int32 or not status.is_cuda):
+        raise ValueError("status must be a CUDA int32 tensor")
+    _call("dit_swiglu_gemm", x.data_ptr(), w.data_ptr(), out.data_ptr(), M, K, F,
+          _ptr(status), _stream(x))
+    return out

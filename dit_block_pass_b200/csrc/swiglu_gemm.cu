@@ -1,0 +1,405 @@
+// swiglu_gemm.cu -- SwiGLU fused into the up-projection GEMM on the sm_100
+// tensor cores: out[m, j] = silu(x W_gate^T)[m, j] * (x W_lin^T)[m, j],
+// written once in bf16; the [M, 2F] product never reaches HBM.
+//
+// The LMSYS report summary at news.cocoloop.cn ("minimax-h3-sglang-h200"),
+// section "Só com três camadas de aceleração somadas chega-se a 6 vezes",
+// names SwiGLU among the fused operators; "SGLang acelera MiniMax-H3 em GPUs
+// H200", first paragraph, says the fusion cuts memory traffic and launches.
+// Fusing the activation into the GEMM that produces its input is the step
+// beyond the one-pass SwiGLU kernel: the 2F-wide product is consumed in the
+// accumulator.
+//
+// Design (one CTA per 128 x 128 output tile, 6 warps):
+//   warp 0   TMA producer: per 64-wide K step, one 128 x 64 tile of x and
+//            two 128 x 64 tiles of W (the gate rows n0.. and the linear rows
+//            F + n0..) land in a 4-stage shared-memory ring (128-byte
+//            swizzle), completing a transaction-count mbarrier.
+//   warp 1   allocates 256 TMEM columns and issues tcgen05.mma (kind::f16,
+//            M = 128, N = 256: gate and linear tiles side by side, K = 16 per
+//            instruction, four per stage) from one thread; tcgen05.commit
+//            frees each stage when its MMAs have read it, and signals the
+//            epilogue after the last one.
+//   warps 2-5 epilogue: tcgen05.ld pulls 32 gate and the matching 32 linear
+//            accumulators per thread (thread = output row), silu(g) * u in
+//            fp32, one rounding to bf16, 64-byte row segments to HBM.
+// The 1-D grid is rasterised in groups of 16 row tiles so that the CTAs
+// resident at one time share their x and W tiles in L2.  x, W tiles beyond
+// M, K or F are zero-filled by TMA; stores past M or F are skipped.
+//
+// Every mbarrier wait is bounded (2 s of %globaltimer); on expiry the CTA
+// records an error in the caller's status word, drains what it issued
+// (bounded as well), frees its TMEM and exits.  No cluster, no multicast.
+#include <cuda.h>
+
+#include <mutex>
+
+#include "common.cuh"
+
+namespace dit {
+namespace {
+
+constexpr int kBM = 128;                    // output rows per CTA
+constexpr int kBN = 128;                    // output columns per CTA (each half)
+constexpr int kBK = 64;                     // K per stage: one 128-byte swizzle row
+constexpr int kStages = 4;
+constexpr int kThreadsG = 192;
+constexpr int kGroupM = 16;                 // raster group (row tiles)
+constexpr uint32_t kTileA = kBM * kBK * 2;            // 16 KB
+constexpr uint32_t kTileB = 2 * kBN * kBK * 2;        // 32 KB (gate + linear)
+constexpr uint32_t kStageBytes = kTileA + kTileB;     // 48 KB
+constexpr uint32_t kTmemCols = 256;
+constexpr size_t kSmemBytes = kStages * kStageBytes + 1024 /*alignment*/ + 256 /*barriers*/;
+constexpr unsigned long long kWaitNs = 2000000000ull;
+
+// ----------------------------------------------------------- PTX helpers
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ unsigned long long now_ns() {
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Wait for the phase of `bar` with the given parity to complete, for at most
+// kWaitNs, or until another role of the CTA has given up (*abort != 0).
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort) {
+    const unsigned long long t0 = now_ns();
+    for (uint32_t i = 0;; ++i) {
+        if (mbar_try(bar, parity)) return true;
+        if ((i & 255u) == 255u) {
+            if (*abort) return false;
+            if (now_ns() - t0 > kWaitNs) return false;
+        }
+    }
+}
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, uint32_t bar,
+                                            int c0, int c1) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1)
+        : "memory");
+}
+
+// Shared-memory matrix descriptor: K-major operand, 128-byte swizzle, rows
+// of 128 bytes in groups of 8 (1024 bytes apart).  Fields: start address,
+// leading offset (16 bytes), stride offset (1024 bytes), all >> 4; version
+// 1; layout type 2 (128-byte swizzle).
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t addr) {
+    uint64_t d = static_cast<uint64_t>((addr >> 4) & 0x3FFFu);
+    d |= static_cast<uint64_t>(16u >> 4) << 16;
+    d |= static_cast<uint64_t>(1024u >> 4) << 32;
+    d |= static_cast<uint64_t>(1) << 46;
+    d |= static_cast<uint64_t>(2) << 61;
+    return d;
+}
+
+// Instruction descriptor of kind::f16: fp32 accumulator, bf16 A and B, both
+// K-major, N = 256, M = 128.
+constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((256u >> 3) << 17) |
+                            ((128u >> 4) << 24);
+
+__device__ __forceinline__ void mma_bf16(uint32_t tmem_d, uint64_t da, uint64_t db,
+                                         uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+        "l"(da), "l"(db), "r"(kIdesc), "r"(accumulate)
+        : "memory");
+}
+
+__device__ __forceinline__ void mma_commit(uint32_t bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::
+                     "r"(bar)
+                 : "memory");
+}
+
+__device__ __forceinline__ void fence_before_sync() {
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void fence_after_sync() {
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+// 32 consecutive fp32 accumulator columns of this thread's TMEM lane.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
+    uint32_t r[32];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+        "%11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, "
+        "%28, %29, %30, %31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+          "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
+          "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+          "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
+          "=r"(r[31])
+        : "r"(taddr));
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+__device__ __forceinline__ void tmem_wait_ld() {
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ float silu_mul(float g, float u) {
+    return __fdividef(g, 1.0f + __expf(-g)) * u;
+}
+
+struct GemmParams {
+    uint16_t* out;
+    int* status;            // device word, set to 1 when a wait expires (may be NULL)
+    int M, K, F;
+    int tiles_m, tiles_n;
+};
+
+__global__ void __launch_bounds__(kThreadsG, 1)
+swiglu_gemm_kernel(const __grid_constant__ CUtensorMap map_x,
+                   const __grid_constant__ CUtensorMap map_wg,
+                   const __grid_constant__ CUtensorMap map_wu, GemmParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    // 1024-byte aligned stages (the swizzle atom), barriers after them
+    const uint32_t raw = smem_u32(smem_raw);
+    const uint32_t base = (raw + 1023u) & ~1023u;
+    uint8_t* gen_base = smem_raw + (base - raw);
+    const uint32_t bar_full = base + kStages * kStageBytes;      // kStages x 8 bytes
+    const uint32_t bar_empty = bar_full + 8 * kStages;
+    const uint32_t bar_accum = bar_empty + 8 * kStages;
+    const uint32_t bar_drain = bar_accum + 8;
+    volatile uint32_t* tmem_slot =
+        reinterpret_cast<volatile uint32_t*>(gen_base + kStages * kStageBytes + 16 * kStages + 16);
+    volatile int* abort = reinterpret_cast<volatile int*>(gen_base + kStages * kStageBytes +
+                                                          16 * kStages + 20);
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+
+    // raster: groups of kGroupM row tiles, column tiles outer within a group
+    const int pid = blockIdx.x;
+    const int per_group = kGroupM * p.tiles_n;
+    const int group = pid / per_group;
+    const int first_m = group * kGroupM;
+    const int gsize = min(p.tiles_m - first_m, kGroupM);
+    const int in_group = pid - group * per_group;
+    const int tm = first_m + in_group % gsize;
+    const int tn = in_group / gsize;
+    const int m0 = tm * kBM, n0 = tn * kBN;
+    const int nk = (p.K + kBK - 1) / kBK;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(bar_full + 8 * s, 1);
+            mbar_init(bar_empty + 8 * s, 1);
+        }
+        mbar_init(bar_accum, 1);
+        mbar_init(bar_drain, 1);
+        *abort = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                         smem_u32(const_cast<uint32_t*>(tmem_slot))),
+                     "r"(kTmemCols)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    fence_before_sync();
+    __syncthreads();
+    fence_after_sync();
+    const uint32_t tmem = *tmem_slot;
+    bool failed = false;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            // producer
+            int issued = 0;
+            for (int kb = 0; kb < nk; ++kb) {
+                const int s = kb % kStages;
+                const uint32_t ph = static_cast<uint32_t>(kb / kStages) & 1u;
+                if (!mbar_wait(bar_empty + 8 * s, ph ^ 1u, abort)) {
+                    failed = true;
+                    break;
+                }
+                const uint32_t sa = base + s * kStageBytes;
+                mbar_expect_tx(bar_full + 8 * s, kStageBytes);
+                tma_load_2d(sa, &map_x, bar_full + 8 * s, kb * kBK, m0);
+                tma_load_2d(sa + kTileA, &map_wg, bar_full + 8 * s, kb * kBK, n0);
+                tma_load_2d(sa + kTileA + kTileB / 2, &map_wu, bar_full + 8 * s, kb * kBK, n0);
+                issued = kb + 1;
+            }
+            if (failed) {
+                // let the copies already issued land before the CTA exits
+                for (int kb = max(0, issued - kStages); kb < issued; ++kb)
+                    mbar_wait(bar_full + 8 * (kb % kStages),
+                              static_cast<uint32_t>(kb / kStages) & 1u, abort);
+            }
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        if (lane == 0) {
+            // MMA issuer
+            for (int kb = 0; kb < nk; ++kb) {
+                const int s = kb % kStages;
+                const uint32_t ph = static_cast<uint32_t>(kb / kStages) & 1u;
+                if (!mbar_wait(bar_full + 8 * s, ph, abort)) {
+                    failed = true;
+                    break;
+                }
+                fence_after_sync();
+                const uint32_t sa = base + s * kStageBytes;
+                const uint32_t sb = sa + kTileA;
+#pragma unroll
+                for (int kk = 0; kk < kBK / 16; ++kk)
+                    mma_bf16(tmem, sw128_desc(sa + kk * 32), sw128_desc(sb + kk * 32),
+                             (kb | kk) != 0 ? 1u : 0u);
+                mma_commit(bar_empty + 8 * s);      // stage free once these MMAs read it
+            }
+            // the accumulator is complete (or, after a failure, every MMA
+            // issued has finished) when this commit arrives
+            mma_commit(failed ? bar_drain : bar_accum);
+            if (failed) mbar_wait(bar_drain, 0, abort);
+        }
+        __syncwarp();
+    } else {
+        // epilogue: warp w reads TMEM lanes 32 * (w % 4) .. + 31
+        const int q = warp & 3;
+        const int row = m0 + 32 * q + lane;
+        if (!mbar_wait(bar_accum, 0, abort)) {
+            failed = true;
+        } else {
+            fence_after_sync();
+            const uint32_t lane_addr = tmem + (static_cast<uint32_t>(32 * q) << 16);
+#pragma unroll 1
+            for (int c = 0; c < kBN / 32; ++c) {
+                float g[32], u[32];
+                tmem_ld32(lane_addr + 32 * c, g);
+                tmem_ld32(lane_addr + kBN + 32 * c, u);
+                tmem_wait_ld();
+                if (row < p.M) {
+                    uint16_t* dst = p.out + static_cast<int64_t>(row) * p.F + n0 + 32 * c;
+#pragma unroll
+                    for (int v = 0; v < 4; ++v) {
+                        if (n0 + 32 * c + 8 * v < p.F) {
+                            float o[8];
+#pragma unroll
+                            for (int i = 0; i < 8; ++i) o[i] = silu_mul(g[8 * v + i], u[8 * v + i]);
+                            *reinterpret_cast<uint4*>(dst + 8 * v) = pack8(o);
+                        }
+                    }
+                }
+            }
+        }
+    }
+    if (failed) {
+        *abort = 1;
+        if (p.status) atomicExch(p.status, 1);
+    }
+    fence_before_sync();
+    __syncthreads();
+    fence_after_sync();
+    if (warp == 1)
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
+                     "r"(kTmemCols)
+                     : "memory");
+}
+
+// ------------------------------------------------------------------ host
+
+using EncodeTiled = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                 const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                 const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                 CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiled encoder() {
+    static std::once_flag once;
+    static EncodeTiled fn = nullptr;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiled>(p);
+    });
+    return fn;
+}
+
+// A [rows, K] bf16 row-major operand read in 64 x 128 boxes, 128-byte swizzle.
+bool make_map(CUtensorMap* map, const void* base, int64_t rows, int K) {
+    const EncodeTiled enc = encoder();
+    if (!enc) return false;
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(rows)};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(K) * 2};
+    const cuuint32_t box[2] = {kBK, 128};
+    const cuuint32_t elem[2] = {1, 1};
+    return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+               box, elem, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+}  // namespace dit
+
+extern "C" int dit_swiglu_gemm(const uint16_t* x, const uint16_t* w, uint16_t* out, int64_t M,
+                               int K, int F, int* status, void* stream) {
+    using namespace dit;
+    if (M < 0 || K <= 0 || F <= 0) return DIT_ERR_SHAPE;
+    if (K % 8 || F % 8) return DIT_ERR_ALIGN;
+    if (M > 0x7FFFFFFFLL - kBM || F > (1 << 30) / 2) return DIT_ERR_SHAPE;
+    if (M == 0) return DIT_OK;
+    if (!x || !w || !out) return DIT_ERR_NULL;
+    if (!aligned16(x) || !aligned16(w) || !aligned16(out)) return DIT_ERR_ALIGN;
+    if (status && reinterpret_cast<uintptr_t>(status) % 4) return DIT_ERR_ALIGN;
+    const size_t out_bytes = static_cast<size_t>(M) * F * 2;
+    if (overlaps(out, out_bytes, x, static_cast<size_t>(M) * K * 2) ||
+        overlaps(out, out_bytes, w, static_cast<size_t>(2) * F * K * 2))
+        return DIT_ERR_OVERLAP;
+    CUtensorMap mx, mg, mu;
+    const uint16_t* w_lin = w + static_cast<int64_t>(F) * K;
+    if (!make_map(&mx, x, M, K) || !make_map(&mg, w, F, K) || !make_map(&mu, w_lin, F, K))
+        return DIT_ERR_LAUNCH;
+    GemmParams p{};
+    p.out = out;
+    p.status = status;
+    p.M = static_cast<int>(M);
+    p.K = K;
+    p.F = F;
+    p.tiles_m = static_cast<int>((M + kBM - 1) / kBM);
+    p.tiles_n = (F + kBN - 1) / kBN;
+    const int64_t ctas = static_cast<int64_t>(p.tiles_m) * p.tiles_n;
+    if (ctas > 0x7FFFFFFF) return DIT_ERR_SHAPE;
+    if (cudaFuncSetAttribute(swiglu_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(kSmemBytes)) != cudaSuccess)
+        return DIT_ERR_LAUNCH;
+    swiglu_gemm_kernel<<<static_cast<unsigned>(ctas), kThreadsG, kSmemBytes, as_stream(stream)>>>(
+        mx, mg, mu, p);
+    return launch_status();
+}

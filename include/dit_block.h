@@ -276,6 +276,27 @@ int cachedit_decide(const double* sums, int R, int B, double threshold,
                     double* rel_out, uint8_t* reuse_out, void* stream);
 
 /*
+ * SwiGLU fused into the up-projection GEMM (tensor cores, sm_100):
+ *     out[m, j] = silu(g) * u,  g = sum_k x[m, k] w[j, k],
+ *                               u = sum_k x[m, k] w[F + j, k]
+ * The LMSYS report (news.cocoloop.cn, "minimax-h3-sglang-h200", section "Só
+ * com três camadas de aceleração somadas chega-se a 6 vezes") names SwiGLU
+ * among the fused operators; here it is fused into the GEMM that produces
+ * its input, so the [M, 2F] product is never written.
+ *   x    device [M, K] bf16, row-major (token-major activations).
+ *   w    device [2F, K] bf16, one row per output feature (the usual linear
+ *        weight layout): rows [0, F) the gate half, [F, 2F) the linear half.
+ *   out  device [M, F] bf16; must not overlap x or w.
+ * K and F multiples of 8; pointers 16-byte aligned.  Products accumulate in
+ * fp32 in the tensor memory; silu(g) * u is formed in fp32 and rounded once
+ * to bf16.  status (optional device int, 4-byte aligned) is set to 1 if a
+ * pipeline wait inside the kernel ran out (a defect, never expected): the
+ * output is then incomplete.  The caller clears it.
+ */
+int dit_swiglu_gemm(const uint16_t* x, const uint16_t* w, uint16_t* out, int64_t M, int K, int F,
+                    int* status, void* stream);
+
+/*
  * Cache-DiT step cache.  The LMSYS report (news.cocoloop.cn,
  * "minimax-h3-sglang-h200", section "Só com três camadas de aceleração
  * somadas chega-se a 6 vezes") reuses results cached between neighbouring

@@ -239,3 +239,16 @@ def test_cache_policy_and_step_cache_errors(lib):
         assert f(A, A + 0x10000, A + 0x20000, 12, None) == E["ALIGN"]
         assert f(A + 2, A + 0x10000, A + 0x20000, 8, None) == E["ALIGN"]
         assert f(A, A + 0x10000, A + 16, 64, None) == E["OVERLAP"]    # partly over an input
+
+
+def test_swiglu_gemm_argument_errors(lib):
+    f = lib.dit_swiglu_gemm
+    assert f(A, A + 0x100000, A + 0x200000, 0, 64, 64, None, None) == 0      # empty M
+    assert f(A, A + 0x100000, A + 0x200000, -1, 64, 64, None, None) == E["SHAPE"]
+    assert f(A, A + 0x100000, A + 0x200000, 4, 0, 64, None, None) == E["SHAPE"]
+    assert f(A, A + 0x100000, A + 0x200000, 4, 60, 64, None, None) == E["ALIGN"]
+    assert f(A, A + 0x100000, A + 0x200000, 4, 64, 12, None, None) == E["ALIGN"]
+    assert f(None, A + 0x100000, A + 0x200000, 4, 64, 64, None, None) == E["NULL"]
+    assert f(A + 8, A + 0x100000, A + 0x200000, 4, 64, 64, None, None) == E["ALIGN"]
+    assert f(A, A + 0x100000, A + 0x200000, 4, 64, 64, A + 2, None) == E["ALIGN"]
+    assert f(A, A + 0x100000, A + 0x100, 4, 64, 64, None, None) == E["OVERLAP"]   # over x
