@@ -10,22 +10,29 @@
 // beyond the one-pass SwiGLU kernel: the 2F-wide product is consumed in the
 // accumulator.
 //
-// Design (one CTA per 128 x 128 output tile, 6 warps):
+// Design: persistent, one CTA of 6 warps per SM, 128 x 128 output tiles
+// taken in a static round robin:
 //   warp 0   TMA producer: per 64-wide K step, one 128 x 64 tile of x and
 //            two 128 x 64 tiles of W (the gate rows n0.. and the linear rows
 //            F + n0..) land in a 4-stage shared-memory ring (128-byte
-//            swizzle), completing a transaction-count mbarrier.
-//   warp 1   allocates 256 TMEM columns and issues tcgen05.mma (kind::f16,
-//            M = 128, N = 256: gate and linear tiles side by side, K = 16 per
-//            instruction, four per stage) from one thread; tcgen05.commit
-//            frees each stage when its MMAs have read it, and signals the
-//            epilogue after the last one.
+//            swizzle), completing a transaction-count mbarrier.  The ring
+//            runs on across tiles.
+//   warp 1   allocates all 512 TMEM columns (two 256-column accumulators)
+//            and issues tcgen05.mma (kind::f16, M = 128, N = 256: gate and
+//            linear tiles side by side, K = 16 per instruction, four per
+//            stage) from one thread; tcgen05.commit frees each stage when
+//            its MMAs have read it and hands a finished accumulator to the
+//            epilogue.
 //   warps 2-5 epilogue: tcgen05.ld pulls 32 gate and the matching 32 linear
 //            accumulators per thread (thread = output row), silu(g) * u in
-//            fp32, one rounding to bf16, 64-byte row segments to HBM.
-// The 1-D grid is rasterised in groups of 16 row tiles so that the CTAs
-// resident at one time share their x and W tiles in L2.  x, W tiles beyond
-// M, K or F are zero-filled by TMA; stores past M or F are skipped.
+//            fp32, one rounding to bf16, 64-byte row segments to HBM.  Once
+//            the last columns are in registers the accumulator goes back to
+//            the MMA warp, so one tile's epilogue overlaps the next tile's
+//            main loop.
+// Tiles are numbered in groups of 16 row tiles (column tiles outer within a
+// group) so that the tiles in flight share their x and W tiles in L2.  x, W
+// tiles beyond M, K or F are zero-filled by TMA; stores past M or F are
+// skipped.
 //
 // Every mbarrier wait is bounded (2 s of %globaltimer); on expiry the CTA
 // records an error in the caller's status word, drains what it issued
@@ -48,7 +55,7 @@ constexpr int kGroupM = 16;                 // raster group (row tiles)
 constexpr uint32_t kTileA = kBM * kBK * 2;            // 16 KB
 constexpr uint32_t kTileB = 2 * kBN * kBK * 2;        // 32 KB (gate + linear)
 constexpr uint32_t kStageBytes = kTileA + kTileB;     // 48 KB
-constexpr uint32_t kTmemCols = 256;
+constexpr uint32_t kTmemCols = 512;                   // two 256-column accumulators
 constexpr size_t kSmemBytes = kStages * kStageBytes + 1024 /*alignment*/ + 256 /*barriers*/;
 constexpr unsigned long long kWaitNs = 2000000000ull;
 
@@ -178,9 +185,25 @@ struct GemmParams {
     uint16_t* out;
     int* status;            // device word, set to 1 when a wait expires (may be NULL)
     int M, K, F;
-    int tiles_m, tiles_n;
+    int tiles_m, tiles_n, tiles;
 };
 
+// Output tile of linear tile id t: groups of kGroupM row tiles, the column
+// tiles outer within a group, so that the tiles in flight at one time share
+// their x and W tiles in L2.
+__device__ __forceinline__ void tile_coords(const GemmParams& p, int t, int& m0, int& n0) {
+    const int per_group = kGroupM * p.tiles_n;
+    const int group = t / per_group;
+    const int first_m = group * kGroupM;
+    const int gsize = min(p.tiles_m - first_m, kGroupM);
+    const int in_group = t - group * per_group;
+    m0 = (first_m + in_group % gsize) * kBM;
+    n0 = (in_group / gsize) * kBN;
+}
+
+// Persistent: CTA b takes tiles b, b + gridDim.x, ...  The K-step ring and
+// the two accumulators (TMEM columns [0, 256) and [256, 512)) run across
+// tiles, so the epilogue of one tile overlaps the main loop of the next.
 __global__ void __launch_bounds__(kThreadsG, 1)
 swiglu_gemm_kernel(const __grid_constant__ CUtensorMap map_x,
                    const __grid_constant__ CUtensorMap map_wg,
@@ -191,26 +214,15 @@ swiglu_gemm_kernel(const __grid_constant__ CUtensorMap map_x,
     const uint32_t base = (raw + 1023u) & ~1023u;
     uint8_t* gen_base = smem_raw + (base - raw);
     const uint32_t bar_full = base + kStages * kStageBytes;      // kStages x 8 bytes
-    const uint32_t bar_empty = bar_full + 8 * kStages;
-    const uint32_t bar_accum = bar_empty + 8 * kStages;
-    const uint32_t bar_drain = bar_accum + 8;
-    volatile uint32_t* tmem_slot =
-        reinterpret_cast<volatile uint32_t*>(gen_base + kStages * kStageBytes + 16 * kStages + 16);
-    volatile int* abort = reinterpret_cast<volatile int*>(gen_base + kStages * kStageBytes +
-                                                          16 * kStages + 20);
+    const uint32_t bar_empty = bar_full + 8 * kStages;           // kStages x 8 bytes
+    const uint32_t bar_tfull = bar_empty + 8 * kStages;          // 2 x 8: accumulator ready
+    const uint32_t bar_tempty = bar_tfull + 16;                  // 2 x 8: accumulator drained
+    const uint32_t bar_drain = bar_tempty + 16;
+    uint8_t* tail = gen_base + kStages * kStageBytes + 16 * kStages + 40;
+    volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(tail);
+    volatile int* abort = reinterpret_cast<volatile int*>(tail + 4);
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-
-    // raster: groups of kGroupM row tiles, column tiles outer within a group
-    const int pid = blockIdx.x;
-    const int per_group = kGroupM * p.tiles_n;
-    const int group = pid / per_group;
-    const int first_m = group * kGroupM;
-    const int gsize = min(p.tiles_m - first_m, kGroupM);
-    const int in_group = pid - group * per_group;
-    const int tm = first_m + in_group % gsize;
-    const int tn = in_group / gsize;
-    const int m0 = tm * kBM, n0 = tn * kBN;
     const int nk = (p.K + kBK - 1) / kBK;
 
     if (threadIdx.x == 0) {
@@ -218,7 +230,10 @@ swiglu_gemm_kernel(const __grid_constant__ CUtensorMap map_x,
             mbar_init(bar_full + 8 * s, 1);
             mbar_init(bar_empty + 8 * s, 1);
         }
-        mbar_init(bar_accum, 1);
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(bar_tfull + 8 * a, 1);
+            mbar_init(bar_tempty + 8 * a, 4);      // one arrival per epilogue warp
+        }
         mbar_init(bar_drain, 1);
         *abort = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -238,70 +253,102 @@ swiglu_gemm_kernel(const __grid_constant__ CUtensorMap map_x,
 
     if (warp == 0) {
         if (lane == 0) {
-            // producer
-            int issued = 0;
-            for (int kb = 0; kb < nk; ++kb) {
-                const int s = kb % kStages;
-                const uint32_t ph = static_cast<uint32_t>(kb / kStages) & 1u;
-                if (!mbar_wait(bar_empty + 8 * s, ph ^ 1u, abort)) {
-                    failed = true;
-                    break;
+            // producer: K steps of every tile, through the ring
+            uint32_t it = 0;
+            for (int t = blockIdx.x; t < p.tiles && !failed; t += gridDim.x) {
+                int m0, n0;
+                tile_coords(p, t, m0, n0);
+                for (int kb = 0; kb < nk; ++kb, ++it) {
+                    const uint32_t s = it % kStages;
+                    const uint32_t ph = (it / kStages) & 1u;
+                    if (!mbar_wait(bar_empty + 8 * s, ph ^ 1u, abort)) {
+                        failed = true;
+                        break;
+                    }
+                    const uint32_t sa = base + s * kStageBytes;
+                    mbar_expect_tx(bar_full + 8 * s, kStageBytes);
+                    tma_load_2d(sa, &map_x, bar_full + 8 * s, kb * kBK, m0);
+                    tma_load_2d(sa + kTileA, &map_wg, bar_full + 8 * s, kb * kBK, n0);
+                    tma_load_2d(sa + kTileA + kTileB / 2, &map_wu, bar_full + 8 * s, kb * kBK,
+                                n0);
                 }
-                const uint32_t sa = base + s * kStageBytes;
-                mbar_expect_tx(bar_full + 8 * s, kStageBytes);
-                tma_load_2d(sa, &map_x, bar_full + 8 * s, kb * kBK, m0);
-                tma_load_2d(sa + kTileA, &map_wg, bar_full + 8 * s, kb * kBK, n0);
-                tma_load_2d(sa + kTileA + kTileB / 2, &map_wu, bar_full + 8 * s, kb * kBK, n0);
-                issued = kb + 1;
             }
             if (failed) {
                 // let the copies already issued land before the CTA exits
-                for (int kb = max(0, issued - kStages); kb < issued; ++kb)
-                    mbar_wait(bar_full + 8 * (kb % kStages),
-                              static_cast<uint32_t>(kb / kStages) & 1u, abort);
+                for (uint32_t j = it > kStages ? it - kStages : 0; j < it; ++j)
+                    mbar_wait(bar_full + 8 * (j % kStages), (j / kStages) & 1u, abort);
             }
         }
         __syncwarp();
     } else if (warp == 1) {
         if (lane == 0) {
             // MMA issuer
-            for (int kb = 0; kb < nk; ++kb) {
-                const int s = kb % kStages;
-                const uint32_t ph = static_cast<uint32_t>(kb / kStages) & 1u;
-                if (!mbar_wait(bar_full + 8 * s, ph, abort)) {
+            uint32_t it = 0, local = 0;
+            for (int t = blockIdx.x; t < p.tiles && !failed; t += gridDim.x, ++local) {
+                const uint32_t acc = local & 1u;
+                const uint32_t aph = (local >> 1) & 1u;
+                // the epilogue has drained this accumulator (the first two pass)
+                if (!mbar_wait(bar_tempty + 8 * acc, aph ^ 1u, abort)) {
                     failed = true;
                     break;
                 }
                 fence_after_sync();
-                const uint32_t sa = base + s * kStageBytes;
-                const uint32_t sb = sa + kTileA;
+                const uint32_t d = tmem + acc * 256u;
+                for (int kb = 0; kb < nk; ++kb, ++it) {
+                    const uint32_t s = it % kStages;
+                    const uint32_t ph = (it / kStages) & 1u;
+                    if (!mbar_wait(bar_full + 8 * s, ph, abort)) {
+                        failed = true;
+                        break;
+                    }
+                    fence_after_sync();
+                    const uint32_t sa = base + s * kStageBytes;
+                    const uint32_t sb = sa + kTileA;
 #pragma unroll
-                for (int kk = 0; kk < kBK / 16; ++kk)
-                    mma_bf16(tmem, sw128_desc(sa + kk * 32), sw128_desc(sb + kk * 32),
-                             (kb | kk) != 0 ? 1u : 0u);
-                mma_commit(bar_empty + 8 * s);      // stage free once these MMAs read it
+                    for (int kk = 0; kk < kBK / 16; ++kk)
+                        mma_bf16(d, sw128_desc(sa + kk * 32), sw128_desc(sb + kk * 32),
+                                 (kb | kk) != 0 ? 1u : 0u);
+                    mma_commit(bar_empty + 8 * s);  // stage free once these MMAs read it
+                }
+                if (!failed) mma_commit(bar_tfull + 8 * acc);
             }
-            // the accumulator is complete (or, after a failure, every MMA
-            // issued has finished) when this commit arrives
-            mma_commit(failed ? bar_drain : bar_accum);
-            if (failed) mbar_wait(bar_drain, 0, abort);
+            if (failed) {
+                // every MMA issued has finished when this commit arrives
+                mma_commit(bar_drain);
+                mbar_wait(bar_drain, 0, abort);
+            }
         }
         __syncwarp();
     } else {
         // epilogue: warp w reads TMEM lanes 32 * (w % 4) .. + 31
         const int q = warp & 3;
-        const int row = m0 + 32 * q + lane;
-        if (!mbar_wait(bar_accum, 0, abort)) {
-            failed = true;
-        } else {
+        uint32_t local = 0;
+        for (int t = blockIdx.x; t < p.tiles; t += gridDim.x, ++local) {
+            int m0, n0;
+            tile_coords(p, t, m0, n0);
+            const uint32_t acc = local & 1u;
+            if (!mbar_wait(bar_tfull + 8 * acc, (local >> 1) & 1u, abort)) {
+                failed = true;
+                break;
+            }
             fence_after_sync();
-            const uint32_t lane_addr = tmem + (static_cast<uint32_t>(32 * q) << 16);
+            const int row = m0 + 32 * q + lane;
+            const uint32_t lane_addr = tmem + acc * 256u + (static_cast<uint32_t>(32 * q) << 16);
 #pragma unroll 1
             for (int c = 0; c < kBN / 32; ++c) {
                 float g[32], u[32];
                 tmem_ld32(lane_addr + 32 * c, g);
                 tmem_ld32(lane_addr + kBN + 32 * c, u);
                 tmem_wait_ld();
+                if (c == kBN / 32 - 1) {
+                    // every column of this accumulator is in registers: hand it back
+                    fence_before_sync();
+                    __syncwarp();
+                    if (lane == 0)
+                        asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(
+                                         bar_tempty + 8 * acc)
+                                     : "memory");
+                }
                 if (row < p.M) {
                     uint16_t* dst = p.out + static_cast<int64_t>(row) * p.F + n0 + 32 * c;
 #pragma unroll
@@ -394,8 +441,12 @@ extern "C" int dit_swiglu_gemm(const uint16_t* x, const uint16_t* w, uint16_t* o
     p.F = F;
     p.tiles_m = static_cast<int>((M + kBM - 1) / kBM);
     p.tiles_n = (F + kBN - 1) / kBN;
-    const int64_t ctas = static_cast<int64_t>(p.tiles_m) * p.tiles_n;
-    if (ctas > 0x7FFFFFFF) return DIT_ERR_SHAPE;
+    const int64_t tiles = static_cast<int64_t>(p.tiles_m) * p.tiles_n;
+    if (tiles > 0x7FFFFFFF) return DIT_ERR_SHAPE;
+    p.tiles = static_cast<int>(tiles);
+    const int sms = device_sm_count();
+    if (sms <= 0) return DIT_ERR_LAUNCH;
+    const int64_t ctas = tiles < sms ? tiles : sms;     // one persistent CTA per SM
     if (cudaFuncSetAttribute(swiglu_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(kSmemBytes)) != cudaSuccess)
         return DIT_ERR_LAUNCH;
