@@ -46,16 +46,19 @@
 namespace dit {
 namespace {
 
-constexpr int kBM = 128;                    // output rows per CTA
-constexpr int kBN = 128;                    // output columns per CTA (each half)
+constexpr int kHalves = 2;                  // 128-row MMAs per tile (sharing the W tile)
+constexpr int kBM = 128 * kHalves;          // output rows per tile
+constexpr int kBN = 128;                    // output columns per tile (each W half)
 constexpr int kBK = 64;                     // K per stage: one 128-byte swizzle row
-constexpr int kStages = 4;
+constexpr int kStages = kHalves == 2 ? 3 : 4;
 constexpr int kThreadsG = 192;
-constexpr int kGroupM = 16;                 // raster group (row tiles)
-constexpr uint32_t kTileA = kBM * kBK * 2;            // 16 KB
+constexpr int kGroupM = 16 / kHalves;       // raster group (row tiles)
+constexpr uint32_t kTileA = kBM * kBK * 2;            // 16 KB per 128 rows
 constexpr uint32_t kTileB = 2 * kBN * kBK * 2;        // 32 KB (gate + linear)
-constexpr uint32_t kStageBytes = kTileA + kTileB;     // 48 KB
-constexpr uint32_t kTmemCols = 512;                   // two 256-column accumulators
+constexpr uint32_t kStageBytes = kTileA + kTileB;
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kAccCols = 256 * kHalves;          // accumulator columns per tile
+constexpr uint32_t kAccBufs = kTmemCols / kAccCols;   // tiles in TMEM at once
 constexpr size_t kSmemBytes = kStages * kStageBytes + 1024 /*alignment*/ + 256 /*barriers*/;
 constexpr unsigned long long kWaitNs = 2000000000ull;
 
@@ -230,7 +233,7 @@ swiglu_gemm_kernel(const __grid_constant__ CUtensorMap map_x,
             mbar_init(bar_full + 8 * s, 1);
             mbar_init(bar_empty + 8 * s, 1);
         }
-        for (int a = 0; a < 2; ++a) {
+        for (uint32_t a = 0; a < kAccBufs; ++a) {
             mbar_init(bar_tfull + 8 * a, 1);
             mbar_init(bar_tempty + 8 * a, 4);      // one arrival per epilogue warp
         }
@@ -267,7 +270,10 @@ swiglu_gemm_kernel(const __grid_constant__ CUtensorMap map_x,
                     }
                     const uint32_t sa = base + s * kStageBytes;
                     mbar_expect_tx(bar_full + 8 * s, kStageBytes);
-                    tma_load_2d(sa, &map_x, bar_full + 8 * s, kb * kBK, m0);
+#pragma unroll
+                    for (int h = 0; h < kHalves; ++h)
+                        tma_load_2d(sa + h * (kTileA / kHalves), &map_x, bar_full + 8 * s,
+                                    kb * kBK, m0 + 128 * h);
                     tma_load_2d(sa + kTileA, &map_wg, bar_full + 8 * s, kb * kBK, n0);
                     tma_load_2d(sa + kTileA + kTileB / 2, &map_wu, bar_full + 8 * s, kb * kBK,
                                 n0);
@@ -285,15 +291,15 @@ swiglu_gemm_kernel(const __grid_constant__ CUtensorMap map_x,
             // MMA issuer
             uint32_t it = 0, local = 0;
             for (int t = blockIdx.x; t < p.tiles && !failed; t += gridDim.x, ++local) {
-                const uint32_t acc = local & 1u;
-                const uint32_t aph = (local >> 1) & 1u;
-                // the epilogue has drained this accumulator (the first two pass)
+                const uint32_t acc = local % kAccBufs;
+                const uint32_t aph = (local / kAccBufs) & 1u;
+                // the epilogue has drained this accumulator (the first use passes)
                 if (!mbar_wait(bar_tempty + 8 * acc, aph ^ 1u, abort)) {
                     failed = true;
                     break;
                 }
                 fence_after_sync();
-                const uint32_t d = tmem + acc * 256u;
+                const uint32_t d = tmem + acc * kAccCols;
                 for (int kb = 0; kb < nk; ++kb, ++it) {
                     const uint32_t s = it % kStages;
                     const uint32_t ph = (it / kStages) & 1u;
@@ -306,8 +312,10 @@ swiglu_gemm_kernel(const __grid_constant__ CUtensorMap map_x,
                     const uint32_t sb = sa + kTileA;
 #pragma unroll
                     for (int kk = 0; kk < kBK / 16; ++kk)
-                        mma_bf16(d, sw128_desc(sa + kk * 32), sw128_desc(sb + kk * 32),
-                                 (kb | kk) != 0 ? 1u : 0u);
+#pragma unroll
+                        for (int h = 0; h < kHalves; ++h)
+                            mma_bf16(d + 256u * h, sw128_desc(sa + h * (kTileA / kHalves) + kk * 32),
+                                     sw128_desc(sb + kk * 32), (kb | kk) != 0 ? 1u : 0u);
                     mma_commit(bar_empty + 8 * s);  // stage free once these MMAs read it
                 }
                 if (!failed) mma_commit(bar_tfull + 8 * acc);
@@ -326,21 +334,23 @@ swiglu_gemm_kernel(const __grid_constant__ CUtensorMap map_x,
         for (int t = blockIdx.x; t < p.tiles; t += gridDim.x, ++local) {
             int m0, n0;
             tile_coords(p, t, m0, n0);
-            const uint32_t acc = local & 1u;
-            if (!mbar_wait(bar_tfull + 8 * acc, (local >> 1) & 1u, abort)) {
+            const uint32_t acc = local % kAccBufs;
+            if (!mbar_wait(bar_tfull + 8 * acc, (local / kAccBufs) & 1u, abort)) {
                 failed = true;
                 break;
             }
             fence_after_sync();
-            const int row = m0 + 32 * q + lane;
-            const uint32_t lane_addr = tmem + acc * 256u + (static_cast<uint32_t>(32 * q) << 16);
 #pragma unroll 1
-            for (int c = 0; c < kBN / 32; ++c) {
+            for (int hc = 0; hc < kHalves * (kBN / 32); ++hc) {
+                const int h = hc / (kBN / 32), c = hc % (kBN / 32);
+                const int row = m0 + 128 * h + 32 * q + lane;
+                const uint32_t lane_addr =
+                    tmem + acc * kAccCols + 256u * h + (static_cast<uint32_t>(32 * q) << 16);
                 float g[32], u[32];
                 tmem_ld32(lane_addr + 32 * c, g);
                 tmem_ld32(lane_addr + kBN + 32 * c, u);
                 tmem_wait_ld();
-                if (c == kBN / 32 - 1) {
+                if (hc == kHalves * (kBN / 32) - 1) {
                     // every column of this accumulator is in registers: hand it back
                     fence_before_sync();
                     __syncwarp();
