@@ -365,6 +365,51 @@ def time_cache_step(chain, steps, warmup, world):
     return out
 
 
+def time_swiglu_gemm(chain, steps, warmup, world):
+    """The up-projection with SwiGLU fused into its epilogue (tcgen05) on the
+    clip's normalised tokens, against the unfused chain it replaces: cuBLAS's
+    bf16 GEMM into [M, 2F], then the one-pass SwiGLU.  Returns ms per launch
+    of both; inputs are larger than L2."""
+    import torch
+    import dit_block_pass_b200 as dbp
+    from dit_block_pass_b200 import workloads as W
+    c, wl = chain, chain.wl
+    M, K, F = wl.M, wl.D, wl.F
+    w = W.normal(wl.seed, 91, 2 * F, K, sigma=K ** -0.5, device=c.dev)
+    x = c.y1.view(M, K)
+    y = c.swi.view(M, 2 * F)
+    st = torch.zeros(1, dtype=torch.int32, device=c.dev)
+    ops = {"fused": lambda: dbp.swiglu_gemm(x, w, out=c.out, status=st),
+           "unfused": lambda: (torch.matmul(x, w.T, out=y), dbp.swiglu(y, out=c.out))}
+    stream = torch.cuda.current_stream()
+    out = {}
+    for name, op in ops.items():
+        for _ in range(warmup):
+            op()
+        barrier_sync(world)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(steps):
+            op()
+        b.record(stream)
+        barrier_sync(world)
+        out[name] = a.elapsed_time(b) / steps
+    if int(st.item()) != 0:
+        raise RuntimeError("swiglu_gemm reported an expired pipeline wait")
+    del w
+    return out
+
+
+def tensor_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["bf16_tflops"]), float(d["bf16_tflops_sustained"]), "measured"
+    except Exception:
+        return 1590.0, 1400.0, "fallback"
+
+
 def time_e2e(chain, steps, warmup, world):
     """The same chain through the public API with inputs on the host: every
     step copies its inputs host->device from pinned memory, runs the chain and
@@ -534,6 +579,8 @@ def main():
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--config", default="h3_5s")
     ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--gemm-steps", type=int, default=10,
+                    help="timed launches of the fused up-projection and of its unfused chain")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
@@ -565,6 +612,7 @@ def main():
         qk_opt = time_qk_options(chain, args.steps, args.warmup, world)
         tok_sets, tok_share = time_token_sets(chain, args.steps, args.warmup, world)
         step_cache = time_cache_step(chain, args.steps, args.warmup, world)
+        gemm_ms = time_swiglu_gemm(chain, args.gemm_steps, 2, world)
     finally:
         if sampler:
             sampler.__exit__(None, None, None)
@@ -599,6 +647,19 @@ def main():
         gbs = 6 * wl.M * wl.D / (ms / 1000.0) / 1e9        # read two, write one
         cache_step[name] = {"ms": round(ms, 4), "GB/s": round(gbs, 1),
                             "frac_of_peak": round(gbs / peak, 4)}
+    burst, sustained, tkind = tensor_peaks()
+    gflop = 2.0 * wl.M * wl.D * 2 * wl.F / 1e9
+    fused_ms = max_over_ranks(gemm_ms["fused"], world)
+    unfused_ms = max_over_ranks(gemm_ms["unfused"], world)
+    tflops = gflop / fused_ms
+    swiglu_gemm = {"kernel": "swiglu_gemm_kernel (tcgen05)", "ms": round(fused_ms, 3),
+                   "TFLOP/s": round(tflops, 1), "bound": "tensor",
+                   "frac_of_burst_peak": round(tflops / burst, 4),
+                   "frac_of_sustained_peak": round(tflops / sustained, 4),
+                   "peak_source": f"{tkind} bf16_tflops {burst} / sustained {sustained}",
+                   "unfused_ms (cuBLAS bf16 GEMM + swiglu_kernel)": round(unfused_ms, 3),
+                   "speedup_vs_unfused": round(unfused_ms / fused_ms, 4),
+                   "shape": f"[{wl.M}, {wl.D}] x [{2 * wl.F}, {wl.D}]^T -> [{wl.M}, {wl.F}]"}
     dom_ms = per_op[OPS.index(DOMINANT)]
     achieved = nbytes[DOMINANT] / (dom_ms / 1000.0) / 1e9
     tr = NCU_TRAFFIC.get(DOMINANT)
@@ -638,7 +699,7 @@ def main():
                        "l2": "every input is larger than L2 (126 MB); no flush",
                        "parallelism": f"{world} independent clip(s), one per GPU"},
             "ops": ops, "qk_options": qk_options, "token_sets": token_sets,
-            "cache_step": cache_step,
+            "cache_step": cache_step, "swiglu_gemm": swiglu_gemm,
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": chain.launches_per_step() * args.steps, "clocks": clocks,
         }

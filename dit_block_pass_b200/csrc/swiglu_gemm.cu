@@ -10,29 +10,32 @@
 // beyond the one-pass SwiGLU kernel: the 2F-wide product is consumed in the
 // accumulator.
 //
-// Design: persistent, one CTA of 6 warps per SM, 128 x 128 output tiles
-// taken in a static round robin:
-//   warp 0   TMA producer: per 64-wide K step, one 128 x 64 tile of x and
-//            two 128 x 64 tiles of W (the gate rows n0.. and the linear rows
-//            F + n0..) land in a 4-stage shared-memory ring (128-byte
-//            swizzle), completing a transaction-count mbarrier.  The ring
-//            runs on across tiles.
-//   warp 1   allocates all 512 TMEM columns (two 256-column accumulators)
-//            and issues tcgen05.mma (kind::f16, M = 128, N = 256: gate and
-//            linear tiles side by side, K = 16 per instruction, four per
-//            stage) from one thread; tcgen05.commit frees each stage when
-//            its MMAs have read it and hands a finished accumulator to the
+// Design: persistent, one CTA of 6 warps per SM, output tiles of 256 rows x
+// 128 columns taken in a static round robin:
+//   warp 0   TMA producer: per 64-wide K step, two 128 x 64 tiles of x (rows
+//            m0.. and m0 + 128..) and two 128 x 64 tiles of W (the gate rows
+//            n0.. and the linear rows F + n0..) land in a 3-stage ring of
+//            64 KB stages (128-byte swizzle), completing a transaction-count
+//            mbarrier.  The ring runs on across tiles.
+//   warp 1   allocates all 512 TMEM columns and issues tcgen05.mma from one
+//            thread: kind::f16, M = 128, N = 256 (gate and linear tiles side
+//            by side), K = 16, two MMAs per K slice (one per 128-row half,
+//            both reading the same W tile: 131 flop per staged byte), four
+//            slices per stage.  tcgen05.commit frees each stage when its
+//            MMAs have read it and hands the finished accumulators to the
 //            epilogue.
 //   warps 2-5 epilogue: tcgen05.ld pulls 32 gate and the matching 32 linear
 //            accumulators per thread (thread = output row), silu(g) * u in
 //            fp32, one rounding to bf16, 64-byte row segments to HBM.  Once
-//            the last columns are in registers the accumulator goes back to
-//            the MMA warp, so one tile's epilogue overlaps the next tile's
-//            main loop.
-// Tiles are numbered in groups of 16 row tiles (column tiles outer within a
+//            the last columns are in registers the accumulators go back to
+//            the MMA warp; the producer has meanwhile filled the ring for
+//            the next tile.
+// Tiles are numbered in groups of 8 row tiles (column tiles outer within a
 // group) so that the tiles in flight share their x and W tiles in L2.  x, W
 // tiles beyond M, K or F are zero-filled by TMA; stores past M or F are
-// skipped.
+// skipped.  Measured on B200 at the sustained tensor peak (the tile shape,
+// the raster group, the epilogue width and streaming stores all measured
+// within noise of each other there).
 //
 // Every mbarrier wait is bounded (2 s of %globaltimer); on expiry the CTA
 // records an error in the caller's status word, drains what it issued
