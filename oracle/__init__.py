@@ -79,6 +79,9 @@ class Oracle:
         L.dito_swiglu_gemm.argtypes = [_u16p, _u16p, _i64, _int, _int, _i64p, _i64, _f64p,
                                        _f64p, _f64p]
         L.dito_swiglu_gemm.restype = _int
+        L.dito_gemm_gated_residual.argtypes = [_u16p, _u16p, _u16p, _f64p, _i64, _i64, _i64,
+                                               _int, _int, _i64p, _i64, _u16p, _f64p, _f64p]
+        L.dito_gemm_gated_residual.restype = _int
         L.dito_residual_store.argtypes = [_u16p, _u16p, _i64, _u16p]
         L.dito_residual_apply.argtypes = [_u16p, _u16p, _i64, _u16p]
         for name in ("dito_adaln_modulate", "dito_gated_residual_adaln", "dito_swiglu",
@@ -254,6 +257,30 @@ class Oracle:
             None if r is None else r.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)), R,
             _p(out, _f64p), _p(ga, _f64p), _p(ua, _f64p)), "swiglu_gemm")
         return out, ga, ua
+
+    def gemm_gated_residual(self, h, w, x, gate, N, rows=None):
+        """h: [M, K] bf16 bits, w: [D, K] bf16 bits, x: [M, D] bf16 bits,
+        gate: [B, D] (B = M / N samples of N token rows).  Returns
+        (x_out [R, D] bf16 bits, dot [R, D] fp64, abs_dot [R, D] fp64) for the
+        rows `rows` (all when None)."""
+        h = _c(h, np.uint16)
+        w = _c(w, np.uint16)
+        x = _c(x, np.uint16)
+        M, K = h.shape
+        D = w.shape[0]
+        if w.shape != (D, K) or x.shape != (M, D):
+            raise ValueError("shapes do not match")
+        gate = _c(gate, np.float64).reshape(-1, D)
+        r = None if rows is None else _c(rows, np.int64)
+        R = M if r is None else r.size
+        out = np.empty((R, D), dtype=np.uint16)
+        dot = np.empty((R, D), dtype=np.float64)
+        ad = np.empty((R, D), dtype=np.float64)
+        _check(self.lib.dito_gemm_gated_residual(
+            _p(h, _u16p), _p(w, _u16p), _p(x, _u16p), _p(gate, _f64p), D, M, N, K, D,
+            None if r is None else r.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)), R,
+            _p(out, _u16p), _p(dot, _f64p), _p(ad, _f64p)), "gemm_gated_residual")
+        return out, dot, ad
 
     def residual_store(self, before, after):
         """R = bf16(after - before), elementwise on bf16 bits."""

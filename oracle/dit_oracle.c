@@ -500,3 +500,48 @@ int dito_swiglu_gemm(const uint16_t* x, const uint16_t* w, int64_t M, int K, int
     }
     return 0;
 }
+
+/* ---------------- gated residual fused into the down-projection GEMM (f2) */
+
+/*
+ * x_out[m, n] = bf16(x[m, n] + gate_b[n] * sum_k h[m, k] * w[n, k])
+ * h: [M, K] bf16 (the block's MLP activations), w: [D, K] bf16 (the
+ * projection weight, one row per output feature), x: [M, D] bf16 (the
+ * residual stream), gate: [B, D] (sample b = m / N of token row m, vectors
+ * mod_batch_stride apart).  This is a2's residual update with its branch
+ * r = h w^T taken straight from the product: [REPORT] names the gated
+ * residual among the fused operators, and the fused form must give what the
+ * unfused chain gives up to the rounding of r, which the fusion removes.
+ * The dot product is summed in fp64 in the order k = 0 .. K-1 (the products
+ * of two bf16 values are exact), then x + gate * dot in fp64 is rounded once
+ * to bf16.  rows (n_rows entries) picks the token rows, or NULL for all M;
+ * x_out is [n_rows, D] and dot (optional) receives the fp64 dot products,
+ * abs_dot (optional) sum_k |h w| for each output.
+ */
+int dito_gemm_gated_residual(const uint16_t* h, const uint16_t* w, const uint16_t* x,
+                             const double* gate, int64_t mod_batch_stride, int64_t M,
+                             int64_t N, int K, int D, const int64_t* rows, int64_t n_rows,
+                             uint16_t* x_out, double* dot, double* abs_dot)
+{
+    if (M < 0 || N <= 0 || K <= 0 || D <= 0 || n_rows < 0 || M % N) return -2;
+    if (!rows) n_rows = M;
+    for (int64_t r = 0; r < n_rows; ++r) {
+        int64_t m = rows ? rows[r] : r;
+        if (m < 0 || m >= M) return -3;
+        const double* g = gate + (m / N) * mod_batch_stride;
+        const uint16_t* hr = h + m * (int64_t)K;
+        for (int n = 0; n < D; ++n) {
+            const uint16_t* wn = w + (int64_t)n * K;
+            double s = 0.0, a = 0.0;
+            for (int k = 0; k < K; ++k) {
+                double t = dito_bf16_to_f64(hr[k]) * dito_bf16_to_f64(wn[k]);
+                s += t;
+                a += fabs(t);
+            }
+            x_out[r * D + n] = dito_f64_to_bf16(dito_bf16_to_f64(x[m * (int64_t)D + n]) + g[n] * s);
+            if (dot) dot[r * D + n] = s;
+            if (abs_dot) abs_dot[r * D + n] = a;
+        }
+    }
+    return 0;
+}

@@ -46,6 +46,12 @@ MUTANTS = {
                                "for (int k = 0; k < K - 1; ++k) {\n                double xv"),
     "gemm_silu_sign": ("out[r * F + j] = g / (1.0 + exp(-g)) * u;",
                        "out[r * F + j] = g / (1.0 + exp(g)) * u;"),
+    "down_gate_by_row": ("const double* g = gate + (m / N) * mod_batch_stride;",
+                         "const double* g = gate + (m % N) * mod_batch_stride;"),
+    "down_weight_column": ("const uint16_t* wn = w + (int64_t)n * K;",
+                           "const uint16_t* wn = w + (int64_t)n;"),
+    "down_gate_added": ("dito_bf16_to_f64(x[m * (int64_t)D + n]) + g[n] * s);",
+                        "dito_bf16_to_f64(x[m * (int64_t)D + n]) + g[n] + s);"),
     "swiglu_exp_sign": ("a / (1.0 + exp(-a))", "a / (1.0 + exp(a))"),
     "swiglu_halves_swapped": ("double a = dito_bf16_to_f64(in[m * 2 * (int64_t)F + j]);",
                               "double a = dito_bf16_to_f64(in[m * 2 * (int64_t)F + F + j]);"),
@@ -95,7 +101,8 @@ MUTANTS = {
 }
 
 PIN_MODULES = ["test_oracle_bf16", "test_oracle_adaln", "test_oracle_swiglu", "test_oracle_qk",
-               "test_oracle_cachedit", "test_oracle_cache_step", "test_oracle_swiglu_gemm"]
+               "test_oracle_cachedit", "test_oracle_cache_step", "test_oracle_swiglu_gemm",
+               "test_oracle_gemm_residual"]
 
 
 def _pins():
