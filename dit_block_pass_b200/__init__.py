@@ -25,7 +25,7 @@ __all__ = [
     "DitError", "library", "library_path", "adaln_modulate", "gated_residual_adaln", "swiglu",
     "qk_rmsnorm_rope3d", "cachedit_workspace_bytes", "cachedit_residual_diff",
     "cachedit_residual_sums", "cachedit_decide", "cachedit_residual_diff_noalloc",
-    "launch_counts", "QKOut", "CachePolicy", "swiglu_gemm", "cachedit_residual_store",
+    "launch_counts", "QKOut", "CachePolicy", "swiglu_gemm", "gemm_gated_residual", "cachedit_residual_store",
     "cachedit_residual_apply", "F32", "BF16", "ROPE_INTERLEAVED", "ROPE_HALF", "NORM_HEAD", "NORM_ROW",
 ]
 
@@ -44,7 +44,7 @@ launch_counts = {
     "qk_rmsnorm_rope3d_ex": 1, "adaln_modulate_tok": 1, "gated_residual_adaln_tok": 1,
     "cachedit_residual_diff": 2, "cachedit_residual_sums": 2, "cachedit_decide": 1,
     "cachedit_residual_diff_noalloc": 2, "cachedit_residual_store": 1,
-    "cachedit_residual_apply": 1, "swiglu_gemm": 1,
+    "cachedit_residual_apply": 1, "swiglu_gemm": 1, "gemm_gated_residual": 1,
 }
 
 
@@ -103,6 +103,8 @@ def library() -> ctypes.CDLL:
                                                    dbl, dbl, i32, i32,
                                                    ctypes.POINTER(QKOut), vp]
             L.dit_swiglu_gemm.argtypes = [vp, vp, vp, i64, i32, i32, vp, vp]
+            L.dit_gemm_gated_residual.argtypes = [vp, vp, vp, vp, vp, i32, i64, i32, i64, i32,
+                                                  i32, vp, vp]
             L.cachedit_residual_store.argtypes = [vp, vp, vp, i64, vp]
             L.cachedit_residual_apply.argtypes = [vp, vp, vp, i64, vp]
             L.dit_cache_policy_init.argtypes = [ctypes.POINTER(CachePolicyStruct), dbl, i32, i32]
@@ -117,6 +119,7 @@ def library() -> ctypes.CDLL:
             for name in ("dit_adaln_modulate", "dit_gated_residual_adaln", "dit_swiglu",
                          "dit_adaln_modulate_tok", "dit_gated_residual_adaln_tok",
                          "cachedit_residual_store", "cachedit_residual_apply", "dit_swiglu_gemm",
+                         "dit_gemm_gated_residual",
                          "dit_cache_policy_init", "dit_cache_policy_decide",
                          "dit_qk_rmsnorm_rope3d", "dit_qk_rmsnorm_rope3d_ex",
                          "cachedit_residual_diff",
@@ -550,3 +553,31 @@ def swiglu_gemm(x: torch.Tensor, w: torch.Tensor, out: Optional[torch.Tensor] = 
     _call("dit_swiglu_gemm", x.data_ptr(), w.data_ptr(), out.data_ptr(), M, K, F,
           _ptr(status), _stream(x))
     return out
+
+
+def gemm_gated_residual(h: torch.Tensor, w: torch.Tensor, x: torch.Tensor, gate: torch.Tensor,
+                        x_out: Optional[torch.Tensor] = None,
+                        status: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """x' = bf16(x + gate_b * (h @ w.T)) on the tensor cores.  h [B, N, K],
+    w [D, K], x [B, N, D] bf16; gate [B, D] or [D] (fp32 or bf16, unit inner
+    stride).  x_out may be x.  Returns x'."""
+    for nm, t in (("h", h), ("w", w), ("x", x)):
+        _need_cuda_bf16(nm, t)
+        if not t.is_contiguous():
+            raise ValueError(f"{nm} must be contiguous")
+    if h.dim() != 3 or x.dim() != 3 or w.dim() != 2:
+        raise ValueError("h and x must be [B, N, .], w [D, K]")
+    B, N, K = h.shape
+    D = w.shape[0]
+    if w.shape[1] != K or x.shape != (B, N, D):
+        raise ValueError("shapes do not match: h [B, N, K], w [D, K], x [B, N, D]")
+    dt, gs = _mod_views(B, D, gate)
+    x_out = torch.empty_like(x) if x_out is None else x_out
+    _need_cuda_bf16("x_out", x_out)
+    if x_out.shape != x.shape or not x_out.is_contiguous():
+        raise ValueError("x_out must match x")
+    if status is not None and (status.dtype != torch.int32 or not status.is_cuda):
+        raise ValueError("status must be a CUDA int32 tensor")
+    _call("dit_gemm_gated_residual", h.data_ptr(), w.data_ptr(), x.data_ptr(), x_out.data_ptr(),
+          gate.data_ptr(), dt, gs, B, N, K, D, _ptr(status), _stream(x))
+    return x_out

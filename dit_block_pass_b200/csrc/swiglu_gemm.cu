@@ -187,16 +187,31 @@ __device__ __forceinline__ float silu_mul(float g, float u) {
     return __fdividef(g, 1.0f + __expf(-g)) * u;
 }
 
+// Epilogues of the one main loop.
+enum Epilogue {
+    kSwiGLU = 0,            // out[m, j] = silu(acc[m, j]) * acc[m, 128 + j]: 128 outputs per tile
+    kGatedResidual = 1,     // out[m, n] = x[m, n] + gate_b[n] * acc[m, n]: 256 outputs per tile
+};
+
 struct GemmParams {
     uint16_t* out;
     int* status;            // device word, set to 1 when a wait expires (may be NULL)
-    int M, K, F;
+    int M, K;
+    int cols;               // output columns (F, or D)
     int tiles_m, tiles_n, tiles;
+    int b1_offset;          // row of the second W box relative to the first (0: own map)
+    // gated residual
+    const uint16_t* x;      // [M, cols] residual stream (may be out)
+    const void* gate;       // [B, cols] per-sample gate, fp32 or bf16
+    int gate_dtype;
+    int64_t gate_stride;
+    int64_t tokens;         // token rows per sample
 };
 
 // Output tile of linear tile id t: groups of kGroupM row tiles, the column
 // tiles outer within a group, so that the tiles in flight at one time share
 // their x and W tiles in L2.
+template <int EPI>
 __device__ __forceinline__ void tile_coords(const GemmParams& p, int t, int& m0, int& n0) {
     const int per_group = kGroupM * p.tiles_n;
     const int group = t / per_group;
@@ -204,16 +219,47 @@ __device__ __forceinline__ void tile_coords(const GemmParams& p, int t, int& m0,
     const int gsize = min(p.tiles_m - first_m, kGroupM);
     const int in_group = t - group * per_group;
     m0 = (first_m + in_group % gsize) * kBM;
-    n0 = (in_group / gsize) * kBN;
+    n0 = (in_group / gsize) * (EPI == kSwiGLU ? kBN : 2 * kBN);
+}
+
+__device__ __forceinline__ float gate_at(const GemmParams& p, int64_t off) {
+    if (p.gate_dtype == DIT_F32) return __ldg(static_cast<const float*>(p.gate) + off);
+    return __uint_as_float(static_cast<uint32_t>(__ldg(static_cast<const uint16_t*>(p.gate) + off))
+                           << 16);
+}
+
+// bf16(x + g * a) for two elements with one rounding of each fp32-exact
+// value: the fp32 fma rounds once, and rounding that to bf16 can differ from
+// rounding the fma's exact value only on an exact bf16 tie (low half
+// 0x8000); that pair is redone in fp64, where g * a (fp32 x fp32) is exact.
+__device__ __noinline__ uint32_t resid_pair_fp64(float x0, float g0, float a0, float x1, float g1,
+                                                 float a1) {
+    const __nv_bfloat16 lo = __double2bfloat16(
+        fma(static_cast<double>(g0), static_cast<double>(a0), static_cast<double>(x0)));
+    const __nv_bfloat16 hi = __double2bfloat16(
+        fma(static_cast<double>(g1), static_cast<double>(a1), static_cast<double>(x1)));
+    return static_cast<uint32_t>(__bfloat16_as_ushort(lo)) |
+           (static_cast<uint32_t>(__bfloat16_as_ushort(hi)) << 16);
+}
+
+__device__ __forceinline__ uint32_t resid_pair(uint32_t xw, float g0, float a0, float g1,
+                                               float a1) {
+    const float x0 = bf16_lo(xw), x1 = bf16_hi(xw);
+    const float s0 = __fmaf_rn(g0, a0, x0);
+    const float s1 = __fmaf_rn(g1, a1, x1);
+    if (((__float_as_uint(s0) & 0xFFFFu) == 0x8000u) | ((__float_as_uint(s1) & 0xFFFFu) == 0x8000u))
+        return resid_pair_fp64(x0, g0, a0, x1, g1, a1);
+    return pack2(s0, s1);
 }
 
 // Persistent: CTA b takes tiles b, b + gridDim.x, ...  The K-step ring and
 // the two accumulators (TMEM columns [0, 256) and [256, 512)) run across
 // tiles, so the epilogue of one tile overlaps the main loop of the next.
+template <int EPI>
 __global__ void __launch_bounds__(kThreadsG, 1)
-swiglu_gemm_kernel(const __grid_constant__ CUtensorMap map_x,
-                   const __grid_constant__ CUtensorMap map_wg,
-                   const __grid_constant__ CUtensorMap map_wu, GemmParams p) {
+gemm_kernel(const __grid_constant__ CUtensorMap map_x,
+            const __grid_constant__ CUtensorMap map_wg,
+            const __grid_constant__ CUtensorMap map_wu, GemmParams p) {
     extern __shared__ uint8_t smem_raw[];
     // 1024-byte aligned stages (the swizzle atom), barriers after them
     const uint32_t raw = smem_u32(smem_raw);
@@ -263,7 +309,7 @@ swiglu_gemm_kernel(const __grid_constant__ CUtensorMap map_x,
             uint32_t it = 0;
             for (int t = blockIdx.x; t < p.tiles && !failed; t += gridDim.x) {
                 int m0, n0;
-                tile_coords(p, t, m0, n0);
+                tile_coords<EPI>(p, t, m0, n0);
                 for (int kb = 0; kb < nk; ++kb, ++it) {
                     const uint32_t s = it % kStages;
                     const uint32_t ph = (it / kStages) & 1u;
@@ -279,7 +325,7 @@ swiglu_gemm_kernel(const __grid_constant__ CUtensorMap map_x,
                                     kb * kBK, m0 + 128 * h);
                     tma_load_2d(sa + kTileA, &map_wg, bar_full + 8 * s, kb * kBK, n0);
                     tma_load_2d(sa + kTileA + kTileB / 2, &map_wu, bar_full + 8 * s, kb * kBK,
-                                n0);
+                                n0 + p.b1_offset);
                 }
             }
             if (failed) {
@@ -336,24 +382,27 @@ swiglu_gemm_kernel(const __grid_constant__ CUtensorMap map_x,
         uint32_t local = 0;
         for (int t = blockIdx.x; t < p.tiles; t += gridDim.x, ++local) {
             int m0, n0;
-            tile_coords(p, t, m0, n0);
+            tile_coords<EPI>(p, t, m0, n0);
             const uint32_t acc = local % kAccBufs;
             if (!mbar_wait(bar_tfull + 8 * acc, (local / kAccBufs) & 1u, abort)) {
                 failed = true;
                 break;
             }
             fence_after_sync();
+            // SwiGLU: per half, 4 chunks of 32 gate + 32 linear columns;
+            // gated residual: per half, 8 chunks of 32 output columns
+            constexpr int kPer = EPI == kSwiGLU ? kBN / 32 : 2 * kBN / 32;
 #pragma unroll 1
-            for (int hc = 0; hc < kHalves * (kBN / 32); ++hc) {
-                const int h = hc / (kBN / 32), c = hc % (kBN / 32);
+            for (int hc = 0; hc < kHalves * kPer; ++hc) {
+                const int h = hc / kPer, c = hc % kPer;
                 const int row = m0 + 128 * h + 32 * q + lane;
                 const uint32_t lane_addr =
                     tmem + acc * kAccCols + 256u * h + (static_cast<uint32_t>(32 * q) << 16);
                 float g[32], u[32];
                 tmem_ld32(lane_addr + 32 * c, g);
-                tmem_ld32(lane_addr + kBN + 32 * c, u);
+                if (EPI == kSwiGLU) tmem_ld32(lane_addr + kBN + 32 * c, u);
                 tmem_wait_ld();
-                if (hc == kHalves * (kBN / 32) - 1) {
+                if (hc == kHalves * kPer - 1) {
                     // every column of this accumulator is in registers: hand it back
                     fence_before_sync();
                     __syncwarp();
@@ -363,14 +412,37 @@ swiglu_gemm_kernel(const __grid_constant__ CUtensorMap map_x,
                                      : "memory");
                 }
                 if (row < p.M) {
-                    uint16_t* dst = p.out + static_cast<int64_t>(row) * p.F + n0 + 32 * c;
+                    const int col0 = n0 + 32 * c;
+                    uint16_t* dst = p.out + static_cast<int64_t>(row) * p.cols + col0;
+                    if (EPI == kSwiGLU) {
 #pragma unroll
-                    for (int v = 0; v < 4; ++v) {
-                        if (n0 + 32 * c + 8 * v < p.F) {
-                            float o[8];
+                        for (int v = 0; v < 4; ++v) {
+                            if (col0 + 8 * v < p.cols) {
+                                float o[8];
 #pragma unroll
-                            for (int i = 0; i < 8; ++i) o[i] = silu_mul(g[8 * v + i], u[8 * v + i]);
-                            *reinterpret_cast<uint4*>(dst + 8 * v) = pack8(o);
+                                for (int i = 0; i < 8; ++i)
+                                    o[i] = silu_mul(g[8 * v + i], u[8 * v + i]);
+                                *reinterpret_cast<uint4*>(dst + 8 * v) = pack8(o);
+                            }
+                        }
+                    } else {
+                        const uint16_t* xs = p.x + static_cast<int64_t>(row) * p.cols + col0;
+                        const int64_t goff = (row / p.tokens) * p.gate_stride + col0;
+#pragma unroll
+                        for (int v = 0; v < 4; ++v) {
+                            if (col0 + 8 * v < p.cols) {
+                                const uint4 xv = *reinterpret_cast<const uint4*>(xs + 8 * v);
+                                float gv[8];
+#pragma unroll
+                                for (int i = 0; i < 8; ++i) gv[i] = gate_at(p, goff + 8 * v + i);
+                                const float* a = g + 8 * v;
+                                uint4 o;
+                                o.x = resid_pair(xv.x, gv[0], a[0], gv[1], a[1]);
+                                o.y = resid_pair(xv.y, gv[2], a[2], gv[3], a[3]);
+                                o.z = resid_pair(xv.z, gv[4], a[4], gv[5], a[5]);
+                                o.w = resid_pair(xv.w, gv[6], a[6], gv[7], a[7]);
+                                *reinterpret_cast<uint4*>(dst + 8 * v) = o;
+                            }
                         }
                     }
                 }
@@ -428,6 +500,40 @@ bool make_map(CUtensorMap* map, const void* base, int64_t rows, int K) {
 }  // namespace
 }  // namespace dit
 
+namespace dit {
+namespace {
+
+// Shared launch: x [M, K], two W views for the B tile's halves, epilogue EPI.
+template <int EPI>
+int launch_gemm(const uint16_t* x, const uint16_t* w0, int64_t w0_rows, const uint16_t* w1,
+                int64_t w1_rows, GemmParams& p, int64_t M, int K, int cols, void* stream) {
+    CUtensorMap mx, m0, m1;
+    if (!make_map(&mx, x, M, K) || !make_map(&m0, w0, w0_rows, K) ||
+        !make_map(&m1, w1, w1_rows, K))
+        return DIT_ERR_LAUNCH;
+    p.M = static_cast<int>(M);
+    p.K = K;
+    p.cols = cols;
+    p.tiles_m = static_cast<int>((M + kBM - 1) / kBM);
+    const int tile_cols = EPI == kSwiGLU ? kBN : 2 * kBN;
+    p.tiles_n = (cols + tile_cols - 1) / tile_cols;
+    const int64_t tiles = static_cast<int64_t>(p.tiles_m) * p.tiles_n;
+    if (tiles > 0x7FFFFFFF) return DIT_ERR_SHAPE;
+    p.tiles = static_cast<int>(tiles);
+    const int sms = device_sm_count();
+    if (sms <= 0) return DIT_ERR_LAUNCH;
+    const int64_t ctas = tiles < sms ? tiles : sms;     // one persistent CTA per SM
+    if (cudaFuncSetAttribute(gemm_kernel<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(kSmemBytes)) != cudaSuccess)
+        return DIT_ERR_LAUNCH;
+    gemm_kernel<EPI><<<static_cast<unsigned>(ctas), kThreadsG, kSmemBytes, as_stream(stream)>>>(
+        mx, m0, m1, p);
+    return launch_status();
+}
+
+}  // namespace
+}  // namespace dit
+
 extern "C" int dit_swiglu_gemm(const uint16_t* x, const uint16_t* w, uint16_t* out, int64_t M,
                                int K, int F, int* status, void* stream) {
     using namespace dit;
@@ -442,28 +548,42 @@ extern "C" int dit_swiglu_gemm(const uint16_t* x, const uint16_t* w, uint16_t* o
     if (overlaps(out, out_bytes, x, static_cast<size_t>(M) * K * 2) ||
         overlaps(out, out_bytes, w, static_cast<size_t>(2) * F * K * 2))
         return DIT_ERR_OVERLAP;
-    CUtensorMap mx, mg, mu;
-    const uint16_t* w_lin = w + static_cast<int64_t>(F) * K;
-    if (!make_map(&mx, x, M, K) || !make_map(&mg, w, F, K) || !make_map(&mu, w_lin, F, K))
-        return DIT_ERR_LAUNCH;
     GemmParams p{};
     p.out = out;
     p.status = status;
-    p.M = static_cast<int>(M);
-    p.K = K;
-    p.F = F;
-    p.tiles_m = static_cast<int>((M + kBM - 1) / kBM);
-    p.tiles_n = (F + kBN - 1) / kBN;
-    const int64_t tiles = static_cast<int64_t>(p.tiles_m) * p.tiles_n;
-    if (tiles > 0x7FFFFFFF) return DIT_ERR_SHAPE;
-    p.tiles = static_cast<int>(tiles);
-    const int sms = device_sm_count();
-    if (sms <= 0) return DIT_ERR_LAUNCH;
-    const int64_t ctas = tiles < sms ? tiles : sms;     // one persistent CTA per SM
-    if (cudaFuncSetAttribute(swiglu_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(kSmemBytes)) != cudaSuccess)
-        return DIT_ERR_LAUNCH;
-    swiglu_gemm_kernel<<<static_cast<unsigned>(ctas), kThreadsG, kSmemBytes, as_stream(stream)>>>(
-        mx, mg, mu, p);
-    return launch_status();
+    p.b1_offset = 0;
+    return launch_gemm<kSwiGLU>(x, w, F, w + static_cast<int64_t>(F) * K, F, p, M, K, F, stream);
+}
+
+extern "C" int dit_gemm_gated_residual(const uint16_t* h, const uint16_t* w, const uint16_t* x,
+                                       uint16_t* x_out, const void* gate, int gate_dtype,
+                                       int64_t gate_batch_stride, int B, int64_t N, int K, int D,
+                                       int* status, void* stream) {
+    using namespace dit;
+    if (B < 0 || N < 0 || K <= 0 || D <= 0 || gate_batch_stride < 0) return DIT_ERR_SHAPE;
+    if (gate_dtype != DIT_F32 && gate_dtype != DIT_BF16) return DIT_ERR_DTYPE;
+    if (K % 8 || D % 8) return DIT_ERR_ALIGN;
+    const int64_t M = static_cast<int64_t>(B) * N;
+    if (M > 0x7FFFFFFFLL - kBM || D > (1 << 30)) return DIT_ERR_SHAPE;
+    if (M == 0) return DIT_OK;
+    if (!h || !w || !x || !x_out || !gate) return DIT_ERR_NULL;
+    if (!aligned16(h) || !aligned16(w) || !aligned16(x) || !aligned16(x_out)) return DIT_ERR_ALIGN;
+    if (reinterpret_cast<uintptr_t>(gate) % (gate_dtype == DIT_F32 ? 4 : 2)) return DIT_ERR_ALIGN;
+    if (status && reinterpret_cast<uintptr_t>(status) % 4) return DIT_ERR_ALIGN;
+    const size_t xb = static_cast<size_t>(M) * D * 2;
+    // x_out may be x itself (each element is read, then written, by one thread)
+    if ((x_out != x && overlaps(x_out, xb, x, xb)) ||
+        overlaps(x_out, xb, h, static_cast<size_t>(M) * K * 2) ||
+        overlaps(x_out, xb, w, static_cast<size_t>(D) * K * 2))
+        return DIT_ERR_OVERLAP;
+    GemmParams p{};
+    p.out = x_out;
+    p.status = status;
+    p.b1_offset = kBN;                 // the tile's second 128 rows of the same W
+    p.x = x;
+    p.gate = gate;
+    p.gate_dtype = gate_dtype;
+    p.gate_stride = gate_batch_stride;
+    p.tokens = N;
+    return launch_gemm<kGatedResidual>(h, w, D, w, D, p, M, K, D, stream);
 }

@@ -297,6 +297,28 @@ int dit_swiglu_gemm(const uint16_t* x, const uint16_t* w, uint16_t* out, int64_t
                     int* status, void* stream);
 
 /*
+ * The gated residual fused into the down-projection GEMM (tensor cores):
+ *     x_out[m, n] = bf16(x[m, n] + gate_b[n] * sum_k h[m, k] w[n, k])
+ * a2's residual update with its branch taken straight from the product, so
+ * the [M, D] branch is never written.  Same main loop as dit_swiglu_gemm.
+ *   h      device [B*N, K] bf16 (the MLP activations, token-major).
+ *   w      device [D, K] bf16, one row per output feature.
+ *   x      device [B*N, D] bf16 residual stream; x_out may be x (in place) or
+ *          must overlap neither x, h nor w.
+ *   gate   device [B, D] of gate_dtype (DIT_F32 or DIT_BF16), gate_batch_stride
+ *          elements between samples (0 broadcasts); token row m uses sample
+ *          m / N.
+ * K and D multiples of 8; h, w, x, x_out 16-byte aligned.  The sum runs in
+ * fp32 in the tensor memory; x + gate * sum is one fp32 fma rounded once to
+ * bf16 (redone in fp64 when the fma lands on a bf16 tie).  status as for
+ * dit_swiglu_gemm.
+ */
+int dit_gemm_gated_residual(const uint16_t* h, const uint16_t* w, const uint16_t* x,
+                            uint16_t* x_out, const void* gate, int gate_dtype,
+                            int64_t gate_batch_stride, int B, int64_t N, int K, int D,
+                            int* status, void* stream);
+
+/*
  * Cache-DiT step cache.  The LMSYS report (news.cocoloop.cn,
  * "minimax-h3-sglang-h200", section "Só com três camadas de aceleração
  * somadas chega-se a 6 vezes") reuses results cached between neighbouring

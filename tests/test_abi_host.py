@@ -252,3 +252,16 @@ def test_swiglu_gemm_argument_errors(lib):
     assert f(A + 8, A + 0x100000, A + 0x200000, 4, 64, 64, None, None) == E["ALIGN"]
     assert f(A, A + 0x100000, A + 0x200000, 4, 64, 64, A + 2, None) == E["ALIGN"]
     assert f(A, A + 0x100000, A + 0x100, 4, 64, 64, None, None) == E["OVERLAP"]   # over x
+
+
+def test_gemm_gated_residual_argument_errors(lib):
+    f = lib.dit_gemm_gated_residual
+    H, W_, X, O, G = A, A + 0x100000, A + 0x200000, A + 0x300000, A + 0x400000
+    assert f(H, W_, X, O, G, 0, 64, 0, 4, 64, 64, None, None) == 0          # empty
+    assert f(H, W_, X, O, G, 0, 64, 1, 4, 60, 64, None, None) == E["ALIGN"]
+    assert f(H, W_, X, O, G, 2, 64, 1, 4, 64, 64, None, None) == E["DTYPE"]
+    assert f(H, W_, X, O, None, 0, 64, 1, 4, 64, 64, None, None) == E["NULL"]
+    assert f(H, W_, X, O, G + 2, 0, 64, 1, 4, 64, 64, None, None) == E["ALIGN"]
+    assert f(H, W_, X, X + 16, G, 0, 64, 1, 4, 64, 64, None, None) == E["OVERLAP"]
+    assert f(H, W_, X, H, G, 0, 64, 1, 4, 64, 64, None, None) == E["OVERLAP"]
+    assert f(H, W_, X, O, G, 0, -1, 1, 4, 64, 64, None, None) == E["SHAPE"]

@@ -1,5 +1,5 @@
-"""SwiGLU fused into the up-projection GEMM (tcgen05) against the fp64
-oracle.  Tolerance, derived from the arithmetic: the tensor cores sum K
+"""SwiGLU fused into the up-projection GEMM and the gated residual fused
+into the down-projection GEMM (tcgen05) against the fp64 oracle.  Tolerance, derived from the arithmetic: the tensor cores sum K
 exact bf16 products in fp32, so |g_gpu - g| <= 2 K 2^-24 sum_k |x w| for any
 summation order (the factor 2 is margin for the unit's internal order);
 that error passes through silu(g) * u with |silu'| <= 1.1, and the result is
@@ -132,3 +132,81 @@ def test_empty_and_errors():
     assert dbp.swiglu_gemm(x, w).shape == (0, 8)
     with pytest.raises(ValueError):
         dbp.swiglu_gemm(torch.zeros(4, 64, dtype=torch.bfloat16, device=DEV), w[:, :32].contiguous())
+
+
+# ------------------------------------------ gated residual, down-projection
+
+
+def _check_resid(orc, h_rows, w, x_rows, gate, N, got, rows_global, what=""):
+    """x' within the derived bound: |g| * 2 K 2^-24 sum|h w| for the
+    accumulation, plus one bf16 ulp for the final rounding."""
+    B = gate.shape[0]
+    # the oracle on the selected rows: pass them as their own samples
+    ref, dot, ad = orc.gemm_gated_residual(bits(h_rows), bits(w), bits(x_rows),
+                                           gate.double().numpy()[rows_global // N], 1)
+    K = h_rows.shape[1]
+    gv = np.abs(gate.double().numpy()[rows_global // N])
+    bound = gv * 2.0 * K * 2.0 ** -24 * ad + _ulp_bf16(orc.bf16_to_f64(ref))
+    out = orc.bf16_to_f64(bits(got))
+    err = np.abs(out - orc.bf16_to_f64(ref))
+    assert not (err > bound).any(), (what, int((err > bound).sum()))
+    assert float(np.mean(err == 0)) > 0.95, (what, float(np.mean(err == 0)))
+    del B
+
+
+@pytest.mark.parametrize("B,N,K,D", [(1, 128, 64, 256), (2, 100, 512, 384), (3, 77, 136, 264),
+                                     (1, 1000, 2048, 1024)])
+@pytest.mark.parametrize("gate_dtype", [torch.float32, torch.bfloat16])
+def test_down_projection_gated_residual(orc, B, N, K, D, gate_dtype):
+    g = torch.Generator().manual_seed(B * 1000 + N + K + D)
+    h = torch.randn(B, N, K, generator=g).to(torch.bfloat16)
+    w = (torch.randn(D, K, generator=g) / K ** 0.5).to(torch.bfloat16)
+    x = torch.randn(B, N, D, generator=g).to(torch.bfloat16)
+    gate = (0.3 * torch.randn(B, D, generator=g)).to(gate_dtype)
+    st = torch.zeros(1, dtype=torch.int32, device=DEV)
+    out = dbp.gemm_gated_residual(h.to(DEV), w.to(DEV), x.to(DEV), gate.to(DEV), status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    M = B * N
+    rows = np.arange(M)
+    _check_resid(orc, h.view(M, K), w, x.view(M, D), gate.float(), N, out.view(M, D).cpu(), rows,
+                 what=f"{B}x{N}x{K}x{D}")
+
+
+def test_down_projection_in_place_and_zero_gate(orc):
+    """In place on x; a zero gate leaves x bit for bit."""
+    B, N, K, D = 2, 200, 256, 512
+    g = torch.Generator().manual_seed(3)
+    h = torch.randn(B, N, K, generator=g).to(torch.bfloat16).to(DEV)
+    w = (torch.randn(D, K, generator=g) / K ** 0.5).to(torch.bfloat16).to(DEV)
+    x = torch.randn(B, N, D, generator=g).to(torch.bfloat16).to(DEV)
+    x0 = x.clone()
+    dbp.gemm_gated_residual(h, w, x, torch.zeros(B, D, device=DEV), x_out=x)
+    torch.cuda.synchronize()
+    assert torch.equal(x.view(torch.int16), x0.view(torch.int16))
+    gate = 0.5 * torch.ones(D, device=DEV)                  # one gate for every sample
+    ref = dbp.gemm_gated_residual(h, w, x0, gate)
+    dbp.gemm_gated_residual(h, w, x, gate, x_out=x)
+    torch.cuda.synchronize()
+    assert torch.equal(x.view(torch.int16), ref.view(torch.int16))
+
+
+def test_down_projection_full_size_sampled_rows(orc):
+    """The h3_5s down-projection: h [124992, 13824], w [5120, 13824]."""
+    wl = W.CONFIGS["h3_5s"]
+    M, K, D = wl.M, wl.F, wl.D
+    gen = torch.Generator(device=DEV).manual_seed(2)
+    h = torch.randn(1, M, K, generator=gen, device=DEV).to(torch.bfloat16)
+    w = (torch.randn(D, K, generator=gen, device=DEV) / K ** 0.5).to(torch.bfloat16)
+    x = torch.randn(1, M, D, generator=gen, device=DEV).to(torch.bfloat16)
+    gate = 0.3 * torch.randn(1, D, generator=gen, device=DEV)
+    st = torch.zeros(1, dtype=torch.int32, device=DEV)
+    out = dbp.gemm_gated_residual(h, w, x, gate, status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    rows = np.array([0, 255, 256, 70001, M - 257, M - 1])
+    idx = torch.from_numpy(rows).to(DEV)
+    _check_resid(orc, h[0, idx].cpu(), w.cpu(), x[0, idx].cpu(), gate.cpu(), M,
+                 out[0, idx].cpu(), rows, what="h3_5s rows")
+    del h, w, x, out
+    torch.cuda.empty_cache()
