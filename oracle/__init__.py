@@ -82,6 +82,11 @@ class Oracle:
         L.dito_gemm_gated_residual.argtypes = [_u16p, _u16p, _u16p, _f64p, _i64, _i64, _i64,
                                                _int, _int, _i64p, _i64, _u16p, _f64p, _f64p]
         L.dito_gemm_gated_residual.restype = _int
+        L.dito_subblock_keep_count.argtypes = [_i64, _dbl]
+        L.dito_subblock_keep_count.restype = _int
+        L.dito_subblock_router.argtypes = [_u16p, _u16p, _i64, _int, _i64, _int, _int, _int, _dbl,
+                                           ctypes.POINTER(ctypes.c_int32), _f64p, _f64p]
+        L.dito_subblock_router.restype = _int
         L.dito_residual_store.argtypes = [_u16p, _u16p, _i64, _u16p]
         L.dito_residual_apply.argtypes = [_u16p, _u16p, _i64, _u16p]
         for name in ("dito_adaln_modulate", "dito_gated_residual_adaln", "dito_swiglu",
@@ -281,6 +286,32 @@ class Oracle:
             None if r is None else r.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)), R,
             _p(out, _u16p), _p(dot, _f64p), _p(ad, _f64p)), "gemm_gated_residual")
         return out, dot, ad
+
+    def subblock_keep_count(self, n_blocks, sparsity):
+        n = self.lib.dito_subblock_keep_count(int(n_blocks), float(sparsity))
+        _check(0 if n > 0 else n, "subblock_keep_count")
+        return n
+
+    def subblock_router(self, q, k, B, H, hd, block, sparsity, row_stride=None):
+        """q, k: [B*N, >= H*hd] bf16 bits (rows `row_stride` apart).  Returns
+        (kept [B, H, n_blocks, n_keep] int32, scores [B, H, n_blocks, n_blocks]
+        fp64)."""
+        q = _c(q, np.uint16)
+        k = _c(k, np.uint16)
+        if row_stride is None:
+            row_stride = q.shape[-1]
+        N = q.size // row_stride // B
+        nb = (N + block - 1) // block
+        n_keep = self.subblock_keep_count(nb, sparsity)
+        kept = np.empty((B, H, nb, n_keep), dtype=np.int32)
+        scores = np.empty((B, H, nb, nb), dtype=np.float64)
+        work = np.empty(2 * nb * hd + 2 * nb, dtype=np.float64)
+        rc = self.lib.dito_subblock_router(_p(q, _u16p), _p(k, _u16p), row_stride, B, N, H, hd,
+                                           block, sparsity,
+                                           kept.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)),
+                                           _p(scores, _f64p), _p(work, _f64p))
+        _check(0 if rc > 0 else rc, "subblock_router")
+        return kept, scores
 
     def residual_store(self, before, after):
         """R = bf16(after - before), elementwise on bf16 bits."""

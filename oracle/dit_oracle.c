@@ -545,3 +545,96 @@ int dito_gemm_gated_residual(const uint16_t* h, const uint16_t* w, const uint16_
     }
     return 0;
 }
+
+/* -------------------------------------------- SubBlock sparse router (f4) */
+
+/*
+ * [REPORT], section "Só com três camadas de aceleração somadas chega-se a 6
+ * vezes": a block-sparse router cuts, from the 10th denoising step on, the
+ * KV blocks that take part in attention, at sparsity 0.75 or 0.80.  The pages
+ * give no rule; the reading here is the plainest one:
+ *   - the N tokens of a sample are cut into blocks of `block` consecutive
+ *     tokens (the last one may be shorter): n_blocks = ceil(N / block);
+ *   - per head, a block's summary is the mean of its rows (q for query
+ *     blocks, k for key blocks);
+ *   - query block i scores key block j by the dot product of the summaries;
+ *   - each query block keeps the n_keep key blocks with the highest scores
+ *     (ties: the lower block index first), n_keep = ceil((1 - sparsity) *
+ *     n_blocks) and at least 1; the kept indices are written in increasing
+ *     order.
+ * q, k: rows of B*N tokens, `row_stride` elements apart, each H heads of hd
+ * values (head h at offset h*hd).  kept: [B, H, n_blocks, n_keep] int32.
+ * scores (optional): [B, H, n_blocks, n_blocks] fp64.  work: 2*n_blocks*hd
+ * + 2*n_blocks doubles.  Returns n_keep, or a negative code.
+ */
+int dito_subblock_keep_count(int64_t n_blocks, double sparsity)
+{
+    if (n_blocks <= 0 || !(sparsity >= 0.0) || !(sparsity < 1.0)) return -2;
+    double want = ceil((1.0 - sparsity) * (double)n_blocks - 1e-9);
+    int64_t keep = (int64_t)want;
+    if (keep < 1) keep = 1;
+    if (keep > n_blocks) keep = n_blocks;
+    return (int)keep;
+}
+
+int dito_subblock_router(const uint16_t* q, const uint16_t* k, int64_t row_stride, int B,
+                         int64_t N, int H, int hd, int block, double sparsity, int32_t* kept,
+                         double* scores, double* work)
+{
+    if (B < 0 || N <= 0 || H < 1 || hd < 1 || block < 1 || row_stride < (int64_t)H * hd)
+        return -2;
+    int64_t nb = (N + block - 1) / block;
+    int n_keep = dito_subblock_keep_count(nb, sparsity);
+    if (n_keep < 0) return n_keep;
+    double* qm = work;                 /* [nb, hd] */
+    double* km = qm + nb * hd;         /* [nb, hd] */
+    double* sc = km + nb * hd;         /* [nb] */
+    int64_t* order = (int64_t*)(sc + nb);   /* [nb], fits in the next nb doubles */
+    for (int b = 0; b < B; ++b)
+        for (int h = 0; h < H; ++h) {
+            /* block means */
+            for (int64_t j = 0; j < nb; ++j) {
+                int64_t t0 = j * block, t1 = t0 + block < N ? t0 + block : N;
+                for (int d = 0; d < hd; ++d) {
+                    double sq = 0.0, sk = 0.0;
+                    for (int64_t t = t0; t < t1; ++t) {
+                        int64_t off = ((int64_t)b * N + t) * row_stride + (int64_t)h * hd + d;
+                        sq += dito_bf16_to_f64(q[off]);
+                        sk += dito_bf16_to_f64(k[off]);
+                    }
+                    qm[j * hd + d] = sq / (double)(t1 - t0);
+                    km[j * hd + d] = sk / (double)(t1 - t0);
+                }
+            }
+            for (int64_t i = 0; i < nb; ++i) {
+                for (int64_t j = 0; j < nb; ++j) {
+                    double s = 0.0;
+                    for (int d = 0; d < hd; ++d) s += qm[i * hd + d] * km[j * hd + d];
+                    sc[j] = s;
+                    order[j] = j;
+                    if (scores) scores[(((int64_t)b * H + h) * nb + i) * nb + j] = s;
+                }
+                /* selection: repeatedly take the best remaining block */
+                int32_t* out = kept + (((int64_t)b * H + h) * nb + i) * n_keep;
+                for (int r = 0; r < n_keep; ++r) {
+                    int64_t best = r;
+                    for (int64_t c = r + 1; c < nb; ++c) {
+                        int64_t oc = order[c], ob = order[best];
+                        if (sc[oc] > sc[ob] || (sc[oc] == sc[ob] && oc < ob)) best = c;
+                    }
+                    int64_t tmp = order[r];
+                    order[r] = order[best];
+                    order[best] = tmp;
+                }
+                /* the kept blocks in increasing order */
+                for (int r = 0; r < n_keep; ++r) out[r] = (int32_t)order[r];
+                for (int r = 1; r < n_keep; ++r)
+                    for (int c = r; c > 0 && out[c - 1] > out[c]; --c) {
+                        int32_t t = out[c];
+                        out[c] = out[c - 1];
+                        out[c - 1] = t;
+                    }
+            }
+        }
+    return n_keep;
+}

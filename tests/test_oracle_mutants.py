@@ -52,6 +52,16 @@ MUTANTS = {
                            "const uint16_t* wn = w + (int64_t)n;"),
     "down_gate_added": ("dito_bf16_to_f64(x[m * (int64_t)D + n]) + g[n] * s);",
                         "dito_bf16_to_f64(x[m * (int64_t)D + n]) + g[n] + s);"),
+    "router_mean_over_full_block": ("qm[j * hd + d] = sq / (double)(t1 - t0);",
+                                    "qm[j * hd + d] = sq / (double)block;"),
+    "router_keeps_lowest": ("if (sc[oc] > sc[ob] || (sc[oc] == sc[ob] && oc < ob)) best = c;",
+                            "if (sc[oc] < sc[ob] || (sc[oc] == sc[ob] && oc < ob)) best = c;"),
+    "router_ties_to_higher_index": ("if (sc[oc] > sc[ob] || (sc[oc] == sc[ob] && oc < ob)) best = c;",
+                                    "if (sc[oc] > sc[ob] || (sc[oc] == sc[ob] && oc > ob)) best = c;"),
+    "router_scores_q_with_q": ("for (int d = 0; d < hd; ++d) s += qm[i * hd + d] * km[j * hd + d];",
+                               "for (int d = 0; d < hd; ++d) s += qm[i * hd + d] * qm[j * hd + d];"),
+    "router_keep_floor": ("double want = ceil((1.0 - sparsity) * (double)n_blocks - 1e-9);",
+                          "double want = floor((1.0 - sparsity) * (double)n_blocks);"),
     "swiglu_exp_sign": ("a / (1.0 + exp(-a))", "a / (1.0 + exp(a))"),
     "swiglu_halves_swapped": ("double a = dito_bf16_to_f64(in[m * 2 * (int64_t)F + j]);",
                               "double a = dito_bf16_to_f64(in[m * 2 * (int64_t)F + F + j]);"),
@@ -102,7 +112,7 @@ MUTANTS = {
 
 PIN_MODULES = ["test_oracle_bf16", "test_oracle_adaln", "test_oracle_swiglu", "test_oracle_qk",
                "test_oracle_cachedit", "test_oracle_cache_step", "test_oracle_swiglu_gemm",
-               "test_oracle_gemm_residual"]
+               "test_oracle_gemm_residual", "test_oracle_subblock"]
 
 
 def _pins():
