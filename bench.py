@@ -400,6 +400,34 @@ def time_swiglu_gemm(chain, steps, warmup, world):
     return out
 
 
+def time_subblock_router(chain, steps, warmup, world):
+    """The SubBlock router on the clip's q and k (blocks of 128 tokens,
+    sparsity 0.75): ms per call (two launches: block means, then scores and
+    selection)."""
+    import torch
+    import dit_block_pass_b200 as dbp
+    c, wl = chain, chain.wl
+    D = wl.D
+    q, k = c.qkv[:, :, :D], c.qkv[:, :, D:2 * D]
+    nb = (wl.N + 127) // 128
+    n_keep = dbp.subblock_keep_count(nb, 0.75)
+    ws = torch.empty(int(dbp.library().dit_subblock_workspace_bytes(wl.B, wl.N, wl.H, wl.hd, 128)),
+                     dtype=torch.uint8, device=c.dev)
+    kept = torch.empty(wl.B, wl.H, nb, n_keep, dtype=torch.int32, device=c.dev)
+    op = lambda: dbp.subblock_router(q, k, wl.H, 128, 0.75, workspace=ws, kept=kept)
+    for _ in range(warmup):
+        op()
+    barrier_sync(world)
+    stream = torch.cuda.current_stream()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(steps):
+        op()
+    b.record(stream)
+    barrier_sync(world)
+    return a.elapsed_time(b) / steps, nb, n_keep
+
+
 def tensor_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -613,6 +641,8 @@ def main():
         tok_sets, tok_share = time_token_sets(chain, args.steps, args.warmup, world)
         step_cache = time_cache_step(chain, args.steps, args.warmup, world)
         gemm_ms = time_swiglu_gemm(chain, args.gemm_steps, 2, world)
+        router_ms, router_nb, router_keep = time_subblock_router(chain, args.steps, args.warmup,
+                                                                 world)
     finally:
         if sampler:
             sampler.__exit__(None, None, None)
@@ -660,6 +690,11 @@ def main():
                    "unfused_ms (cuBLAS bf16 GEMM + swiglu_kernel)": round(unfused_ms, 3),
                    "speedup_vs_unfused": round(unfused_ms / fused_ms, 4),
                    "shape": f"[{wl.M}, {wl.D}] x [{2 * wl.F}, {wl.D}]^T -> [{wl.M}, {wl.F}]"}
+    router_ms = max_over_ranks(router_ms, world)
+    router_gbs = 4.0 * wl.M * wl.D / (router_ms / 1000.0) / 1e9        # read q and k once
+    subblock = {"ms": round(router_ms, 4), "GB/s": round(router_gbs, 1),
+                "frac_of_peak": round(router_gbs / peak, 4), "block": 128, "sparsity": 0.75,
+                "key_blocks": router_nb, "kept_per_query_block": router_keep}
     dom_ms = per_op[OPS.index(DOMINANT)]
     achieved = nbytes[DOMINANT] / (dom_ms / 1000.0) / 1e9
     tr = NCU_TRAFFIC.get(DOMINANT)
@@ -699,7 +734,7 @@ def main():
                        "l2": "every input is larger than L2 (126 MB); no flush",
                        "parallelism": f"{world} independent clip(s), one per GPU"},
             "ops": ops, "qk_options": qk_options, "token_sets": token_sets,
-            "cache_step": cache_step, "swiglu_gemm": swiglu_gemm,
+            "cache_step": cache_step, "swiglu_gemm": swiglu_gemm, "subblock_router": subblock,
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": chain.launches_per_step() * args.steps, "clocks": clocks,
         }

@@ -25,7 +25,8 @@ __all__ = [
     "DitError", "library", "library_path", "adaln_modulate", "gated_residual_adaln", "swiglu",
     "qk_rmsnorm_rope3d", "cachedit_workspace_bytes", "cachedit_residual_diff",
     "cachedit_residual_sums", "cachedit_decide", "cachedit_residual_diff_noalloc",
-    "launch_counts", "QKOut", "CachePolicy", "swiglu_gemm", "gemm_gated_residual", "cachedit_residual_store",
+    "launch_counts", "QKOut", "CachePolicy", "swiglu_gemm", "gemm_gated_residual",
+    "subblock_keep_count", "subblock_router", "cachedit_residual_store",
     "cachedit_residual_apply", "F32", "BF16", "ROPE_INTERLEAVED", "ROPE_HALF", "NORM_HEAD", "NORM_ROW",
 ]
 
@@ -45,6 +46,7 @@ launch_counts = {
     "cachedit_residual_diff": 2, "cachedit_residual_sums": 2, "cachedit_decide": 1,
     "cachedit_residual_diff_noalloc": 2, "cachedit_residual_store": 1,
     "cachedit_residual_apply": 1, "swiglu_gemm": 1, "gemm_gated_residual": 1,
+    "subblock_router": 2,
 }
 
 
@@ -103,6 +105,11 @@ def library() -> ctypes.CDLL:
                                                    dbl, dbl, i32, i32,
                                                    ctypes.POINTER(QKOut), vp]
             L.dit_swiglu_gemm.argtypes = [vp, vp, vp, i64, i32, i32, vp, vp]
+            L.dit_subblock_keep_count.argtypes = [i64, dbl]
+            L.dit_subblock_workspace_bytes.argtypes = [i32, i64, i32, i32, i32]
+            L.dit_subblock_workspace_bytes.restype = sz
+            L.dit_subblock_router.argtypes = [vp, vp, i64, i32, i64, i32, i32, i32, dbl, vp, vp,
+                                              sz, vp]
             L.dit_gemm_gated_residual.argtypes = [vp, vp, vp, vp, vp, i32, i64, i32, i64, i32,
                                                   i32, vp, vp]
             L.cachedit_residual_store.argtypes = [vp, vp, vp, i64, vp]
@@ -119,7 +126,8 @@ def library() -> ctypes.CDLL:
             for name in ("dit_adaln_modulate", "dit_gated_residual_adaln", "dit_swiglu",
                          "dit_adaln_modulate_tok", "dit_gated_residual_adaln_tok",
                          "cachedit_residual_store", "cachedit_residual_apply", "dit_swiglu_gemm",
-                         "dit_gemm_gated_residual",
+                         "dit_gemm_gated_residual", "dit_subblock_keep_count",
+                         "dit_subblock_router",
                          "dit_cache_policy_init", "dit_cache_policy_decide",
                          "dit_qk_rmsnorm_rope3d", "dit_qk_rmsnorm_rope3d_ex",
                          "cachedit_residual_diff",
@@ -581,3 +589,50 @@ def gemm_gated_residual(h: torch.Tensor, w: torch.Tensor, x: torch.Tensor, gate:
     _call("dit_gemm_gated_residual", h.data_ptr(), w.data_ptr(), x.data_ptr(), x_out.data_ptr(),
           gate.data_ptr(), dt, gs, B, N, K, D, _ptr(status), _stream(x))
     return x_out
+
+
+# ------------------------------------------------------------ SubBlock router
+
+
+def subblock_keep_count(n_blocks: int, sparsity: float) -> int:
+    n = library().dit_subblock_keep_count(int(n_blocks), float(sparsity))
+    if n < 0:
+        raise DitError("dit_subblock_keep_count", n, library().dit_status_string(n).decode())
+    return n
+
+
+def subblock_router(q: torch.Tensor, k: torch.Tensor, heads: int, block: int = 128,
+                    sparsity: float = 0.75, workspace: Optional[torch.Tensor] = None,
+                    kept: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """The kept key blocks of every query block: int32 [B, H, n_blocks,
+    n_keep], increasing.  q and k are [B, N, H*hd] views (e.g. slices of a
+    fused qkv buffer) sharing one row stride."""
+    _need_cuda_bf16("q", q)
+    _need_cuda_bf16("k", k)
+    B, N, width = q.shape
+    if k.shape != q.shape or width % heads:
+        raise ValueError("q and k must be [B, N, H*hd] of the same shape")
+    hd = width // heads
+    rs = _token_rows("q", q, B, N, width)
+    if _token_rows("k", k, B, N, width) != rs:
+        raise ValueError("q and k must share the row stride")
+    nb = (N + block - 1) // block
+    if not 0.0 <= sparsity < 1.0:
+        raise ValueError("sparsity must be in [0, 1)")
+    if nb == 0 or B == 0:
+        return torch.empty(B, heads, nb, 0, dtype=torch.int32, device=q.device)
+    n_keep = subblock_keep_count(nb, sparsity)
+    need = int(library().dit_subblock_workspace_bytes(B, N, heads, hd, block))
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    if workspace.numel() * workspace.element_size() < need:
+        raise ValueError(f"workspace needs {need} bytes")
+    if kept is None:
+        kept = torch.empty(B, heads, nb, n_keep, dtype=torch.int32, device=q.device)
+    if kept.dtype != torch.int32 or kept.numel() != B * heads * nb * n_keep or \
+            not kept.is_contiguous():
+        raise ValueError(f"kept must be a contiguous int32 [B, H, {nb}, {n_keep}] tensor")
+    _call("dit_subblock_router", q.data_ptr(), k.data_ptr(), rs, B, N, heads, hd, block,
+          float(sparsity), kept.data_ptr(), workspace.data_ptr(),
+          workspace.numel() * workspace.element_size(), _stream(q))
+    return kept

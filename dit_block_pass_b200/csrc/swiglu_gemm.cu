@@ -10,8 +10,8 @@
 // beyond the one-pass SwiGLU kernel: the 2F-wide product is consumed in the
 // accumulator.
 //
-// Design: persistent, one CTA of 6 warps per SM, output tiles of 256 rows x
-// 128 columns taken in a static round robin:
+// Design: persistent, one CTA of 10 warps per SM, output tiles of 256 rows x
+// 128 (SwiGLU) or 256 (gated residual) columns taken in a static round robin:
 //   warp 0   TMA producer: per 64-wide K step, two 128 x 64 tiles of x (rows
 //            m0.. and m0 + 128..) and two 128 x 64 tiles of W (the gate rows
 //            n0.. and the linear rows F + n0..) land in a 3-stage ring of
@@ -24,18 +24,21 @@
 //            slices per stage.  tcgen05.commit frees each stage when its
 //            MMAs have read it and hands the finished accumulators to the
 //            epilogue.
-//   warps 2-5 epilogue: tcgen05.ld pulls 32 gate and the matching 32 linear
-//            accumulators per thread (thread = output row), silu(g) * u in
-//            fp32, one rounding to bf16, 64-byte row segments to HBM.  Once
-//            the last columns are in registers the accumulators go back to
-//            the MMA warp; the producer has meanwhile filled the ring for
-//            the next tile.
+//   warps 2-9 epilogue: two warps per TMEM lane quarter, each taking half
+//            of the column chunks; tcgen05.ld pulls 32 accumulators per
+//            thread (thread = output row): gate and the matching linear
+//            columns -> silu(g) * u, or output columns -> x + gate * acc
+//            (gate rows read 16 bytes at a time when aligned); one rounding
+//            to bf16, 64-byte row segments to HBM.  Once the last columns
+//            are in registers the accumulators go back to the MMA warp; the
+//            producer has meanwhile filled the ring for the next tile.
 // Tiles are numbered in groups of 8 row tiles (column tiles outer within a
 // group) so that the tiles in flight share their x and W tiles in L2.  x, W
 // tiles beyond M, K or F are zero-filled by TMA; stores past M or F are
-// skipped.  Measured on B200 at the sustained tensor peak (the tile shape,
-// the raster group, the epilogue width and streaming stores all measured
-// within noise of each other there).
+// skipped.  The SwiGLU form runs at the sustained tensor peak of B200 (raster
+// groups, streaming stores and the epilogue width measured within noise
+// there); the heavier residual epilogue gained 8 % from the second epilogue
+// warp per lane quarter and vector gate loads.
 //
 // Every mbarrier wait is bounded (2 s of %globaltimer); on expiry the CTA
 // records an error in the caller's status word, drains what it issued
@@ -54,7 +57,8 @@ constexpr int kBM = 128 * kHalves;          // output rows per tile
 constexpr int kBN = 128;                    // output columns per tile (each W half)
 constexpr int kBK = 64;                     // K per stage: one 128-byte swizzle row
 constexpr int kStages = kHalves == 2 ? 3 : 4;
-constexpr int kThreadsG = 192;
+constexpr int kEpiWarps = 8;
+constexpr int kThreadsG = 64 + 32 * kEpiWarps;
 constexpr int kGroupM = 16 / kHalves;       // raster group (row tiles)
 constexpr uint32_t kTileA = kBM * kBK * 2;            // 16 KB per 128 rows
 constexpr uint32_t kTileB = 2 * kBN * kBK * 2;        // 32 KB (gate + linear)
@@ -206,6 +210,7 @@ struct GemmParams {
     int gate_dtype;
     int64_t gate_stride;
     int64_t tokens;         // token rows per sample
+    bool gate_vec;          // every gate row is 16-byte aligned
 };
 
 // Output tile of linear tile id t: groups of kGroupM row tiles, the column
@@ -284,7 +289,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap map_x,
         }
         for (uint32_t a = 0; a < kAccBufs; ++a) {
             mbar_init(bar_tfull + 8 * a, 1);
-            mbar_init(bar_tempty + 8 * a, 4);      // one arrival per epilogue warp
+            mbar_init(bar_tempty + 8 * a, kEpiWarps);   // one arrival per epilogue warp
         }
         mbar_init(bar_drain, 1);
         *abort = 0;
@@ -379,6 +384,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap map_x,
     } else {
         // epilogue: warp w reads TMEM lanes 32 * (w % 4) .. + 31
         const int q = warp & 3;
+        const int cg = (warp - 2) / 4;          // which share of the column chunks
         uint32_t local = 0;
         for (int t = blockIdx.x; t < p.tiles; t += gridDim.x, ++local) {
             int m0, n0;
@@ -391,10 +397,11 @@ gemm_kernel(const __grid_constant__ CUtensorMap map_x,
             fence_after_sync();
             // SwiGLU: per half, 4 chunks of 32 gate + 32 linear columns;
             // gated residual: per half, 8 chunks of 32 output columns
-            constexpr int kPer = EPI == kSwiGLU ? kBN / 32 : 2 * kBN / 32;
+            constexpr int kAll = EPI == kSwiGLU ? kBN / 32 : 2 * kBN / 32;
+            constexpr int kPer = kAll / (kEpiWarps / 4);
 #pragma unroll 1
             for (int hc = 0; hc < kHalves * kPer; ++hc) {
-                const int h = hc / kPer, c = hc % kPer;
+                const int h = hc / kPer, c = kPer * cg + hc % kPer;
                 const int row = m0 + 128 * h + 32 * q + lane;
                 const uint32_t lane_addr =
                     tmem + acc * kAccCols + 256u * h + (static_cast<uint32_t>(32 * q) << 16);
@@ -433,8 +440,23 @@ gemm_kernel(const __grid_constant__ CUtensorMap map_x,
                             if (col0 + 8 * v < p.cols) {
                                 const uint4 xv = *reinterpret_cast<const uint4*>(xs + 8 * v);
                                 float gv[8];
+                                if (p.gate_vec) {
+                                    if (p.gate_dtype == DIT_F32) {
+                                        const float4* gp = reinterpret_cast<const float4*>(
+                                            static_cast<const float*>(p.gate) + goff + 8 * v);
+                                        const float4 ga = __ldg(gp), gb = __ldg(gp + 1);
+                                        gv[0] = ga.x; gv[1] = ga.y; gv[2] = ga.z; gv[3] = ga.w;
+                                        gv[4] = gb.x; gv[5] = gb.y; gv[6] = gb.z; gv[7] = gb.w;
+                                    } else {
+                                        unpack8(__ldg(reinterpret_cast<const uint4*>(
+                                                    static_cast<const uint16_t*>(p.gate) + goff +
+                                                    8 * v)),
+                                                gv);
+                                    }
+                                } else {
 #pragma unroll
-                                for (int i = 0; i < 8; ++i) gv[i] = gate_at(p, goff + 8 * v + i);
+                                    for (int i = 0; i < 8; ++i) gv[i] = gate_at(p, goff + 8 * v + i);
+                                }
                                 const float* a = g + 8 * v;
                                 uint4 o;
                                 o.x = resid_pair(xv.x, gv[0], a[0], gv[1], a[1]);
@@ -585,5 +607,6 @@ extern "C" int dit_gemm_gated_residual(const uint16_t* h, const uint16_t* w, con
     p.gate_dtype = gate_dtype;
     p.gate_stride = gate_batch_stride;
     p.tokens = N;
+    p.gate_vec = aligned16(gate) && gate_batch_stride % (gate_dtype == DIT_F32 ? 4 : 8) == 0;
     return launch_gemm<kGatedResidual>(h, w, D, w, D, p, M, K, D, stream);
 }

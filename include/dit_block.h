@@ -319,6 +319,33 @@ int dit_gemm_gated_residual(const uint16_t* h, const uint16_t* w, const uint16_t
                             int* status, void* stream);
 
 /*
+ * SubBlock block-sparse attention router.  The LMSYS report (news.cocoloop.cn,
+ * "minimax-h3-sglang-h200", section "Só com três camadas de aceleração
+ * somadas chega-se a 6 vezes") cuts, from the 10th denoising step on, the KV
+ * blocks that take part in attention, at sparsity 0.75 or 0.80, and gives no
+ * rule.  Reading: the N tokens of a sample are cut into blocks of `block`
+ * consecutive tokens (the last may be shorter), n_blocks = ceil(N / block);
+ * per head, a block's summary is the mean of its rows; query block i scores
+ * key block j by the dot product of the summaries (fp32) and keeps the
+ * n_keep = dit_subblock_keep_count(n_blocks, sparsity) = max(1,
+ * ceil((1 - sparsity) n_blocks)) best key blocks, ties to the lower index.
+ *   q, k       device rows of B*N tokens, row_stride elements apart (a fused
+ *              qkv buffer works), H heads of hd values each (hd multiple of
+ *              8, <= 256; H*hd <= DIT_MAX_D); 16-byte aligned.
+ *   kept       device int32 [B, H, n_blocks, n_keep]: the kept key blocks of
+ *              each query block, in increasing order.
+ *   workspace  device, >= dit_subblock_workspace_bytes(...) bytes (the block
+ *              means, [B, 2, n_blocks, H*hd] fp32), 16-byte aligned.
+ * 0 <= sparsity < 1 (else DIT_ERR_VALUE); n_blocks <= 8192.  Which steps use
+ * the router (the report: from the 10th) is the caller's choice.
+ */
+int dit_subblock_keep_count(int64_t n_blocks, double sparsity);
+size_t dit_subblock_workspace_bytes(int B, int64_t N, int H, int hd, int block);
+int dit_subblock_router(const uint16_t* q, const uint16_t* k, int64_t row_stride, int B,
+                        int64_t N, int H, int hd, int block, double sparsity, int32_t* kept,
+                        void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * Cache-DiT step cache.  The LMSYS report (news.cocoloop.cn,
  * "minimax-h3-sglang-h200", section "Só com três camadas de aceleração
  * somadas chega-se a 6 vezes") reuses results cached between neighbouring

@@ -265,3 +265,23 @@ def test_gemm_gated_residual_argument_errors(lib):
     assert f(H, W_, X, X + 16, G, 0, 64, 1, 4, 64, 64, None, None) == E["OVERLAP"]
     assert f(H, W_, X, H, G, 0, 64, 1, 4, 64, 64, None, None) == E["OVERLAP"]
     assert f(H, W_, X, O, G, 0, -1, 1, 4, 64, 64, None, None) == E["SHAPE"]
+
+
+def test_subblock_router_host(lib):
+    """The keep count equals the oracle's; argument errors launch nothing."""
+    import oracle
+    orc = oracle.default()
+    for nb in (1, 3, 8, 100, 977, 1922, 8192):
+        for sp in (0.0, 0.5, 0.75, 0.8, 0.99):
+            assert lib.dit_subblock_keep_count(nb, sp) == orc.subblock_keep_count(nb, sp)
+    assert lib.dit_subblock_keep_count(10, 1.0) == E["VALUE"]
+    f = lib.dit_subblock_router
+    ws = lib.dit_subblock_workspace_bytes(1, 256, 2, 64, 128)
+    assert ws == 2 * 2 * 2 * 64 * 4
+    assert f(A, A + 0x1000, 128, 1, 0, 2, 64, 128, 0.75, A + 0x2000, A + 0x3000, ws, None) == 0
+    assert f(A, A + 0x1000, 128, 1, 256, 2, 60, 128, 0.75, A + 0x2000, A + 0x3000, ws, None) == E["SHAPE"]
+    assert f(A, A + 0x1000, 128, 1, 256, 2, 64, 128, 1.0, A + 0x2000, A + 0x3000, ws, None) == E["VALUE"]
+    assert f(A, A + 0x1000, 128, 1, 256, 2, 64, 128, 0.75, A + 0x2000, A + 0x3000, ws - 4, None) == E["WORKSPACE"]
+    assert f(A, None, 128, 1, 256, 2, 64, 128, 0.75, A + 0x2000, A + 0x3000, ws, None) == E["NULL"]
+    assert f(A, A + 0x1000, 120, 1, 256, 2, 64, 128, 0.75, A + 0x2000, A + 0x3000, ws, None) == E["SHAPE"]
+    assert f(A, A + 0x1000, 128, 1, 128 * 8193, 2, 64, 128, 0.75, A + 0x2000, A + 0x3000, ws, None) == E["SHAPE"]
