@@ -87,6 +87,10 @@ class Oracle:
         L.dito_subblock_router.argtypes = [_u16p, _u16p, _i64, _int, _i64, _int, _int, _int, _dbl,
                                            ctypes.POINTER(ctypes.c_int32), _f64p, _f64p]
         L.dito_subblock_router.restype = _int
+        L.dito_block_sparse_attention.argtypes = [_u16p, _u16p, _u16p, _i64, _int, _i64, _int,
+                                                  _int, _int, ctypes.POINTER(ctypes.c_int32),
+                                                  _int, _dbl, _f64p, _f64p]
+        L.dito_block_sparse_attention.restype = _int
         L.dito_residual_store.argtypes = [_u16p, _u16p, _i64, _u16p]
         L.dito_residual_apply.argtypes = [_u16p, _u16p, _i64, _u16p]
         for name in ("dito_adaln_modulate", "dito_gated_residual_adaln", "dito_swiglu",
@@ -312,6 +316,28 @@ class Oracle:
                                            _p(scores, _f64p), _p(work, _f64p))
         _check(0 if rc > 0 else rc, "subblock_router")
         return kept, scores
+
+    def block_sparse_attention(self, q, k, v, B, H, hd, block, kept, scale=None,
+                               row_stride=None):
+        """q, k, v: [B*N, >= H*hd] bf16 bits; kept: [B, H, n_blocks, n_keep]
+        int32.  Returns out [B*N, H*hd] fp64."""
+        q = _c(q, np.uint16)
+        k = _c(k, np.uint16)
+        v = _c(v, np.uint16)
+        if row_stride is None:
+            row_stride = q.shape[-1]
+        N = q.size // row_stride // B
+        kept = _c(kept, np.int32)
+        n_keep = kept.shape[-1]
+        if scale is None:
+            scale = 1.0 / np.sqrt(hd)
+        out = np.empty((B * N, H * hd), dtype=np.float64)
+        work = np.empty(n_keep * block, dtype=np.float64)
+        _check(self.lib.dito_block_sparse_attention(
+            _p(q, _u16p), _p(k, _u16p), _p(v, _u16p), row_stride, B, N, H, hd, block,
+            kept.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)), n_keep, float(scale),
+            _p(out, _f64p), _p(work, _f64p)), "block_sparse_attention")
+        return out
 
     def residual_store(self, before, after):
         """R = bf16(after - before), elementwise on bf16 bits."""

@@ -62,6 +62,10 @@ MUTANTS = {
                                "for (int d = 0; d < hd; ++d) s += qm[i * hd + d] * qm[j * hd + d];"),
     "router_keep_floor": ("double want = ceil((1.0 - sparsity) * (double)n_blocks - 1e-9);",
                           "double want = floor((1.0 - sparsity) * (double)n_blocks);"),
+    "attn_scale_dropped": ("                        s *= scale;\n", "\n"),
+    "attn_not_normalised": ("double pw = work[n++] / l;", "double pw = work[n++];"),
+    "attn_values_from_k": ("const uint16_t* vu = v + ((int64_t)b * N + u) * row_stride",
+                           "const uint16_t* vu = k + ((int64_t)b * N + u) * row_stride"),
     "swiglu_exp_sign": ("a / (1.0 + exp(-a))", "a / (1.0 + exp(a))"),
     "swiglu_halves_swapped": ("double a = dito_bf16_to_f64(in[m * 2 * (int64_t)F + j]);",
                               "double a = dito_bf16_to_f64(in[m * 2 * (int64_t)F + F + j]);"),
@@ -112,7 +116,8 @@ MUTANTS = {
 
 PIN_MODULES = ["test_oracle_bf16", "test_oracle_adaln", "test_oracle_swiglu", "test_oracle_qk",
                "test_oracle_cachedit", "test_oracle_cache_step", "test_oracle_swiglu_gemm",
-               "test_oracle_gemm_residual", "test_oracle_subblock"]
+               "test_oracle_gemm_residual", "test_oracle_subblock",
+               "test_oracle_sparse_attention"]
 
 
 def _pins():
