@@ -89,7 +89,8 @@ class Oracle:
         L.dito_subblock_router.restype = _int
         L.dito_block_sparse_attention.argtypes = [_u16p, _u16p, _u16p, _i64, _int, _i64, _int,
                                                   _int, _int, ctypes.POINTER(ctypes.c_int32),
-                                                  _int, _dbl, _f64p, _f64p]
+                                                  _int, _dbl, ctypes.POINTER(ctypes.c_int64),
+                                                  _i64, _f64p, _f64p]
         L.dito_block_sparse_attention.restype = _int
         L.dito_residual_store.argtypes = [_u16p, _u16p, _i64, _u16p]
         L.dito_residual_apply.argtypes = [_u16p, _u16p, _i64, _u16p]
@@ -318,9 +319,10 @@ class Oracle:
         return kept, scores
 
     def block_sparse_attention(self, q, k, v, B, H, hd, block, kept, scale=None,
-                               row_stride=None):
+                               row_stride=None, rows=None):
         """q, k, v: [B*N, >= H*hd] bf16 bits; kept: [B, H, n_blocks, n_keep]
-        int32.  Returns out [B*N, H*hd] fp64."""
+        int32.  Returns out [R, H*hd] fp64 for the query rows `rows` (b*N + t;
+        all B*N when None)."""
         q = _c(q, np.uint16)
         k = _c(k, np.uint16)
         v = _c(v, np.uint16)
@@ -331,11 +333,14 @@ class Oracle:
         n_keep = kept.shape[-1]
         if scale is None:
             scale = 1.0 / np.sqrt(hd)
-        out = np.empty((B * N, H * hd), dtype=np.float64)
+        r = None if rows is None else _c(rows, np.int64)
+        R = B * N if r is None else r.size
+        out = np.empty((R, H * hd), dtype=np.float64)
         work = np.empty(n_keep * block, dtype=np.float64)
         _check(self.lib.dito_block_sparse_attention(
             _p(q, _u16p), _p(k, _u16p), _p(v, _u16p), row_stride, B, N, H, hd, block,
             kept.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)), n_keep, float(scale),
+            None if r is None else r.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)), R,
             _p(out, _f64p), _p(work, _f64p)), "block_sparse_attention")
         return out
 

@@ -646,57 +646,63 @@ int dito_subblock_router(const uint16_t* q, const uint16_t* k, int64_t row_strid
  * with u over the tokens of the kept key blocks kept[b, h, i, 0..n_keep) of
  * the same sample (the last block may be shorter).  Non-causal.  fp64: the
  * scores, the max-shifted exponentials, the normaliser and the weighted sum.
- * q, k, v rows `row_stride` apart, H heads of hd; out: [B*N, H*hd] fp64.
- * work: the scores of one query token (n_keep * block doubles).
+ * q, k, v rows `row_stride` apart, H heads of hd.  rows (n_rows entries)
+ * picks the query rows (b*N + t) to compute, or NULL for all B*N; out:
+ * [n_rows, H*hd] fp64.  work: the scores of one query token (n_keep * block
+ * doubles).
  */
 int dito_block_sparse_attention(const uint16_t* q, const uint16_t* k, const uint16_t* v,
                                 int64_t row_stride, int B, int64_t N, int H, int hd, int block,
-                                const int32_t* kept, int n_keep, double scale, double* out,
-                                double* work)
+                                const int32_t* kept, int n_keep, double scale,
+                                const int64_t* rows, int64_t n_rows, double* out, double* work)
 {
-    if (B < 0 || N <= 0 || H < 1 || hd < 1 || block < 1 || n_keep < 1 ||
+    if (B < 0 || N <= 0 || H < 1 || hd < 1 || block < 1 || n_keep < 1 || n_rows < 0 ||
         row_stride < (int64_t)H * hd)
         return -2;
     int64_t nb = (N + block - 1) / block;
-    for (int b = 0; b < B; ++b)
-        for (int h = 0; h < H; ++h)
-            for (int64_t t = 0; t < N; ++t) {
-                int64_t i = t / block;
-                const int32_t* kb = kept + (((int64_t)b * H + h) * nb + i) * n_keep;
-                const uint16_t* qt = q + ((int64_t)b * N + t) * row_stride + (int64_t)h * hd;
-                int64_t n = 0;
-                double mx = -INFINITY;
-                for (int r = 0; r < n_keep; ++r) {
-                    int64_t j = kb[r];
-                    if (j < 0 || j >= nb) return -3;
-                    int64_t u1 = (j + 1) * block < N ? (j + 1) * block : N;
-                    for (int64_t u = j * block; u < u1; ++u) {
-                        const uint16_t* ku = k + ((int64_t)b * N + u) * row_stride + (int64_t)h * hd;
-                        double s = 0.0;
-                        for (int d = 0; d < hd; ++d)
-                            s += dito_bf16_to_f64(qt[d]) * dito_bf16_to_f64(ku[d]);
-                        s *= scale;
-                        work[n++] = s;
-                        if (s > mx) mx = s;
-                    }
-                }
-                double l = 0.0;
-                for (int64_t e = 0; e < n; ++e) {
-                    work[e] = exp(work[e] - mx);
-                    l += work[e];
-                }
-                double* ot = out + ((int64_t)b * N + t) * ((int64_t)H * hd) + (int64_t)h * hd;
-                for (int d = 0; d < hd; ++d) ot[d] = 0.0;
-                n = 0;
-                for (int r = 0; r < n_keep; ++r) {
-                    int64_t j = kb[r];
-                    int64_t u1 = (j + 1) * block < N ? (j + 1) * block : N;
-                    for (int64_t u = j * block; u < u1; ++u) {
-                        const uint16_t* vu = v + ((int64_t)b * N + u) * row_stride + (int64_t)h * hd;
-                        double pw = work[n++] / l;
-                        for (int d = 0; d < hd; ++d) ot[d] += pw * dito_bf16_to_f64(vu[d]);
-                    }
+    if (!rows) n_rows = (int64_t)B * N;
+    for (int64_t r_out = 0; r_out < n_rows; ++r_out)
+        for (int h = 0; h < H; ++h) {
+            int64_t row = rows ? rows[r_out] : r_out;
+            if (row < 0 || row >= (int64_t)B * N) return -3;
+            int b = (int)(row / N);
+            int64_t t = row - (int64_t)b * N;
+            int64_t i = t / block;
+            const int32_t* kb = kept + (((int64_t)b * H + h) * nb + i) * n_keep;
+            const uint16_t* qt = q + ((int64_t)b * N + t) * row_stride + (int64_t)h * hd;
+            int64_t n = 0;
+            double mx = -INFINITY;
+            for (int r = 0; r < n_keep; ++r) {
+                int64_t j = kb[r];
+                if (j < 0 || j >= nb) return -3;
+                int64_t u1 = (j + 1) * block < N ? (j + 1) * block : N;
+                for (int64_t u = j * block; u < u1; ++u) {
+                    const uint16_t* ku = k + ((int64_t)b * N + u) * row_stride + (int64_t)h * hd;
+                    double s = 0.0;
+                    for (int d = 0; d < hd; ++d)
+                        s += dito_bf16_to_f64(qt[d]) * dito_bf16_to_f64(ku[d]);
+                    s *= scale;
+                    work[n++] = s;
+                    if (s > mx) mx = s;
                 }
             }
+            double l = 0.0;
+            for (int64_t e = 0; e < n; ++e) {
+                work[e] = exp(work[e] - mx);
+                l += work[e];
+            }
+            double* ot = out + r_out * ((int64_t)H * hd) + (int64_t)h * hd;
+            for (int d = 0; d < hd; ++d) ot[d] = 0.0;
+            n = 0;
+            for (int r = 0; r < n_keep; ++r) {
+                int64_t j = kb[r];
+                int64_t u1 = (j + 1) * block < N ? (j + 1) * block : N;
+                for (int64_t u = j * block; u < u1; ++u) {
+                    const uint16_t* vu = v + ((int64_t)b * N + u) * row_stride + (int64_t)h * hd;
+                    double pw = work[n++] / l;
+                    for (int d = 0; d < hd; ++d) ot[d] += pw * dito_bf16_to_f64(vu[d]);
+                }
+            }
+        }
     return 0;
 }

@@ -62,7 +62,7 @@ MUTANTS = {
                                "for (int d = 0; d < hd; ++d) s += qm[i * hd + d] * qm[j * hd + d];"),
     "router_keep_floor": ("double want = ceil((1.0 - sparsity) * (double)n_blocks - 1e-9);",
                           "double want = floor((1.0 - sparsity) * (double)n_blocks);"),
-    "attn_scale_dropped": ("                        s *= scale;\n", "\n"),
+    "attn_scale_dropped": ("                    s *= scale;\n", "\n"),
     "attn_not_normalised": ("double pw = work[n++] / l;", "double pw = work[n++];"),
     "attn_values_from_k": ("const uint16_t* vu = v + ((int64_t)b * N + u) * row_stride",
                            "const uint16_t* vu = k + ((int64_t)b * N + u) * row_stride"),

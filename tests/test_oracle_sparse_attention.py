@@ -82,3 +82,14 @@ def test_samples_and_heads_are_independent(orc):
     out = orc.block_sparse_attention(q, k, v, B, H, hd, blk, kept)
     one = orc.block_sparse_attention(q[N:], k[N:], v[N:], 1, H, hd, blk, kept[1:])
     assert np.allclose(out[N:], one, rtol=0, atol=0)
+
+
+def test_row_selection(orc):
+    B, N, H, hd, blk = 2, 12, 2, 8, 4
+    q, k, v = _qkv(orc, 7, B, N, H, hd)
+    kept = np.array([[[[0], [2], [1]], [[1], [1], [0]]], [[[2], [0], [1]], [[0], [1], [2]]]],
+                    dtype=np.int32)
+    full = orc.block_sparse_attention(q, k, v, B, H, hd, blk, kept)
+    rows = np.array([23, 0, 13, 5])
+    part = orc.block_sparse_attention(q, k, v, B, H, hd, blk, kept, rows=rows)
+    assert np.array_equal(part, full[rows])
