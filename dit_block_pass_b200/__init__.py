@@ -26,7 +26,7 @@ __all__ = [
     "qk_rmsnorm_rope3d", "cachedit_workspace_bytes", "cachedit_residual_diff",
     "cachedit_residual_sums", "cachedit_decide", "cachedit_residual_diff_noalloc",
     "launch_counts", "QKOut", "CachePolicy", "swiglu_gemm", "gemm_gated_residual",
-    "subblock_keep_count", "subblock_router", "cachedit_residual_store",
+    "subblock_keep_count", "subblock_router", "block_sparse_attention", "cachedit_residual_store",
     "cachedit_residual_apply", "F32", "BF16", "ROPE_INTERLEAVED", "ROPE_HALF", "NORM_HEAD", "NORM_ROW",
 ]
 
@@ -46,7 +46,7 @@ launch_counts = {
     "cachedit_residual_diff": 2, "cachedit_residual_sums": 2, "cachedit_decide": 1,
     "cachedit_residual_diff_noalloc": 2, "cachedit_residual_store": 1,
     "cachedit_residual_apply": 1, "swiglu_gemm": 1, "gemm_gated_residual": 1,
-    "subblock_router": 2,
+    "subblock_router": 2, "block_sparse_attention": 1,
 }
 
 
@@ -105,6 +105,8 @@ def library() -> ctypes.CDLL:
                                                    dbl, dbl, i32, i32,
                                                    ctypes.POINTER(QKOut), vp]
             L.dit_swiglu_gemm.argtypes = [vp, vp, vp, i64, i32, i32, vp, vp]
+            L.dit_block_sparse_attention.argtypes = [vp, vp, vp, i64, vp, i64, i32, i64, i32,
+                                                     i32, i32, vp, i32, dbl, vp, vp]
             L.dit_subblock_keep_count.argtypes = [i64, dbl]
             L.dit_subblock_workspace_bytes.argtypes = [i32, i64, i32, i32, i32]
             L.dit_subblock_workspace_bytes.restype = sz
@@ -127,7 +129,7 @@ def library() -> ctypes.CDLL:
                          "dit_adaln_modulate_tok", "dit_gated_residual_adaln_tok",
                          "cachedit_residual_store", "cachedit_residual_apply", "dit_swiglu_gemm",
                          "dit_gemm_gated_residual", "dit_subblock_keep_count",
-                         "dit_subblock_router",
+                         "dit_subblock_router", "dit_block_sparse_attention",
                          "dit_cache_policy_init", "dit_cache_policy_decide",
                          "dit_qk_rmsnorm_rope3d", "dit_qk_rmsnorm_rope3d_ex",
                          "cachedit_residual_diff",
@@ -636,3 +638,39 @@ def subblock_router(q: torch.Tensor, k: torch.Tensor, heads: int, block: int = 1
           float(sparsity), kept.data_ptr(), workspace.data_ptr(),
           workspace.numel() * workspace.element_size(), _stream(q))
     return kept
+
+
+def block_sparse_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, heads: int,
+                           kept: torch.Tensor, scale: Optional[float] = None,
+                           out: Optional[torch.Tensor] = None,
+                           status: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Attention of every query block over its kept key blocks (blocks of
+    128 tokens, head size 128).  q, k, v: [B, N, H*128] views sharing one row
+    stride (e.g. slices of a fused qkv buffer); kept: int32 [B, H, n_blocks,
+    n_keep] from subblock_router.  Returns [B, N, H*128] bf16."""
+    for nm, t in (("q", q), ("k", k), ("v", v)):
+        _need_cuda_bf16(nm, t)
+    B, N, width = q.shape
+    if k.shape != q.shape or v.shape != q.shape or width % heads:
+        raise ValueError("q, k and v must be [B, N, H*hd] of the same shape")
+    hd = width // heads
+    rs = _token_rows("q", q, B, N, width)
+    if _token_rows("k", k, B, N, width) != rs or _token_rows("v", v, B, N, width) != rs:
+        raise ValueError("q, k and v must share the row stride")
+    if kept.dtype != torch.int32 or kept.dim() != 4 or not kept.is_contiguous() or \
+            kept.shape[:3] != (B, heads, (N + 127) // 128):
+        raise ValueError("kept must be a contiguous int32 [B, H, n_blocks, n_keep] tensor")
+    if out is None:
+        out = torch.empty(B, N, width, dtype=torch.bfloat16, device=q.device)
+    _need_cuda_bf16("out", out)
+    os_ = _token_rows("out", out, B, N, width)
+    if scale is None:
+        scale = hd ** -0.5
+    if status is not None and (status.dtype != torch.int32 or not status.is_cuda):
+        raise ValueError("status must be a CUDA int32 tensor")
+    if B * N == 0:
+        return out
+    _call("dit_block_sparse_attention", q.data_ptr(), k.data_ptr(), v.data_ptr(), rs,
+          out.data_ptr(), os_, B, N, heads, hd, 128, kept.data_ptr(), kept.shape[3],
+          float(scale), _ptr(status), _stream(q))
+    return out

@@ -1,0 +1,355 @@
+// sparse_attention.cu -- block-sparse attention over the SubBlock router's
+// kept key blocks, on the sm_100 tensor cores.
+//
+// The LMSYS report summary at news.cocoloop.cn ("minimax-h3-sglang-h200"),
+// section "Só com três camadas de aceleração somadas chega-se a 6 vezes":
+// SubBlock attention lets a block-sparse router cut the KV blocks that take
+// part in attention.  For token t of query block i and head h:
+//     out[t, h] = sum_u softmax_u(scale * q[t, h] . k[u, h]) v[u, h]
+// over the tokens u of the kept key blocks of (b, h, i); non-causal; blocks
+// of 128 tokens, head size 128.
+//
+// Design: one CTA of 6 warps per (query block, head, sample); S = Q K^T and
+// O = P V on the tensor cores with fp32 accumulators in TMEM (two S buffers
+// and O: 384 of 512 columns), online softmax on the CUDA cores:
+//   warp 0    TMA: the 128 x 128 Q tile once, then K and V tiles of each
+//             kept block into a 2-stage ring (128-byte swizzle).
+//   warp 1    one thread issues tcgen05.mma: S_n = Q K_n^T (K-major A and B)
+//             into S buffer n mod 2 as soon as K_n is in and that buffer was
+//             read, then O += P_{n-1} V_{n-1} (P from shared memory, K-major;
+//             V MN-major), so block n's scores overlap block n-1's softmax.
+//   warps 2-5 softmax, thread = query row (TMEM lane): tcgen05.ld the S row,
+//             running max and sum in the exp2 domain, masking keys past the
+//             sample's last token; after the previous P V has finished, the
+//             O row is rescaled in TMEM (tcgen05.ld / st) when its max moved,
+//             and P is written as bf16 into shared memory in the tensor
+//             cores' 128-byte swizzled K-major layout.  At the end O / l is
+//             written as bf16.
+// Every mbarrier wait is bounded (tcgen05.cuh); on expiry the CTA records an
+// error in the caller's status word and exits after freeing its TMEM.
+#include "tcgen05.cuh"
+
+namespace dit {
+namespace {
+
+using namespace tc;
+
+constexpr int kBlk = 128;                       // tokens per block (rows of every tile)
+constexpr int kHd = 128;                        // head size
+constexpr int kThreadsA = 192;
+constexpr uint32_t kTile = kBlk * kHd * 2;      // 32 KB: one 128 x 128 bf16 tile
+constexpr uint32_t kHalfTile = kTile / 2;       // 16 KB: 64 columns (one swizzle atom wide)
+constexpr uint32_t kTmemColsA = 512;
+constexpr uint32_t kColO = 256;                 // O in TMEM columns [256, 384)
+// Q, 2 x (K, V), P, then barriers
+constexpr size_t kSmemA = 6 * kTile + 1024 + 256;
+constexpr uint32_t kIdescS = idesc_f16(128, 128, false, false);    // S = Q K^T
+constexpr uint32_t kIdescO = idesc_f16(128, 128, false, true);     // O += P V (V MN-major)
+
+struct AttnParams {
+    const int32_t* kept;        // [B, H, nb, n_keep]
+    uint16_t* out;
+    int64_t out_stride;         // elements between output rows
+    int* status;
+    int64_t N;
+    int H, nb, n_keep;
+    float scale_log2;           // scale * log2(e)
+};
+
+__global__ void __launch_bounds__(kThreadsA, 1)
+block_sparse_attention_kernel(const __grid_constant__ CUtensorMap map_q,
+                              const __grid_constant__ CUtensorMap map_k,
+                              const __grid_constant__ CUtensorMap map_v, AttnParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_u32(smem_raw);
+    const uint32_t base = (raw + 1023u) & ~1023u;
+    uint8_t* gen_base = smem_raw + (base - raw);
+    const uint32_t sQ = base;
+    const uint32_t sK0 = base + kTile;              // stage s: K at sK0 + s * 2 * kTile
+    const uint32_t sP = base + 5 * kTile;
+    uint8_t* gP = gen_base + 5 * kTile;
+    const uint32_t bar = base + 6 * kTile;
+    const uint32_t bar_q = bar;                     // Q landed
+    const uint32_t bar_kv_full = bar + 8;           // [2]
+    const uint32_t bar_kv_empty = bar + 24;         // [2]
+    const uint32_t bar_s_full = bar + 40;           // [2]
+    const uint32_t bar_s_free = bar + 56;           // [2], 4 arrivals
+    const uint32_t bar_p_full = bar + 72;           // 4 arrivals
+    const uint32_t bar_o_done = bar + 80;
+    const uint32_t bar_drain = bar + 88;
+    volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(gen_base + 6 * kTile + 96);
+    volatile int* abort = reinterpret_cast<volatile int*>(gen_base + 6 * kTile + 100);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int i = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+    const int nk = p.n_keep;
+    const int32_t* kept = p.kept + ((static_cast<int64_t>(b) * p.H + h) * p.nb + i) * nk;
+    const int row0 = static_cast<int>(static_cast<int64_t>(b) * p.N);   // first row of the sample
+
+    if (threadIdx.x == 0) {
+        mbar_init(bar_q, 1);
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(bar_kv_full + 8 * s, 1);
+            mbar_init(bar_kv_empty + 8 * s, 1);
+            mbar_init(bar_s_full + 8 * s, 1);
+            mbar_init(bar_s_free + 8 * s, 4);
+        }
+        mbar_init(bar_p_full, 4);
+        mbar_init(bar_o_done, 1);
+        mbar_init(bar_drain, 1);
+        *abort = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == 1) tmem_alloc(smem_u32(const_cast<uint32_t*>(tmem_slot)), kTmemColsA);
+    fence_before_sync();
+    __syncthreads();
+    fence_after_sync();
+    const uint32_t tmem = *tmem_slot;
+    bool failed = false;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            // the Q tile, then K and V of every kept block
+            const int col = h * kHd;
+            mbar_expect_tx(bar_q, kTile);
+            tma_load_2d(sQ, &map_q, bar_q, col, row0 + i * kBlk);
+            tma_load_2d(sQ + kHalfTile, &map_q, bar_q, col + 64, row0 + i * kBlk);
+            int issued = 0;
+            for (int n = 0; n < nk; ++n) {
+                const int s = n & 1;
+                if (!mbar_wait(bar_kv_empty + 8 * s, ((n >> 1) & 1) ^ 1, abort)) {
+                    failed = true;
+                    break;
+                }
+                const int row = row0 + __ldg(kept + n) * kBlk;
+                const uint32_t sk = sK0 + s * 2 * kTile, sv = sk + kTile;
+                const uint32_t fb = bar_kv_full + 8 * s;
+                mbar_expect_tx(fb, 2 * kTile);
+                tma_load_2d(sk, &map_k, fb, col, row);
+                tma_load_2d(sk + kHalfTile, &map_k, fb, col + 64, row);
+                tma_load_2d(sv, &map_v, fb, col, row);
+                tma_load_2d(sv + kHalfTile, &map_v, fb, col + 64, row);
+                issued = n + 1;
+            }
+            mbar_wait(bar_q, 0, abort);
+            if (failed) {
+                for (int n = issued > 2 ? issued - 2 : 0; n < issued; ++n)
+                    mbar_wait(bar_kv_full + 8 * (n & 1), (n >> 1) & 1, abort);
+            }
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        if (lane == 0) {
+            // S_n = Q K_n^T, then O += P_{n-1} V_{n-1}
+            if (!mbar_wait(bar_q, 0, abort)) failed = true;
+            for (int n = 0; n <= nk && !failed; ++n) {
+                if (n < nk) {
+                    const int s = n & 1;
+                    if (!mbar_wait(bar_kv_full + 8 * s, (n >> 1) & 1, abort) ||
+                        (n >= 2 && !mbar_wait(bar_s_free + 8 * s, ((n - 2) >> 1) & 1, abort))) {
+                        failed = true;
+                        break;
+                    }
+                    fence_after_sync();
+                    const uint32_t sk = sK0 + s * 2 * kTile;
+#pragma unroll
+                    for (int kk = 0; kk < kHd / 16; ++kk) {
+                        const uint32_t off = (kk >> 2) * kHalfTile + (kk & 3) * 32;
+                        mma_f16(tmem + 128u * s, sw128_desc(sQ + off), sw128_desc(sk + off),
+                                kIdescS, kk != 0 ? 1u : 0u);
+                    }
+                    mma_commit(bar_s_full + 8 * s);
+                }
+                if (n >= 1) {
+                    const int m = n - 1;
+                    if (!mbar_wait(bar_p_full, m & 1, abort)) {
+                        failed = true;
+                        break;
+                    }
+                    fence_after_sync();
+                    const uint32_t sv = sK0 + (m & 1) * 2 * kTile + kTile;
+#pragma unroll
+                    for (int kk = 0; kk < kBlk / 16; ++kk) {
+                        // A: P, K-major over keys; B: V, MN-major (d contiguous),
+                        // 16 keys = two 8-row groups per step
+                        const uint32_t pa = sP + (kk >> 2) * kHalfTile + (kk & 3) * 32;
+                        mma_f16(tmem + kColO, sw128_desc(pa), sw128_desc_mn(sv + kk * 2048, kHalfTile),
+                                kIdescO, (m | kk) != 0 ? 1u : 0u);
+                    }
+                    mma_commit(bar_o_done);
+                    mma_commit(bar_kv_empty + 8 * (m & 1));
+                }
+            }
+            if (failed) {
+                mma_commit(bar_drain);
+                mbar_wait(bar_drain, 0, abort);
+            }
+        }
+        __syncwarp();
+    } else {
+        // softmax: thread = query row r (TMEM lane)
+        const int q = warp & 3;
+        const int r = 32 * q + lane;
+        const uint32_t lane_off = static_cast<uint32_t>(32 * q) << 16;
+        float m_run = -INFINITY, l_run = 0.0f;
+        for (int n = 0; n < nk; ++n) {
+            const int s = n & 1;
+            if (!mbar_wait(bar_s_full + 8 * s, (n >> 1) & 1, abort)) {
+                failed = true;
+                break;
+            }
+            fence_after_sync();
+            float sc[kBlk];
+#pragma unroll
+            for (int c = 0; c < kBlk / 32; ++c)
+                tmem_ld32(tmem + lane_off + 128u * s + 32 * c,
+                          *reinterpret_cast<float(*)[32]>(sc + 32 * c));
+            tmem_wait_ld();
+            fence_before_sync();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar_s_free + 8 * s);
+            // keys past the sample's last token do not take part
+            const int64_t j = __ldg(kept + n);
+            const int64_t left = p.N - j * kBlk;
+            const int valid = left >= kBlk ? kBlk : (left > 0 ? static_cast<int>(left) : 0);
+            float mx = m_run;
+#pragma unroll
+            for (int c = 0; c < kBlk; ++c) {
+                sc[c] = c < valid ? sc[c] * p.scale_log2 : -INFINITY;
+                mx = fmaxf(mx, sc[c]);
+            }
+            const float alpha = exp2f(m_run - mx);      // 0 on the first block
+            float sum = 0.0f;
+#pragma unroll
+            for (int c = 0; c < kBlk; ++c) {
+                sc[c] = exp2f(sc[c] - mx);
+                sum += sc[c];
+            }
+            l_run = l_run * alpha + sum;
+            m_run = mx;
+            if (n >= 1) {
+                // the previous P V is done: P is free and O holds the sum so far
+                if (!mbar_wait(bar_o_done, (n - 1) & 1, abort)) {
+                    failed = true;
+                    break;
+                }
+                fence_after_sync();
+                if (__any_sync(0xffffffffu, alpha != 1.0f)) {
+#pragma unroll 1
+                    for (int c = 0; c < kHd / 32; ++c) {
+                        float o[32];
+                        tmem_ld32(tmem + lane_off + kColO + 32 * c, o);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) o[e] *= alpha;
+                        tmem_st32(tmem + lane_off + kColO + 32 * c, o);
+                    }
+                    tmem_wait_st();
+                }
+            }
+            // P row r as bf16, K-major with the 128-byte swizzle: keys
+            // [64a, 64a + 64) in atom a, 16-byte chunk c of the row at chunk
+            // c ^ (r mod 8)
+#pragma unroll
+            for (int a = 0; a < 2; ++a) {
+                uint8_t* rowp = gP + a * kHalfTile + r * 128;
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    float f[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) f[e] = sc[64 * a + 8 * c + e];
+                    *reinterpret_cast<uint4*>(rowp + ((c ^ (r & 7)) << 4)) = pack8(f);
+                }
+            }
+            fence_proxy_async_smem();
+            fence_before_sync();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar_p_full);
+        }
+        if (!failed && nk > 0) {
+            if (!mbar_wait(bar_o_done, (nk - 1) & 1, abort)) {
+                failed = true;
+            } else {
+                fence_after_sync();
+                const int64_t tok = static_cast<int64_t>(i) * kBlk + r;
+                const float inv_l = 1.0f / l_run;
+#pragma unroll 1
+                for (int c = 0; c < kHd / 32; ++c) {
+                    float o[32];
+                    tmem_ld32(tmem + lane_off + kColO + 32 * c, o);
+                    tmem_wait_ld();
+                    if (tok < p.N) {
+                        uint16_t* dst = p.out + (row0 + tok) * p.out_stride + h * kHd + 32 * c;
+#pragma unroll
+                        for (int v = 0; v < 4; ++v) {
+                            float f[8];
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) f[e] = o[8 * v + e] * inv_l;
+                            *reinterpret_cast<uint4*>(dst + 8 * v) = pack8(f);
+                        }
+                    }
+                }
+            }
+        }
+    }
+    if (failed) {
+        *abort = 1;
+        if (p.status) atomicExch(p.status, 1);
+    }
+    fence_before_sync();
+    __syncthreads();
+    fence_after_sync();
+    if (warp == 1) tmem_dealloc(tmem, kTmemColsA);
+}
+
+}  // namespace
+}  // namespace dit
+
+extern "C" int dit_block_sparse_attention(const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                                          int64_t row_stride, uint16_t* out, int64_t out_stride,
+                                          int B, int64_t N, int H, int hd, int block,
+                                          const int32_t* kept, int n_keep, double scale,
+                                          int* status, void* stream) {
+    using namespace dit;
+    if (B < 0 || N < 0 || H < 1 || n_keep < 1) return DIT_ERR_SHAPE;
+    if (hd != kHd || block != kBlk) return DIT_ERR_SHAPE;
+    const int64_t D = static_cast<int64_t>(H) * hd;
+    if (row_stride < D || out_stride < D) return DIT_ERR_SHAPE;
+    if (row_stride % 8 || out_stride % 8) return DIT_ERR_ALIGN;
+    if (!(scale > 0.0) || scale > 1e30) return DIT_ERR_VALUE;
+    if (B == 0 || N == 0) return DIT_OK;
+    const int64_t nb = (N + kBlk - 1) / kBlk;
+    if (n_keep > nb || B > 65535 || H > 65535) return DIT_ERR_SHAPE;
+    const int64_t rows = static_cast<int64_t>(B) * N;
+    if (rows + kBlk > 0x7FFFFFFF) return DIT_ERR_SHAPE;
+    if (!q || !k || !v || !out || !kept) return DIT_ERR_NULL;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) ||
+        reinterpret_cast<uintptr_t>(kept) % 4)
+        return DIT_ERR_ALIGN;
+    if (status && reinterpret_cast<uintptr_t>(status) % 4) return DIT_ERR_ALIGN;
+    const size_t ob = static_cast<size_t>(rows - 1) * out_stride * 2 + D * 2;
+    const size_t ib = static_cast<size_t>(rows - 1) * row_stride * 2 + D * 2;
+    if (overlaps(out, ob, q, ib) || overlaps(out, ob, k, ib) || overlaps(out, ob, v, ib))
+        return DIT_ERR_OVERLAP;
+    CUtensorMap mq, mk, mv;
+    if (!make_map(&mq, q, rows, D, row_stride) || !make_map(&mk, k, rows, D, row_stride) ||
+        !make_map(&mv, v, rows, D, row_stride))
+        return DIT_ERR_LAUNCH;
+    AttnParams p{};
+    p.kept = kept;
+    p.out = out;
+    p.out_stride = out_stride;
+    p.status = status;
+    p.N = N;
+    p.H = H;
+    p.nb = static_cast<int>(nb);
+    p.n_keep = n_keep;
+    p.scale_log2 = static_cast<float>(scale * 1.4426950408889634);
+    if (cudaFuncSetAttribute(block_sparse_attention_kernel,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(kSmemA)) != cudaSuccess)
+        return DIT_ERR_LAUNCH;
+    block_sparse_attention_kernel<<<dim3(static_cast<unsigned>(nb), H, B), kThreadsA, kSmemA,
+                                    as_stream(stream)>>>(mq, mk, mv, p);
+    return launch_status();
+}

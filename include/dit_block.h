@@ -346,6 +346,30 @@ int dit_subblock_router(const uint16_t* q, const uint16_t* k, int64_t row_stride
                         void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * Block-sparse attention over the router's kept key blocks (tensor cores):
+ * for token t of query block i, head h,
+ *     out[t, h] = sum_u softmax_u(scale * q[t, h] . k[u, h]) v[u, h]
+ * over the tokens u of the key blocks kept[b, h, i, 0..n_keep) of the same
+ * sample (as returned by dit_subblock_router); non-causal.
+ *   q, k, v     device rows of B*N tokens, row_stride elements apart (a fused
+ *               qkv buffer works), H heads of hd = 128; 16-byte aligned.
+ *   out         device rows, out_stride elements apart, H*128 wide; must not
+ *               overlap q, k or v.
+ *   block       128 (the tile height); n_keep <= n_blocks.
+ *   kept        device int32 [B, H, n_blocks, n_keep]; an index outside
+ *               [0, n_blocks) contributes no keys (its rows may come out NaN).
+ *   scale       the softmax scale, e.g. 1/sqrt(128).
+ * S = Q K^T and O = P V run on tcgen05 with fp32 accumulators; the softmax
+ * is fp32 in the exp2 domain and P enters the second product as bf16.
+ * status as for dit_swiglu_gemm.
+ */
+int dit_block_sparse_attention(const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                               int64_t row_stride, uint16_t* out, int64_t out_stride,
+                               int B, int64_t N, int H, int hd, int block,
+                               const int32_t* kept, int n_keep, double scale,
+                               int* status, void* stream);
+
+/*
  * Cache-DiT step cache.  The LMSYS report (news.cocoloop.cn,
  * "minimax-h3-sglang-h200", section "Só com três camadas de aceleração
  * somadas chega-se a 6 vezes") reuses results cached between neighbouring
