@@ -428,6 +428,39 @@ def time_subblock_router(chain, steps, warmup, world):
     return a.elapsed_time(b) / steps, nb, n_keep
 
 
+def time_sparse_attention(chain, steps, world):
+    """SubBlock attention on the clip's q, k, v at sparsity 0.75: the kept
+    lists from the router, then the block-sparse attention (tcgen05); the
+    dense attention of the library (torch scaled_dot_product_attention) for
+    context.  Returns (sparse ms, dense ms, kept blocks, key blocks)."""
+    import torch
+    import dit_block_pass_b200 as dbp
+    c, wl = chain, chain.wl
+    D, H = wl.D, wl.H
+    q, k, v = c.qkv[:, :, :D], c.qkv[:, :, D:2 * D], c.qkv[:, :, 2 * D:]
+    kept = dbp.subblock_router(q, k, H, 128, 0.75)
+    out = torch.empty(wl.B, wl.N, D, dtype=torch.bfloat16, device=c.dev)
+    st = torch.zeros(1, dtype=torch.int32, device=c.dev)
+    qh, kh, vh = (t.reshape(wl.B, wl.N, H, wl.hd).transpose(1, 2) for t in (q, k, v))
+    ops = {"sparse": lambda: dbp.block_sparse_attention(q, k, v, H, kept, out=out, status=st),
+           "dense": lambda: torch.nn.functional.scaled_dot_product_attention(qh, kh, vh)}
+    stream = torch.cuda.current_stream()
+    res = {}
+    for name, op in ops.items():
+        op()
+        barrier_sync(world)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(steps):
+            op()
+        b.record(stream)
+        barrier_sync(world)
+        res[name] = a.elapsed_time(b) / steps
+    if int(st.item()) != 0:
+        raise RuntimeError("block_sparse_attention reported an expired pipeline wait")
+    return res["sparse"], res["dense"], kept.shape[3], kept.shape[2]
+
+
 def tensor_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -607,6 +640,8 @@ def main():
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--config", default="h3_5s")
     ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--attn-steps", type=int, default=3,
+                    help="timed launches of the block-sparse attention and of dense attention")
     ap.add_argument("--gemm-steps", type=int, default=10,
                     help="timed launches of the fused up-projection and of its unfused chain")
     ap.add_argument("--no-e2e", action="store_true")
@@ -643,6 +678,8 @@ def main():
         gemm_ms = time_swiglu_gemm(chain, args.gemm_steps, 2, world)
         router_ms, router_nb, router_keep = time_subblock_router(chain, args.steps, args.warmup,
                                                                  world)
+        attn_ms, dense_ms, attn_keep, attn_nb = time_sparse_attention(chain, args.attn_steps,
+                                                                      world)
     finally:
         if sampler:
             sampler.__exit__(None, None, None)
@@ -695,6 +732,15 @@ def main():
     subblock = {"ms": round(router_ms, 4), "GB/s": round(router_gbs, 1),
                 "frac_of_peak": round(router_gbs / peak, 4), "block": 128, "sparsity": 0.75,
                 "key_blocks": router_nb, "kept_per_query_block": router_keep}
+    attn_ms = max_over_ranks(attn_ms, world)
+    dense_ms = max_over_ranks(dense_ms, world)
+    attn_tflop = 4.0 * 128 ** 3 * attn_nb * attn_keep * wl.H * wl.B / 1e12
+    sparse_attention = {"kernel": "block_sparse_attention_kernel (tcgen05)", "ms": round(attn_ms, 3),
+                        "TFLOP/s": round(attn_tflop / (attn_ms / 1000.0), 1), "bound": "tensor",
+                        "frac_of_burst_peak": round(attn_tflop / (attn_ms / 1000.0) / burst, 4),
+                        "sparsity": 0.75, "kept_blocks": attn_keep, "key_blocks": attn_nb,
+                        "dense_library_ms (torch scaled_dot_product_attention)": round(dense_ms, 3),
+                        "speedup_vs_dense": round(dense_ms / attn_ms, 3)}
     dom_ms = per_op[OPS.index(DOMINANT)]
     achieved = nbytes[DOMINANT] / (dom_ms / 1000.0) / 1e9
     tr = NCU_TRAFFIC.get(DOMINANT)
@@ -735,6 +781,7 @@ def main():
                        "parallelism": f"{world} independent clip(s), one per GPU"},
             "ops": ops, "qk_options": qk_options, "token_sets": token_sets,
             "cache_step": cache_step, "swiglu_gemm": swiglu_gemm, "subblock_router": subblock,
+            "sparse_attention": sparse_attention,
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": chain.launches_per_step() * args.steps, "clocks": clocks,
         }

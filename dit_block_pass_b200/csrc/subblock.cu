@@ -15,13 +15,14 @@
 //                           sums the rows of block j of sample b of tensor t
 //                           (q or k) for every column, 16-byte loads, fp32,
 //                           and writes the means [B, 2, n_blocks, H*hd].
-//   subblock_select_kernel  CTA (query-block group, h, b): the group's query
-//                           means in shared memory, one pass over the key
-//                           means of head h (L2 resident) for all scores,
-//                           then per query block a bitonic sort of 64-bit
-//                           keys (order-preserving score bits, then the
-//                           inverted block index) and a second, ascending
-//                           sort of the n_keep winners' indices.
+//   subblock_select_kernel  CTA (up to 8 query blocks, h, b): the query means
+//                           in shared memory, one pass over the key means of
+//                           head h (L2 resident) for all scores, then one
+//                           warp per query block: a radix select of the
+//                           n_keep-th largest score (four 8-bit histogram
+//                           passes) and an ordered ballot compaction that
+//                           writes the kept indices in increasing order,
+//                           ties at the threshold to the lower index.
 #include <cmath>
 
 #include "common.cuh"
@@ -79,42 +80,75 @@ __device__ __forceinline__ uint32_t ordered(float f) {
     return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
-// Bitonic sort of n (a power of two) 64-bit keys in shared memory by the
-// whole CTA, descending or ascending.
-__device__ __forceinline__ void bitonic(unsigned long long* keys, int n, bool descending) {
-    for (int size = 2; size <= n; size <<= 1) {
-        for (int stride = size >> 1; stride > 0; stride >>= 1) {
-            for (int e = threadIdx.x; e < n / 2; e += kSelThreads) {
-                const int lo = 2 * e - (e & (stride - 1));
-                const int hi = lo + stride;
-                // sub-sequences alternate direction; the last merge goes the
-                // requested way
-                const bool first = ((lo & size) == 0) == descending;
-                const unsigned long long a = keys[lo], c = keys[hi];
-                if (first ? (a < c) : (a > c)) {
-                    keys[lo] = c;
-                    keys[hi] = a;
-                }
-            }
-            __syncthreads();
+// One warp picks one query block's kept key blocks from its fp32 scores
+// sc[0..nb) in shared memory: four 8-bit histogram passes over the
+// order-preserving score codes find the n_keep-th largest code T, then the
+// kept indices -- every code above T and the lowest-index ties at T -- are
+// written in increasing order with ballots.  Same order as sorting (score
+// descending, index ascending) and taking the first n_keep.
+__device__ void warp_select(const float* sc, int nb, int n_keep, unsigned* hist, int32_t* out,
+                            int lane) {
+    uint32_t prefix = 0, mask = 0;
+    int need = n_keep;              // keys still wanted among those matching the prefix
+    for (int pass = 0; pass < 4; ++pass) {
+        const int shift = 24 - 8 * pass;
+        for (int e = lane; e < 256; e += 32) hist[e] = 0;
+        __syncwarp();
+        for (int j = lane; j < nb; j += 32) {
+            const uint32_t c = ordered(sc[j]);
+            if ((c & mask) == prefix) atomicAdd(&hist[(c >> shift) & 255u], 1u);
         }
+        __syncwarp();
+        int digit = 0, above = 0;
+        if (lane == 0) {
+            // from the top digit down, the first bin that reaches `need`
+            int acc = 0, d = 255;
+            for (; d > 0; --d) {
+                const int cnt = static_cast<int>(hist[d]);
+                if (acc + cnt >= need) break;
+                acc += cnt;
+            }
+            digit = d;
+            above = acc;
+        }
+        digit = __shfl_sync(0xffffffffu, digit, 0);
+        above = __shfl_sync(0xffffffffu, above, 0);
+        need -= above;
+        prefix |= static_cast<uint32_t>(digit) << shift;
+        mask |= 255u << shift;
+        __syncwarp();
+    }
+    // prefix is T; `need` ties at T are taken, lowest indices first
+    int written = 0, eq_seen = 0;
+    const unsigned below = (1u << lane) - 1u;
+    for (int j0 = 0; j0 < nb; j0 += 32) {
+        const int j = j0 + lane;
+        const uint32_t c = j < nb ? ordered(sc[j]) : 0u;
+        const bool gt = j < nb && c > prefix;
+        const bool eq = j < nb && c == prefix;
+        const unsigned eqm = __ballot_sync(0xffffffffu, eq);
+        const bool take = gt || (eq && eq_seen + __popc(eqm & below) < need);
+        const unsigned tm = __ballot_sync(0xffffffffu, take);
+        if (take) out[written + __popc(tm & below)] = j;
+        written += __popc(tm);
+        eq_seen += __popc(eqm);
     }
 }
 
-// CTA (g, h, b): query blocks i = g*QB .. g*QB + QB - 1 of head h, sample b.
-// Shared memory: qmean [QB][hd] fp32, scores [QB][nb_pad] fp32, keys
-// [nb_pad] u64.
+// CTA (g, h, b): query blocks i = g*QB .. g*QB + QB - 1 of head h, sample b;
+// all 8 warps compute the scores, then warp r selects query block r.
+// Shared memory: qmean [QB][hd] fp32, scores [QB][nb] fp32, 256-bin
+// histograms [8].
 __global__ void __launch_bounds__(kSelThreads)
-subblock_select_kernel(const float* __restrict__ pooled, int nb, int nb_pad, int D, int hd,
-                       int QB, int n_keep, int keep_pad, int32_t* __restrict__ kept) {
+subblock_select_kernel(const float* __restrict__ pooled, int nb, int D, int hd, int QB,
+                       int n_keep, int32_t* __restrict__ kept) {
     extern __shared__ __align__(16) unsigned char sm[];
     const int h = blockIdx.y, b = blockIdx.z;
     const int i0 = blockIdx.x * QB;
     const int nq = min(QB, nb - i0);
     float* qmean = reinterpret_cast<float*>(sm);                       // QB * hd
-    float* scores = qmean + QB * hd;                                   // QB * nb_pad
-    unsigned long long* keys =
-        reinterpret_cast<unsigned long long*>(scores + static_cast<int64_t>(QB) * nb_pad);
+    float* scores = qmean + QB * hd;                                   // QB * nb
+    unsigned* hist = reinterpret_cast<unsigned*>(scores + static_cast<int64_t>(QB) * nb);
     const float* qsrc = pooled + (static_cast<int64_t>(b) * 2 + 0) * nb * D + h * hd;
     const float* ksrc = pooled + (static_cast<int64_t>(b) * 2 + 1) * nb * D + h * hd;
     for (int e = threadIdx.x; e < nq * hd; e += kSelThreads) {
@@ -126,13 +160,13 @@ subblock_select_kernel(const float* __restrict__ pooled, int nb, int nb_pad, int
     // fp32, d in increasing order
     for (int j = threadIdx.x; j < nb; j += kSelThreads) {
         const float4* kv = reinterpret_cast<const float4*>(ksrc + static_cast<int64_t>(j) * D);
-        float acc[16];
+        float acc[8];
 #pragma unroll
-        for (int r = 0; r < 16; ++r) acc[r] = 0.0f;
+        for (int r = 0; r < 8; ++r) acc[r] = 0.0f;
         for (int d4 = 0; d4 < hd / 4; ++d4) {
             const float4 kk = __ldg(kv + d4);
 #pragma unroll
-            for (int r = 0; r < 16; ++r) {
+            for (int r = 0; r < 8; ++r) {
                 if (r < nq) {
                     const float* qm = qmean + r * hd + 4 * d4;
                     acc[r] = __fmaf_rn(qm[0], kk.x, acc[r]);
@@ -143,38 +177,16 @@ subblock_select_kernel(const float* __restrict__ pooled, int nb, int nb_pad, int
             }
         }
 #pragma unroll
-        for (int r = 0; r < 16; ++r)
-            if (r < nq) scores[static_cast<int64_t>(r) * nb_pad + j] = acc[r];
+        for (int r = 0; r < 8; ++r)
+            if (r < nq) scores[static_cast<int64_t>(r) * nb + j] = acc[r];
     }
     __syncthreads();
-    for (int r = 0; r < nq; ++r) {
-        // keys: score bits, then the inverted index, so that a descending
-        // sort puts equal scores in increasing index order; padding sorts last
-        for (int j = threadIdx.x; j < nb_pad; j += kSelThreads) {
-            keys[j] = j < nb ? (static_cast<unsigned long long>(
-                                    ordered(scores[static_cast<int64_t>(r) * nb_pad + j]))
-                                << 32) |
-                                   (0xFFFFFFFFu - static_cast<uint32_t>(j))
-                             : 0ull;
-        }
-        __syncthreads();
-        bitonic(keys, nb_pad, true);
-        // the kept block indices, then sorted ascending (padding last)
-        unsigned long long idx[kMaxBlocks / kSelThreads];
-        int c = 0;
-        for (int e = threadIdx.x; e < keep_pad; e += kSelThreads, ++c)
-            idx[c] = e < n_keep ? static_cast<unsigned long long>(
-                                      0xFFFFFFFFu - static_cast<uint32_t>(keys[e] & 0xFFFFFFFFull))
-                                : ~0ull;
-        __syncthreads();
-        c = 0;
-        for (int e = threadIdx.x; e < keep_pad; e += kSelThreads, ++c) keys[e] = idx[c];
-        __syncthreads();
-        bitonic(keys, keep_pad, false);
-        int32_t* out = kept + ((static_cast<int64_t>(b) * gridDim.y + h) * nb + i0 + r) * n_keep;
-        for (int e = threadIdx.x; e < n_keep; e += kSelThreads)
-            out[e] = static_cast<int32_t>(keys[e]);
-        __syncthreads();
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (warp < nq) {
+        int32_t* out =
+            kept + ((static_cast<int64_t>(b) * gridDim.y + h) * nb + i0 + warp) * n_keep;
+        warp_select(scores + static_cast<int64_t>(warp) * nb, nb, n_keep, hist + 256 * warp, out,
+                    lane);
     }
 }
 
@@ -185,12 +197,6 @@ int keep_count(int64_t n_blocks, double sparsity) {
     if (keep < 1) keep = 1;
     if (keep > n_blocks) keep = n_blocks;
     return static_cast<int>(keep);
-}
-
-int pad_pow2(int n) {
-    int p = 1;
-    while (p < n) p <<= 1;
-    return p;
 }
 
 }  // namespace
@@ -234,17 +240,15 @@ extern "C" int dit_subblock_router(const uint16_t* q, const uint16_t* k, int64_t
         block, nb, static_cast<int>(D / 8), pooled);
     int rc = launch_status();
     if (rc) return rc;
-    const int nb_pad = pad_pow2(nb);
-    const int keep_pad = pad_pow2(n_keep);
-    // query blocks per CTA: as many as fit in about 96 KB of scores (<= 16)
-    int QB = 16;
-    while (QB > 1 && static_cast<size_t>(QB) * nb_pad * 4 > 96 * 1024) QB >>= 1;
-    const size_t smem = static_cast<size_t>(QB) * hd * 4 + static_cast<size_t>(QB) * nb_pad * 4 +
-                        static_cast<size_t>(nb_pad) * 8;
+    // query blocks per CTA (one per warp): as many as fit in about 96 KB of scores
+    int QB = 8;
+    while (QB > 1 && static_cast<size_t>(QB) * nb * 4 > 96 * 1024) QB >>= 1;
+    const size_t smem = static_cast<size_t>(QB) * hd * 4 + static_cast<size_t>(QB) * nb * 4 +
+                        8 * 256 * sizeof(unsigned);
     if (cudaFuncSetAttribute(subblock_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(smem)) != cudaSuccess)
         return DIT_ERR_LAUNCH;
     subblock_select_kernel<<<dim3((nb + QB - 1) / QB, H, B), kSelThreads, smem, st>>>(
-        pooled, nb, nb_pad, static_cast<int>(D), hd, QB, n_keep, keep_pad, kept);
+        pooled, nb, static_cast<int>(D), hd, QB, n_keep, kept);
     return launch_status();
 }
