@@ -92,6 +92,7 @@ struct GemmParams {
     int cols;               // output columns (F, or D)
     int tiles_m, tiles_n, tiles;
     int b1_offset;          // row of the second W box relative to the first (0: own map)
+    int stall;              // test hook: the producer issues nothing, every wait runs out
     // gated residual
     const uint16_t* x;      // [M, cols] residual stream (may be out)
     const void* gate;       // [B, cols] per-sample gate, fp32 or bf16
@@ -200,7 +201,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap map_x,
         if (lane == 0) {
             // producer: K steps of every tile, through the ring
             uint32_t it = 0;
-            for (int t = blockIdx.x; t < p.tiles && !failed; t += gridDim.x) {
+            for (int t = blockIdx.x; t < p.tiles && !failed && !p.stall; t += gridDim.x) {
                 int m0, n0;
                 tile_coords<EPI>(p, t, m0, n0);
                 for (int kb = 0; kb < nk; ++kb, ++it) {
@@ -429,6 +430,22 @@ extern "C" int dit_swiglu_gemm(const uint16_t* x, const uint16_t* w, uint16_t* o
     p.out = out;
     p.status = status;
     p.b1_offset = 0;
+    return launch_gemm<kSwiGLU>(x, w, F, w + static_cast<int64_t>(F) * K, F, p, M, K, F, stream);
+}
+
+extern "C" int dit_swiglu_gemm_stall_test(const uint16_t* x, const uint16_t* w, uint16_t* out,
+                                          int64_t M, int K, int F, int* status, void* stream) {
+    using namespace dit;
+    if (M <= 0 || M > 4096 || K <= 0 || K > 4096 || F <= 0 || F > 4096) return DIT_ERR_SHAPE;
+    if (K % 8 || F % 8) return DIT_ERR_ALIGN;
+    if (!x || !w || !out || !status) return DIT_ERR_NULL;
+    if (!aligned16(x) || !aligned16(w) || !aligned16(out) ||
+        reinterpret_cast<uintptr_t>(status) % 4)
+        return DIT_ERR_ALIGN;
+    GemmParams p{};
+    p.out = out;
+    p.status = status;
+    p.stall = 1;
     return launch_gemm<kSwiGLU>(x, w, F, w + static_cast<int64_t>(F) * K, F, p, M, K, F, stream);
 }
 

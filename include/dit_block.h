@@ -297,6 +297,16 @@ int dit_swiglu_gemm(const uint16_t* x, const uint16_t* w, uint16_t* out, int64_t
                     int* status, void* stream);
 
 /*
+ * Test hook for the failure path of the tensor-core kernels: the same launch
+ * as dit_swiglu_gemm with its copy warp disabled, so that every pipeline wait
+ * runs out (after about 2 s) and the kernel writes 1 to *status, frees its
+ * tensor memory and returns, leaving the context usable.  Small shapes only
+ * (M, K, F <= 4096); status is required.  Not for production use.
+ */
+int dit_swiglu_gemm_stall_test(const uint16_t* x, const uint16_t* w, uint16_t* out, int64_t M,
+                               int K, int F, int* status, void* stream);
+
+/*
  * The gated residual fused into the down-projection GEMM (tensor cores):
  *     x_out[m, n] = bf16(x[m, n] + gate_b[n] * sum_k h[m, k] w[n, k])
  * a2's residual update with its branch taken straight from the product, so

@@ -210,3 +210,25 @@ def test_down_projection_full_size_sampled_rows(orc):
                  out[0, idx].cpu(), rows, what="h3_5s rows")
     del h, w, x, out
     torch.cuda.empty_cache()
+
+
+def test_an_expired_wait_is_reported_and_the_context_survives(orc):
+    """Failure path: with the copy warp disabled (test hook) every pipeline
+    wait runs out after its 2 s bound; the kernel reports through the status
+    word, frees its tensor memory and returns, and the next launch works."""
+    M, K, F = 128, 64, 128
+    x, w = _inputs(M, K, F, 11)
+    xg, wg = x.to(DEV), w.to(DEV)
+    out = torch.zeros(M, F, dtype=torch.bfloat16, device=DEV)
+    st = torch.zeros(1, dtype=torch.int32, device=DEV)
+    L = dbp.library()
+    rc = L.dit_swiglu_gemm_stall_test(xg.data_ptr(), wg.data_ptr(), out.data_ptr(), M, K, F,
+                                      st.data_ptr(), torch.cuda.current_stream().cuda_stream)
+    assert rc == 0
+    torch.cuda.synchronize()
+    assert int(st.item()) == 1
+    st.zero_()
+    good = dbp.swiglu_gemm(xg, wg, status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    _check(orc, x, w, good.cpu(), what="after the stall")
