@@ -9,21 +9,24 @@
 // over the tokens u of the kept key blocks of (b, h, i); non-causal; blocks
 // of 128 tokens, head size 128.
 //
-// Design: one CTA of 6 warps per (query block, head, sample); S = Q K^T and
-// O = P V on the tensor cores with fp32 accumulators in TMEM (two S buffers
-// and O: 384 of 512 columns), online softmax on the CUDA cores:
-//   warp 0    TMA: the 128 x 128 Q tile once, then K and V tiles of each
-//             kept block into a 2-stage ring (128-byte swizzle).
-//   warp 1    one thread issues tcgen05.mma: S_n = Q K_n^T (K-major A and B)
-//             into S buffer n mod 2 as soon as K_n is in and that buffer was
-//             read, then O += P_{n-1} V_{n-1} (P from shared memory, K-major;
-//             V MN-major), so block n's scores overlap block n-1's softmax.
+// Design: one CTA of 6 warps per (query block, head, sample), two CTAs per SM
+// (96 KB of shared memory and 256 of the 512 TMEM columns each), so that one
+// CTA's softmax runs while the other's products use the tensor cores:
+//   warp 0    TMA: the 128 x 128 Q tile once, then K and V of each kept
+//             block, one buffer each (128-byte swizzle): K_{n+1} lands while
+//             block n's softmax runs, V_{n+1} while S_{n+1} and its softmax run.
+//   warp 1    one thread issues tcgen05.mma: S_n = Q K_n^T (shared-memory
+//             operands, fp32 into TMEM columns [0, 128)), then, once the
+//             softmax has written P_n, O += P_n V_n with P read from TMEM
+//             (the A operand in tensor memory, two bf16 per column over S_n's
+//             first 64 columns) and V as an MN-major shared-memory operand
+//             (no transpose).  S_{n+1} is issued after P_n V_n has read P_n.
 //   warps 2-5 softmax, thread = query row (TMEM lane): tcgen05.ld the S row,
-//             running max and sum in the exp2 domain, masking keys past the
-//             sample's last token; after the previous P V has finished, the
-//             O row is rescaled in TMEM (tcgen05.ld / st) when its max moved,
-//             and P is written as bf16 into shared memory in the tensor
-//             cores' 128-byte swizzled K-major layout.  At the end O / l is
+//             mask keys past the sample's last token, weights 2^(s - m) in
+//             fp32 with lazy rescaling (the reference max m moves, and O and
+//             the row sum are rescaled in TMEM, only when a row's block max
+//             exceeds m by more than 8, so weights stay below 2^8), and P
+//             written back into TMEM as bf16 pairs.  At the end O / l is
 //             written as bf16.
 // Every mbarrier wait is bounded (tcgen05.cuh); on expiry the CTA records an
 // error in the caller's status word and exits after freeing its TMEM.
@@ -39,12 +42,24 @@ constexpr int kHd = 128;                        // head size
 constexpr int kThreadsA = 192;
 constexpr uint32_t kTile = kBlk * kHd * 2;      // 32 KB: one 128 x 128 bf16 tile
 constexpr uint32_t kHalfTile = kTile / 2;       // 16 KB: 64 columns (one swizzle atom wide)
-constexpr uint32_t kTmemColsA = 512;
-constexpr uint32_t kColO = 256;                 // O in TMEM columns [256, 384)
-// Q, 2 x (K, V), P, then barriers
-constexpr size_t kSmemA = 6 * kTile + 1024 + 256;
+constexpr uint32_t kTmemColsA = 256;           // two CTAs share an SM's 512 columns
+constexpr uint32_t kColO = 128;                 // S (and P over it) in [0, 128), O in [128, 256)
+// Q, K, V, then barriers
+constexpr size_t kSmemA = 3 * kTile + 1024 + 256;
 constexpr uint32_t kIdescS = idesc_f16(128, 128, false, false);    // S = Q K^T
 constexpr uint32_t kIdescO = idesc_f16(128, 128, false, true);     // O += P V (V MN-major)
+
+// D (TMEM) += A (TMEM, K-major: row m in lane m, two bf16 per column) * B
+// (shared-memory descriptor).
+__device__ __forceinline__ void mma_f16_ts(uint32_t tmem_d, uint32_t tmem_a, uint64_t db,
+                                           uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(tmem_d),
+        "r"(tmem_a), "l"(db), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
 
 struct AttnParams {
     const int32_t* kept;        // [B, H, nb, n_keep]
@@ -56,7 +71,7 @@ struct AttnParams {
     float scale_log2;           // scale * log2(e)
 };
 
-__global__ void __launch_bounds__(kThreadsA, 1)
+__global__ void __launch_bounds__(kThreadsA, 2)
 block_sparse_attention_kernel(const __grid_constant__ CUtensorMap map_q,
                               const __grid_constant__ CUtensorMap map_k,
                               const __grid_constant__ CUtensorMap map_v, AttnParams p) {
@@ -64,21 +79,17 @@ block_sparse_attention_kernel(const __grid_constant__ CUtensorMap map_q,
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
     uint8_t* gen_base = smem_raw + (base - raw);
-    const uint32_t sQ = base;
-    const uint32_t sK0 = base + kTile;              // stage s: K at sK0 + s * 2 * kTile
-    const uint32_t sP = base + 5 * kTile;
-    uint8_t* gP = gen_base + 5 * kTile;
-    const uint32_t bar = base + 6 * kTile;
-    const uint32_t bar_q = bar;                     // Q landed
-    const uint32_t bar_kv_full = bar + 8;           // [2]
-    const uint32_t bar_kv_empty = bar + 24;         // [2]
-    const uint32_t bar_s_full = bar + 40;           // [2]
-    const uint32_t bar_s_free = bar + 56;           // [2], 4 arrivals
-    const uint32_t bar_p_full = bar + 72;           // 4 arrivals
-    const uint32_t bar_o_done = bar + 80;
-    const uint32_t bar_drain = bar + 88;
-    volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(gen_base + 6 * kTile + 96);
-    volatile int* abort = reinterpret_cast<volatile int*>(gen_base + 6 * kTile + 100);
+    const uint32_t sQ = base, sK = base + kTile, sV = base + 2 * kTile;
+    const uint32_t bar = base + 3 * kTile;
+    const uint32_t bar_q = bar;
+    const uint32_t bar_k_full = bar + 8, bar_k_empty = bar + 16;
+    const uint32_t bar_v_full = bar + 24, bar_v_empty = bar + 32;
+    const uint32_t bar_s_full = bar + 40;           // S_n in TMEM
+    const uint32_t bar_p_full = bar + 48;           // P_n in TMEM, O rescaled (4 arrivals)
+    const uint32_t bar_o_done = bar + 56;           // P_n V_n done: S/P columns and O free
+    const uint32_t bar_drain = bar + 64;
+    volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(gen_base + 3 * kTile + 80);
+    volatile int* abort = reinterpret_cast<volatile int*>(gen_base + 3 * kTile + 84);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int i = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
@@ -88,12 +99,11 @@ block_sparse_attention_kernel(const __grid_constant__ CUtensorMap map_q,
 
     if (threadIdx.x == 0) {
         mbar_init(bar_q, 1);
-        for (int s = 0; s < 2; ++s) {
-            mbar_init(bar_kv_full + 8 * s, 1);
-            mbar_init(bar_kv_empty + 8 * s, 1);
-            mbar_init(bar_s_full + 8 * s, 1);
-            mbar_init(bar_s_free + 8 * s, 4);
-        }
+        mbar_init(bar_k_full, 1);
+        mbar_init(bar_k_empty, 1);
+        mbar_init(bar_v_full, 1);
+        mbar_init(bar_v_empty, 1);
+        mbar_init(bar_s_full, 1);
         mbar_init(bar_p_full, 4);
         mbar_init(bar_o_done, 1);
         mbar_init(bar_drain, 1);
@@ -109,76 +119,73 @@ block_sparse_attention_kernel(const __grid_constant__ CUtensorMap map_q,
 
     if (warp == 0) {
         if (lane == 0) {
-            // the Q tile, then K and V of every kept block
+            // the Q tile, then K and V of every kept block (one buffer each:
+            // K_{n+1} lands while the softmax of block n runs, V_{n+1} while
+            // S_{n+1} and its softmax run)
             const int col = h * kHd;
             mbar_expect_tx(bar_q, kTile);
             tma_load_2d(sQ, &map_q, bar_q, col, row0 + i * kBlk);
             tma_load_2d(sQ + kHalfTile, &map_q, bar_q, col + 64, row0 + i * kBlk);
-            int issued = 0;
+            int issued_k = 0, issued_v = 0;
             for (int n = 0; n < nk; ++n) {
-                const int s = n & 1;
-                if (!mbar_wait(bar_kv_empty + 8 * s, ((n >> 1) & 1) ^ 1, abort)) {
+                const int row = row0 + __ldg(kept + n) * kBlk;
+                if (!mbar_wait(bar_k_empty, (n & 1) ^ 1, abort)) {
                     failed = true;
                     break;
                 }
-                const int row = row0 + __ldg(kept + n) * kBlk;
-                const uint32_t sk = sK0 + s * 2 * kTile, sv = sk + kTile;
-                const uint32_t fb = bar_kv_full + 8 * s;
-                mbar_expect_tx(fb, 2 * kTile);
-                tma_load_2d(sk, &map_k, fb, col, row);
-                tma_load_2d(sk + kHalfTile, &map_k, fb, col + 64, row);
-                tma_load_2d(sv, &map_v, fb, col, row);
-                tma_load_2d(sv + kHalfTile, &map_v, fb, col + 64, row);
-                issued = n + 1;
+                mbar_expect_tx(bar_k_full, kTile);
+                tma_load_2d(sK, &map_k, bar_k_full, col, row);
+                tma_load_2d(sK + kHalfTile, &map_k, bar_k_full, col + 64, row);
+                issued_k = n + 1;
+                if (!mbar_wait(bar_v_empty, (n & 1) ^ 1, abort)) {
+                    failed = true;
+                    break;
+                }
+                mbar_expect_tx(bar_v_full, kTile);
+                tma_load_2d(sV, &map_v, bar_v_full, col, row);
+                tma_load_2d(sV + kHalfTile, &map_v, bar_v_full, col + 64, row);
+                issued_v = n + 1;
             }
             mbar_wait(bar_q, 0, abort);
             if (failed) {
-                for (int n = issued > 2 ? issued - 2 : 0; n < issued; ++n)
-                    mbar_wait(bar_kv_full + 8 * (n & 1), (n >> 1) & 1, abort);
+                if (issued_k) mbar_wait(bar_k_full, (issued_k - 1) & 1, abort);
+                if (issued_v) mbar_wait(bar_v_full, (issued_v - 1) & 1, abort);
             }
         }
         __syncwarp();
     } else if (warp == 1) {
         if (lane == 0) {
-            // S_n = Q K_n^T, then O += P_{n-1} V_{n-1}
             if (!mbar_wait(bar_q, 0, abort)) failed = true;
-            for (int n = 0; n <= nk && !failed; ++n) {
-                if (n < nk) {
-                    const int s = n & 1;
-                    if (!mbar_wait(bar_kv_full + 8 * s, (n >> 1) & 1, abort) ||
-                        (n >= 2 && !mbar_wait(bar_s_free + 8 * s, ((n - 2) >> 1) & 1, abort))) {
-                        failed = true;
-                        break;
-                    }
-                    fence_after_sync();
-                    const uint32_t sk = sK0 + s * 2 * kTile;
-#pragma unroll
-                    for (int kk = 0; kk < kHd / 16; ++kk) {
-                        const uint32_t off = (kk >> 2) * kHalfTile + (kk & 3) * 32;
-                        mma_f16(tmem + 128u * s, sw128_desc(sQ + off), sw128_desc(sk + off),
-                                kIdescS, kk != 0 ? 1u : 0u);
-                    }
-                    mma_commit(bar_s_full + 8 * s);
+            for (int n = 0; n < nk && !failed; ++n) {
+                // S_n = Q K_n^T, once K_n is in and P_{n-1} V_{n-1} has read the
+                // columns S_n overwrites
+                if (!mbar_wait(bar_k_full, n & 1, abort) ||
+                    (n >= 1 && !mbar_wait(bar_o_done, (n - 1) & 1, abort))) {
+                    failed = true;
+                    break;
                 }
-                if (n >= 1) {
-                    const int m = n - 1;
-                    if (!mbar_wait(bar_p_full, m & 1, abort)) {
-                        failed = true;
-                        break;
-                    }
-                    fence_after_sync();
-                    const uint32_t sv = sK0 + (m & 1) * 2 * kTile + kTile;
+                fence_after_sync();
 #pragma unroll
-                    for (int kk = 0; kk < kBlk / 16; ++kk) {
-                        // A: P, K-major over keys; B: V, MN-major (d contiguous),
-                        // 16 keys = two 8-row groups per step
-                        const uint32_t pa = sP + (kk >> 2) * kHalfTile + (kk & 3) * 32;
-                        mma_f16(tmem + kColO, sw128_desc(pa), sw128_desc_mn(sv + kk * 2048, kHalfTile),
-                                kIdescO, (m | kk) != 0 ? 1u : 0u);
-                    }
-                    mma_commit(bar_o_done);
-                    mma_commit(bar_kv_empty + 8 * (m & 1));
+                for (int kk = 0; kk < kHd / 16; ++kk) {
+                    const uint32_t off = (kk >> 2) * kHalfTile + (kk & 3) * 32;
+                    mma_f16(tmem, sw128_desc(sQ + off), sw128_desc(sK + off), kIdescS,
+                            kk != 0 ? 1u : 0u);
                 }
+                mma_commit(bar_s_full);
+                mma_commit(bar_k_empty);
+                // O += P_n V_n once the softmax has written P_n (over S_n) and
+                // rescaled O
+                if (!mbar_wait(bar_p_full, n & 1, abort) || !mbar_wait(bar_v_full, n & 1, abort)) {
+                    failed = true;
+                    break;
+                }
+                fence_after_sync();
+#pragma unroll
+                for (int kk = 0; kk < kBlk / 16; ++kk)
+                    mma_f16_ts(tmem + kColO, tmem + 8 * kk, sw128_desc_mn(sV + kk * 2048, kHalfTile),
+                               kIdescO, (n | kk) != 0 ? 1u : 0u);
+                mma_commit(bar_o_done);
+                mma_commit(bar_v_empty);
             }
             if (failed) {
                 mma_commit(bar_drain);
@@ -193,8 +200,7 @@ block_sparse_attention_kernel(const __grid_constant__ CUtensorMap map_q,
         const uint32_t lane_off = static_cast<uint32_t>(32 * q) << 16;
         float m_run = -INFINITY, l_run = 0.0f;
         for (int n = 0; n < nk; ++n) {
-            const int s = n & 1;
-            if (!mbar_wait(bar_s_full + 8 * s, (n >> 1) & 1, abort)) {
+            if (!__all_sync(0xffffffffu, mbar_wait(bar_s_full, n & 1, abort))) {
                 failed = true;
                 break;
             }
@@ -202,23 +208,25 @@ block_sparse_attention_kernel(const __grid_constant__ CUtensorMap map_q,
             float sc[kBlk];
 #pragma unroll
             for (int c = 0; c < kBlk / 32; ++c)
-                tmem_ld32(tmem + lane_off + 128u * s + 32 * c,
-                          *reinterpret_cast<float(*)[32]>(sc + 32 * c));
+                tmem_ld32(tmem + lane_off + 32 * c, *reinterpret_cast<float(*)[32]>(sc + 32 * c));
             tmem_wait_ld();
-            fence_before_sync();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bar_s_free + 8 * s);
             // keys past the sample's last token do not take part
             const int64_t j = __ldg(kept + n);
             const int64_t left = p.N - j * kBlk;
             const int valid = left >= kBlk ? kBlk : (left > 0 ? static_cast<int>(left) : 0);
-            float mx = m_run;
+            float mr = -INFINITY;
 #pragma unroll
             for (int c = 0; c < kBlk; ++c) {
                 sc[c] = c < valid ? sc[c] * p.scale_log2 : -INFINITY;
-                mx = fmaxf(mx, sc[c]);
+                mr = fmaxf(mr, sc[c]);
             }
-            const float alpha = exp2f(m_run - mx);      // 0 on the first block
+            // lazy rescaling: the reference max moves (and O and l are
+            // rescaled) only when some row's block max exceeds it by more than
+            // 8, so the weights stay below 2^8 and most blocks skip the O
+            // round trip through TMEM
+            const bool move = __any_sync(0xffffffffu, mr > m_run + 8.0f);
+            const float mx = move ? fmaxf(m_run, mr) : m_run;
+            const float alpha = move ? exp2f(m_run - mx) : 1.0f;   // 0 on the first block
             float sum = 0.0f;
 #pragma unroll
             for (int c = 0; c < kBlk; ++c) {
@@ -227,47 +235,35 @@ block_sparse_attention_kernel(const __grid_constant__ CUtensorMap map_q,
             }
             l_run = l_run * alpha + sum;
             m_run = mx;
-            if (n >= 1) {
-                // the previous P V is done: P is free and O holds the sum so far
-                if (!mbar_wait(bar_o_done, (n - 1) & 1, abort)) {
-                    failed = true;
-                    break;
-                }
-                fence_after_sync();
-                if (__any_sync(0xffffffffu, alpha != 1.0f)) {
+            if (n >= 1 && move) {
+                // P_{n-1} V_{n-1} is done (S_n was issued after it), so O holds
+                // the sum so far
 #pragma unroll 1
-                    for (int c = 0; c < kHd / 32; ++c) {
-                        float o[32];
-                        tmem_ld32(tmem + lane_off + kColO + 32 * c, o);
-                        tmem_wait_ld();
+                for (int c = 0; c < kHd / 32; ++c) {
+                    float o[32];
+                    tmem_ld32(tmem + lane_off + kColO + 32 * c, o);
+                    tmem_wait_ld();
 #pragma unroll
-                        for (int e = 0; e < 32; ++e) o[e] *= alpha;
-                        tmem_st32(tmem + lane_off + kColO + 32 * c, o);
-                    }
-                    tmem_wait_st();
+                    for (int e = 0; e < 32; ++e) o[e] *= alpha;
+                    tmem_st32(tmem + lane_off + kColO + 32 * c, o);
                 }
             }
-            // P row r as bf16, K-major with the 128-byte swizzle: keys
-            // [64a, 64a + 64) in atom a, 16-byte chunk c of the row at chunk
-            // c ^ (r mod 8)
+            // P_n as bf16 pairs over S_n's first 64 columns (row r in lane r)
 #pragma unroll
-            for (int a = 0; a < 2; ++a) {
-                uint8_t* rowp = gP + a * kHalfTile + r * 128;
+            for (int c = 0; c < 2; ++c) {
+                float w[32];
 #pragma unroll
-                for (int c = 0; c < 8; ++c) {
-                    float f[8];
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) f[e] = sc[64 * a + 8 * c + e];
-                    *reinterpret_cast<uint4*>(rowp + ((c ^ (r & 7)) << 4)) = pack8(f);
-                }
+                for (int e = 0; e < 32; ++e)
+                    w[e] = __uint_as_float(pack2(sc[64 * c + 2 * e], sc[64 * c + 2 * e + 1]));
+                tmem_st32(tmem + lane_off + 32 * c, w);
             }
-            fence_proxy_async_smem();
+            tmem_wait_st();
             fence_before_sync();
             __syncwarp();
             if (lane == 0) mbar_arrive(bar_p_full);
         }
         if (!failed && nk > 0) {
-            if (!mbar_wait(bar_o_done, (nk - 1) & 1, abort)) {
+            if (!__all_sync(0xffffffffu, mbar_wait(bar_o_done, (nk - 1) & 1, abort))) {
                 failed = true;
             } else {
                 fence_after_sync();
