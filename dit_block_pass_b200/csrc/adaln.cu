@@ -45,6 +45,7 @@ struct RowParams {
     int64_t set_stride;         // elements between the sets of one sample
     int n_sets;
     bool mod_vec;               // every set's vectors can be read 16 bytes at a time
+    int staged_sets;            // sets staged in shared memory (1, or 2 for AdaLN)
 };
 
 __device__ __forceinline__ float mod_at(const void* p, int dtype, int64_t i) {
@@ -122,6 +123,11 @@ template <bool TOK>
 __device__ __forceinline__ void modulation8(const RowParams& p, const float4* s_lo, int Dv,
                                             int v, const void* m, int set, bool one_plus,
                                             float (&f)[8]) {
+    if (TOK && set > 0 && set < p.staged_sets) {
+        // a second staged set follows the first (4 * Dv float4s apart)
+        lds8(s_lo + 4 * Dv, s_lo + 5 * Dv, v, f);
+        return;
+    }
     if (TOK && set != 0) {
         if (set < 0) {
 #pragma unroll
@@ -142,12 +148,25 @@ __device__ __forceinline__ void modulation8(const RowParams& p, const float4* s_
 // Stage the modulation vectors of sample blockIdx.y in shared memory:
 // shift and (1 + scale) (and gate), each as [lo Dv][hi Dv] float4 halves.
 template <bool GATED>
+__device__ __forceinline__ void stage_one_set(const RowParams& p, float4* smem, int nthreads,
+                                              int64_t mb);
+
+template <bool GATED>
 __device__ __forceinline__ void stage_modulation(const RowParams& p, float4* smem, int nthreads) {
+    const int64_t mb = static_cast<int64_t>(blockIdx.y) * p.mod_stride;
+    stage_one_set<GATED>(p, smem, nthreads, mb);
+    // AdaLN with per-token sets: set 1 too, 4 * Dv float4s after set 0
+    if (!GATED && p.staged_sets > 1)
+        stage_one_set<GATED>(p, smem + 4 * p.Dv, nthreads, mb + p.set_stride);
+}
+
+template <bool GATED>
+__device__ __forceinline__ void stage_one_set(const RowParams& p, float4* smem, int nthreads,
+                                              int64_t mb) {
     const int Dv = p.Dv;
     float4* s_sh = smem;
     float4* s_sc = smem + 2 * Dv;
     float4* s_g = smem + 4 * Dv;
-    const int64_t mb = static_cast<int64_t>(blockIdx.y) * p.mod_stride;
     for (int v = threadIdx.x; v < Dv; v += nthreads) {
         float sh[8], sc[8], g[8];
 #pragma unroll
@@ -194,17 +213,36 @@ __device__ __forceinline__ void ln_finish_store(const RowParams& p, const float4
     }
     q = warp_sum(q);
     const float rstd = rsqrtf(__fmaf_rn(q, p.inv_D, p.eps));
+    // the set is decided once per row, outside the unrolled loops, so that a
+    // staged row's shared-memory loads can be issued ahead as without sets
+    if (!TOK || (set >= 0 && set < p.staged_sets)) {
+        const int so = TOK ? 4 * Dv * set : 0;
 #pragma unroll
-    for (int j = 0; j < VPL; ++j) {
-        const int v = j * 32 + lane;
-        if (v < Dv) {
-            float f[8], sh[8], sc[8];
-            unpack8(xv[j], f);
-            modulation8<TOK>(p, s_sh, Dv, v, p.shift, set, false, sh);
-            modulation8<TOK>(p, s_sc, Dv, v, p.scale, set, true, sc);
+        for (int j = 0; j < VPL; ++j) {
+            const int v = j * 32 + lane;
+            if (v < Dv) {
+                float f[8], sh[8], sc[8];
+                unpack8(xv[j], f);
+                lds8(s_sh + so, s_sh + so + Dv, v, sh);
+                lds8(s_sc + so, s_sc + so + Dv, v, sc);
 #pragma unroll
-            for (int i = 0; i < 8; ++i) f[i] = __fmaf_rn((f[i] - mu) * rstd, sc[i], sh[i]);
-            st_stream(p.y + base + v, pack8(f));
+                for (int i = 0; i < 8; ++i) f[i] = __fmaf_rn((f[i] - mu) * rstd, sc[i], sh[i]);
+                st_stream(p.y + base + v, pack8(f));
+            }
+        }
+    } else {
+#pragma unroll
+        for (int j = 0; j < VPL; ++j) {
+            const int v = j * 32 + lane;
+            if (v < Dv) {
+                float f[8], sh[8], sc[8];
+                unpack8(xv[j], f);
+                modulation8<TOK>(p, s_sh, Dv, v, p.shift, set, false, sh);
+                modulation8<TOK>(p, s_sc, Dv, v, p.scale, set, true, sc);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) f[i] = __fmaf_rn((f[i] - mu) * rstd, sc[i], sh[i]);
+                st_stream(p.y + base + v, pack8(f));
+            }
         }
     }
 }
@@ -258,6 +296,69 @@ __device__ __forceinline__ void cp_async16(void* smem_dst, const void* gsrc) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d), "l"(gsrc) : "memory");
 }
 
+// First pass of a gated row (the lane's vectors of one half): x + gate * r
+// to x_out, kept in xv, and the sum of (x_out - x0).  STAGED reads the gate
+// from the shared-memory stage (set 0), otherwise from the row's set.
+template <int VPL, bool TOK, bool STAGED>
+__device__ __forceinline__ float gated_first_pass(const RowParams& p, const float4* s_g,
+                                                  const uint4* stage, uint4 (&xv)[VPL],
+                                                  int64_t base, int lane, int half, int set,
+                                                  float x0) {
+    const int Dv = p.Dv;
+    float s = 0.0f;
+#pragma unroll
+    for (int j = 0; j < VPL; ++j) {
+        const int v = 64 * j + 32 * half + lane;
+        if (v < Dv) {
+            const uint4 rv = stage[j * 32 + lane];
+            float g[8];
+            if (STAGED) lds8(s_g, s_g + Dv, v, g);
+            else modulation8<TOK>(p, s_g, Dv, v, p.gate, set, false, g);
+            uint4 o;
+            o.x = gated_pair(xv[j].x, rv.x, g[0], g[1]);
+            o.y = gated_pair(xv[j].y, rv.y, g[2], g[3]);
+            o.z = gated_pair(xv[j].z, rv.z, g[4], g[5]);
+            o.w = gated_pair(xv[j].w, rv.w, g[6], g[7]);
+            xv[j] = o;
+            st_stream(p.x_out + base + v, o);
+            float f[8];
+            unpack8(o, f);
+            float t = 0.0f;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) t += f[i];
+            s += __fmaf_rn(-8.0f, x0, t);
+        }
+    }
+    return s;
+}
+
+// Last pass of a gated row: y = (x_out - mu) * rstd * (1 + scale) + shift.
+template <int VPL, bool TOK, bool STAGED>
+__device__ __forceinline__ void gated_last_pass(const RowParams& p, const float4* s_sh,
+                                                const float4* s_sc, const uint4 (&xv)[VPL],
+                                                int64_t base, int lane, int half, int set,
+                                                float mu, float rstd) {
+    const int Dv = p.Dv;
+#pragma unroll
+    for (int j = 0; j < VPL; ++j) {
+        const int v = 64 * j + 32 * half + lane;
+        if (v < Dv) {
+            float f[8], sh[8], sc[8];
+            unpack8(xv[j], f);
+            if (STAGED) {
+                lds8(s_sh, s_sh + Dv, v, sh);
+                lds8(s_sc, s_sc + Dv, v, sc);
+            } else {
+                modulation8<TOK>(p, s_sh, Dv, v, p.shift, set, false, sh);
+                modulation8<TOK>(p, s_sc, Dv, v, p.scale, set, true, sc);
+            }
+#pragma unroll
+            for (int i = 0; i < 8; ++i) f[i] = __fmaf_rn((f[i] - mu) * rstd, sc[i], sh[i]);
+            st_stream(p.y + base + v, pack8(f));
+        }
+    }
+}
+
 // Gated residual + AdaLN: one warp PAIR per row.  Warp h (0, 1) of a pair
 // holds vectors v = 64*j + 32*h + lane of the row (each warp instruction
 // still covers 512 contiguous bytes), so a lane keeps VPL = ceil(D/512)
@@ -309,29 +410,36 @@ gated_rows_kernel(RowParams p) {
         const float x0 = __shfl_sync(0xffffffffu, bf16_lo(xv[0].x), 0);
         // each lane reads back only the vectors it copied itself
         asm volatile("cp.async.wait_group 0;" ::: "memory");
+        // the set is decided once per row, outside the unrolled loops
+        const bool staged = !TOK || set == 0;
         float s = 0.0f;
+        if (!TOK) {
 #pragma unroll
-        for (int j = 0; j < VPL; ++j) {
-            const int v = 64 * j + 32 * half + lane;
-            if (v < Dv) {
-                const uint4 rv = stage[j * 32 + lane];
-                float g[8];
-                if (TOK) modulation8<TOK>(p, s_g, Dv, v, p.gate, set, false, g);
-                else lds8(s_g, s_g + Dv, v, g);
-                uint4 o;
-                o.x = gated_pair(xv[j].x, rv.x, g[0], g[1]);
-                o.y = gated_pair(xv[j].y, rv.y, g[2], g[3]);
-                o.z = gated_pair(xv[j].z, rv.z, g[4], g[5]);
-                o.w = gated_pair(xv[j].w, rv.w, g[6], g[7]);
-                xv[j] = o;
-                st_stream(p.x_out + base + v, o);
-                float f[8];
-                unpack8(o, f);
-                float t = 0.0f;
+            for (int j = 0; j < VPL; ++j) {
+                const int v = 64 * j + 32 * half + lane;
+                if (v < Dv) {
+                    const uint4 rv = stage[j * 32 + lane];
+                    float g[8];
+                    lds8(s_g, s_g + Dv, v, g);
+                    uint4 o;
+                    o.x = gated_pair(xv[j].x, rv.x, g[0], g[1]);
+                    o.y = gated_pair(xv[j].y, rv.y, g[2], g[3]);
+                    o.z = gated_pair(xv[j].z, rv.z, g[4], g[5]);
+                    o.w = gated_pair(xv[j].w, rv.w, g[6], g[7]);
+                    xv[j] = o;
+                    st_stream(p.x_out + base + v, o);
+                    float f[8];
+                    unpack8(o, f);
+                    float t = 0.0f;
 #pragma unroll
-                for (int i = 0; i < 8; ++i) t += f[i];
-                s += __fmaf_rn(-8.0f, x0, t);
+                    for (int i = 0; i < 8; ++i) t += f[i];
+                    s += __fmaf_rn(-8.0f, x0, t);
+                }
             }
+        } else if (staged) {
+            s = gated_first_pass<VPL, TOK, true>(p, s_g, stage, xv, base, lane, half, set, x0);
+        } else {
+            s = gated_first_pass<VPL, TOK, false>(p, s_g, stage, xv, base, lane, half, set, x0);
         }
         s = warp_sum(s);
         if (lane == 0) {
@@ -361,23 +469,25 @@ gated_rows_kernel(RowParams p) {
         asm volatile("bar.sync %0, 64;" ::"r"(bar) : "memory");
         const float rstd =
             rsqrtf(__fmaf_rn(red[pair][1][0] + red[pair][1][1], p.inv_D, p.eps));
+        if (!TOK) {
 #pragma unroll
-        for (int j = 0; j < VPL; ++j) {
-            const int v = 64 * j + 32 * half + lane;
-            if (v < Dv) {
-                float f[8], sh[8], sc[8];
-                unpack8(xv[j], f);
-                if (TOK) {
-                    modulation8<TOK>(p, s_sh, Dv, v, p.shift, set, false, sh);
-                    modulation8<TOK>(p, s_sc, Dv, v, p.scale, set, true, sc);
-                } else {
+            for (int j = 0; j < VPL; ++j) {
+                const int v = 64 * j + 32 * half + lane;
+                if (v < Dv) {
+                    float f[8], sh[8], sc[8];
+                    unpack8(xv[j], f);
                     lds8(s_sh, s_sh + Dv, v, sh);
                     lds8(s_sc, s_sc + Dv, v, sc);
-                }
 #pragma unroll
-                for (int i = 0; i < 8; ++i) f[i] = __fmaf_rn((f[i] - mu) * rstd, sc[i], sh[i]);
-                st_stream(p.y + base + v, pack8(f));
+                    for (int i = 0; i < 8; ++i)
+                        f[i] = __fmaf_rn((f[i] - mu) * rstd, sc[i], sh[i]);
+                    st_stream(p.y + base + v, pack8(f));
+                }
             }
+        } else if (staged) {
+            gated_last_pass<VPL, TOK, true>(p, s_sh, s_sc, xv, base, lane, half, set, mu, rstd);
+        } else {
+            gated_last_pass<VPL, TOK, false>(p, s_sh, s_sc, xv, base, lane, half, set, mu, rstd);
         }
     }
 }
@@ -404,9 +514,11 @@ RowLaunch pick_kernel(bool gated, int Dv) {
         return {nullptr, 0, 0};
     }
     const int need = (Dv + 63) / 64;   // a warp pair shares a row
+    // 24 warps (80 registers each) for short rows; the per-token form keeps
+    // 16, since its second code path spills at 80 registers
 #define DIT_VPL_CASE(V)                                                                   \
     if (need <= V) {                                                                      \
-        constexpr int WG = (V <= 10) ? 24 : 16;                                           \
+        constexpr int WG = (V <= 10 && !TOK) ? 24 : 16;                                   \
         return {gated_rows_kernel<V, WG, TOK>, WG * 32,                                   \
                 mod + static_cast<size_t>(WG) * V * 32 * sizeof(uint4)};                  \
     }
@@ -417,8 +529,9 @@ RowLaunch pick_kernel(bool gated, int Dv) {
 }
 
 int launch_rows(const RowParams& p, bool gated, int B, cudaStream_t stream) {
-    const RowLaunch L = p.set_index ? pick_kernel<true>(gated, p.Dv)
-                                    : pick_kernel<false>(gated, p.Dv);
+    RowLaunch L = p.set_index ? pick_kernel<true>(gated, p.Dv)
+                              : pick_kernel<false>(gated, p.Dv);
+    if (L.kernel && !gated && p.staged_sets > 1) L.smem *= 2;     // the second staged set
     if (!L.kernel) return DIT_ERR_SHAPE;
     // opt in whenever dynamic shared memory is used (static arrays count
     // toward the 48 KB default too)
@@ -469,6 +582,12 @@ int set_checks(RowParams& p, const uint8_t* set_index, int n_sets, int64_t set_s
     bool vec = p.mod_stride % per16 == 0 && set_stride % per16 == 0;
     for (int i = 0; i < n_mods; ++i) vec = vec && aligned16(mods[i]);
     p.mod_vec = vec;
+    // AdaLN stages set 1 beside set 0 when both fit in about 100 KB
+    // (2 CTAs per SM); the gated form keeps its shared memory for the stage
+    p.staged_sets = (n_mods == 2 && n_sets >= 2 &&
+                     2 * static_cast<size_t>(p.Dv) * 4 * sizeof(float4) <= 100 * 1024)
+                        ? 2
+                        : 1;
     return DIT_OK;
 }
 

@@ -69,9 +69,12 @@ __device__ __forceinline__ float w_at(const void* p, int dtype, int i) {
     return __uint_as_float(static_cast<uint32_t>(static_cast<const uint16_t*>(p)[i]) << 16);
 }
 
-// Eight weights of elements e .. e+7 (fp32 or bf16; 16-byte aligned rows).
-__device__ __forceinline__ void w8_at(const void* w, int dtype, int e, float (&f)[8]) {
-    if (dtype == DIT_F32) {
+// Eight weights of elements e .. e+7 (fp32 when WF32, else bf16; 16-byte
+// aligned rows).  The dtype is a template argument so that an unrolled loop
+// of these loads has no branch between them.
+template <bool WF32>
+__device__ __forceinline__ void w8_of(const void* w, int e, float (&f)[8]) {
+    if (WF32) {
         const float4* q = reinterpret_cast<const float4*>(static_cast<const float*>(w) + e);
         const float4 a = __ldg(q), b = __ldg(q + 1);
         f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w;
@@ -227,10 +230,10 @@ __device__ __forceinline__ void qk_head_tensor(const uint4 (&v)[NVL], uint4* oro
 // Whole-row norm of one tensor row held as NVL lane-vectors v: the row's
 // sum of squares first (a warp reduction), then the weighted, rotated
 // values.  The weight has one entry per element of the row.
-template <int HD, int NVL, int LAYOUT>
+template <int HD, int NVL, int LAYOUT, bool WF32>
 __device__ __forceinline__ void qk_row_tensor(uint4 (&v)[NVL], uint4* orow, int64_t osh, int nvr,
-                                              int lane, const void* w, int w_dtype,
-                                              const float* cs, const float* sn, float eps) {
+                                              int lane, const void* w, const float* cs,
+                                              const float* sn, float eps) {
     constexpr int LPH = HD / 8;
     constexpr int HALF = LPH / 2;
     const bool first = ((lane % LPH) & HALF) == 0;
@@ -249,12 +252,27 @@ __device__ __forceinline__ void qk_row_tensor(uint4 (&v)[NVL], uint4* orow, int6
 #pragma unroll
     for (int j = 0; j < NVL; ++j)
         asm volatile("" : "+r"(v[j].x), "+r"(v[j].y), "+r"(v[j].z), "+r"(v[j].w));
+    // the weights of vector j + PD are requested before vector j is stored
+    // (a store is a compiler barrier for loads), so the weight loads run PD
+    // vectors ahead of their use
+    constexpr int PD = NVL < 2 ? NVL : 2;
+    float wr[PD][8];
+#pragma unroll
+    for (int d = 0; d < PD; ++d) {
+        const int idx = d * 32 + lane;
+        w8_of<WF32>(w, (idx < nvr ? idx : 0) * 8, wr[d]);
+    }
 #pragma unroll
     for (int j = 0; j < NVL; ++j) {
         const int idx = j * 32 + lane;
         float f[8], wv[8], o8[8];
         unpack8(v[j], f);
-        w8_at(w, w_dtype, (idx < nvr ? idx : 0) * 8, wv);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) wv[i] = wr[j % PD][i];
+        if (j + PD < NVL) {
+            const int nidx = (j + PD) * 32 + lane;
+            w8_of<WF32>(w, (nidx < nvr ? nidx : 0) * 8, wr[j % PD]);
+        }
         if (LAYOUT == 0) {
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
@@ -312,10 +330,14 @@ qk_rmsnorm_rope3d_kernel(QKParams p) {
 
     float cs[NP], sn[NP];
     token_angles<HD, LAYOUT>(p, s_omega, tok, lane % LPH, cs, sn);
-    if (MODE == 2)
-        qk_row_tensor<HD, NVL, LAYOUT>(v, out_row(p.o0, p, tok), p.osh, p.nvr, lane, p.w0,
-                                       p.w_dtype, cs, sn, p.eps);
-    else
+    if (MODE == 2) {
+        if (p.w_dtype == DIT_F32)
+            qk_row_tensor<HD, NVL, LAYOUT, true>(v, out_row(p.o0, p, tok), p.osh, p.nvr, lane,
+                                                 p.w0, cs, sn, p.eps);
+        else
+            qk_row_tensor<HD, NVL, LAYOUT, false>(v, out_row(p.o0, p, tok), p.osh, p.nvr, lane,
+                                                  p.w0, cs, sn, p.eps);
+    } else
         qk_head_tensor<HD, NVL, LAYOUT, MODE == 0>(v, out_row(p.o0, p, tok), p.osh, p.nvr, lane,
                                                    p.w0, p.w_dtype, cs, sn, p.eps);
     if (row1) {
@@ -324,10 +346,14 @@ qk_rmsnorm_rope3d_kernel(QKParams p) {
 #pragma unroll
         for (int j = 0; j < NVL; ++j)
             v[j] = (j * 32 + lane < p.nvr) ? stage[j * 32] : make_uint4(0, 0, 0, 0);
-        if (MODE == 2)
-            qk_row_tensor<HD, NVL, LAYOUT>(v, out_row(p.o1, p, tok), p.osh, p.nvr, lane, p.w1,
-                                           p.w_dtype, cs, sn, p.eps);
-        else
+        if (MODE == 2) {
+            if (p.w_dtype == DIT_F32)
+                qk_row_tensor<HD, NVL, LAYOUT, true>(v, out_row(p.o1, p, tok), p.osh, p.nvr,
+                                                     lane, p.w1, cs, sn, p.eps);
+            else
+                qk_row_tensor<HD, NVL, LAYOUT, false>(v, out_row(p.o1, p, tok), p.osh, p.nvr,
+                                                      lane, p.w1, cs, sn, p.eps);
+        } else
             qk_head_tensor<HD, NVL, LAYOUT, MODE == 0>(v, out_row(p.o1, p, tok), p.osh, p.nvr,
                                                        lane, p.w1, p.w_dtype, cs, sn, p.eps);
     }
