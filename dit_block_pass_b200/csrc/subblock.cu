@@ -18,9 +18,10 @@
 //   subblock_select_kernel  CTA (up to 8 query blocks, h, b): the query means
 //                           in shared memory, one pass over the key means of
 //                           head h (L2 resident) for all scores, then one
-//                           warp per query block: a radix select of the
-//                           n_keep-th largest score (four 8-bit histogram
-//                           passes) and an ordered ballot compaction that
+//                           warp per query block: the n_keep-th largest
+//                           score found bit by bit with warp-wide counts
+//                           (the scores in registers up to 1024 key
+//                           blocks) and an ordered ballot compaction that
 //                           writes the kept indices in increasing order,
 //                           ties at the threshold to the lower index.
 #include <cmath>
@@ -32,6 +33,7 @@ namespace {
 
 constexpr int kPoolThreads = 256;
 constexpr int kSelThreads = 256;
+constexpr int kKeysPerThread = 4;       // key blocks per thread and pass of the score loop
 constexpr int kMaxBlocks = 8192;           // key blocks per sample
 
 // Means of the rows of one block, every column: thread t takes column
@@ -81,53 +83,75 @@ __device__ __forceinline__ uint32_t ordered(float f) {
 }
 
 // One warp picks one query block's kept key blocks from its fp32 scores
-// sc[0..nb) in shared memory: four 8-bit histogram passes over the
-// order-preserving score codes find the n_keep-th largest code T, then the
-// kept indices -- every code above T and the lowest-index ties at T -- are
-// written in increasing order with ballots.  Same order as sorting (score
-// descending, index ascending) and taking the first n_keep.
-__device__ void warp_select(const float* sc, int nb, int n_keep, unsigned* hist, int32_t* out,
-                            int lane) {
-    uint32_t prefix = 0, mask = 0;
-    int need = n_keep;              // keys still wanted among those matching the prefix
-    for (int pass = 0; pass < 4; ++pass) {
-        const int shift = 24 - 8 * pass;
-        for (int e = lane; e < 256; e += 32) hist[e] = 0;
-        __syncwarp();
-        for (int j = lane; j < nb; j += 32) {
-            const uint32_t c = ordered(sc[j]);
-            if ((c & mask) == prefix) atomicAdd(&hist[(c >> shift) & 255u], 1u);
-        }
-        __syncwarp();
-        int digit = 0, above = 0;
-        if (lane == 0) {
-            // from the top digit down, the first bin that reaches `need`
-            int acc = 0, d = 255;
-            for (; d > 0; --d) {
-                const int cnt = static_cast<int>(hist[d]);
-                if (acc + cnt >= need) break;
-                acc += cnt;
-            }
-            digit = d;
-            above = acc;
-        }
-        digit = __shfl_sync(0xffffffffu, digit, 0);
-        above = __shfl_sync(0xffffffffu, above, 0);
-        need -= above;
-        prefix |= static_cast<uint32_t>(digit) << shift;
-        mask |= 255u << shift;
-        __syncwarp();
+// sc[0..nb) in shared memory.  The n_keep-th largest order-preserving code T
+// is the largest T with at least n_keep codes >= T, fixed one bit at a time
+// from the top (32 warp-wide counts; no shared-memory atomics, which the
+// clustered top bytes of the codes would serialise); then the kept indices --
+// every code above T and the lowest-index ties at T -- are written in
+// increasing order with ballots.  Same order as sorting (score descending,
+// index ascending) and taking the first n_keep.  This form: nb <= 32 * KPL,
+// the lane's codes in registers; warp_select_smem below: any nb, the codes
+// re-read from shared memory in every count.
+template <int KPL>
+__device__ void warp_select_reg(const float* sc, int nb, int n_keep, int32_t* out, int lane) {
+    uint32_t c[KPL];
+#pragma unroll
+    for (int k = 0; k < KPL; ++k) {
+        const int j = k * 32 + lane;
+        c[k] = j < nb ? ordered(sc[j]) : 0u;
     }
-    // prefix is T; `need` ties at T are taken, lowest indices first
+    // a candidate is never 0, so the padding codes (0) are never counted
+    uint32_t T = 0;
+    for (int bit = 31; bit >= 0; --bit) {
+        const uint32_t cand = T | (1u << bit);
+        unsigned cnt = 0;
+#pragma unroll
+        for (int k = 0; k < KPL; ++k) cnt += c[k] >= cand ? 1u : 0u;
+        if (__reduce_add_sync(0xffffffffu, cnt) >= static_cast<unsigned>(n_keep)) T = cand;
+    }
+    unsigned gt = 0;
+#pragma unroll
+    for (int k = 0; k < KPL; ++k) gt += c[k] > T ? 1u : 0u;
+    // `need` ties at T are taken, lowest indices first
+    const int need = n_keep - static_cast<int>(__reduce_add_sync(0xffffffffu, gt));
+    int written = 0, eq_seen = 0;
+    const unsigned below = (1u << lane) - 1u;
+#pragma unroll
+    for (int k = 0; k < KPL; ++k) {
+        if (k * 32 >= nb) break;
+        const int j = k * 32 + lane;
+        const bool live = j < nb;
+        const bool g = live && c[k] > T;
+        const bool eq = live && c[k] == T;
+        const unsigned eqm = __ballot_sync(0xffffffffu, eq);
+        const bool take = g || (eq && eq_seen + __popc(eqm & below) < need);
+        const unsigned tm = __ballot_sync(0xffffffffu, take);
+        if (take) out[written + __popc(tm & below)] = j;
+        written += __popc(tm);
+        eq_seen += __popc(eqm);
+    }
+}
+
+__device__ void warp_select_smem(const float* sc, int nb, int n_keep, int32_t* out, int lane) {
+    uint32_t T = 0;
+    for (int bit = 31; bit >= 0; --bit) {
+        const uint32_t cand = T | (1u << bit);
+        unsigned cnt = 0;
+        for (int j = lane; j < nb; j += 32) cnt += ordered(sc[j]) >= cand ? 1u : 0u;
+        if (__reduce_add_sync(0xffffffffu, cnt) >= static_cast<unsigned>(n_keep)) T = cand;
+    }
+    unsigned gt = 0;
+    for (int j = lane; j < nb; j += 32) gt += ordered(sc[j]) > T ? 1u : 0u;
+    const int need = n_keep - static_cast<int>(__reduce_add_sync(0xffffffffu, gt));
     int written = 0, eq_seen = 0;
     const unsigned below = (1u << lane) - 1u;
     for (int j0 = 0; j0 < nb; j0 += 32) {
         const int j = j0 + lane;
         const uint32_t c = j < nb ? ordered(sc[j]) : 0u;
-        const bool gt = j < nb && c > prefix;
-        const bool eq = j < nb && c == prefix;
+        const bool g = j < nb && c > T;
+        const bool eq = j < nb && c == T;
         const unsigned eqm = __ballot_sync(0xffffffffu, eq);
-        const bool take = gt || (eq && eq_seen + __popc(eqm & below) < need);
+        const bool take = g || (eq && eq_seen + __popc(eqm & below) < need);
         const unsigned tm = __ballot_sync(0xffffffffu, take);
         if (take) out[written + __popc(tm & below)] = j;
         written += __popc(tm);
@@ -137,8 +161,7 @@ __device__ void warp_select(const float* sc, int nb, int n_keep, unsigned* hist,
 
 // CTA (g, h, b): query blocks i = g*QB .. g*QB + QB - 1 of head h, sample b;
 // all 8 warps compute the scores, then warp r selects query block r.
-// Shared memory: qmean [QB][hd] fp32, scores [QB][nb] fp32, 256-bin
-// histograms [8].
+// Shared memory: qmean [8][hd] fp32, scores [QB][nb] fp32.
 __global__ void __launch_bounds__(kSelThreads)
 subblock_select_kernel(const float* __restrict__ pooled, int nb, int D, int hd, int QB,
                        int n_keep, int32_t* __restrict__ kept) {
@@ -146,47 +169,74 @@ subblock_select_kernel(const float* __restrict__ pooled, int nb, int D, int hd, 
     const int h = blockIdx.y, b = blockIdx.z;
     const int i0 = blockIdx.x * QB;
     const int nq = min(QB, nb - i0);
-    float* qmean = reinterpret_cast<float*>(sm);                       // QB * hd
-    float* scores = qmean + QB * hd;                                   // QB * nb
-    unsigned* hist = reinterpret_cast<unsigned*>(scores + static_cast<int64_t>(QB) * nb);
+    float* qmean = reinterpret_cast<float*>(sm);                       // 8 * hd
+    float* scores = qmean + 8 * hd;                                    // QB * nb
     const float* qsrc = pooled + (static_cast<int64_t>(b) * 2 + 0) * nb * D + h * hd;
     const float* ksrc = pooled + (static_cast<int64_t>(b) * 2 + 1) * nb * D + h * hd;
-    for (int e = threadIdx.x; e < nq * hd; e += kSelThreads) {
+    // rows past the last query block are zeros (their scores are not kept),
+    // so the score loop below has no per-row test
+    for (int e = threadIdx.x; e < 8 * hd; e += kSelThreads) {
         const int r = e / hd, d = e - r * hd;
-        qmean[r * hd + d] = qsrc[static_cast<int64_t>(i0 + r) * D + d];
+        qmean[r * hd + d] = r < nq ? qsrc[static_cast<int64_t>(i0 + r) * D + d] : 0.0f;
     }
     __syncthreads();
-    // scores: thread t takes key blocks t, t + 256, ...; dot products in
-    // fp32, d in increasing order
-    for (int j = threadIdx.x; j < nb; j += kSelThreads) {
-        const float4* kv = reinterpret_cast<const float4*>(ksrc + static_cast<int64_t>(j) * D);
-        float acc[8];
+    // scores: thread t takes key blocks t + 256 u (u < kKeysPerThread) per
+    // pass; each 16-byte query read feeds 16 FMAs.  Dot products in fp32,
+    // d in increasing order.  hd % 8 == 0, so every float4 is aligned.
+    const float4* q4 = reinterpret_cast<const float4*>(qmean);
+    const int hd4 = hd / 4;
+    for (int jb = 0; jb < nb; jb += kKeysPerThread * kSelThreads) {
+        const float4* kv[kKeysPerThread];
+        bool live[kKeysPerThread];
 #pragma unroll
-        for (int r = 0; r < 8; ++r) acc[r] = 0.0f;
-        for (int d4 = 0; d4 < hd / 4; ++d4) {
-            const float4 kk = __ldg(kv + d4);
+        for (int u = 0; u < kKeysPerThread; ++u) {
+            const int j = jb + u * kSelThreads + threadIdx.x;
+            live[u] = j < nb;
+            kv[u] = reinterpret_cast<const float4*>(ksrc + static_cast<int64_t>(live[u] ? j : 0) * D);
+        }
+        float acc[kKeysPerThread][8];
+#pragma unroll
+        for (int u = 0; u < kKeysPerThread; ++u)
+#pragma unroll
+            for (int r = 0; r < 8; ++r) acc[u][r] = 0.0f;
+        for (int d4 = 0; d4 < hd4; ++d4) {
+            float4 kk[kKeysPerThread];
+#pragma unroll
+            for (int u = 0; u < kKeysPerThread; ++u) kk[u] = __ldg(kv[u] + d4);
 #pragma unroll
             for (int r = 0; r < 8; ++r) {
-                if (r < nq) {
-                    const float* qm = qmean + r * hd + 4 * d4;
-                    acc[r] = __fmaf_rn(qm[0], kk.x, acc[r]);
-                    acc[r] = __fmaf_rn(qm[1], kk.y, acc[r]);
-                    acc[r] = __fmaf_rn(qm[2], kk.z, acc[r]);
-                    acc[r] = __fmaf_rn(qm[3], kk.w, acc[r]);
+                const float4 qq = q4[r * hd4 + d4];
+#pragma unroll
+                for (int u = 0; u < kKeysPerThread; ++u) {
+                    acc[u][r] = __fmaf_rn(qq.x, kk[u].x, acc[u][r]);
+                    acc[u][r] = __fmaf_rn(qq.y, kk[u].y, acc[u][r]);
+                    acc[u][r] = __fmaf_rn(qq.z, kk[u].z, acc[u][r]);
+                    acc[u][r] = __fmaf_rn(qq.w, kk[u].w, acc[u][r]);
                 }
             }
         }
 #pragma unroll
-        for (int r = 0; r < 8; ++r)
-            if (r < nq) scores[static_cast<int64_t>(r) * nb + j] = acc[r];
+        for (int u = 0; u < kKeysPerThread; ++u) {
+            const int j = jb + u * kSelThreads + threadIdx.x;
+#pragma unroll
+            for (int r = 0; r < 8; ++r)
+                if (live[u] && r < nq) scores[static_cast<int64_t>(r) * nb + j] = acc[u][r];
+        }
     }
     __syncthreads();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (warp < nq) {
         int32_t* out =
             kept + ((static_cast<int64_t>(b) * gridDim.y + h) * nb + i0 + warp) * n_keep;
-        warp_select(scores + static_cast<int64_t>(warp) * nb, nb, n_keep, hist + 256 * warp, out,
-                    lane);
+        const float* sc = scores + static_cast<int64_t>(warp) * nb;
+        if (nb <= 256)
+            warp_select_reg<8>(sc, nb, n_keep, out, lane);
+        else if (nb <= 512)
+            warp_select_reg<16>(sc, nb, n_keep, out, lane);
+        else if (nb <= 1024)
+            warp_select_reg<32>(sc, nb, n_keep, out, lane);
+        else
+            warp_select_smem(sc, nb, n_keep, out, lane);
     }
 }
 
@@ -243,8 +293,7 @@ extern "C" int dit_subblock_router(const uint16_t* q, const uint16_t* k, int64_t
     // query blocks per CTA (one per warp): as many as fit in about 96 KB of scores
     int QB = 8;
     while (QB > 1 && static_cast<size_t>(QB) * nb * 4 > 96 * 1024) QB >>= 1;
-    const size_t smem = static_cast<size_t>(QB) * hd * 4 + static_cast<size_t>(QB) * nb * 4 +
-                        8 * 256 * sizeof(unsigned);
+    const size_t smem = static_cast<size_t>(8) * hd * 4 + static_cast<size_t>(QB) * nb * 4;
     if (cudaFuncSetAttribute(subblock_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(smem)) != cudaSuccess)
         return DIT_ERR_LAUNCH;
