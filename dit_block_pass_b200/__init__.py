@@ -46,7 +46,7 @@ launch_counts = {
     "cachedit_residual_diff": 2, "cachedit_residual_sums": 2, "cachedit_decide": 1,
     "cachedit_residual_diff_noalloc": 2, "cachedit_residual_store": 1,
     "cachedit_residual_apply": 1, "swiglu_gemm": 1, "gemm_gated_residual": 1,
-    "subblock_router": 2, "block_sparse_attention": 1,
+    "subblock_router": 3, "block_sparse_attention": 1,
 }
 
 

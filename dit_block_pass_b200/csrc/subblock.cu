@@ -10,17 +10,18 @@
 // product of the two means and keeps the n_keep = ceil((1 - s) n_blocks)
 // best key blocks (ties to the lower index), listed in increasing order.
 //
-// Two kernels:
+// Three kernels:
 //   subblock_pool_kernel    one pass over q and k (HBM bound): CTA (j, b, t)
 //                           sums the rows of block j of sample b of tensor t
 //                           (q or k) for every column, 16-byte loads, fp32,
 //                           and writes the means [B, 2, n_blocks, H*hd].
-//   subblock_select_kernel  CTA (up to 8 query blocks, h, b): the query means
-//                           in shared memory, one pass over the key means of
-//                           head h (L2 resident) for all scores, then one
-//                           warp per query block: the n_keep-th largest
-//                           score found bit by bit with warp-wide counts
-//                           (the scores in registers up to 1024 key
+//   subblock_scores_kernel  per (sample, head) the n_blocks x n_blocks fp32
+//                           scores as a tiled GEMM of the L2-resident means
+//                           (128 x 128 tiles, 8 x 8 per thread), into the
+//                           workspace after the means.
+//   subblock_select_kernel  one warp per query block: the n_keep-th largest
+//                           score of its row found bit by bit with warp-wide
+//                           counts (the row in registers up to 2048 key
 //                           blocks) and an ordered ballot compaction that
 //                           writes the kept indices in increasing order,
 //                           ties at the threshold to the lower index.
@@ -33,7 +34,8 @@ namespace {
 
 constexpr int kPoolThreads = 256;
 constexpr int kSelThreads = 256;
-constexpr int kKeysPerThread = 4;       // key blocks per thread and pass of the score loop
+constexpr int kScoreTile = 128;          // query x key blocks per score tile
+constexpr int kScoreDK = 32;             // d per staged slice of the score GEMM
 constexpr int kMaxBlocks = 8192;           // key blocks per sample
 
 // Means of the rows of one block, every column: thread t takes column
@@ -159,85 +161,96 @@ __device__ void warp_select_smem(const float* sc, int nb, int n_keep, int32_t* o
     }
 }
 
-// CTA (g, h, b): query blocks i = g*QB .. g*QB + QB - 1 of head h, sample b;
-// all 8 warps compute the scores, then warp r selects query block r.
-// Shared memory: qmean [8][hd] fp32, scores [QB][nb] fp32.
+// Scores of one (sample, head) as a tiled fp32 GEMM: CTA (t, h, b) forms
+// the 128 x 128 tile t of scores[b, h, i, j] = sum_d qm[i, d] km[j, d] from
+// the block means, staging 32-wide d slices of both operands transposed in
+// shared memory.  Thread (ty, tx) keeps an 8 x 8 tile: query rows 4ty.. and
+// 64 + 4ty.., key columns 4tx.. and 64 + 4tx.., so that each 16-byte read of
+// a warp covers contiguous words.  Every score is the fp32 fmaf chain over
+// d = 0, 1, ..., hd - 1 from +0 (no padded terms: a zero product could turn
+// a -0 score into +0 and reorder an exact tie).
 __global__ void __launch_bounds__(kSelThreads)
-subblock_select_kernel(const float* __restrict__ pooled, int nb, int D, int hd, int QB,
-                       int n_keep, int32_t* __restrict__ kept) {
-    extern __shared__ __align__(16) unsigned char sm[];
+subblock_scores_kernel(const float* __restrict__ pooled, int nb, int D, int hd,
+                       float* __restrict__ scores) {
+    __shared__ __align__(16) float qs[kScoreDK][kScoreTile + 4];
+    __shared__ __align__(16) float ks[kScoreDK][kScoreTile + 4];
+    const int tiles = (nb + kScoreTile - 1) / kScoreTile;
+    const int i0 = (blockIdx.x / tiles) * kScoreTile, j0 = (blockIdx.x % tiles) * kScoreTile;
     const int h = blockIdx.y, b = blockIdx.z;
-    const int i0 = blockIdx.x * QB;
-    const int nq = min(QB, nb - i0);
-    float* qmean = reinterpret_cast<float*>(sm);                       // 8 * hd
-    float* scores = qmean + 8 * hd;                                    // QB * nb
     const float* qsrc = pooled + (static_cast<int64_t>(b) * 2 + 0) * nb * D + h * hd;
     const float* ksrc = pooled + (static_cast<int64_t>(b) * 2 + 1) * nb * D + h * hd;
-    // rows past the last query block are zeros (their scores are not kept),
-    // so the score loop below has no per-row test
-    for (int e = threadIdx.x; e < 8 * hd; e += kSelThreads) {
-        const int r = e / hd, d = e - r * hd;
-        qmean[r * hd + d] = r < nq ? qsrc[static_cast<int64_t>(i0 + r) * D + d] : 0.0f;
-    }
-    __syncthreads();
-    // scores: thread t takes key blocks t + 256 u (u < kKeysPerThread) per
-    // pass; each 16-byte query read feeds 16 FMAs.  Dot products in fp32,
-    // d in increasing order.  hd % 8 == 0, so every float4 is aligned.
-    const float4* q4 = reinterpret_cast<const float4*>(qmean);
-    const int hd4 = hd / 4;
-    for (int jb = 0; jb < nb; jb += kKeysPerThread * kSelThreads) {
-        const float4* kv[kKeysPerThread];
-        bool live[kKeysPerThread];
+    const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+    constexpr int kHalf = kScoreTile / 2;
+    float acc[8][8];
 #pragma unroll
-        for (int u = 0; u < kKeysPerThread; ++u) {
-            const int j = jb + u * kSelThreads + threadIdx.x;
-            live[u] = j < nb;
-            kv[u] = reinterpret_cast<const float4*>(ksrc + static_cast<int64_t>(live[u] ? j : 0) * D);
+    for (int r = 0; r < 8; ++r)
+#pragma unroll
+        for (int c = 0; c < 8; ++c) acc[r][c] = 0.0f;
+    for (int d0 = 0; d0 < hd; d0 += kScoreDK) {
+        const int dn = min(kScoreDK, hd - d0);          // a multiple of 8
+        for (int e = threadIdx.x; e < kScoreTile * (kScoreDK / 4); e += kSelThreads) {
+            const int r = e / (kScoreDK / 4), c4 = e % (kScoreDK / 4);
+            float4 a = make_float4(0.f, 0.f, 0.f, 0.f), bk = a;
+            if (4 * c4 < dn) {
+                if (i0 + r < nb)
+                    a = *reinterpret_cast<const float4*>(qsrc + static_cast<int64_t>(i0 + r) * D +
+                                                         d0 + 4 * c4);
+                if (j0 + r < nb)
+                    bk = *reinterpret_cast<const float4*>(ksrc + static_cast<int64_t>(j0 + r) * D +
+                                                          d0 + 4 * c4);
+            }
+            qs[4 * c4 + 0][r] = a.x; qs[4 * c4 + 1][r] = a.y;
+            qs[4 * c4 + 2][r] = a.z; qs[4 * c4 + 3][r] = a.w;
+            ks[4 * c4 + 0][r] = bk.x; ks[4 * c4 + 1][r] = bk.y;
+            ks[4 * c4 + 2][r] = bk.z; ks[4 * c4 + 3][r] = bk.w;
         }
-        float acc[kKeysPerThread][8];
+        __syncthreads();
 #pragma unroll
-        for (int u = 0; u < kKeysPerThread; ++u)
+        for (int d = 0; d < kScoreDK; ++d) {
+            if (d < dn) {
+                const float4 q0 = *reinterpret_cast<const float4*>(&qs[d][4 * ty]);
+                const float4 q1 = *reinterpret_cast<const float4*>(&qs[d][kHalf + 4 * ty]);
+                const float4 k0 = *reinterpret_cast<const float4*>(&ks[d][4 * tx]);
+                const float4 k1 = *reinterpret_cast<const float4*>(&ks[d][kHalf + 4 * tx]);
+                const float qv[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
+                const float kv[8] = {k0.x, k0.y, k0.z, k0.w, k1.x, k1.y, k1.z, k1.w};
 #pragma unroll
-            for (int r = 0; r < 8; ++r) acc[u][r] = 0.0f;
-        for (int d4 = 0; d4 < hd4; ++d4) {
-            float4 kk[kKeysPerThread];
+                for (int r = 0; r < 8; ++r)
 #pragma unroll
-            for (int u = 0; u < kKeysPerThread; ++u) kk[u] = __ldg(kv[u] + d4);
-#pragma unroll
-            for (int r = 0; r < 8; ++r) {
-                const float4 qq = q4[r * hd4 + d4];
-#pragma unroll
-                for (int u = 0; u < kKeysPerThread; ++u) {
-                    acc[u][r] = __fmaf_rn(qq.x, kk[u].x, acc[u][r]);
-                    acc[u][r] = __fmaf_rn(qq.y, kk[u].y, acc[u][r]);
-                    acc[u][r] = __fmaf_rn(qq.z, kk[u].z, acc[u][r]);
-                    acc[u][r] = __fmaf_rn(qq.w, kk[u].w, acc[u][r]);
-                }
+                    for (int c = 0; c < 8; ++c) acc[r][c] = __fmaf_rn(qv[r], kv[c], acc[r][c]);
             }
         }
+        __syncthreads();
+    }
+    float* out = scores + (static_cast<int64_t>(b) * gridDim.y + h) * nb * nb;
 #pragma unroll
-        for (int u = 0; u < kKeysPerThread; ++u) {
-            const int j = jb + u * kSelThreads + threadIdx.x;
+    for (int r = 0; r < 8; ++r) {
+        const int i = i0 + (r < 4 ? 4 * ty + r : kHalf + 4 * ty + r - 4);
 #pragma unroll
-            for (int r = 0; r < 8; ++r)
-                if (live[u] && r < nq) scores[static_cast<int64_t>(r) * nb + j] = acc[u][r];
+        for (int c = 0; c < 8; ++c) {
+            const int j = j0 + (c < 4 ? 4 * tx + c : kHalf + 4 * tx + c - 4);
+            if (i < nb && j < nb) out[static_cast<int64_t>(i) * nb + j] = acc[r][c];
         }
     }
-    __syncthreads();
+}
+
+// CTA (g, h, b): warp w selects query block i = 8 g + w of head h, sample b
+// from its score row; KPL > 0: nb <= 32 KPL, the row in registers.
+template <int KPL>
+__global__ void __launch_bounds__(kSelThreads)
+subblock_select_kernel(const float* __restrict__ scores, int nb, int n_keep,
+                       int32_t* __restrict__ kept) {
+    const int h = blockIdx.y, b = blockIdx.z;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    if (warp < nq) {
-        int32_t* out =
-            kept + ((static_cast<int64_t>(b) * gridDim.y + h) * nb + i0 + warp) * n_keep;
-        const float* sc = scores + static_cast<int64_t>(warp) * nb;
-        if (nb <= 256)
-            warp_select_reg<8>(sc, nb, n_keep, out, lane);
-        else if (nb <= 512)
-            warp_select_reg<16>(sc, nb, n_keep, out, lane);
-        else if (nb <= 1024)
-            warp_select_reg<32>(sc, nb, n_keep, out, lane);
-        else
-            warp_select_smem(sc, nb, n_keep, out, lane);
-    }
+    const int i = blockIdx.x * (kSelThreads / 32) + warp;
+    if (i >= nb) return;
+    const int64_t row = (static_cast<int64_t>(b) * gridDim.y + h) * nb + i;
+    const float* sc = scores + row * nb;
+    int32_t* out = kept + row * n_keep;
+    if constexpr (KPL > 0)
+        warp_select_reg<KPL>(sc, nb, n_keep, out, lane);
+    else
+        warp_select_smem(sc, nb, n_keep, out, lane);
 }
 
 int keep_count(int64_t n_blocks, double sparsity) {
@@ -259,7 +272,9 @@ extern "C" int dit_subblock_keep_count(int64_t n_blocks, double sparsity) {
 extern "C" size_t dit_subblock_workspace_bytes(int B, int64_t N, int H, int hd, int block) {
     if (B < 0 || N < 0 || H < 1 || hd < 1 || block < 1) return 0;
     const int64_t nb = (N + block - 1) / block;
-    return static_cast<size_t>(B) * 2 * nb * H * hd * sizeof(float);
+    // the block means [B, 2, nb, H*hd], then the scores [B, H, nb, nb], fp32
+    return (static_cast<size_t>(B) * 2 * nb * H * hd + static_cast<size_t>(B) * H * nb * nb) *
+           sizeof(float);
 }
 
 extern "C" int dit_subblock_router(const uint16_t* q, const uint16_t* k, int64_t row_stride,
@@ -290,14 +305,22 @@ extern "C" int dit_subblock_router(const uint16_t* q, const uint16_t* k, int64_t
         block, nb, static_cast<int>(D / 8), pooled);
     int rc = launch_status();
     if (rc) return rc;
-    // query blocks per CTA (one per warp): as many as fit in about 96 KB of scores
-    int QB = 8;
-    while (QB > 1 && static_cast<size_t>(QB) * nb * 4 > 96 * 1024) QB >>= 1;
-    const size_t smem = static_cast<size_t>(8) * hd * 4 + static_cast<size_t>(QB) * nb * 4;
-    if (cudaFuncSetAttribute(subblock_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(smem)) != cudaSuccess)
-        return DIT_ERR_LAUNCH;
-    subblock_select_kernel<<<dim3((nb + QB - 1) / QB, H, B), kSelThreads, smem, st>>>(
-        pooled, nb, static_cast<int>(D), hd, QB, n_keep, kept);
+    float* scores = pooled + static_cast<int64_t>(B) * 2 * nb * D;
+    const int64_t tiles = (nb + kScoreTile - 1) / kScoreTile;
+    subblock_scores_kernel<<<dim3(static_cast<unsigned>(tiles * tiles), H, B), kSelThreads, 0,
+                             st>>>(pooled, nb, static_cast<int>(D), hd, scores);
+    rc = launch_status();
+    if (rc) return rc;
+    const dim3 sel((nb + 7) / 8, H, B);
+    if (nb <= 256)
+        subblock_select_kernel<8><<<sel, kSelThreads, 0, st>>>(scores, nb, n_keep, kept);
+    else if (nb <= 512)
+        subblock_select_kernel<16><<<sel, kSelThreads, 0, st>>>(scores, nb, n_keep, kept);
+    else if (nb <= 1024)
+        subblock_select_kernel<32><<<sel, kSelThreads, 0, st>>>(scores, nb, n_keep, kept);
+    else if (nb <= 2048)
+        subblock_select_kernel<64><<<sel, kSelThreads, 0, st>>>(scores, nb, n_keep, kept);
+    else
+        subblock_select_kernel<0><<<sel, kSelThreads, 0, st>>>(scores, nb, n_keep, kept);
     return launch_status();
 }

@@ -345,7 +345,8 @@ int dit_gemm_gated_residual(const uint16_t* h, const uint16_t* w, const uint16_t
  *   kept       device int32 [B, H, n_blocks, n_keep]: the kept key blocks of
  *              each query block, in increasing order.
  *   workspace  device, >= dit_subblock_workspace_bytes(...) bytes (the block
- *              means, [B, 2, n_blocks, H*hd] fp32), 16-byte aligned.
+ *              means [B, 2, n_blocks, H*hd], then the scores [B, H, n_blocks,
+ *              n_blocks], both fp32), 16-byte aligned.
  * 0 <= sparsity < 1 (else DIT_ERR_VALUE); n_blocks <= 8192.  Which steps use
  * the router (the report: from the 10th) is the caller's choice.
  */

@@ -277,7 +277,7 @@ def test_subblock_router_host(lib):
     assert lib.dit_subblock_keep_count(10, 1.0) == E["VALUE"]
     f = lib.dit_subblock_router
     ws = lib.dit_subblock_workspace_bytes(1, 256, 2, 64, 128)
-    assert ws == 2 * 2 * 2 * 64 * 4
+    assert ws == (2 * 2 * 2 * 64 + 2 * 2 * 2) * 4       # block means, then scores
     assert f(A, A + 0x1000, 128, 1, 0, 2, 64, 128, 0.75, A + 0x2000, A + 0x3000, ws, None) == 0
     assert f(A, A + 0x1000, 128, 1, 256, 2, 60, 128, 0.75, A + 0x2000, A + 0x3000, ws, None) == E["SHAPE"]
     assert f(A, A + 0x1000, 128, 1, 256, 2, 64, 128, 1.0, A + 0x2000, A + 0x3000, ws, None) == E["VALUE"]
