@@ -11,10 +11,11 @@
 // best key blocks (ties to the lower index), listed in increasing order.
 //
 // Three kernels:
-//   subblock_pool_kernel    one pass over q and k (HBM bound): CTA (j, b, t)
-//                           sums the rows of block j of sample b of tensor t
-//                           (q or k) for every column, 16-byte loads, fp32,
-//                           and writes the means [B, 2, n_blocks, H*hd].
+//   subblock_pool_kernel    one pass over q and k (HBM bound): CTA (j, b, t,
+//                           column chunk) sums the rows of block j of sample
+//                           b of tensor t (q or k), a 16-byte column vector
+//                           per thread, fp32, and writes the means
+//                           [B, 2, n_blocks, H*hd].
 //   subblock_scores_kernel  per (sample, head) the n_blocks x n_blocks fp32
 //                           scores as a tiled GEMM of the L2-resident means
 //                           (128 x 128 tiles, 8 x 8 per thread), into the
@@ -32,50 +33,51 @@
 namespace dit {
 namespace {
 
-constexpr int kPoolThreads = 256;
+constexpr int kPoolThreads = 128;
 constexpr int kSelThreads = 256;
 constexpr int kScoreTile = 128;          // query x key blocks per score tile
 constexpr int kScoreDK = 32;             // d per staged slice of the score GEMM
 constexpr int kMaxBlocks = 8192;           // key blocks per sample
 
-// Means of the rows of one block, every column: thread t takes column
-// vectors t, t + 256, ...; fp32 sums over at most `block` rows, one divide.
+// Means of the rows of one block: CTA (j, b, 2 c + t) takes column vectors
+// 128 c .. 128 c + 127 of block j, sample b, tensor t (q or k), one per
+// thread; fp32 sums over at most `block` rows in row order (8 rows in
+// flight), one divide.
 __global__ void __launch_bounds__(kPoolThreads)
 subblock_pool_kernel(const uint4* __restrict__ q, const uint4* __restrict__ k, int64_t stride_v,
                      int64_t N, int block, int nb, int Dv, float* __restrict__ pooled) {
-    const int j = blockIdx.x, b = blockIdx.y, t = blockIdx.z;
+    const int j = blockIdx.x, b = blockIdx.y, t = blockIdx.z & 1;
+    const int v = (blockIdx.z >> 1) * kPoolThreads + threadIdx.x;
+    if (v >= Dv) return;
     const uint4* src = t == 0 ? q : k;
     const int64_t r0 = static_cast<int64_t>(j) * block;
     const int64_t r1 = r0 + block < N ? r0 + block : N;
     const float count = static_cast<float>(r1 - r0);
     float* out = pooled + ((static_cast<int64_t>(b) * 2 + t) * nb + j) * (static_cast<int64_t>(Dv) * 8);
-    for (int v = threadIdx.x; v < Dv; v += kPoolThreads) {
-        float s[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-        const uint4* p = src + (static_cast<int64_t>(b) * N + r0) * stride_v + v;
-        int64_t r = r0;
-        // four rows in flight at a time
-        for (; r + 4 <= r1; r += 4, p += 4 * stride_v) {
-            uint4 a[4];
+    float s[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    const uint4* p = src + (static_cast<int64_t>(b) * N + r0) * stride_v + v;
+    int64_t r = r0;
+    for (; r + 8 <= r1; r += 8, p += 8 * stride_v) {
+        uint4 a[8];
 #pragma unroll
-            for (int u = 0; u < 4; ++u) a[u] = ld_stream(p + u * stride_v);
+        for (int u = 0; u < 8; ++u) a[u] = ld_stream(p + u * stride_v);
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                float f[8];
-                unpack8(a[u], f);
-#pragma unroll
-                for (int i = 0; i < 8; ++i) s[i] += f[i];
-            }
-        }
-        for (; r < r1; ++r, p += stride_v) {
+        for (int u = 0; u < 8; ++u) {
             float f[8];
-            unpack8(ld_stream(p), f);
+            unpack8(a[u], f);
 #pragma unroll
             for (int i = 0; i < 8; ++i) s[i] += f[i];
         }
-        float4* o = reinterpret_cast<float4*>(out + 8 * v);
-        o[0] = make_float4(s[0] / count, s[1] / count, s[2] / count, s[3] / count);
-        o[1] = make_float4(s[4] / count, s[5] / count, s[6] / count, s[7] / count);
     }
+    for (; r < r1; ++r, p += stride_v) {
+        float f[8];
+        unpack8(ld_stream(p), f);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) s[i] += f[i];
+    }
+    float4* o = reinterpret_cast<float4*>(out + 8 * v);
+    o[0] = make_float4(s[0] / count, s[1] / count, s[2] / count, s[3] / count);
+    o[1] = make_float4(s[4] / count, s[5] / count, s[6] / count, s[7] / count);
 }
 
 // Order-preserving map of a float to uint32 (larger float -> larger code).
@@ -161,6 +163,22 @@ __device__ void warp_select_smem(const float* sc, int nb, int n_keep, int32_t* o
     }
 }
 
+// One d step of a thread's 8 x 8 score tile (see subblock_scores_kernel).
+__device__ __forceinline__ void score_step(const float* qrow, const float* krow, int tx, int ty,
+                                           float (&acc)[8][8]) {
+    constexpr int kHalf = kScoreTile / 2;
+    const float4 q0 = *reinterpret_cast<const float4*>(qrow + 4 * ty);
+    const float4 q1 = *reinterpret_cast<const float4*>(qrow + kHalf + 4 * ty);
+    const float4 k0 = *reinterpret_cast<const float4*>(krow + 4 * tx);
+    const float4 k1 = *reinterpret_cast<const float4*>(krow + kHalf + 4 * tx);
+    const float qv[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
+    const float kv[8] = {k0.x, k0.y, k0.z, k0.w, k1.x, k1.y, k1.z, k1.w};
+#pragma unroll
+    for (int r = 0; r < 8; ++r)
+#pragma unroll
+        for (int c = 0; c < 8; ++c) acc[r][c] = __fmaf_rn(qv[r], kv[c], acc[r][c]);
+}
+
 // Scores of one (sample, head) as a tiled fp32 GEMM: CTA (t, h, b) forms
 // the 128 x 128 tile t of scores[b, h, i, j] = sum_d qm[i, d] km[j, d] from
 // the block means, staging 32-wide d slices of both operands transposed in
@@ -205,20 +223,15 @@ subblock_scores_kernel(const float* __restrict__ pooled, int nb, int D, int hd,
             ks[4 * c4 + 2][r] = bk.z; ks[4 * c4 + 3][r] = bk.w;
         }
         __syncthreads();
+        // a full slice runs without a per-step test (a branch in the unrolled
+        // loop would keep the shared-memory reads from being issued ahead)
+        if (dn == kScoreDK) {
 #pragma unroll
-        for (int d = 0; d < kScoreDK; ++d) {
-            if (d < dn) {
-                const float4 q0 = *reinterpret_cast<const float4*>(&qs[d][4 * ty]);
-                const float4 q1 = *reinterpret_cast<const float4*>(&qs[d][kHalf + 4 * ty]);
-                const float4 k0 = *reinterpret_cast<const float4*>(&ks[d][4 * tx]);
-                const float4 k1 = *reinterpret_cast<const float4*>(&ks[d][kHalf + 4 * tx]);
-                const float qv[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
-                const float kv[8] = {k0.x, k0.y, k0.z, k0.w, k1.x, k1.y, k1.z, k1.w};
+            for (int d = 0; d < kScoreDK; ++d) score_step(qs[d], ks[d], tx, ty, acc);
+        } else {
 #pragma unroll
-                for (int r = 0; r < 8; ++r)
-#pragma unroll
-                    for (int c = 0; c < 8; ++c) acc[r][c] = __fmaf_rn(qv[r], kv[c], acc[r][c]);
-            }
+            for (int d = 0; d < kScoreDK; ++d)
+                if (d < dn) score_step(qs[d], ks[d], tx, ty, acc);
         }
         __syncthreads();
     }
@@ -300,7 +313,8 @@ extern "C" int dit_subblock_router(const uint16_t* q, const uint16_t* k, int64_t
     if (!workspace || workspace_bytes < need || !aligned16(workspace)) return DIT_ERR_WORKSPACE;
     float* pooled = static_cast<float*>(workspace);
     cudaStream_t st = as_stream(stream);
-    subblock_pool_kernel<<<dim3(nb, B, 2), kPoolThreads, 0, st>>>(
+    const int chunks = static_cast<int>((D / 8 + kPoolThreads - 1) / kPoolThreads);
+    subblock_pool_kernel<<<dim3(nb, B, 2 * chunks), kPoolThreads, 0, st>>>(
         reinterpret_cast<const uint4*>(q), reinterpret_cast<const uint4*>(k), row_stride / 8, N,
         block, nb, static_cast<int>(D / 8), pooled);
     int rc = launch_status();
