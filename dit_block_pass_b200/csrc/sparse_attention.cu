@@ -16,12 +16,16 @@
 //             block, one buffer each (128-byte swizzle): K_{n+1} lands while
 //             block n's softmax runs, V_{n+1} while S_{n+1} and its softmax run.
 //   warp 1    one thread issues tcgen05.mma: S_n = Q K_n^T (shared-memory
-//             operands, fp32 into TMEM columns [0, 128)), then, once the
-//             softmax has written P_n, O += P_n V_n with P read from TMEM
-//             (the A operand in tensor memory, two bf16 per column over S_n's
-//             first 64 columns) and V as an MN-major shared-memory operand
-//             (no transpose).  S_{n+1} is issued after P_n V_n has read P_n.
-//   warps 2-5 softmax, thread = query row (TMEM lane): tcgen05.ld the S row,
+//             operands, fp32 into TMEM columns [0, 128)) as two N = 64 halves,
+//             and, once the softmax has written P_n, O += P_n V_n with P read
+//             from TMEM (the A operand in tensor memory, two bf16 per column
+//             over S_n's first 64 columns) and V as an MN-major shared-memory
+//             operand (no transpose).  Keys 64..127 of S_{n+1} go into the
+//             columns P_n does not use as soon as the softmax has read S_n
+//             (so they run during softmax n and P_n V_n); keys 0..63 follow
+//             once P_n V_n has read P_n.
+//   warps 2-5 softmax, thread = query row (TMEM lane): tcgen05.ld the S row
+//             (then report S_n read),
 //             mask keys past the sample's last token, weights 2^(s - m) in
 //             fp32 with lazy rescaling (the reference max m moves, and O and
 //             the row sum are rescaled in TMEM, only when a row's block max
@@ -46,7 +50,7 @@ constexpr uint32_t kTmemColsA = 256;           // two CTAs share an SM's 512 col
 constexpr uint32_t kColO = 128;                 // S (and P over it) in [0, 128), O in [128, 256)
 // Q, K, V, then barriers
 constexpr size_t kSmemA = 3 * kTile + 1024 + 256;
-constexpr uint32_t kIdescS = idesc_f16(128, 128, false, false);    // S = Q K^T
+constexpr uint32_t kIdescS64 = idesc_f16(128, 64, false, false);   // half of S = Q K^T
 constexpr uint32_t kIdescO = idesc_f16(128, 128, false, true);     // O += P V (V MN-major)
 
 // D (TMEM) += A (TMEM, K-major: row m in lane m, two bf16 per column) * B
@@ -59,6 +63,18 @@ __device__ __forceinline__ void mma_f16_ts(uint32_t tmem_d, uint32_t tmem_a, uin
         "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(tmem_d),
         "r"(tmem_a), "l"(db), "r"(idesc), "r"(accumulate)
         : "memory");
+}
+
+// Keys k0 .. k0 + 63 of S = Q K^T (k0 = 0 or 64) into TMEM columns k0 ..
+// k0 + 63: eight M = 128, N = 64, K = 16 products; rows k0.. of each 64-wide
+// K half start k0 * 128 bytes in (a multiple of the 1024-byte swizzle atom).
+__device__ __forceinline__ void issue_s(uint32_t tmem, uint32_t sQ, uint32_t sK, int k0) {
+#pragma unroll
+    for (int kk = 0; kk < kHd / 16; ++kk) {
+        const uint32_t off = (kk >> 2) * kHalfTile + (kk & 3) * 32;
+        mma_f16(tmem + k0, sw128_desc(sQ + off), sw128_desc(sK + off + k0 * 128), kIdescS64,
+                kk != 0 ? 1u : 0u);
+    }
 }
 
 struct AttnParams {
@@ -88,6 +104,7 @@ block_sparse_attention_kernel(const __grid_constant__ CUtensorMap map_q,
     const uint32_t bar_p_full = bar + 48;           // P_n in TMEM, O rescaled (4 arrivals)
     const uint32_t bar_o_done = bar + 56;           // P_n V_n done: S/P columns and O free
     const uint32_t bar_drain = bar + 64;
+    const uint32_t bar_s_free = bar + 72;           // S_n read into registers (4 arrivals)
     volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(gen_base + 3 * kTile + 80);
     volatile int* abort = reinterpret_cast<volatile int*>(gen_base + 3 * kTile + 84);
 
@@ -107,6 +124,7 @@ block_sparse_attention_kernel(const __grid_constant__ CUtensorMap map_q,
         mbar_init(bar_p_full, 4);
         mbar_init(bar_o_done, 1);
         mbar_init(bar_drain, 1);
+        mbar_init(bar_s_free, 4);
         *abort = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
@@ -156,36 +174,58 @@ block_sparse_attention_kernel(const __grid_constant__ CUtensorMap map_q,
     } else if (warp == 1) {
         if (lane == 0) {
             if (!mbar_wait(bar_q, 0, abort)) failed = true;
+            // S_0, both key halves
+            if (!failed && nk > 0) {
+                if (!mbar_wait(bar_k_full, 0, abort)) {
+                    failed = true;
+                } else {
+                    fence_after_sync();
+                    issue_s(tmem, sQ, sK, 64);
+                    issue_s(tmem, sQ, sK, 0);
+                    mma_commit(bar_s_full);
+                    mma_commit(bar_k_empty);
+                }
+            }
             for (int n = 0; n < nk && !failed; ++n) {
-                // S_n = Q K_n^T, once K_n is in and P_{n-1} V_{n-1} has read the
-                // columns S_n overwrites
-                if (!mbar_wait(bar_k_full, n & 1, abort) ||
-                    (n >= 1 && !mbar_wait(bar_o_done, (n - 1) & 1, abort))) {
+                const bool more = n + 1 < nk;
+                // keys 64..127 of S_{n+1} (columns P_n does not use) once the
+                // softmax has read S_n and K_{n+1} is in, and P_n V_n once P_n
+                // is written: whichever is ready first
+                bool b_done = !more, pv_done = false;
+                const unsigned long long t0 = now_ns();
+                for (uint32_t it = 0; !(b_done && pv_done); ++it) {
+                    if (!b_done && mbar_try(bar_s_free, n & 1) &&
+                        mbar_try(bar_k_full, (n + 1) & 1)) {
+                        fence_after_sync();
+                        issue_s(tmem, sQ, sK, 64);
+                        b_done = true;
+                    }
+                    if (!pv_done && mbar_try(bar_p_full, n & 1) && mbar_try(bar_v_full, n & 1)) {
+                        fence_after_sync();
+#pragma unroll
+                        for (int kk = 0; kk < kBlk / 16; ++kk)
+                            mma_f16_ts(tmem + kColO, tmem + 8 * kk,
+                                       sw128_desc_mn(sV + kk * 2048, kHalfTile), kIdescO,
+                                       (n | kk) != 0 ? 1u : 0u);
+                        mma_commit(bar_o_done);
+                        mma_commit(bar_v_empty);
+                        pv_done = true;
+                    }
+                    if ((it & 255u) == 255u && (*abort || now_ns() - t0 > kWaitNs)) {
+                        failed = true;
+                        break;
+                    }
+                }
+                if (failed || !more) continue;
+                // keys 0..63 of S_{n+1} overwrite P_n: after P_n V_n has read it
+                if (!mbar_wait(bar_o_done, n & 1, abort)) {
                     failed = true;
                     break;
                 }
                 fence_after_sync();
-#pragma unroll
-                for (int kk = 0; kk < kHd / 16; ++kk) {
-                    const uint32_t off = (kk >> 2) * kHalfTile + (kk & 3) * 32;
-                    mma_f16(tmem, sw128_desc(sQ + off), sw128_desc(sK + off), kIdescS,
-                            kk != 0 ? 1u : 0u);
-                }
+                issue_s(tmem, sQ, sK, 0);
                 mma_commit(bar_s_full);
                 mma_commit(bar_k_empty);
-                // O += P_n V_n once the softmax has written P_n (over S_n) and
-                // rescaled O
-                if (!mbar_wait(bar_p_full, n & 1, abort) || !mbar_wait(bar_v_full, n & 1, abort)) {
-                    failed = true;
-                    break;
-                }
-                fence_after_sync();
-#pragma unroll
-                for (int kk = 0; kk < kBlk / 16; ++kk)
-                    mma_f16_ts(tmem + kColO, tmem + 8 * kk, sw128_desc_mn(sV + kk * 2048, kHalfTile),
-                               kIdescO, (n | kk) != 0 ? 1u : 0u);
-                mma_commit(bar_o_done);
-                mma_commit(bar_v_empty);
             }
             if (failed) {
                 mma_commit(bar_drain);
@@ -210,6 +250,10 @@ block_sparse_attention_kernel(const __grid_constant__ CUtensorMap map_q,
             for (int c = 0; c < kBlk / 32; ++c)
                 tmem_ld32(tmem + lane_off + 32 * c, *reinterpret_cast<float(*)[32]>(sc + 32 * c));
             tmem_wait_ld();
+            // S_n is in registers: its columns 64..127 may take S_{n+1}
+            fence_before_sync();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar_s_free);
             // keys past the sample's last token do not take part
             const int64_t j = __ldg(kept + n);
             const int64_t left = p.N - j * kBlk;
