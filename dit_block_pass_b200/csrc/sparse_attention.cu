@@ -25,9 +25,10 @@
 //             (so they run during softmax n and P_n V_n); keys 0..63 follow
 //             once P_n V_n has read P_n.
 //   warps 2-5 softmax, thread = query row (TMEM lane): tcgen05.ld the S row
-//             (then report S_n read),
-//             mask keys past the sample's last token, weights 2^(s - m) in
-//             fp32 with lazy rescaling (the reference max m moves, and O and
+//             (then report S_n read), mask keys past the sample's last token,
+//             the row max of the raw scores in four chains, weights
+//             2^(s * scale * log2 e - m) with one fma each, in fp32 with
+//             lazy rescaling (the reference max m moves, and O and
 //             the row sum are rescaled in TMEM, only when a row's block max
 //             exceeds m by more than 8, so weights stay below 2^8), and P
 //             written back into TMEM as bf16 pairs.  At the end O / l is
@@ -258,12 +259,16 @@ block_sparse_attention_kernel(const __grid_constant__ CUtensorMap map_q,
             const int64_t j = __ldg(kept + n);
             const int64_t left = p.N - j * kBlk;
             const int valid = left >= kBlk ? kBlk : (left > 0 ? static_cast<int>(left) : 0);
-            float mr = -INFINITY;
+            // the row max of the raw scores (scale > 0 and rounding is monotonic,
+            // so scaling the max equals the max of the scaled scores), in four
+            // independent chains
+            float mq[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
             for (int c = 0; c < kBlk; ++c) {
-                sc[c] = c < valid ? sc[c] * p.scale_log2 : -INFINITY;
-                mr = fmaxf(mr, sc[c]);
+                sc[c] = c < valid ? sc[c] : -INFINITY;
+                mq[c & 3] = fmaxf(mq[c & 3], sc[c]);
             }
+            const float mr = fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3])) * p.scale_log2;
             // lazy rescaling: the reference max moves (and O and l are
             // rescaled) only when some row's block max exceeds it by more than
             // 8, so the weights stay below 2^8 and most blocks skip the O
@@ -271,10 +276,11 @@ block_sparse_attention_kernel(const __grid_constant__ CUtensorMap map_q,
             const bool move = __any_sync(0xffffffffu, mr > m_run + 8.0f);
             const float mx = move ? fmaxf(m_run, mr) : m_run;
             const float alpha = move ? exp2f(m_run - mx) : 1.0f;   // 0 on the first block
+            const float nmx = -mx;
             float sum = 0.0f;
 #pragma unroll
             for (int c = 0; c < kBlk; ++c) {
-                sc[c] = exp2f(sc[c] - mx);
+                sc[c] = exp2f(fmaf(sc[c], p.scale_log2, nmx));
                 sum += sc[c];
             }
             l_run = l_run * alpha + sum;
