@@ -42,7 +42,8 @@
 //
 // Every mbarrier wait is bounded (2 s of %globaltimer); on expiry the CTA
 // records an error in the caller's status word, drains what it issued
-// (bounded as well), frees its TMEM and exits.  No cluster, no multicast.
+// (bounded as well), frees its TMEM and exits.  No cluster launch: every TMA
+// load fills this CTA's own shared memory.
 #include "tcgen05.cuh"
 
 namespace dit {
