@@ -165,10 +165,10 @@ block_sparse_attention_kernel(const __grid_constant__ CUtensorMap map_q,
                 tma_load_2d(sV + kHalfTile, &map_v, bar_v_full, col + 64, row);
                 issued_v = n + 1;
             }
-            mbar_wait(bar_q, 0, abort);
+            mbar_wait_drain(bar_q, 0);           // the Q copy lands before the CTA exits
             if (failed) {
-                if (issued_k) mbar_wait(bar_k_full, (issued_k - 1) & 1, abort);
-                if (issued_v) mbar_wait(bar_v_full, (issued_v - 1) & 1, abort);
+                if (issued_k) mbar_wait_drain(bar_k_full, (issued_k - 1) & 1);
+                if (issued_v) mbar_wait_drain(bar_v_full, (issued_v - 1) & 1);
             }
         }
         __syncwarp();
@@ -230,7 +230,7 @@ block_sparse_attention_kernel(const __grid_constant__ CUtensorMap map_q,
             }
             if (failed) {
                 mma_commit(bar_drain);
-                mbar_wait(bar_drain, 0, abort);
+                mbar_wait_drain(bar_drain, 0);
             }
         }
         __syncwarp();

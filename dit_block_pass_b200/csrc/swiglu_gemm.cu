@@ -226,7 +226,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap map_x,
             if (failed) {
                 // let the copies already issued land before the CTA exits
                 for (uint32_t j = it > kStages ? it - kStages : 0; j < it; ++j)
-                    mbar_wait(bar_full + 8 * (j % kStages), (j / kStages) & 1u, abort);
+                    mbar_wait_drain(bar_full + 8 * (j % kStages), (j / kStages) & 1u);
             }
         }
         __syncwarp();
@@ -267,7 +267,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap map_x,
             if (failed) {
                 // every MMA issued has finished when this commit arrives
                 mma_commit(bar_drain);
-                mbar_wait(bar_drain, 0, abort);
+                mbar_wait_drain(bar_drain, 0);
             }
         }
         __syncwarp();
