@@ -217,6 +217,21 @@ def _set_views(B: int, N: int, D: int, set_index: torch.Tensor, *mods: torch.Ten
     return dt, strides[0], strides[1], S
 
 
+def _result_buffers(prev: torch.Tensor, B: int, rel: Optional[torch.Tensor],
+                    reuse: Optional[torch.Tensor]):
+    """The Cache-DiT outputs: caller tensors are checked before the kernel
+    writes B float64 and B uint8 values through their pointers (contiguous,
+    on prev's device, at least B elements); None allocates them."""
+    rel = torch.empty(B, dtype=torch.float64, device=prev.device) if rel is None else rel
+    reuse = torch.empty(B, dtype=torch.uint8, device=prev.device) if reuse is None else reuse
+    for nm, t, dt in (("rel", rel, torch.float64), ("reuse", reuse, torch.uint8)):
+        if not isinstance(t, torch.Tensor) or t.dtype != dt or t.device != prev.device or \
+                not t.is_contiguous() or t.numel() < B:
+            raise ValueError(f"{nm} must be a contiguous {dt} tensor of at least {B} elements "
+                             f"on {prev.device}")
+    return rel, reuse
+
+
 def _rows3(name: str, t: torch.Tensor):
     if t.dim() != 3 or not t.is_contiguous():
         raise ValueError(f"{name} must be a contiguous [B, N, D] tensor")
@@ -395,8 +410,9 @@ def _workspace(prev: torch.Tensor, workspace: Optional[torch.Tensor]) -> torch.T
     need = cachedit_workspace_bytes(B, N, D)
     if workspace is None:
         workspace = torch.empty(need, dtype=torch.uint8, device=prev.device)
-    if workspace.numel() * workspace.element_size() < need or not workspace.is_contiguous():
-        raise ValueError(f"workspace needs {need} contiguous bytes")
+    if workspace.numel() * workspace.element_size() < need or not workspace.is_contiguous() \
+            or workspace.device != prev.device:
+        raise ValueError(f"workspace needs {need} contiguous bytes on {prev.device}")
     return workspace
 
 
@@ -411,8 +427,7 @@ def cachedit_residual_diff(prev: torch.Tensor, cur: torch.Tensor, threshold: flo
     if cur.shape != prev.shape or not cur.is_contiguous():
         raise ValueError("cur must match prev")
     ws = _workspace(prev, workspace)
-    rel = torch.empty(B, dtype=torch.float64, device=prev.device) if rel is None else rel
-    reuse = torch.empty(B, dtype=torch.uint8, device=prev.device) if reuse is None else reuse
+    rel, reuse = _result_buffers(prev, B, rel, reuse)
     _call("cachedit_residual_diff", prev.data_ptr(), cur.data_ptr(), B, N, D, float(threshold),
           rel.data_ptr(), reuse.data_ptr(), ws.data_ptr(), ws.numel() * ws.element_size(),
           _stream(prev))
@@ -430,6 +445,10 @@ def cachedit_residual_sums(prev: torch.Tensor, cur: torch.Tensor,
         raise ValueError("cur must match prev")
     ws = _workspace(prev, workspace)
     sums = torch.empty(B, 2, dtype=torch.float64, device=prev.device) if sums is None else sums
+    if sums.dtype != torch.float64 or sums.device != prev.device or not sums.is_contiguous() \
+            or sums.numel() < 2 * B:
+        raise ValueError(f"sums must be a contiguous float64 tensor of at least {2 * B} "
+                         f"elements on {prev.device}")
     _call("cachedit_residual_sums", prev.data_ptr(), cur.data_ptr(), B, N, D, sums.data_ptr(),
           ws.data_ptr(), ws.numel() * ws.element_size(), _stream(prev))
     return sums
@@ -465,8 +484,7 @@ def cachedit_residual_diff_noalloc(prev: torch.Tensor, cur: torch.Tensor, thresh
     B, N, D = _rows3("prev", prev)
     if cur.shape != prev.shape or not cur.is_contiguous():
         raise ValueError("cur must match prev")
-    rel = torch.empty(B, dtype=torch.float64, device=prev.device) if rel is None else rel
-    reuse = torch.empty(B, dtype=torch.uint8, device=prev.device) if reuse is None else reuse
+    rel, reuse = _result_buffers(prev, B, rel, reuse)
     _call("cachedit_residual_diff_noalloc", prev.data_ptr(), cur.data_ptr(), B, N, D,
           float(threshold), rel.data_ptr(), reuse.data_ptr(), _stream(prev))
     return rel, reuse

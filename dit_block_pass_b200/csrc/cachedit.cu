@@ -277,9 +277,11 @@ extern "C" int cachedit_decide(const double* sums, int R, int B, double threshol
 // which every GPU that loads the library holds until the process exits.
 //
 // Host code must not pass the array's name to a kernel (on the host it is a
-// stand-in, not a device address); the device address is looked up once per
-// device with cudaGetSymbolAddress, on the first call made with that device
-// current, and cached.
+// stand-in, not a device address); the device address comes from
+// cudaGetSymbolAddress with that device current.  It is looked up again on
+// every call made outside stream capture (a cudaDeviceReset reloads the
+// module at a new address), and a call made while its stream is capturing
+// uses the address the last uncaptured call on that device found.
 namespace dit {
 namespace {
 
@@ -291,12 +293,17 @@ constexpr int kMaxDevices = 64;
 std::mutex g_scratch_mu;
 double* g_scratch_ptr[kMaxDevices] = {};
 
-// Device address of the scratch array on the current device (looked up once).
-double* scratch_address() {
+// Device address of the scratch array on the current device: looked up
+// when the stream is not capturing, else the one cached by an earlier call
+// (NULL if there was none).
+double* scratch_address(cudaStream_t stream) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+    const bool capturing =
+        cudaStreamIsCapturing(stream, &cap) != cudaSuccess || cap != cudaStreamCaptureStatusNone;
     std::lock_guard<std::mutex> lock(g_scratch_mu);
-    if (!g_scratch_ptr[dev]) {
+    if (!capturing) {
         void* p = nullptr;
         if (cudaGetSymbolAddress(&p, g_cachedit_scratch) != cudaSuccess) return nullptr;
         g_scratch_ptr[dev] = static_cast<double*>(p);
@@ -317,7 +324,7 @@ extern "C" int cachedit_residual_diff_noalloc(const uint16_t* prev, const uint16
     if (B > kStaticMaxSamples) return DIT_ERR_SHAPE;
     if (!rel_out || !reuse_out) return DIT_ERR_NULL;
     if (isnan(threshold)) return DIT_ERR_VALUE;
-    double* scratch = scratch_address();
+    double* scratch = scratch_address(as_stream(stream));
     if (!scratch) return DIT_ERR_LAUNCH;
     const int64_t nvs = N * D / 8;
     const int G = partial_slots(B, nvs, 1);

@@ -450,9 +450,11 @@ int dit_cache_policy_decide(dit_cache_policy* policy, double rel);
  * Limits: B <= 64 samples, and (partial-sum slots per sample) x B <= 4096
  * (always true for B <= 64 on current GPUs); beyond them it returns
  * DIT_ERR_SHAPE (B) or DIT_ERR_WORKSPACE (slots) and launches nothing.
- * Set-up: the first call on each device looks up the array's device address
- * (cudaGetSymbolAddress) with that device current and caches it; make that
- * first call before any stream capture on the device.
+ * Set-up: a call whose stream is not capturing looks up the array's device
+ * address (cudaGetSymbolAddress) with the current device and caches it, so
+ * the address stays right after a cudaDeviceReset; a call made while its
+ * stream is capturing uses the cached address.  Make the first call on each
+ * device before any stream capture on it (else DIT_ERR_LAUNCH).
  * Sharing: every call on a device uses the same array, which keeps the last
  * call's contents; each call writes every slot it reads before reading it,
  * so nothing needs clearing, but calls that overlap on the GPU (different

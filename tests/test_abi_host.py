@@ -285,3 +285,27 @@ def test_subblock_router_host(lib):
     assert f(A, None, 128, 1, 256, 2, 64, 128, 0.75, A + 0x2000, A + 0x3000, ws, None) == E["NULL"]
     assert f(A, A + 0x1000, 120, 1, 256, 2, 64, 128, 0.75, A + 0x2000, A + 0x3000, ws, None) == E["SHAPE"]
     assert f(A, A + 0x1000, 128, 1, 128 * 8193, 2, 64, 128, 0.75, A + 0x2000, A + 0x3000, ws, None) == E["SHAPE"]
+
+
+def test_cachedit_result_buffers_are_checked_before_the_call():
+    """rel [B] float64 and reuse [B] uint8 reach the kernel as raw pointers,
+    so the binding rejects a wrong dtype, a short or strided tensor, or one on
+    another device before any call (checked here on CPU tensors)."""
+    import torch
+    import dit_block_pass_b200 as dbp
+    prev = torch.zeros(3, 4, 8, dtype=torch.bfloat16)
+    rel, reuse = dbp._result_buffers(prev, 3, None, None)
+    assert rel.dtype == torch.float64 and reuse.dtype == torch.uint8 and rel.numel() == 3
+    ok_rel, ok_reuse = torch.zeros(3, dtype=torch.float64), torch.zeros(3, dtype=torch.uint8)
+    assert dbp._result_buffers(prev, 3, ok_rel, ok_reuse)[0] is ok_rel
+    bad = [
+        (torch.zeros(3, dtype=torch.float32), ok_reuse),           # rel float32
+        (torch.zeros(2, dtype=torch.float64), ok_reuse),           # rel too short
+        (torch.zeros(6, dtype=torch.float64)[::2], ok_reuse),      # rel strided
+        (ok_rel, torch.zeros(3, dtype=torch.int32)),               # reuse int32
+        (ok_rel, torch.zeros(2, dtype=torch.uint8)),               # reuse too short
+        (ok_rel, torch.zeros(3, dtype=torch.uint8, device="meta")),  # another device
+    ]
+    for r, u in bad:
+        with pytest.raises(ValueError):
+            dbp._result_buffers(prev, 3, r, u)

@@ -117,7 +117,7 @@ def test_fullsize_qk_rope(orc, name):
     assert np.array_equal(sel[:, 2 * D:], hb[:, 2 * D:]), "v changed"
 
 
-@pytest.mark.parametrize("name", ["h3_5s", "cfg_av"])
+@pytest.mark.parametrize("name", ["h3_5s", "h3_10s", "cfg_av"])
 def test_fullsize_cachedit(orc, name):
     wl = W.CONFIGS[name]
     B, N, D = wl.B, wl.N, wl.D
