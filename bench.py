@@ -12,9 +12,15 @@ flush is needed between steps.  Device time comes from CUDA events on the
 launching stream, bracketed by a barrier and a synchronize, max over ranks.
 
 Usage:
-  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
-Under torchrun each rank runs an independent clip (weak scaling; the ops are
-token-local, so the data path has no collective).
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference] [--shard]
+With --gpus N > 1 and no torchrun environment the script starts N ranks
+itself under torch.distributed.run (one process per GPU, NCCL).  By default
+each rank runs an independent clip (weak scaling; the ops are token-local, so
+the data path has no collective) and the line also carries `sharded_clip`:
+one clip sequence-sharded across the ranks, with the Cache-DiT all-gather
+inside the step (strong scaling).  --shard makes the sharded clip the
+headline.  The line also times the 10 s clip and the CFG pair with joint
+audio (`configs`) outside the headline's timed region.
 """
 from __future__ import annotations
 
@@ -39,13 +45,12 @@ OPS = ["adaln_modulate", "qk_rmsnorm_rope3d", "gated_residual_adaln", "swiglu",
 DOMINANT = "swiglu"
 
 # DRAM traffic from ncu (dram__bytes_read.sum + dram__bytes_write.sum of one
-# launch on the 32,256-token h3_slice, per token; a pure stream scales with
-# the token count).  Valid only while the kernel source is unchanged (hash of
-# the .cu file without comments); reported as null otherwise.
-NCU_TRAFFIC = {
-    "swiglu": {"file": "swiglu.cu", "sha": "a9e07b0f774729cf",
-               "bytes_per_token": 2620278488 / 32256},
-}
+# launch of each op's kernels on the 32,256-token h3_slice, per token; every
+# op is a stream, so traffic scales with the token count).  An entry is valid
+# only while its kernel source is unchanged (hash of the .cu file without
+# comments and blank space); it is reported as null otherwise.
+NCU_SLICE_TOKENS = 32256
+NCU_TRAFFIC = {}
 
 
 def algorithmic_bytes(wl) -> dict:
@@ -192,6 +197,63 @@ class Chain:
     def launches_per_step(self):
         import dit_block_pass_b200 as dbp
         return sum(dbp.launch_counts[o] for o in OPS)
+
+
+class ShardChain(Chain):
+    """This rank's contiguous token shard [n0, n1) of every sample of one
+    clip: the same chain on the shard, QK with the shard's global token
+    offset (or its slice of the explicit positions), and the Cache-DiT check
+    as shard sums, an all-gather of 2*B doubles and a fixed-order decide."""
+
+    def __init__(self, wl, device, rank, world):
+        import torch
+        from dit_block_pass_b200 import workloads as W
+        from dit_block_pass_b200.sharding import shard_range
+        self.wl = wl
+        self.dev = device
+        self.n0, self.n1 = shard_range(wl.N, rank, world)
+        B, N, D, F = wl.B, wl.N, wl.D, wl.F
+        n = self.n1 - self.n0
+        self.tokens = B * n
+        rows = (torch.arange(B)[:, None] * N + torch.arange(self.n0, self.n1)[None, :]).reshape(-1)
+        g = lambda s_, w: W.token_rows(wl, s_, w, device=device, row_ids=rows)
+        self.x = g(W.S_X, D).view(B, n, D)
+        self.r = g(W.S_R, D).view(B, n, D)
+        self.qkv = g(W.S_QKV, 3 * D).view(B, n, 3 * D)
+        self.swi = g(W.S_SWIGLU, 2 * F)
+        prev, cur = W.cache_pair(wl, device=device, row_ids=rows)
+        self.prev, self.cur = prev.view(B, n, D), cur.view(B, n, D)
+        self.mod = W.modulation(wl, device=device)
+        self.wq, self.wk = W.norm_weights(wl, device=device)
+        pos = W.positions(wl)
+        self.pos = None if pos is None else pos[rows].contiguous().to(device)
+        self.y1 = torch.empty_like(self.x)
+        self.xo = torch.empty_like(self.x)
+        self.y2 = torch.empty_like(self.x)
+        self.out = torch.empty(B * n, F, dtype=torch.bfloat16, device=device)
+        torch.cuda.synchronize(device)
+
+    def ops(self):
+        import dit_block_pass_b200 as dbp
+        from dit_block_pass_b200.sharding import cachedit_residual_diff_sharded
+        wl, D, m = self.wl, self.wl.D, self.mod
+        grid = None if self.pos is not None else (wl.T, wl.Hg, wl.Wg)
+        off = 0 if self.pos is not None else self.n0
+        return [
+            lambda: dbp.adaln_modulate(self.x, m[:, 0], m[:, 1], wl.eps, out=self.y1),
+            lambda: dbp.qk_rmsnorm_rope3d(self.qkv[:, :, :D], self.qkv[:, :, D:2 * D], self.wq,
+                                          self.wk, wl.H, wl.pairs, grid=grid, pos=self.pos,
+                                          pos_offset=off, theta=wl.theta, eps=wl.eps),
+            lambda: dbp.gated_residual_adaln(self.x, self.r, m[:, 2], m[:, 3], m[:, 4], wl.eps,
+                                             x_out=self.xo, y=self.y2),
+            lambda: dbp.swiglu(self.swi, out=self.out),
+            lambda: cachedit_residual_diff_sharded(self.prev, self.cur, wl.thresholds[0]),
+        ]
+
+    def launches_per_step(self):
+        import dit_block_pass_b200 as dbp
+        return sum(dbp.launch_counts[o] for o in OPS[:-1]) + \
+            dbp.launch_counts["cachedit_residual_sums"] + dbp.launch_counts["cachedit_decide"]
 
 
 def dist_setup(args):
@@ -397,6 +459,51 @@ def time_swiglu_gemm(chain, steps, warmup, world):
     if int(st.item()) != 0:
         raise RuntimeError("swiglu_gemm reported an expired pipeline wait")
     del w
+    return out
+
+
+def time_gemm_residual(chain, steps, warmup, world):
+    """The down-projection with the gated residual fused into its epilogue
+    (tcgen05): x' = bf16(x + gate * (h W^T)), h [M, F], W [D, F], on the
+    clip's tensors.  Times the fused GEMM alone, cuBLAS's bf16 GEMM alone,
+    and the two ways to reach (x', y = AdaLN(x')): fused GEMM then
+    adaln_modulate, against cuBLAS GEMM into [M, D] then
+    gated_residual_adaln.  Returns ms per launch of each."""
+    import torch
+    import dit_block_pass_b200 as dbp
+    from dit_block_pass_b200 import workloads as W
+    c, wl = chain, chain.wl
+    B, N, D, F = wl.B, wl.N, wl.D, wl.F
+    w = W.normal(wl.seed, 92, D, F, sigma=F ** -0.5, device=c.dev)
+    h = c.out.view(B, N, F)
+    branch = torch.empty(B, N, D, dtype=torch.bfloat16, device=c.dev)
+    m = c.mod
+    st = torch.zeros(1, dtype=torch.int32, device=c.dev)
+    ops = {
+        "fused_gemm": lambda: dbp.gemm_gated_residual(h, w, c.x, m[:, 2], x_out=c.xo, status=st),
+        "cublas_gemm": lambda: torch.matmul(h, w.T, out=branch),
+        "fused_chain": lambda: (dbp.gemm_gated_residual(h, w, c.x, m[:, 2], x_out=c.xo, status=st),
+                                dbp.adaln_modulate(c.xo, m[:, 3], m[:, 4], wl.eps, out=c.y2)),
+        "unfused_chain": lambda: (torch.matmul(h, w.T, out=branch),
+                                  dbp.gated_residual_adaln(c.x, branch, m[:, 2], m[:, 3], m[:, 4],
+                                                           wl.eps, x_out=c.xo, y=c.y2)),
+    }
+    stream = torch.cuda.current_stream()
+    out = {}
+    for name, op in ops.items():
+        for _ in range(warmup):
+            op()
+        barrier_sync(world)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(steps):
+            op()
+        b.record(stream)
+        barrier_sync(world)
+        out[name] = max_over_ranks(a.elapsed_time(b) / steps, world)
+    if int(st.item()) != 0:
+        raise RuntimeError("gemm_gated_residual reported an expired pipeline wait")
+    del w, branch
     return out
 
 
@@ -611,14 +718,24 @@ def run_reference(args, wl):
     """The reference arm: the fp64 oracle as it stands, on the host cores."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
-    if world > 1 and rank != 0:
-        return
+    if world > 1:
+        # count the ranks that started (gloo on the host), then only rank 0 works
+        import datetime
+        import torch
+        import torch.distributed as dist
+        dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=60))
+        t = torch.ones(1)
+        dist.all_reduce(t)
+        world = int(t.item())
+        dist.destroy_process_group()
+        if rank != 0:
+            return
     rate, pool, passes, threads = oracle_chain_rate(
         wl, budget_s=args.ref_budget, threads=host_threads(), steps=max(1, args.steps))
     per_step = pool * passes
     line = {
         "impl": "reference", "metric": METRIC, "value": rate, "unit": "tokens/s",
-        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1000.0 * per_step / rate, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": wl.describe(), "tokens_per_step_sampled": per_step},
@@ -632,6 +749,170 @@ def run_reference(args, wl):
     print(json.dumps(line), flush=True)
 
 
+def op_report(nbytes: dict, per_op, tokens: int, peak: float, traffic: dict) -> dict:
+    """Per-op ms, GB/s, fraction of the HBM peak and tokens/s; with the ncu
+    traffic of a full launch (and its ratio to the algorithmic bytes) where
+    a capture of the current kernel source exists."""
+    ops = {}
+    for name, ms in zip(OPS, per_op):
+        gbs = nbytes[name] / (ms / 1000.0) / 1e9
+        ops[name] = {"ms": round(ms, 4), "GB/s": round(gbs, 1),
+                     "frac_of_peak": round(gbs / peak, 4),
+                     "tokens_per_s": round(tokens / (ms / 1000.0), 1),
+                     "algorithmic_bytes": nbytes[name]}
+        t = traffic.get(name)
+        ops[name]["traffic"] = t
+        ops[name]["traffic_over_algorithmic"] = (round(t / nbytes[name], 4) if t else None)
+    return ops
+
+
+def ncu_traffic(tokens: int) -> dict:
+    """DRAM bytes of one full launch of each op, from the slice captures
+    whose kernel source still matches; absent entries are null."""
+    out = {}
+    for name, tr in NCU_TRAFFIC.items():
+        if tr["sha"] == source_sha(tr["file"]):
+            out[name] = round(tr["bytes_per_token"] * tokens)
+    return out
+
+
+def time_config(name: str, dev, steps: int, warmup: int, world: int, peak: float) -> dict:
+    """Per-op and chain timings of another workload (one clip per rank),
+    with its own buffers, outside the headline's timed region."""
+    import torch
+    from dit_block_pass_b200 import workloads as W
+    wl = W.CONFIGS[name]
+    chain = Chain(wl, dev)
+    total_ms, per_op = time_device(chain, steps, warmup, world)
+    per_op = [max_over_ranks(ms, world) for ms in per_op]
+    total_ms = max_over_ranks(total_ms, world)
+    nbytes = algorithmic_bytes(wl)
+    ms_step = total_ms / steps
+    chain_bytes = sum(nbytes[o] for o in OPS)
+    res = {"workload": wl.describe(), "steps": steps, "warmup": warmup,
+           "ms_per_step": round(ms_step, 4),
+           "tokens_per_s": round(world * wl.M / (ms_step / 1000.0), 1),
+           "chain_GB/s": round(chain_bytes / (ms_step / 1000.0) / 1e9, 1),
+           "chain_frac_of_peak": round(chain_bytes / (ms_step / 1000.0) / 1e9 / peak, 4),
+           "ops": op_report(nbytes, per_op, wl.M, peak, ncu_traffic(wl.M))}
+    del chain
+    torch.cuda.synchronize(dev)
+    torch.cuda.empty_cache()
+    return res
+
+
+def time_sharded_clip(wl, dev, steps: int, warmup: int, world: int, rank: int) -> dict:
+    """One clip sequence-sharded across the ranks: per step every rank runs
+    the chain on its token shard and the Cache-DiT check with its all-gather.
+    Returns the max-over-ranks ms per step and the clip's tokens/s."""
+    import torch
+    chain = ShardChain(wl, dev, rank, world)
+    total_ms, per_op = time_device(chain, steps, warmup, world)
+    total_ms = max_over_ranks(total_ms, world)
+    per_op = [max_over_ranks(ms, world) for ms in per_op]
+    ms_step = total_ms / steps
+    res = {"workload": wl.describe(), "ranks": world, "scaling": "strong",
+           "tokens_per_rank": f"{chain.n1 - chain.n0} (rank {rank}); clip {wl.N}",
+           "ms_per_step": round(ms_step, 4),
+           "tokens_per_s": round(wl.M / (ms_step / 1000.0), 1),
+           "ms_per_op (max over ranks)": {o: round(ms, 4) for o, ms in zip(OPS, per_op)},
+           "collective": "all_gather of 2*B float64 per rank (Cache-DiT sums), fixed-order "
+                         "decide on every rank",
+           "gpu_launches": chain.launches_per_step() * steps}
+    del chain
+    torch.cuda.synchronize(dev)
+    torch.cuda.empty_cache()
+    return res
+
+
+def extra_report(ex: dict, wl, nbytes: dict, peak: float, world: int) -> dict:
+    """JSON objects of the rows timed beside the chain (QK options, per-token
+    sets, step cache, fused GEMMs, router, block-sparse attention)."""
+    out = {}
+    qk_options = {}
+    for name, ms in ex["qk"].items():
+        ms = max_over_ranks(ms, world)
+        gbs = nbytes["qk_rmsnorm_rope3d"] / (ms / 1000.0) / 1e9
+        qk_options[name] = {"ms": round(ms, 4), "GB/s": round(gbs, 1),
+                            "frac_of_peak": round(gbs / peak, 4)}
+    out["qk_options"] = qk_options
+    tok_sets, tok_share = ex["tok"]
+    token_sets = {"tokens_on_set_1": round(tok_share, 4)}
+    for name, ms in tok_sets.items():
+        ms = max_over_ranks(ms, world)
+        gbs = nbytes[name] / (ms / 1000.0) / 1e9
+        token_sets[name] = {"ms": round(ms, 4), "GB/s": round(gbs, 1),
+                            "frac_of_peak": round(gbs / peak, 4)}
+    out["token_sets"] = token_sets
+    cache_step = {}
+    for name, ms in ex["cache"].items():
+        ms = max_over_ranks(ms, world)
+        gbs = 6 * wl.M * wl.D / (ms / 1000.0) / 1e9        # read two, write one
+        cache_step[name] = {"ms": round(ms, 4), "GB/s": round(gbs, 1),
+                            "frac_of_peak": round(gbs / peak, 4)}
+    out["cache_step"] = cache_step
+    burst, sustained, tkind = tensor_peaks()
+    gemm_ms = ex["gemm"]
+    gflop = 2.0 * wl.M * wl.D * 2 * wl.F / 1e9
+    fused_ms = max_over_ranks(gemm_ms["fused"], world)
+    unfused_ms = max_over_ranks(gemm_ms["unfused"], world)
+    tflops = gflop / fused_ms
+    out["swiglu_gemm"] = {
+        "kernel": "gemm_kernel<kSwiGLU> (tcgen05)", "ms": round(fused_ms, 3),
+        "TFLOP/s": round(tflops, 1), "bound": "tensor",
+        "frac_of_burst_peak": round(tflops / burst, 4),
+        "frac_of_sustained_peak": round(tflops / sustained, 4),
+        "peak_source": f"{tkind} bf16_tflops {burst} / sustained {sustained}",
+        "unfused_ms (cuBLAS bf16 GEMM + swiglu_kernel)": round(unfused_ms, 3),
+        "speedup_vs_unfused": round(unfused_ms / fused_ms, 4),
+        "shape": f"[{wl.M}, {wl.D}] x [{2 * wl.F}, {wl.D}]^T -> [{wl.M}, {wl.F}]"}
+    g = ex["gres"]
+    gflop_d = 2.0 * wl.M * wl.F * wl.D / 1e9
+    tfl = gflop_d / g["fused_gemm"]
+    out["gemm_gated_residual"] = {
+        "kernel": "gemm_kernel<kGatedResidual> (tcgen05)", "ms": round(g["fused_gemm"], 3),
+        "TFLOP/s": round(tfl, 1), "bound": "tensor",
+        "frac_of_burst_peak": round(tfl / burst, 4),
+        "frac_of_sustained_peak": round(tfl / sustained, 4),
+        "cublas_gemm_ms (bf16 GEMM into [M, D] alone)": round(g["cublas_gemm"], 3),
+        "fused_chain_ms (fused GEMM + adaln_modulate)": round(g["fused_chain"], 3),
+        "unfused_chain_ms (cuBLAS GEMM + gated_residual_adaln)": round(g["unfused_chain"], 3),
+        "speedup_vs_unfused": round(g["unfused_chain"] / g["fused_chain"], 4),
+        "shape": f"[{wl.M}, {wl.F}] x [{wl.D}, {wl.F}]^T + gated residual -> [{wl.M}, {wl.D}]"}
+    router_ms, router_nb, router_keep = ex["router"]
+    router_ms = max_over_ranks(router_ms, world)
+    router_gbs = 4.0 * wl.M * wl.D / (router_ms / 1000.0) / 1e9        # read q and k once
+    out["subblock_router"] = {
+        "ms": round(router_ms, 4), "GB/s": round(router_gbs, 1),
+        "frac_of_peak": round(router_gbs / peak, 4), "block": 128, "sparsity": 0.75,
+        "key_blocks": router_nb, "kept_per_query_block": router_keep}
+    attn_ms, dense_ms, attn_keep, attn_nb = ex["attn"]
+    attn_ms = max_over_ranks(attn_ms, world)
+    dense_ms = max_over_ranks(dense_ms, world)
+    attn_tflop = 4.0 * 128 ** 3 * attn_nb * attn_keep * wl.H * wl.B / 1e12
+    out["sparse_attention"] = {
+        "kernel": "block_sparse_attention_kernel (tcgen05)", "ms": round(attn_ms, 3),
+        "TFLOP/s": round(attn_tflop / (attn_ms / 1000.0), 1), "bound": "tensor",
+        "frac_of_burst_peak": round(attn_tflop / (attn_ms / 1000.0) / burst, 4),
+        "sparsity": 0.75, "kept_blocks": attn_keep, "key_blocks": attn_nb,
+        "dense_library_ms (torch scaled_dot_product_attention)": round(dense_ms, 3),
+        "speedup_vs_dense": round(dense_ms / attn_ms, 3)}
+    return out
+
+
+def relaunch_under_torchrun(n: int) -> int:
+    """Start n ranks of this script under torch.distributed.run (one per GPU,
+    rendezvous on 127.0.0.1) and return its exit code."""
+    import socket
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1",
+           f"--nproc-per-node={n}", "--master-addr", "127.0.0.1", "--master-port", str(port),
+           os.path.abspath(__file__), *sys.argv[1:]]
+    return subprocess.call(cmd)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -639,11 +920,18 @@ def main():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--config", default="h3_5s")
+    ap.add_argument("--shard", action="store_true",
+                    help="headline = one clip sequence-sharded across the ranks")
+    ap.add_argument("--configs", default="h3_10s,cfg_av",
+                    help="other workloads timed after the headline (comma list, or none)")
+    ap.add_argument("--config-steps", type=int, default=40)
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--attn-steps", type=int, default=3,
                     help="timed launches of the block-sparse attention and of dense attention")
     ap.add_argument("--gemm-steps", type=int, default=10,
-                    help="timed launches of the fused up-projection and of its unfused chain")
+                    help="timed launches of the fused GEMMs and of their unfused chains")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="time the chain only (no option, GEMM, router or attention rows)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
@@ -652,6 +940,14 @@ def main():
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "native" and args.steps > 20:
         raise SystemExit("use at least 3 warm-up steps for a timed run")
+    if args.gpus < 1:
+        raise SystemExit("--gpus must be at least 1")
+    world_env = os.environ.get("WORLD_SIZE")
+    if world_env is None and args.gpus > 1:
+        # one process per GPU: start the ranks rather than run one GPU silently
+        raise SystemExit(relaunch_under_torchrun(args.gpus))
+    if world_env is not None and int(world_env) != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world_env}: they must agree")
 
     from dit_block_pass_b200 import workloads as W
     wl = W.CONFIGS[args.config]
@@ -665,98 +961,66 @@ def main():
     build.build()
     world, rank, local = dist_setup(args)
     dev = torch.device(f"cuda:{local}")
-    chain = Chain(wl, dev)
+    peak, peak_kind = hbm_peak()
+    nbytes = algorithmic_bytes(wl)
+    extras = {}
 
     sampler = ClockSampler(local) if not args.no_clocks else None
     if sampler:
         sampler.__enter__()
     try:
+        if args.shard:
+            chain = ShardChain(wl, dev, rank, world)
+        else:
+            chain = Chain(wl, dev)
         total_ms, per_op = time_device(chain, args.steps, args.warmup, world)
-        qk_opt = time_qk_options(chain, args.steps, args.warmup, world)
-        tok_sets, tok_share = time_token_sets(chain, args.steps, args.warmup, world)
-        step_cache = time_cache_step(chain, args.steps, args.warmup, world)
-        gemm_ms = time_swiglu_gemm(chain, args.gemm_steps, 2, world)
-        router_ms, router_nb, router_keep = time_subblock_router(chain, args.steps, args.warmup,
-                                                                 world)
-        attn_ms, dense_ms, attn_keep, attn_nb = time_sparse_attention(chain, args.attn_steps,
-                                                                      world)
+        launches = chain.launches_per_step() * args.steps
+        tokens = chain.tokens if args.shard else wl.M
+        if not args.no_extras and not args.shard:
+            extras["qk"] = time_qk_options(chain, args.steps, args.warmup, world)
+            extras["tok"] = time_token_sets(chain, args.steps, args.warmup, world)
+            extras["cache"] = time_cache_step(chain, args.steps, args.warmup, world)
+            extras["gemm"] = time_swiglu_gemm(chain, args.gemm_steps, 2, world)
+            extras["gres"] = time_gemm_residual(chain, args.gemm_steps, 2, world)
+            extras["router"] = time_subblock_router(chain, args.steps, args.warmup, world)
+            extras["attn"] = time_sparse_attention(chain, args.attn_steps, world)
+        e2e = None
+        if not args.no_e2e and not args.shard:
+            ms_e2e, h2d, d2h = time_e2e(chain, args.e2e_steps, 1, world)
+            e2e = {"value": world * tokens / (ms_e2e / 1000.0), "unit": "tokens/s",
+                   "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                   "ms_per_step": round(ms_e2e, 3)}
+        del chain
+        torch.cuda.synchronize(dev)
+        torch.cuda.empty_cache()
+        configs = {}
+        if not args.shard:
+            for name in [c for c in args.configs.split(",") if c and c != "none"]:
+                configs[name] = time_config(name, dev, args.config_steps, 3, world, peak)
+        sharded = None
+        if world > 1 and not args.shard:
+            sharded = time_sharded_clip(wl, dev, args.config_steps, 3, world, rank)
     finally:
         if sampler:
             sampler.__exit__(None, None, None)
     total_ms = max_over_ranks(total_ms, world)
+    per_op = [max_over_ranks(ms, world) for ms in per_op]
     ms_step = total_ms / args.steps
-    tokens = wl.M
-    value = world * tokens * args.steps / (total_ms / 1000.0)
+    if args.shard:
+        value = wl.M * args.steps / (total_ms / 1000.0)      # one clip over all ranks
+    else:
+        value = world * wl.M * args.steps / (total_ms / 1000.0)
 
-    peak, peak_kind = hbm_peak()
-    nbytes = algorithmic_bytes(wl)
-    ops = {}
-    for name, ms in zip(OPS, per_op):
-        gbs = nbytes[name] / (ms / 1000.0) / 1e9
-        ops[name] = {"ms": round(ms, 4), "GB/s": round(gbs, 1),
-                     "frac_of_peak": round(gbs / peak, 4),
-                     "tokens_per_s": round(tokens / (ms / 1000.0), 1)}
-    qk_options = {}
-    for name, ms in qk_opt.items():
-        ms = max_over_ranks(ms, world)
-        gbs = nbytes["qk_rmsnorm_rope3d"] / (ms / 1000.0) / 1e9
-        qk_options[name] = {"ms": round(ms, 4), "GB/s": round(gbs, 1),
-                            "frac_of_peak": round(gbs / peak, 4)}
-    token_sets = {"tokens_on_set_1": round(tok_share, 4)}
-    for name, ms in tok_sets.items():
-        ms = max_over_ranks(ms, world)
-        gbs = nbytes[name] / (ms / 1000.0) / 1e9
-        token_sets[name] = {"ms": round(ms, 4), "GB/s": round(gbs, 1),
-                            "frac_of_peak": round(gbs / peak, 4)}
-    cache_step = {}
-    for name, ms in step_cache.items():
-        ms = max_over_ranks(ms, world)
-        gbs = 6 * wl.M * wl.D / (ms / 1000.0) / 1e9        # read two, write one
-        cache_step[name] = {"ms": round(ms, 4), "GB/s": round(gbs, 1),
-                            "frac_of_peak": round(gbs / peak, 4)}
-    burst, sustained, tkind = tensor_peaks()
-    gflop = 2.0 * wl.M * wl.D * 2 * wl.F / 1e9
-    fused_ms = max_over_ranks(gemm_ms["fused"], world)
-    unfused_ms = max_over_ranks(gemm_ms["unfused"], world)
-    tflops = gflop / fused_ms
-    swiglu_gemm = {"kernel": "swiglu_gemm_kernel (tcgen05)", "ms": round(fused_ms, 3),
-                   "TFLOP/s": round(tflops, 1), "bound": "tensor",
-                   "frac_of_burst_peak": round(tflops / burst, 4),
-                   "frac_of_sustained_peak": round(tflops / sustained, 4),
-                   "peak_source": f"{tkind} bf16_tflops {burst} / sustained {sustained}",
-                   "unfused_ms (cuBLAS bf16 GEMM + swiglu_kernel)": round(unfused_ms, 3),
-                   "speedup_vs_unfused": round(unfused_ms / fused_ms, 4),
-                   "shape": f"[{wl.M}, {wl.D}] x [{2 * wl.F}, {wl.D}]^T -> [{wl.M}, {wl.F}]"}
-    router_ms = max_over_ranks(router_ms, world)
-    router_gbs = 4.0 * wl.M * wl.D / (router_ms / 1000.0) / 1e9        # read q and k once
-    subblock = {"ms": round(router_ms, 4), "GB/s": round(router_gbs, 1),
-                "frac_of_peak": round(router_gbs / peak, 4), "block": 128, "sparsity": 0.75,
-                "key_blocks": router_nb, "kept_per_query_block": router_keep}
-    attn_ms = max_over_ranks(attn_ms, world)
-    dense_ms = max_over_ranks(dense_ms, world)
-    attn_tflop = 4.0 * 128 ** 3 * attn_nb * attn_keep * wl.H * wl.B / 1e12
-    sparse_attention = {"kernel": "block_sparse_attention_kernel (tcgen05)", "ms": round(attn_ms, 3),
-                        "TFLOP/s": round(attn_tflop / (attn_ms / 1000.0), 1), "bound": "tensor",
-                        "frac_of_burst_peak": round(attn_tflop / (attn_ms / 1000.0) / burst, 4),
-                        "sparsity": 0.75, "kept_blocks": attn_keep, "key_blocks": attn_nb,
-                        "dense_library_ms (torch scaled_dot_product_attention)": round(dense_ms, 3),
-                        "speedup_vs_dense": round(dense_ms / attn_ms, 3)}
+    ops = op_report(nbytes, per_op, tokens, peak, ncu_traffic(tokens))
+    line_extras = {}
+    if extras:
+        line_extras = extra_report(extras, wl, nbytes, peak, world)
     dom_ms = per_op[OPS.index(DOMINANT)]
-    achieved = nbytes[DOMINANT] / (dom_ms / 1000.0) / 1e9
-    tr = NCU_TRAFFIC.get(DOMINANT)
-    traffic = (round(tr["bytes_per_token"] * tokens)
-               if tr and tr["sha"] == source_sha(tr["file"]) else None)
+    achieved = ops[DOMINANT]["algorithmic_bytes"] / (dom_ms / 1000.0) / 1e9
     roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
-                "frac": round(achieved / peak, 4), "traffic": traffic,
+                "frac": round(achieved / peak, 4), "traffic": ops[DOMINANT]["traffic"],
                 "kernel": "swiglu_kernel", "peak_source": f"{peak_kind} hbm_gbs (copy)",
-                "algorithmic_bytes": nbytes[DOMINANT]}
-
-    e2e = None
-    if not args.no_e2e:
-        ms_e2e, h2d, d2h = time_e2e(chain, args.e2e_steps, 1, world)
-        e2e = {"value": world * tokens / (ms_e2e / 1000.0), "unit": "tokens/s",
-               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-               "ms_per_step": round(ms_e2e, 3)}
+                "algorithmic_bytes": ops[DOMINANT]["algorithmic_bytes"]}
 
     cpu = None
     if world == 1 and not args.no_cpu and rank == 0:
@@ -765,25 +1029,36 @@ def main():
                "sample": f"{pool} random token rows of the clip, {passes} pass(es) over them "
                          f"(about {args.cpu_budget:.0f} s), whole chain per row, rows split "
                          f"over {threads} host threads"}
+        single = {}
+        for name, budget in (("tiny", 2.0), ("small", 5.0)):
+            r1, p1, n1, _ = oracle_chain_rate(W.CONFIGS[name], budget, 1)
+            single[name] = {"value": r1, "unit": "tokens/s", "cores": 1,
+                            "sample": f"{p1} token rows, {n1} pass(es), whole chain per row"}
+        cpu["single_thread"] = single
 
     clocks = sampler.summary() if sampler else None
     if rank == 0:
+        if args.shard:
+            par = f"one clip sequence-sharded over {world} rank(s) (token shards, " \
+                  f"Cache-DiT all-gather)"
+        else:
+            par = f"{world} independent clip(s), one per GPU"
         line = {
             "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "higher_is_better": True, "scaling": "strong" if args.shard else "weak",
+            "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded counter-based generator, H3-shaped)",
             "config": {"workload": wl.describe(),
                        "chain": "adaln_modulate -> qk_rmsnorm_rope3d -> gated_residual_adaln "
                                 "-> swiglu, + cachedit_residual_diff",
                        "tokens_per_step_per_gpu": tokens,
                        "l2": "every input is larger than L2 (126 MB); no flush",
-                       "parallelism": f"{world} independent clip(s), one per GPU"},
-            "ops": ops, "qk_options": qk_options, "token_sets": token_sets,
-            "cache_step": cache_step, "swiglu_gemm": swiglu_gemm, "subblock_router": subblock,
-            "sparse_attention": sparse_attention,
+                       "parallelism": par},
+            "ops": ops, **line_extras, "configs": configs or None,
+            "sharded_clip": sharded,
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
-            "gpu_launches": chain.launches_per_step() * args.steps, "clocks": clocks,
+            "gpu_launches": launches, "clocks": clocks,
         }
         print(json.dumps(line), flush=True)
     if world > 1:

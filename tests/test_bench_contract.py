@@ -40,7 +40,21 @@ def test_reference_arm_prints_the_contract_line():
     assert e2e["h2d_bytes_per_step"] == 0 and e2e["d2h_bytes_per_step"] == 0
 
 
-def test_reference_arm_is_silent_on_other_ranks():
-    res = _run({"WORLD_SIZE": "2", "RANK": "1", "LOCAL_RANK": "1"}, args=("--gpus", "2"))
+def test_gpus_n_starts_n_ranks_and_only_rank_0_prints():
+    """--gpus 2 with no torchrun environment starts two ranks itself (never one
+    process silently); the ranks count themselves over gloo, so n_gpus is the
+    number that ran, and only rank 0 prints a line."""
+    env = {k: v for k, v in os.environ.items()
+           if k not in ("WORLD_SIZE", "RANK", "LOCAL_RANK", "MASTER_ADDR", "MASTER_PORT")}
+    cmd = [sys.executable, "bench.py", "--impl", "reference", "--steps", "1", "--warmup", "3",
+           "--ref-budget", "1", "--gpus", "2"]
+    res = subprocess.run(cmd, cwd=ROOT, env=env, capture_output=True, text=True, timeout=300)
     assert res.returncode == 0, res.stderr[-2000:]
-    assert not [ln for ln in res.stdout.splitlines() if ln.startswith("{")]
+    lines = [ln for ln in res.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1, res.stdout
+    assert json.loads(lines[0])["n_gpus"] == 2
+
+
+def test_gpus_must_agree_with_the_launcher():
+    res = _run({"WORLD_SIZE": "2", "RANK": "1", "LOCAL_RANK": "1"}, args=("--gpus", "4"))
+    assert res.returncode != 0
