@@ -509,8 +509,11 @@ def time_gemm_residual(chain, steps, warmup, world):
 
 def time_subblock_router(chain, steps, warmup, world):
     """The SubBlock router on the clip's q and k (blocks of 128 tokens,
-    sparsity 0.75): ms per call (two launches: block means, then scores and
-    selection)."""
+    sparsity 0.75), two ways: the router reading q and k (block means, then
+    scores and selection), and the QK operator writing the block means as it
+    rotates q and k, then the router from those means.  Returns ms per call
+    of: the router alone, the QK operator alone, the QK operator with means,
+    and the router from means; plus the block counts."""
     import torch
     import dit_block_pass_b200 as dbp
     c, wl = chain, chain.wl
@@ -521,18 +524,32 @@ def time_subblock_router(chain, steps, warmup, world):
     ws = torch.empty(int(dbp.library().dit_subblock_workspace_bytes(wl.B, wl.N, wl.H, wl.hd, 128)),
                      dtype=torch.uint8, device=c.dev)
     kept = torch.empty(wl.B, wl.H, nb, n_keep, dtype=torch.int32, device=c.dev)
-    op = lambda: dbp.subblock_router(q, k, wl.H, 128, 0.75, workspace=ws, kept=kept)
-    for _ in range(warmup):
-        op()
-    barrier_sync(world)
+    means = torch.empty(wl.B, 2, nb, D, dtype=torch.float32, device=c.dev)
+    grid = None if c.pos is not None else (wl.T, wl.Hg, wl.Wg)
+    qk = lambda **kw: dbp.qk_rmsnorm_rope3d(q, k, c.wq, c.wk, wl.H, wl.pairs, grid=grid,
+                                            pos=c.pos, theta=wl.theta, eps=wl.eps, **kw)
+    ops = {
+        "router": lambda: dbp.subblock_router(q, k, wl.H, 128, 0.75, workspace=ws, kept=kept),
+        "qk": lambda: qk(),
+        "qk_pooled": lambda: qk(block_means=means, block=128),
+        "router_means": lambda: dbp.subblock_router_means(means, wl.N, wl.H, 128, 0.75,
+                                                          workspace=ws, kept=kept),
+    }
     stream = torch.cuda.current_stream()
-    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    a.record(stream)
-    for _ in range(steps):
-        op()
-    b.record(stream)
-    barrier_sync(world)
-    return a.elapsed_time(b) / steps, nb, n_keep
+    out = {}
+    for name, op in ops.items():
+        for _ in range(warmup):
+            op()
+        barrier_sync(world)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(steps):
+            op()
+        b.record(stream)
+        barrier_sync(world)
+        out[name] = max_over_ranks(a.elapsed_time(b) / steps, world)
+    del ws, kept, means
+    return out, nb, n_keep
 
 
 def time_sparse_attention(chain, steps, world):
@@ -879,13 +896,21 @@ def extra_report(ex: dict, wl, nbytes: dict, peak: float, world: int) -> dict:
         "unfused_chain_ms (cuBLAS GEMM + gated_residual_adaln)": round(g["unfused_chain"], 3),
         "speedup_vs_unfused": round(g["unfused_chain"] / g["fused_chain"], 4),
         "shape": f"[{wl.M}, {wl.F}] x [{wl.D}, {wl.F}]^T + gated residual -> [{wl.M}, {wl.D}]"}
-    router_ms, router_nb, router_keep = ex["router"]
-    router_ms = max_over_ranks(router_ms, world)
-    router_gbs = 4.0 * wl.M * wl.D / (router_ms / 1000.0) / 1e9        # read q and k once
+    rt, router_nb, router_keep = ex["router"]
+    router_gbs = 4.0 * wl.M * wl.D / (rt["router"] / 1000.0) / 1e9        # read q and k once
+    qk_gbs = nbytes["qk_rmsnorm_rope3d"] / (rt["qk_pooled"] / 1000.0) / 1e9
+    unfused = rt["qk"] + rt["router"]
+    fused = rt["qk_pooled"] + rt["router_means"]
     out["subblock_router"] = {
-        "ms": round(router_ms, 4), "GB/s": round(router_gbs, 1),
+        "ms": round(rt["router"], 4), "GB/s": round(router_gbs, 1),
         "frac_of_peak": round(router_gbs / peak, 4), "block": 128, "sparsity": 0.75,
-        "key_blocks": router_nb, "kept_per_query_block": router_keep}
+        "key_blocks": router_nb, "kept_per_query_block": router_keep,
+        "qk_with_block_means_ms": round(rt["qk_pooled"], 4),
+        "qk_with_block_means_frac_of_peak (q, k bytes only)": round(qk_gbs / peak, 4),
+        "router_from_means_ms": round(rt["router_means"], 4),
+        "qk_then_router_ms": round(unfused, 4),
+        "qk_with_means_then_router_ms": round(fused, 4),
+        "saved_ms": round(unfused - fused, 4)}
     attn_ms, dense_ms, attn_keep, attn_nb = ex["attn"]
     attn_ms = max_over_ranks(attn_ms, world)
     dense_ms = max_over_ranks(dense_ms, world)

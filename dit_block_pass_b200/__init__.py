@@ -26,7 +26,8 @@ __all__ = [
     "qk_rmsnorm_rope3d", "cachedit_workspace_bytes", "cachedit_residual_diff",
     "cachedit_residual_sums", "cachedit_decide", "cachedit_residual_diff_noalloc",
     "launch_counts", "QKOut", "CachePolicy", "swiglu_gemm", "gemm_gated_residual",
-    "subblock_keep_count", "subblock_router", "block_sparse_attention", "cachedit_residual_store",
+    "subblock_keep_count", "subblock_router", "subblock_router_means", "block_sparse_attention",
+    "cachedit_residual_store",
     "cachedit_residual_apply", "F32", "BF16", "ROPE_INTERLEAVED", "ROPE_HALF", "NORM_HEAD", "NORM_ROW",
 ]
 
@@ -46,7 +47,8 @@ launch_counts = {
     "cachedit_residual_diff": 2, "cachedit_residual_sums": 2, "cachedit_decide": 1,
     "cachedit_residual_diff_noalloc": 2, "cachedit_residual_store": 1,
     "cachedit_residual_apply": 1, "swiglu_gemm": 1, "gemm_gated_residual": 1,
-    "subblock_router": 3, "block_sparse_attention": 1,
+    "subblock_router": 3, "block_sparse_attention": 1, "qk_rmsnorm_rope3d_pooled": 1,
+    "subblock_router_means": 2,
 }
 
 
@@ -104,6 +106,13 @@ def library() -> ctypes.CDLL:
                                                    i32, i32, i32, i32, vp, i64, i32, i32, i32,
                                                    dbl, dbl, i32, i32,
                                                    ctypes.POINTER(QKOut), vp]
+            L.dit_qk_rmsnorm_rope3d_pooled.argtypes = [vp, vp, i64, vp, vp, i32, i32, i64, i32,
+                                                       i32, i32, i32, i32, vp, i64, i32, i32,
+                                                       i32, dbl, dbl, i32, i32, vp, vp]
+            L.dit_subblock_means_workspace_bytes.argtypes = [i32, i64, i32, i32]
+            L.dit_subblock_means_workspace_bytes.restype = sz
+            L.dit_subblock_router_means.argtypes = [vp, i32, i64, i32, i32, i32, dbl, vp, vp, sz,
+                                                    vp]
             L.dit_swiglu_gemm.argtypes = [vp, vp, vp, i64, i32, i32, vp, vp]
             L.dit_block_sparse_attention.argtypes = [vp, vp, vp, i64, vp, i64, i32, i64, i32,
                                                      i32, i32, vp, i32, dbl, vp, vp]
@@ -134,6 +143,7 @@ def library() -> ctypes.CDLL:
                          "dit_subblock_router", "dit_block_sparse_attention",
                          "dit_cache_policy_init", "dit_cache_policy_decide",
                          "dit_qk_rmsnorm_rope3d", "dit_qk_rmsnorm_rope3d_ex",
+                         "dit_qk_rmsnorm_rope3d_pooled", "dit_subblock_router_means",
                          "cachedit_residual_diff",
                          "cachedit_residual_sums", "cachedit_decide"):
                 getattr(L, name).restype = i32
@@ -332,7 +342,8 @@ def qk_rmsnorm_rope3d(q: Optional[torch.Tensor], k: Optional[torch.Tensor],
                       theta: float = 10000.0, eps: float = 1e-6,
                       rope_layout: int = ROPE_INTERLEAVED, norm_width: int = NORM_HEAD,
                       q_out: Optional[torch.Tensor] = None,
-                      k_out: Optional[torch.Tensor] = None) -> None:
+                      k_out: Optional[torch.Tensor] = None,
+                      block_means: Optional[torch.Tensor] = None, block: int = 128) -> None:
     """In place on q and k ([B, N, H*hd] views, e.g. slices of a fused qkv
     buffer): RMSNorm with weight w, then 3D RoPE with pair split
     ``pairs`` = (t, h, w).  Positions come from ``grid`` = (T, Hg, Wg) (token
@@ -342,7 +353,11 @@ def qk_rmsnorm_rope3d(q: Optional[torch.Tensor], k: Optional[torch.Tensor],
     pairs (2p, 2p+1), ROPE_HALF pairs (p, p + hd/2).  With ``q_out``/``k_out``
     ([B, N, H, hd] views with any strides and a contiguous last dimension,
     e.g. ``torch.empty(B, H, N, hd).transpose(1, 2)`` for the head-major
-    layout attention reads) q and k are only read and the results go there."""
+    layout attention reads) q and k are only read and the results go there.
+    With ``block_means`` (fp32 [B, 2, ceil(N/block), H*hd], contiguous) the
+    call is in place with the per-head norm and also writes the mean of each
+    block of ``block`` tokens of the rotated q ([:, 0]) and k ([:, 1]), the
+    input of ``subblock_router_means``."""
     ref = q if q is not None else k
     if ref is None:
         raise ValueError("q and k cannot both be None")
@@ -377,6 +392,20 @@ def qk_rmsnorm_rope3d(q: Optional[torch.Tensor], k: Optional[torch.Tensor],
             raise ValueError("give grid=(T, Hg, Wg) or pos")
         T, Hg, Wg = grid
     pt, ph, pw = pairs
+    if block_means is not None:
+        nb = (N + block - 1) // block
+        if q is None or k is None or q_out is not None or k_out is not None or \
+                norm_width != NORM_HEAD:
+            raise ValueError("block_means needs q and k, in place, with the per-head norm")
+        if block_means.dtype != torch.float32 or not block_means.is_contiguous() or \
+                block_means.device != ref.device or \
+                tuple(block_means.shape) != (B, 2, nb, width):
+            raise ValueError(f"block_means must be a contiguous float32 [{B}, 2, {nb}, {width}] "
+                             f"tensor on {ref.device}")
+        _call("dit_qk_rmsnorm_rope3d_pooled", _ptr(q), _ptr(k), rs, _ptr(w_q), _ptr(w_k), w_dt,
+              B, N, heads, hd, T, Hg, Wg, _ptr(pos), int(pos_offset), pt, ph, pw, float(theta),
+              float(eps), int(rope_layout), int(block), block_means.data_ptr(), _stream(ref))
+        return
     out = None
     if q_out is not None or k_out is not None:
         strides = None
@@ -657,6 +686,41 @@ def subblock_router(q: torch.Tensor, k: torch.Tensor, heads: int, block: int = 1
     _call("dit_subblock_router", q.data_ptr(), k.data_ptr(), rs, B, N, heads, hd, block,
           float(sparsity), kept.data_ptr(), workspace.data_ptr(),
           workspace.numel() * workspace.element_size(), _stream(q))
+    return kept
+
+
+def subblock_router_means(block_means: torch.Tensor, N: int, heads: int, block: int = 128,
+                          sparsity: float = 0.75, workspace: Optional[torch.Tensor] = None,
+                          kept: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """The router from block means (``qk_rmsnorm_rope3d(..., block_means=)``):
+    fp32 [B, 2, n_blocks, H*hd] -> kept int32 [B, H, n_blocks, n_keep]."""
+    if block_means.dtype != torch.float32 or not block_means.is_cuda or \
+            not block_means.is_contiguous() or block_means.dim() != 4 or \
+            block_means.shape[1] != 2:
+        raise ValueError("block_means must be a contiguous CUDA float32 [B, 2, n_blocks, H*hd]")
+    B, _, nb, width = block_means.shape
+    if nb != (N + block - 1) // block or width % heads:
+        raise ValueError("block_means does not match N, block and heads")
+    hd = width // heads
+    if not 0.0 <= sparsity < 1.0:
+        raise ValueError("sparsity must be in [0, 1)")
+    if nb == 0 or B == 0:
+        return torch.empty(B, heads, nb, 0, dtype=torch.int32, device=block_means.device)
+    n_keep = subblock_keep_count(nb, sparsity)
+    need = int(library().dit_subblock_means_workspace_bytes(B, N, heads, block))
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=block_means.device)
+    if workspace.numel() * workspace.element_size() < need or \
+            workspace.device != block_means.device or not workspace.is_contiguous():
+        raise ValueError(f"workspace needs {need} contiguous bytes")
+    if kept is None:
+        kept = torch.empty(B, heads, nb, n_keep, dtype=torch.int32, device=block_means.device)
+    if kept.dtype != torch.int32 or kept.numel() != B * heads * nb * n_keep or \
+            not kept.is_contiguous() or kept.device != block_means.device:
+        raise ValueError(f"kept must be a contiguous int32 [B, H, {nb}, {n_keep}] tensor")
+    _call("dit_subblock_router_means", block_means.data_ptr(), B, N, heads, hd, block,
+          float(sparsity), kept.data_ptr(), workspace.data_ptr(),
+          workspace.numel() * workspace.element_size(), _stream(block_means))
     return kept
 
 

@@ -359,6 +359,199 @@ qk_rmsnorm_rope3d_kernel(QKParams p) {
     }
 }
 
+// ---------------------------------------------------------------------------
+// QK RMSNorm + 3D RoPE in place that also writes the mean of each block of
+// `block` consecutive tokens of the rotated q and k (the SubBlock router's
+// block summaries), so the router does not read q and k again.
+//
+// Work split: CTA (g, j, b) takes head group g (32*V row vectors: V vectors
+// per lane, whole heads since hd/8 divides 32) of token block j of sample b;
+// its 4 warps take consecutive quarters of the block's tokens.  Each warp
+// keeps kPoolStages tokens in flight through a private cp.async ring (a lane
+// copies, and later reads, only its own vectors), normalises and rotates
+// one token at a time, stores it in place, and adds the bf16-rounded results
+// to fp32 sums in token order.  The four warps' sums are then added in warp
+// order and divided by the block's token count once: the summation order is
+// fixed, so the means repeat bit for bit run to run.
+constexpr int kPoolWarps = 4;
+constexpr int kPoolStages = 4;
+constexpr int kPoolV = 2;            // vectors per lane per tensor
+
+template <int HD, int LAYOUT, int V>
+__global__ void __launch_bounds__(kPoolWarps * 32, 4)
+qk_rope_pool_kernel(QKParams p, int block, int nb, float* __restrict__ means) {
+    constexpr int LPH = HD / 8;             // lanes per head
+    constexpr int HALF = LPH / 2;
+    constexpr int NP = LAYOUT == 0 ? 4 : 8; // rotation pairs per lane
+    constexpr int SV = 2 * V;               // vectors per lane per token: q, then k
+    extern __shared__ uint4 pool_ring[];    // [warp][stage][SV][32 lanes]
+    __shared__ double s_omega[HD / 2];
+    __shared__ __align__(16) float s_w[2][HD];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int g = blockIdx.x, j = blockIdx.y, b = blockIdx.z;
+    const int v0 = g * 32 * V + lane;       // this lane's first row vector
+    const int sub = lane % LPH;
+    const bool first = (sub & HALF) == 0;
+    bool valid[V];
+#pragma unroll
+    for (int u = 0; u < V; ++u) valid[u] = v0 + 32 * u < p.nvr;
+    const int64_t n0 = static_cast<int64_t>(j) * block;
+    const int count = static_cast<int>((n0 + block < p.N ? n0 + block : p.N) - n0);
+    const int per = (block + kPoolWarps - 1) / kPoolWarps;
+    const int lo = warp * per < count ? warp * per : count;
+    const int hi = lo + per < count ? lo + per : count;
+    const int64_t row0 = static_cast<int64_t>(b) * p.N + n0;   // global row of token 0
+    uint4* ring = pool_ring + warp * (kPoolStages * SV * 32) + lane;
+
+    // copy token t's vectors into ring stage s (one commit group per token,
+    // empty past the warp's range so the group count stays uniform)
+    auto issue = [&](int t, int s) {
+        if (t < hi) {
+            const int64_t row = row0 + t;
+#pragma unroll
+            for (int u = 0; u < V; ++u) {
+                if (valid[u]) {
+                    cp_async16(ring + (s * SV + u) * 32, p.t0 + row * p.stride_v + v0 + 32 * u);
+                    cp_async16(ring + (s * SV + V + u) * 32,
+                               p.t1 + row * p.stride_v + v0 + 32 * u);
+                }
+            }
+        }
+        asm volatile("cp.async.commit_group;" ::: "memory");
+    };
+#pragma unroll
+    for (int s = 0; s < kPoolStages; ++s) issue(lo + s, s);
+
+    omega_table<HD>(p, s_omega);
+    for (int e = threadIdx.x; e < 2 * HD; e += blockDim.x)
+        s_w[e / HD][e % HD] = w_at(e < HD ? p.w0 : p.w1, p.w_dtype, e % HD);
+    __syncthreads();
+
+    float acc[2][V][8];
+#pragma unroll
+    for (int t = 0; t < 2; ++t)
+#pragma unroll
+        for (int u = 0; u < V; ++u)
+#pragma unroll
+            for (int i = 0; i < 8; ++i) acc[t][u][i] = 0.0f;
+
+    int s = 0;
+    for (int t = lo; t < hi; ++t) {
+        asm volatile("cp.async.wait_group %0;" ::"n"(kPoolStages - 1) : "memory");
+        uint4 v[SV];
+#pragma unroll
+        for (int x = 0; x < SV; ++x) v[x] = ring[(s * SV + x) * 32];
+        const int64_t row = row0 + t;
+        float cs[NP], sn[NP];
+        token_angles<HD, LAYOUT>(p, s_omega, row, sub, cs, sn);
+#pragma unroll
+        for (int ten = 0; ten < 2; ++ten) {
+            const float* w = s_w[ten];
+            uint4* orow = (ten == 0 ? p.o0 : p.o1) + row * p.stride_v + v0;
+            // per-lane coefficients with the weight folded in (as the
+            // one-token-per-warp kernel)
+            float A[8], Bc[8], C[4], Dd[4];
+            if (LAYOUT == 0) {
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const float wa = w[8 * sub + 2 * k], wb = w[8 * sub + 2 * k + 1];
+                    A[k] = wa * cs[k]; Bc[k] = -(wb * sn[k]); C[k] = wa * sn[k]; Dd[k] = wb * cs[k];
+                }
+            } else {
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const float wo = w[8 * sub + i], wp = w[8 * (sub ^ HALF) + i];
+                    A[i] = wo * cs[i];
+                    Bc[i] = (first ? -wp : wp) * sn[i];
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < V; ++u) {
+                const uint4 x = v[ten * V + u];
+                float f[8];
+                unpack8(x, f);
+                float ss = 0.0f;
+#pragma unroll
+                for (int i = 0; i < 8; ++i) ss = __fmaf_rn(f[i], f[i], ss);
+#pragma unroll
+                for (int o = LPH / 2; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+                const float inv = rsqrtf(__fmaf_rn(ss, 1.0f / static_cast<float>(HD), p.eps));
+                float o8[8];
+                if (LAYOUT == 0) {
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        o8[2 * k] = inv * __fmaf_rn(f[2 * k], A[k], f[2 * k + 1] * Bc[k]);
+                        o8[2 * k + 1] = inv * __fmaf_rn(f[2 * k], C[k], f[2 * k + 1] * Dd[k]);
+                    }
+                } else {
+                    uint4 pv;
+                    pv.x = __shfl_xor_sync(0xffffffffu, x.x, HALF);
+                    pv.y = __shfl_xor_sync(0xffffffffu, x.y, HALF);
+                    pv.z = __shfl_xor_sync(0xffffffffu, x.z, HALF);
+                    pv.w = __shfl_xor_sync(0xffffffffu, x.w, HALF);
+                    float fp[8];
+                    unpack8(pv, fp);
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) o8[i] = inv * __fmaf_rn(f[i], A[i], fp[i] * Bc[i]);
+                }
+                const uint4 packed = pack8(o8);
+                if (valid[u]) st_stream(orow + 32 * u, packed);
+                float r8[8];
+                unpack8(packed, r8);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) acc[ten][u][i] += r8[i];
+            }
+        }
+        // the stage's vectors are consumed: refill it with token t + stages
+        issue(t + kPoolStages, s);
+        s = s + 1 == kPoolStages ? 0 : s + 1;
+    }
+    asm volatile("cp.async.wait_group 0;" ::: "memory");
+    __syncthreads();
+    // warp sums -> shared memory [warp][tensor][u][lane][8], then warp order
+    float* cmb = reinterpret_cast<float*>(pool_ring);
+#pragma unroll
+    for (int t = 0; t < 2; ++t)
+#pragma unroll
+        for (int u = 0; u < V; ++u) {
+            float4* d = reinterpret_cast<float4*>(cmb + (((warp * 2 + t) * V + u) * 32 + lane) * 8);
+            d[0] = make_float4(acc[t][u][0], acc[t][u][1], acc[t][u][2], acc[t][u][3]);
+            d[1] = make_float4(acc[t][u][4], acc[t][u][5], acc[t][u][6], acc[t][u][7]);
+        }
+    __syncthreads();
+    const float cnt = static_cast<float>(count);
+    const int64_t D = static_cast<int64_t>(p.nvr) * 8;
+    for (int c = warp; c < 2 * V; c += kPoolWarps) {
+        const int t = c / V, u = c % V;
+        float sum[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        for (int w = 0; w < kPoolWarps; ++w) {
+            const float* src = cmb + (((w * 2 + t) * V + u) * 32 + lane) * 8;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) sum[i] += src[i];
+        }
+        if (valid[u]) {
+            float4* dst = reinterpret_cast<float4*>(
+                means + ((static_cast<int64_t>(b) * 2 + t) * nb + j) * D +
+                static_cast<int64_t>(v0 + 32 * u) * 8);
+            dst[0] = make_float4(sum[0] / cnt, sum[1] / cnt, sum[2] / cnt, sum[3] / cnt);
+            dst[1] = make_float4(sum[4] / cnt, sum[5] / cnt, sum[6] / cnt, sum[7] / cnt);
+        }
+    }
+}
+
+using PoolKernel = void (*)(QKParams, int, int, float*);
+
+template <int LAYOUT>
+PoolKernel pick_pool(int hd) {
+    switch (hd) {
+        case 32: return qk_rope_pool_kernel<32, LAYOUT, kPoolV>;
+        case 64: return qk_rope_pool_kernel<64, LAYOUT, kPoolV>;
+        case 128: return qk_rope_pool_kernel<128, LAYOUT, kPoolV>;
+        case 256: return qk_rope_pool_kernel<256, LAYOUT, kPoolV>;
+        default: return nullptr;
+    }
+}
+
 using QKKernel = void (*)(QKParams);
 
 struct Pick {
@@ -589,4 +782,76 @@ extern "C" int dit_qk_rmsnorm_rope3d(uint16_t* q, uint16_t* k, int64_t row_strid
     return dit_qk_rmsnorm_rope3d_ex(q, k, row_stride, w_q, w_k, w_dtype, B, N, H, hd, T, Hg, Wg,
                                     pos, pos_offset, pairs_t, pairs_h, pairs_w, theta, eps,
                                     DIT_ROPE_INTERLEAVED, DIT_NORM_HEAD, nullptr, stream);
+}
+
+extern "C" int dit_qk_rmsnorm_rope3d_pooled(uint16_t* q, uint16_t* k, int64_t row_stride,
+                                            const void* w_q, const void* w_k, int w_dtype, int B,
+                                            int64_t N, int H, int hd, int T, int Hg, int Wg,
+                                            const int32_t* pos, int64_t pos_offset, int pairs_t,
+                                            int pairs_h, int pairs_w, double theta, double eps,
+                                            int rope_layout, int block, float* block_means,
+                                            void* stream) {
+    using namespace dit;
+    if (w_dtype != DIT_F32 && w_dtype != DIT_BF16) return DIT_ERR_DTYPE;
+    if (B < 0 || N < 0 || H < 1 || block < 1) return DIT_ERR_SHAPE;
+    if (hd != 32 && hd != 64 && hd != 128 && hd != 256) return DIT_ERR_SHAPE;
+    if (rope_layout != DIT_ROPE_INTERLEAVED && rope_layout != DIT_ROPE_HALF) return DIT_ERR_VALUE;
+    if (pairs_t < 1 || pairs_h < 1 || pairs_w < 1 || pairs_t + pairs_h + pairs_w != hd / 2)
+        return DIT_ERR_SHAPE;
+    const int64_t width = static_cast<int64_t>(H) * hd;
+    if (width > DIT_MAX_D || row_stride < width) return DIT_ERR_SHAPE;
+    if (row_stride % 8) return DIT_ERR_ALIGN;
+    if (!(theta > 0.0) || theta > 1e300 || !(eps >= 0.0) || eps > 1e30) return DIT_ERR_VALUE;
+    if (B > 65535 || (B > 0 && N > (INT64_MAX / 4) / row_stride / B)) return DIT_ERR_SHAPE;
+    if (!pos) {
+        if (T < 1 || Hg < 1 || Wg < 1 || pos_offset < 0) return DIT_ERR_SHAPE;
+        const int64_t cells = static_cast<int64_t>(T) * Hg * Wg;
+        if (cells > INT32_MAX || pos_offset + N > cells) return DIT_ERR_SHAPE;
+    } else if (reinterpret_cast<uintptr_t>(pos) % 4) {
+        return DIT_ERR_ALIGN;
+    }
+    const int64_t nb = (N + block - 1) / block;
+    if (nb > 65535) return DIT_ERR_SHAPE;
+    if (B == 0 || N == 0) return DIT_OK;
+    if (!q || !k || !block_means) return DIT_ERR_NULL;
+    int st;
+    if ((st = check_w(w_q, w_dtype)) || (st = check_w(w_k, w_dtype))) return st;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(block_means)) return DIT_ERR_ALIGN;
+    const int64_t rows = static_cast<int64_t>(B) * N;
+    if (rows_overlap(q, k, rows, row_stride, width)) return DIT_ERR_OVERLAP;
+    const size_t mbytes = static_cast<size_t>(B) * 2 * nb * width * sizeof(float);
+    const size_t qbytes = 2 * static_cast<size_t>((rows - 1) * row_stride + width);
+    if (overlaps(block_means, mbytes, q, qbytes) || overlaps(block_means, mbytes, k, qbytes))
+        return DIT_ERR_OVERLAP;
+
+    QKParams p{};
+    p.t0 = reinterpret_cast<const uint4*>(q);
+    p.t1 = reinterpret_cast<const uint4*>(k);
+    p.o0 = reinterpret_cast<uint4*>(q);
+    p.o1 = reinterpret_cast<uint4*>(k);
+    p.w0 = w_q;
+    p.w1 = w_k;
+    p.w_dtype = w_dtype;
+    p.stride_v = row_stride / 8;
+    p.rows = rows;
+    p.N = N;
+    p.nvr = static_cast<int>(width / 8);
+    p.Hg = Hg;
+    p.Wg = Wg;
+    p.pos = pos;
+    p.pos_offset = pos_offset;
+    p.pt = pairs_t;
+    p.ph = pairs_h;
+    p.pw = pairs_w;
+    p.theta = theta;
+    p.eps = static_cast<float>(eps);
+    const PoolKernel kern = rope_layout == DIT_ROPE_HALF ? pick_pool<DIT_ROPE_HALF>(hd)
+                                                         : pick_pool<DIT_ROPE_INTERLEAVED>(hd);
+    if (!kern) return DIT_ERR_SHAPE;
+    const int groups = (p.nvr + 32 * kPoolV - 1) / (32 * kPoolV);
+    const size_t smem = static_cast<size_t>(kPoolWarps) * kPoolStages * 2 * kPoolV * 32 *
+                        sizeof(uint4);
+    kern<<<dim3(groups, static_cast<unsigned>(nb), B), kPoolWarps * 32, smem,
+           as_stream(stream)>>>(p, block, static_cast<int>(nb), block_means);
+    return launch_status();
 }

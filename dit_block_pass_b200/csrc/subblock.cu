@@ -290,6 +290,63 @@ extern "C" size_t dit_subblock_workspace_bytes(int B, int64_t N, int H, int hd, 
            sizeof(float);
 }
 
+namespace dit {
+namespace {
+
+// Scores and selection from the block means [B, 2, nb, H*hd] (fp32) into
+// the scores buffer [B, H, nb, nb].
+int route_from_means(const float* pooled, int B, int nb, int H, int hd, int n_keep,
+                     int32_t* kept, float* scores, cudaStream_t st) {
+    const int64_t D = static_cast<int64_t>(H) * hd;
+    const int64_t tiles = (nb + kScoreTile - 1) / kScoreTile;
+    subblock_scores_kernel<<<dim3(static_cast<unsigned>(tiles * tiles), H, B), kSelThreads, 0,
+                             st>>>(pooled, nb, static_cast<int>(D), hd, scores);
+    int rc = launch_status();
+    if (rc) return rc;
+    const dim3 sel((nb + 7) / 8, H, B);
+    if (nb <= 256)
+        subblock_select_kernel<8><<<sel, kSelThreads, 0, st>>>(scores, nb, n_keep, kept);
+    else if (nb <= 512)
+        subblock_select_kernel<16><<<sel, kSelThreads, 0, st>>>(scores, nb, n_keep, kept);
+    else if (nb <= 1024)
+        subblock_select_kernel<32><<<sel, kSelThreads, 0, st>>>(scores, nb, n_keep, kept);
+    else if (nb <= 2048)
+        subblock_select_kernel<64><<<sel, kSelThreads, 0, st>>>(scores, nb, n_keep, kept);
+    else
+        subblock_select_kernel<0><<<sel, kSelThreads, 0, st>>>(scores, nb, n_keep, kept);
+    return launch_status();
+}
+
+}  // namespace
+}  // namespace dit
+
+extern "C" size_t dit_subblock_means_workspace_bytes(int B, int64_t N, int H, int block) {
+    if (B < 0 || N < 0 || H < 1 || block < 1) return 0;
+    const int64_t nb = (N + block - 1) / block;
+    return static_cast<size_t>(B) * H * nb * nb * sizeof(float);
+}
+
+extern "C" int dit_subblock_router_means(const float* block_means, int B, int64_t N, int H,
+                                         int hd, int block, double sparsity, int32_t* kept,
+                                         void* workspace, size_t workspace_bytes, void* stream) {
+    using namespace dit;
+    if (B < 0 || N < 0 || H < 1 || block < 1) return DIT_ERR_SHAPE;
+    if (hd < 8 || hd > 256 || hd % 8) return DIT_ERR_SHAPE;
+    if (static_cast<int64_t>(H) * hd > DIT_MAX_D) return DIT_ERR_SHAPE;
+    if (!(sparsity >= 0.0) || !(sparsity < 1.0)) return DIT_ERR_VALUE;
+    if (B == 0 || N == 0) return DIT_OK;
+    const int64_t nb64 = (N + block - 1) / block;
+    if (nb64 > kMaxBlocks || B > 65535) return DIT_ERR_SHAPE;
+    const int nb = static_cast<int>(nb64);
+    if (!block_means || !kept) return DIT_ERR_NULL;
+    if (!aligned16(block_means) || reinterpret_cast<uintptr_t>(kept) % 4) return DIT_ERR_ALIGN;
+    if (!workspace || !aligned16(workspace) ||
+        workspace_bytes < dit_subblock_means_workspace_bytes(B, N, H, block))
+        return DIT_ERR_WORKSPACE;
+    return route_from_means(block_means, B, nb, H, hd, keep_count(nb, sparsity), kept,
+                            static_cast<float*>(workspace), as_stream(stream));
+}
+
 extern "C" int dit_subblock_router(const uint16_t* q, const uint16_t* k, int64_t row_stride,
                                    int B, int64_t N, int H, int hd, int block, double sparsity,
                                    int32_t* kept, void* workspace, size_t workspace_bytes,
@@ -320,21 +377,5 @@ extern "C" int dit_subblock_router(const uint16_t* q, const uint16_t* k, int64_t
     int rc = launch_status();
     if (rc) return rc;
     float* scores = pooled + static_cast<int64_t>(B) * 2 * nb * D;
-    const int64_t tiles = (nb + kScoreTile - 1) / kScoreTile;
-    subblock_scores_kernel<<<dim3(static_cast<unsigned>(tiles * tiles), H, B), kSelThreads, 0,
-                             st>>>(pooled, nb, static_cast<int>(D), hd, scores);
-    rc = launch_status();
-    if (rc) return rc;
-    const dim3 sel((nb + 7) / 8, H, B);
-    if (nb <= 256)
-        subblock_select_kernel<8><<<sel, kSelThreads, 0, st>>>(scores, nb, n_keep, kept);
-    else if (nb <= 512)
-        subblock_select_kernel<16><<<sel, kSelThreads, 0, st>>>(scores, nb, n_keep, kept);
-    else if (nb <= 1024)
-        subblock_select_kernel<32><<<sel, kSelThreads, 0, st>>>(scores, nb, n_keep, kept);
-    else if (nb <= 2048)
-        subblock_select_kernel<64><<<sel, kSelThreads, 0, st>>>(scores, nb, n_keep, kept);
-    else
-        subblock_select_kernel<0><<<sel, kSelThreads, 0, st>>>(scores, nb, n_keep, kept);
-    return launch_status();
+    return route_from_means(pooled, B, nb, H, hd, n_keep, kept, scores, st);
 }

@@ -232,6 +232,34 @@ int dit_qk_rmsnorm_rope3d_ex(uint16_t* q, uint16_t* k, int64_t row_stride,
                              const dit_qk_out* out, void* stream);
 
 /*
+ * dit_qk_rmsnorm_rope3d_ex in place with per-head norm (DIT_NORM_HEAD), that
+ * also writes the SubBlock router's block summaries of its results, so the
+ * router need not read q and k again (the LMSYS report, news.cocoloop.cn,
+ * "minimax-h3-sglang-h200", section "Só com três camadas de aceleração
+ * somadas chega-se a 6 vezes": fused operators cut memory traffic; SubBlock
+ * attention routes over KV blocks).
+ *   block        tokens per router block, >= 1; n_blocks = ceil(N / block),
+ *                counted from the first token of each sample in this call,
+ *                <= 65535.
+ *   block_means  device fp32 [B, 2, n_blocks, H*hd], 16-byte aligned, not
+ *                overlapping q or k: [b][0][j] is the mean over block j's
+ *                tokens of the rotated q rows as stored (bf16), [b][1][j] the
+ *                same for k (the last block may hold fewer tokens).  Each
+ *                mean is an fp32 sum in a fixed order divided once by the
+ *                token count, so results repeat run to run.  It is the input
+ *                of dit_subblock_router_means.
+ * q and k are both required (DIT_ERR_NULL); other arguments, errors and
+ * limits as dit_qk_rmsnorm_rope3d_ex (rope_layout as there; B <= 65535).
+ */
+int dit_qk_rmsnorm_rope3d_pooled(uint16_t* q, uint16_t* k, int64_t row_stride,
+                                 const void* w_q, const void* w_k, int w_dtype,
+                                 int B, int64_t N, int H, int hd,
+                                 int T, int Hg, int Wg, const int32_t* pos, int64_t pos_offset,
+                                 int pairs_t, int pairs_h, int pairs_w,
+                                 double theta, double eps, int rope_layout, int block,
+                                 float* block_means, void* stream);
+
+/*
  * Cache-DiT residual-difference check between neighbouring denoising steps.
  *   Per sample b:  rel_b   = sum_{n,d} |cur - prev| / sum_{n,d} |prev|
  *                  reuse_b = rel_b < threshold       (strict)
@@ -355,6 +383,22 @@ size_t dit_subblock_workspace_bytes(int B, int64_t N, int H, int hd, int block);
 int dit_subblock_router(const uint16_t* q, const uint16_t* k, int64_t row_stride, int B,
                         int64_t N, int H, int hd, int block, double sparsity, int32_t* kept,
                         void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * The SubBlock router from block means already computed (for example by
+ * dit_qk_rmsnorm_rope3d_pooled): the scores and the selection of
+ * dit_subblock_router, without reading q and k.
+ *   block_means  device fp32 [B, 2, n_blocks, H*hd] (q means, then k means),
+ *                16-byte aligned; n_blocks = ceil(N / block) <= 8192.
+ *   workspace    device, >= dit_subblock_means_workspace_bytes(B, N, H, block)
+ *                bytes (the scores [B, H, n_blocks, n_blocks] fp32),
+ *                16-byte aligned.
+ * kept, sparsity, hd limits and errors as dit_subblock_router.
+ */
+size_t dit_subblock_means_workspace_bytes(int B, int64_t N, int H, int block);
+int dit_subblock_router_means(const float* block_means, int B, int64_t N, int H, int hd,
+                              int block, double sparsity, int32_t* kept, void* workspace,
+                              size_t workspace_bytes, void* stream);
 
 /*
  * Block-sparse attention over the router's kept key blocks (tensor cores):
