@@ -108,7 +108,7 @@ def library() -> ctypes.CDLL:
                                                    ctypes.POINTER(QKOut), vp]
             L.dit_qk_rmsnorm_rope3d_pooled.argtypes = [vp, vp, i64, vp, vp, i32, i32, i64, i32,
                                                        i32, i32, i32, i32, vp, i64, i32, i32,
-                                                       i32, dbl, dbl, i32, i32, vp, vp]
+                                                       i32, dbl, dbl, i32, i32, vp, vp, vp]
             L.dit_subblock_means_workspace_bytes.argtypes = [i32, i64, i32, i32]
             L.dit_subblock_means_workspace_bytes.restype = sz
             L.dit_subblock_router_means.argtypes = [vp, i32, i64, i32, i32, i32, dbl, vp, vp, sz,
@@ -343,7 +343,8 @@ def qk_rmsnorm_rope3d(q: Optional[torch.Tensor], k: Optional[torch.Tensor],
                       rope_layout: int = ROPE_INTERLEAVED, norm_width: int = NORM_HEAD,
                       q_out: Optional[torch.Tensor] = None,
                       k_out: Optional[torch.Tensor] = None,
-                      block_means: Optional[torch.Tensor] = None, block: int = 128) -> None:
+                      block_means: Optional[torch.Tensor] = None, block: int = 128,
+                      status: Optional[torch.Tensor] = None) -> None:
     """In place on q and k ([B, N, H*hd] views, e.g. slices of a fused qkv
     buffer): RMSNorm with weight w, then 3D RoPE with pair split
     ``pairs`` = (t, h, w).  Positions come from ``grid`` = (T, Hg, Wg) (token
@@ -357,7 +358,8 @@ def qk_rmsnorm_rope3d(q: Optional[torch.Tensor], k: Optional[torch.Tensor],
     With ``block_means`` (fp32 [B, 2, ceil(N/block), H*hd], contiguous) the
     call is in place with the per-head norm and also writes the mean of each
     block of ``block`` tokens of the rotated q ([:, 0]) and k ([:, 1]), the
-    input of ``subblock_router_means``."""
+    input of ``subblock_router_means``; ``status`` (int32 CUDA scalar) is set to
+    1 if a wait of that path's copy pipeline expired."""
     ref = q if q is not None else k
     if ref is None:
         raise ValueError("q and k cannot both be None")
@@ -397,6 +399,8 @@ def qk_rmsnorm_rope3d(q: Optional[torch.Tensor], k: Optional[torch.Tensor],
         if q is None or k is None or q_out is not None or k_out is not None or \
                 norm_width != NORM_HEAD:
             raise ValueError("block_means needs q and k, in place, with the per-head norm")
+        if status is not None and (status.dtype != torch.int32 or not status.is_cuda):
+            raise ValueError("status must be a CUDA int32 tensor")
         if block_means.dtype != torch.float32 or not block_means.is_contiguous() or \
                 block_means.device != ref.device or \
                 tuple(block_means.shape) != (B, 2, nb, width):
@@ -404,7 +408,8 @@ def qk_rmsnorm_rope3d(q: Optional[torch.Tensor], k: Optional[torch.Tensor],
                              f"tensor on {ref.device}")
         _call("dit_qk_rmsnorm_rope3d_pooled", _ptr(q), _ptr(k), rs, _ptr(w_q), _ptr(w_k), w_dt,
               B, N, heads, hd, T, Hg, Wg, _ptr(pos), int(pos_offset), pt, ph, pw, float(theta),
-              float(eps), int(rope_layout), int(block), block_means.data_ptr(), _stream(ref))
+              float(eps), int(rope_layout), int(block), block_means.data_ptr(), _ptr(status),
+              _stream(ref))
         return
     out = None
     if q_out is not None or k_out is not None:

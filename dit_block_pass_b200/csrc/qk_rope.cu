@@ -34,7 +34,7 @@
 // fp64, and sin/cos are taken in fp32 on the reduced angle, which keeps the
 // rotation accurate to a few fp32 ulp for positions in the hundreds.  HBM
 // bound.
-#include "common.cuh"
+#include "tcgen05.cuh"
 
 namespace dit {
 namespace {
@@ -366,58 +366,114 @@ qk_rmsnorm_rope3d_kernel(QKParams p) {
 //
 // Work split: CTA (g, j, b) takes head group g (32*V row vectors: V vectors
 // per lane, whole heads since hd/8 divides 32) of token block j of sample b;
-// its 4 warps take consecutive quarters of the block's tokens.  Each warp
-// keeps kPoolStages tokens in flight through a private cp.async ring (a lane
-// copies, and later reads, only its own vectors), normalises and rotates
-// one token at a time, stores it in place, and adds the bf16-rounded results
-// to fp32 sums in token order.  The four warps' sums are then added in warp
-// order and divided by the block's token count once: the summation order is
-// fixed, so the means repeat bit for bit run to run.
+// its 4 warps take consecutive quarters of the block's tokens.  The group's
+// slice of a token row is contiguous, so one lane of each warp brings a
+// token's q and k slices into a private ring of kPoolStages stages with two
+// bulk copies (completion counted on the stage's mbarrier); the warp then
+// normalises and rotates the token from shared memory, stores it in place,
+// and adds the bf16-rounded results to fp32 sums in token order.  The four
+// warps' sums are added in warp order and divided by the block's token count
+// once: the summation order is fixed, so the means repeat bit for bit.
+//
+// Angles: a lane always holds the same rotation pairs.  When a token sits one
+// step further along w than the warp's previous token (same t and h), the
+// w-axis pairs advance by one rotation by their frequency (t and h pairs
+// stay); otherwise, and at least every kRecur tokens, every angle is formed
+// afresh (fp64 reduction, fp32 sin/cos).  The recurrence adds at most a few
+// fp32 ulp per step, far below a bf16 ulp of the result.
 constexpr int kPoolWarps = 4;
-constexpr int kPoolStages = 4;
+constexpr int kPoolStages = 6;
 constexpr int kPoolV = 2;            // vectors per lane per tensor
+constexpr int kRecur = 128;          // longest run of recurrence steps
+
+__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes,
+                                         uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
+            "r"(dst),
+        "l"(src), "r"(bytes), "r"(bar)
+        : "memory");
+}
+
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float& lo, float& hi) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+
+// The token's (t, h, w) position (grid index or explicit table).
+__device__ __forceinline__ void token_pos(const QKParams& p, int64_t tok, int& t, int& h,
+                                          int& w) {
+    if (p.pos) {
+        t = p.pos[3 * tok + 0];
+        h = p.pos[3 * tok + 1];
+        w = p.pos[3 * tok + 2];
+    } else {
+        const int hw = p.Hg * p.Wg;
+        const int g = static_cast<int>(p.pos_offset + tok % p.N);
+        t = g / hw;
+        const int rem = g - t * hw;
+        h = rem / p.Wg;
+        w = rem - h * p.Wg;
+    }
+}
 
 template <int HD, int LAYOUT, int V>
 __global__ void __launch_bounds__(kPoolWarps * 32, 4)
-qk_rope_pool_kernel(QKParams p, int block, int nb, float* __restrict__ means) {
+qk_rope_pool_kernel(QKParams p, int block, int nb, float* __restrict__ means, int* status) {
     constexpr int LPH = HD / 8;             // lanes per head
     constexpr int HALF = LPH / 2;
     constexpr int NP = LAYOUT == 0 ? 4 : 8; // rotation pairs per lane
     constexpr int SV = 2 * V;               // vectors per lane per token: q, then k
-    extern __shared__ uint4 pool_ring[];    // [warp][stage][SV][32 lanes]
+    constexpr uint32_t kStage = SV * 32 * 16;
+    extern __shared__ __align__(128) uint8_t pool_smem[];
     __shared__ double s_omega[HD / 2];
     __shared__ __align__(16) float s_w[2][HD];
+    __shared__ int s_abort;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int g = blockIdx.x, j = blockIdx.y, b = blockIdx.z;
-    const int v0 = g * 32 * V + lane;       // this lane's first row vector
+    const int vbase = g * 32 * V;
+    const int v0 = vbase + lane;            // this lane's first row vector
+    const int nvec = p.nvr - vbase < 32 * V ? p.nvr - vbase : 32 * V;
+    const uint32_t chunk = static_cast<uint32_t>(nvec) * 16;   // bytes per tensor and token
     const int sub = lane % LPH;
     const bool first = (sub & HALF) == 0;
     bool valid[V];
 #pragma unroll
-    for (int u = 0; u < V; ++u) valid[u] = v0 + 32 * u < p.nvr;
+    for (int u = 0; u < V; ++u) valid[u] = 32 * u + lane < nvec;
     const int64_t n0 = static_cast<int64_t>(j) * block;
     const int count = static_cast<int>((n0 + block < p.N ? n0 + block : p.N) - n0);
     const int per = (block + kPoolWarps - 1) / kPoolWarps;
     const int lo = warp * per < count ? warp * per : count;
     const int hi = lo + per < count ? lo + per : count;
     const int64_t row0 = static_cast<int64_t>(b) * p.N + n0;   // global row of token 0
-    uint4* ring = pool_ring + warp * (kPoolStages * SV * 32) + lane;
+    const uint32_t ring = tc::smem_u32(pool_smem) + warp * kPoolStages * kStage;
+    const uint32_t bars = tc::smem_u32(pool_smem) + kPoolWarps * kPoolStages * kStage +
+                          warp * kPoolStages * 8;
 
-    // copy token t's vectors into ring stage s (one commit group per token,
-    // empty past the warp's range so the group count stays uniform)
+    if (threadIdx.x == 0) s_abort = 0;
+    if (lane == 0) {
+        for (int s = 0; s < kPoolStages; ++s) tc::mbar_init(bars + 8 * s, 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    __syncwarp();
+    // token t's q and k slices into stage s (lane 0)
     auto issue = [&](int t, int s) {
-        if (t < hi) {
+        if (lane == 0 && t < hi) {
             const int64_t row = row0 + t;
-#pragma unroll
-            for (int u = 0; u < V; ++u) {
-                if (valid[u]) {
-                    cp_async16(ring + (s * SV + u) * 32, p.t0 + row * p.stride_v + v0 + 32 * u);
-                    cp_async16(ring + (s * SV + V + u) * 32,
-                               p.t1 + row * p.stride_v + v0 + 32 * u);
-                }
-            }
+            tc::mbar_expect_tx(bars + 8 * s, 2 * chunk);
+            bulk_g2s(ring + s * kStage, p.t0 + row * p.stride_v + vbase, chunk, bars + 8 * s);
+            bulk_g2s(ring + s * kStage + V * 32 * 16, p.t1 + row * p.stride_v + vbase, chunk,
+                     bars + 8 * s);
         }
-        asm volatile("cp.async.commit_group;" ::: "memory");
     };
 #pragma unroll
     for (int s = 0; s < kPoolStages; ++s) issue(lo + s, s);
@@ -427,35 +483,84 @@ qk_rope_pool_kernel(QKParams p, int block, int nb, float* __restrict__ means) {
         s_w[e / HD][e % HD] = w_at(e < HD ? p.w0 : p.w1, p.w_dtype, e % HD);
     __syncthreads();
 
-    float acc[2][V][8];
+    // this lane's pairs: index, and the per-token step of w-axis pairs
+    float stc[NP], sts[NP], cs[NP], sn[NP];
+#pragma unroll
+    for (int k = 0; k < NP; ++k) {
+        const int pr = LAYOUT == 0 ? 4 * sub + k : 8 * (sub % HALF) + k;
+        if (pr >= p.pt + p.ph) {
+            double sd, cd;
+            sincos(s_omega[pr], &sd, &cd);
+            stc[k] = static_cast<float>(cd);
+            sts[k] = static_cast<float>(sd);
+        } else {
+            stc[k] = 1.0f;
+            sts[k] = 0.0f;
+        }
+        cs[k] = 1.0f;
+        sn[k] = 0.0f;
+    }
+    int pt_ = -1, ph_ = -1, pw_ = -1, run = kRecur;
+
+    uint64_t acc[2][V][4];
 #pragma unroll
     for (int t = 0; t < 2; ++t)
 #pragma unroll
         for (int u = 0; u < V; ++u)
 #pragma unroll
-            for (int i = 0; i < 8; ++i) acc[t][u][i] = 0.0f;
+            for (int i = 0; i < 4; ++i) acc[t][u][i] = 0ull;
 
-    int s = 0;
+    bool failed = false;
+    int done = lo;                          // tokens whose stage was consumed
     for (int t = lo; t < hi; ++t) {
-        asm volatile("cp.async.wait_group %0;" ::"n"(kPoolStages - 1) : "memory");
+        const int k = t - lo;
+        const int s = k % kPoolStages;
+        if (!__all_sync(0xffffffffu, tc::mbar_wait(bars + 8 * s, (k / kPoolStages) & 1,
+                                                     &s_abort))) {
+            failed = true;
+            break;
+        }
+        const uint4* st = reinterpret_cast<const uint4*>(pool_smem + (ring - tc::smem_u32(pool_smem)) +
+                                                         s * kStage);
         uint4 v[SV];
 #pragma unroll
-        for (int x = 0; x < SV; ++x) v[x] = ring[(s * SV + x) * 32];
+        for (int x = 0; x < SV; ++x) v[x] = st[x * 32 + lane];
+        __syncwarp();
+        issue(t + kPoolStages, s);          // every lane has read the stage
+        done = t + 1;
         const int64_t row = row0 + t;
-        float cs[NP], sn[NP];
-        token_angles<HD, LAYOUT>(p, s_omega, row, sub, cs, sn);
+        int tt, th, tw;
+        token_pos(p, row, tt, th, tw);
+        if (tt == pt_ && th == ph_ && tw == pw_ + 1 && run < kRecur) {
+#pragma unroll
+            for (int q = 0; q < NP; ++q) {
+                const float c = cs[q], d = sn[q];
+                cs[q] = __fmaf_rn(c, stc[q], -(d * sts[q]));
+                sn[q] = __fmaf_rn(d, stc[q], c * sts[q]);
+            }
+            ++run;
+        } else {
+            token_angles<HD, LAYOUT>(p, s_omega, row, sub, cs, sn);
+            run = 0;
+        }
+        pt_ = tt;
+        ph_ = th;
+        pw_ = tw;
 #pragma unroll
         for (int ten = 0; ten < 2; ++ten) {
             const float* w = s_w[ten];
             uint4* orow = (ten == 0 ? p.o0 : p.o1) + row * p.stride_v + v0;
-            // per-lane coefficients with the weight folded in (as the
-            // one-token-per-warp kernel)
             float A[8], Bc[8], C[4], Dd[4];
             if (LAYOUT == 0) {
+                const float4 wa = *reinterpret_cast<const float4*>(w + 8 * sub);
+                const float4 wb = *reinterpret_cast<const float4*>(w + 8 * sub + 4);
+                const float wv[8] = {wa.x, wa.y, wa.z, wa.w, wb.x, wb.y, wb.z, wb.w};
 #pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    const float wa = w[8 * sub + 2 * k], wb = w[8 * sub + 2 * k + 1];
-                    A[k] = wa * cs[k]; Bc[k] = -(wb * sn[k]); C[k] = wa * sn[k]; Dd[k] = wb * cs[k];
+                for (int q = 0; q < 4; ++q) {
+                    A[q] = wv[2 * q] * cs[q];
+                    Bc[q] = -(wv[2 * q + 1] * sn[q]);
+                    C[q] = wv[2 * q] * sn[q];
+                    Dd[q] = wv[2 * q + 1] * cs[q];
                 }
             } else {
 #pragma unroll
@@ -479,9 +584,9 @@ qk_rope_pool_kernel(QKParams p, int block, int nb, float* __restrict__ means) {
                 float o8[8];
                 if (LAYOUT == 0) {
 #pragma unroll
-                    for (int k = 0; k < 4; ++k) {
-                        o8[2 * k] = inv * __fmaf_rn(f[2 * k], A[k], f[2 * k + 1] * Bc[k]);
-                        o8[2 * k + 1] = inv * __fmaf_rn(f[2 * k], C[k], f[2 * k + 1] * Dd[k]);
+                    for (int q = 0; q < 4; ++q) {
+                        o8[2 * q] = inv * __fmaf_rn(f[2 * q], A[q], f[2 * q + 1] * Bc[q]);
+                        o8[2 * q + 1] = inv * __fmaf_rn(f[2 * q], C[q], f[2 * q + 1] * Dd[q]);
                     }
                 } else {
                     uint4 pv;
@@ -499,26 +604,39 @@ qk_rope_pool_kernel(QKParams p, int block, int nb, float* __restrict__ means) {
                 float r8[8];
                 unpack8(packed, r8);
 #pragma unroll
-                for (int i = 0; i < 8; ++i) acc[ten][u][i] += r8[i];
+                for (int i = 0; i < 4; ++i)
+                    acc[ten][u][i] = f2_add(acc[ten][u][i], f2_pack(r8[2 * i], r8[2 * i + 1]));
             }
         }
-        // the stage's vectors are consumed: refill it with token t + stages
-        issue(t + kPoolStages, s);
-        s = s + 1 == kPoolStages ? 0 : s + 1;
     }
-    asm volatile("cp.async.wait_group 0;" ::: "memory");
+    if (failed) {
+        s_abort = 1;
+        if (status) atomicExch(status, 1);
+        // the copies this warp issued land before the CTA exits
+        if (lane == 0) {
+            for (int t = done; t < hi && t < done + kPoolStages; ++t) {
+                const int k = t - lo;
+                tc::mbar_wait_drain(bars + 8 * (k % kPoolStages), (k / kPoolStages) & 1);
+            }
+        }
+        __syncwarp();
+    }
     __syncthreads();
     // warp sums -> shared memory [warp][tensor][u][lane][8], then warp order
-    float* cmb = reinterpret_cast<float*>(pool_ring);
+    float* cmb = reinterpret_cast<float*>(pool_smem);
 #pragma unroll
     for (int t = 0; t < 2; ++t)
 #pragma unroll
         for (int u = 0; u < V; ++u) {
+            float a[8];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) f2_unpack(acc[t][u][i], a[2 * i], a[2 * i + 1]);
             float4* d = reinterpret_cast<float4*>(cmb + (((warp * 2 + t) * V + u) * 32 + lane) * 8);
-            d[0] = make_float4(acc[t][u][0], acc[t][u][1], acc[t][u][2], acc[t][u][3]);
-            d[1] = make_float4(acc[t][u][4], acc[t][u][5], acc[t][u][6], acc[t][u][7]);
+            d[0] = make_float4(a[0], a[1], a[2], a[3]);
+            d[1] = make_float4(a[4], a[5], a[6], a[7]);
         }
     __syncthreads();
+    if (s_abort) return;
     const float cnt = static_cast<float>(count);
     const int64_t D = static_cast<int64_t>(p.nvr) * 8;
     for (int c = warp; c < 2 * V; c += kPoolWarps) {
@@ -539,7 +657,7 @@ qk_rope_pool_kernel(QKParams p, int block, int nb, float* __restrict__ means) {
     }
 }
 
-using PoolKernel = void (*)(QKParams, int, int, float*);
+using PoolKernel = void (*)(QKParams, int, int, float*, int*);
 
 template <int LAYOUT>
 PoolKernel pick_pool(int hd) {
@@ -790,7 +908,7 @@ extern "C" int dit_qk_rmsnorm_rope3d_pooled(uint16_t* q, uint16_t* k, int64_t ro
                                             const int32_t* pos, int64_t pos_offset, int pairs_t,
                                             int pairs_h, int pairs_w, double theta, double eps,
                                             int rope_layout, int block, float* block_means,
-                                            void* stream) {
+                                            int* status, void* stream) {
     using namespace dit;
     if (w_dtype != DIT_F32 && w_dtype != DIT_BF16) return DIT_ERR_DTYPE;
     if (B < 0 || N < 0 || H < 1 || block < 1) return DIT_ERR_SHAPE;
@@ -849,9 +967,14 @@ extern "C" int dit_qk_rmsnorm_rope3d_pooled(uint16_t* q, uint16_t* k, int64_t ro
                                                          : pick_pool<DIT_ROPE_INTERLEAVED>(hd);
     if (!kern) return DIT_ERR_SHAPE;
     const int groups = (p.nvr + 32 * kPoolV - 1) / (32 * kPoolV);
-    const size_t smem = static_cast<size_t>(kPoolWarps) * kPoolStages * 2 * kPoolV * 32 *
-                        sizeof(uint4);
+    if (status && reinterpret_cast<uintptr_t>(status) % 4) return DIT_ERR_ALIGN;
+    // the rings, then one mbarrier per stage and warp
+    const size_t smem = static_cast<size_t>(kPoolWarps) * kPoolStages * (2 * kPoolV * 32 * 16 + 8);
+    if (smem > 48 * 1024 &&
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem)) != cudaSuccess)
+        return DIT_ERR_LAUNCH;
     kern<<<dim3(groups, static_cast<unsigned>(nb), B), kPoolWarps * 32, smem,
-           as_stream(stream)>>>(p, block, static_cast<int>(nb), block_means);
+           as_stream(stream)>>>(p, block, static_cast<int>(nb), block_means, status);
     return launch_status();
 }

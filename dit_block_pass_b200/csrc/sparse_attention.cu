@@ -24,10 +24,12 @@
 //             columns P_n does not use as soon as the softmax has read S_n
 //             (so they run during softmax n and P_n V_n); keys 0..63 follow
 //             once P_n V_n has read P_n.
-//   warps 2-5 softmax, thread = query row (TMEM lane): tcgen05.ld the S row
-//             (then report S_n read), mask keys past the sample's last token,
-//             the row max of the raw scores in four chains, weights
-//             2^(s * scale * log2 e - m) with one fma each, in fp32 with
+//   warps 2-5 softmax, thread = query row (TMEM lane): keys past the
+//             sample's last token are set to -inf in TMEM (only a partial
+//             block needs it), tcgen05.ld the S row (then report S_n read),
+//             the row max of the raw scores in four chains of three-input
+//             maxima, weights 2^(s * scale * log2 e - m) with one paired fma
+//             per two weights and ex2.approx, row sums in paired adds, with
 //             lazy rescaling (the reference max m moves, and O and
 //             the row sum are rescaled in TMEM, only when a row's block max
 //             exceeds m by more than 8, so weights stay below 2^8), and P
@@ -44,7 +46,14 @@ using namespace tc;
 
 constexpr int kBlk = 128;                       // tokens per block (rows of every tile)
 constexpr int kHd = 128;                        // head size
-constexpr int kThreadsA = 192;
+constexpr int kThreadsA = 256;                  // two warpgroups
+// Register split (setmaxnreg): the kernel is launched with 128 registers per
+// thread (two CTAs of 256 threads fill the SM's 65,536); the copy/MMA
+// warpgroup gives up to 40 and the softmax warpgroup takes 216, which adds up
+// to the launch total: 128 * (40 + 216) = 256 * 128.
+constexpr int kRegsLaunch = 128;
+constexpr int kRegsLow = 56;
+constexpr int kRegsHigh = 2 * kRegsLaunch - kRegsLow;
 constexpr uint32_t kTile = kBlk * kHd * 2;      // 32 KB: one 128 x 128 bf16 tile
 constexpr uint32_t kHalfTile = kTile / 2;       // 16 KB: 64 columns (one swizzle atom wide)
 constexpr uint32_t kTmemColsA = 256;           // two CTAs share an SM's 512 columns
@@ -64,6 +73,61 @@ __device__ __forceinline__ void mma_f16_ts(uint32_t tmem_d, uint32_t tmem_a, uin
         "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(tmem_d),
         "r"(tmem_a), "l"(db), "r"(idesc), "r"(accumulate)
         : "memory");
+}
+
+// fp32 pairs in one 64-bit register (sm_100 paired arithmetic).
+__device__ __forceinline__ uint64_t pack_f2(float lo, float hi) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ void unpack_f2(uint64_t v, float& lo, float& hi) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t fma_f2(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+__device__ __forceinline__ uint64_t add_f2(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+// max of three (sm_100)
+__device__ __forceinline__ float max3(float a, float b, float c) {
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+// 2^x on the special-function unit, subnormal results flushed to zero (a
+// weight below 2^-126 of the row's reference is lost in bf16 P anyway).
+__device__ __forceinline__ float ex2_ftz(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// -inf into columns valid .. 127 of this warp's 32 rows of S (tensor
+// memory address `row_base`): whole 32-column chunks at once, the chunk
+// holding the boundary one column at a time.
+__device__ __forceinline__ void mask_tail(uint32_t row_base, int valid) {
+    float ninf[32];
+#pragma unroll
+    for (int e = 0; e < 32; ++e) ninf[e] = -INFINITY;
+    for (int c = 0; c < kBlk / 32; ++c) {
+        const int c0 = 32 * c;
+        if (c0 >= valid) {
+            tmem_st32(row_base + c0, ninf);
+        } else if (c0 + 32 > valid) {
+            for (int col = valid; col < c0 + 32; ++col)
+                asm volatile("tcgen05.st.sync.aligned.32x32b.x1.b32 [%0], {%1};" ::"r"(
+                                 row_base + static_cast<uint32_t>(col)),
+                             "r"(__float_as_uint(-INFINITY))
+                             : "memory");
+        }
+    }
+    tmem_wait_st();
 }
 
 // Keys k0 .. k0 + 63 of S = Q K^T (k0 = 0 or 64) into TMEM columns k0 ..
@@ -136,6 +200,9 @@ block_sparse_attention_kernel(const __grid_constant__ CUtensorMap map_q,
     const uint32_t tmem = *tmem_slot;
     bool failed = false;
 
+    if (warp < 4) {
+    // copy and MMA warpgroup (warps 2 and 3 only wait at the end)
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsLow));
     if (warp == 0) {
         if (lane == 0) {
             // the Q tile, then K and V of every kept block (one buffer each:
@@ -234,18 +301,28 @@ block_sparse_attention_kernel(const __grid_constant__ CUtensorMap map_q,
             }
         }
         __syncwarp();
+    }
     } else {
-        // softmax: thread = query row r (TMEM lane)
+        // softmax warpgroup: thread = query row r (TMEM lane)
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsHigh));
         const int q = warp & 3;
         const int r = 32 * q + lane;
         const uint32_t lane_off = static_cast<uint32_t>(32 * q) << 16;
         float m_run = -INFINITY, l_run = 0.0f;
         for (int n = 0; n < nk; ++n) {
+            // keys past the sample's last token do not take part
+            const int64_t j = __ldg(kept + n);
+            const int64_t left = p.N - j * kBlk;
+            const int valid = left >= kBlk ? kBlk : (left > 0 ? static_cast<int>(left) : 0);
             if (!__all_sync(0xffffffffu, mbar_wait(bar_s_full, n & 1, abort))) {
                 failed = true;
                 break;
             }
             fence_after_sync();
+            // a sample's last block may be partial: its missing keys' scores
+            // become -inf in tensor memory (the same block for every row, so
+            // the branch is uniform), and full blocks need no mask at all
+            if (valid < kBlk) mask_tail(tmem + lane_off, valid);
             float sc[kBlk];
 #pragma unroll
             for (int c = 0; c < kBlk / 32; ++c)
@@ -255,34 +332,42 @@ block_sparse_attention_kernel(const __grid_constant__ CUtensorMap map_q,
             fence_before_sync();
             __syncwarp();
             if (lane == 0) mbar_arrive(bar_s_free);
-            // keys past the sample's last token do not take part
-            const int64_t j = __ldg(kept + n);
-            const int64_t left = p.N - j * kBlk;
-            const int valid = left >= kBlk ? kBlk : (left > 0 ? static_cast<int>(left) : 0);
             // the row max of the raw scores (scale > 0 and rounding is monotonic,
             // so scaling the max equals the max of the scaled scores), in four
-            // independent chains
-            float mq[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+            // independent chains of three-input maxima
+            float mq[4] = {fmaxf(sc[0], sc[4]), fmaxf(sc[1], sc[5]), fmaxf(sc[2], sc[6]),
+                           fmaxf(sc[3], sc[7])};
 #pragma unroll
-            for (int c = 0; c < kBlk; ++c) {
-                sc[c] = c < valid ? sc[c] : -INFINITY;
-                mq[c & 3] = fmaxf(mq[c & 3], sc[c]);
+            for (int c = 8; c < kBlk; c += 8) {
+#pragma unroll
+                for (int e = 0; e < 4; ++e) mq[e] = max3(mq[e], sc[c + e], sc[c + 4 + e]);
             }
-            const float mr = fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3])) * p.scale_log2;
+            const float mr = max3(mq[0], mq[1], fmaxf(mq[2], mq[3])) * p.scale_log2;
             // lazy rescaling: the reference max moves (and O and l are
             // rescaled) only when some row's block max exceeds it by more than
             // 8, so the weights stay below 2^8 and most blocks skip the O
             // round trip through TMEM
             const bool move = __any_sync(0xffffffffu, mr > m_run + 8.0f);
             const float mx = move ? fmaxf(m_run, mr) : m_run;
-            const float alpha = move ? exp2f(m_run - mx) : 1.0f;   // 0 on the first block
-            const float nmx = -mx;
-            float sum = 0.0f;
+            const float alpha = move ? ex2_ftz(m_run - mx) : 1.0f;   // 0 on the first block
+            const uint64_t sc2 = pack_f2(p.scale_log2, p.scale_log2);
+            const uint64_t nm2 = pack_f2(-mx, -mx);
+            // weights 2^(s * scale * log2 e - m): one paired fma per two
+            // weights, the exponential on the special-function unit, and the
+            // row sum in four paired chains
+            uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
-            for (int c = 0; c < kBlk; ++c) {
-                sc[c] = exp2f(fmaf(sc[c], p.scale_log2, nmx));
-                sum += sc[c];
+            for (int c = 0; c < kBlk; c += 2) {
+                float a, b;
+                unpack_f2(fma_f2(pack_f2(sc[c], sc[c + 1]), sc2, nm2), a, b);
+                sc[c] = ex2_ftz(a);
+                sc[c + 1] = ex2_ftz(b);
+                acc[(c >> 1) & 3] = add_f2(acc[(c >> 1) & 3], pack_f2(sc[c], sc[c + 1]));
             }
+            float s0, s1, s2, s3;
+            unpack_f2(add_f2(acc[0], acc[1]), s0, s1);
+            unpack_f2(add_f2(acc[2], acc[3]), s2, s3);
+            const float sum = (s0 + s2) + (s1 + s3);
             l_run = l_run * alpha + sum;
             m_run = mx;
             if (n >= 1 && move) {
@@ -391,6 +476,12 @@ extern "C" int dit_block_sparse_attention(const uint16_t* q, const uint16_t* k, 
     p.nb = static_cast<int>(nb);
     p.n_keep = n_keep;
     p.scale_log2 = static_cast<float>(scale * 1.4426950408889634);
+    // the register split inside the kernel assumes the launch count it was
+    // sized for; any other count could make setmaxnreg.inc wait forever
+    cudaFuncAttributes fa{};
+    if (cudaFuncGetAttributes(&fa, block_sparse_attention_kernel) != cudaSuccess ||
+        fa.numRegs != kRegsLaunch)
+        return DIT_ERR_LAUNCH;
     if (cudaFuncSetAttribute(block_sparse_attention_kernel,
                              cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(kSmemA)) != cudaSuccess)

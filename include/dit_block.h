@@ -248,6 +248,9 @@ int dit_qk_rmsnorm_rope3d_ex(uint16_t* q, uint16_t* k, int64_t row_stride,
  *                mean is an fp32 sum in a fixed order divided once by the
  *                token count, so results repeat run to run.  It is the input
  *                of dit_subblock_router_means.
+ *   status       optional device int: set to 1 if a wait of the kernel's
+ *                copy pipeline ran out (bounded at 2 s; the means of the
+ *                affected blocks are then left unwritten).  NULL: not reported.
  * q and k are both required (DIT_ERR_NULL); other arguments, errors and
  * limits as dit_qk_rmsnorm_rope3d_ex (rope_layout as there; B <= 65535).
  */
@@ -257,7 +260,7 @@ int dit_qk_rmsnorm_rope3d_pooled(uint16_t* q, uint16_t* k, int64_t row_stride,
                                  int T, int Hg, int Wg, const int32_t* pos, int64_t pos_offset,
                                  int pairs_t, int pairs_h, int pairs_w,
                                  double theta, double eps, int rope_layout, int block,
-                                 float* block_means, void* stream);
+                                 float* block_means, int* status, void* stream);
 
 /*
  * Cache-DiT residual-difference check between neighbouring denoising steps.

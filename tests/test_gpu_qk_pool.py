@@ -158,8 +158,8 @@ def test_pooled_argument_errors():
     f = L.dit_qk_rmsnorm_rope3d_pooled
     # block 0, k NULL, means overlapping q
     assert f(A, A + 256, 256, w.data_ptr(), w.data_ptr(), 0, 1, 64, 2, 64, 1, 8, 8, None, 0, 12,
-             10, 10, 1e4, 1e-6, 0, 0, m.data_ptr(), None) == -2
+             10, 10, 1e4, 1e-6, 0, 0, m.data_ptr(), None, None) == -2
     assert f(A, None, 256, w.data_ptr(), w.data_ptr(), 0, 1, 64, 2, 64, 1, 8, 8, None, 0, 12,
-             10, 10, 1e4, 1e-6, 0, 16, m.data_ptr(), None) == -1
+             10, 10, 1e4, 1e-6, 0, 16, m.data_ptr(), None, None) == -1
     assert f(A, A + 256, 256, w.data_ptr(), w.data_ptr(), 0, 1, 64, 2, 64, 1, 8, 8, None, 0, 12,
-             10, 10, 1e4, 1e-6, 0, 16, A, None) == -7
+             10, 10, 1e4, 1e-6, 0, 16, A, None, None) == -7
