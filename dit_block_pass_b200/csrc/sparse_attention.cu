@@ -9,34 +9,37 @@
 // over the tokens u of the kept key blocks of (b, h, i); non-causal; blocks
 // of 128 tokens, head size 128.
 //
-// Design: one CTA of 6 warps per (query block, head, sample), two CTAs per SM
-// (96 KB of shared memory and 256 of the 512 TMEM columns each), so that one
-// CTA's softmax runs while the other's products use the tensor cores:
-//   warp 0    TMA: the 128 x 128 Q tile once, then K and V of each kept
-//             block, one buffer each (128-byte swizzle): K_{n+1} lands while
-//             block n's softmax runs, V_{n+1} while S_{n+1} and its softmax run.
-//   warp 1    one thread issues tcgen05.mma: S_n = Q K_n^T (shared-memory
-//             operands, fp32 into TMEM columns [0, 128)) as two N = 64 halves,
-//             and, once the softmax has written P_n, O += P_n V_n with P read
-//             from TMEM (the A operand in tensor memory, two bf16 per column
-//             over S_n's first 64 columns) and V as an MN-major shared-memory
-//             operand (no transpose).  Keys 64..127 of S_{n+1} go into the
-//             columns P_n does not use as soon as the softmax has read S_n
-//             (so they run during softmax n and P_n V_n); keys 0..63 follow
-//             once P_n V_n has read P_n.
-//   warps 2-5 softmax, thread = query row (TMEM lane): keys past the
+// Design: one CTA of two warpgroups per (query block, head, sample), two
+// CTAs per SM (113 KB of shared memory and 256 of the 512 TMEM columns
+// each).  The kept keys are walked in steps of 64 (two per kept block), and
+// every stage is software pipelined so that the softmax warps never wait on
+// the tensor core in steady state:
+//   TMEM      S buffers A = columns [0, 64) and B = [64, 128) (step h uses
+//             h % 2), O = [128, 256) in fp32.  P_h, the step's weights as
+//             bf16 pairs, overwrites the first 32 columns of its S buffer.
+//   warp 0    TMA of the 128 x 128 Q tile once, then the K half-tile (64 keys
+//             x 128) of every step into a 3-slot ring.
+//   warp 2    TMA of the V half-tile of every step into a 2-slot ring.
+//   warp 1    one thread issues tcgen05.mma: S_h = Q K_h^T (N = 64) into its
+//             buffer, and, once the softmax has written P_h, O += P_h V_h
+//             (P from TMEM, V as an MN-major shared-memory operand).  S_{h+2}
+//             reuses S_h's buffer once P_h V_h has read P_h, so S_{h+1} is
+//             computed while the softmax works on step h.
+//   warps 4-7 softmax, thread = query row (TMEM lane): keys past the
 //             sample's last token are set to -inf in TMEM (only a partial
-//             block needs it), tcgen05.ld the S row (then report S_n read),
-//             the row max of the raw scores in four chains of three-input
-//             maxima, weights 2^(s * scale * log2 e - m) with one paired fma
-//             per two weights and ex2.approx, row sums in paired adds, with
-//             lazy rescaling (the reference max m moves, and O and
-//             the row sum are rescaled in TMEM, only when a row's block max
-//             exceeds m by more than 8, so weights stay below 2^8), and P
-//             written back into TMEM as bf16 pairs.  At the end O / l is
-//             written as bf16.
-// Every mbarrier wait is bounded (tcgen05.cuh); on expiry the CTA records an
-// error in the caller's status word and exits after freeing its TMEM.
+//             block needs it), tcgen05.ld the 64 scores, the row max in
+//             three-input maxima, weights 2^(s * scale * log2 e - m) with one
+//             paired fma per two weights and ex2.approx, row sums in paired
+//             adds, lazy rescaling (the reference max m moves, and O and the
+//             row sum are rescaled in TMEM after P_{h-1} V_{h-1} is done, only
+//             when a row's step max exceeds m by more than 8, so weights stay
+//             below 2^8), and P written back as bf16 pairs.  At the end
+//             O / l is written as bf16.
+// Registers are split with setmaxnreg: the copy/MMA warpgroup runs on 80
+// per thread and the softmax warpgroup on 176.  Every mbarrier wait is
+// bounded (tcgen05.cuh); on expiry the CTA records an error in the caller's
+// status word and exits after its copies and products have drained and its
+// TMEM is freed.
 #include "tcgen05.cuh"
 
 namespace dit {
@@ -44,23 +47,29 @@ namespace {
 
 using namespace tc;
 
-constexpr int kBlk = 128;                       // tokens per block (rows of every tile)
+constexpr int kBlk = 128;                       // tokens per block (rows of a Q tile)
 constexpr int kHd = 128;                        // head size
+constexpr int kStepKeys = 64;                   // keys per pipeline step
 constexpr int kThreadsA = 256;                  // two warpgroups
 // Register split (setmaxnreg): the kernel is launched with 128 registers per
 // thread (two CTAs of 256 threads fill the SM's 65,536); the copy/MMA
-// warpgroup gives up to 40 and the softmax warpgroup takes 216, which adds up
-// to the launch total: 128 * (40 + 216) = 256 * 128.
+// warpgroup gives up to 80 and the softmax warpgroup takes 176, which adds up
+// to the launch total: 128 * (80 + 176) = 256 * 128.
 constexpr int kRegsLaunch = 128;
-constexpr int kRegsLow = 56;
+constexpr int kRegsLow = 80;
 constexpr int kRegsHigh = 2 * kRegsLaunch - kRegsLow;
-constexpr uint32_t kTile = kBlk * kHd * 2;      // 32 KB: one 128 x 128 bf16 tile
-constexpr uint32_t kHalfTile = kTile / 2;       // 16 KB: 64 columns (one swizzle atom wide)
-constexpr uint32_t kTmemColsA = 256;           // two CTAs share an SM's 512 columns
-constexpr uint32_t kColO = 128;                 // S (and P over it) in [0, 128), O in [128, 256)
-// Q, K, V, then barriers
-constexpr size_t kSmemA = 3 * kTile + 1024 + 256;
-constexpr uint32_t kIdescS64 = idesc_f16(128, 64, false, false);   // half of S = Q K^T
+constexpr uint32_t kTile = kBlk * kHd * 2;      // 32 KB: the 128 x 128 bf16 Q tile
+constexpr uint32_t kHalfTile = kTile / 2;       // 16 KB: 64 keys x 128, or 128 rows x 64
+constexpr uint32_t kSub = kHalfTile / 2;        // 8 KB: 64 keys x 64 (one swizzle atom wide)
+constexpr int kKSlots = 3, kVSlots = 2;
+constexpr uint32_t kTmemColsA = 256;            // two CTAs share an SM's 512 columns
+constexpr uint32_t kColO = 128;
+constexpr uint32_t kDataBytes = kTile + (kKSlots + kVSlots) * kHalfTile;   // 112 KB
+// 1 KB for the alignment of the 128-byte swizzle atoms; the barriers live in
+// whichever part of it the alignment leaves free (113 KB per CTA, so two
+// CTAs and their reserved 1 KB each fill the SM's 228 KB)
+constexpr size_t kSmemA = kDataBytes + 1024;
+constexpr uint32_t kIdescS64 = idesc_f16(128, 64, false, false);   // S_h = Q K_h^T
 constexpr uint32_t kIdescO = idesc_f16(128, 128, false, true);     // O += P V (V MN-major)
 
 // D (TMEM) += A (TMEM, K-major: row m in lane m, two bf16 per column) * B
@@ -108,14 +117,14 @@ __device__ __forceinline__ float ex2_ftz(float x) {
     return y;
 }
 
-// -inf into columns valid .. 127 of this warp's 32 rows of S (tensor
-// memory address `row_base`): whole 32-column chunks at once, the chunk
-// holding the boundary one column at a time.
+// -inf into columns valid .. 63 of this warp's 32 rows of a step's S
+// buffer (tensor memory address `row_base`): a whole 32-column chunk at
+// once, the chunk holding the boundary one column at a time.
 __device__ __forceinline__ void mask_tail(uint32_t row_base, int valid) {
     float ninf[32];
 #pragma unroll
     for (int e = 0; e < 32; ++e) ninf[e] = -INFINITY;
-    for (int c = 0; c < kBlk / 32; ++c) {
+    for (int c = 0; c < kStepKeys / 32; ++c) {
         const int c0 = 32 * c;
         if (c0 >= valid) {
             tmem_st32(row_base + c0, ninf);
@@ -130,16 +139,28 @@ __device__ __forceinline__ void mask_tail(uint32_t row_base, int valid) {
     tmem_wait_st();
 }
 
-// Keys k0 .. k0 + 63 of S = Q K^T (k0 = 0 or 64) into TMEM columns k0 ..
-// k0 + 63: eight M = 128, N = 64, K = 16 products; rows k0.. of each 64-wide
-// K half start k0 * 128 bytes in (a multiple of the 1024-byte swizzle atom).
-__device__ __forceinline__ void issue_s(uint32_t tmem, uint32_t sQ, uint32_t sK, int k0) {
+// S_h = Q K_h^T into TMEM columns col .. col + 63: eight M = 128, N = 64,
+// K = 16 products over the head dimension.  Q is two 16 KB halves (64 of the
+// head dimension each, 128 rows); a K half-tile is two 8 KB halves (64 of
+// the head dimension each, 64 keys).
+__device__ __forceinline__ void issue_s(uint32_t tmem_col, uint32_t sQ, uint32_t sK) {
 #pragma unroll
     for (int kk = 0; kk < kHd / 16; ++kk) {
-        const uint32_t off = (kk >> 2) * kHalfTile + (kk & 3) * 32;
-        mma_f16(tmem + k0, sw128_desc(sQ + off), sw128_desc(sK + off + k0 * 128), kIdescS64,
-                kk != 0 ? 1u : 0u);
+        const uint32_t in = (kk & 3) * 32;
+        mma_f16(tmem_col, sw128_desc(sQ + (kk >> 2) * kHalfTile + in),
+                sw128_desc(sK + (kk >> 2) * kSub + in), kIdescS64, kk != 0 ? 1u : 0u);
     }
+}
+
+// O += P_h V_h: four M = 128, N = 128, K = 16 products over the step's 64
+// keys; P_h from TMEM (two bf16 per column from column p_col), V_h as an
+// MN-major operand (16 keys = 2 KB per product, the second 64 of the head
+// dimension kSub further).
+__device__ __forceinline__ void issue_pv(uint32_t tmem, uint32_t p_col, uint32_t sV, bool first) {
+#pragma unroll
+    for (int kk = 0; kk < kStepKeys / 16; ++kk)
+        mma_f16_ts(tmem + kColO, tmem + p_col + 8 * kk, sw128_desc_mn(sV + kk * 2048, kSub),
+                   kIdescO, (first && kk == 0) ? 0u : 1u);
 }
 
 struct AttnParams {
@@ -152,6 +173,14 @@ struct AttnParams {
     float scale_log2;           // scale * log2(e)
 };
 
+// Keys of step h that exist: the sample's tokens of kept block kept[h/2],
+// half h%2 (0 .. 64).
+__device__ __forceinline__ int step_valid(const int32_t* kept, int h, int64_t N) {
+    const int64_t left = N - static_cast<int64_t>(__ldg(kept + (h >> 1))) * kBlk -
+                         static_cast<int64_t>(h & 1) * kStepKeys;
+    return left >= kStepKeys ? kStepKeys : (left > 0 ? static_cast<int>(left) : 0);
+}
+
 __global__ void __launch_bounds__(kThreadsA, 2)
 block_sparse_attention_kernel(const __grid_constant__ CUtensorMap map_q,
                               const __grid_constant__ CUtensorMap map_k,
@@ -159,37 +188,46 @@ block_sparse_attention_kernel(const __grid_constant__ CUtensorMap map_q,
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
-    uint8_t* gen_base = smem_raw + (base - raw);
-    const uint32_t sQ = base, sK = base + kTile, sV = base + 2 * kTile;
-    const uint32_t bar = base + 3 * kTile;
+    const uint32_t sQ = base;
+    const uint32_t sK0 = base + kTile;                       // K slot s at sK0 + s * kHalfTile
+    const uint32_t sV0 = sK0 + kKSlots * kHalfTile;          // V slot s at sV0 + s * kHalfTile
+    // barriers and flags: before the aligned data if the alignment left
+    // room for them, else after it (the 1 KB slack holds them either way)
+    const uint32_t bar = base - raw >= 256 ? raw : base + kDataBytes;
+    uint8_t* gen_bar = smem_raw + (bar - raw);
     const uint32_t bar_q = bar;
-    const uint32_t bar_k_full = bar + 8, bar_k_empty = bar + 16;
-    const uint32_t bar_v_full = bar + 24, bar_v_empty = bar + 32;
-    const uint32_t bar_s_full = bar + 40;           // S_n in TMEM
-    const uint32_t bar_p_full = bar + 48;           // P_n in TMEM, O rescaled (4 arrivals)
-    const uint32_t bar_o_done = bar + 56;           // P_n V_n done: S/P columns and O free
-    const uint32_t bar_drain = bar + 64;
-    const uint32_t bar_s_free = bar + 72;           // S_n read into registers (4 arrivals)
-    volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(gen_base + 3 * kTile + 80);
-    volatile int* abort = reinterpret_cast<volatile int*>(gen_base + 3 * kTile + 84);
+    const uint32_t bar_k_full = bar + 8, bar_k_empty = bar + 32;     // [kKSlots]
+    const uint32_t bar_v_full = bar + 56, bar_v_empty = bar + 72;    // [kVSlots]
+    const uint32_t bar_s_full = bar + 88;                            // [2] S_h in TMEM
+    const uint32_t bar_p_full = bar + 104;                           // [2] P_h written (4 arrivals)
+    const uint32_t bar_o_done = bar + 120;                           // P_h V_h done (phase h)
+    const uint32_t bar_drain = bar + 128;
+    volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(gen_bar + 136);
+    volatile int* abort = reinterpret_cast<volatile int*>(gen_bar + 140);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int i = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
     const int nk = p.n_keep;
+    const int steps = 2 * nk;
     const int32_t* kept = p.kept + ((static_cast<int64_t>(b) * p.H + h) * p.nb + i) * nk;
     const int row0 = static_cast<int>(static_cast<int64_t>(b) * p.N);   // first row of the sample
 
     if (threadIdx.x == 0) {
         mbar_init(bar_q, 1);
-        mbar_init(bar_k_full, 1);
-        mbar_init(bar_k_empty, 1);
-        mbar_init(bar_v_full, 1);
-        mbar_init(bar_v_empty, 1);
-        mbar_init(bar_s_full, 1);
-        mbar_init(bar_p_full, 4);
+        for (int s = 0; s < kKSlots; ++s) {
+            mbar_init(bar_k_full + 8 * s, 1);
+            mbar_init(bar_k_empty + 8 * s, 1);
+        }
+        for (int s = 0; s < kVSlots; ++s) {
+            mbar_init(bar_v_full + 8 * s, 1);
+            mbar_init(bar_v_empty + 8 * s, 1);
+        }
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(bar_s_full + 8 * s, 1);
+            mbar_init(bar_p_full + 8 * s, 4);
+        }
         mbar_init(bar_o_done, 1);
         mbar_init(bar_drain, 1);
-        mbar_init(bar_s_free, 4);
         *abort = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
@@ -201,99 +239,97 @@ block_sparse_attention_kernel(const __grid_constant__ CUtensorMap map_q,
     bool failed = false;
 
     if (warp < 4) {
-    // copy and MMA warpgroup (warps 2 and 3 only wait at the end)
+    // copy and MMA warpgroup (warp 3 only waits at the end)
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsLow));
+    const int col = h * kHd;
     if (warp == 0) {
         if (lane == 0) {
-            // the Q tile, then K and V of every kept block (one buffer each:
-            // K_{n+1} lands while the softmax of block n runs, V_{n+1} while
-            // S_{n+1} and its softmax run)
-            const int col = h * kHd;
+            // Q once, then the K half-tile of every step into the 3-slot ring
             mbar_expect_tx(bar_q, kTile);
             tma_load_2d(sQ, &map_q, bar_q, col, row0 + i * kBlk);
             tma_load_2d(sQ + kHalfTile, &map_q, bar_q, col + 64, row0 + i * kBlk);
-            int issued_k = 0, issued_v = 0;
-            for (int n = 0; n < nk; ++n) {
-                const int row = row0 + __ldg(kept + n) * kBlk;
-                if (!mbar_wait(bar_k_empty, (n & 1) ^ 1, abort)) {
+            int issued = 0;
+            for (int st = 0; st < steps; ++st) {
+                const int s = st % kKSlots;
+                if (!mbar_wait(bar_k_empty + 8 * s, ((st / kKSlots) & 1) ^ 1, abort)) {
                     failed = true;
                     break;
                 }
-                mbar_expect_tx(bar_k_full, kTile);
-                tma_load_2d(sK, &map_k, bar_k_full, col, row);
-                tma_load_2d(sK + kHalfTile, &map_k, bar_k_full, col + 64, row);
-                issued_k = n + 1;
-                if (!mbar_wait(bar_v_empty, (n & 1) ^ 1, abort)) {
-                    failed = true;
-                    break;
-                }
-                mbar_expect_tx(bar_v_full, kTile);
-                tma_load_2d(sV, &map_v, bar_v_full, col, row);
-                tma_load_2d(sV + kHalfTile, &map_v, bar_v_full, col + 64, row);
-                issued_v = n + 1;
+                const int row = row0 + __ldg(kept + (st >> 1)) * kBlk + (st & 1) * kStepKeys;
+                const uint32_t dst = sK0 + s * kHalfTile;
+                mbar_expect_tx(bar_k_full + 8 * s, kHalfTile);
+                tma_load_2d(dst, &map_k, bar_k_full + 8 * s, col, row);
+                tma_load_2d(dst + kSub, &map_k, bar_k_full + 8 * s, col + 64, row);
+                issued = st + 1;
             }
             mbar_wait_drain(bar_q, 0);           // the Q copy lands before the CTA exits
             if (failed) {
-                if (issued_k) mbar_wait_drain(bar_k_full, (issued_k - 1) & 1);
-                if (issued_v) mbar_wait_drain(bar_v_full, (issued_v - 1) & 1);
+                for (int st = issued - kKSlots > 0 ? issued - kKSlots : 0; st < issued; ++st)
+                    mbar_wait_drain(bar_k_full + 8 * (st % kKSlots), (st / kKSlots) & 1);
+            }
+        }
+        __syncwarp();
+    } else if (warp == 2) {
+        if (lane == 0) {
+            // the V half-tile of every step into the 2-slot ring
+            int issued = 0;
+            for (int st = 0; st < steps; ++st) {
+                const int s = st % kVSlots;
+                if (!mbar_wait(bar_v_empty + 8 * s, ((st / kVSlots) & 1) ^ 1, abort)) {
+                    failed = true;
+                    break;
+                }
+                const int row = row0 + __ldg(kept + (st >> 1)) * kBlk + (st & 1) * kStepKeys;
+                const uint32_t dst = sV0 + s * kHalfTile;
+                mbar_expect_tx(bar_v_full + 8 * s, kHalfTile);
+                tma_load_2d(dst, &map_v, bar_v_full + 8 * s, col, row);
+                tma_load_2d(dst + kSub, &map_v, bar_v_full + 8 * s, col + 64, row);
+                issued = st + 1;
+            }
+            if (failed) {
+                for (int st = issued - kVSlots > 0 ? issued - kVSlots : 0; st < issued; ++st)
+                    mbar_wait_drain(bar_v_full + 8 * (st % kVSlots), (st / kVSlots) & 1);
             }
         }
         __syncwarp();
     } else if (warp == 1) {
         if (lane == 0) {
             if (!mbar_wait(bar_q, 0, abort)) failed = true;
-            // S_0, both key halves
-            if (!failed && nk > 0) {
-                if (!mbar_wait(bar_k_full, 0, abort)) {
-                    failed = true;
-                } else {
-                    fence_after_sync();
-                    issue_s(tmem, sQ, sK, 64);
-                    issue_s(tmem, sQ, sK, 0);
-                    mma_commit(bar_s_full);
-                    mma_commit(bar_k_empty);
-                }
-            }
-            for (int n = 0; n < nk && !failed; ++n) {
-                const bool more = n + 1 < nk;
-                // keys 64..127 of S_{n+1} (columns P_n does not use) once the
-                // softmax has read S_n and K_{n+1} is in, and P_n V_n once P_n
-                // is written: whichever is ready first
-                bool b_done = !more, pv_done = false;
-                const unsigned long long t0 = now_ns();
-                for (uint32_t it = 0; !(b_done && pv_done); ++it) {
-                    if (!b_done && mbar_try(bar_s_free, n & 1) &&
-                        mbar_try(bar_k_full, (n + 1) & 1)) {
-                        fence_after_sync();
-                        issue_s(tmem, sQ, sK, 64);
-                        b_done = true;
-                    }
-                    if (!pv_done && mbar_try(bar_p_full, n & 1) && mbar_try(bar_v_full, n & 1)) {
-                        fence_after_sync();
-#pragma unroll
-                        for (int kk = 0; kk < kBlk / 16; ++kk)
-                            mma_f16_ts(tmem + kColO, tmem + 8 * kk,
-                                       sw128_desc_mn(sV + kk * 2048, kHalfTile), kIdescO,
-                                       (n | kk) != 0 ? 1u : 0u);
-                        mma_commit(bar_o_done);
-                        mma_commit(bar_v_empty);
-                        pv_done = true;
-                    }
-                    if ((it & 255u) == 255u && (*abort || now_ns() - t0 > kWaitNs)) {
-                        failed = true;
-                        break;
-                    }
-                }
-                if (failed || !more) continue;
-                // keys 0..63 of S_{n+1} overwrite P_n: after P_n V_n has read it
-                if (!mbar_wait(bar_o_done, n & 1, abort)) {
+            // S_0 and S_1 into buffers A and B
+            for (int st = 0; st < 2 && st < steps && !failed; ++st) {
+                if (!mbar_wait(bar_k_full + 8 * st, 0, abort)) {
                     failed = true;
                     break;
                 }
                 fence_after_sync();
-                issue_s(tmem, sQ, sK, 0);
-                mma_commit(bar_s_full);
-                mma_commit(bar_k_empty);
+                issue_s(tmem + kStepKeys * st, sQ, sK0 + st * kHalfTile);
+                mma_commit(bar_s_full + 8 * st);
+                mma_commit(bar_k_empty + 8 * st);
+            }
+            for (int st = 0; st < steps && !failed; ++st) {
+                const int x = st & 1;
+                // P_h V_h once the softmax has written P_h and V_h is in
+                if (!mbar_wait(bar_p_full + 8 * x, (st >> 1) & 1, abort) ||
+                    !mbar_wait(bar_v_full + 8 * (st % kVSlots), (st / kVSlots) & 1, abort)) {
+                    failed = true;
+                    break;
+                }
+                fence_after_sync();
+                issue_pv(tmem, kStepKeys * x, sV0 + (st % kVSlots) * kHalfTile, st == 0);
+                mma_commit(bar_o_done);
+                mma_commit(bar_v_empty + 8 * (st % kVSlots));
+                // S_{h+2} reuses this buffer: after P_h V_h has read P_h
+                const int nx = st + 2;
+                if (nx >= steps) continue;
+                if (!mbar_wait(bar_o_done, st & 1, abort) ||
+                    !mbar_wait(bar_k_full + 8 * (nx % kKSlots), (nx / kKSlots) & 1, abort)) {
+                    failed = true;
+                    break;
+                }
+                fence_after_sync();
+                issue_s(tmem + kStepKeys * x, sQ, sK0 + (nx % kKSlots) * kHalfTile);
+                mma_commit(bar_s_full + 8 * x);
+                mma_commit(bar_k_empty + 8 * (nx % kKSlots));
             }
             if (failed) {
                 mma_commit(bar_drain);
@@ -309,47 +345,42 @@ block_sparse_attention_kernel(const __grid_constant__ CUtensorMap map_q,
         const int r = 32 * q + lane;
         const uint32_t lane_off = static_cast<uint32_t>(32 * q) << 16;
         float m_run = -INFINITY, l_run = 0.0f;
-        for (int n = 0; n < nk; ++n) {
+        for (int st = 0; st < steps; ++st) {
+            const int x = st & 1;
+            const uint32_t sbuf = tmem + lane_off + kStepKeys * x;
             // keys past the sample's last token do not take part
-            const int64_t j = __ldg(kept + n);
-            const int64_t left = p.N - j * kBlk;
-            const int valid = left >= kBlk ? kBlk : (left > 0 ? static_cast<int>(left) : 0);
-            if (!__all_sync(0xffffffffu, mbar_wait(bar_s_full, n & 1, abort))) {
+            const int valid = step_valid(kept, st, p.N);
+            if (!__all_sync(0xffffffffu, mbar_wait(bar_s_full + 8 * x, (st >> 1) & 1, abort))) {
                 failed = true;
                 break;
             }
             fence_after_sync();
-            // a sample's last block may be partial: its missing keys' scores
-            // become -inf in tensor memory (the same block for every row, so
-            // the branch is uniform), and full blocks need no mask at all
-            if (valid < kBlk) mask_tail(tmem + lane_off, valid);
-            float sc[kBlk];
-#pragma unroll
-            for (int c = 0; c < kBlk / 32; ++c)
-                tmem_ld32(tmem + lane_off + 32 * c, *reinterpret_cast<float(*)[32]>(sc + 32 * c));
+            // a partial step's missing keys become -inf in tensor memory (the
+            // same for every row, so the branch is uniform); full steps need
+            // no mask at all
+            if (valid < kStepKeys) mask_tail(sbuf, valid);
+            float sc[kStepKeys];
+            tmem_ld32(sbuf, *reinterpret_cast<float(*)[32]>(sc));
+            tmem_ld32(sbuf + 32, *reinterpret_cast<float(*)[32]>(sc + 32));
             tmem_wait_ld();
-            // S_n is in registers: its columns 64..127 may take S_{n+1}
-            fence_before_sync();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bar_s_free);
             // the row max of the raw scores (scale > 0 and rounding is monotonic,
             // so scaling the max equals the max of the scaled scores), in four
             // independent chains of three-input maxima
             float mq[4] = {fmaxf(sc[0], sc[4]), fmaxf(sc[1], sc[5]), fmaxf(sc[2], sc[6]),
                            fmaxf(sc[3], sc[7])};
 #pragma unroll
-            for (int c = 8; c < kBlk; c += 8) {
+            for (int c = 8; c < kStepKeys; c += 8) {
 #pragma unroll
                 for (int e = 0; e < 4; ++e) mq[e] = max3(mq[e], sc[c + e], sc[c + 4 + e]);
             }
             const float mr = max3(mq[0], mq[1], fmaxf(mq[2], mq[3])) * p.scale_log2;
             // lazy rescaling: the reference max moves (and O and l are
-            // rescaled) only when some row's block max exceeds it by more than
-            // 8, so the weights stay below 2^8 and most blocks skip the O
+            // rescaled) only when some row's step max exceeds it by more than
+            // 8, so the weights stay below 2^8 and most steps skip the O
             // round trip through TMEM
             const bool move = __any_sync(0xffffffffu, mr > m_run + 8.0f);
             const float mx = move ? fmaxf(m_run, mr) : m_run;
-            const float alpha = move ? ex2_ftz(m_run - mx) : 1.0f;   // 0 on the first block
+            const float alpha = move ? ex2_ftz(m_run - mx) : 1.0f;   // 0 on the first step
             const uint64_t sc2 = pack_f2(p.scale_log2, p.scale_log2);
             const uint64_t nm2 = pack_f2(-mx, -mx);
             // weights 2^(s * scale * log2 e - m): one paired fma per two
@@ -357,11 +388,11 @@ block_sparse_attention_kernel(const __grid_constant__ CUtensorMap map_q,
             // row sum in four paired chains
             uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
-            for (int c = 0; c < kBlk; c += 2) {
-                float a, b;
-                unpack_f2(fma_f2(pack_f2(sc[c], sc[c + 1]), sc2, nm2), a, b);
+            for (int c = 0; c < kStepKeys; c += 2) {
+                float a, bb;
+                unpack_f2(fma_f2(pack_f2(sc[c], sc[c + 1]), sc2, nm2), a, bb);
                 sc[c] = ex2_ftz(a);
-                sc[c + 1] = ex2_ftz(b);
+                sc[c + 1] = ex2_ftz(bb);
                 acc[(c >> 1) & 3] = add_f2(acc[(c >> 1) & 3], pack_f2(sc[c], sc[c + 1]));
             }
             float s0, s1, s2, s3;
@@ -370,9 +401,14 @@ block_sparse_attention_kernel(const __grid_constant__ CUtensorMap map_q,
             const float sum = (s0 + s2) + (s1 + s3);
             l_run = l_run * alpha + sum;
             m_run = mx;
-            if (n >= 1 && move) {
-                // P_{n-1} V_{n-1} is done (S_n was issued after it), so O holds
-                // the sum so far
+            if (st >= 1 && move) {
+                // O holds the sum up to step h-1 once P_{h-1} V_{h-1} is done
+                // (P_h is not written yet, so that is the latest product)
+                if (!__all_sync(0xffffffffu, mbar_wait(bar_o_done, (st - 1) & 1, abort))) {
+                    failed = true;
+                    break;
+                }
+                fence_after_sync();
 #pragma unroll 1
                 for (int c = 0; c < kHd / 32; ++c) {
                     float o[32];
@@ -383,22 +419,21 @@ block_sparse_attention_kernel(const __grid_constant__ CUtensorMap map_q,
                     tmem_st32(tmem + lane_off + kColO + 32 * c, o);
                 }
             }
-            // P_n as bf16 pairs over S_n's first 64 columns (row r in lane r)
-#pragma unroll
-            for (int c = 0; c < 2; ++c) {
+            // P_h as bf16 pairs over the buffer's first 32 columns (row r in lane r)
+            {
                 float w[32];
 #pragma unroll
                 for (int e = 0; e < 32; ++e)
-                    w[e] = __uint_as_float(pack2(sc[64 * c + 2 * e], sc[64 * c + 2 * e + 1]));
-                tmem_st32(tmem + lane_off + 32 * c, w);
+                    w[e] = __uint_as_float(pack2(sc[2 * e], sc[2 * e + 1]));
+                tmem_st32(sbuf, w);
             }
             tmem_wait_st();
             fence_before_sync();
             __syncwarp();
-            if (lane == 0) mbar_arrive(bar_p_full);
+            if (lane == 0) mbar_arrive(bar_p_full + 8 * x);
         }
-        if (!failed && nk > 0) {
-            if (!__all_sync(0xffffffffu, mbar_wait(bar_o_done, (nk - 1) & 1, abort))) {
+        if (!failed && steps > 0) {
+            if (!__all_sync(0xffffffffu, mbar_wait(bar_o_done, (steps - 1) & 1, abort))) {
                 failed = true;
             } else {
                 fence_after_sync();
@@ -463,8 +498,9 @@ extern "C" int dit_block_sparse_attention(const uint16_t* q, const uint16_t* k, 
     if (overlaps(out, ob, q, ib) || overlaps(out, ob, k, ib) || overlaps(out, ob, v, ib))
         return DIT_ERR_OVERLAP;
     CUtensorMap mq, mk, mv;
-    if (!make_map(&mq, q, rows, D, row_stride) || !make_map(&mk, k, rows, D, row_stride) ||
-        !make_map(&mv, v, rows, D, row_stride))
+    if (!make_map(&mq, q, rows, D, row_stride) ||
+        !make_map(&mk, k, rows, D, row_stride, kStepKeys) ||
+        !make_map(&mv, v, rows, D, row_stride, kStepKeys))
         return DIT_ERR_LAUNCH;
     AttnParams p{};
     p.kept = kept;

@@ -223,16 +223,15 @@ inline EncodeTiled encoder() {
     return fn;
 }
 
-// A [rows, K] bf16 row-major operand read in 64 x 128 boxes, 128-byte swizzle.
 // A bf16 row-major operand [rows, cols] (row_stride elements apart) read in
-// 64 x 128 boxes (64 along the row, 128 rows), 128-byte swizzle, zero fill.
+// 64 x box_rows boxes (64 along the row), 128-byte swizzle, zero fill.
 inline bool make_map(CUtensorMap* map, const void* base, int64_t rows, int64_t cols,
-                     int64_t row_stride) {
+                     int64_t row_stride, uint32_t box_rows = 128) {
     const EncodeTiled enc = encoder();
     if (!enc) return false;
     const cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
     const cuuint64_t strides[1] = {static_cast<cuuint64_t>(row_stride) * 2};
-    const cuuint32_t box[2] = {64, 128};
+    const cuuint32_t box[2] = {64, box_rows};
     const cuuint32_t elem[2] = {1, 1};
     return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
                box, elem, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
