@@ -50,7 +50,18 @@ DOMINANT = "swiglu"
 # only while its kernel source is unchanged (hash of the .cu file without
 # comments and blank space); it is reported as null otherwise.
 NCU_SLICE_TOKENS = 32256
-NCU_TRAFFIC = {}
+NCU_TRAFFIC = {
+    "adaln_modulate": {"file": "adaln.cu", "sha": "92e8ba1a144a009a",
+                       "bytes_per_token": 606011392 / NCU_SLICE_TOKENS},
+    "qk_rmsnorm_rope3d": {"file": "qk_rope.cu", "sha": "7956bd20f689261b",
+                          "bytes_per_token": 1263253248 / NCU_SLICE_TOKENS},
+    "gated_residual_adaln": {"file": "adaln.cu", "sha": "92e8ba1a144a009a",
+                             "bytes_per_token": 1265638912 / NCU_SLICE_TOKENS},
+    "swiglu": {"file": "swiglu.cu", "sha": "a9e07b0f774729cf",
+               "bytes_per_token": 2620489264 / NCU_SLICE_TOKENS},
+    "cachedit_residual_diff": {"file": "cachedit.cu", "sha": "9a1487d46a877c49",
+                               "bytes_per_token": 665030400 / NCU_SLICE_TOKENS},
+}
 
 
 def algorithmic_bytes(wl) -> dict:
