@@ -23,8 +23,9 @@
 //   warp 1    one thread issues tcgen05.mma: S_h = Q K_h^T (N = 64) into its
 //             buffer, and, once the softmax has written P_h, O += P_h V_h
 //             (P from TMEM, V as an MN-major shared-memory operand).  S_{h+2}
-//             reuses S_h's buffer once P_h V_h has read P_h, so S_{h+1} is
-//             computed while the softmax works on step h.
+//             reuses S_h's buffer: it is issued right after P_h V_h, which
+//             the tensor core runs first, so S_{h+1} and S_{h+2} are computed
+//             while the softmax works on steps h and h+1.
 //   warps 4-7 softmax, thread = query row (TMEM lane): keys past the
 //             sample's last token are set to -inf in TMEM (only a partial
 //             block needs it), tcgen05.ld the 64 scores, the row max in
@@ -318,11 +319,14 @@ block_sparse_attention_kernel(const __grid_constant__ CUtensorMap map_q,
                 issue_pv(tmem, kStepKeys * x, sV0 + (st % kVSlots) * kHalfTile, st == 0);
                 mma_commit(bar_o_done);
                 mma_commit(bar_v_empty + 8 * (st % kVSlots));
-                // S_{h+2} reuses this buffer: after P_h V_h has read P_h
+                // S_{h+2} reuses this buffer.  The products this thread issues
+                // run on the tensor core in issue order, so S_{h+2} writes the
+                // buffer after P_h V_h has read P_h from it; waiting for
+                // P_h V_h to complete first gave bit-identical outputs and
+                // cost 6 % at h3_5s
                 const int nx = st + 2;
                 if (nx >= steps) continue;
-                if (!mbar_wait(bar_o_done, st & 1, abort) ||
-                    !mbar_wait(bar_k_full + 8 * (nx % kKSlots), (nx / kKSlots) & 1, abort)) {
+                if (!mbar_wait(bar_k_full + 8 * (nx % kKSlots), (nx / kKSlots) & 1, abort)) {
                     failed = true;
                     break;
                 }
