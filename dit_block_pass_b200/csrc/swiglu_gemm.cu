@@ -29,9 +29,10 @@
 //            thread (thread = output row): gate and the matching linear
 //            columns -> silu(g) * u, or output columns -> x + gate * acc
 //            (gate rows read 16 bytes at a time when aligned); one rounding
-//            to bf16, 64-byte row segments to HBM.  Once the last columns
-//            are in registers the accumulators go back to the MMA warp; the
-//            producer has meanwhile filled the ring for the next tile.
+//            to bf16, 64-byte row segments to HBM.  Each 128-row half goes
+//            back to the MMA warp once its last columns are in registers
+//            (half 0 first), so the next tile's first K steps run on half 0
+//            while half 1 drains; the producer has meanwhile filled the ring.
 // Tiles are numbered in groups of 8 row tiles (column tiles outer within a
 // group) so that the tiles in flight share their x and W tiles in L2.  x, W
 // tiles beyond M, K or F are zero-filled by TMA; stores past M or F are
@@ -147,9 +148,10 @@ __device__ __forceinline__ uint32_t resid_pair(uint32_t xw, float g0, float a0, 
     return pack2(s0, s1);
 }
 
-// Persistent: CTA b takes tiles b, b + gridDim.x, ...  The K-step ring and
-// the two accumulators (TMEM columns [0, 256) and [256, 512)) run across
-// tiles, so the epilogue of one tile overlaps the main loop of the next.
+// Persistent: CTA b takes tiles b, b + gridDim.x, ...  The K-step ring runs
+// across tiles, and the two accumulator halves (TMEM columns [0, 256) and
+// [256, 512)) are released separately, so the epilogue of one tile overlaps
+// the first K steps of the next.
 template <int EPI>
 __global__ void __launch_bounds__(kThreadsG, 1)
 gemm_kernel(const __grid_constant__ CUtensorMap map_x,
@@ -163,7 +165,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap map_x,
     const uint32_t bar_full = base + kStages * kStageBytes;      // kStages x 8 bytes
     const uint32_t bar_empty = bar_full + 8 * kStages;           // kStages x 8 bytes
     const uint32_t bar_tfull = bar_empty + 8 * kStages;          // 2 x 8: accumulator ready
-    const uint32_t bar_tempty = bar_tfull + 16;                  // 2 x 8: accumulator drained
+    const uint32_t bar_tempty = bar_tfull + 16;                  // 2 x 8: half h drained
     const uint32_t bar_drain = bar_tempty + 16;
     uint8_t* tail = gen_base + kStages * kStageBytes + 16 * kStages + 40;
     volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(tail);
@@ -177,10 +179,9 @@ gemm_kernel(const __grid_constant__ CUtensorMap map_x,
             mbar_init(bar_full + 8 * s, 1);
             mbar_init(bar_empty + 8 * s, 1);
         }
-        for (uint32_t a = 0; a < kAccBufs; ++a) {
-            mbar_init(bar_tfull + 8 * a, 1);
-            mbar_init(bar_tempty + 8 * a, kEpiWarps);   // one arrival per epilogue warp
-        }
+        for (uint32_t a = 0; a < kAccBufs; ++a) mbar_init(bar_tfull + 8 * a, 1);
+        for (int h = 0; h < kHalves; ++h)
+            mbar_init(bar_tempty + 8 * h, kEpiWarps);   // one arrival per epilogue warp
         mbar_init(bar_drain, 1);
         *abort = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -232,18 +233,32 @@ gemm_kernel(const __grid_constant__ CUtensorMap map_x,
         __syncwarp();
     } else if (warp == 1) {
         if (lane == 0) {
-            // MMA issuer
+            // MMA issuer.  The accumulator holds both 128-row halves of a tile
+            // (all 512 columns); the epilogue releases each half on its own
+            // barrier, half 0 first.  A tile starts once half 0 is free: its
+            // first K steps issue half 0's products only and keep their ring
+            // stages until half 1 is free too (at most kStages of them), then
+            // half 1 catches up in K order, so the epilogue of the previous
+            // tile overlaps the start of this one.
             uint32_t it = 0, local = 0;
             for (int t = blockIdx.x; t < p.tiles && !failed; t += gridDim.x, ++local) {
-                const uint32_t acc = local % kAccBufs;
-                const uint32_t aph = (local / kAccBufs) & 1u;
-                // the epilogue has drained this accumulator (the first use passes)
-                if (!mbar_wait(bar_tempty + 8 * acc, aph ^ 1u, abort)) {
+                const uint32_t free_ph = (local & 1u) ^ 1u;    // the first tile passes
+                if (!mbar_wait(bar_tempty, free_ph, abort)) {
                     failed = true;
                     break;
                 }
                 fence_after_sync();
-                const uint32_t d = tmem + acc * kAccCols;
+                bool h1 = mbar_test(bar_tempty + 8, free_ph);
+                if (h1) fence_after_sync();
+                const uint32_t it0 = it;
+                int pend = 0;                   // first K step whose half-1 products are not issued
+                auto issue_half = [&](int kb, int h) {
+                    const uint32_t sa = base + ((it0 + kb) % kStages) * kStageBytes;
+#pragma unroll
+                    for (int kk = 0; kk < kBK / 16; ++kk)
+                        mma_bf16(tmem + 256u * h, sw128_desc(sa + h * (kTileA / kHalves) + kk * 32),
+                                 sw128_desc(sa + kTileA + kk * 32), (kb | kk) != 0 ? 1u : 0u);
+                };
                 for (int kb = 0; kb < nk; ++kb, ++it) {
                     const uint32_t s = it % kStages;
                     const uint32_t ph = (it / kStages) & 1u;
@@ -252,17 +267,39 @@ gemm_kernel(const __grid_constant__ CUtensorMap map_x,
                         break;
                     }
                     fence_after_sync();
-                    const uint32_t sa = base + s * kStageBytes;
-                    const uint32_t sb = sa + kTileA;
-#pragma unroll
-                    for (int kk = 0; kk < kBK / 16; ++kk)
-#pragma unroll
-                        for (int h = 0; h < kHalves; ++h)
-                            mma_bf16(d + 256u * h, sw128_desc(sa + h * (kTileA / kHalves) + kk * 32),
-                                     sw128_desc(sb + kk * 32), (kb | kk) != 0 ? 1u : 0u);
-                    mma_commit(bar_empty + 8 * s);  // stage free once these MMAs read it
+                    issue_half(kb, 0);
+                    if (!h1) {
+                        h1 = mbar_test(bar_tempty + 8, free_ph);
+                        // every ring stage is held: half 1 must be free before the next step
+                        if (!h1 && kb + 1 - pend >= kStages) {
+                            if (!mbar_wait(bar_tempty + 8, free_ph, abort)) {
+                                failed = true;
+                                break;
+                            }
+                            h1 = true;
+                        }
+                        if (h1) fence_after_sync();
+                    }
+                    if (h1) {
+                        for (; pend <= kb; ++pend) {
+                            issue_half(pend, 1);
+                            // stage free once both halves' products have read it
+                            mma_commit(bar_empty + 8 * ((it0 + pend) % kStages));
+                        }
+                    }
                 }
-                if (!failed) mma_commit(bar_tfull + 8 * acc);
+                if (!failed && pend < nk) {
+                    if (!mbar_wait(bar_tempty + 8, free_ph, abort)) {
+                        failed = true;
+                    } else {
+                        fence_after_sync();
+                        for (; pend < nk; ++pend) {
+                            issue_half(pend, 1);
+                            mma_commit(bar_empty + 8 * ((it0 + pend) % kStages));
+                        }
+                    }
+                }
+                if (!failed) mma_commit(bar_tfull);
             }
             if (failed) {
                 // every MMA issued has finished when this commit arrives
@@ -299,13 +336,13 @@ gemm_kernel(const __grid_constant__ CUtensorMap map_x,
                 tmem_ld32(lane_addr + 32 * c, g);
                 if (EPI == kSwiGLU) tmem_ld32(lane_addr + kBN + 32 * c, u);
                 tmem_wait_ld();
-                if (hc == kHalves * kPer - 1) {
-                    // every column of this accumulator is in registers: hand it back
+                if (hc % kPer == kPer - 1) {
+                    // this half's columns are all in registers: hand it back
                     fence_before_sync();
                     __syncwarp();
                     if (lane == 0)
                         asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(
-                                         bar_tempty + 8 * acc)
+                                         bar_tempty + 8 * h)
                                      : "memory");
                 }
                 if (row < p.M) {
