@@ -272,6 +272,19 @@ def dist_setup(args):
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world == 1 and args.shard:
+        # one rank: the sharded path still runs its all-gather, over a group of one
+        import datetime
+        import socket
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        with socket.socket() as sk:
+            sk.bind(("127.0.0.1", 0))
+            port = sk.getsockname()[1]
+        dist.init_process_group("nccl", init_method=f"tcp://127.0.0.1:{port}", rank=0,
+                                world_size=1, timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device(f"cuda:{local}"))
+        return world, rank, local
     if world > 1:
         import datetime
         import torch.distributed as dist
@@ -1097,8 +1110,8 @@ def main():
             "gpu_launches": launches, "clocks": clocks,
         }
         print(json.dumps(line), flush=True)
-    if world > 1:
-        import torch.distributed as dist
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized():
         dist.barrier()
         dist.destroy_process_group()
 
