@@ -451,6 +451,31 @@ def time_cache_step(chain, steps, warmup, world):
     return out
 
 
+def time_alternating(ops: dict, steps: int, warmup: int, world: int, rounds: int = 4) -> dict:
+    """ms per launch of each op, timed in `rounds` alternating rounds (every
+    op once per round, in order) of max(1, steps // rounds) launches each,
+    the median over rounds: ops that run at the power cap are compared under
+    the same power and thermal state rather than one after the other."""
+    import torch
+    stream = torch.cuda.current_stream()
+    per = max(1, steps // rounds)
+    for op in ops.values():
+        for _ in range(warmup):
+            op()
+    times = {name: [] for name in ops}
+    for _ in range(rounds):
+        for name, op in ops.items():
+            barrier_sync(world)
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            for _ in range(per):
+                op()
+            b.record(stream)
+            barrier_sync(world)
+            times[name].append(a.elapsed_time(b) / per)
+    return {name: max_over_ranks(statistics.median(t), world) for name, t in times.items()}
+
+
 def time_swiglu_gemm(chain, steps, warmup, world):
     """The up-projection with SwiGLU fused into its epilogue (tcgen05) on the
     clip's normalised tokens, against the unfused chain it replaces: cuBLAS's
@@ -467,19 +492,7 @@ def time_swiglu_gemm(chain, steps, warmup, world):
     st = torch.zeros(1, dtype=torch.int32, device=c.dev)
     ops = {"fused": lambda: dbp.swiglu_gemm(x, w, out=c.out, status=st),
            "unfused": lambda: (torch.matmul(x, w.T, out=y), dbp.swiglu(y, out=c.out))}
-    stream = torch.cuda.current_stream()
-    out = {}
-    for name, op in ops.items():
-        for _ in range(warmup):
-            op()
-        barrier_sync(world)
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record(stream)
-        for _ in range(steps):
-            op()
-        b.record(stream)
-        barrier_sync(world)
-        out[name] = a.elapsed_time(b) / steps
+    out = time_alternating(ops, steps, warmup, world)
     if int(st.item()) != 0:
         raise RuntimeError("swiglu_gemm reported an expired pipeline wait")
     del w
@@ -512,19 +525,7 @@ def time_gemm_residual(chain, steps, warmup, world):
                                   dbp.gated_residual_adaln(c.x, branch, m[:, 2], m[:, 3], m[:, 4],
                                                            wl.eps, x_out=c.xo, y=c.y2)),
     }
-    stream = torch.cuda.current_stream()
-    out = {}
-    for name, op in ops.items():
-        for _ in range(warmup):
-            op()
-        barrier_sync(world)
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record(stream)
-        for _ in range(steps):
-            op()
-        b.record(stream)
-        barrier_sync(world)
-        out[name] = max_over_ranks(a.elapsed_time(b) / steps, world)
+    out = time_alternating(ops, steps, warmup, world)
     if int(st.item()) != 0:
         raise RuntimeError("gemm_gated_residual reported an expired pipeline wait")
     del w, branch
@@ -977,7 +978,7 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--attn-steps", type=int, default=3,
                     help="timed launches of the block-sparse attention and of dense attention")
-    ap.add_argument("--gemm-steps", type=int, default=10,
+    ap.add_argument("--gemm-steps", type=int, default=12,
                     help="timed launches of the fused GEMMs and of their unfused chains")
     ap.add_argument("--no-extras", action="store_true",
                     help="time the chain only (no option, GEMM, router or attention rows)")

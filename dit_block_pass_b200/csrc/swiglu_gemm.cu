@@ -33,7 +33,7 @@
 //            back to the MMA warp once its last columns are in registers
 //            (half 0 first), so the next tile's first K steps run on half 0
 //            while half 1 drains; the producer has meanwhile filled the ring.
-// Tiles are numbered in groups of 8 row tiles (column tiles outer within a
+// Tiles are numbered in groups of row tiles (column tiles outer within a
 // group) so that the tiles in flight share their x and W tiles in L2.  x, W
 // tiles beyond M, K or F are zero-filled by TMA; stores past M or F are
 // skipped.  The SwiGLU form runs at the sustained tensor peak of B200 (raster
@@ -57,7 +57,17 @@ constexpr int kBK = 64;                     // K per stage: one 128-byte swizzle
 constexpr int kStages = kHalves == 2 ? 3 : 4;
 constexpr int kEpiWarps = 8;
 constexpr int kThreadsG = 64 + 32 * kEpiWarps;
-constexpr int kGroupM = 16 / kHalves;       // raster group (row tiles)
+// Raster groups (row tiles whose column tiles run together so that the tiles
+// in flight share their x and W tiles in L2), measured at the H3 shapes:
+// SwiGLU [124992, 5120] x [27648, 5120]^T best at 8-12 (16 and more thrash L2:
+// 32 cost 12 %, 64 cost 24 %), the down-projection [124992, 13824] x
+// [5120, 13824]^T best at 4-5 (8: +2-4 %, 16: +8 %).  Outputs do not depend on it.
+#ifndef GEMM_GROUP_SWIGLU
+#define GEMM_GROUP_SWIGLU 12
+#endif
+#ifndef GEMM_GROUP_RESID
+#define GEMM_GROUP_RESID 5
+#endif
 constexpr uint32_t kTileA = kBM * kBK * 2;            // 16 KB per 128 rows
 constexpr uint32_t kTileB = 2 * kBN * kBK * 2;        // 32 KB (gate + linear)
 constexpr uint32_t kStageBytes = kTileA + kTileB;
@@ -93,6 +103,7 @@ struct GemmParams {
     int M, K;
     int cols;               // output columns (F, or D)
     int tiles_m, tiles_n, tiles;
+    int group_m;            // raster group: row tiles whose column tiles run together
     int b1_offset;          // row of the second W box relative to the first (0: own map)
     int stall;              // test hook: the producer issues nothing, every wait runs out
     // gated residual
@@ -109,10 +120,10 @@ struct GemmParams {
 // their x and W tiles in L2.
 template <int EPI>
 __device__ __forceinline__ void tile_coords(const GemmParams& p, int t, int& m0, int& n0) {
-    const int per_group = kGroupM * p.tiles_n;
+    const int per_group = p.group_m * p.tiles_n;
     const int group = t / per_group;
-    const int first_m = group * kGroupM;
-    const int gsize = min(p.tiles_m - first_m, kGroupM);
+    const int first_m = group * p.group_m;
+    const int gsize = min(p.tiles_m - first_m, p.group_m);
     const int in_group = t - group * per_group;
     m0 = (first_m + in_group % gsize) * kBM;
     n0 = (in_group / gsize) * (EPI == kSwiGLU ? kBN : 2 * kBN);
@@ -436,6 +447,7 @@ int launch_gemm(const uint16_t* x, const uint16_t* w0, int64_t w0_rows, const ui
     const int64_t tiles = static_cast<int64_t>(p.tiles_m) * p.tiles_n;
     if (tiles > 0x7FFFFFFF) return DIT_ERR_SHAPE;
     p.tiles = static_cast<int>(tiles);
+    p.group_m = EPI == kSwiGLU ? GEMM_GROUP_SWIGLU : GEMM_GROUP_RESID;
     const int sms = device_sm_count();
     if (sms <= 0) return DIT_ERR_LAUNCH;
     const int64_t ctas = tiles < sms ? tiles : sms;     // one persistent CTA per SM
