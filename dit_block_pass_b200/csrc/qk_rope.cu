@@ -483,6 +483,12 @@ qk_rope_pool_kernel(QKParams p, int block, int nb, float* __restrict__ means, in
         s_w[e / HD][e % HD] = w_at(e < HD ? p.w0 : p.w1, p.w_dtype, e % HD);
     __syncthreads();
 
+    // interleaved pairs: this lane's 8 weights of q and of k stay in registers
+    float wl[2][8];
+#pragma unroll
+    for (int ten = 0; ten < 2; ++ten)
+#pragma unroll
+        for (int i = 0; i < 8; ++i) wl[ten][i] = LAYOUT == 0 ? s_w[ten][8 * sub + i] : 0.0f;
     // this lane's pairs: index, and the per-token step of w-axis pairs
     float stc[NP], sts[NP], cs[NP], sn[NP];
 #pragma unroll
@@ -501,6 +507,10 @@ qk_rope_pool_kernel(QKParams p, int block, int nb, float* __restrict__ means, in
         sn[k] = 0.0f;
     }
     int pt_ = -1, ph_ = -1, pw_ = -1, run = kRecur;
+    // grid positions advance token by token (w, then h, then t carry): one
+    // division for the warp's first token, none after
+    int gt = 0, gh = 0, gw = 0;
+    if (!p.pos && lo < hi) token_pos(p, row0 + lo, gt, gh, gw);
 
     uint64_t acc[2][V][4];
 #pragma unroll
@@ -530,7 +540,20 @@ qk_rope_pool_kernel(QKParams p, int block, int nb, float* __restrict__ means, in
         done = t + 1;
         const int64_t row = row0 + t;
         int tt, th, tw;
-        token_pos(p, row, tt, th, tw);
+        if (p.pos) {
+            token_pos(p, row, tt, th, tw);
+        } else {
+            tt = gt;
+            th = gh;
+            tw = gw;
+            if (++gw == p.Wg) {
+                gw = 0;
+                if (++gh == p.Hg) {
+                    gh = 0;
+                    ++gt;
+                }
+            }
+        }
         if (tt == pt_ && th == ph_ && tw == pw_ + 1 && run < kRecur) {
 #pragma unroll
             for (int q = 0; q < NP; ++q) {
@@ -552,15 +575,12 @@ qk_rope_pool_kernel(QKParams p, int block, int nb, float* __restrict__ means, in
             uint4* orow = (ten == 0 ? p.o0 : p.o1) + row * p.stride_v + v0;
             float A[8], Bc[8], C[4], Dd[4];
             if (LAYOUT == 0) {
-                const float4 wa = *reinterpret_cast<const float4*>(w + 8 * sub);
-                const float4 wb = *reinterpret_cast<const float4*>(w + 8 * sub + 4);
-                const float wv[8] = {wa.x, wa.y, wa.z, wa.w, wb.x, wb.y, wb.z, wb.w};
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
-                    A[q] = wv[2 * q] * cs[q];
-                    Bc[q] = -(wv[2 * q + 1] * sn[q]);
-                    C[q] = wv[2 * q] * sn[q];
-                    Dd[q] = wv[2 * q + 1] * cs[q];
+                    A[q] = wl[ten][2 * q] * cs[q];
+                    Bc[q] = -(wl[ten][2 * q + 1] * sn[q]);
+                    C[q] = wl[ten][2 * q] * sn[q];
+                    Dd[q] = wl[ten][2 * q + 1] * cs[q];
                 }
             } else {
 #pragma unroll
