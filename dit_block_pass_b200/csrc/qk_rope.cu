@@ -55,6 +55,7 @@ struct QKParams {
     bool o_rows;            // output token rows are evenly spaced: osb == N * osn
     int64_t rows;           // B * N
     int64_t N;
+    bool rows32;            // B * N < 2^31: token indices fit 32 bits
     int nvr;                // vectors per tensor row = H * hd / 8
     int Hg, Wg;
     const int32_t* pos;
@@ -139,9 +140,13 @@ __device__ __forceinline__ void token_angles(const QKParams& p, const double* s_
         pos3[1] = p.pos[3 * tok + 1];
         pos3[2] = p.pos[3 * tok + 2];
     } else {
-        // grid index < 2^31 (checked on the host)
+        // grid index < 2^31 (checked on the host); a 32-bit modulo when the
+        // token indices allow it (a 64-bit one costs several times more)
         const int hw = p.Hg * p.Wg;
-        const int g = static_cast<int>(p.pos_offset + tok % p.N);
+        const int64_t n = p.rows32 ? static_cast<int64_t>(static_cast<uint32_t>(tok) %
+                                                          static_cast<uint32_t>(p.N))
+                                   : tok % p.N;
+        const int g = static_cast<int>(p.pos_offset + n);
         const int t = g / hw;
         const int rem = g - t * hw;
         const int h = rem / p.Wg;
@@ -882,6 +887,7 @@ extern "C" int dit_qk_rmsnorm_rope3d_ex(uint16_t* q, uint16_t* k, int64_t row_st
     p.o_rows = osb == N * osn;
     p.rows = rows;
     p.N = N;
+    p.rows32 = rows < (int64_t(1) << 31);
     p.nvr = static_cast<int>(width / 8);
     p.Hg = Hg;
     p.Wg = Wg;
@@ -973,6 +979,7 @@ extern "C" int dit_qk_rmsnorm_rope3d_pooled(uint16_t* q, uint16_t* k, int64_t ro
     p.stride_v = row_stride / 8;
     p.rows = rows;
     p.N = N;
+    p.rows32 = rows < (int64_t(1) << 31);
     p.nvr = static_cast<int>(width / 8);
     p.Hg = Hg;
     p.Wg = Wg;
