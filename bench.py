@@ -53,8 +53,8 @@ NCU_SLICE_TOKENS = 32256
 NCU_TRAFFIC = {
     "adaln_modulate": {"file": "adaln.cu", "sha": "92e8ba1a144a009a",
                        "bytes_per_token": 606011392 / NCU_SLICE_TOKENS},
-    "qk_rmsnorm_rope3d": {"file": "qk_rope.cu", "sha": "7956bd20f689261b",
-                          "bytes_per_token": 1263253248 / NCU_SLICE_TOKENS},
+    "qk_rmsnorm_rope3d": {"file": "qk_rope.cu", "sha": "e122628529cadd84",
+                          "bytes_per_token": 1262753536 / NCU_SLICE_TOKENS},
     "gated_residual_adaln": {"file": "adaln.cu", "sha": "92e8ba1a144a009a",
                              "bytes_per_token": 1265638912 / NCU_SLICE_TOKENS},
     "swiglu": {"file": "swiglu.cu", "sha": "a9e07b0f774729cf",
