@@ -546,8 +546,11 @@ def time_subblock_router(chain, steps, warmup, world):
     q, k = c.qkv[:, :, :D], c.qkv[:, :, D:2 * D]
     nb = (wl.N + 127) // 128
     n_keep = dbp.subblock_keep_count(nb, 0.75)
-    ws = torch.empty(int(dbp.library().dit_subblock_workspace_bytes(wl.B, wl.N, wl.H, wl.hd, 128)),
+    L = dbp.library()
+    ws = torch.empty(max(int(L.dit_subblock_workspace_bytes(wl.B, wl.N, wl.H, wl.hd, 128)),
+                         int(L.dit_subblock_means_workspace_bytes(wl.B, wl.N, wl.H, wl.hd, 128))),
                      dtype=torch.uint8, device=c.dev)
+    status = torch.zeros(1, dtype=torch.int32, device=c.dev)
     kept = torch.empty(wl.B, wl.H, nb, n_keep, dtype=torch.int32, device=c.dev)
     means = torch.empty(wl.B, 2, nb, D, dtype=torch.float32, device=c.dev)
     grid = None if c.pos is not None else (wl.T, wl.Hg, wl.Wg)
@@ -556,9 +559,9 @@ def time_subblock_router(chain, steps, warmup, world):
     ops = {
         "router": lambda: dbp.subblock_router(q, k, wl.H, 128, 0.75, workspace=ws, kept=kept),
         "qk": lambda: qk(),
-        "qk_pooled": lambda: qk(block_means=means, block=128),
+        "qk_pooled": lambda: qk(block_means=means, block=128, status=status),
         "router_means": lambda: dbp.subblock_router_means(means, wl.N, wl.H, 128, 0.75,
-                                                          workspace=ws, kept=kept),
+                                                          workspace=ws, kept=kept, status=status),
     }
     stream = torch.cuda.current_stream()
     out = {}
@@ -573,6 +576,8 @@ def time_subblock_router(chain, steps, warmup, world):
         b.record(stream)
         barrier_sync(world)
         out[name] = max_over_ranks(a.elapsed_time(b) / steps, world)
+    if int(status.item()):
+        raise RuntimeError("the QK operator with means or the router reported an expired wait")
     del ws, kept, means
     return out, nb, n_keep
 

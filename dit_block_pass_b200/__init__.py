@@ -48,7 +48,7 @@ launch_counts = {
     "cachedit_residual_diff_noalloc": 2, "cachedit_residual_store": 1,
     "cachedit_residual_apply": 1, "swiglu_gemm": 1, "gemm_gated_residual": 1,
     "subblock_router": 3, "block_sparse_attention": 1, "qk_rmsnorm_rope3d_pooled": 1,
-    "subblock_router_means": 2,
+    "subblock_router_means": 3,        # 2 when hd is not a multiple of 32
 }
 
 
@@ -109,10 +109,10 @@ def library() -> ctypes.CDLL:
             L.dit_qk_rmsnorm_rope3d_pooled.argtypes = [vp, vp, i64, vp, vp, i32, i32, i64, i32,
                                                        i32, i32, i32, i32, vp, i64, i32, i32,
                                                        i32, dbl, dbl, i32, i32, vp, vp, vp]
-            L.dit_subblock_means_workspace_bytes.argtypes = [i32, i64, i32, i32]
+            L.dit_subblock_means_workspace_bytes.argtypes = [i32, i64, i32, i32, i32]
             L.dit_subblock_means_workspace_bytes.restype = sz
             L.dit_subblock_router_means.argtypes = [vp, i32, i64, i32, i32, i32, dbl, vp, vp, sz,
-                                                    vp]
+                                                    vp, vp]
             L.dit_swiglu_gemm.argtypes = [vp, vp, vp, i64, i32, i32, vp, vp]
             L.dit_block_sparse_attention.argtypes = [vp, vp, vp, i64, vp, i64, i32, i64, i32,
                                                      i32, i32, vp, i32, dbl, vp, vp]
@@ -696,9 +696,12 @@ def subblock_router(q: torch.Tensor, k: torch.Tensor, heads: int, block: int = 1
 
 def subblock_router_means(block_means: torch.Tensor, N: int, heads: int, block: int = 128,
                           sparsity: float = 0.75, workspace: Optional[torch.Tensor] = None,
-                          kept: Optional[torch.Tensor] = None) -> torch.Tensor:
+                          kept: Optional[torch.Tensor] = None,
+                          status: Optional[torch.Tensor] = None) -> torch.Tensor:
     """The router from block means (``qk_rmsnorm_rope3d(..., block_means=)``):
-    fp32 [B, 2, n_blocks, H*hd] -> kept int32 [B, H, n_blocks, n_keep]."""
+    fp32 [B, 2, n_blocks, H*hd] -> kept int32 [B, H, n_blocks, n_keep].
+    ``status`` (int32 CUDA scalar) is set to 1 if a wait of the tensor-core
+    score kernel expired."""
     if block_means.dtype != torch.float32 or not block_means.is_cuda or \
             not block_means.is_contiguous() or block_means.dim() != 4 or \
             block_means.shape[1] != 2:
@@ -712,7 +715,7 @@ def subblock_router_means(block_means: torch.Tensor, N: int, heads: int, block: 
     if nb == 0 or B == 0:
         return torch.empty(B, heads, nb, 0, dtype=torch.int32, device=block_means.device)
     n_keep = subblock_keep_count(nb, sparsity)
-    need = int(library().dit_subblock_means_workspace_bytes(B, N, heads, block))
+    need = int(library().dit_subblock_means_workspace_bytes(B, N, heads, hd, block))
     if workspace is None:
         workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=block_means.device)
     if workspace.numel() * workspace.element_size() < need or \
@@ -723,9 +726,11 @@ def subblock_router_means(block_means: torch.Tensor, N: int, heads: int, block: 
     if kept.dtype != torch.int32 or kept.numel() != B * heads * nb * n_keep or \
             not kept.is_contiguous() or kept.device != block_means.device:
         raise ValueError(f"kept must be a contiguous int32 [B, H, {nb}, {n_keep}] tensor")
+    if status is not None and (status.dtype != torch.int32 or not status.is_cuda):
+        raise ValueError("status must be a CUDA int32 tensor")
     _call("dit_subblock_router_means", block_means.data_ptr(), B, N, heads, hd, block,
           float(sparsity), kept.data_ptr(), workspace.data_ptr(),
-          workspace.numel() * workspace.element_size(), _stream(block_means))
+          workspace.numel() * workspace.element_size(), _ptr(status), _stream(block_means))
     return kept
 
 

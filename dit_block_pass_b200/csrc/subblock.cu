@@ -20,6 +20,15 @@
 //                           scores as a tiled GEMM of the L2-resident means
 //                           (128 x 128 tiles, 8 x 8 per thread), into the
 //                           workspace after the means.
+//   tf32_split_kernel       for the router from means: each mean split into
+//                           a tf32 high part (low 13 mantissa bits cleared)
+//                           and the remainder.
+//   subblock_scores_tc_kernel  the same scores on the tensor cores: per
+//                           128 query x 64 key block tile, the hi and lo
+//                           parts brought by TMA (128-byte swizzle) 32
+//                           head-dimension values at a time through a
+//                           two-slot ring, hi.hi + hi.lo + lo.hi accumulated
+//                           in TMEM by kind::tf32 products.
 //   subblock_select_kernel  one warp per query block: the n_keep-th largest
 //                           score of its row found bit by bit with warp-wide
 //                           counts (the row in registers up to 2048 key
@@ -28,7 +37,7 @@
 //                           ties at the threshold to the lower index.
 #include <cmath>
 
-#include "common.cuh"
+#include "tcgen05.cuh"
 
 namespace dit {
 namespace {
@@ -97,21 +106,60 @@ __device__ __forceinline__ uint32_t ordered(float f) {
 // the lane's codes in registers; warp_select_smem below: any nb, the codes
 // re-read from shared memory in every count.
 template <int KPL>
-__device__ void warp_select_reg(const float* sc, int nb, int n_keep, int32_t* out, int lane) {
+__device__ void warp_select_reg(const float* sc, int nb, int n_keep, int32_t* out, int lane,
+                                uint32_t* stage) {
     uint32_t c[KPL];
 #pragma unroll
     for (int k = 0; k < KPL; ++k) {
         const int j = k * 32 + lane;
         c[k] = j < nb ? ordered(sc[j]) : 0u;
     }
-    // a candidate is never 0, so the padding codes (0) are never counted
+    // a candidate is never 0, so the padding codes (0) are never counted.
+    // T: the bits of the threshold found so far (bits >= `bit` + 1); n_ge_t,
+    // n_ge_u: the codes >= T and >= U = T + 2^(bit+1).  Once the bucket
+    // [T, U) holds at most 32 codes they are gathered one per lane and the
+    // remaining bits are found on those alone.
     uint32_t T = 0;
-    for (int bit = 31; bit >= 0; --bit) {
+    unsigned n_ge_t = static_cast<unsigned>(nb), n_ge_u = 0;
+    int bit = 31;
+    for (; bit >= 0 && n_ge_t - n_ge_u > 32u; --bit) {
         const uint32_t cand = T | (1u << bit);
         unsigned cnt = 0;
 #pragma unroll
         for (int k = 0; k < KPL; ++k) cnt += c[k] >= cand ? 1u : 0u;
-        if (__reduce_add_sync(0xffffffffu, cnt) >= static_cast<unsigned>(n_keep)) T = cand;
+        cnt = __reduce_add_sync(0xffffffffu, cnt);
+        if (cnt >= static_cast<unsigned>(n_keep)) {
+            T = cand;
+            n_ge_t = cnt;
+        } else {
+            n_ge_u = cnt;
+        }
+    }
+    if (bit >= 0) {
+        // the bucket: nonzero codes whose bits above `bit` are T's
+        const int sh = bit + 1;
+        unsigned mine = 0;
+#pragma unroll
+        for (int k = 0; k < KPL; ++k)
+            mine += (c[k] != 0u && (sh == 32 || (c[k] >> sh) == (T >> sh))) ? 1u : 0u;
+        unsigned off = mine;                        // inclusive scan over the lanes
+#pragma unroll
+        for (int d = 1; d < 32; d <<= 1) {
+            const unsigned o = __shfl_up_sync(0xffffffffu, off, d);
+            if (lane >= d) off += o;
+        }
+        off -= mine;
+#pragma unroll
+        for (int k = 0; k < KPL; ++k)
+            if (c[k] != 0u && (sh == 32 || (c[k] >> sh) == (T >> sh))) stage[off++] = c[k];
+        __syncwarp();
+        const uint32_t e = lane < static_cast<int>(n_ge_t - n_ge_u) ? stage[lane] : 0u;
+        __syncwarp();
+        for (; bit >= 0; --bit) {
+            const uint32_t cand = T | (1u << bit);
+            const unsigned cnt = n_ge_u + __reduce_add_sync(0xffffffffu, e >= cand ? 1u : 0u);
+            if (cnt >= static_cast<unsigned>(n_keep)) T = cand;
+        }
     }
     unsigned gt = 0;
 #pragma unroll
@@ -260,10 +308,197 @@ subblock_select_kernel(const float* __restrict__ scores, int nb, int n_keep,
     const int64_t row = (static_cast<int64_t>(b) * gridDim.y + h) * nb + i;
     const float* sc = scores + row * nb;
     int32_t* out = kept + row * n_keep;
+    __shared__ uint32_t stage[kSelThreads];
     if constexpr (KPL > 0)
-        warp_select_reg<KPL>(sc, nb, n_keep, out, lane);
+        warp_select_reg<KPL>(sc, nb, n_keep, out, lane, stage + 32 * warp);
     else
         warp_select_smem(sc, nb, n_keep, out, lane);
+}
+
+// ---------------------------------------------------------------------------
+// Scores on the tensor cores for the router from precomputed means.  The
+// scores are a dense contraction (query-block means x key-block means over
+// the head dimension), but a selection threshold must be resolved to about
+// 2^-14 of the largest score, finer than one TF32 product (11 significant
+// bits).  Each mean is therefore split as a = hi + lo, hi = a with its low 13
+// mantissa bits cleared (exactly a TF32 value) and lo = a - hi (exact), and
+// the products hi*hi + hi*lo + lo*hi are accumulated in fp32 (the three-pass
+// split-TF32 method; the dropped lo*lo term and lo's own rounding to TF32 are
+// each below 2^-22 of the product).
+constexpr int kTcM = 128;        // query blocks per tile (TMEM lanes)
+constexpr int kTcN = 64;         // key blocks per tile (TMEM columns)
+constexpr int kTcChunk = 32;     // head-dimension values per 128-byte swizzle row
+constexpr int kTcSlots = 2;      // chunks in flight
+constexpr uint32_t kTcSlotBytes = 2 * (kTcM + kTcN) * kTcChunk * 4;   // hi and lo: 48 KB
+constexpr int kTcSmem = kTcSlots * kTcSlotBytes + 1024;
+
+// hi / lo of n fp32 values (n multiple of 4).
+__global__ void __launch_bounds__(256)
+tf32_split_kernel(const float4* __restrict__ src, float4* __restrict__ hi, float4* __restrict__ lo,
+                  int64_t n4) {
+    for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n4;
+         i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const float4 a = src[i];
+        float4 h, l;
+        h.x = __uint_as_float(__float_as_uint(a.x) & 0xFFFFE000u); l.x = a.x - h.x;
+        h.y = __uint_as_float(__float_as_uint(a.y) & 0xFFFFE000u); l.y = a.y - h.y;
+        h.z = __uint_as_float(__float_as_uint(a.z) & 0xFFFFE000u); l.z = a.z - h.z;
+        h.w = __uint_as_float(__float_as_uint(a.w) & 0xFFFFE000u); l.w = a.w - h.w;
+        hi[i] = h;
+        lo[i] = l;
+    }
+}
+
+// kind::tf32: fp32 accumulator, TF32 A and B, both K-major.
+constexpr uint32_t idesc_tf32(int M, int N) {
+    return (1u << 4) | (2u << 7) | (2u << 10) | ((static_cast<uint32_t>(N) >> 3) << 17) |
+           ((static_cast<uint32_t>(M) >> 4) << 24);
+}
+constexpr uint32_t kIdescTf32 = idesc_tf32(kTcM, kTcN);
+
+__device__ __forceinline__ void mma_tf32(uint32_t tmem_d, uint64_t da, uint64_t db,
+                                         uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+        "l"(da), "l"(db), "r"(kIdescTf32), "r"(accumulate)
+        : "memory");
+}
+
+// CTA (tile, h, b): scores[b, h, i0 .. i0+127, j0 .. j0+63].  Warp 0 brings
+// the hi and lo tiles of both operands 32 head-dimension values (one chunk)
+// at a time into a two-slot ring; one thread of warp 1 issues each chunk's
+// 3 x 4 products as soon as it lands and frees its slot with a commit; the
+// four warps read the accumulator (thread = query block), pass their 32
+// rows through shared memory (the ring, free once the products are done)
+// and store them row by row, a warp per 64-score row segment.  Two CTAs
+// share an SM, so one's copies overlap the other's products and stores.
+// Rows past n_blocks are computed on whatever the copy brought (the next
+// group's rows, or zeros past the array) and never stored.
+__global__ void __launch_bounds__(128, 2)
+subblock_scores_tc_kernel(const __grid_constant__ CUtensorMap map_hi_a,
+                          const __grid_constant__ CUtensorMap map_lo_a,
+                          const __grid_constant__ CUtensorMap map_hi_b,
+                          const __grid_constant__ CUtensorMap map_lo_b, int nb, int hd,
+                          float* __restrict__ scores, int* status) {
+    extern __shared__ uint8_t tc_smem_raw[];
+    __shared__ uint64_t s_bar[2 * kTcSlots + 1];
+    __shared__ uint32_t s_tmem;
+    __shared__ int s_abort;
+    const uint32_t raw = tc::smem_u32(tc_smem_raw);
+    const uint32_t base = (raw + 1023u) & ~1023u;
+    const int chunks = hd / kTcChunk;
+    constexpr uint32_t a_bytes = kTcM * kTcChunk * 4;      // 16 KB
+    constexpr uint32_t b_bytes = kTcN * kTcChunk * 4;      // 8 KB
+    // slot layout: A hi, A lo, B hi, B lo
+    const uint32_t bar_full = tc::smem_u32(&s_bar[0]);
+    const uint32_t bar_empty = tc::smem_u32(&s_bar[kTcSlots]);
+    const uint32_t bar_done = tc::smem_u32(&s_bar[2 * kTcSlots]);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int tiles_j = (nb + kTcN - 1) / kTcN;
+    const int i0 = (blockIdx.x / tiles_j) * kTcM, j0 = (blockIdx.x % tiles_j) * kTcN;
+    const int h = blockIdx.y, b = blockIdx.z;
+    const int H = gridDim.y;
+    if (threadIdx.x == 0) {
+        for (int c = 0; c <= 2 * kTcSlots; ++c) tc::mbar_init(tc::smem_u32(&s_bar[c]), 1);
+        s_abort = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == 1) tc::tmem_alloc(tc::smem_u32(&s_tmem), kTcN);
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tmem = s_tmem;
+    if (warp == 0) {
+        if (lane == 0) {
+            const int qrow = (b * 2 + 0) * nb + i0, krow = (b * 2 + 1) * nb + j0;
+            int issued = 0;
+            for (int c = 0; c < chunks; ++c) {
+                const int slot = c % kTcSlots;
+                if (c >= kTcSlots &&
+                    !tc::mbar_wait(bar_empty + 8 * slot, ((c / kTcSlots) - 1) & 1, &s_abort)) {
+                    s_abort = 1;
+                    break;
+                }
+                const uint32_t sa = base + slot * kTcSlotBytes, bar = bar_full + 8 * slot;
+                const int col = h * hd + c * kTcChunk;
+                tc::mbar_expect_tx(bar, kTcSlotBytes);
+                tc::tma_load_2d(sa, &map_hi_a, bar, col, qrow);
+                tc::tma_load_2d(sa + 2 * a_bytes, &map_hi_b, bar, col, krow);
+                tc::tma_load_2d(sa + a_bytes, &map_lo_a, bar, col, qrow);
+                tc::tma_load_2d(sa + 2 * a_bytes + b_bytes, &map_lo_b, bar, col, krow);
+                issued = c + 1;
+            }
+            // the copies land before the CTA exits: the last chunk of each
+            // slot (earlier ones were consumed before their slot was reused)
+            for (int c = issued > kTcSlots ? issued - kTcSlots : 0; c < issued; ++c)
+                tc::mbar_wait_drain(bar_full + 8 * (c % kTcSlots), (c / kTcSlots) & 1);
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        if (lane == 0) {
+            uint32_t acc = 0;
+            for (int c = 0; c < chunks; ++c) {
+                const int slot = c % kTcSlots;
+                if (!tc::mbar_wait(bar_full + 8 * slot, (c / kTcSlots) & 1, &s_abort)) {
+                    s_abort = 1;
+                    break;
+                }
+                tc::fence_after_sync();
+                const uint32_t sa = base + slot * kTcSlotBytes;
+#pragma unroll
+                for (int kk = 0; kk < kTcChunk / 8; ++kk) {
+                    const uint32_t o = kk * 32;
+                    const uint64_t ah = tc::sw128_desc(sa + o);
+                    const uint64_t al = tc::sw128_desc(sa + a_bytes + o);
+                    const uint64_t bh = tc::sw128_desc(sa + 2 * a_bytes + o);
+                    const uint64_t bl = tc::sw128_desc(sa + 2 * a_bytes + b_bytes + o);
+                    mma_tf32(tmem, ah, bh, acc);
+                    mma_tf32(tmem, ah, bl, 1u);
+                    mma_tf32(tmem, al, bh, 1u);
+                    acc = 1u;
+                }
+                tc::mma_commit(bar_empty + 8 * slot);
+            }
+            // also after a failed wait: the commit then tracks the products
+            // already issued, on chunks that had landed
+            tc::mma_commit(bar_done);
+        }
+        __syncwarp();
+    }
+    // epilogue: thread = query block i0 + 32 * warp + lane (TMEM lane); the
+    // commit is issued in every case, so the drain wait ends; the loads are
+    // skipped warp-uniformly after a failure.
+    __syncthreads();
+    bool failed = s_abort != 0;
+    if (!__all_sync(0xffffffffu, tc::mbar_wait_drain(bar_done, 0))) failed = true;
+    if (!failed) {
+        tc::fence_after_sync();
+        float v[kTcN];
+        const uint32_t lane_addr = tmem + (static_cast<uint32_t>(32 * warp) << 16);
+        tc::tmem_ld32(lane_addr, *reinterpret_cast<float(*)[32]>(v));
+        tc::tmem_ld32(lane_addr + 32, *reinterpret_cast<float(*)[32]>(v + 32));
+        tc::tmem_wait_ld();
+        // the warp's 32 x 64 scores through shared memory, rows kTcN + 1
+        // apart (no bank conflicts either way)
+        float* st = reinterpret_cast<float*>(tc_smem_raw + (base - raw)) + warp * 32 * (kTcN + 1);
+#pragma unroll
+        for (int jj = 0; jj < kTcN; ++jj) st[lane * (kTcN + 1) + jj] = v[jj];
+        __syncwarp();
+        const int rows = nb - (i0 + 32 * warp) < 32 ? nb - (i0 + 32 * warp) : 32;
+        float* out = scores + ((static_cast<int64_t>(b) * H + h) * nb + i0 + 32 * warp) * nb + j0;
+        const bool c0 = j0 + lane < nb, c1 = j0 + 32 + lane < nb;
+        for (int r = 0; r < rows; ++r) {
+            if (c0) out[static_cast<int64_t>(r) * nb + lane] = st[r * (kTcN + 1) + lane];
+            if (c1) out[static_cast<int64_t>(r) * nb + 32 + lane] = st[r * (kTcN + 1) + 32 + lane];
+        }
+    }
+    if (failed && lane == 0 && status) atomicExch(status, 1);
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    if (warp == 1) tc::tmem_dealloc(tmem, kTcN);
 }
 
 int keep_count(int64_t n_blocks, double sparsity) {
@@ -293,16 +528,9 @@ extern "C" size_t dit_subblock_workspace_bytes(int B, int64_t N, int H, int hd, 
 namespace dit {
 namespace {
 
-// Scores and selection from the block means [B, 2, nb, H*hd] (fp32) into
-// the scores buffer [B, H, nb, nb].
-int route_from_means(const float* pooled, int B, int nb, int H, int hd, int n_keep,
-                     int32_t* kept, float* scores, cudaStream_t st) {
-    const int64_t D = static_cast<int64_t>(H) * hd;
-    const int64_t tiles = (nb + kScoreTile - 1) / kScoreTile;
-    subblock_scores_kernel<<<dim3(static_cast<unsigned>(tiles * tiles), H, B), kSelThreads, 0,
-                             st>>>(pooled, nb, static_cast<int>(D), hd, scores);
-    int rc = launch_status();
-    if (rc) return rc;
+// The n_keep largest scores of each row of scores [B, H, nb, nb] into kept.
+int select_kept(const float* scores, int B, int nb, int H, int n_keep, int32_t* kept,
+                cudaStream_t st) {
     const dim3 sel((nb + 7) / 8, H, B);
     if (nb <= 256)
         subblock_select_kernel<8><<<sel, kSelThreads, 0, st>>>(scores, nb, n_keep, kept);
@@ -317,18 +545,71 @@ int route_from_means(const float* pooled, int B, int nb, int H, int hd, int n_ke
     return launch_status();
 }
 
+// Scores and selection from the block means [B, 2, nb, H*hd] (fp32) into
+// the scores buffer [B, H, nb, nb].
+int route_from_means(const float* pooled, int B, int nb, int H, int hd, int n_keep,
+                     int32_t* kept, float* scores, cudaStream_t st) {
+    const int64_t D = static_cast<int64_t>(H) * hd;
+    const int64_t tiles = (nb + kScoreTile - 1) / kScoreTile;
+    subblock_scores_kernel<<<dim3(static_cast<unsigned>(tiles * tiles), H, B), kSelThreads, 0,
+                             st>>>(pooled, nb, static_cast<int>(D), hd, scores);
+    int rc = launch_status();
+    if (rc) return rc;
+    return select_kept(scores, B, nb, H, n_keep, kept, st);
+}
+
+size_t round256(size_t n) { return (n + 255) & ~static_cast<size_t>(255); }
+
+// Whether the router from means takes the tensor-core scores (whole
+// 32-value chunks of the head dimension).
+bool tc_scores(int hd) { return hd % kTcChunk == 0; }
+
+// Tensor-core scores: split the means into hi / lo in the workspace, then one
+// CTA per 128 x 64 tile.
+int scores_tc(const float* means, int B, int nb, int H, int hd, float* scores, float* hi,
+              float* lo, int* status, cudaStream_t st) {
+    const int64_t D = static_cast<int64_t>(H) * hd;
+    const int64_t rows = static_cast<int64_t>(B) * 2 * nb;
+    const int64_t n4 = rows * D / 4;
+    const int sms = device_sm_count();
+    if (sms <= 0) return DIT_ERR_LAUNCH;
+    int64_t g = (n4 + 255) / 256;
+    if (g > static_cast<int64_t>(sms) * 8) g = static_cast<int64_t>(sms) * 8;
+    tf32_split_kernel<<<static_cast<unsigned>(g), 256, 0, st>>>(
+        reinterpret_cast<const float4*>(means), reinterpret_cast<float4*>(hi),
+        reinterpret_cast<float4*>(lo), n4);
+    int rc = launch_status();
+    if (rc) return rc;
+    CUtensorMap mha, mla, mhb, mlb;
+    if (!tc::make_map_f32(&mha, hi, rows, D, D, kTcM) || !tc::make_map_f32(&mla, lo, rows, D, D, kTcM) ||
+        !tc::make_map_f32(&mhb, hi, rows, D, D, kTcN) || !tc::make_map_f32(&mlb, lo, rows, D, D, kTcN))
+        return DIT_ERR_LAUNCH;
+    const size_t smem = kTcSmem;
+    if (cudaFuncSetAttribute(subblock_scores_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             kTcSmem) != cudaSuccess)
+        return DIT_ERR_LAUNCH;
+    const int64_t tiles = static_cast<int64_t>((nb + kTcM - 1) / kTcM) * ((nb + kTcN - 1) / kTcN);
+    subblock_scores_tc_kernel<<<dim3(static_cast<unsigned>(tiles), H, B), 128, smem, st>>>(
+        mha, mla, mhb, mlb, nb, hd, scores, status);
+    return launch_status();
+}
 }  // namespace
 }  // namespace dit
 
-extern "C" size_t dit_subblock_means_workspace_bytes(int B, int64_t N, int H, int block) {
-    if (B < 0 || N < 0 || H < 1 || block < 1) return 0;
+extern "C" size_t dit_subblock_means_workspace_bytes(int B, int64_t N, int H, int hd, int block) {
+    if (B < 0 || N < 0 || H < 1 || hd < 1 || block < 1) return 0;
     const int64_t nb = (N + block - 1) / block;
-    return static_cast<size_t>(B) * H * nb * nb * sizeof(float);
+    const size_t scores = static_cast<size_t>(B) * H * nb * nb * sizeof(float);
+    if (!dit::tc_scores(hd)) return scores;
+    // the scores, then the hi and lo parts of the means
+    const size_t means = static_cast<size_t>(B) * 2 * nb * H * hd * sizeof(float);
+    return dit::round256(scores) + 2 * dit::round256(means);
 }
 
 extern "C" int dit_subblock_router_means(const float* block_means, int B, int64_t N, int H,
                                          int hd, int block, double sparsity, int32_t* kept,
-                                         void* workspace, size_t workspace_bytes, void* stream) {
+                                         void* workspace, size_t workspace_bytes, int* status,
+                                         void* stream) {
     using namespace dit;
     if (B < 0 || N < 0 || H < 1 || block < 1) return DIT_ERR_SHAPE;
     if (hd < 8 || hd > 256 || hd % 8) return DIT_ERR_SHAPE;
@@ -340,11 +621,21 @@ extern "C" int dit_subblock_router_means(const float* block_means, int B, int64_
     const int nb = static_cast<int>(nb64);
     if (!block_means || !kept) return DIT_ERR_NULL;
     if (!aligned16(block_means) || reinterpret_cast<uintptr_t>(kept) % 4) return DIT_ERR_ALIGN;
+    if (status && reinterpret_cast<uintptr_t>(status) % 4) return DIT_ERR_ALIGN;
     if (!workspace || !aligned16(workspace) ||
-        workspace_bytes < dit_subblock_means_workspace_bytes(B, N, H, block))
+        workspace_bytes < dit_subblock_means_workspace_bytes(B, N, H, hd, block))
         return DIT_ERR_WORKSPACE;
-    return route_from_means(block_means, B, nb, H, hd, keep_count(nb, sparsity), kept,
-                            static_cast<float*>(workspace), as_stream(stream));
+    float* scores = static_cast<float*>(workspace);
+    if (!tc_scores(hd))
+        return route_from_means(block_means, B, nb, H, hd, keep_count(nb, sparsity), kept, scores,
+                                as_stream(stream));
+    const size_t sb = round256(static_cast<size_t>(B) * H * nb * nb * sizeof(float));
+    const size_t mb = round256(static_cast<size_t>(B) * 2 * nb * H * hd * sizeof(float));
+    uint8_t* w = static_cast<uint8_t*>(workspace);
+    int rc = scores_tc(block_means, B, nb, H, hd, scores, reinterpret_cast<float*>(w + sb),
+                       reinterpret_cast<float*>(w + sb + mb), status, as_stream(stream));
+    if (rc) return rc;
+    return select_kept(scores, B, nb, H, keep_count(nb, sparsity), kept, as_stream(stream));
 }
 
 extern "C" int dit_subblock_router(const uint16_t* q, const uint16_t* k, int64_t row_stride,

@@ -252,5 +252,21 @@ inline bool make_map(CUtensorMap* map, const void* base, int64_t rows, int64_t c
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// An fp32 row-major operand [rows, cols] (row_stride elements apart) read in
+// 32 x box_rows boxes (32 fp32 = one 128-byte swizzle row), zero fill.
+inline bool make_map_f32(CUtensorMap* map, const void* base, int64_t rows, int64_t cols,
+                         int64_t row_stride, uint32_t box_rows) {
+    const EncodeTiled enc = encoder();
+    if (!enc) return false;
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(row_stride) * 4};
+    const cuuint32_t box[2] = {32, box_rows};
+    const cuuint32_t elem[2] = {1, 1};
+    return enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void*>(base), dims, strides,
+               box, elem, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 }  // namespace tc
 }  // namespace dit

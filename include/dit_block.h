@@ -393,15 +393,23 @@ int dit_subblock_router(const uint16_t* q, const uint16_t* k, int64_t row_stride
  * dit_subblock_router, without reading q and k.
  *   block_means  device fp32 [B, 2, n_blocks, H*hd] (q means, then k means),
  *                16-byte aligned; n_blocks = ceil(N / block) <= 8192.
- *   workspace    device, >= dit_subblock_means_workspace_bytes(B, N, H, block)
- *                bytes (the scores [B, H, n_blocks, n_blocks] fp32),
- *                16-byte aligned.
+ *   workspace    device, >= dit_subblock_means_workspace_bytes(B, N, H, hd,
+ *                block) bytes (the scores [B, H, n_blocks, n_blocks] fp32;
+ *                for hd a multiple of 32, also the high and low tf32 parts
+ *                of the means), 16-byte aligned.
+ *   status       optional device int: set to 1 if a wait of the tensor-core
+ *                score kernel ran out (bounded at 2 s; the scores of the
+ *                affected tiles are then left unwritten).  NULL: not reported.
+ * For hd a multiple of 32 the scores are taken on the tensor cores
+ * as three tf32 products (hi.hi + hi.lo + lo.hi, the means split into a tf32
+ * high part and the remainder), which keeps them within a few fp32 rounding
+ * steps of the fp32 sum; other hd use fp32 FMAs.
  * kept, sparsity, hd limits and errors as dit_subblock_router.
  */
-size_t dit_subblock_means_workspace_bytes(int B, int64_t N, int H, int block);
+size_t dit_subblock_means_workspace_bytes(int B, int64_t N, int H, int hd, int block);
 int dit_subblock_router_means(const float* block_means, int B, int64_t N, int H, int hd,
                               int block, double sparsity, int32_t* kept, void* workspace,
-                              size_t workspace_bytes, void* stream);
+                              size_t workspace_bytes, int* status, void* stream);
 
 /*
  * Block-sparse attention over the router's kept key blocks (tensor cores):

@@ -163,3 +163,69 @@ def test_pooled_argument_errors():
              10, 10, 1e4, 1e-6, 0, 16, m.data_ptr(), None, None) == -1
     assert f(A, A + 256, 256, w.data_ptr(), w.data_ptr(), 0, 1, 64, 2, 64, 1, 8, 8, None, 0, 12,
              10, 10, 1e4, 1e-6, 0, 16, A, None, None) == -7
+
+
+ROUTER_MEANS = [
+    # B, N, H, hd, block, sparsity: several 128 x 64 score tiles with ragged
+    # edges (tensor-core scores for hd a multiple of 32: 1 to 5 chunks
+    # through the two-slot ring), and hd that takes the fp32 FMA scores (48)
+    (2, 4800, 2, 128, 8, 0.75),      # 600 blocks: 5 x 10 tiles, last 88 x 24
+    (1, 2016, 3, 96, 8, 0.8),        # 3 chunks of 32
+    (1, 8 * 2100, 1, 32, 8, 0.75),   # 2,100 blocks (selection past 2,048)
+    (2, 1000, 2, 64, 16, 0.5),       # 63 blocks: one ragged tile
+    (1, 3000, 2, 48, 16, 0.75),
+    (1, 1500, 1, 160, 8, 0.75),      # 5 chunks
+    (1, 700, 2, 256, 8, 0.75),       # 8 chunks
+]
+
+
+@pytest.mark.parametrize("B,N,H,hd,block,sp", ROUTER_MEANS)
+def test_router_from_given_means(orc, B, N, H, hd, block, sp):
+    """The router from means given directly: fp32 means of random bf16 q and
+    k (exact means rounded once to fp32).  The scores the call leaves at the
+    front of its workspace are checked one by one against the oracle's
+    (fp64 means, fp64 sums) within the bound of the arithmetic used:
+      fp32 FMA sums:      hd 2^-24 sum|q_d k_d|
+      tf32 split (3 products of a high part with 10 stored bits and the
+      remainder truncated to tf32): 3 2^-20 per product, plus 3 hd / 8
+      tensor-core accumulations of at most 2^-23 each,
+    both plus 2 2^-24 for the rounding of the means to fp32; and the kept
+    lists as the router test."""
+    D = H * hd
+    g = torch.Generator().manual_seed(N + hd)
+    x = torch.randn(B * N, 2 * D, generator=g).to(torch.bfloat16)
+    xb = bits(x)
+    nb = (N + block - 1) // block
+    m, _, _ = _means64(xb, orc, B, N, block)                       # [B, nb, 2D]
+    means = np.stack([m[:, :, :D], m[:, :, D:]], axis=1)           # [B, 2, nb, D]
+    L = dbp.library()
+    need = int(L.dit_subblock_means_workspace_bytes(B, N, H, hd, block))
+    assert need >= B * H * nb * nb * 4
+    ws = torch.full((need,), 0xFF, dtype=torch.uint8, device=DEV)
+    st = torch.zeros(1, dtype=torch.int32, device=DEV)
+    gm = torch.from_numpy(means.astype(np.float32)).to(DEV)
+    kept = dbp.subblock_router_means(gm, N, H, block, sp, workspace=ws, status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    ref, S = orc.subblock_router(xb[:, :D], xb[:, D:], B, H, hd, block, sp)
+    got_s = ws[:B * H * nb * nb * 4].view(torch.float32).cpu().numpy().reshape(B, H, nb, nb)
+    mq = means[:, 0].reshape(B, nb, H, hd).transpose(0, 2, 1, 3)    # [B, H, nb, hd]
+    mk = means[:, 1].reshape(B, nb, H, hd).transpose(0, 2, 1, 3)
+    absdot = np.einsum("bhid,bhjd->bhij", np.abs(mq), np.abs(mk))
+    tc = hd % 32 == 0
+    rel = (3 * 2.0 ** -20 + 3 * hd / 8 * 2.0 ** -23) if tc else hd * 2.0 ** -24
+    tol = (rel + 2 * 2.0 ** -24) * absdot + 1e-30
+    err = np.abs(got_s - S)
+    assert np.all(err <= tol), (float((err / tol).max()), np.unravel_index(np.argmax(err / tol), err.shape))
+    n_keep = ref.shape[-1]
+    _check_rows(kept.cpu().numpy(), ref, S, n_keep, f"means {B}x{N}x{H}x{hd}/{block}")
+
+
+def test_router_means_workspace_sizes():
+    L = dbp.library()
+    nb = (1000 + 15) // 16
+    scores = 2 * 3 * nb * nb * 4
+    assert L.dit_subblock_means_workspace_bytes(2, 1000, 3, 48, 16) == scores
+    big = L.dit_subblock_means_workspace_bytes(2, 1000, 3, 64, 16)
+    assert big >= scores + 2 * (2 * 2 * nb * 3 * 64 * 4)
+    assert L.dit_subblock_means_workspace_bytes(2, 1000, 3, 64, 0) == 0
