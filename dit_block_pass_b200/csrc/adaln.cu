@@ -390,14 +390,17 @@ gated_rows_kernel(RowParams p) {
     const float n1 = 8.0f * static_cast<float>((Dv / 64) * 32 + (rem > 32 ? rem - 32 : 0));
     const int64_t row0 = static_cast<int64_t>(blockIdx.y) * p.N;
     const int64_t rstep = static_cast<int64_t>(gridDim.x) * PAIRS;
+    bool r_issued = false;                      // this row's r copies went out last row
     for (int64_t n = static_cast<int64_t>(blockIdx.x) * PAIRS + pair; n < p.N; n += rstep) {
         const int64_t base = (row0 + n) * Dv;
+        if (!r_issued) {
 #pragma unroll
-        for (int j = 0; j < VPL; ++j) {
-            const int v = 64 * j + 32 * half + lane;
-            if (v < Dv) cp_async16(stage + j * 32 + lane, p.r + base + v);
+            for (int j = 0; j < VPL; ++j) {
+                const int v = 64 * j + 32 * half + lane;
+                if (v < Dv) cp_async16(stage + j * 32 + lane, p.r + base + v);
+            }
+            asm volatile("cp.async.commit_group;" ::: "memory");
         }
-        asm volatile("cp.async.commit_group;" ::: "memory");
         uint4 xv[VPL];
 #pragma unroll
         for (int j = 0; j < VPL; ++j) {
@@ -440,6 +443,20 @@ gated_rows_kernel(RowParams p) {
             s = gated_first_pass<VPL, TOK, true>(p, s_g, stage, xv, base, lane, half, set, x0);
         } else {
             s = gated_first_pass<VPL, TOK, false>(p, s_g, stage, xv, base, lane, half, set, x0);
+        }
+        // the stage is free (each lane read back its own vectors): the next
+        // row's r copies go out now and travel while this row's statistics
+        // and y are computed
+        const int64_t nn = n + rstep;
+        r_issued = nn < p.N;
+        if (r_issued) {
+            const uint4* rn = p.r + (row0 + nn) * Dv;
+#pragma unroll
+            for (int j = 0; j < VPL; ++j) {
+                const int v = 64 * j + 32 * half + lane;
+                if (v < Dv) cp_async16(stage + j * 32 + lane, rn + v);
+            }
+            asm volatile("cp.async.commit_group;" ::: "memory");
         }
         s = warp_sum(s);
         if (lane == 0) {

@@ -155,19 +155,34 @@ __device__ void warp_select_reg(const float* sc, int nb, int n_keep, int32_t* ou
         __syncwarp();
         const uint32_t e = lane < static_cast<int>(n_ge_t - n_ge_u) ? stage[lane] : 0u;
         __syncwarp();
+        const unsigned above = n_ge_u;              // codes above the bucket
         for (; bit >= 0; --bit) {
             const uint32_t cand = T | (1u << bit);
-            const unsigned cnt = n_ge_u + __reduce_add_sync(0xffffffffu, e >= cand ? 1u : 0u);
-            if (cnt >= static_cast<unsigned>(n_keep)) T = cand;
+            const unsigned cnt = above + __reduce_add_sync(0xffffffffu, e >= cand ? 1u : 0u);
+            if (cnt >= static_cast<unsigned>(n_keep)) {
+                T = cand;
+                n_ge_t = cnt;
+            } else {
+                n_ge_u = cnt;
+            }
         }
     }
-    unsigned gt = 0;
-#pragma unroll
-    for (int k = 0; k < KPL; ++k) gt += c[k] > T ? 1u : 0u;
+    // now U = T + 1: n_ge_u codes lie above T and n_ge_t - n_ge_u equal it;
     // `need` ties at T are taken, lowest indices first
-    const int need = n_keep - static_cast<int>(__reduce_add_sync(0xffffffffu, gt));
+    const int need = n_keep - static_cast<int>(n_ge_u);
     int written = 0, eq_seen = 0;
     const unsigned below = (1u << lane) - 1u;
+    if (static_cast<unsigned>(need) == n_ge_t - n_ge_u) {      // every tie is taken
+#pragma unroll
+        for (int k = 0; k < KPL; ++k) {
+            if (k * 32 >= nb) break;
+            const bool take = c[k] >= T;                      // padding (0) is below T
+            const unsigned tm = __ballot_sync(0xffffffffu, take);
+            if (take) out[written + __popc(tm & below)] = k * 32 + lane;
+            written += __popc(tm);
+        }
+        return;
+    }
 #pragma unroll
     for (int k = 0; k < KPL; ++k) {
         if (k * 32 >= nb) break;
