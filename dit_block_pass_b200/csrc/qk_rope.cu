@@ -300,13 +300,78 @@ __device__ __forceinline__ void qk_row_tensor(uint4 (&v)[NVL], uint4* orow, int6
     }
 }
 
+// Rotate-half pairs with the whole-row norm: a lane holds both members of
+// its pairs.  Lane-vector j of a lane is row vector paired_idx(j, lane):
+// each 64-vector span of the row holds 64 / (hd/8) whole heads, lane group
+// g = lane / (hd/16) takes head g of the span, and the lane takes vector
+// lane mod (hd/16) of that head's first half (j even) and the same vector
+// of its second half (j odd).  The hd/16 lanes of a group read consecutive
+// vectors, so every load and store still covers whole 32-byte sectors.
+template <int HD>
+__device__ __forceinline__ int paired_idx(int j, int lane) {
+    constexpr int LPH = HD / 8, HALF = LPH / 2;
+    return (j >> 1) * 64 + (lane / HALF) * LPH + (j & 1) * HALF + lane % HALF;
+}
+
+// Whole-row norm and rotate-half rotation of a row held in the paired
+// layout (NVL even): the same arithmetic per element as qk_row_tensor,
+// with each pair's partner in the lane's own registers.
+template <int HD, int NVL, bool WF32>
+__device__ __forceinline__ void qk_row_tensor_paired(uint4 (&v)[NVL], uint4* orow, int64_t osh,
+                                                     int nvr, int lane, const void* w,
+                                                     const float* cs, const float* sn,
+                                                     float eps) {
+    static_assert(NVL % 2 == 0, "paired rows hold whole pairs");
+    float ss = 0.0f;
+#pragma unroll
+    for (int j = 0; j < NVL; ++j) {
+        float f[8];
+        unpack8(v[j], f);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) ss = __fmaf_rn(f[i], f[i], ss);
+    }
+    ss = warp_sum(ss);
+    const float inv = rsqrtf(__fmaf_rn(ss, 1.0f / static_cast<float>(nvr * 8), eps));
+#pragma unroll
+    for (int j = 0; j < NVL; ++j)
+        asm volatile("" : "+r"(v[j].x), "+r"(v[j].y), "+r"(v[j].z), "+r"(v[j].w));
+    // the pair's weights are loaded as it is processed: loading them a pair
+    // ahead spills at 128 registers and measured slower
+#pragma unroll
+    for (int j = 0; j < NVL; j += 2) {
+        const int i0 = paired_idx<HD>(j, lane), i1 = paired_idx<HD>(j + 1, lane);
+        const bool ok = i0 < nvr;
+        float wa[8], wb[8], u0[8], u1[8], o0[8], o1[8];
+        w8_of<WF32>(w, (ok ? i0 : 0) * 8, wa);
+        w8_of<WF32>(w, (ok ? i1 : 0) * 8, wb);
+        unpack8(v[j], u0);
+        unpack8(v[j + 1], u1);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            u0[i] = u0[i] * inv * wa[i];
+            u1[i] = u1[i] * inv * wb[i];
+        }
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            o0[i] = __fmaf_rn(u0[i], cs[i], -u1[i] * sn[i]);
+            o1[i] = __fmaf_rn(u1[i], cs[i], u0[i] * sn[i]);
+        }
+        if (ok) {
+            st_stream(out_vec<HD, false>(orow, osh, i0), pack8(o0));
+            st_stream(out_vec<HD, false>(orow, osh, i1), pack8(o1));
+        }
+    }
+}
+
 // MODE 0: per-head norm, heads adjacent in the output; 1: per-head norm,
-// strided heads (e.g. a head-major output); 2: whole-row norm.
+// strided heads (e.g. a head-major output); 2: whole-row norm (with
+// rotate-half pairs in the paired layout, NVL being even there).
 template <int HD, int NVL, int LAYOUT, int MODE>
 __global__ void __launch_bounds__(kThreads, (NVL <= 20 ? 2 : 1))
 qk_rmsnorm_rope3d_kernel(QKParams p) {
     constexpr int LPH = HD / 8;             // lanes per head
     constexpr int NP = LAYOUT == 0 ? 4 : 8; // rotation pairs per lane
+    constexpr bool PAIRED = LAYOUT == 1 && MODE == 2 && NVL % 2 == 0;
     extern __shared__ uint4 qk_stage[];
     __shared__ double s_omega[HD / 2];      // frequency of each rotation pair
     const int lane = threadIdx.x & 31;
@@ -320,14 +385,17 @@ qk_rmsnorm_rope3d_kernel(QKParams p) {
     if (live) {
         if (row1) {
 #pragma unroll
-            for (int j = 0; j < NVL; ++j)
-                if (j * 32 + lane < p.nvr) cp_async16(stage + j * 32, row1 + j * 32 + lane);
+            for (int j = 0; j < NVL; ++j) {
+                const int idx = PAIRED ? paired_idx<HD>(j, lane) : j * 32 + lane;
+                if (idx < p.nvr) cp_async16(stage + j * 32, row1 + idx);
+            }
             asm volatile("cp.async.commit_group;" ::: "memory");
         }
 #pragma unroll
-        for (int j = 0; j < NVL; ++j)
-            v[j] = (j * 32 + lane < p.nvr) ? ld_inplace(row0 + j * 32 + lane)
-                                           : make_uint4(0, 0, 0, 0);
+        for (int j = 0; j < NVL; ++j) {
+            const int idx = PAIRED ? paired_idx<HD>(j, lane) : j * 32 + lane;
+            v[j] = idx < p.nvr ? ld_inplace(row0 + idx) : make_uint4(0, 0, 0, 0);
+        }
     }
     omega_table<HD>(p, s_omega);
     __syncthreads();
@@ -335,7 +403,14 @@ qk_rmsnorm_rope3d_kernel(QKParams p) {
 
     float cs[NP], sn[NP];
     token_angles<HD, LAYOUT>(p, s_omega, tok, lane % LPH, cs, sn);
-    if (MODE == 2) {
+    if constexpr (PAIRED) {
+        if (p.w_dtype == DIT_F32)
+            qk_row_tensor_paired<HD, NVL, true>(v, out_row(p.o0, p, tok), p.osh, p.nvr, lane,
+                                                p.w0, cs, sn, p.eps);
+        else
+            qk_row_tensor_paired<HD, NVL, false>(v, out_row(p.o0, p, tok), p.osh, p.nvr, lane,
+                                                 p.w0, cs, sn, p.eps);
+    } else if (MODE == 2) {
         if (p.w_dtype == DIT_F32)
             qk_row_tensor<HD, NVL, LAYOUT, true>(v, out_row(p.o0, p, tok), p.osh, p.nvr, lane,
                                                  p.w0, cs, sn, p.eps);
@@ -349,9 +424,18 @@ qk_rmsnorm_rope3d_kernel(QKParams p) {
         // each lane reads back only the vectors it copied itself
         asm volatile("cp.async.wait_group 0;" ::: "memory");
 #pragma unroll
-        for (int j = 0; j < NVL; ++j)
-            v[j] = (j * 32 + lane < p.nvr) ? stage[j * 32] : make_uint4(0, 0, 0, 0);
-        if (MODE == 2) {
+        for (int j = 0; j < NVL; ++j) {
+            const int idx = PAIRED ? paired_idx<HD>(j, lane) : j * 32 + lane;
+            v[j] = idx < p.nvr ? stage[j * 32] : make_uint4(0, 0, 0, 0);
+        }
+        if constexpr (PAIRED) {
+            if (p.w_dtype == DIT_F32)
+                qk_row_tensor_paired<HD, NVL, true>(v, out_row(p.o1, p, tok), p.osh, p.nvr,
+                                                    lane, p.w1, cs, sn, p.eps);
+            else
+                qk_row_tensor_paired<HD, NVL, false>(v, out_row(p.o1, p, tok), p.osh, p.nvr,
+                                                     lane, p.w1, cs, sn, p.eps);
+        } else if (MODE == 2) {
             if (p.w_dtype == DIT_F32)
                 qk_row_tensor<HD, NVL, LAYOUT, true>(v, out_row(p.o1, p, tok), p.osh, p.nvr,
                                                      lane, p.w1, cs, sn, p.eps);
@@ -900,7 +984,11 @@ extern "C" int dit_qk_rmsnorm_rope3d_ex(uint16_t* q, uint16_t* k, int64_t row_st
     p.eps = static_cast<float>(eps);
 
     const int mode = norm_width == DIT_NORM_ROW ? 2 : (osh == hd ? 0 : 1);
-    const Pick pk = pick(hd, rope_layout, mode, (p.nvr + 31) / 32);
+    // rotate-half with the whole-row norm holds the row in whole 64-vector
+    // spans (an even count of lane-vectors)
+    const int nvl = mode == 2 && rope_layout == DIT_ROPE_HALF ? 2 * ((p.nvr + 63) / 64)
+                                                              : (p.nvr + 31) / 32;
+    const Pick pk = pick(hd, rope_layout, mode, nvl);
     if (!pk.kernel) return DIT_ERR_SHAPE;
     // the second tensor's stage
     const size_t smem =
