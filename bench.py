@@ -51,12 +51,12 @@ DOMINANT = "swiglu"
 # comments and blank space); it is reported as null otherwise.
 NCU_SLICE_TOKENS = 32256
 NCU_TRAFFIC = {
-    "adaln_modulate": {"file": "adaln.cu", "sha": "92e8ba1a144a009a",
-                       "bytes_per_token": 606011392 / NCU_SLICE_TOKENS},
+    "adaln_modulate": {"file": "adaln.cu", "sha": "b4f26979a5cdeb0e",
+                       "bytes_per_token": 608085760 / NCU_SLICE_TOKENS},
     "qk_rmsnorm_rope3d": {"file": "qk_rope.cu", "sha": "e122628529cadd84",
                           "bytes_per_token": 1262753536 / NCU_SLICE_TOKENS},
-    "gated_residual_adaln": {"file": "adaln.cu", "sha": "92e8ba1a144a009a",
-                             "bytes_per_token": 1265638912 / NCU_SLICE_TOKENS},
+    "gated_residual_adaln": {"file": "adaln.cu", "sha": "b4f26979a5cdeb0e",
+                             "bytes_per_token": 1265792512 / NCU_SLICE_TOKENS},
     "swiglu": {"file": "swiglu.cu", "sha": "a9e07b0f774729cf",
                "bytes_per_token": 2620489264 / NCU_SLICE_TOKENS},
     "cachedit_residual_diff": {"file": "cachedit.cu", "sha": "9a1487d46a877c49",
