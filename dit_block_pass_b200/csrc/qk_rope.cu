@@ -449,6 +449,149 @@ qk_rmsnorm_rope3d_kernel(QKParams p) {
 }
 
 // ---------------------------------------------------------------------------
+// Whole-row norm, persistent (rows of up to 20 lane-vectors, H*hd <= 5120):
+// one CTA of kRowWarps warps per SM.  The per-element weights of q and k are
+// staged once per CTA in shared memory (fp32, lo/hi float4 halves, so a warp
+// reads them without bank conflicts) instead of passing through L1 for every
+// token, and each warp streams its rows (q then k of each of its tokens)
+// through one shared-memory stage: as soon as a row's values are in
+// registers and summed, the next row's copy is issued into the stage, so
+// one row per warp is always in flight.  The arithmetic per element is the
+// one-shot whole-row kernel's (same lane-vectors, same order of the sums).
+constexpr int kRowWarps = 16;
+constexpr int kRowMaxNVL = 20;
+
+template <int HD, int NVL, int LAYOUT>
+__device__ __forceinline__ void row_copy(const uint4* row, uint4* stage, int nvr, int lane) {
+#pragma unroll
+    for (int j = 0; j < NVL; ++j) {
+        const int idx = LAYOUT == 1 ? paired_idx<HD>(j, lane) : j * 32 + lane;
+        if (idx < nvr) cp_async16(stage + j * 32, row + idx);
+    }
+    asm volatile("cp.async.commit_group;" ::: "memory");
+}
+
+// Weighted rotation and store of a row normalised by inv, the weights read
+// from the shared-memory copy s_w (s_w[idx]: elements 8 idx .. 8 idx + 3,
+// s_w[nvr + idx]: the next four).
+template <int HD, int NVL, int LAYOUT>
+__device__ __forceinline__ void qk_row_rotate_smem(const uint4 (&v)[NVL], uint4* orow, int64_t osh,
+                                                   int nvr, int lane, const float4* s_w,
+                                                   float inv, const float* cs, const float* sn) {
+    if constexpr (LAYOUT == 0) {
+#pragma unroll
+        for (int j = 0; j < NVL; ++j) {
+            const int idx = j * 32 + lane;
+            if (idx < nvr) {
+                float f[8], o8[8];
+                unpack8(v[j], f);
+                const float4 a = s_w[idx], b = s_w[nvr + idx];
+                const float wv[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const float u0 = f[2 * k] * inv * wv[2 * k];
+                    const float u1 = f[2 * k + 1] * inv * wv[2 * k + 1];
+                    o8[2 * k] = __fmaf_rn(u0, cs[k], -u1 * sn[k]);
+                    o8[2 * k + 1] = __fmaf_rn(u0, sn[k], u1 * cs[k]);
+                }
+                st_stream(out_vec<HD, false>(orow, osh, idx), pack8(o8));
+            }
+        }
+    } else {
+#pragma unroll
+        for (int j = 0; j < NVL; j += 2) {
+            const int i0 = paired_idx<HD>(j, lane), i1 = paired_idx<HD>(j + 1, lane);
+            if (i0 < nvr) {
+                float u0[8], u1[8], o0[8], o1[8];
+                unpack8(v[j], u0);
+                unpack8(v[j + 1], u1);
+                const float4 a0 = s_w[i0], b0 = s_w[nvr + i0];
+                const float4 a1 = s_w[i1], b1 = s_w[nvr + i1];
+                const float wa[8] = {a0.x, a0.y, a0.z, a0.w, b0.x, b0.y, b0.z, b0.w};
+                const float wb[8] = {a1.x, a1.y, a1.z, a1.w, b1.x, b1.y, b1.z, b1.w};
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    u0[i] = u0[i] * inv * wa[i];
+                    u1[i] = u1[i] * inv * wb[i];
+                }
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    o0[i] = __fmaf_rn(u0[i], cs[i], -u1[i] * sn[i]);
+                    o1[i] = __fmaf_rn(u1[i], cs[i], u0[i] * sn[i]);
+                }
+                st_stream(out_vec<HD, false>(orow, osh, i0), pack8(o0));
+                st_stream(out_vec<HD, false>(orow, osh, i1), pack8(o1));
+            }
+        }
+    }
+}
+
+template <int HD, int NVL, int LAYOUT>
+__global__ void __launch_bounds__(kRowWarps * 32, 1)
+qk_row_persistent_kernel(QKParams p) {
+    static_assert(LAYOUT == 0 || NVL % 2 == 0, "paired rows hold whole pairs");
+    constexpr int LPH = HD / 8;
+    constexpr int NP = LAYOUT == 0 ? 4 : 8;
+    extern __shared__ float4 qk_rows_smem[];
+    __shared__ double s_omega[HD / 2];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int nvr = p.nvr;
+    const int ntens = p.t1 ? 2 : 1;
+    uint4* stage = reinterpret_cast<uint4*>(qk_rows_smem + 2 * nvr * ntens) + warp * (NVL * 32) + lane;
+    const int64_t tstep = static_cast<int64_t>(gridDim.x) * kRowWarps;
+    int64_t tok = static_cast<int64_t>(blockIdx.x) * kRowWarps + warp;
+    if (tok < p.rows) row_copy<HD, NVL, LAYOUT>(p.t0 + tok * p.stride_v, stage, nvr, lane);
+    // the weights, while the first rows travel
+    for (int t = 0; t < ntens; ++t) {
+        const void* w = t ? p.w1 : p.w0;
+        float4* sw = qk_rows_smem + 2 * nvr * t;
+        for (int v = threadIdx.x; v < nvr; v += blockDim.x) {
+            float f[8];
+            if (p.w_dtype == DIT_F32)
+                w8_of<true>(w, 8 * v, f);
+            else
+                w8_of<false>(w, 8 * v, f);
+            sw[v] = make_float4(f[0], f[1], f[2], f[3]);
+            sw[nvr + v] = make_float4(f[4], f[5], f[6], f[7]);
+        }
+    }
+    omega_table<HD>(p, s_omega);
+    __syncthreads();
+    for (; tok < p.rows; tok += tstep) {
+        float cs[NP], sn[NP];
+        token_angles<HD, LAYOUT>(p, s_omega, tok, lane % LPH, cs, sn);
+        for (int t = 0; t < ntens; ++t) {
+            asm volatile("cp.async.wait_group 0;" ::: "memory");
+            uint4 v[NVL];
+            float ss = 0.0f;
+#pragma unroll
+            for (int j = 0; j < NVL; ++j) {
+                const int idx = LAYOUT == 1 ? paired_idx<HD>(j, lane) : j * 32 + lane;
+                v[j] = idx < nvr ? stage[j * 32] : make_uint4(0, 0, 0, 0);
+                float f[8];
+                unpack8(v[j], f);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) ss = __fmaf_rn(f[i], f[i], ss);
+            }
+            ss = warp_sum(ss);
+            const float inv = rsqrtf(__fmaf_rn(ss, 1.0f / static_cast<float>(nvr * 8), p.eps));
+            // every lane's stage values are in the sum: the next row's copy
+            const bool same = t + 1 < ntens;
+            const int64_t ntok = same ? tok : tok + tstep;
+            if (ntok < p.rows)
+                row_copy<HD, NVL, LAYOUT>((same ? p.t1 : p.t0) + ntok * p.stride_v, stage, nvr,
+                                          lane);
+#pragma unroll
+            for (int j = 0; j < NVL; ++j)
+                asm volatile("" : "+r"(v[j].x), "+r"(v[j].y), "+r"(v[j].z), "+r"(v[j].w));
+            qk_row_rotate_smem<HD, NVL, LAYOUT>(v, out_row(t ? p.o1 : p.o0, p, tok), p.osh, nvr,
+                                                lane, qk_rows_smem + 2 * nvr * t, inv, cs, sn);
+        }
+    }
+    asm volatile("cp.async.wait_group 0;" ::: "memory");
+}
+
+// ---------------------------------------------------------------------------
 // QK RMSNorm + 3D RoPE in place that also writes the mean of each block of
 // `block` consecutive tokens of the rotated q and k (the SubBlock router's
 // block summaries), so the router does not read q and k again.
@@ -821,6 +964,34 @@ Pick pick(int hd, int layout, int mode, int nvl) {
     }
 }
 
+template <int HD, int LAYOUT>
+Pick pick_row_nvl(int nvl) {
+#define DIT_ROW_CASE(V)                                                              \
+    if (nvl <= V) return Pick{qk_row_persistent_kernel<HD, V, LAYOUT>, V};
+    if constexpr (LAYOUT == 0) {
+        DIT_ROW_CASE(1) DIT_ROW_CASE(2) DIT_ROW_CASE(3) DIT_ROW_CASE(4) DIT_ROW_CASE(6)
+        DIT_ROW_CASE(8) DIT_ROW_CASE(10) DIT_ROW_CASE(12) DIT_ROW_CASE(16) DIT_ROW_CASE(20)
+    } else {
+        DIT_ROW_CASE(2) DIT_ROW_CASE(4) DIT_ROW_CASE(6) DIT_ROW_CASE(8) DIT_ROW_CASE(10)
+        DIT_ROW_CASE(12) DIT_ROW_CASE(16) DIT_ROW_CASE(20)
+    }
+#undef DIT_ROW_CASE
+    return Pick{};
+}
+
+// The persistent whole-row kernel for rows of up to kRowMaxNVL lane-vectors.
+Pick pick_row(int hd, int layout, int nvl) {
+    if (nvl > kRowMaxNVL) return Pick{};
+    const bool half = layout == DIT_ROPE_HALF;
+    switch (hd) {
+        case 32: return half ? pick_row_nvl<32, 1>(nvl) : pick_row_nvl<32, 0>(nvl);
+        case 64: return half ? pick_row_nvl<64, 1>(nvl) : pick_row_nvl<64, 0>(nvl);
+        case 128: return half ? pick_row_nvl<128, 1>(nvl) : pick_row_nvl<128, 0>(nvl);
+        case 256: return half ? pick_row_nvl<256, 1>(nvl) : pick_row_nvl<256, 0>(nvl);
+        default: return Pick{};
+    }
+}
+
 // Rows i of q and k (i < rows, `rs` elements apart, `w` wide) overlap iff
 // some row difference m in (-rows, rows) puts k within w elements of q.
 bool rows_overlap(const void* q, const void* k, int64_t rows, int64_t rs, int64_t w) {
@@ -988,6 +1159,24 @@ extern "C" int dit_qk_rmsnorm_rope3d_ex(uint16_t* q, uint16_t* k, int64_t row_st
     // spans (an even count of lane-vectors)
     const int nvl = mode == 2 && rope_layout == DIT_ROPE_HALF ? 2 * ((p.nvr + 63) / 64)
                                                               : (p.nvr + 31) / 32;
+    if (mode == 2) {
+        const Pick rk = pick_row(hd, rope_layout, nvl);
+        if (rk.kernel) {
+            const int ntens = p.t1 ? 2 : 1;
+            const size_t rsmem = static_cast<size_t>(2 * p.nvr * ntens) * sizeof(float4) +
+                                 static_cast<size_t>(kRowWarps) * rk.nvl * 32 * sizeof(uint4);
+            if (cudaFuncSetAttribute(rk.kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     static_cast<int>(rsmem)) != cudaSuccess)
+                return DIT_ERR_LAUNCH;
+            const int sms = device_sm_count();
+            const int occ = occupancy(reinterpret_cast<const void*>(rk.kernel), kRowWarps * 32, rsmem);
+            if (sms <= 0 || occ <= 0) return DIT_ERR_LAUNCH;
+            int64_t ctas = (rows + kRowWarps - 1) / kRowWarps;
+            if (ctas > static_cast<int64_t>(sms) * occ) ctas = static_cast<int64_t>(sms) * occ;
+            rk.kernel<<<static_cast<unsigned>(ctas), kRowWarps * 32, rsmem, as_stream(stream)>>>(p);
+            return launch_status();
+        }
+    }
     const Pick pk = pick(hd, rope_layout, mode, nvl);
     if (!pk.kernel) return DIT_ERR_SHAPE;
     // the second tensor's stage
