@@ -53,8 +53,8 @@ NCU_SLICE_TOKENS = 32256
 NCU_TRAFFIC = {
     "adaln_modulate": {"file": "adaln.cu", "sha": "b4f26979a5cdeb0e",
                        "bytes_per_token": 608085760 / NCU_SLICE_TOKENS},
-    "qk_rmsnorm_rope3d": {"file": "qk_rope.cu", "sha": "9975a63606d189a1",
-                          "bytes_per_token": 1263007744 / NCU_SLICE_TOKENS},
+    "qk_rmsnorm_rope3d": {"file": "qk_rope.cu", "sha": "b057e79cd2493df0",
+                          "bytes_per_token": 1263321856 / NCU_SLICE_TOKENS},
     "gated_residual_adaln": {"file": "adaln.cu", "sha": "b4f26979a5cdeb0e",
                              "bytes_per_token": 1265792512 / NCU_SLICE_TOKENS},
     "swiglu": {"file": "swiglu.cu", "sha": "a9e07b0f774729cf",
