@@ -117,6 +117,67 @@ def test_fullsize_qk_rope(orc, name):
     assert np.array_equal(sel[:, 2 * D:], hb[:, 2 * D:]), "v changed"
 
 
+@pytest.mark.parametrize("layout", [dbp.ROPE_INTERLEAVED, dbp.ROPE_HALF])
+@pytest.mark.parametrize("name", ["h3_5s", "cfg_av"])
+def test_fullsize_qk_whole_row_norm(orc, name, layout):
+    """The whole-row norm options at full size (the persistent row kernel,
+    as the benchmark times it), sampled rows against the oracle."""
+    wl = W.CONFIGS[name]
+    B, N, D, M = wl.B, wl.N, wl.D, wl.M
+    rows = W.sample_rows(wl, SAMPLE)
+    qkv = W.token_rows(wl, W.S_QKV, 3 * D, device=DEV)
+    qh = W.token_rows(wl, W.S_QKV, 3 * D, row_ids=rows)
+    _same_rows(qkv[rows.to(DEV)], qh)
+    wq, wk = W.row_norm_weights(wl, device=DEV)
+    v3 = qkv.view(B, N, 3 * D)
+    pos = W.positions(wl, device=DEV)
+    dbp.qk_rmsnorm_rope3d(v3[:, :, :D], v3[:, :, D:2 * D], wq, wk, wl.H, wl.pairs,
+                          grid=None if pos is not None else (wl.T, wl.Hg, wl.Wg), pos=pos,
+                          theta=wl.theta, eps=wl.eps, rope_layout=layout,
+                          norm_width=dbp.NORM_ROW)
+    sel = bits(qkv[rows.to(DEV)])
+    del qkv, v3
+    _free()
+    if pos is not None:
+        p = pos.cpu().numpy()[rows.numpy()]
+    else:
+        p = orc.grid_positions(wl.T, wl.Hg, wl.Wg, 0, N)[(rows % N).numpy()]
+    hb = bits(qh)
+    for t, w in ((0, wq), (1, wk)):
+        ref = orc.qk_rmsnorm_rope3d_ex(hb[:, t * D:(t + 1) * D], w.cpu().double().numpy(), wl.H,
+                                       wl.hd, np.ascontiguousarray(p), wl.pairs, wl.theta, wl.eps,
+                                       layout=layout, norm=dbp.NORM_ROW)
+        compare_bf16(sel[:, t * D:(t + 1) * D], ref, f"{name} {'qk'[t]} layout {layout}")
+    assert np.array_equal(sel[:, 2 * D:], hb[:, 2 * D:]), "v changed"
+
+
+def test_fullsize_qk_means_then_router(orc):
+    """h3_5s: the QK operator with block means, then the router from those
+    means (tensor-core scores, 977 blocks), against the oracle router on the
+    kernel's own q and k for two heads (within the fp32 tie band)."""
+    from test_gpu_subblock import _check_rows
+    wl = W.CONFIGS["h3_5s"]
+    N, D, H, hd = wl.N, wl.D, wl.H, wl.hd
+    qkv = W.token_rows(wl, W.S_QKV, 3 * D, device=DEV).view(1, N, 3 * D)
+    wq, wk = W.norm_weights(wl, device=DEV)
+    nb = (N + 127) // 128
+    means = torch.empty(1, 2, nb, D, dtype=torch.float32, device=DEV)
+    st = torch.zeros(1, dtype=torch.int32, device=DEV)
+    dbp.qk_rmsnorm_rope3d(qkv[:, :, :D], qkv[:, :, D:2 * D], wq, wk, H, wl.pairs,
+                          grid=(wl.T, wl.Hg, wl.Wg), theta=wl.theta, eps=wl.eps,
+                          block_means=means, block=128, status=st)
+    kept = dbp.subblock_router_means(means, N, H, 128, 0.75, status=st).cpu().numpy()
+    assert int(st.item()) == 0
+    for h in (0, 29):
+        q = bits(qkv[0, :, h * hd:(h + 1) * hd])
+        k = bits(qkv[0, :, D + h * hd:D + (h + 1) * hd])
+        ref, S = orc.subblock_router(q, k, 1, 1, hd, 128, 0.75)
+        assert ref.shape[-1] == 245
+        _check_rows(kept[0, h], ref[0, 0], S[0, 0], 245, f"h3 means head {h}")
+    del qkv, means
+    _free()
+
+
 @pytest.mark.parametrize("name", ["h3_5s", "h3_10s", "cfg_av"])
 def test_fullsize_cachedit(orc, name):
     wl = W.CONFIGS[name]
