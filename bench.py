@@ -627,41 +627,75 @@ def tensor_peaks():
 
 def time_e2e(chain, steps, warmup, world):
     """The same chain through the public API with inputs on the host: every
-    step copies its inputs host->device from pinned memory, runs the chain and
-    reads every output back device->host.  Returns (ms per step, h2d bytes,
+    step copies all of its inputs host->device from pinned memory, runs the
+    chain and reads every output back device->host.  Two device buffer sets
+    alternate between steps, with the copies in on one stream, the chain on a
+    second and the copies out on a third, so step i's inputs travel while
+    step i-1 computes and step i-2's outputs travel back (the link carries
+    both directions at once); a set is refilled only after its outputs have
+    been read back.  The timed region runs from the first timed step's first
+    copy in to the last one's last copy out.  Returns (ms per step, h2d bytes,
     d2h bytes)."""
+    import copy
+
     import torch
     c = chain
-    ins = [c.x, c.r, c.qkv, c.swi, c.prev, c.cur]
-    outs = [c.y1, c.qkv, c.xo, c.y2, c.out, c.rel, c.reuse]
-    host_in = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in ins]
-    for h, t in zip(host_in, ins):
-        h.copy_(t)
-    host_out = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in outs]
-    h2d = sum(t.numel() * t.element_size() for t in ins)
-    d2h = sum(t.numel() * t.element_size() for t in outs)
-    ops = c.ops()
-    stream = torch.cuda.current_stream()
+    names_in = ["x", "r", "qkv", "swi", "prev", "cur"]
+    names_out = ["y1", "qkv", "xo", "y2", "out", "rel", "reuse"]
+    c2 = copy.copy(c)
+    for n in dict.fromkeys(names_in + names_out + ["ws"]):
+        setattr(c2, n, torch.empty_like(getattr(c, n)))
+    sets = [c, c2]
+    ops = [s_.ops() for s_ in sets]
+    host_in = [torch.empty(getattr(c, n).shape, dtype=getattr(c, n).dtype, pin_memory=True)
+               for n in names_in]
+    for h, n in zip(host_in, names_in):
+        h.copy_(getattr(c, n))
+    host_out = [torch.empty(getattr(c, n).shape, dtype=getattr(c, n).dtype, pin_memory=True)
+                for n in names_out]
+    h2d = sum(h.numel() * h.element_size() for h in host_in)
+    d2h = sum(h.numel() * h.element_size() for h in host_out)
+    s_in, s_comp, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
+    in_done = [torch.cuda.Event(), torch.cuda.Event()]
+    comp_done = [torch.cuda.Event(), torch.cuda.Event()]
+    freed = [torch.cuda.Event(), torch.cuda.Event()]
+    used = [False, False]
 
-    def step():
-        for h, t in zip(host_in, ins):
-            t.copy_(h, non_blocking=True)
-        for op in ops:
-            op()
-        for h, t in zip(host_out, outs):
-            h.copy_(t, non_blocking=True)
+    def step(i):
+        k = i % 2
+        s_ = sets[k]
+        with torch.cuda.stream(s_in):
+            if used[k]:
+                s_in.wait_event(freed[k])
+            for h, n in zip(host_in, names_in):
+                getattr(s_, n).copy_(h, non_blocking=True)
+            in_done[k].record(s_in)
+        with torch.cuda.stream(s_comp):
+            s_comp.wait_event(in_done[k])
+            for op in ops[k]:
+                op()
+            comp_done[k].record(s_comp)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(comp_done[k])
+            for h, n in zip(host_out, names_out):
+                h.copy_(getattr(s_, n), non_blocking=True)
+            freed[k].record(s_out)
+        used[k] = True
 
-    for _ in range(warmup):
-        step()
+    for i in range(warmup):
+        step(i)
+    torch.cuda.synchronize()
     barrier_sync(world)
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    a.record(stream)
-    for _ in range(steps):
-        step()
-    b.record(stream)
+    a.record(s_in)
+    for i in range(warmup, warmup + steps):
+        step(i)
+    b.record(s_out)
+    torch.cuda.synchronize()
     barrier_sync(world)
     ms = max_over_ranks(a.elapsed_time(b), world) / steps
-    del host_in, host_out
+    del host_in, host_out, c2, sets, ops
+    torch.cuda.empty_cache()
     return ms, h2d, d2h
 
 
@@ -980,7 +1014,7 @@ def main():
     ap.add_argument("--configs", default="h3_10s,cfg_av",
                     help="other workloads timed after the headline (comma list, or none)")
     ap.add_argument("--config-steps", type=int, default=40)
-    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--e2e-steps", type=int, default=8)
     ap.add_argument("--attn-steps", type=int, default=3,
                     help="timed launches of the block-sparse attention and of dense attention")
     ap.add_argument("--gemm-steps", type=int, default=12,
@@ -1044,7 +1078,7 @@ def main():
             extras["attn"] = time_sparse_attention(chain, args.attn_steps, world)
         e2e = None
         if not args.no_e2e and not args.shard:
-            ms_e2e, h2d, d2h = time_e2e(chain, args.e2e_steps, 1, world)
+            ms_e2e, h2d, d2h = time_e2e(chain, args.e2e_steps, 2, world)
             e2e = {"value": world * tokens / (ms_e2e / 1000.0), "unit": "tokens/s",
                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                    "ms_per_step": round(ms_e2e, 3)}
