@@ -23,12 +23,17 @@
 // reduction inside its lane group, and the RMSNorm weight is folded into
 // per-lane rotation coefficients once per token and tensor.  Whole-row norm:
 // the row's sum of squares is a warp reduction over every vector the lane
-// holds, and the per-element weights are read through L1.
+// holds; rows up to 5,120 wide take a persistent kernel that stages the
+// per-element weights in shared memory once per CTA and streams each warp's
+// rows through one stage, wider rows the one-shot kernel with the weights
+// read through L1.
 //
 // Rotation: a lane always holds the same rotation pairs of a head (4 pairs
-// inside its vector when pairs are interleaved; 8 pairs shared with the lane
-// hd/16 away when they are (p, p + hd/2)), so it computes their angles once
-// per token and reuses them for every head of q and k.  The hd/2
+// inside its vector when pairs are interleaved; 8 pairs (p, p + hd/2) when
+// they are rotate-half, the partner elements fetched from the lane hd/16 away
+// with a shuffle, or, for the whole-row norm, held by the lane itself in a
+// paired layout), so it computes their angles once per token and reuses them
+// for every head of q and k.  The hd/2
 // frequencies are computed in fp64 once per CTA into shared memory while the
 // rows load; the angles pos*omega are formed and reduced modulo 2*pi in
 // fp64, and sin/cos are taken in fp32 on the reduced angle, which keeps the
