@@ -44,23 +44,25 @@ OPS = ["adaln_modulate", "qk_rmsnorm_rope3d", "gated_residual_adaln", "swiglu",
        "cachedit_residual_diff"]
 DOMINANT = "swiglu"
 
-# DRAM traffic from ncu (dram__bytes_read.sum + dram__bytes_write.sum of one
-# launch of each op's kernels on the 32,256-token h3_slice, per token; every
-# op is a stream, so traffic scales with the token count).  An entry is valid
-# only while its kernel source is unchanged (hash of the .cu file without
-# comments and blank space); it is reported as null otherwise.
-NCU_SLICE_TOKENS = 32256
+# DRAM traffic from ncu (dram__bytes_read.sum + dram__bytes_write.sum) of
+# one full launch of each op's main kernel on the 5 s clip (124,992 tokens; a
+# one-pass capture, see profiles/dram_traffic_h3_5s.md), per token; every op
+# is a stream, so for the other configs traffic scales with the token count.
+# An entry is valid only while its kernel source is unchanged (hash of the
+# .cu file without comments and blank space); it is reported as null
+# otherwise.
+NCU_TOKENS = 124992
 NCU_TRAFFIC = {
     "adaln_modulate": {"file": "adaln.cu", "sha": "b4f26979a5cdeb0e",
-                       "bytes_per_token": 608085760 / NCU_SLICE_TOKENS},
+                       "bytes_per_token": 2507664128 / NCU_TOKENS},
     "qk_rmsnorm_rope3d": {"file": "qk_rope.cu", "sha": "b057e79cd2493df0",
-                          "bytes_per_token": 1263321856 / NCU_SLICE_TOKENS},
+                          "bytes_per_token": 5056747008 / NCU_TOKENS},
     "gated_residual_adaln": {"file": "adaln.cu", "sha": "b4f26979a5cdeb0e",
-                             "bytes_per_token": 1265792512 / NCU_SLICE_TOKENS},
+                             "bytes_per_token": 5064393472 / NCU_TOKENS},
     "swiglu": {"file": "swiglu.cu", "sha": "a9e07b0f774729cf",
-               "bytes_per_token": 2620489264 / NCU_SLICE_TOKENS},
+               "bytes_per_token": 10308000512 / NCU_TOKENS},
     "cachedit_residual_diff": {"file": "cachedit.cu", "sha": "9a1487d46a877c49",
-                               "bytes_per_token": 665030400 / NCU_SLICE_TOKENS},
+                               "bytes_per_token": 2560026112 / NCU_TOKENS},
 }
 
 
@@ -848,8 +850,9 @@ def op_report(nbytes: dict, per_op, tokens: int, peak: float, traffic: dict) -> 
 
 
 def ncu_traffic(tokens: int) -> dict:
-    """DRAM bytes of one full launch of each op, from the slice captures
-    whose kernel source still matches; absent entries are null."""
+    """DRAM bytes of one full launch of each op over `tokens` tokens, from
+    the full-size captures whose kernel source still matches; absent
+    entries are null."""
     out = {}
     for name, tr in NCU_TRAFFIC.items():
         if tr["sha"] == source_sha(tr["file"]):
