@@ -559,7 +559,8 @@ def time_subblock_router(chain, steps, warmup, world):
     qk = lambda **kw: dbp.qk_rmsnorm_rope3d(q, k, c.wq, c.wk, wl.H, wl.pairs, grid=grid,
                                             pos=c.pos, theta=wl.theta, eps=wl.eps, **kw)
     ops = {
-        "router": lambda: dbp.subblock_router(q, k, wl.H, 128, 0.75, workspace=ws, kept=kept),
+        "router": lambda: dbp.subblock_router(q, k, wl.H, 128, 0.75, workspace=ws, kept=kept,
+                                              status=status),
         "qk": lambda: qk(),
         "qk_pooled": lambda: qk(block_means=means, block=128, status=status),
         "router_means": lambda: dbp.subblock_router_means(means, wl.N, wl.H, 128, 0.75,

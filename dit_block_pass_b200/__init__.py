@@ -47,7 +47,7 @@ launch_counts = {
     "cachedit_residual_diff": 2, "cachedit_residual_sums": 2, "cachedit_decide": 1,
     "cachedit_residual_diff_noalloc": 2, "cachedit_residual_store": 1,
     "cachedit_residual_apply": 1, "swiglu_gemm": 1, "gemm_gated_residual": 1,
-    "subblock_router": 3, "block_sparse_attention": 1, "qk_rmsnorm_rope3d_pooled": 1,
+    "subblock_router": 4, "block_sparse_attention": 1, "qk_rmsnorm_rope3d_pooled": 1,
     "subblock_router_means": 3,        # 2 when hd is not a multiple of 32
 }
 
@@ -120,7 +120,7 @@ def library() -> ctypes.CDLL:
             L.dit_subblock_workspace_bytes.argtypes = [i32, i64, i32, i32, i32]
             L.dit_subblock_workspace_bytes.restype = sz
             L.dit_subblock_router.argtypes = [vp, vp, i64, i32, i64, i32, i32, i32, dbl, vp, vp,
-                                              sz, vp]
+                                              sz, vp, vp]
             L.dit_swiglu_gemm_stall_test.argtypes = [vp, vp, vp, i64, i32, i32, vp, vp]
             L.dit_gemm_gated_residual.argtypes = [vp, vp, vp, vp, vp, i32, i64, i32, i64, i32,
                                                   i32, vp, vp]
@@ -659,10 +659,12 @@ def subblock_keep_count(n_blocks: int, sparsity: float) -> int:
 
 def subblock_router(q: torch.Tensor, k: torch.Tensor, heads: int, block: int = 128,
                     sparsity: float = 0.75, workspace: Optional[torch.Tensor] = None,
-                    kept: Optional[torch.Tensor] = None) -> torch.Tensor:
+                    kept: Optional[torch.Tensor] = None,
+                    status: Optional[torch.Tensor] = None) -> torch.Tensor:
     """The kept key blocks of every query block: int32 [B, H, n_blocks,
     n_keep], increasing.  q and k are [B, N, H*hd] views (e.g. slices of a
-    fused qkv buffer) sharing one row stride."""
+    fused qkv buffer) sharing one row stride.  ``status`` (int32 CUDA
+    scalar) is set to 1 if a wait of the tensor-core score kernel expired."""
     _need_cuda_bf16("q", q)
     _need_cuda_bf16("k", k)
     B, N, width = q.shape
@@ -688,9 +690,11 @@ def subblock_router(q: torch.Tensor, k: torch.Tensor, heads: int, block: int = 1
     if kept.dtype != torch.int32 or kept.numel() != B * heads * nb * n_keep or \
             not kept.is_contiguous():
         raise ValueError(f"kept must be a contiguous int32 [B, H, {nb}, {n_keep}] tensor")
+    if status is not None and (status.dtype != torch.int32 or not status.is_cuda):
+        raise ValueError("status must be a CUDA int32 tensor")
     _call("dit_subblock_router", q.data_ptr(), k.data_ptr(), rs, B, N, heads, hd, block,
           float(sparsity), kept.data_ptr(), workspace.data_ptr(),
-          workspace.numel() * workspace.element_size(), _stream(q))
+          workspace.numel() * workspace.element_size(), _ptr(status), _stream(q))
     return kept
 
 

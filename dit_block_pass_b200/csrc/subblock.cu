@@ -535,9 +535,11 @@ extern "C" int dit_subblock_keep_count(int64_t n_blocks, double sparsity) {
 extern "C" size_t dit_subblock_workspace_bytes(int B, int64_t N, int H, int hd, int block) {
     if (B < 0 || N < 0 || H < 1 || hd < 1 || block < 1) return 0;
     const int64_t nb = (N + block - 1) / block;
-    // the block means [B, 2, nb, H*hd], then the scores [B, H, nb, nb], fp32
-    return (static_cast<size_t>(B) * 2 * nb * H * hd + static_cast<size_t>(B) * H * nb * nb) *
-           sizeof(float);
+    // the block means [B, 2, nb, H*hd] fp32 (256-byte rounded), then what
+    // the router from means needs
+    const size_t means = static_cast<size_t>(B) * 2 * nb * H * hd * sizeof(float);
+    return ((means + 255) & ~static_cast<size_t>(255)) +
+           dit_subblock_means_workspace_bytes(B, N, H, hd, block);
 }
 
 namespace dit {
@@ -608,6 +610,21 @@ int scores_tc(const float* means, int B, int nb, int H, int hd, float* scores, f
         mha, mla, mhb, mlb, nb, hd, scores, status);
     return launch_status();
 }
+// Scores and selection from block means, in a workspace laid out as
+// dit_subblock_means_workspace_bytes describes.
+int route_means_ws(const float* means, int B, int nb, int H, int hd, int n_keep, int32_t* kept,
+                   void* workspace, int* status, cudaStream_t st) {
+    float* scores = static_cast<float*>(workspace);
+    if (!tc_scores(hd)) return route_from_means(means, B, nb, H, hd, n_keep, kept, scores, st);
+    const size_t sb = round256(static_cast<size_t>(B) * H * nb * nb * sizeof(float));
+    const size_t mb = round256(static_cast<size_t>(B) * 2 * nb * H * hd * sizeof(float));
+    uint8_t* w = static_cast<uint8_t*>(workspace);
+    const int rc = scores_tc(means, B, nb, H, hd, scores, reinterpret_cast<float*>(w + sb),
+                             reinterpret_cast<float*>(w + sb + mb), status, st);
+    if (rc) return rc;
+    return select_kept(scores, B, nb, H, n_keep, kept, st);
+}
+
 }  // namespace
 }  // namespace dit
 
@@ -640,23 +657,14 @@ extern "C" int dit_subblock_router_means(const float* block_means, int B, int64_
     if (!workspace || !aligned16(workspace) ||
         workspace_bytes < dit_subblock_means_workspace_bytes(B, N, H, hd, block))
         return DIT_ERR_WORKSPACE;
-    float* scores = static_cast<float*>(workspace);
-    if (!tc_scores(hd))
-        return route_from_means(block_means, B, nb, H, hd, keep_count(nb, sparsity), kept, scores,
-                                as_stream(stream));
-    const size_t sb = round256(static_cast<size_t>(B) * H * nb * nb * sizeof(float));
-    const size_t mb = round256(static_cast<size_t>(B) * 2 * nb * H * hd * sizeof(float));
-    uint8_t* w = static_cast<uint8_t*>(workspace);
-    int rc = scores_tc(block_means, B, nb, H, hd, scores, reinterpret_cast<float*>(w + sb),
-                       reinterpret_cast<float*>(w + sb + mb), status, as_stream(stream));
-    if (rc) return rc;
-    return select_kept(scores, B, nb, H, keep_count(nb, sparsity), kept, as_stream(stream));
+    return route_means_ws(block_means, B, nb, H, hd, keep_count(nb, sparsity), kept, workspace,
+                          status, as_stream(stream));
 }
 
 extern "C" int dit_subblock_router(const uint16_t* q, const uint16_t* k, int64_t row_stride,
                                    int B, int64_t N, int H, int hd, int block, double sparsity,
                                    int32_t* kept, void* workspace, size_t workspace_bytes,
-                                   void* stream) {
+                                   int* status, void* stream) {
     using namespace dit;
     if (B < 0 || N < 0 || H < 1 || block < 1) return DIT_ERR_SHAPE;
     if (hd < 8 || hd > 256 || hd % 8) return DIT_ERR_SHAPE;
@@ -672,6 +680,7 @@ extern "C" int dit_subblock_router(const uint16_t* q, const uint16_t* k, int64_t
     if (!q || !k || !kept) return DIT_ERR_NULL;
     if (!aligned16(q) || !aligned16(k) || reinterpret_cast<uintptr_t>(kept) % 4)
         return DIT_ERR_ALIGN;
+    if (status && reinterpret_cast<uintptr_t>(status) % 4) return DIT_ERR_ALIGN;
     const size_t need = dit_subblock_workspace_bytes(B, N, H, hd, block);
     if (!workspace || workspace_bytes < need || !aligned16(workspace)) return DIT_ERR_WORKSPACE;
     float* pooled = static_cast<float*>(workspace);
@@ -682,6 +691,7 @@ extern "C" int dit_subblock_router(const uint16_t* q, const uint16_t* k, int64_t
         block, nb, static_cast<int>(D / 8), pooled);
     int rc = launch_status();
     if (rc) return rc;
-    float* scores = pooled + static_cast<int64_t>(B) * 2 * nb * D;
-    return route_from_means(pooled, B, nb, H, hd, n_keep, kept, scores, st);
+    const size_t mb = round256(static_cast<size_t>(B) * 2 * nb * D * sizeof(float));
+    return route_means_ws(pooled, B, nb, H, hd, n_keep, kept,
+                          static_cast<uint8_t*>(workspace) + mb, status, st);
 }

@@ -376,8 +376,11 @@ int dit_gemm_gated_residual(const uint16_t* h, const uint16_t* w, const uint16_t
  *   kept       device int32 [B, H, n_blocks, n_keep]: the kept key blocks of
  *              each query block, in increasing order.
  *   workspace  device, >= dit_subblock_workspace_bytes(...) bytes (the block
- *              means [B, 2, n_blocks, H*hd], then the scores [B, H, n_blocks,
- *              n_blocks], both fp32), 16-byte aligned.
+ *              means [B, 2, n_blocks, H*hd] fp32, then the workspace of
+ *              dit_subblock_router_means), 16-byte aligned.
+ *   status     optional device int, as dit_subblock_router_means.
+ * The scores are taken as dit_subblock_router_means takes them (tensor cores
+ * for hd a multiple of 32).
  * 0 <= sparsity < 1 (else DIT_ERR_VALUE); n_blocks <= 8192.  Which steps use
  * the router (the report: from the 10th) is the caller's choice.
  */
@@ -385,7 +388,7 @@ int dit_subblock_keep_count(int64_t n_blocks, double sparsity);
 size_t dit_subblock_workspace_bytes(int B, int64_t N, int H, int hd, int block);
 int dit_subblock_router(const uint16_t* q, const uint16_t* k, int64_t row_stride, int B,
                         int64_t N, int H, int hd, int block, double sparsity, int32_t* kept,
-                        void* workspace, size_t workspace_bytes, void* stream);
+                        void* workspace, size_t workspace_bytes, int* status, void* stream);
 
 /*
  * The SubBlock router from block means already computed (for example by

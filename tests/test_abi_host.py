@@ -277,14 +277,17 @@ def test_subblock_router_host(lib):
     assert lib.dit_subblock_keep_count(10, 1.0) == E["VALUE"]
     f = lib.dit_subblock_router
     ws = lib.dit_subblock_workspace_bytes(1, 256, 2, 64, 128)
-    assert ws == (2 * 2 * 2 * 64 + 2 * 2 * 2) * 4       # block means, then scores
-    assert f(A, A + 0x1000, 128, 1, 0, 2, 64, 128, 0.75, A + 0x2000, A + 0x3000, ws, None) == 0
-    assert f(A, A + 0x1000, 128, 1, 256, 2, 60, 128, 0.75, A + 0x2000, A + 0x3000, ws, None) == E["SHAPE"]
-    assert f(A, A + 0x1000, 128, 1, 256, 2, 64, 128, 1.0, A + 0x2000, A + 0x3000, ws, None) == E["VALUE"]
-    assert f(A, A + 0x1000, 128, 1, 256, 2, 64, 128, 0.75, A + 0x2000, A + 0x3000, ws - 4, None) == E["WORKSPACE"]
-    assert f(A, None, 128, 1, 256, 2, 64, 128, 0.75, A + 0x2000, A + 0x3000, ws, None) == E["NULL"]
-    assert f(A, A + 0x1000, 120, 1, 256, 2, 64, 128, 0.75, A + 0x2000, A + 0x3000, ws, None) == E["SHAPE"]
-    assert f(A, A + 0x1000, 128, 1, 128 * 8193, 2, 64, 128, 0.75, A + 0x2000, A + 0x3000, ws, None) == E["SHAPE"]
+    # block means (256-byte rounded), then the scores and the split means
+    assert ws == 2048 + lib.dit_subblock_means_workspace_bytes(1, 256, 2, 64, 128)
+    assert lib.dit_subblock_means_workspace_bytes(1, 256, 2, 64, 128) == 256 + 2 * 2048
+    assert lib.dit_subblock_workspace_bytes(1, 256, 2, 48, 128) == 1536 + 32  # fp32 scores only
+    assert f(A, A + 0x1000, 128, 1, 0, 2, 64, 128, 0.75, A + 0x2000, A + 0x3000, ws, None, None) == 0
+    assert f(A, A + 0x1000, 128, 1, 256, 2, 60, 128, 0.75, A + 0x2000, A + 0x3000, ws, None, None) == E["SHAPE"]
+    assert f(A, A + 0x1000, 128, 1, 256, 2, 64, 128, 1.0, A + 0x2000, A + 0x3000, ws, None, None) == E["VALUE"]
+    assert f(A, A + 0x1000, 128, 1, 256, 2, 64, 128, 0.75, A + 0x2000, A + 0x3000, ws - 4, None, None) == E["WORKSPACE"]
+    assert f(A, None, 128, 1, 256, 2, 64, 128, 0.75, A + 0x2000, A + 0x3000, ws, None, None) == E["NULL"]
+    assert f(A, A + 0x1000, 120, 1, 256, 2, 64, 128, 0.75, A + 0x2000, A + 0x3000, ws, None, None) == E["SHAPE"]
+    assert f(A, A + 0x1000, 128, 1, 128 * 8193, 2, 64, 128, 0.75, A + 0x2000, A + 0x3000, ws, None, None) == E["SHAPE"]
 
 
 def test_cachedit_result_buffers_are_checked_before_the_call():

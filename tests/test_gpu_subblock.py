@@ -1,10 +1,13 @@
-"""The SubBlock router on the GPU against the oracle.  Scores are fp32 on
-the GPU and fp64 in the oracle, so where two key blocks' scores lie within
-the fp32 error of the selection threshold either may be kept: the test
-checks that the kept list is valid (n_keep distinct increasing indices) and
-agrees with the oracle's everywhere else.  The bound: the block means sum
-at most `block` bf16 values and the score sums hd products, all in fp32;
-tau = 2^-14 max_j |score_ij| covers both with a wide margin."""
+"""The SubBlock router on the GPU against the oracle.  Scores are fp32 sums
+on the GPU (three tf32 products of split means on the tensor cores for hd a
+multiple of 32, fp32 FMAs otherwise) and fp64 in the oracle, so where two key
+blocks' scores lie within the fp32 error of the selection threshold either may
+be kept: the test checks that the kept list is valid (n_keep distinct
+increasing indices) and agrees with the oracle's everywhere else.  The bound:
+the block means sum at most `block` bf16 values in fp32, and a score carries
+at most about (3 hd / 8) 2^-23 + 3 2^-20 of sum|q_d k_d| (the split-tf32 bound
+checked score by score in test_gpu_qk_pool.py); tau = 2^-14 max_j |score_ij|
+covers both with a wide margin."""
 import numpy as np
 import pytest
 import torch
