@@ -57,7 +57,9 @@ def _qkv(B, N, H, hd, seed):
 @pytest.mark.parametrize("B,N,H,hd,block,sp", [(2, 1000, 3, 64, 128, 0.75), (1, 8192, 4, 128, 128, 0.8),
                                                (2, 77, 2, 32, 16, 0.5), (1, 3000, 2, 128, 64, 0.0),
                                                (1, 4096 * 3 + 5, 2, 64, 8, 0.75),
-                                               (1, 8 * 2100, 1, 32, 8, 0.75)])
+                                               (1, 8 * 2100, 1, 32, 8, 0.75),
+                                               (2, 1000, 3, 40, 16, 0.75),    # fp32 FMA scores
+                                               (1, 1500, 2, 256, 8, 0.8)])    # 8 tf32 chunks
 def test_router_matches_oracle(orc, B, N, H, hd, block, sp):
     qkv = _qkv(B, N, H, hd, N + H)
     D = H * hd
