@@ -24,7 +24,7 @@
 //                           a tf32 high part (low 13 mantissa bits cleared)
 //                           and the remainder.
 //   subblock_scores_tc_kernel  the same scores on the tensor cores: per
-//                           128 query x 64 key block tile, the hi and lo
+//                           128 query x 256 key block tile, the hi and lo
 //                           parts brought by TMA (128-byte swizzle) 32
 //                           head-dimension values at a time through a
 //                           two-slot ring, hi.hi + hi.lo + lo.hi accumulated
@@ -341,10 +341,10 @@ subblock_select_kernel(const float* __restrict__ scores, int nb, int n_keep,
 // split-TF32 method; the dropped lo*lo term and lo's own rounding to TF32 are
 // each below 2^-22 of the product).
 constexpr int kTcM = 128;        // query blocks per tile (TMEM lanes)
-constexpr int kTcN = 64;         // key blocks per tile (TMEM columns)
+constexpr int kTcN = 256;        // key blocks per tile (TMEM columns)
 constexpr int kTcChunk = 32;     // head-dimension values per 128-byte swizzle row
 constexpr int kTcSlots = 2;      // chunks in flight
-constexpr uint32_t kTcSlotBytes = 2 * (kTcM + kTcN) * kTcChunk * 4;   // hi and lo: 48 KB
+constexpr uint32_t kTcSlotBytes = 2 * (kTcM + kTcN) * kTcChunk * 4;   // hi and lo: 96 KB
 constexpr int kTcSmem = kTcSlots * kTcSlotBytes + 1024;
 
 // hi / lo of n fp32 values (n multiple of 4).
@@ -381,17 +381,19 @@ __device__ __forceinline__ void mma_tf32(uint32_t tmem_d, uint64_t da, uint64_t 
         : "memory");
 }
 
-// CTA (tile, h, b): scores[b, h, i0 .. i0+127, j0 .. j0+63].  Warp 0 brings
-// the hi and lo tiles of both operands 32 head-dimension values (one chunk)
-// at a time into a two-slot ring; one thread of warp 1 issues each chunk's
-// 3 x 4 products as soon as it lands and frees its slot with a commit; the
-// four warps read the accumulator (thread = query block), pass their 32
+// CTA (tile, h, b): scores[b, h, i0 .. i0+127, j0 .. j0+255].  Warp 0
+// brings the hi and lo tiles of both operands 32 head-dimension values (one
+// chunk) at a time into a two-slot ring (96 KB a slot, one CTA per SM); one
+// thread of warp 1 issues each chunk's 3 x 4 products (N = 256) as soon as
+// it lands and frees its slot with a commit; the four warps read the
+// accumulator 64 columns at a time (thread = query block), pass their 32
 // rows through shared memory (the ring, free once the products are done)
-// and store them row by row, a warp per 64-score row segment.  Two CTAs
-// share an SM, so one's copies overlap the other's products and stores.
-// Rows past n_blocks are computed on whatever the copy brought (the next
-// group's rows, or zeros past the array) and never stored.
-__global__ void __launch_bounds__(128, 2)
+// and store them row by row, a warp per 64-score row segment.  (128 x 64
+// tiles with two CTAs per SM read the query means four times as often and
+// measured 7 % slower for the whole call.)  Rows past n_blocks are computed
+// on whatever the copy brought (the next group's rows, or zeros past the
+// array) and never stored.
+__global__ void __launch_bounds__(128, 1)
 subblock_scores_tc_kernel(const __grid_constant__ CUtensorMap map_hi_a,
                           const __grid_constant__ CUtensorMap map_lo_a,
                           const __grid_constant__ CUtensorMap map_hi_b,
@@ -405,7 +407,7 @@ subblock_scores_tc_kernel(const __grid_constant__ CUtensorMap map_hi_a,
     const uint32_t base = (raw + 1023u) & ~1023u;
     const int chunks = hd / kTcChunk;
     constexpr uint32_t a_bytes = kTcM * kTcChunk * 4;      // 16 KB
-    constexpr uint32_t b_bytes = kTcN * kTcChunk * 4;      // 8 KB
+    constexpr uint32_t b_bytes = kTcN * kTcChunk * 4;      // 32 KB
     // slot layout: A hi, A lo, B hi, B lo
     const uint32_t bar_full = tc::smem_u32(&s_bar[0]);
     const uint32_t bar_empty = tc::smem_u32(&s_bar[kTcSlots]);
@@ -490,23 +492,30 @@ subblock_scores_tc_kernel(const __grid_constant__ CUtensorMap map_hi_a,
     if (!__all_sync(0xffffffffu, tc::mbar_wait_drain(bar_done, 0))) failed = true;
     if (!failed) {
         tc::fence_after_sync();
-        float v[kTcN];
+        constexpr int kCh = 64;             // columns per epilogue chunk
         const uint32_t lane_addr = tmem + (static_cast<uint32_t>(32 * warp) << 16);
-        tc::tmem_ld32(lane_addr, *reinterpret_cast<float(*)[32]>(v));
-        tc::tmem_ld32(lane_addr + 32, *reinterpret_cast<float(*)[32]>(v + 32));
-        tc::tmem_wait_ld();
-        // the warp's 32 x 64 scores through shared memory, rows kTcN + 1
-        // apart (no bank conflicts either way)
-        float* st = reinterpret_cast<float*>(tc_smem_raw + (base - raw)) + warp * 32 * (kTcN + 1);
-#pragma unroll
-        for (int jj = 0; jj < kTcN; ++jj) st[lane * (kTcN + 1) + jj] = v[jj];
-        __syncwarp();
+        // the warp's 32 x 64 scores of a chunk through shared memory, rows
+        // kCh + 1 apart (no bank conflicts either way)
+        float* st = reinterpret_cast<float*>(tc_smem_raw + (base - raw)) + warp * 32 * (kCh + 1);
         const int rows = nb - (i0 + 32 * warp) < 32 ? nb - (i0 + 32 * warp) : 32;
         float* out = scores + ((static_cast<int64_t>(b) * H + h) * nb + i0 + 32 * warp) * nb + j0;
-        const bool c0 = j0 + lane < nb, c1 = j0 + 32 + lane < nb;
-        for (int r = 0; r < rows; ++r) {
-            if (c0) out[static_cast<int64_t>(r) * nb + lane] = st[r * (kTcN + 1) + lane];
-            if (c1) out[static_cast<int64_t>(r) * nb + 32 + lane] = st[r * (kTcN + 1) + 32 + lane];
+        for (int c = 0; c < kTcN / kCh && j0 + c * kCh < nb; ++c) {
+            float v[kCh];
+            tc::tmem_ld32(lane_addr + c * kCh, *reinterpret_cast<float(*)[32]>(v));
+            tc::tmem_ld32(lane_addr + c * kCh + 32, *reinterpret_cast<float(*)[32]>(v + 32));
+            tc::tmem_wait_ld();
+#pragma unroll
+            for (int jj = 0; jj < kCh; ++jj) st[lane * (kCh + 1) + jj] = v[jj];
+            __syncwarp();
+            const int jc = j0 + c * kCh;
+            const bool c0 = jc + lane < nb, c1 = jc + 32 + lane < nb;
+            for (int r = 0; r < rows; ++r) {
+                if (c0) out[static_cast<int64_t>(r) * nb + c * kCh + lane] = st[r * (kCh + 1) + lane];
+                if (c1)
+                    out[static_cast<int64_t>(r) * nb + c * kCh + 32 + lane] =
+                        st[r * (kCh + 1) + 32 + lane];
+            }
+            __syncwarp();
         }
     }
     if (failed && lane == 0 && status) atomicExch(status, 1);
@@ -582,7 +591,7 @@ size_t round256(size_t n) { return (n + 255) & ~static_cast<size_t>(255); }
 bool tc_scores(int hd) { return hd % kTcChunk == 0; }
 
 // Tensor-core scores: split the means into hi / lo in the workspace, then one
-// CTA per 128 x 64 tile.
+// CTA per 128 x 256 tile.
 int scores_tc(const float* means, int B, int nb, int H, int hd, float* scores, float* hi,
               float* lo, int* status, cudaStream_t st) {
     const int64_t D = static_cast<int64_t>(H) * hd;

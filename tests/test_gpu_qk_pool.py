@@ -166,12 +166,12 @@ def test_pooled_argument_errors():
 
 
 ROUTER_MEANS = [
-    # B, N, H, hd, block, sparsity: several 128 x 64 score tiles with ragged
-    # edges (tensor-core scores for hd a multiple of 32: 1 to 5 chunks
+    # B, N, H, hd, block, sparsity: several 128 x 256 score tiles with ragged
+    # edges (tensor-core scores for hd a multiple of 32: 1 to 8 chunks
     # through the two-slot ring), and hd that takes the fp32 FMA scores (48)
-    (2, 4800, 2, 128, 8, 0.75),      # 600 blocks: 5 x 10 tiles, last 88 x 24
+    (2, 4800, 2, 128, 8, 0.75),      # 600 blocks: 5 x 3 tiles, last 88 x 88
     (1, 2016, 3, 96, 8, 0.8),        # 3 chunks of 32
-    (1, 8 * 2100, 1, 32, 8, 0.75),   # 2,100 blocks (selection past 2,048)
+    (1, 8 * 2100, 1, 32, 8, 0.75),   # 2,100 blocks: 17 x 9 tiles (selection past 2,048)
     (2, 1000, 2, 64, 16, 0.5),       # 63 blocks: one ragged tile
     (1, 3000, 2, 48, 16, 0.75),
     (1, 1500, 1, 160, 8, 0.75),      # 5 chunks
