@@ -10,29 +10,31 @@
 // product of the two means and keeps the n_keep = ceil((1 - s) n_blocks)
 // best key blocks (ties to the lower index), listed in increasing order.
 //
-// Three kernels:
+// Kernels (the router on q and k pools, then scores and selects; the router
+// from means, fed by the QK operator, starts at the scores):
 //   subblock_pool_kernel    one pass over q and k (HBM bound): CTA (j, b, t,
 //                           column chunk) sums the rows of block j of sample
 //                           b of tensor t (q or k), a 16-byte column vector
 //                           per thread, fp32, and writes the means
-//                           [B, 2, n_blocks, H*hd].
-//   subblock_scores_kernel  per (sample, head) the n_blocks x n_blocks fp32
-//                           scores as a tiled GEMM of the L2-resident means
-//                           (128 x 128 tiles, 8 x 8 per thread), into the
-//                           workspace after the means.
-//   tf32_split_kernel       for the router from means: each mean split into
-//                           a tf32 high part (low 13 mantissa bits cleared)
+//                           [B, 2, n_blocks, H*hd] at the workspace's start.
+//   tf32_split_kernel       for hd a multiple of 32: each mean split into a
+//                           tf32 high part (low 13 mantissa bits cleared)
 //                           and the remainder.
-//   subblock_scores_tc_kernel  the same scores on the tensor cores: per
-//                           128 query x 256 key block tile, the hi and lo
-//                           parts brought by TMA (128-byte swizzle) 32
-//                           head-dimension values at a time through a
-//                           two-slot ring, hi.hi + hi.lo + lo.hi accumulated
-//                           in TMEM by kind::tf32 products.
+//   subblock_scores_tc_kernel  per (sample, head) the n_blocks x n_blocks
+//                           scores on the tensor cores: per 128 query x 256
+//                           key block tile, the hi and lo parts brought by
+//                           TMA (128-byte swizzle) 32 head-dimension values
+//                           at a time through a two-slot ring, hi.hi +
+//                           hi.lo + lo.hi accumulated in TMEM by kind::tf32
+//                           products.
+//   subblock_scores_kernel  the same scores for other head sizes, as a tiled
+//                           fp32 GEMM of the L2-resident means (128 x 128
+//                           tiles, 8 x 8 per thread).
 //   subblock_select_kernel  one warp per query block: the n_keep-th largest
 //                           score of its row found bit by bit with warp-wide
 //                           counts (the row in registers up to 2048 key
-//                           blocks) and an ordered ballot compaction that
+//                           blocks; the last candidates gathered one per
+//                           lane) and an ordered ballot compaction that
 //                           writes the kept indices in increasing order,
 //                           ties at the threshold to the lower index.
 #include <cmath>
