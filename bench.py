@@ -20,7 +20,11 @@ the data path has no collective) and the line also carries `sharded_clip`:
 one clip sequence-sharded across the ranks, with the Cache-DiT all-gather
 inside the step (strong scaling).  --shard makes the sharded clip the
 headline.  The line also times the 10 s clip and the CFG pair with joint
-audio (`configs`) outside the headline's timed region.
+audio (`configs`) outside the headline's timed region, and `e2e`: the same
+chain through the public API with every step's inputs copied in from pinned
+host memory and every output read back, two device buffer sets alternating
+over three streams (copies in, chain, copies out) so both copy directions
+overlap each other and the compute.
 """
 from __future__ import annotations
 
