@@ -632,7 +632,7 @@ def tensor_peaks():
         return 1590.0, 1400.0, "fallback"
 
 
-def time_e2e(chain, steps, warmup, world):
+def time_e2e(chain, steps, warmup, world, keep_outputs=False):
     """The same chain through the public API with inputs on the host: every
     step copies all of its inputs host->device from pinned memory, runs the
     chain and reads every output back device->host.  Two device buffer sets
@@ -642,7 +642,8 @@ def time_e2e(chain, steps, warmup, world):
     both directions at once); a set is refilled only after its outputs have
     been read back.  The timed region runs from the first timed step's first
     copy in to the last one's last copy out.  Returns (ms per step, h2d bytes,
-    d2h bytes)."""
+    d2h bytes), and with keep_outputs the host inputs and the last step's host
+    outputs by name as well."""
     import copy
 
     import torch
@@ -701,8 +702,11 @@ def time_e2e(chain, steps, warmup, world):
     torch.cuda.synchronize()
     barrier_sync(world)
     ms = max_over_ranks(a.elapsed_time(b), world) / steps
+    kept = (dict(zip(names_in, host_in)), dict(zip(names_out, host_out))) if keep_outputs else None
     del host_in, host_out, c2, sets, ops
     torch.cuda.empty_cache()
+    if keep_outputs:
+        return ms, h2d, d2h, kept[0], kept[1]
     return ms, h2d, d2h
 
 
