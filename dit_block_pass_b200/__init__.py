@@ -122,6 +122,8 @@ def library() -> ctypes.CDLL:
             L.dit_subblock_router.argtypes = [vp, vp, i64, i32, i64, i32, i32, i32, dbl, vp, vp,
                                               sz, vp, vp]
             L.dit_swiglu_gemm_stall_test.argtypes = [vp, vp, vp, i64, i32, i32, vp, vp]
+            L.dit_subblock_scores_stall_test.argtypes = [vp, i32, i64, i32, i32, i32, vp, sz, vp,
+                                                         vp]
             L.dit_gemm_gated_residual.argtypes = [vp, vp, vp, vp, vp, i32, i64, i32, i64, i32,
                                                   i32, vp, vp]
             L.cachedit_residual_store.argtypes = [vp, vp, vp, i64, vp]
@@ -139,7 +141,7 @@ def library() -> ctypes.CDLL:
                          "dit_adaln_modulate_tok", "dit_gated_residual_adaln_tok",
                          "cachedit_residual_store", "cachedit_residual_apply", "dit_swiglu_gemm",
                          "dit_gemm_gated_residual", "dit_subblock_keep_count",
-                         "dit_swiglu_gemm_stall_test",
+                         "dit_swiglu_gemm_stall_test", "dit_subblock_scores_stall_test",
                          "dit_subblock_router", "dit_block_sparse_attention",
                          "dit_cache_policy_init", "dit_cache_policy_decide",
                          "dit_qk_rmsnorm_rope3d", "dit_qk_rmsnorm_rope3d_ex",

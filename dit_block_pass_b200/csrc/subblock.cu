@@ -400,7 +400,7 @@ subblock_scores_tc_kernel(const __grid_constant__ CUtensorMap map_hi_a,
                           const __grid_constant__ CUtensorMap map_lo_a,
                           const __grid_constant__ CUtensorMap map_hi_b,
                           const __grid_constant__ CUtensorMap map_lo_b, int nb, int hd,
-                          float* __restrict__ scores, int* status) {
+                          float* __restrict__ scores, int* status, int stall) {
     extern __shared__ uint8_t tc_smem_raw[];
     __shared__ uint64_t s_bar[2 * kTcSlots + 1];
     __shared__ uint32_t s_tmem;
@@ -433,7 +433,8 @@ subblock_scores_tc_kernel(const __grid_constant__ CUtensorMap map_hi_a,
         if (lane == 0) {
             const int qrow = (b * 2 + 0) * nb + i0, krow = (b * 2 + 1) * nb + j0;
             int issued = 0;
-            for (int c = 0; c < chunks; ++c) {
+            // stall (a test hook): no copy is issued, so every wait runs out
+            for (int c = 0; c < chunks && !stall; ++c) {
                 const int slot = c % kTcSlots;
                 if (c >= kTcSlots &&
                     !tc::mbar_wait(bar_empty + 8 * slot, ((c / kTcSlots) - 1) & 1, &s_abort)) {
@@ -595,7 +596,7 @@ bool tc_scores(int hd) { return hd % kTcChunk == 0; }
 // Tensor-core scores: split the means into hi / lo in the workspace, then one
 // CTA per 128 x 256 tile.
 int scores_tc(const float* means, int B, int nb, int H, int hd, float* scores, float* hi,
-              float* lo, int* status, cudaStream_t st) {
+              float* lo, int* status, cudaStream_t st, int stall = 0) {
     const int64_t D = static_cast<int64_t>(H) * hd;
     const int64_t rows = static_cast<int64_t>(B) * 2 * nb;
     const int64_t n4 = rows * D / 4;
@@ -618,7 +619,7 @@ int scores_tc(const float* means, int B, int nb, int H, int hd, float* scores, f
         return DIT_ERR_LAUNCH;
     const int64_t tiles = static_cast<int64_t>((nb + kTcM - 1) / kTcM) * ((nb + kTcN - 1) / kTcN);
     subblock_scores_tc_kernel<<<dim3(static_cast<unsigned>(tiles), H, B), 128, smem, st>>>(
-        mha, mla, mhb, mlb, nb, hd, scores, status);
+        mha, mla, mhb, mlb, nb, hd, scores, status, stall);
     return launch_status();
 }
 // Scores and selection from block means, in a workspace laid out as
@@ -670,6 +671,28 @@ extern "C" int dit_subblock_router_means(const float* block_means, int B, int64_
         return DIT_ERR_WORKSPACE;
     return route_means_ws(block_means, B, nb, H, hd, keep_count(nb, sparsity), kept, workspace,
                           status, as_stream(stream));
+}
+
+extern "C" int dit_subblock_scores_stall_test(const float* block_means, int B, int64_t N, int H,
+                                              int hd, int block, void* workspace,
+                                              size_t workspace_bytes, int* status, void* stream) {
+    using namespace dit;
+    if (B < 1 || N < 1 || H < 1 || block < 1 || !tc_scores(hd)) return DIT_ERR_SHAPE;
+    if (static_cast<int64_t>(H) * hd > DIT_MAX_D) return DIT_ERR_SHAPE;
+    const int64_t nb64 = (N + block - 1) / block;
+    if (nb64 > 512 || B > 4) return DIT_ERR_SHAPE;        // small shapes only
+    const int nb = static_cast<int>(nb64);
+    if (!block_means || !status) return DIT_ERR_NULL;
+    if (!aligned16(block_means) || reinterpret_cast<uintptr_t>(status) % 4) return DIT_ERR_ALIGN;
+    if (!workspace || !aligned16(workspace) ||
+        workspace_bytes < dit_subblock_means_workspace_bytes(B, N, H, hd, block))
+        return DIT_ERR_WORKSPACE;
+    const size_t sb = round256(static_cast<size_t>(B) * H * nb * nb * sizeof(float));
+    const size_t mb = round256(static_cast<size_t>(B) * 2 * nb * H * hd * sizeof(float));
+    uint8_t* w = static_cast<uint8_t*>(workspace);
+    return scores_tc(block_means, B, nb, H, hd, reinterpret_cast<float*>(w),
+                     reinterpret_cast<float*>(w + sb), reinterpret_cast<float*>(w + sb + mb),
+                     status, as_stream(stream), 1);
 }
 
 extern "C" int dit_subblock_router(const uint16_t* q, const uint16_t* k, int64_t row_stride,

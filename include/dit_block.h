@@ -415,6 +415,19 @@ int dit_subblock_router_means(const float* block_means, int B, int64_t N, int H,
                               size_t workspace_bytes, int* status, void* stream);
 
 /*
+ * Test hook for the failure path of the tensor-core score kernel: the split
+ * and the score launch of dit_subblock_router_means with the kernel's copy
+ * thread issuing nothing, so that every wait runs out (after about 2 s) and
+ * the kernel writes 1 to *status, frees its tensor memory and returns,
+ * leaving the context usable; the scores are left unwritten and nothing is
+ * selected.  hd a multiple of 32, B <= 4, n_blocks <= 512; status is
+ * required.  Not for production use.
+ */
+int dit_subblock_scores_stall_test(const float* block_means, int B, int64_t N, int H, int hd,
+                                   int block, void* workspace, size_t workspace_bytes,
+                                   int* status, void* stream);
+
+/*
  * Block-sparse attention over the router's kept key blocks (tensor cores):
  * for token t of query block i, head h,
  *     out[t, h] = sum_u softmax_u(scale * q[t, h] . k[u, h]) v[u, h]

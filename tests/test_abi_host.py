@@ -288,6 +288,13 @@ def test_subblock_router_host(lib):
     assert f(A, None, 128, 1, 256, 2, 64, 128, 0.75, A + 0x2000, A + 0x3000, ws, None, None) == E["NULL"]
     assert f(A, A + 0x1000, 120, 1, 256, 2, 64, 128, 0.75, A + 0x2000, A + 0x3000, ws, None, None) == E["SHAPE"]
     assert f(A, A + 0x1000, 128, 1, 128 * 8193, 2, 64, 128, 0.75, A + 0x2000, A + 0x3000, ws, None, None) == E["SHAPE"]
+    # the score kernel's stall hook refuses what it does not test, before any launch
+    g = lib.dit_subblock_scores_stall_test
+    mws = lib.dit_subblock_means_workspace_bytes(1, 256, 2, 64, 128)
+    assert g(A, 1, 256, 2, 64, 128, A + 0x2000, mws, None, None) == E["NULL"]           # status
+    assert g(A, 1, 256, 2, 48, 128, A + 0x2000, mws, A + 0x100, None) == E["SHAPE"]      # FMA path
+    assert g(A, 1, 256 * 1024, 2, 64, 8, A + 0x2000, mws, A + 0x100, None) == E["SHAPE"]  # too big
+    assert g(A, 1, 256, 2, 64, 128, A + 0x2000, mws - 16, A + 0x100, None) == E["WORKSPACE"]
 
 
 def test_cachedit_result_buffers_are_checked_before_the_call():

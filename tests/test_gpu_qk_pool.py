@@ -229,3 +229,32 @@ def test_router_means_workspace_sizes():
     big = L.dit_subblock_means_workspace_bytes(2, 1000, 3, 64, 16)
     assert big >= scores + 2 * (2 * 2 * nb * 3 * 64 * 4)
     assert L.dit_subblock_means_workspace_bytes(2, 1000, 3, 64, 0) == 0
+
+
+def test_router_scores_expired_wait_is_reported_and_the_context_survives(orc):
+    """Failure path of the tensor-core score kernel: with its copy thread
+    issuing nothing (test hook) every wait runs out after its 2 s bound; the
+    kernel reports through the status word, frees its tensor memory and
+    returns, and the router works in the same context afterwards."""
+    B, N, H, hd, block = 1, 1024, 2, 64, 64
+    D = H * hd
+    g = torch.Generator().manual_seed(5)
+    x = torch.randn(B * N, 2 * D, generator=g).to(torch.bfloat16)
+    xb = bits(x)
+    m, _, _ = _means64(xb, orc, B, N, block)
+    gm = torch.from_numpy(np.stack([m[:, :, :D], m[:, :, D:]], axis=1).astype(np.float32)).to(DEV)
+    L = dbp.library()
+    need = int(L.dit_subblock_means_workspace_bytes(B, N, H, hd, block))
+    ws = torch.empty(need, dtype=torch.uint8, device=DEV)
+    st = torch.zeros(1, dtype=torch.int32, device=DEV)
+    rc = L.dit_subblock_scores_stall_test(gm.data_ptr(), B, N, H, hd, block, ws.data_ptr(), need,
+                                          st.data_ptr(), torch.cuda.current_stream().cuda_stream)
+    assert rc == 0
+    torch.cuda.synchronize()
+    assert int(st.item()) == 1
+    st.zero_()
+    kept = dbp.subblock_router_means(gm, N, H, block, 0.75, status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    ref, S = orc.subblock_router(xb[:, :D], xb[:, D:], B, H, hd, block, 0.75)
+    _check_rows(kept.cpu().numpy(), ref, S, ref.shape[-1], "after the stall")
