@@ -116,6 +116,9 @@ def library() -> ctypes.CDLL:
             L.dit_swiglu_gemm.argtypes = [vp, vp, vp, i64, i32, i32, vp, vp]
             L.dit_block_sparse_attention.argtypes = [vp, vp, vp, i64, vp, i64, i32, i64, i32,
                                                      i32, i32, vp, i32, dbl, vp, vp]
+            L.dit_block_sparse_attention_stall_test.argtypes = [vp, vp, vp, i64, vp, i64, i32,
+                                                                i64, i32, i32, i32, vp, i32,
+                                                                dbl, vp, vp]
             L.dit_subblock_keep_count.argtypes = [i64, dbl]
             L.dit_subblock_workspace_bytes.argtypes = [i32, i64, i32, i32, i32]
             L.dit_subblock_workspace_bytes.restype = sz
@@ -142,6 +145,7 @@ def library() -> ctypes.CDLL:
                          "cachedit_residual_store", "cachedit_residual_apply", "dit_swiglu_gemm",
                          "dit_gemm_gated_residual", "dit_subblock_keep_count",
                          "dit_swiglu_gemm_stall_test", "dit_subblock_scores_stall_test",
+                         "dit_block_sparse_attention_stall_test",
                          "dit_subblock_router", "dit_block_sparse_attention",
                          "dit_cache_policy_init", "dit_cache_policy_decide",
                          "dit_qk_rmsnorm_rope3d", "dit_qk_rmsnorm_rope3d_ex",

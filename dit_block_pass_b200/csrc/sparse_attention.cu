@@ -172,6 +172,7 @@ struct AttnParams {
     int64_t N;
     int H, nb, n_keep;
     float scale_log2;           // scale * log2(e)
+    int stall;                  // test hook: the copy warps issue nothing, every wait runs out
 };
 
 // Keys of step h that exist: the sample's tokens of kept block kept[h/2],
@@ -244,7 +245,7 @@ block_sparse_attention_kernel(const __grid_constant__ CUtensorMap map_q,
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsLow));
     const int col = h * kHd;
     if (warp == 0) {
-        if (lane == 0) {
+        if (lane == 0 && !p.stall) {
             // Q once, then the K half-tile of every step into the 3-slot ring
             mbar_expect_tx(bar_q, kTile);
             tma_load_2d(sQ, &map_q, bar_q, col, row0 + i * kBlk);
@@ -271,7 +272,7 @@ block_sparse_attention_kernel(const __grid_constant__ CUtensorMap map_q,
         }
         __syncwarp();
     } else if (warp == 2) {
-        if (lane == 0) {
+        if (lane == 0 && !p.stall) {
             // the V half-tile of every step into the 2-slot ring
             int issued = 0;
             for (int st = 0; st < steps; ++st) {
@@ -472,15 +473,10 @@ block_sparse_attention_kernel(const __grid_constant__ CUtensorMap map_q,
     if (warp == 1) tmem_dealloc(tmem, kTmemColsA);
 }
 
-}  // namespace
-}  // namespace dit
-
-extern "C" int dit_block_sparse_attention(const uint16_t* q, const uint16_t* k, const uint16_t* v,
-                                          int64_t row_stride, uint16_t* out, int64_t out_stride,
-                                          int B, int64_t N, int H, int hd, int block,
-                                          const int32_t* kept, int n_keep, double scale,
-                                          int* status, void* stream) {
-    using namespace dit;
+int sparse_attention(const uint16_t* q, const uint16_t* k, const uint16_t* v, int64_t row_stride,
+                     uint16_t* out, int64_t out_stride, int B, int64_t N, int H, int hd,
+                     int block, const int32_t* kept, int n_keep, double scale, int* status,
+                     void* stream, int stall) {
     if (B < 0 || N < 0 || H < 1 || n_keep < 1) return DIT_ERR_SHAPE;
     if (hd != kHd || block != kBlk) return DIT_ERR_SHAPE;
     const int64_t D = static_cast<int64_t>(H) * hd;
@@ -516,6 +512,7 @@ extern "C" int dit_block_sparse_attention(const uint16_t* q, const uint16_t* k, 
     p.nb = static_cast<int>(nb);
     p.n_keep = n_keep;
     p.scale_log2 = static_cast<float>(scale * 1.4426950408889634);
+    p.stall = stall;
     // the register split inside the kernel assumes the launch count it was
     // sized for; any other count could make setmaxnreg.inc wait forever
     cudaFuncAttributes fa{};
@@ -529,4 +526,28 @@ extern "C" int dit_block_sparse_attention(const uint16_t* q, const uint16_t* k, 
     block_sparse_attention_kernel<<<dim3(static_cast<unsigned>(nb), H, B), kThreadsA, kSmemA,
                                     as_stream(stream)>>>(mq, mk, mv, p);
     return launch_status();
+}
+
+}  // namespace
+}  // namespace dit
+
+extern "C" int dit_block_sparse_attention(const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                                          int64_t row_stride, uint16_t* out, int64_t out_stride,
+                                          int B, int64_t N, int H, int hd, int block,
+                                          const int32_t* kept, int n_keep, double scale,
+                                          int* status, void* stream) {
+    return dit::sparse_attention(q, k, v, row_stride, out, out_stride, B, N, H, hd, block, kept,
+                                 n_keep, scale, status, stream, 0);
+}
+
+extern "C" int dit_block_sparse_attention_stall_test(const uint16_t* q, const uint16_t* k,
+                                                     const uint16_t* v, int64_t row_stride,
+                                                     uint16_t* out, int64_t out_stride, int B,
+                                                     int64_t N, int H, int hd, int block,
+                                                     const int32_t* kept, int n_keep,
+                                                     double scale, int* status, void* stream) {
+    if (!status) return DIT_ERR_NULL;
+    if (B < 1 || N < 1 || B * N > 1024 || H > 4) return DIT_ERR_SHAPE;      // small shapes only
+    return dit::sparse_attention(q, k, v, row_stride, out, out_stride, B, N, H, hd, block, kept,
+                                 n_keep, scale, status, stream, 1);
 }

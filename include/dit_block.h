@@ -452,6 +452,20 @@ int dit_block_sparse_attention(const uint16_t* q, const uint16_t* k, const uint1
                                int* status, void* stream);
 
 /*
+ * Test hook for the failure path of the block-sparse attention kernel: the
+ * same launch as dit_block_sparse_attention with its copy warps issuing
+ * nothing, so that every wait runs out (after about 2 s) and the kernel
+ * writes 1 to *status, frees its tensor memory and returns, leaving the
+ * context usable; out is left unwritten.  B*N <= 1024, H <= 4; status is
+ * required.  Not for production use.
+ */
+int dit_block_sparse_attention_stall_test(const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                                          int64_t row_stride, uint16_t* out, int64_t out_stride,
+                                          int B, int64_t N, int H, int hd, int block,
+                                          const int32_t* kept, int n_keep, double scale,
+                                          int* status, void* stream);
+
+/*
  * Cache-DiT step cache.  The LMSYS report (news.cocoloop.cn,
  * "minimax-h3-sglang-h200", section "Só com três camadas de aceleração
  * somadas chega-se a 6 vezes") reuses results cached between neighbouring

@@ -131,3 +131,39 @@ def test_attention_errors():
     assert L.dit_block_sparse_attention(q.data_ptr(), k.data_ptr(), v.data_ptr(), 768,
                                         x.data_ptr(), 768, 1, 256, 2, 128, 128, kept.data_ptr(),
                                         1, 0.1, None, None) == -7          # out over the inputs
+
+
+def test_an_expired_wait_is_reported_and_the_context_survives(orc):
+    """Failure path: with the copy warps issuing nothing (test hook) every
+    wait of the pipeline runs out after its 2 s bound; the kernel reports
+    through the status word, frees its tensor memory and returns, and the
+    next launch in the same context is correct."""
+    B, N, H = 1, 256, 1
+    D = H * HD
+    g = torch.Generator().manual_seed(3)
+    qkv = torch.randn(B, N, 3 * D, generator=g).to(torch.bfloat16)
+    x = qkv.to(DEV)
+    q, k, v = x[:, :, :D], x[:, :, D:2 * D], x[:, :, 2 * D:]
+    kept = dbp.subblock_router(k, k, H, 128, 0.5)
+    out = torch.zeros(B, N, D, dtype=torch.bfloat16, device=DEV)
+    st = torch.zeros(1, dtype=torch.int32, device=DEV)
+    L = dbp.library()
+    rc = L.dit_block_sparse_attention_stall_test(
+        q.data_ptr(), k.data_ptr(), v.data_ptr(), 3 * D, out.data_ptr(), D, B, N, H, HD, 128,
+        kept.data_ptr(), kept.shape[-1], HD ** -0.5, st.data_ptr(),
+        torch.cuda.current_stream().cuda_stream)
+    assert rc == 0
+    torch.cuda.synchronize()
+    assert int(st.item()) == 1
+    assert L.dit_block_sparse_attention_stall_test(
+        q.data_ptr(), k.data_ptr(), v.data_ptr(), 3 * D, out.data_ptr(), D, B, N, H, HD, 128,
+        kept.data_ptr(), kept.shape[-1], HD ** -0.5, None, None) == -1     # status required
+    st.zero_()
+    good = dbp.block_sparse_attention(q, k, v, H, kept, status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    flat = bits(qkv.view(B * N, 3 * D))
+    ref = orc.block_sparse_attention(flat[:, :D], flat[:, D:2 * D], flat[:, 2 * D:], B, H, HD,
+                                     128, kept.cpu().numpy())
+    got = orc.bf16_to_f64(bits(good.view(B * N, D)))
+    assert np.abs(got - ref).max() < 0.02
