@@ -109,6 +109,9 @@ def library() -> ctypes.CDLL:
             L.dit_qk_rmsnorm_rope3d_pooled.argtypes = [vp, vp, i64, vp, vp, i32, i32, i64, i32,
                                                        i32, i32, i32, i32, vp, i64, i32, i32,
                                                        i32, dbl, dbl, i32, i32, vp, vp, vp]
+            L.dit_qk_rmsnorm_rope3d_pooled_stall_test.argtypes = [
+                vp, vp, i64, vp, vp, i32, i32, i64, i32, i32, i32, i32, i32, vp, i64, i32, i32,
+                i32, dbl, dbl, i32, i32, vp, vp, vp]
             L.dit_subblock_means_workspace_bytes.argtypes = [i32, i64, i32, i32, i32]
             L.dit_subblock_means_workspace_bytes.restype = sz
             L.dit_subblock_router_means.argtypes = [vp, i32, i64, i32, i32, i32, dbl, vp, vp, sz,
@@ -146,6 +149,7 @@ def library() -> ctypes.CDLL:
                          "dit_gemm_gated_residual", "dit_subblock_keep_count",
                          "dit_swiglu_gemm_stall_test", "dit_subblock_scores_stall_test",
                          "dit_block_sparse_attention_stall_test",
+                         "dit_qk_rmsnorm_rope3d_pooled_stall_test",
                          "dit_subblock_router", "dit_block_sparse_attention",
                          "dit_cache_policy_init", "dit_cache_policy_decide",
                          "dit_qk_rmsnorm_rope3d", "dit_qk_rmsnorm_rope3d_ex",

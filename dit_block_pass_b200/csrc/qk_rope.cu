@@ -665,7 +665,8 @@ __device__ __forceinline__ void token_pos(const QKParams& p, int64_t tok, int& t
 
 template <int HD, int LAYOUT, int V>
 __global__ void __launch_bounds__(kPoolWarps * 32, 4)
-qk_rope_pool_kernel(QKParams p, int block, int nb, float* __restrict__ means, int* status) {
+qk_rope_pool_kernel(QKParams p, int block, int nb, float* __restrict__ means, int* status,
+                    int stall) {
     constexpr int LPH = HD / 8;             // lanes per head
     constexpr int HALF = LPH / 2;
     constexpr int NP = LAYOUT == 0 ? 4 : 8; // rotation pairs per lane
@@ -704,7 +705,7 @@ qk_rope_pool_kernel(QKParams p, int block, int nb, float* __restrict__ means, in
     __syncwarp();
     // token t's q and k slices into stage s (lane 0)
     auto issue = [&](int t, int s) {
-        if (lane == 0 && t < hi) {
+        if (lane == 0 && t < hi && !stall) {       // stall: a test hook, no copy goes out
             const int64_t row = row0 + t;
             tc::mbar_expect_tx(bars + 8 * s, 2 * chunk);
             bulk_g2s(ring + s * kStage, p.t0 + row * p.stride_v + vbase, chunk, bars + 8 * s);
@@ -869,8 +870,9 @@ qk_rope_pool_kernel(QKParams p, int block, int nb, float* __restrict__ means, in
     if (failed) {
         s_abort = 1;
         if (status) atomicExch(status, 1);
-        // the copies this warp issued land before the CTA exits
-        if (lane == 0) {
+        // the copies this warp issued land before the CTA exits (none when
+        // stalled)
+        if (lane == 0 && !stall) {
             for (int t = done; t < hi && t < done + kPoolStages; ++t) {
                 const int k = t - lo;
                 tc::mbar_wait_drain(bars + 8 * (k % kPoolStages), (k / kPoolStages) & 1);
@@ -914,7 +916,7 @@ qk_rope_pool_kernel(QKParams p, int block, int nb, float* __restrict__ means, in
     }
 }
 
-using PoolKernel = void (*)(QKParams, int, int, float*, int*);
+using PoolKernel = void (*)(QKParams, int, int, float*, int*, int);
 
 template <int LAYOUT>
 PoolKernel pick_pool(int hd) {
@@ -1210,14 +1212,14 @@ extern "C" int dit_qk_rmsnorm_rope3d(uint16_t* q, uint16_t* k, int64_t row_strid
                                     DIT_ROPE_INTERLEAVED, DIT_NORM_HEAD, nullptr, stream);
 }
 
-extern "C" int dit_qk_rmsnorm_rope3d_pooled(uint16_t* q, uint16_t* k, int64_t row_stride,
-                                            const void* w_q, const void* w_k, int w_dtype, int B,
-                                            int64_t N, int H, int hd, int T, int Hg, int Wg,
-                                            const int32_t* pos, int64_t pos_offset, int pairs_t,
-                                            int pairs_h, int pairs_w, double theta, double eps,
-                                            int rope_layout, int block, float* block_means,
-                                            int* status, void* stream) {
-    using namespace dit;
+namespace dit {
+namespace {
+
+int qk_pooled(uint16_t* q, uint16_t* k, int64_t row_stride, const void* w_q, const void* w_k,
+              int w_dtype, int B, int64_t N, int H, int hd, int T, int Hg, int Wg,
+              const int32_t* pos, int64_t pos_offset, int pairs_t, int pairs_h, int pairs_w,
+              double theta, double eps, int rope_layout, int block, float* block_means,
+              int* status, void* stream, int stall) {
     if (w_dtype != DIT_F32 && w_dtype != DIT_BF16) return DIT_ERR_DTYPE;
     if (B < 0 || N < 0 || H < 1 || block < 1) return DIT_ERR_SHAPE;
     if (hd != 32 && hd != 64 && hd != 128 && hd != 256) return DIT_ERR_SHAPE;
@@ -1284,6 +1286,33 @@ extern "C" int dit_qk_rmsnorm_rope3d_pooled(uint16_t* q, uint16_t* k, int64_t ro
                              static_cast<int>(smem)) != cudaSuccess)
         return DIT_ERR_LAUNCH;
     kern<<<dim3(groups, static_cast<unsigned>(nb), B), kPoolWarps * 32, smem,
-           as_stream(stream)>>>(p, block, static_cast<int>(nb), block_means, status);
+           as_stream(stream)>>>(p, block, static_cast<int>(nb), block_means, status, stall);
     return launch_status();
+}
+
+}  // namespace
+}  // namespace dit
+
+extern "C" int dit_qk_rmsnorm_rope3d_pooled(uint16_t* q, uint16_t* k, int64_t row_stride,
+                                            const void* w_q, const void* w_k, int w_dtype, int B,
+                                            int64_t N, int H, int hd, int T, int Hg, int Wg,
+                                            const int32_t* pos, int64_t pos_offset, int pairs_t,
+                                            int pairs_h, int pairs_w, double theta, double eps,
+                                            int rope_layout, int block, float* block_means,
+                                            int* status, void* stream) {
+    return dit::qk_pooled(q, k, row_stride, w_q, w_k, w_dtype, B, N, H, hd, T, Hg, Wg, pos,
+                          pos_offset, pairs_t, pairs_h, pairs_w, theta, eps, rope_layout, block,
+                          block_means, status, stream, 0);
+}
+
+extern "C" int dit_qk_rmsnorm_rope3d_pooled_stall_test(
+    uint16_t* q, uint16_t* k, int64_t row_stride, const void* w_q, const void* w_k, int w_dtype,
+    int B, int64_t N, int H, int hd, int T, int Hg, int Wg, const int32_t* pos,
+    int64_t pos_offset, int pairs_t, int pairs_h, int pairs_w, double theta, double eps,
+    int rope_layout, int block, float* block_means, int* status, void* stream) {
+    if (!status) return DIT_ERR_NULL;
+    if (B < 1 || N < 1 || static_cast<int64_t>(B) * N > 4096) return DIT_ERR_SHAPE;
+    return dit::qk_pooled(q, k, row_stride, w_q, w_k, w_dtype, B, N, H, hd, T, Hg, Wg, pos,
+                          pos_offset, pairs_t, pairs_h, pairs_w, theta, eps, rope_layout, block,
+                          block_means, status, stream, 1);
 }

@@ -263,6 +263,22 @@ int dit_qk_rmsnorm_rope3d_pooled(uint16_t* q, uint16_t* k, int64_t row_stride,
                                  float* block_means, int* status, void* stream);
 
 /*
+ * Test hook for the failure path of dit_qk_rmsnorm_rope3d_pooled: the same
+ * launch with no copy issued, so that every wait of the copy ring runs out
+ * (after about 2 s) and the kernel writes 1 to *status and returns, leaving
+ * the context usable; q, k and the means are left unwritten.  B*N <= 4096;
+ * status is required.  Not for production use.
+ */
+int dit_qk_rmsnorm_rope3d_pooled_stall_test(uint16_t* q, uint16_t* k, int64_t row_stride,
+                                            const void* w_q, const void* w_k, int w_dtype,
+                                            int B, int64_t N, int H, int hd,
+                                            int T, int Hg, int Wg, const int32_t* pos,
+                                            int64_t pos_offset, int pairs_t, int pairs_h,
+                                            int pairs_w, double theta, double eps,
+                                            int rope_layout, int block, float* block_means,
+                                            int* status, void* stream);
+
+/*
  * Cache-DiT residual-difference check between neighbouring denoising steps.
  *   Per sample b:  rel_b   = sum_{n,d} |cur - prev| / sum_{n,d} |prev|
  *                  reuse_b = rel_b < threshold       (strict)

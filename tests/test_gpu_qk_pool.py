@@ -258,3 +258,40 @@ def test_router_scores_expired_wait_is_reported_and_the_context_survives(orc):
     assert int(st.item()) == 0
     ref, S = orc.subblock_router(xb[:, :D], xb[:, D:], B, H, hd, block, 0.75)
     _check_rows(kept.cpu().numpy(), ref, S, ref.shape[-1], "after the stall")
+
+
+def test_pooled_expired_wait_is_reported_and_the_context_survives(orc):
+    """Failure path of the QK operator with block means: with no copy issued
+    (test hook) every wait of the copy ring runs out after its 2 s bound; the
+    kernel reports through the status word and returns without touching q, k
+    or the means, and the next launch in the same context is correct."""
+    wl = W.Workload("stall", B=1, T=2, Hg=4, Wg=6, D=4 * 64, H=4, hd=64, F=8, pairs=(12, 10, 10))
+    N, D = wl.N, wl.D
+    qkv_h = W.token_rows(wl, W.S_QKV, 3 * D)
+    wq, wk = W.norm_weights(wl)
+    x = qkv_h.to(DEV).view(1, N, 3 * D)
+    before = x.clone()
+    means = torch.full((1, 2, (N + 15) // 16, D), 7.0, dtype=torch.float32, device=DEV)
+    st = torch.zeros(1, dtype=torch.int32, device=DEV)
+    L = dbp.library()
+    wqg, wkg = wq.to(DEV), wk.to(DEV)
+    rc = L.dit_qk_rmsnorm_rope3d_pooled_stall_test(
+        x.data_ptr(), x.data_ptr() + 2 * D, 3 * D, wqg.data_ptr(), wkg.data_ptr(), 0, 1, N,
+        wl.H, wl.hd, wl.T, wl.Hg, wl.Wg, None, 0, *wl.pairs, wl.theta, wl.eps, 0, 16,
+        means.data_ptr(), st.data_ptr(), torch.cuda.current_stream().cuda_stream)
+    assert rc == 0
+    torch.cuda.synchronize()
+    assert int(st.item()) == 1
+    assert torch.equal(x.view(torch.int16), before.view(torch.int16))
+    assert bool((means == 7.0).all())
+    st.zero_()
+    dbp.qk_rmsnorm_rope3d(x[:, :, :D], x[:, :, D:2 * D], wqg, wkg, wl.H, wl.pairs,
+                          grid=(wl.T, wl.Hg, wl.Wg), theta=wl.theta, eps=wl.eps,
+                          block_means=means, block=16, status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    hb = bits(qkv_h)
+    p = np.ascontiguousarray(orc.grid_positions(wl.T, wl.Hg, wl.Wg, 0, N).reshape(-1, 3))
+    ref = orc.qk_rmsnorm_rope3d_ex(hb[:, :D], wq.double().numpy(), wl.H, wl.hd, p, wl.pairs,
+                                   wl.theta, wl.eps, layout=0)
+    compare_bf16(bits(x.view(N, 3 * D))[:, :D], ref, "q after the stall")
