@@ -59,8 +59,8 @@ NCU_TOKENS = 124992
 NCU_TRAFFIC = {
     "adaln_modulate": {"file": "adaln.cu", "sha": "b4f26979a5cdeb0e",
                        "bytes_per_token": 2507664128 / NCU_TOKENS},
-    "qk_rmsnorm_rope3d": {"file": "qk_rope.cu", "sha": "b057e79cd2493df0",
-                          "bytes_per_token": 5056747008 / NCU_TOKENS},
+    "qk_rmsnorm_rope3d": {"file": "qk_rope.cu", "sha": "d014d3875c6ecca7",
+                          "bytes_per_token": 5057144832 / NCU_TOKENS},
     "gated_residual_adaln": {"file": "adaln.cu", "sha": "b4f26979a5cdeb0e",
                              "bytes_per_token": 5064393472 / NCU_TOKENS},
     "swiglu": {"file": "swiglu.cu", "sha": "a9e07b0f774729cf",
