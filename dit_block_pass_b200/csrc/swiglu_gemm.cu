@@ -61,12 +61,13 @@ constexpr int kThreadsG = 64 + 32 * kEpiWarps;
 // in flight share their x and W tiles in L2), measured at the H3 shapes:
 // SwiGLU [124992, 5120] x [27648, 5120]^T best at 8-12 (16 and more thrash L2:
 // 32 cost 12 %, 64 cost 24 %), the down-projection [124992, 13824] x
-// [5120, 13824]^T best at 4-5 (8: +2-4 %, 16: +8 %).  Outputs do not depend on it.
+// [5120, 13824]^T best at 4 (3, 5, 6, 7: +1-2 %; 8: +2-4 %, 16: +8 %).
+// Outputs do not depend on it.
 #ifndef GEMM_GROUP_SWIGLU
 #define GEMM_GROUP_SWIGLU 12
 #endif
 #ifndef GEMM_GROUP_RESID
-#define GEMM_GROUP_RESID 5
+#define GEMM_GROUP_RESID 4
 #endif
 constexpr uint32_t kTileA = kBM * kBK * 2;            // 16 KB per 128 rows
 constexpr uint32_t kTileB = 2 * kBN * kBK * 2;        // 32 KB (gate + linear)
